@@ -1,0 +1,354 @@
+"""Benchmark of the Gated DeltaNet token mixer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One JSON line on rank 0. A "step" is one gdn_prefill call (gate prologue + chunk
+kernel) on the 35B-A3B GDN layer shape: B=1, T=4096, 16 QK / 32 V heads,
+d=128, bf16 q/k/v/o, fp32 gates and state, zero initial state, final state
+written. `value` is prefill tokens/s over the whole job (all ranks; each rank
+runs its own copy of the workload, so scaling is weak). The same line carries
+the decode measurement (256 sequences x 64 V heads, 1000 consecutive in-place
+steps of gdn_decode_step) under "decode".
+
+Timing: W untimed warm-up steps; then K steps, each preceded by an L2 flush
+(a 512 MiB write, outside the timed window) and bracketed by CUDA events on
+the launching stream; a barrier and a device synchronise on both sides of the
+timed region; the max over ranks. `e2e` repeats the prefill through the public
+Python API from pinned host buffers, host<->device copies inside the timing.
+The CPU baseline is the fp64 oracle (test infrastructure) timed on this host.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "prefill_35b"
+METRIC = "GDN prefill tokens/s and decode steps/s on 1 B200, % of roofline"
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(
+            p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def prefill_bytes(T, N, H_qk, H_v, d, io_bytes, with_initial):
+    """Algorithmic HBM bytes of one gdn_prefill call: q, k, v read, o written,
+    a and b read, the final state written (and the initial state read if given)."""
+    b = 2 * T * H_qk * d * io_bytes + 2 * T * H_v * d * io_bytes + 2 * T * H_v * 4
+    b += N * H_v * d * d * 4 * (2 if with_initial else 1)
+    return b
+
+
+def prefill_flops(T, N, H_qk, H_v, d, C=64):
+    """Algorithmic tensor flops: the in-chunk products QK^T and KK^T per QK head,
+    and per V head the solve-applied T Y (C^2 d), the intra-chunk P Vnew (C^2 d),
+    and the state products K S^T, Q S^T and the state update (3 x 2 C d^2 per
+    chunk)."""
+    return T * (H_qk * 4 * C * d + H_v * (4 * C * d + 6 * d * d))
+
+
+def decode_bytes(N, H_qk, H_v, d, io_bytes):
+    return 2 * N * H_v * d * d * 4 + N * (2 * H_qk * d + 2 * H_v * d) * io_bytes + 2 * N * H_v * 4
+
+
+class Clocks:
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = [r.split(", ") for r in (getattr(self, "out", "") or "").strip().splitlines()]
+        rows = [r for r in rows if len(r) >= 9]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _max_over_ranks(x: float, ws: int, device) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def run_ours(args):
+    from linear_attention_sequence_delta_b200 import gdn
+    from linear_attention_sequence_delta_b200.inputs import (DECODE_STEPS, DECODE_WORKLOAD,
+                                                             WORKLOADS, make_decode_inputs,
+                                                             make_prefill_inputs)
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    gdn.load_library()
+    hbm, tc_burst, tc_sust, peak_src = _peaks()
+    W = WORKLOADS[WORKLOAD]
+    P = make_prefill_inputs(**W, seed=rank, device=dev)
+    T, H_qk, d = P.q.shape
+    H_v = P.v.shape[1]
+    N = P.num_seqs
+    o = torch.empty((T, H_v, d), device=dev, dtype=P.q.dtype)
+    Sf = torch.empty((N, H_v, d, d), device=dev, dtype=torch.float32)
+    wsz = gdn.workspace_size(N, T, H_qk, H_v, d, d)
+    work = torch.empty((max(wsz, 1),), device=dev, dtype=torch.uint8)
+    flush = torch.empty((512 << 20,), device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        gdn.gdn_prefill(P.q, P.k, P.v, P.a, P.b, P.A_log, P.dt_bias, P.cu_seqlens, None,
+                        out=o, final_state=Sf, workspace=work)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    clocks = Clocks(local)
+    _barrier(ws)
+    torch.cuda.synchronize()
+    with clocks:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)  # L2 flush, outside the events
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        _barrier(ws)
+        # ---- decode: 1000 consecutive steps on the 397B-A17B GDN shape ----
+        dec = None
+        if not args.no_decode:
+            D = make_decode_inputs(steps=args.decode_steps, seed=rank, device=dev,
+                                   **DECODE_WORKLOAD)
+            od = torch.empty_like(D.v[0])
+            for t in range(min(3, args.decode_steps)):  # warm-up on a copy of the state
+                gdn.gdn_decode_step(D.q[t], D.k[t], D.v[t], D.a[t], D.b[t], D.A_log, D.dt_bias,
+                                    D.state.clone(), out=od)
+            torch.cuda.synchronize()
+            _barrier(ws)
+            d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            d0.record(stream)
+            for t in range(args.decode_steps):
+                gdn.gdn_decode_step(D.q[t], D.k[t], D.v[t], D.a[t], D.b[t], D.A_log, D.dt_bias,
+                                    D.state, out=od)
+            d1.record(stream)
+            torch.cuda.synchronize()
+            dec_ms = _max_over_ranks(d0.elapsed_time(d1), ws, dev)
+            Nd, H_qkd, H_vd = D.q.shape[1], D.q.shape[2], D.v.shape[2]
+            per_step_s = dec_ms / 1e3 / args.decode_steps
+            db = decode_bytes(Nd, H_qkd, H_vd, d, 2)
+            dec = {"value": ws * args.decode_steps / (dec_ms / 1e3), "unit": "steps/s",
+                   "tokens_per_s": ws * Nd * args.decode_steps / (dec_ms / 1e3),
+                   "steps": args.decode_steps, "us_per_step": per_step_s * 1e6,
+                   "workload": f"decode: {Nd} seqs x 1 token, H_qk={H_qkd}, H_v={H_vd}, d={d}, "
+                               "bf16 q/k/v/o, fp32 state ~N(0,0.02^2) in place",
+                   "roofline": {"bound": "hbm", "achieved": db / per_step_s / 1e9,
+                                "peak": hbm, "unit": "GB/s",
+                                "frac": db / per_step_s / 1e9 / hbm, "traffic": None,
+                                "algorithmic_bytes": db, "peak_source": peak_src},
+                   "gpu_launches": args.decode_steps}
+            del D
+    kern_ms = [a.elapsed_time(b) for a, b in ev]
+    ms = _max_over_ranks(sum(kern_ms) / len(kern_ms), ws, dev)
+    tok_s = ws * T / (ms / 1e3)
+    byts = prefill_bytes(T, N, H_qk, H_v, d, 2, with_initial=False)
+    flops = prefill_flops(T, N, H_qk, H_v, d)
+    achieved = byts / (ms / 1e3) / 1e9
+    t_roof = max(byts / (hbm * 1e9), flops / (tc_burst * 1e12))
+
+    # ---- e2e through the public API from pinned host buffers ----
+    host = {k_: getattr(P, k_).cpu().pin_memory() for k_ in
+            ("q", "k", "v", "a", "b", "A_log", "dt_bias", "cu_seqlens")}
+    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    S_h = torch.empty(Sf.shape, dtype=Sf.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = o_h.numel() * o_h.element_size() + S_h.numel() * S_h.element_size()
+
+    def e2e_step():
+        dv = {k_: t.to(dev, non_blocking=True) for k_, t in host.items()}
+        oo, ss = gdn.gdn_prefill(dv["q"], dv["k"], dv["v"], dv["a"], dv["b"], dv["A_log"],
+                                 dv["dt_bias"], dv["cu_seqlens"], None)
+        o_h.copy_(oo, non_blocking=True)
+        S_h.copy_(ss, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    _barrier(ws)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / args.steps, ws, dev)
+
+    line = {
+        "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "prefill_35b: B=1, T=4096, H_qk=16, H_v=32, d=128, bf16 q/k/v/o, "
+                               "fp32 gates/state, zero initial state, final state written",
+                   "global_batch": ws, "seq_len": T, "parallelism": f"replicas x{ws}",
+                   "l2": "flushed (512 MiB write) before every timed step"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None, "algorithmic_bytes": byts,
+                     "kernel": "gdn_prefill (gate prologue + chunk kernel)",
+                     "peak_source": peak_src,
+                     "tensor": {"algorithmic_flops": flops, "achieved_tflops":
+                                flops / (ms / 1e3) / 1e12, "peak_tflops": tc_burst,
+                                "frac": flops / (ms / 1e3) / 1e12 / tc_burst},
+                     "frac_of_slower_roof": t_roof / (ms / 1e3)},
+        "e2e": {"value": ws * T / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * args.steps + (args.decode_steps if dec else 0),
+        "clocks": clocks.summary(),
+        "decode": dec,
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(P)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(P, heads=None):
+    """The fp64 oracle on this host's cores, on a bounded sample of the workload."""
+    import numpy as np
+
+    import oracle
+    H_v = P.v.shape[1]
+    heads = heads or H_v
+    r = H_v // P.q.shape[1]
+    Q = P.q.cpu()
+    K = P.k.cpu()
+    hs = list(range(heads))
+    js = sorted({h // r for h in hs})
+    t0 = time.perf_counter()
+    oracle.forward(Q[:, js[0]:js[-1] + 1], K[:, js[0]:js[-1] + 1], P.v[:, :heads].cpu(),
+                   P.a[:, :heads].cpu(), P.b[:, :heads].cpu(), P.A_log[:heads].cpu(),
+                   P.dt_bias[:heads].cpu(), P.cu_seqlens.cpu().numpy().astype(np.int64))
+    dt = time.perf_counter() - t0
+    T = P.q.shape[0]
+    return {"value": T * heads / H_v / dt, "unit": "tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{heads} of {H_v} V heads x {T} tokens ({dt:.2f} s), scaled to all heads"}
+
+
+def run_reference(args):
+    """The oracle (a plain sequential fp64 CPU program) as the reference arm."""
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return
+    from linear_attention_sequence_delta_b200.inputs import WORKLOADS, make_prefill_inputs
+    P = make_prefill_inputs(**WORKLOADS[WORKLOAD], seed=0)
+    heads = 8
+    for _ in range(args.warmup):
+        cpu_baseline(P, heads=2)  # untimed warm-up (page in the library and the inputs)
+    vals = []
+    for _ in range(args.steps):
+        vals.append(cpu_baseline(P, heads=heads))
+    v = statistics.median(x["value"] for x in vals)
+    T = P.q.shape[0]
+    line = {
+        "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": T / v * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": "prefill_35b: B=1, T=4096, H_qk=16, H_v=32, d=128, bf16 q/k/v "
+                               "(upcast exactly), fp64 arithmetic", "global_batch": 1,
+                   "seq_len": T, "parallelism": "host cores (OpenMP)"},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "kind": "oracle",
+                         "cores": vals[0]["cores"], "sample": vals[0]["sample"]},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

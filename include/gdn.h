@@ -1,0 +1,148 @@
+/*
+ * gdn.h -- C ABI of the Gated DeltaNet token-mixer library (libgdn.so).
+ *
+ * The library computes the gated delta rule of the Qwen3.5 linear-attention
+ * layers on one NVIDIA B200 (sm_100a):
+ *
+ *   per V head h, with QK head j = h / (H_v / H_qk):
+ *     q_t, k_t <- q_t / ||q_t||, k_t / ||k_t||   (eps 1e-6 inside the root)
+ *     g_t      = -exp(A_log[h]) * softplus(a_t + dt_bias[h]),  alpha_t = exp(g_t)
+ *     beta_t   = sigmoid(b_t)
+ *     S_t      = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *     o_t      = S_t (scale * q_t)
+ *
+ *   "Qwen3.5-MoE-35B-A3B architecture teardown", section 3.3 (the delta rule
+ *   and the prefill / decode split), 3.4 (QK heads shared by V heads), 3.5 (QK
+ *   L2 norm), 3.7 (the chunkwise prefill in seven steps);
+ *   "Qwen3.5 observation notes", sections "DeltaNet", "Gated DeltaNet" and
+ *   "Qwen3_5MoeGatedDeltaNet" (gates, decay before the read, the dispatch
+ *   between the chunked and the recurrent kernel, initial / final state).
+ *
+ * Conventions shared by every call:
+ *   - Pointers are DEVICE pointers unless stated, 16-byte aligned. The caller
+ *     owns every buffer; the library allocates nothing on any call.
+ *   - Tensors are dense, row-major, in the shapes given:
+ *       q, k        [T, H_qk, d_k]      v, o   [T, H_v, d_v]
+ *       a, b        [T, H_v]            A_log, dt_bias  [H_v]
+ *       state       [N, H_v, d_v, d_k]  value-major: o = S q, S[i][c] with
+ *                                       i a value index and c a key index.
+ *                                       (The pages' HF layout is the transpose.)
+ *     T is the packed token count; sequence n owns tokens cu_seqlens[n] ..
+ *     cu_seqlens[n+1]-1 (cu_seqlens: int32, device, N+1 entries, cu[0] = 0,
+ *     non-decreasing, cu[N] = T).
+ *   - io_dtype selects the type of q, k, v and o (GDN_BF16 or GDN_FP32). The
+ *     gates and the state are always fp32 (the pages' mamba_ssm_dtype float32).
+ *   - Supported shapes: d_k = d_v in {64, 128}; H_v a multiple of H_qk.
+ *   - `stream` is a cudaStream_t (NULL: the legacy default stream). Every call
+ *     is stream-ordered and asynchronous; nothing is synchronised.
+ *   - Errors: every call returns a gdn_status. Arguments are checked on the
+ *     host before anything is launched; a bad argument launches nothing.
+ *     Content errors that only the device can see (bad cu_seqlens, a bounded
+ *     wait that ran out) set a device status word that gdn_sync_status()
+ *     returns and clears. No call traps, asserts or aborts.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1, /* null / misaligned pointer, bad size or count       */
+    GDN_ERR_UNSUPPORTED = 2, /* a shape or type this build does not implement     */
+    GDN_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required        */
+    GDN_ERR_CUDA = 4,        /* a CUDA runtime call failed (launch, attribute)    */
+    GDN_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out                */
+    GDN_ERR_BAD_SEQLENS = 6  /* cu_seqlens not non-decreasing / out of range      */
+} gdn_status;
+
+typedef enum { GDN_BF16 = 0, GDN_FP32 = 1 } gdn_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* gdn_status_string(int status);
+
+/* Library ABI version: major * 10000 + minor * 100 + patch. */
+int gdn_version(void);
+
+/*
+ * Bytes of device workspace gdn_prefill needs for these sizes (the per-token
+ * chunk-cumulative log-decay G and beta, fp32 [T, H_v] each, plus alignment).
+ * Returns 0 for invalid sizes.
+ */
+size_t gdn_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t H_qk,
+                                  int32_t H_v, int32_t d_k, int32_t d_v);
+
+/*
+ * gdn_gates -- the gate prologue ("Qwen3.5 observation notes",
+ * "Qwen3_5MoeGatedDeltaNet": beta = sigmoid(b), g = -exp(A_log) *
+ * softplus(a + dt_bias); "Qwen3.5-MoE-35B-A3B architecture teardown", 3.7
+ * step 3: the cumulative sum of g inside each 64-token chunk).
+ *   a, b              [T, H_v] fp32          (in)
+ *   A_log, dt_bias    [H_v] fp32             (in)
+ *   cu_seqlens        [N+1] int32            (in) chunks restart at each sequence
+ *   g_chunk_cumsum    [T, H_v] fp32 or NULL  (out) inclusive cumsum of g per chunk
+ *   g                 [T, H_v] fp32 or NULL  (out) the log-decay itself
+ *   beta              [T, H_v] fp32 or NULL  (out)
+ * g is computed as 0 where softplus(...) is 0, so alpha = 1 there (no NaN),
+ * and is clamped below at -128, where alpha = exp(g) is already 0 in fp32; the
+ * clamp keeps the in-chunk sums finite when alpha = 0 (g = -inf).
+ */
+int gdn_gates(const float* a, const float* b, const float* A_log, const float* dt_bias,
+              const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens, int32_t H_v,
+              float* g_chunk_cumsum, float* g, float* beta, void* stream);
+
+/*
+ * gdn_prefill -- the chunked prefill (the pages' chunk_gated_delta_rule with
+ * use_qk_l2norm_in_kernel=True; "Qwen3.5-MoE-35B-A3B architecture teardown",
+ * 3.7 steps 1-7, chunk size 64). Runs the gate prologue, then the chunk kernel.
+ *   q, k, v           io_dtype, shapes above (in)
+ *   a, b, A_log, dt_bias  fp32 (in)
+ *   initial_state     [N, H_v, d_v, d_k] fp32 or NULL (zeros)          (in)
+ *   cu_seqlens        [N+1] int32                                        (in)
+ *   scale             multiplier on the normalised query (1.0f = none)
+ *   o                 [T, H_v, d_v] io_dtype                              (out)
+ *   final_state       [N, H_v, d_v, d_k] fp32 or NULL (not written)      (out)
+ *                     may alias initial_state (each state is read before it
+ *                     is written, by the same block)
+ *   workspace         >= gdn_prefill_workspace_size(...) bytes, 256-byte aligned
+ * Empty sequences are allowed: their final state equals their initial state.
+ */
+int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
+                const float* a, const float* b, const float* A_log, const float* dt_bias,
+                const float* initial_state, const int32_t* cu_seqlens, int32_t num_seqs,
+                int64_t total_tokens, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
+                float scale, void* o, float* final_state, void* workspace,
+                size_t workspace_bytes, void* stream);
+
+/*
+ * gdn_decode_step -- one token for each of N sequences, the state updated in
+ * place (the pages' recurrent_gated_delta_rule for seq_len == 1; "Qwen3.5
+ * observation notes", "Qwen3_5MoeGatedDeltaNet": state *= exp(g), kv_mem,
+ * delta = (v - kv_mem) * beta, state += k delta^T, out = read-out with q).
+ *   q, k   [N, H_qk, d_k] io_dtype   v [N, H_v, d_v] io_dtype          (in)
+ *   a, b   [N, H_v] fp32             A_log, dt_bias [H_v] fp32          (in)
+ *   state  [N, H_v, d_v, d_k] fp32                                (in/out)
+ *   o      [N, H_v, d_v] io_dtype                                      (out)
+ */
+int gdn_decode_step(const void* q, const void* k, const void* v, int32_t io_dtype,
+                    const float* a, const float* b, const float* A_log, const float* dt_bias,
+                    float* state, int32_t num_seqs, int32_t H_qk, int32_t H_v, int32_t d_k,
+                    int32_t d_v, float scale, void* o, void* stream);
+
+/*
+ * Synchronise `stream`, then return and clear the device status word of the
+ * current device (GDN_OK, GDN_ERR_BAD_SEQLENS or GDN_ERR_TIMEOUT), or
+ * GDN_ERR_CUDA if the synchronisation itself failed.
+ */
+int gdn_sync_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

@@ -1,0 +1,8 @@
+"""Gated DeltaNet token mixer on NVIDIA B200 (sm_100a).
+
+The compute lives in libgdn.so (CUDA kernels behind the C ABI of
+include/gdn.h); `gdn` is its ctypes binding and `inputs` draws seeded
+synthetic inputs of the Qwen3.5 GDN layer shapes.
+"""
+from .gdn import (GDNError, gdn_decode_step, gdn_gates, gdn_prefill, gdn_sync_status,  # noqa: F401
+                  load_library, workspace_size)

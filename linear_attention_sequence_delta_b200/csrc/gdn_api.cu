@@ -1,0 +1,173 @@
+// C ABI of libgdn.so: argument checks, workspace carving and kernel dispatch.
+// Declarations and the contract of every entry point are in include/gdn.h.
+#include <math.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "gdn_internal.cuh"
+
+namespace gdn {
+
+// One status word per device: kernels record content errors (bad cu_seqlens,
+// an expired bounded wait) here instead of trapping.
+__device__ int g_status_word;
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::atomic<int*> g_status_ptr[kMaxDevices];
+std::mutex g_status_mu;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline bool aligned(const void* p, size_t a) {
+    return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+inline int to_status(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
+
+int check_heads(int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v) {
+    if (H_qk <= 0 || H_v <= 0 || d_k <= 0 || d_v <= 0) return GDN_ERR_INVALID_ARG;
+    if (H_v % H_qk != 0) return GDN_ERR_INVALID_ARG;
+    if (d_k != d_v || (d_k != 64 && d_k != 128)) return GDN_ERR_UNSUPPORTED;
+    return GDN_OK;
+}
+
+size_t gate_bytes(int64_t T, int32_t H_v) { return align_up((size_t)T * H_v * sizeof(float), 256); }
+}  // namespace
+
+int* device_status_ptr() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    int* p = g_status_ptr[dev].load(std::memory_order_acquire);
+    if (p) return p;
+    std::lock_guard<std::mutex> lk(g_status_mu);
+    p = g_status_ptr[dev].load(std::memory_order_relaxed);
+    if (!p) {
+        void* addr = nullptr;
+        if (cudaGetSymbolAddress(&addr, g_status_word) != cudaSuccess) return nullptr;
+        p = static_cast<int*>(addr);
+        g_status_ptr[dev].store(p, std::memory_order_release);
+    }
+    return p;
+}
+
+}  // namespace gdn
+
+using namespace gdn;
+
+extern "C" {
+
+const char* gdn_status_string(int status) {
+    switch (status) {
+        case GDN_OK: return "GDN_OK";
+        case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG";
+        case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
+        case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE";
+        case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+        case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
+        case GDN_ERR_BAD_SEQLENS: return "GDN_ERR_BAD_SEQLENS";
+        default: return "GDN_ERR_UNKNOWN";
+    }
+}
+
+int gdn_version(void) { return 100; }
+
+size_t gdn_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t H_qk,
+                                  int32_t H_v, int32_t d_k, int32_t d_v) {
+    if (num_seqs < 0 || total_tokens < 0) return 0;
+    if (check_heads(H_qk, H_v, d_k, d_v) != GDN_OK) return 0;
+    return 2 * gate_bytes(total_tokens, H_v);
+}
+
+int gdn_gates(const float* a, const float* b, const float* A_log, const float* dt_bias,
+              const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens, int32_t H_v,
+              float* g_chunk_cumsum, float* g, float* beta, void* stream) {
+    if (num_seqs < 0 || total_tokens < 0 || H_v <= 0) return GDN_ERR_INVALID_ARG;
+    if (num_seqs == 0 && total_tokens != 0) return GDN_ERR_INVALID_ARG;
+    if (num_seqs == 0 || (!g_chunk_cumsum && !g && !beta)) return GDN_OK;
+    if (!a || !b || !A_log || !dt_bias || !cu_seqlens) return GDN_ERR_INVALID_ARG;
+    if (!aligned(a, 4) || !aligned(b, 4) || !aligned(g_chunk_cumsum, 4) || !aligned(g, 4) ||
+        !aligned(beta, 4))
+        return GDN_ERR_INVALID_ARG;
+    int* st = device_status_ptr();
+    if (!st) return GDN_ERR_CUDA;
+    return to_status(launch_gates(a, b, A_log, dt_bias, cu_seqlens, num_seqs, total_tokens, H_v,
+                                  g_chunk_cumsum, g, beta, st, (cudaStream_t)stream));
+}
+
+int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
+                const float* a, const float* b, const float* A_log, const float* dt_bias,
+                const float* initial_state, const int32_t* cu_seqlens, int32_t num_seqs,
+                int64_t total_tokens, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
+                float scale, void* o, float* final_state, void* workspace,
+                size_t workspace_bytes, void* stream) {
+    if (io_dtype != GDN_BF16 && io_dtype != GDN_FP32) return GDN_ERR_INVALID_ARG;
+    if (num_seqs < 0 || total_tokens < 0) return GDN_ERR_INVALID_ARG;
+    if (num_seqs == 0 && total_tokens != 0) return GDN_ERR_INVALID_ARG;
+    int hs = check_heads(H_qk, H_v, d_k, d_v);
+    if (hs != GDN_OK) return hs;
+    if (!isfinite(scale)) return GDN_ERR_INVALID_ARG;
+    if (num_seqs == 0) return GDN_OK;
+    if ((int64_t)num_seqs * H_v * (d_v / 32) >= (int64_t)1 << 31) return GDN_ERR_UNSUPPORTED;
+    if (!cu_seqlens || !A_log || !dt_bias) return GDN_ERR_INVALID_ARG;
+    if (total_tokens > 0 && (!q || !k || !v || !a || !b || !o)) return GDN_ERR_INVALID_ARG;
+    const void* ptrs16[] = {q, k, v, o, initial_state, final_state};
+    for (const void* p : ptrs16)
+        if (!aligned(p, 16)) return GDN_ERR_INVALID_ARG;
+    if (!aligned(a, 4) || !aligned(b, 4)) return GDN_ERR_INVALID_ARG;
+    const size_t need = gdn_prefill_workspace_size(num_seqs, total_tokens, H_qk, H_v, d_k, d_v);
+    if (workspace_bytes < need || (need > 0 && !workspace)) return GDN_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return GDN_ERR_WORKSPACE;
+
+    int* st = device_status_ptr();
+    if (!st) return GDN_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    float* G = static_cast<float*>(workspace);
+    float* beta = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                           gate_bytes(total_tokens, H_v));
+    if (total_tokens > 0) {
+        cudaError_t e = launch_gates(a, b, A_log, dt_bias, cu_seqlens, num_seqs, total_tokens,
+                                     H_v, G, nullptr, beta, st, s);
+        if (e != cudaSuccess) return GDN_ERR_CUDA;
+    }
+    return to_status(launch_prefill_simt(q, k, v, io_dtype, G, beta, initial_state, cu_seqlens,
+                                         num_seqs, total_tokens, H_qk, H_v, d_k, scale, o,
+                                         final_state, st, s));
+}
+
+int gdn_decode_step(const void* q, const void* k, const void* v, int32_t io_dtype,
+                    const float* a, const float* b, const float* A_log, const float* dt_bias,
+                    float* state, int32_t num_seqs, int32_t H_qk, int32_t H_v, int32_t d_k,
+                    int32_t d_v, float scale, void* o, void* stream) {
+    if (io_dtype != GDN_BF16 && io_dtype != GDN_FP32) return GDN_ERR_INVALID_ARG;
+    if (num_seqs < 0) return GDN_ERR_INVALID_ARG;
+    int hs = check_heads(H_qk, H_v, d_k, d_v);
+    if (hs != GDN_OK) return hs;
+    if (!isfinite(scale)) return GDN_ERR_INVALID_ARG;
+    if (num_seqs == 0) return GDN_OK;
+    if ((int64_t)num_seqs * H_v >= (int64_t)1 << 31) return GDN_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !a || !b || !A_log || !dt_bias || !state || !o)
+        return GDN_ERR_INVALID_ARG;
+    const void* ptrs16[] = {q, k, v, o, state};
+    for (const void* p : ptrs16)
+        if (!aligned(p, 16)) return GDN_ERR_INVALID_ARG;
+    if (!aligned(a, 4) || !aligned(b, 4)) return GDN_ERR_INVALID_ARG;
+    return to_status(launch_decode(q, k, v, io_dtype, a, b, A_log, dt_bias, state, num_seqs,
+                                   H_qk, H_v, d_k, scale, o, (cudaStream_t)stream));
+}
+
+int gdn_sync_status(void* stream) {
+    int* st = device_status_ptr();
+    if (!st) return GDN_ERR_CUDA;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return GDN_ERR_CUDA;
+    int val = 0;
+    if (cudaMemcpy(&val, st, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    const int zero = 0;
+    if (val != 0 && cudaMemcpy(st, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    return val;
+}
+
+}  // extern "C"

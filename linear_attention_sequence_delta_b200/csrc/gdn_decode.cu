@@ -1,0 +1,188 @@
+// Single-token decode: one step of the gated delta rule per (sequence, V head),
+// the fp32 state updated in place ("Qwen3.5 observation notes",
+// "Qwen3_5MoeGatedDeltaNet", the recurrent kernel for seq_len == 1).
+//
+// With the value-major state S[i][c] (i: value index, c: key index) every value
+// row evolves on its own:
+//   S_i <- alpha S_i;  delta_i = beta (v_i - S_i . k);  S_i <- S_i + delta_i k;
+//   o_i = S_i . q = alpha (S_old_i . q) + delta_i (k . q)
+// so one pass that reads a row, forms two dot products (with k and q), and
+// writes the row back does the whole step. The kernel is HBM-bound: 2 * 4 * d^2
+// bytes of state per head move per token, against ~7 d^2 flops.
+//
+// Mapping: one 128-thread block per (sequence, head). A warp covers four rows at
+// a time, eight lanes per row, each lane holding d/8 consecutive-by-float4
+// elements (offsets 4p + 32m), so every load and store instruction moves four
+// fully used 128-byte lines. The two dot products reduce over the eight lanes
+// of a row with three xor shuffles each. Loads of two row groups are issued
+// before any arithmetic so each lane keeps 2 * d/32 16-byte loads in flight.
+#include "gdn_internal.cuh"
+
+namespace gdn {
+
+namespace {
+
+template <typename IO, int NE>
+__device__ __forceinline__ void load_vec(const IO* p, float (&out)[NE]);
+
+template <>
+__device__ __forceinline__ void load_vec<float, 4>(const float* p, float (&out)[4]) {
+    const float4 x = *reinterpret_cast<const float4*>(p);
+    out[0] = x.x; out[1] = x.y; out[2] = x.z; out[3] = x.w;
+}
+
+template <>
+__device__ __forceinline__ void load_vec<__nv_bfloat16, 4>(const __nv_bfloat16* p,
+                                                          float (&out)[4]) {
+    const uint2 x = *reinterpret_cast<const uint2*>(p);
+    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&x.x);
+    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&x.y);
+    const float2 l = __bfloat1622float2(lo), h = __bfloat1622float2(hi);
+    out[0] = l.x; out[1] = l.y; out[2] = h.x; out[3] = h.y;
+}
+
+constexpr int kRowGroupsInFlight = 2;
+
+template <typename IO, int D>
+__global__ void __launch_bounds__(128, 4) decode_kernel(
+    const IO* __restrict__ q, const IO* __restrict__ k, const IO* __restrict__ v,
+    const float* __restrict__ a, const float* __restrict__ b,
+    const float* __restrict__ A_log, const float* __restrict__ dt_bias,
+    float* __restrict__ state, int H_qk, int H_v, float scale, IO* __restrict__ o) {
+    constexpr int NV = D / 32;               // float4 chunks per lane per row
+    constexpr int ROWS_PER_WARP = D / 4;     // 4 warps share the D rows
+    constexpr int ITERS = ROWS_PER_WARP / 4; // 4 rows per warp-iteration
+    constexpr int B = kRowGroupsInFlight;
+    static_assert(ITERS % B == 0, "row groups must tile the warp's rows");
+
+    const int unit = blockIdx.x;  // n * H_v + h
+    const int n = unit / H_v;
+    const int h = unit - n * H_v;
+    const int j = h / (H_v / H_qk);
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int p = lane & 7;   // position inside the row
+    const int rg = lane >> 3; // which of the four rows
+
+    // normalised q and k, in the lane's column pattern (cols 4p + 32m .. +3)
+    float kr[NV][4], qr[NV][4];
+    const IO* qp = q + ((size_t)n * H_qk + j) * D;
+    const IO* kp = k + ((size_t)n * H_qk + j) * D;
+#pragma unroll
+    for (int m = 0; m < NV; ++m) {
+        load_vec<IO, 4>(qp + 4 * p + 32 * m, qr[m]);
+        load_vec<IO, 4>(kp + 4 * p + 32 * m, kr[m]);
+    }
+    float sq = 0.f, sk = 0.f;
+#pragma unroll
+    for (int m = 0; m < NV; ++m)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            sq = fmaf(qr[m][e], qr[m][e], sq);
+            sk = fmaf(kr[m][e], kr[m][e], sk);
+        }
+#pragma unroll
+    for (int x = 1; x < 8; x <<= 1) {
+        sq += __shfl_xor_sync(0xffffffffu, sq, x);
+        sk += __shfl_xor_sync(0xffffffffu, sk, x);
+    }
+    const float rq = scale / sqrtf(sq + kL2Eps);
+    const float rk = 1.f / sqrtf(sk + kL2Eps);
+    float kq = 0.f;
+#pragma unroll
+    for (int m = 0; m < NV; ++m)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            qr[m][e] *= rq;
+            kr[m][e] *= rk;
+            kq = fmaf(kr[m][e], qr[m][e], kq);
+        }
+#pragma unroll
+    for (int x = 1; x < 8; x <<= 1) kq += __shfl_xor_sync(0xffffffffu, kq, x);
+
+    const float alpha = expf(gate_g(a[unit], A_log[h], dt_bias[h]));
+    const float beta = gate_beta(b[unit]);
+
+    float* S = state + (size_t)unit * D * D;
+    const IO* vp = v + (size_t)unit * D;
+    IO* op = o + (size_t)unit * D;
+
+#pragma unroll 1
+    for (int it0 = 0; it0 < ITERS; it0 += B) {
+        float4 s[B][NV];
+        float vi[B];
+#pragma unroll
+        for (int bb = 0; bb < B; ++bb) {
+            const int row = warp * ROWS_PER_WARP + (it0 + bb) * 4 + rg;
+            const float* rp = S + (size_t)row * D + 4 * p;
+#pragma unroll
+            for (int m = 0; m < NV; ++m) s[bb][m] = __ldcs(reinterpret_cast<const float4*>(rp + 32 * m));
+            vi[bb] = to_f32(vp[row]);
+        }
+#pragma unroll
+        for (int bb = 0; bb < B; ++bb) {
+            const int row = warp * ROWS_PER_WARP + (it0 + bb) * 4 + rg;
+            float dk = 0.f, dq = 0.f;
+#pragma unroll
+            for (int m = 0; m < NV; ++m) {
+                dk = fmaf(s[bb][m].x, kr[m][0], dk); dq = fmaf(s[bb][m].x, qr[m][0], dq);
+                dk = fmaf(s[bb][m].y, kr[m][1], dk); dq = fmaf(s[bb][m].y, qr[m][1], dq);
+                dk = fmaf(s[bb][m].z, kr[m][2], dk); dq = fmaf(s[bb][m].z, qr[m][2], dq);
+                dk = fmaf(s[bb][m].w, kr[m][3], dk); dq = fmaf(s[bb][m].w, qr[m][3], dq);
+            }
+#pragma unroll
+            for (int x = 1; x < 8; x <<= 1) {
+                dk += __shfl_xor_sync(0xffffffffu, dk, x);
+                dq += __shfl_xor_sync(0xffffffffu, dq, x);
+            }
+            // read with the decayed state, then write
+            const float delta = beta * (vi[bb] - alpha * dk);
+            float* rp = S + (size_t)row * D + 4 * p;
+#pragma unroll
+            for (int m = 0; m < NV; ++m) {
+                float4 w;
+                w.x = fmaf(alpha, s[bb][m].x, delta * kr[m][0]);
+                w.y = fmaf(alpha, s[bb][m].y, delta * kr[m][1]);
+                w.z = fmaf(alpha, s[bb][m].z, delta * kr[m][2]);
+                w.w = fmaf(alpha, s[bb][m].w, delta * kr[m][3]);
+                __stcs(reinterpret_cast<float4*>(rp + 32 * m), w);
+            }
+            if (p == 0) op[row] = from_f32<IO>(fmaf(alpha, dq, delta * kq));
+        }
+    }
+}
+
+template <typename IO, int D>
+cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const float* a,
+                            const float* b, const float* A_log, const float* dt_bias,
+                            float* state, int32_t N, int32_t H_qk, int32_t H_v, float scale,
+                            void* o, cudaStream_t s) {
+    const int64_t units = (int64_t)N * H_v;
+    if (units == 0) return cudaSuccess;
+    decode_kernel<IO, D><<<(unsigned)units, 128, 0, s>>>(
+        static_cast<const IO*>(q), static_cast<const IO*>(k), static_cast<const IO*>(v), a, b,
+        A_log, dt_bias, state, H_qk, H_v, scale, static_cast<IO*>(o));
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const void* q, const void* k, const void* v, int io_dtype,
+                          const float* a, const float* b, const float* A_log,
+                          const float* dt_bias, float* state, int32_t N, int32_t H_qk,
+                          int32_t H_v, int32_t d, float scale, void* o, cudaStream_t s) {
+    if (io_dtype == GDN_BF16) {
+        if (d == 128)
+            return launch_decode_t<__nv_bfloat16, 128>(q, k, v, a, b, A_log, dt_bias, state, N,
+                                                       H_qk, H_v, scale, o, s);
+        return launch_decode_t<__nv_bfloat16, 64>(q, k, v, a, b, A_log, dt_bias, state, N, H_qk,
+                                                  H_v, scale, o, s);
+    }
+    if (d == 128)
+        return launch_decode_t<float, 128>(q, k, v, a, b, A_log, dt_bias, state, N, H_qk, H_v,
+                                           scale, o, s);
+    return launch_decode_t<float, 64>(q, k, v, a, b, A_log, dt_bias, state, N, H_qk, H_v, scale,
+                                      o, s);
+}
+
+}  // namespace gdn

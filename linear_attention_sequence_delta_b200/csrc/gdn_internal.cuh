@@ -1,0 +1,90 @@
+// Internal declarations shared by the kernel translation units of libgdn.so.
+// Not part of the public ABI (that is include/gdn.h).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gdn.h"
+
+namespace gdn {
+
+constexpr int kChunk = 64;          // chunk length of the prefill (teardown, 3.7 step 2)
+constexpr float kL2Eps = 1e-6f;     // inside the square root of the QK L2 norm
+// Lower clamp of the per-token log-decay g. exp(-128) is 0 in fp32, so alpha is
+// unchanged (exactly 0) by the clamp, but the in-chunk cumulative sums stay
+// finite: a gate of alpha = 0 (g = -inf, e.g. exp(A_log) overflowing) would
+// otherwise turn G_i - G_j into inf - inf = NaN.
+constexpr float kMinLogDecay = -128.f;
+
+// Device status word values (written by kernels, read by gdn_sync_status).
+constexpr int kStatusBadSeqlens = GDN_ERR_BAD_SEQLENS;
+constexpr int kStatusTimeout = GDN_ERR_TIMEOUT;
+
+// ---- small device helpers ---------------------------------------------------
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T x);
+template <>
+__device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+    return __bfloat162float(x);
+}
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// softplus(x) = log(1 + e^x) in the overflow-free form max(x,0) + log1p(e^-|x|).
+__device__ __forceinline__ float softplus_f32(float x) {
+    return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x)));
+}
+
+// g = -exp(A_log) * softplus(a + dt_bias); 0 when the softplus is 0 (alpha = 1);
+// clamped below at kMinLogDecay (where alpha is 0 in fp32 either way).
+__device__ __forceinline__ float gate_g(float a, float A_log, float dt_bias) {
+    const float sp = softplus_f32(a + dt_bias);
+    return sp > 0.f ? fmaxf(-expf(A_log) * sp, kMinLogDecay) : 0.f;
+}
+
+__device__ __forceinline__ float gate_beta(float b) { return 1.f / (1.f + expf(-b)); }
+
+__device__ __forceinline__ void set_status(int* status, int code) {
+    if (status) atomicCAS(status, 0, code);
+}
+
+// ---- host launchers (one per kernel family) ----------------------------------
+
+// Status word of the current device (a __device__ int of this library).
+int* device_status_ptr();
+
+cudaError_t launch_gates(const float* a, const float* b, const float* A_log,
+                         const float* dt_bias, const int32_t* cu_seqlens, int32_t num_seqs,
+                         int64_t total_tokens, int32_t H_v, float* G, float* g, float* beta,
+                         int* status, cudaStream_t s);
+
+cudaError_t launch_decode(const void* q, const void* k, const void* v, int io_dtype,
+                          const float* a, const float* b, const float* A_log,
+                          const float* dt_bias, float* state, int32_t N, int32_t H_qk,
+                          int32_t H_v, int32_t d, float scale, void* o, cudaStream_t s);
+
+cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, int io_dtype,
+                                const float* G, const float* beta, const float* S0,
+                                const int32_t* cu_seqlens, int32_t N, int64_t T, int32_t H_qk,
+                                int32_t H_v, int32_t d, float scale, void* o, float* S_final,
+                                int* status, cudaStream_t s);
+
+}  // namespace gdn

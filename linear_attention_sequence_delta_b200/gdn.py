@@ -1,0 +1,178 @@
+"""Python binding of libgdn.so (argument marshalling only).
+
+Every step of the computation runs in the library's CUDA kernels; this module
+only checks tensor metadata, allocates outputs/workspace through torch, and
+passes raw pointers and the current CUDA stream across the C ABI declared in
+include/gdn.h. There is no fallback: if the library is missing or cannot be
+loaded, every call raises.
+
+The three calls keep the C names:
+  gdn_gates(a, b, A_log, dt_bias, cu_seqlens, ...)
+  gdn_prefill(q, k, v, a, b, A_log, dt_bias, cu_seqlens, initial_state=None, ...)
+  gdn_decode_step(q, k, v, a, b, A_log, dt_bias, state, ...)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdn.so")
+
+GDN_BF16, GDN_FP32 = 0, 1
+_STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "GDN_ERR_WORKSPACE",
+           4: "GDN_ERR_CUDA", 5: "GDN_ERR_TIMEOUT", 6: "GDN_ERR_BAD_SEQLENS"}
+
+# Every symbol include/gdn.h declares (the tests check the library exports them all).
+EXPORTS = ["gdn_status_string", "gdn_version", "gdn_prefill_workspace_size", "gdn_gates",
+           "gdn_prefill", "gdn_decode_step", "gdn_sync_status"]
+
+
+class GDNError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_STATUS.get(status, status)}")
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libgdn.so (built by `python -m linear_attention_sequence_delta_b200.build`)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libgdn.so not found at {path}; build it with "
+                           "`python -m linear_attention_sequence_delta_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, i32, i64, f32, sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
+                            ctypes.c_size_t)
+    lib.gdn_status_string.restype = ctypes.c_char_p
+    lib.gdn_status_string.argtypes = [ctypes.c_int]
+    lib.gdn_version.restype = ctypes.c_int
+    lib.gdn_prefill_workspace_size.restype = sz
+    lib.gdn_prefill_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32]
+    lib.gdn_gates.restype = ctypes.c_int
+    lib.gdn_gates.argtypes = [P, P, P, P, P, i32, i64, i32, P, P, P, P]
+    lib.gdn_prefill.restype = ctypes.c_int
+    lib.gdn_prefill.argtypes = [P, P, P, i32, P, P, P, P, P, P, i32, i64, i32, i32, i32, i32, f32,
+                                P, P, P, sz, P]
+    lib.gdn_decode_step.restype = ctypes.c_int
+    lib.gdn_decode_step.argtypes = [P, P, P, i32, P, P, P, P, P, i32, i32, i32, i32, i32, f32, P,
+                                    P]
+    lib.gdn_sync_status.restype = ctypes.c_int
+    lib.gdn_sync_status.argtypes = [P]
+    _lib = lib
+    return lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _io_dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GDN_BF16
+    if t.dtype == torch.float32:
+        return GDN_FP32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise GDNError(status, where)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("all tensors must be CUDA tensors")
+            if not t.is_contiguous():
+                raise ValueError("all tensors must be contiguous")
+
+
+def workspace_size(num_seqs, total_tokens, H_qk, H_v, d_k, d_v) -> int:
+    return int(load_library().gdn_prefill_workspace_size(num_seqs, total_tokens, H_qk, H_v, d_k,
+                                                         d_v))
+
+
+def gdn_gates(a, b, A_log, dt_bias, cu_seqlens, *, want_cumsum=True, want_g=True,
+              want_beta=True) -> Tuple[Optional[torch.Tensor], ...]:
+    """Returns (g_chunk_cumsum, g, beta), fp32 [T, H_v] each (None where not asked for)."""
+    lib = load_library()
+    _need_cuda(a, b, A_log, dt_bias, cu_seqlens)
+    T, H_v = a.shape
+    mk = lambda w: torch.empty((T, H_v), device=a.device, dtype=torch.float32) if w else None
+    G, g, beta = mk(want_cumsum), mk(want_g), mk(want_beta)
+    st = lib.gdn_gates(_ptr(a), _ptr(b), _ptr(A_log), _ptr(dt_bias), _ptr(cu_seqlens),
+                       cu_seqlens.numel() - 1, T, H_v, _ptr(G), _ptr(g), _ptr(beta),
+                       _stream(a.device))
+    _check(st, "gdn_gates")
+    return G, g, beta
+
+
+def gdn_prefill(q, k, v, a, b, A_log, dt_bias, cu_seqlens, initial_state=None, *,
+                scale: float = 1.0, output_final_state: bool = True, out=None,
+                final_state=None, workspace=None):
+    """Chunked prefill over a packed batch. Returns (o, final_state or None).
+
+    q, k [T, H_qk, d_k]; v [T, H_v, d_v] (bf16 or fp32, all the same);
+    a, b [T, H_v] fp32; A_log, dt_bias [H_v] fp32; cu_seqlens int32 [N+1];
+    initial_state [N, H_v, d_v, d_k] fp32 or None.
+    """
+    lib = load_library()
+    _need_cuda(q, k, v, a, b, A_log, dt_bias, cu_seqlens, initial_state, out, final_state,
+               workspace)
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k and v must share one dtype")
+    io = _io_dtype(q)
+    T, H_qk, d_k = q.shape
+    _, H_v, d_v = v.shape
+    N = cu_seqlens.numel() - 1
+    o = out if out is not None else torch.empty((T, H_v, d_v), device=q.device, dtype=q.dtype)
+    if output_final_state and final_state is None:
+        final_state = torch.empty((N, H_v, d_v, d_k), device=q.device, dtype=torch.float32)
+    if not output_final_state:
+        final_state = None
+    need = lib.gdn_prefill_workspace_size(N, T, H_qk, H_v, d_k, d_v)
+    if workspace is None:
+        workspace = torch.empty((max(int(need), 1),), device=q.device, dtype=torch.uint8)
+    st = lib.gdn_prefill(_ptr(q), _ptr(k), _ptr(v), io, _ptr(a), _ptr(b), _ptr(A_log),
+                         _ptr(dt_bias), _ptr(initial_state), _ptr(cu_seqlens), N, T, H_qk, H_v,
+                         d_k, d_v, float(scale), _ptr(o), _ptr(final_state), _ptr(workspace),
+                         workspace.numel(), _stream(q.device))
+    _check(st, "gdn_prefill")
+    return o, final_state
+
+
+def gdn_decode_step(q, k, v, a, b, A_log, dt_bias, state, *, scale: float = 1.0, out=None):
+    """One token per sequence; `state` [N, H_v, d_v, d_k] fp32 is updated in place.
+
+    q, k [N, H_qk, d_k]; v [N, H_v, d_v]; a, b [N, H_v]. Returns o [N, H_v, d_v].
+    """
+    lib = load_library()
+    _need_cuda(q, k, v, a, b, A_log, dt_bias, state, out)
+    io = _io_dtype(q)
+    N, H_qk, d_k = q.shape
+    _, H_v, d_v = v.shape
+    o = out if out is not None else torch.empty((N, H_v, d_v), device=q.device, dtype=q.dtype)
+    st = lib.gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), io, _ptr(a), _ptr(b), _ptr(A_log),
+                             _ptr(dt_bias), _ptr(state), N, H_qk, H_v, d_k, d_v, float(scale),
+                             _ptr(o), _stream(q.device))
+    _check(st, "gdn_decode_step")
+    return o
+
+
+def gdn_sync_status(device=None) -> int:
+    """Synchronise the current stream and return (and clear) the device status word."""
+    lib = load_library()
+    return int(lib.gdn_sync_status(_stream(device)))

@@ -1,0 +1,152 @@
+"""The C ABI on the host: exports, status strings, workspace sizing and argument
+checks. No CUDA call is made here: every case is rejected before any launch,
+so these run on a machine without a GPU. Pointer values are fake and aligned
+(or deliberately misaligned); they are never dereferenced.
+"""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+from linear_attention_sequence_delta_b200 import build, gdn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return gdn.load_library()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "gdn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_[a-z_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(lib):
+    decl = _declared()
+    assert set(decl) == set(gdn.EXPORTS)
+    for name in decl:
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code, name in gdn._STATUS.items():
+        assert lib.gdn_status_string(code).decode() == name
+    assert lib.gdn_status_string(99).decode() == "GDN_ERR_UNKNOWN"
+    assert lib.gdn_version() >= 100
+
+
+def test_workspace_size(lib):
+    ws = lib.gdn_prefill_workspace_size
+    assert ws(1, 4096, 16, 32, 128, 128) == 2 * 4096 * 32 * 4
+    assert ws(1, 3, 1, 1, 64, 64) == 2 * 256  # each part rounded up to 256 bytes
+    assert ws(0, 0, 16, 32, 128, 128) == 0
+    assert ws(1, 10, 16, 24, 128, 128) == 0   # H_v % H_qk != 0
+    assert ws(1, 10, 16, 32, 96, 96) == 0     # unsupported head dim
+    assert ws(-1, 10, 16, 32, 128, 128) == 0
+
+
+F = 0x7F0000000000  # fake, 256-byte aligned "device" address
+
+
+def _prefill_args(**over):
+    a = dict(q=F, k=F + 0x1000, v=F + 0x2000, io=gdn.GDN_BF16, a=F + 0x3000, b=F + 0x4000,
+             A_log=F + 0x5000, dt_bias=F + 0x6000, S0=None, cu=F + 0x7000, N=1, T=128, H_qk=2,
+             H_v=4, d_k=64, d_v=64, scale=1.0, o=F + 0x8000, Sf=None, ws=F + 0x10000,
+             ws_bytes=1 << 20, stream=None)
+    a.update(over)
+    return a
+
+
+def _call_prefill(lib, **over):
+    a = _prefill_args(**over)
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.gdn_prefill(v(a["q"]), v(a["k"]), v(a["v"]), a["io"], v(a["a"]), v(a["b"]),
+                           v(a["A_log"]), v(a["dt_bias"]), v(a["S0"]), v(a["cu"]), a["N"], a["T"],
+                           a["H_qk"], a["H_v"], a["d_k"], a["d_v"], a["scale"], v(a["o"]),
+                           v(a["Sf"]), v(a["ws"]), a["ws_bytes"], v(a["stream"]))
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(io=7), 1),
+    (dict(H_v=3), 1),                   # not a multiple of H_qk
+    (dict(H_qk=0), 1),
+    (dict(d_k=96, d_v=96), 2),
+    (dict(d_k=64, d_v=128), 2),
+    (dict(N=-1), 1),
+    (dict(T=-5), 1),
+    (dict(N=0, T=4), 1),
+    (dict(scale=math.nan), 1),
+    (dict(scale=math.inf), 1),
+    (dict(q=None), 1),
+    (dict(cu=None), 1),
+    (dict(o=None), 1),
+    (dict(A_log=None), 1),
+    (dict(q=F + 8), 1),                  # misaligned
+    (dict(o=F + 4), 1),
+    (dict(S0=F + 2), 1),
+    (dict(Sf=F + 12), 1),
+    (dict(a=F + 2), 1),
+    (dict(ws_bytes=100), 3),
+    (dict(ws=None), 3),
+    (dict(ws=F + 16), 3),               # workspace must be 256-byte aligned
+])
+def test_prefill_rejects(lib, over, code):
+    assert _call_prefill(lib, **over) == code
+
+
+def test_prefill_empty_batch_is_noop(lib):
+    # N = 0, T = 0: nothing to do, no CUDA call, success
+    assert _call_prefill(lib, N=0, T=0, q=None, k=None, v=None, o=None, ws=None,
+                         ws_bytes=0) == 0
+
+
+def _call_decode(lib, **over):
+    a = dict(q=F, k=F + 0x1000, v=F + 0x2000, io=gdn.GDN_BF16, a=F + 0x3000, b=F + 0x4000,
+             A_log=F + 0x5000, dt_bias=F + 0x6000, S=F + 0x10000, N=8, H_qk=2, H_v=4, d_k=128,
+             d_v=128, scale=1.0, o=F + 0x8000, stream=None)
+    a.update(over)
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.gdn_decode_step(v(a["q"]), v(a["k"]), v(a["v"]), a["io"], v(a["a"]), v(a["b"]),
+                               v(a["A_log"]), v(a["dt_bias"]), v(a["S"]), a["N"], a["H_qk"],
+                               a["H_v"], a["d_k"], a["d_v"], a["scale"], v(a["o"]),
+                               v(a["stream"]))
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(io=-1), 1), (dict(H_v=5), 1), (dict(d_k=32, d_v=32), 2), (dict(N=-2), 1),
+    (dict(S=None), 1), (dict(S=F + 4), 1), (dict(q=F + 2), 1), (dict(b=None), 1),
+    (dict(scale=math.nan), 1),
+])
+def test_decode_rejects(lib, over, code):
+    assert _call_decode(lib, **over) == code
+
+
+def test_decode_zero_sequences_is_noop(lib):
+    assert _call_decode(lib, N=0) == 0
+
+
+def test_gates_rejects(lib):
+    v = ctypes.c_void_p
+    g = lib.gdn_gates
+    assert g(v(F), v(F), v(F), v(F), v(F), -1, 4, 4, v(F), None, None, None) == 1
+    assert g(v(F), v(F), v(F), v(F), v(F), 1, 4, 0, v(F), None, None, None) == 1
+    assert g(None, v(F), v(F), v(F), v(F), 1, 4, 4, v(F), None, None, None) == 1
+    assert g(v(F + 2), v(F), v(F), v(F), v(F), 1, 4, 4, v(F), None, None, None) == 1
+    # nothing asked for: success without a launch
+    assert g(v(F), v(F), v(F), v(F), v(F), 1, 4, 4, None, None, None, None) == 0
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    saved = gdn._lib
+    try:
+        gdn._lib = None
+        with pytest.raises(RuntimeError, match="libgdn.so not found"):
+            gdn.load_library(str(tmp_path / "missing.so"))
+    finally:
+        gdn._lib = saved

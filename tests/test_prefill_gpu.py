@@ -1,0 +1,166 @@
+"""gdn_prefill (gate prologue + chunk kernel) against the fp64 oracle.
+
+Tolerance (max|gpu - oracle| / max|oracle|, on o and on the final states
+separately): 1e-4 with fp32 q/k/v/o, 1e-2 with bf16 q/k/v/o. The oracle reads
+the same bf16-rounded inputs, upcast exactly.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_attention_sequence_delta_b200 import gdn_prefill, gdn_sync_status
+from linear_attention_sequence_delta_b200.inputs import WORKLOADS, make_prefill_inputs
+from tests.parity_util import TOL_BF16, TOL_FP32, oracle_prefill_heads, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(P, scale=1.0):
+    Pd = P.to("cuda")
+    o, Sf = gdn_prefill(Pd.q, Pd.k, Pd.v, Pd.a, Pd.b, Pd.A_log, Pd.dt_bias, Pd.cu_seqlens,
+                        Pd.initial_state, scale=scale)
+    assert gdn_sync_status() == 0
+    return o, Sf
+
+
+def _full_oracle(P, scale=1.0):
+    return oracle.forward(P.q, P.k, P.v, P.a, P.b, P.A_log, P.dt_bias,
+                          P.cu_seqlens.cpu().numpy(), P.initial_state, scale=scale)
+
+
+def _check(P, tol, scale=1.0):
+    o, Sf = _run(P, scale)
+    o_ref, S_ref = _full_oracle(P, scale)
+    eo, es = rel_err(o, o_ref), rel_err(Sf, S_ref)
+    assert eo <= tol and es <= tol, (eo, es)
+    return eo, es
+
+
+def test_tiny_fp32_workload():
+    """B=1, T=256, 2 QK / 4 V heads, d=64, fp32 I/O: the 1e-4 precision mode."""
+    P = make_prefill_inputs(**WORKLOADS["tiny_fp32"], seed=0)
+    _check(P, TOL_FP32)
+
+
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 127, 200])
+def test_ragged_lengths(T, io):
+    P = make_prefill_inputs([T], H_qk=2, H_v=4, d_k=128, d_v=128, io_dtype=io, state_std=0.05,
+                            seed=T)
+    _check(P, TOL_FP32 if io == torch.float32 else TOL_BF16)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_varlen_with_empty_sequences(d):
+    P = make_prefill_inputs([70, 0, 1, 64, 129, 0, 5], H_qk=1, H_v=3, d_k=d, d_v=d,
+                            io_dtype=torch.float32, state_std=0.1, seed=11)
+    _check(P, TOL_FP32)
+
+
+def test_slow_decay_long_carry():
+    """A_log = -4 (alpha near 0.98 per token) keeps state alive across many chunks."""
+    P = make_prefill_inputs([777], H_qk=2, H_v=4, d_k=128, d_v=128, io_dtype=torch.float32,
+                            seed=3)
+    P.A_log.fill_(-4.0)
+    _check(P, TOL_FP32)
+    Pb = make_prefill_inputs([777], H_qk=2, H_v=4, d_k=128, d_v=128, seed=3)
+    Pb.A_log.fill_(-4.0)
+    _check(Pb, TOL_BF16)
+
+
+def test_pages_init_distribution_and_strong_writes():
+    """A_log = log U(0, 16) as in the pages' parameter init, beta near 1 (b = 4)."""
+    P = make_prefill_inputs([300], H_qk=2, H_v=4, d_k=128, d_v=128, io_dtype=torch.float32,
+                            seed=4)
+    g = torch.Generator().manual_seed(9)
+    P.A_log.copy_(torch.log(torch.rand(4, generator=g) * 16 + 1e-3))
+    P.b.fill_(4.0)
+    _check(P, TOL_FP32)
+
+
+def test_extreme_gates():
+    """alpha = 1 (a -> -inf), beta = 0 (b -> -inf) and alpha = 0 (A_log = 100) tokens."""
+    P = make_prefill_inputs([150], H_qk=1, H_v=3, d_k=64, d_v=64, io_dtype=torch.float32,
+                            state_std=0.1, seed=8)
+    P.a[10:20, 0] = -1e30
+    P.b[30:40, 1] = -1e30
+    P.A_log[2] = 100.0
+    _check(P, TOL_FP32)
+
+
+def test_scale_and_final_state_alias():
+    P = make_prefill_inputs([100, 37], H_qk=2, H_v=4, d_k=64, d_v=64, io_dtype=torch.float32,
+                            state_std=0.1, seed=21)
+    Pd = P.to("cuda")
+    S = Pd.initial_state.clone()
+    o, Sf = gdn_prefill(Pd.q, Pd.k, Pd.v, Pd.a, Pd.b, Pd.A_log, Pd.dt_bias, Pd.cu_seqlens, S,
+                        scale=0.125, final_state=S)
+    assert Sf.data_ptr() == S.data_ptr()
+    o_ref, S_ref = _full_oracle(P, scale=0.125)
+    assert rel_err(o, o_ref) <= TOL_FP32 and rel_err(S, S_ref) <= TOL_FP32
+
+
+def test_split_prefill_resume_equals_single():
+    P = make_prefill_inputs([300], H_qk=2, H_v=4, d_k=128, d_v=128, io_dtype=torch.float32,
+                            seed=5)
+    Pd = P.to("cuda")
+    args = lambda s: (Pd.q[s], Pd.k[s], Pd.v[s], Pd.a[s], Pd.b[s], Pd.A_log, Pd.dt_bias)
+    cu = lambda n: torch.tensor([0, n], dtype=torch.int32, device="cuda")
+    o, Sf = gdn_prefill(*args(slice(0, 300)), cu(300))
+    o1, S1 = gdn_prefill(*args(slice(0, 130)), cu(130))
+    o2, S2 = gdn_prefill(*args(slice(130, 300)), cu(170), S1)
+    torch.cuda.synchronize()
+    assert rel_err(torch.cat([o1, o2]), o.cpu().numpy()) <= 1e-5
+    assert rel_err(S2, Sf.cpu().numpy()) <= 1e-5
+
+
+def test_bad_seqlens_reported_on_device():
+    P = make_prefill_inputs([64, 64], H_qk=1, H_v=2, d_k=64, d_v=64, io_dtype=torch.float32)
+    Pd = P.to("cuda")
+    bad = torch.tensor([0, 100, 90], dtype=torch.int32, device="cuda")  # decreasing
+    gdn_prefill(Pd.q, Pd.k, Pd.v, Pd.a, Pd.b, Pd.A_log, Pd.dt_bias, bad)
+    assert gdn_sync_status() == 6
+    assert gdn_sync_status() == 0  # cleared
+
+
+# ---------------------------------------------------------- full workloads ----
+
+def test_prefill_35b_layer_full():
+    """B=1, T=4096, 16 QK / 32 V heads, d=128, bf16: every output against the oracle."""
+    P = make_prefill_inputs(**WORKLOADS["prefill_35b"], seed=0)
+    _check(P, TOL_BF16)
+
+
+def test_prefill_397b_long_sampled():
+    """B=4, T=16384, 16 QK / 64 V heads: the full launch, sampled (sequence, head) units."""
+    P = make_prefill_inputs(**WORKLOADS["prefill_397b_long"], seed=0, device="cuda")
+    o, Sf = gdn_prefill(P.q, P.k, P.v, P.a, P.b, P.A_log, P.dt_bias, P.cu_seqlens, None)
+    assert gdn_sync_status() == 0
+    units = [(0, 0), (1, 17), (3, 63)]
+    ref = {}
+    for n, h in units:
+        ref.update(oracle_prefill_heads(P, [h], seqs=[n]))
+    cu = P.cu_seqlens.cpu().tolist()
+    for (n, h), (o_ref, S_ref) in ref.items():
+        assert rel_err(o[cu[n]:cu[n + 1], h], o_ref) <= TOL_BF16
+        assert rel_err(Sf[n, h], S_ref) <= TOL_BF16
+    assert torch.isfinite(o.float()).all() and torch.isfinite(Sf).all()
+
+
+def test_varlen_64_sampled():
+    """64 sequences, lengths U[128, 8192], nonzero initial states: sampled units."""
+    P = make_prefill_inputs(**WORKLOADS["varlen_64"], seed=0, device="cuda")
+    o, Sf = gdn_prefill(P.q, P.k, P.v, P.a, P.b, P.A_log, P.dt_bias, P.cu_seqlens,
+                        P.initial_state)
+    assert gdn_sync_status() == 0
+    cu = P.cu_seqlens.cpu().tolist()
+    lens = np.diff(cu)
+    seqs = [int(np.argmin(lens)), int(np.argmax(lens)), 31]
+    ref = oracle_prefill_heads(P, [0, 13, 31], seqs=seqs)
+    for (n, h), (o_ref, S_ref) in ref.items():
+        assert rel_err(o[cu[n]:cu[n + 1], h], o_ref) <= TOL_BF16
+        assert rel_err(Sf[n, h], S_ref) <= TOL_BF16
+    assert torch.isfinite(o.float()).all() and torch.isfinite(Sf).all()
