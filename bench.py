@@ -181,8 +181,8 @@ def run_ours(args):
         # ---- decode: 1000 consecutive steps on the 397B-A17B GDN shape ----
         dec = None
         if not args.no_decode:
-            D = make_decode_inputs(steps=args.decode_steps, seed=rank, device=dev,
-                                   **DECODE_WORKLOAD)
+            dw = dict(DECODE_WORKLOAD, num_seqs=args.decode_seqs)
+            D = make_decode_inputs(steps=args.decode_steps, seed=rank, device=dev, **dw)
             od = torch.empty_like(D.v[0])
             for t in range(min(3, args.decode_steps)):  # warm-up on a copy of the state
                 gdn.gdn_decode_step(D.q[t], D.k[t], D.v[t], D.a[t], D.b[t], D.A_log, D.dt_bias,
@@ -219,7 +219,44 @@ def run_ours(args):
     achieved = byts / (ms / 1e3) / 1e9
     t_roof = max(byts / (hbm * 1e9), flops / (tc_burst * 1e12))
 
-    # ---- e2e through the public API from pinned host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        e2e = _e2e(args, P, o, Sf, ws, dev, stream)
+
+    line = {
+        "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "prefill_35b: B=1, T=4096, H_qk=16, H_v=32, d=128, bf16 q/k/v/o, "
+                               "fp32 gates/state, zero initial state, final state written",
+                   "global_batch": ws, "seq_len": T, "parallelism": f"replicas x{ws}",
+                   "l2": "flushed (512 MiB write) before every timed step"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None, "algorithmic_bytes": byts,
+                     "kernel": "gdn_prefill (gate prologue + chunk kernel)",
+                     "peak_source": peak_src,
+                     "tensor": {"algorithmic_flops": flops, "achieved_tflops":
+                                flops / (ms / 1e3) / 1e12, "peak_tflops": tc_burst,
+                                "frac": flops / (ms / 1e3) / 1e12 / tc_burst},
+                     "frac_of_slower_roof": t_roof / (ms / 1e3)},
+        "e2e": e2e,
+        "gpu_launches": 2 * args.steps + (args.decode_steps if dec else 0),
+        "clocks": clocks.summary(),
+        "decode": dec,
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(P)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def _e2e(args, P, o, Sf, ws, dev, stream):
+    from linear_attention_sequence_delta_b200 import gdn
+    T = P.q.shape[0]
     host = {k_: getattr(P, k_).cpu().pin_memory() for k_ in
             ("q", "k", "v", "a", "b", "A_log", "dt_bias", "cu_seqlens")}
     o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
@@ -245,37 +282,8 @@ def run_ours(args):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / args.steps, ws, dev)
-
-    line = {
-        "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": ws,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic",
-        "config": {"workload": "prefill_35b: B=1, T=4096, H_qk=16, H_v=32, d=128, bf16 q/k/v/o, "
-                               "fp32 gates/state, zero initial state, final state written",
-                   "global_batch": ws, "seq_len": T, "parallelism": f"replicas x{ws}",
-                   "l2": "flushed (512 MiB write) before every timed step"},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": None, "algorithmic_bytes": byts,
-                     "kernel": "gdn_prefill (gate prologue + chunk kernel)",
-                     "peak_source": peak_src,
-                     "tensor": {"algorithmic_flops": flops, "achieved_tflops":
-                                flops / (ms / 1e3) / 1e12, "peak_tflops": tc_burst,
-                                "frac": flops / (ms / 1e3) / 1e12 / tc_burst},
-                     "frac_of_slower_roof": t_roof / (ms / 1e3)},
-        "e2e": {"value": ws * T / (e2e_ms / 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": 2 * args.steps + (args.decode_steps if dec else 0),
-        "clocks": clocks.summary(),
-        "decode": dec,
-    }
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(P)
-    if ws > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+    return {"value": ws * T / (e2e_ms / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
 
 def cpu_baseline(P, heads=None):
@@ -339,8 +347,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--decode-seqs", type=int, default=256,
+                    help="sequences per decode step (256 = the decode workload; smaller values "
+                         "only for profiling captures)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
