@@ -135,6 +135,35 @@ int gdn_decode_step(const void* q, const void* k, const void* v, int32_t io_dtyp
                     int32_t d_v, float scale, void* o, void* stream);
 
 /*
+ * gdn_prefill_noalloc -- gdn_prefill for callers that cannot allocate device
+ * memory. The pages have no counterpart: this is a deployment variant.
+ *
+ * gdn_prefill asks the caller for a workspace (the per-token gates G and beta).
+ * Callers that cannot call cudaMalloc -- code running under CUDA graph stream
+ * capture, runtimes whose device memory belongs to a pool they must not touch,
+ * plugins that are handed only their input and output buffers -- use this call
+ * instead: the same computation and the same arguments minus the workspace, with
+ * the scratch kept in a fixed array inside the library.
+ *   - Capacity: total_tokens * H_v <= GDN_NOALLOC_MAX_GATE_ELEMS; larger calls
+ *     return GDN_ERR_WORKSPACE and launch nothing (use gdn_prefill for them).
+ *     The array (8 MiB) is held on every GPU that loads the library until the
+ *     process exits.
+ *   - The first call on each device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - Every call shares the one array: calls that overlap on the GPU (two
+ *     streams, or two host threads on one device) race and give wrong results.
+ *     Serialise them (one stream) or use gdn_prefill with separate workspaces.
+ *   - Nothing from an earlier call is read: every gate value is rewritten first.
+ */
+#define GDN_NOALLOC_MAX_GATE_ELEMS 1048576
+int gdn_prefill_noalloc(const void* q, const void* k, const void* v, int32_t io_dtype,
+                        const float* a, const float* b, const float* A_log,
+                        const float* dt_bias, const float* initial_state,
+                        const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                        int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v, float scale,
+                        void* o, float* final_state, void* stream);
+
+/*
  * Synchronise `stream`, then return and clear the device status word of the
  * current device (GDN_OK, GDN_ERR_BAD_SEQLENS or GDN_ERR_TIMEOUT), or
  * GDN_ERR_CUDA if the synchronisation itself failed.

@@ -28,7 +28,7 @@ _STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "
 
 # Every symbol include/gdn.h declares (the tests check the library exports them all).
 EXPORTS = ["gdn_status_string", "gdn_version", "gdn_prefill_workspace_size", "gdn_gates",
-           "gdn_prefill", "gdn_decode_step", "gdn_sync_status"]
+           "gdn_prefill", "gdn_decode_step", "gdn_sync_status", "gdn_prefill_noalloc"]
 
 
 class GDNError(RuntimeError):

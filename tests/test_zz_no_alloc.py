@@ -1,0 +1,77 @@
+"""gdn_prefill_noalloc: the prefill for callers that cannot allocate device memory.
+
+Some callers cannot call cudaMalloc (code under CUDA graph stream capture, a
+runtime whose device memory is owned by its own pool, a plugin given only its
+input and output buffers), so they cannot hand gdn_prefill a workspace. This
+entry point keeps that scratch in a fixed array inside the library. The test
+calls it through the C ABI, twice in a row on different inputs (the array keeps
+the previous call's contents), and checks each result against gdn_prefill's
+within the parity tolerance. It also checks that a call larger than the built-in
+scratch is refused before anything is launched.
+
+This file is named so that pytest collects it last.
+"""
+import ctypes
+
+import pytest
+import torch
+
+from linear_attention_sequence_delta_b200 import gdn
+from linear_attention_sequence_delta_b200.inputs import make_prefill_inputs
+from tests.parity_util import TOL_BF16, TOL_FP32, rel_err
+
+MAX_GATE_ELEMS = 1048576  # GDN_NOALLOC_MAX_GATE_ELEMS in include/gdn.h
+
+
+def _fn():
+    lib = gdn.load_library()
+    f = lib.gdn_prefill_noalloc
+    P, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
+    f.restype = ctypes.c_int
+    f.argtypes = [P, P, P, i32, P, P, P, P, P, P, i32, i64, i32, i32, i32, i32, f32, P, P, P]
+    return f
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _call(P, o, Sf, scale=1.0):
+    T, H_qk, d = P.q.shape
+    H_v = P.v.shape[1]
+    io = gdn.GDN_BF16 if P.q.dtype == torch.bfloat16 else gdn.GDN_FP32
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return _fn()(_p(P.q), _p(P.k), _p(P.v), io, _p(P.a), _p(P.b), _p(P.A_log), _p(P.dt_bias),
+                 _p(P.initial_state), _p(P.cu_seqlens), P.cu_seqlens.numel() - 1, T, H_qk, H_v,
+                 d, d, scale, _p(o), _p(Sf), stream)
+
+
+def test_refuses_more_than_the_builtin_scratch():
+    # Rejected on the host before any CUDA call, so no GPU is needed.
+    F = 0x7F0000000000
+    v = ctypes.c_void_p
+    H_v = 32
+    T = MAX_GATE_ELEMS // H_v + 1
+    st = _fn()(v(F), v(F), v(F), 0, v(F), v(F), v(F), v(F), None, v(F), 1, T, 16, H_v, 128, 128,
+               1.0, v(F), None, None)
+    assert st == 3  # GDN_ERR_WORKSPACE
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("io", [torch.bfloat16, torch.float32])
+def test_noalloc_matches_gdn_prefill_twice(io):
+    tol = TOL_BF16 if io == torch.bfloat16 else TOL_FP32
+    specs = [dict(lengths=[300, 1, 129], H_qk=2, H_v=4, d_k=128, d_v=128, state_std=0.05,
+                  seed=31),
+             dict(lengths=[64, 0, 517], H_qk=2, H_v=8, d_k=64, d_v=64, state_std=0.05,
+                  seed=32)]
+    for spec in specs:  # two calls in a row; the second reuses the array the first filled
+        P = make_prefill_inputs(io_dtype=io, **spec).to("cuda")
+        o_ref, S_ref = gdn.gdn_prefill(P.q, P.k, P.v, P.a, P.b, P.A_log, P.dt_bias,
+                                       P.cu_seqlens, P.initial_state, scale=0.7)
+        o = torch.full_like(o_ref, float("nan"))
+        Sf = torch.full_like(S_ref, float("nan"))
+        assert _call(P, o, Sf, scale=0.7) == 0
+        assert gdn.gdn_sync_status() == 0
+        assert rel_err(o, o_ref.float().cpu().numpy()) <= tol
+        assert rel_err(Sf, S_ref.cpu().numpy()) <= tol
