@@ -110,6 +110,8 @@ int gdn_gates(const float* a, const float* b, const float* A_log, const float* d
  *                     may alias initial_state (each state is read before it
  *                     is written, by the same block)
  *   workspace         >= gdn_prefill_workspace_size(...) bytes, 256-byte aligned
+ *                     (the tensor-core path computes the gates in-kernel and
+ *                     leaves the workspace untouched)
  * Empty sequences are allowed: their final state equals their initial state.
  */
 int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
@@ -118,6 +120,20 @@ int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
                 int64_t total_tokens, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
                 float scale, void* o, float* final_state, void* workspace,
                 size_t workspace_bytes, void* stream);
+
+/*
+ * Process-wide choice of the gdn_prefill implementation (for A/B comparison and
+ * tests; the default is GDN_IMPL_AUTO):
+ *   GDN_IMPL_AUTO         tensor cores (tcgen05) for bf16 I/O with d = 128, the
+ *                         fp32 CUDA-core kernel otherwise (fp32 I/O, d = 64);
+ *   GDN_IMPL_CUDA_CORE    the fp32 CUDA-core kernel for every call;
+ *   GDN_IMPL_TENSOR_CORE  tensor cores only; gdn_prefill then returns
+ *                         GDN_ERR_UNSUPPORTED for shapes/types they do not cover.
+ * Returns the previous setting, or -GDN_ERR_INVALID_ARG for an unknown value.
+ * Not synchronised with calls in flight on other host threads.
+ */
+enum { GDN_IMPL_AUTO = 0, GDN_IMPL_CUDA_CORE = 1, GDN_IMPL_TENSOR_CORE = 2 };
+int gdn_set_prefill_impl(int32_t impl);
 
 /*
  * gdn_decode_step -- one token for each of N sequences, the state updated in

@@ -15,6 +15,7 @@ __device__ int g_status_word;
 
 namespace {
 constexpr int kMaxDevices = 64;
+std::atomic<int> g_prefill_impl{GDN_IMPL_AUTO};
 std::atomic<int*> g_status_ptr[kMaxDevices];
 std::mutex g_status_mu;
 
@@ -120,9 +121,17 @@ int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
     if (workspace_bytes < need || (need > 0 && !workspace)) return GDN_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return GDN_ERR_WORKSPACE;
 
+    const int impl = g_prefill_impl.load(std::memory_order_relaxed);
+    const bool tc_ok = io_dtype == GDN_BF16 && d_k == 128;
+    if (impl == GDN_IMPL_TENSOR_CORE && !tc_ok) return GDN_ERR_UNSUPPORTED;
     int* st = device_status_ptr();
     if (!st) return GDN_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
+    if (tc_ok && impl != GDN_IMPL_CUDA_CORE) {
+        return to_status(launch_prefill_tc(q, k, v, a, b, A_log, dt_bias, initial_state,
+                                           cu_seqlens, num_seqs, total_tokens, H_qk, H_v, scale,
+                                           o, final_state, st, s));
+    }
     float* G = static_cast<float*>(workspace);
     float* beta = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                            gate_bytes(total_tokens, H_v));
@@ -155,6 +164,12 @@ int gdn_decode_step(const void* q, const void* k, const void* v, int32_t io_dtyp
     if (!aligned(a, 4) || !aligned(b, 4)) return GDN_ERR_INVALID_ARG;
     return to_status(launch_decode(q, k, v, io_dtype, a, b, A_log, dt_bias, state, num_seqs,
                                    H_qk, H_v, d_k, scale, o, (cudaStream_t)stream));
+}
+
+int gdn_set_prefill_impl(int32_t impl) {
+    if (impl != GDN_IMPL_AUTO && impl != GDN_IMPL_CUDA_CORE && impl != GDN_IMPL_TENSOR_CORE)
+        return -GDN_ERR_INVALID_ARG;
+    return g_prefill_impl.exchange(impl);
 }
 
 int gdn_sync_status(void* stream) {

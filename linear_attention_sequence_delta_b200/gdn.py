@@ -28,7 +28,9 @@ _STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "
 
 # Every symbol include/gdn.h declares (the tests check the library exports them all).
 EXPORTS = ["gdn_status_string", "gdn_version", "gdn_prefill_workspace_size", "gdn_gates",
-           "gdn_prefill", "gdn_decode_step", "gdn_sync_status", "gdn_prefill_noalloc"]
+           "gdn_prefill", "gdn_decode_step", "gdn_sync_status", "gdn_prefill_noalloc",
+           "gdn_set_prefill_impl"]
+GDN_IMPL_AUTO, GDN_IMPL_CUDA_CORE, GDN_IMPL_TENSOR_CORE = 0, 1, 2
 
 
 class GDNError(RuntimeError):
@@ -66,6 +68,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                     P]
     lib.gdn_sync_status.restype = ctypes.c_int
     lib.gdn_sync_status.argtypes = [P]
+    lib.gdn_set_prefill_impl.restype = ctypes.c_int
+    lib.gdn_set_prefill_impl.argtypes = [i32]
     _lib = lib
     return lib
 
@@ -170,6 +174,14 @@ def gdn_decode_step(q, k, v, a, b, A_log, dt_bias, state, *, scale: float = 1.0,
                              _ptr(o), _stream(q.device))
     _check(st, "gdn_decode_step")
     return o
+
+
+def set_prefill_impl(impl: int) -> int:
+    """Choose the gdn_prefill implementation process-wide; returns the previous choice."""
+    prev = int(load_library().gdn_set_prefill_impl(int(impl)))
+    if prev < 0:
+        raise GDNError(-prev, "gdn_set_prefill_impl")
+    return prev
 
 
 def gdn_sync_status(device=None) -> int:

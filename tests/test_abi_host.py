@@ -150,3 +150,10 @@ def test_binding_fails_loudly_without_library(tmp_path):
             gdn.load_library(str(tmp_path / "missing.so"))
     finally:
         gdn._lib = saved
+
+
+def test_set_prefill_impl(lib):
+    assert lib.gdn_set_prefill_impl(1) == 0
+    assert lib.gdn_set_prefill_impl(2) == 1
+    assert lib.gdn_set_prefill_impl(7) == -1      # invalid: unchanged
+    assert lib.gdn_set_prefill_impl(0) == 2

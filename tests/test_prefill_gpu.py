@@ -164,3 +164,41 @@ def test_varlen_64_sampled():
         assert rel_err(o[cu[n]:cu[n + 1], h], o_ref) <= TOL_BF16
         assert rel_err(Sf[n, h], S_ref) <= TOL_BF16
     assert torch.isfinite(o.float()).all() and torch.isfinite(Sf).all()
+
+
+@pytest.fixture
+def impl_switch():
+    from linear_attention_sequence_delta_b200 import gdn
+    prev = gdn.set_prefill_impl(gdn.GDN_IMPL_AUTO)
+    yield gdn
+    gdn.set_prefill_impl(prev)
+
+
+@pytest.mark.parametrize("impl", ["cuda_core", "tensor_core"])
+@pytest.mark.parametrize("lengths", [[1], [63], [64], [65], [127], [200], [5, 0, 130, 64]])
+def test_bf16_both_implementations(impl_switch, impl, lengths):
+    g = impl_switch
+    g.set_prefill_impl(g.GDN_IMPL_CUDA_CORE if impl == "cuda_core" else g.GDN_IMPL_TENSOR_CORE)
+    P = make_prefill_inputs(lengths, H_qk=2, H_v=4, d_k=128, d_v=128, state_std=0.05,
+                            seed=sum(lengths) + 7)
+    _check(P, TOL_BF16)
+
+
+def test_tensor_core_stress_gates(impl_switch):
+    """Slow decay, strong writes and extreme gates through the tensor-core path."""
+    g = impl_switch
+    g.set_prefill_impl(g.GDN_IMPL_TENSOR_CORE)
+    P = make_prefill_inputs([500], H_qk=1, H_v=4, d_k=128, d_v=128, state_std=0.1, seed=12)
+    P.A_log[0] = -4.0                 # alpha near 0.98: long carry across chunks
+    P.b[:, 1] = 4.0                   # beta near 1
+    P.a[100:130, 2] = -1e30           # alpha = 1 run
+    P.A_log[3] = 100.0                # alpha = 0 every token
+    _check(P, TOL_BF16)
+
+
+def test_tensor_core_rejects_fp32(impl_switch):
+    g = impl_switch
+    g.set_prefill_impl(g.GDN_IMPL_TENSOR_CORE)
+    P = make_prefill_inputs([64], H_qk=1, H_v=1, d_k=128, d_v=128, io_dtype=torch.float32)
+    with pytest.raises(g.GDNError):
+        _run(P)
