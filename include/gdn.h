@@ -70,9 +70,12 @@ const char* gdn_status_string(int status);
 int gdn_version(void);
 
 /*
- * Bytes of device workspace gdn_prefill needs for these sizes (the per-token
- * chunk-cumulative log-decay G and beta, fp32 [T, H_v] each, plus alignment).
- * Returns 0 for invalid sizes.
+ * Bytes of device workspace gdn_prefill needs for these sizes. For d = 128 it
+ * covers the tensor-core path: the chunk offsets of the sequences plus one
+ * 17,664-byte record (the chunk's T and P matrices and per-token factors) per
+ * (64-token chunk, V head), i.e. about 276 bytes per token and V head (with one
+ * extra chunk per sequence); for d = 64 (CUDA-core path) it is the per-token G
+ * and beta, fp32 [T, H_v] each. Returns 0 for invalid sizes.
  */
 size_t gdn_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t H_qk,
                                   int32_t H_v, int32_t d_k, int32_t d_v);
@@ -110,8 +113,8 @@ int gdn_gates(const float* a, const float* b, const float* A_log, const float* d
  *                     may alias initial_state (each state is read before it
  *                     is written, by the same block)
  *   workspace         >= gdn_prefill_workspace_size(...) bytes, 256-byte aligned
- *                     (the tensor-core path computes the gates in-kernel and
- *                     leaves the workspace untouched)
+ *                     (the tensor-core path keeps its per-chunk intermediates
+ *                     there; they are fully rewritten on every call)
  * Empty sequences are allowed: their final state equals their initial state.
  */
 int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
@@ -124,8 +127,9 @@ int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
 /*
  * Process-wide choice of the gdn_prefill implementation (for A/B comparison and
  * tests; the default is GDN_IMPL_AUTO):
- *   GDN_IMPL_AUTO         tensor cores (tcgen05) for bf16 I/O with d = 128, the
- *                         fp32 CUDA-core kernel otherwise (fp32 I/O, d = 64);
+ *   GDN_IMPL_AUTO         tensor cores (tcgen05) for bf16 I/O with d = 128 and at
+ *                         most 16 V heads per QK head, the fp32 CUDA-core
+ *                         kernel otherwise (fp32 I/O, d = 64);
  *   GDN_IMPL_CUDA_CORE    the fp32 CUDA-core kernel for every call;
  *   GDN_IMPL_TENSOR_CORE  tensor cores only; gdn_prefill then returns
  *                         GDN_ERR_UNSUPPORTED for shapes/types they do not cover.

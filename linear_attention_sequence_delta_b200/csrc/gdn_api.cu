@@ -78,7 +78,10 @@ size_t gdn_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_
                                   int32_t H_v, int32_t d_k, int32_t d_v) {
     if (num_seqs < 0 || total_tokens < 0) return 0;
     if (check_heads(H_qk, H_v, d_k, d_v) != GDN_OK) return 0;
-    return 2 * gate_bytes(total_tokens, H_v);
+    const size_t simt = 2 * gate_bytes(total_tokens, H_v);
+    if (d_k != 128) return simt;
+    const size_t tc = prefill_tc_workspace_bytes(num_seqs, total_tokens, H_v);
+    return tc > simt ? tc : simt;
 }
 
 int gdn_gates(const float* a, const float* b, const float* A_log, const float* dt_bias,
@@ -122,7 +125,8 @@ int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
     if (!aligned(workspace, 256)) return GDN_ERR_WORKSPACE;
 
     const int impl = g_prefill_impl.load(std::memory_order_relaxed);
-    const bool tc_ok = io_dtype == GDN_BF16 && d_k == 128;
+    const bool tc_ok =
+        io_dtype == GDN_BF16 && d_k == 128 && prefill_tc_supported(H_qk, H_v);
     if (impl == GDN_IMPL_TENSOR_CORE && !tc_ok) return GDN_ERR_UNSUPPORTED;
     int* st = device_status_ptr();
     if (!st) return GDN_ERR_CUDA;
@@ -130,7 +134,7 @@ int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
     if (tc_ok && impl != GDN_IMPL_CUDA_CORE) {
         return to_status(launch_prefill_tc(q, k, v, a, b, A_log, dt_bias, initial_state,
                                            cu_seqlens, num_seqs, total_tokens, H_qk, H_v, scale,
-                                           o, final_state, st, s));
+                                           o, final_state, workspace, st, s));
     }
     float* G = static_cast<float*>(workspace);
     float* beta = reinterpret_cast<float*>(static_cast<char*>(workspace) +

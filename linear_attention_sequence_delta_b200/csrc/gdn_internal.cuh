@@ -87,11 +87,15 @@ cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, int
                                 int32_t H_v, int32_t d, float scale, void* o, float* S_final,
                                 int* status, cudaStream_t s);
 
-// Tensor-core prefill (bf16 I/O, d = 128); the gate prologue is fused in.
+// Tensor-core prefill (bf16 I/O, d = 128): chunk offsets, the state-independent
+// prep kernel, then the chain kernel. The workspace holds the chunk offsets and
+// one record (T, P and per-token factors) per (chunk, V head).
+size_t prefill_tc_workspace_bytes(int32_t N, int64_t T, int32_t H_v);
+bool prefill_tc_supported(int32_t H_qk, int32_t H_v);
 cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const float* a,
                               const float* b, const float* A_log, const float* dt_bias,
                               const float* S0, const int32_t* cu_seqlens, int32_t N, int64_t T,
                               int32_t H_qk, int32_t H_v, float scale, void* o, float* S_final,
-                              int* status, cudaStream_t s);
+                              void* workspace, int* status, cudaStream_t s);
 
 }  // namespace gdn
