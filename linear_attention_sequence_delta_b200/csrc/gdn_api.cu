@@ -78,6 +78,7 @@ size_t gdn_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_
                                   int32_t H_v, int32_t d_k, int32_t d_v) {
     if (num_seqs < 0 || total_tokens < 0) return 0;
     if (check_heads(H_qk, H_v, d_k, d_v) != GDN_OK) return 0;
+    if (num_seqs == 0) return 0;  // an empty batch launches nothing
     const size_t simt = 2 * gate_bytes(total_tokens, H_v);
     if (d_k != 128) return simt;
     const size_t tc = prefill_tc_workspace_bytes(num_seqs, total_tokens, H_v);

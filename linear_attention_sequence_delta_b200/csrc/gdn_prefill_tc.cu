@@ -38,7 +38,9 @@
 //                  with the 128x128 fp32 state resident in tensor memory (lane
 //                  i = value row i). A loader warp fills a 3-deep ring with the
 //                  raw K/Q/V rows (cp.async) and the prepared T/P/factors (one
-//                  bulk copy); four warps run the state-dependent steps. Every
+//                  bulk copy); eight warps (two per lane quarter, each owning
+//                  half the columns of its rows) run the state-dependent steps,
+//                  the state's decay rescale overlapping the first MMA. Every
 //                  A operand (the bf16 state, Y^T, Vn^T and the decay-scaled
 //                  Vn^T) is written to tensor memory by the threads owning
 //                  those rows, and V^T itself is produced in tensor memory by
@@ -523,7 +525,8 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
 }
 
 // ==================================== chain =======================================
-constexpr int kChainThreads = 160;   // warps 0-3 state chain, warp 4 loader
+constexpr int kChainThreads = 288;   // warps 0-7 state chain, warp 8 loader
+constexpr int kChain = 256;
 constexpr int kRing = 3;
 // shared memory map (bytes from a 1024-byte aligned base)
 constexpr uint32_t SLOT_KQ = 0;        // [2][128 rows][128 B] raw K then Q, sw128
@@ -539,12 +542,14 @@ constexpr size_t kChainSmem = CS_BAR + 128 + 1024;
 
 // tensor memory columns (512 allocated)
 constexpr uint32_t TM_S = 0;      // 128: state, fp32
-constexpr uint32_t TM_S0B = 128;  // 64: state as bf16 pairs (MMA A operand)
-constexpr uint32_t TM_D1 = 192;   // 128: S0 K^T | S0 Q^T; then Y^T as bf16 pairs in 192..223
+constexpr uint32_t TM_S0B = 128;  // 64: state as bf16 pairs (A operand); then Y^T pairs
+constexpr uint32_t TM_D1 = 192;   // 128: S0 K^T | S0 Q^T
 constexpr uint32_t TM_D34 = 320;  // 64: Vn^T, then (P Vn)^T
 constexpr uint32_t TM_DV = 384;   // 64: V^T; then Vn^T (384..415) and scaled Vn^T (416..447)
 constexpr uint32_t kTmemCols = 512;
 
+// Two warps share each TMEM lane quarter: warp w owns value rows 32 (w & 3) ..
+// + 31 and, of every 64- or 128-column quantity of those rows, the half w >> 2.
 __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
     const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
     const float* __restrict__ S0g, const int32_t* __restrict__ cu_seqlens,
@@ -557,7 +562,8 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
     uint64_t* empty = full + kRing;
     uint64_t* mbar = full + 2 * kRing;
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + CS_TMEM);
-    volatile int* s_err = reinterpret_cast<volatile int*>(sm + CS_ERR);
+    volatile int* s_err = reinterpret_cast<volatile int*>(sm + CS_ERR);       // chain warps
+    volatile int* s_lerr = reinterpret_cast<volatile int*>(sm + CS_ERR + 4);  // loader warp
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -581,12 +587,13 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
         }
         mbar_init(mbar, 1);
         *s_err = 0;
+        *s_lerr = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp < 4) {  // the 64x64 bf16 identity (B operand of the V^T MMA)
+    if (warp < 8) {  // the 64x64 bf16 identity (B operand of the V^T MMA)
 #pragma unroll
-        for (int it = 0; it < 4; ++it) {
-            const int idx = tid + 128 * it;  // 0..511
+        for (int it = 0; it < 2; ++it) {
+            const int idx = tid + kChain * it;  // 0..511
             const int row = idx >> 3, ch = idx & 7;
             uint4 w = make_uint4(0u, 0u, 0u, 0u);
             if ((row >> 3) == ch) (&w.x)[(row & 7) >> 1] = 0x3F80u << (16 * (row & 1));
@@ -599,17 +606,17 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ================================ loader =======================================
+        int issued = 0;
 #pragma unroll 1
         for (int c = 0; c < nchunks; ++c) {
             const int st = c % kRing;
             bool ok = true;
             if (c >= kRing)
                 ok = mbar_wait_bounded(&empty[st], ((c / kRing) - 1) & 1, kWaitCycles);
-            if (!ok) *s_err = 1;
-            __syncwarp();
-            if (*s_err) break;
+            if (!ok) *s_lerr = 1;
+            if (__any_sync(0xffffffffu, !ok || *s_err != 0)) break;  // uniform over the warp
             uint8_t* slot = sm + st * kSlotBytes;
             const int64_t t0 = s0 + (int64_t)c * kC;
             const int L = (int)min((int64_t)kC, s1 - t0);
@@ -633,15 +640,27 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
                             v + ((size_t)tok * H_v + h) * kD + ch * 8, live ? 16u : 0u);
             }
             cp_async_mbar_arrive_noinc(&full[st]);
+            issued = c + 1;
         }
         cp_async_commit();
         cp_async_wait<0>();
+        // Drain the record copies: the last phase of each slot has completed (at
+        // once on the normal path, where the chain consumed it) before the block
+        // may leave with nothing in flight into its shared memory.
+        if (lane == 0) {
+            for (int c = issued - 1; c >= 0 && c >= issued - kRing; --c)
+                if (!mbar_wait_bounded(&full[c % kRing], (c / kRing) & 1, kWaitCycles)) *s_lerr = 1;
+        }
+        __syncwarp();
     } else {
         // ================================ chain ========================================
-        const uint32_t ctl = tmem + ((uint32_t)(warp * 32) << 16);
-        const size_t sbase = ((size_t)n * H_v + h) * kD * kD + (size_t)tid * kD;
+        const int qd = warp & 3;              // TMEM lane quarter
+        const int hh = warp >> 2;             // column half
+        const int row = qd * 32 + lane;       // value row i = TMEM lane
+        const uint32_t ctl = tmem + ((uint32_t)(qd * 32) << 16);
+        const size_t sbase = ((size_t)n * H_v + h) * kD * kD + (size_t)row * kD + 64 * hh;
 #pragma unroll 1
-        for (int cb = 0; cb < 4; ++cb) {  // initial state -> TMEM
+        for (int cb = 0; cb < 2; ++cb) {  // initial state -> TMEM (this thread's 64 columns)
             float x[32];
             if (S0g) {
                 const float4* src = reinterpret_cast<const float4*>(S0g + sbase + 32 * cb);
@@ -654,7 +673,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
 #pragma unroll
                 for (int e = 0; e < 32; ++e) x[e] = 0.f;
             }
-            tmem_st32(ctl + TM_S + 32 * cb, x);
+            tmem_st32(ctl + TM_S + 64 * hh + 32 * cb, x);
         }
         tmem_wait_st();
 
@@ -663,9 +682,9 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
             const bool ok = mbar_wait_bounded(mbar, mphase, kWaitCycles);
             mphase ^= 1u;
             if (!ok) *s_err = 1;
-            named_bar_sync(1, 128);
+            const bool bad = named_bar_any(1, kChain, !ok);
             tc_fence_after();
-            return *s_err == 0;
+            return !bad;
         };
 
 #pragma unroll 1
@@ -674,38 +693,28 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
             const bool ok = mbar_wait_bounded(&full[st], (c / kRing) & 1, kWaitCycles);
             if (!ok) *s_err = 1;
             fence_proxy_async_smem();  // the loader's cp.async rows -> tensor core reads
-            named_bar_sync(1, 128);
-            if (*s_err) break;
+            if (named_bar_any(1, kChain, !ok)) break;
             uint8_t* slot = sm + st * kSlotBytes;
             const float* rg = reinterpret_cast<const float*>(slot + SLOT_REC + REC_G);
             const uint32_t kq = smem_u32(slot + SLOT_KQ);
             const int64_t t0 = s0 + (int64_t)c * kC;
             const int L = (int)min((int64_t)kC, s1 - t0);
 
-            // ---- state: bf16 copy (MMA operand), then S <- gamma S --------------------
-            const float gamma = rg[RG_GAMMA];
-#pragma unroll 1
-            for (int cb = 0; cb < 4; cb += 2) {
-                float x[32], y[32];
-                tmem_ld32x2_sync(ctl + TM_S + 32 * cb, ctl + TM_S + 32 * cb + 32, x, y);
+            // ---- state: bf16 copy (A operand of the first MMA) ----------------------
+            float sx[32], sy[32];
+            tmem_ld32x2_sync(ctl + TM_S + 64 * hh, ctl + TM_S + 64 * hh + 32, sx, sy);
+            {
                 uint32_t pk[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
-                tmem_st16(ctl + TM_S0B + 16 * cb, pk);
+                for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(sx[2 * e], sx[2 * e + 1]);
+                tmem_st16(ctl + TM_S0B + 32 * hh, pk);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(y[2 * e], y[2 * e + 1]);
-                tmem_st16(ctl + TM_S0B + 16 * cb + 16, pk);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    x[e] *= gamma;
-                    y[e] *= gamma;
-                }
-                tmem_st32(ctl + TM_S + 32 * cb, x);
-                tmem_st32(ctl + TM_S + 32 * cb + 32, y);
+                for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(sy[2 * e], sy[2 * e + 1]);
+                tmem_st16(ctl + TM_S0B + 32 * hh + 16, pk);
             }
             tmem_wait_st();
             tc_fence_before();
-            named_bar_sync(1, 128);
+            named_bar_sync(1, kChain);
             tc_fence_after();
             if (tid == 0) {
                 constexpr uint32_t id_d1 = idesc_bf16_f32(128, 128, 0, 0);
@@ -723,35 +732,43 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
                                 smem_desc_sw128(idt + ks * 32, 16, 1024), id_v, ks > 0);
                 mma_commit(mbar);
             }
+            // S <- e^{G_L} S while the MMAs run (they read only the bf16 copy)
+            {
+                const float gamma = rg[RG_GAMMA];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    sx[e] *= gamma;
+                    sy[e] *= gamma;
+                }
+                tmem_st32(ctl + TM_S + 64 * hh, sx);
+                tmem_st32(ctl + TM_S + 64 * hh + 32, sy);
+            }
             if (!mma_wait()) break;
 
-            // ---- Y^T = beta (V - e^G rk X)^T, row i = tid, as bf16 pairs into TMEM -----
+            // ---- Y^T = beta (V - e^G rk X)^T for this thread's 32 tokens -> TMEM -------
             {
-                const float4* bbe = reinterpret_cast<const float4*>(rg + RG_BBE);
-#pragma unroll 1
-                for (int hf = 0; hf < 2; ++hf) {
-                    float x[32], vv[32];
-                    tmem_ld32x2_sync(ctl + TM_D1 + 32 * hf, ctl + TM_DV + 32 * hf, x, vv);
-                    uint32_t pk[16];
+                const float4* bbe = reinterpret_cast<const float4*>(rg + RG_BBE) + 16 * hh;
+                float x[32], vv[32];
+                tmem_ld32x2_sync(ctl + TM_D1 + 32 * hh, ctl + TM_DV + 32 * hh, x, vv);
+                uint32_t pk[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float4 f = bbe[16 * hf + e];
-                        pk[e] = pack_bf16x2(fmaf(f.x, vv[2 * e], -f.y * x[2 * e]),
-                                            fmaf(f.z, vv[2 * e + 1], -f.w * x[2 * e + 1]));
-                    }
-                    tmem_st16(ctl + TM_D1 + 16 * hf, pk);
+                for (int e = 0; e < 16; ++e) {
+                    const float4 f = bbe[e];
+                    pk[e] = pack_bf16x2(fmaf(f.x, vv[2 * e], -f.y * x[2 * e]),
+                                        fmaf(f.z, vv[2 * e + 1], -f.w * x[2 * e + 1]));
                 }
+                tmem_st16(ctl + TM_S0B + 16 * hh, pk);  // the bf16 state copy is consumed
             }
             tmem_wait_st();
             tc_fence_before();
-            named_bar_sync(1, 128);
+            named_bar_sync(1, kChain);
             tc_fence_after();
             if (tid == 0) {
                 constexpr uint32_t id = idesc_bf16_f32(128, 64, 0, 0);
                 const uint32_t tt = smem_u32(slot + SLOT_REC + REC_T);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ts(tmem + TM_D34, tmem + TM_D1 + 8 * ks,
+                    mma_bf16_ts(tmem + TM_D34, tmem + TM_S0B + 8 * ks,
                                 smem_desc_sw128(tt + ks * 32, 16, 1024), id, ks > 0);
                 mma_commit(mbar);
             }
@@ -759,27 +776,24 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
 
             // ---- Vn^T -> bf16 pairs in TMEM, and the decay-scaled copy ---------------
             {
-                const float4* egl4 = reinterpret_cast<const float4*>(rg + RG_EGL);
-#pragma unroll 1
-                for (int hf = 0; hf < 2; ++hf) {
-                    float x[32];
-                    tmem_ld32_sync(ctl + TM_D34 + 32 * hf, x);
-                    uint32_t pk[16], ps[16];
+                const float4* egl4 = reinterpret_cast<const float4*>(rg + RG_EGL) + 8 * hh;
+                float x[32];
+                tmem_ld32_sync(ctl + TM_D34 + 32 * hh, x);
+                uint32_t pk[16], ps[16];
 #pragma unroll
-                    for (int e4 = 0; e4 < 8; ++e4) {
-                        const float4 w = egl4[8 * hf + e4];
-                        pk[2 * e4] = pack_bf16x2(x[4 * e4], x[4 * e4 + 1]);
-                        pk[2 * e4 + 1] = pack_bf16x2(x[4 * e4 + 2], x[4 * e4 + 3]);
-                        ps[2 * e4] = pack_bf16x2(x[4 * e4] * w.x, x[4 * e4 + 1] * w.y);
-                        ps[2 * e4 + 1] = pack_bf16x2(x[4 * e4 + 2] * w.z, x[4 * e4 + 3] * w.w);
-                    }
-                    tmem_st16(ctl + TM_DV + 16 * hf, pk);
-                    tmem_st16(ctl + TM_DV + 32 + 16 * hf, ps);
+                for (int e4 = 0; e4 < 8; ++e4) {
+                    const float4 w = egl4[e4];
+                    pk[2 * e4] = pack_bf16x2(x[4 * e4], x[4 * e4 + 1]);
+                    pk[2 * e4 + 1] = pack_bf16x2(x[4 * e4 + 2], x[4 * e4 + 3]);
+                    ps[2 * e4] = pack_bf16x2(x[4 * e4] * w.x, x[4 * e4 + 1] * w.y);
+                    ps[2 * e4 + 1] = pack_bf16x2(x[4 * e4 + 2] * w.z, x[4 * e4 + 3] * w.w);
                 }
+                tmem_st16(ctl + TM_DV + 16 * hh, pk);
+                tmem_st16(ctl + TM_DV + 32 + 16 * hh, ps);
             }
-            tmem_wait_st();
+            tmem_wait_st();  // also covers the rescaled state stored above
             tc_fence_before();
-            named_bar_sync(1, 128);
+            named_bar_sync(1, kChain);
             tc_fence_after();
             if (tid == 0) {
                 constexpr uint32_t id_o = idesc_bf16_f32(128, 64, 0, 0);
@@ -799,16 +813,15 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
 
             // ---- O = e^G rq (Q S0^T) + P Vn: staged as [t][i] rows, 16-byte stores ----
             uint16_t* Ost = reinterpret_cast<uint16_t*>(sm + CS_O);
-            const float4* eg4 = reinterpret_cast<const float4*>(rg + RG_EGQ);
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
+            {
+                const float4* eg4 = reinterpret_cast<const float4*>(rg + RG_EGQ) + 8 * hh;
                 float xq[32], xi[32];
-                tmem_ld32x2_sync(ctl + TM_D1 + 64 + 32 * half, ctl + TM_D34 + 32 * half, xq, xi);
+                tmem_ld32x2_sync(ctl + TM_D1 + 64 + 32 * hh, ctl + TM_D34 + 32 * hh, xq, xi);
 #pragma unroll
                 for (int e4 = 0; e4 < 8; ++e4) {
-                    const float4 w = eg4[8 * half + e4];
+                    const float4 w = eg4[e4];
                     const int e = 4 * e4;
-                    uint16_t* dst = Ost + (32 * half + e) * kD + tid;
+                    uint16_t* dst = Ost + (32 * hh + e) * kD + row;
                     const __nv_bfloat162 o01 = __floats2bfloat162_rn(fmaf(w.x, xq[e], xi[e]),
                                                                      fmaf(w.y, xq[e + 1], xi[e + 1]));
                     const __nv_bfloat162 o23 = __floats2bfloat162_rn(fmaf(w.z, xq[e + 2], xi[e + 2]),
@@ -819,12 +832,12 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
                     dst[3 * kD] = __bfloat16_as_ushort(o23.y);
                 }
             }
-            named_bar_sync(1, 128);
+            named_bar_sync(1, kChain);
             // the slot is no longer read (the last MMA on it has completed): release it
             if (tid == 0) mbar_arrive(&empty[st]);
 #pragma unroll
-            for (int it = 0; it < 8; ++it) {
-                const int idx = tid + 128 * it;  // 0 .. 1023
+            for (int it = 0; it < 4; ++it) {
+                const int idx = tid + kChain * it;  // 0 .. 1023
                 const int t = idx >> 4, ch = idx & 15;
                 if (t < L)
                     *reinterpret_cast<uint4*>(o + ((size_t)(t0 + t) * H_v + h) * kD + ch * 8) =
@@ -834,9 +847,9 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
         if (!*s_err && Sfg) {
             float* dst = Sfg + sbase;
 #pragma unroll 1
-            for (int cb = 0; cb < 4; ++cb) {
+            for (int cb = 0; cb < 2; ++cb) {
                 float x[32];
-                tmem_ld32_sync(ctl + TM_S + 32 * cb, x);
+                tmem_ld32_sync(ctl + TM_S + 64 * hh + 32 * cb, x);
                 float4* d4 = reinterpret_cast<float4*>(dst + 32 * cb);
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
@@ -848,7 +861,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (tid == 0 && *s_err) set_status(status, kStatusTimeout);
+    if (tid == 0 && (*s_err || *s_lerr)) set_status(status, kStatusTimeout);
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 

@@ -304,6 +304,21 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Named barrier that also ORs a predicate over the participating threads: every
+// thread gets the same answer, so a decision taken on it is uniform.
+__device__ __forceinline__ bool named_bar_any(int id, int nthreads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.or.pred p, %2, %3, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+
 // Byte offset of the 16-byte chunk `chunk` (0..7) of row `row` inside a tile of
 // 128-byte rows stored with the 128-byte swizzle (chunk index XOR row % 8). The
 // tile base must be 1024-byte aligned.

@@ -43,7 +43,13 @@ def test_status_strings(lib):
 
 def test_workspace_size(lib):
     ws = lib.gdn_prefill_workspace_size
-    assert ws(1, 4096, 16, 32, 128, 128) == 2 * 4096 * 32 * 4
+    a256 = lambda x: (x + 255) // 256 * 256
+    # d = 128: chunk offsets (N + 1 int32) + one 17,664-byte record per (chunk, V head),
+    # with at most ceil(T / 64) + N chunks over all sequences
+    assert ws(1, 4096, 16, 32, 128, 128) == a256(2 * 4) + (64 + 1) * 32 * 17664
+    assert ws(4, 4 * 16384, 16, 64, 128, 128) == a256(5 * 4) + (1024 + 4) * 64 * 17664
+    # never below the CUDA-core path's need (G and beta, fp32 [T, H_v] each)
+    assert ws(1, 3, 1, 1, 128, 128) >= 2 * 256
     assert ws(1, 3, 1, 1, 64, 64) == 2 * 256  # each part rounded up to 256 bytes
     assert ws(0, 0, 16, 32, 128, 128) == 0
     assert ws(1, 10, 16, 24, 128, 128) == 0   # H_v % H_qk != 0
