@@ -48,6 +48,8 @@
 //
 // Every wait is bounded; on expiry a block records GDN_ERR_TIMEOUT in the status
 // word, leaves its loops, drains its copies, frees its tensor memory and exits.
+#include <cuda.h>
+
 #include "gdn_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -525,45 +527,63 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
 }
 
 // ==================================== chain =======================================
-constexpr int kChainThreads = 288;   // warps 0-7 state chain, warp 8 loader
+constexpr int kChainThreads = 384;  // warps 0-7 state chain, warps 8-11 output and loads
 constexpr int kChain = 256;
+constexpr int kOut = 128;
 constexpr int kRing = 3;
 // shared memory map (bytes from a 1024-byte aligned base)
-constexpr uint32_t SLOT_KQ = 0;        // [2][128 rows][128 B] raw K then Q, sw128
-constexpr uint32_t SLOT_V = 32768;     // [2][64 rows][128 B] V, sw128
+constexpr uint32_t SLOT_KQ = 0;        // [2 col blocks][K rows 0-63, Q rows 64-127][128 B], sw128
+constexpr uint32_t SLOT_V = 32768;     // [2 col blocks][64 rows][128 B] V, sw128
 constexpr uint32_t SLOT_REC = 49152;   // the (chunk, V head) record: T, P, factors
 constexpr uint32_t kSlotBytes = 67584;
-constexpr uint32_t CS_ID = kRing * kSlotBytes;   // [64][128 B] bf16 identity, sw128
-constexpr uint32_t CS_O = CS_ID + 8192;          // [64 t][128 i] bf16 output staging
-constexpr uint32_t CS_BAR = CS_O + 16384;        // full[3], empty[3], mma
+constexpr uint32_t kSlotTx = 6 * 8192 + kRecBytes;  // six 64x64 tiles + the record
+constexpr uint32_t CS_ID = kRing * kSlotBytes;      // [64][128 B] bf16 identity, sw128
+constexpr uint32_t CS_BAR = CS_ID + 8192;           // full[3], mma, out, ofree, drain
 constexpr uint32_t CS_TMEM = CS_BAR + 64;
 constexpr uint32_t CS_ERR = CS_BAR + 68;
 constexpr size_t kChainSmem = CS_BAR + 128 + 1024;
 
 // tensor memory columns (512 allocated)
 constexpr uint32_t TM_S = 0;      // 128: state, fp32
-constexpr uint32_t TM_S0B = 128;  // 64: state as bf16 pairs (A operand); then Y^T pairs
-constexpr uint32_t TM_D1 = 192;   // 128: S0 K^T | S0 Q^T
-constexpr uint32_t TM_D34 = 320;  // 64: Vn^T, then (P Vn)^T
-constexpr uint32_t TM_DV = 384;   // 64: V^T; then Vn^T (384..415) and scaled Vn^T (416..447)
+constexpr uint32_t TM_S0B = 128;  // 64: state as bf16 pairs; later the decay-scaled Vn^T pairs
+constexpr uint32_t TM_D1K = 192;  // 64: S0 K^T
+constexpr uint32_t TM_D1Q = 256;  // 64: S0 Q^T
+constexpr uint32_t TM_DV = 320;   // 64: V^T; Y^T pairs overwrite columns 0-15 and 32-47
+constexpr uint32_t TM_D3 = 384;   // 64: Vn^T; Vn^T pairs overwrite columns 0-15 and 32-47
+constexpr uint32_t TM_D4 = 448;   // 64: (P Vn)^T
 constexpr uint32_t kTmemCols = 512;
 
-// Two warps share each TMEM lane quarter: warp w owns value rows 32 (w & 3) ..
-// + 31 and, of every 64- or 128-column quantity of those rows, the half w >> 2.
+// Column (in 32-bit words) of the K=16 slice ks of a 64-token bf16 operand that
+// two warps wrote in place over the fp32 columns they had read: tokens 0-31 at
+// +0..15, tokens 32-63 at +32..47.
+__device__ __forceinline__ uint32_t split_pairs_col(int ks) {
+    return (uint32_t)((ks >> 1) * 32 + (ks & 1) * 8);
+}
+
+// One block per (sequence, V head). Warps 0-7 carry the state: two warps share
+// each TMEM lane quarter, warp w owning value rows 32 (w & 3) .. + 31 and, of
+// every 64- or 128-column quantity of those rows, the half w >> 2; warp 0 also
+// issues the MMAs. Warps 8-11 (one per lane quarter) turn each chunk's output
+// accumulators into o and, once a chunk's ring slot is no longer read, load the
+// chunk three ahead into it (TMA tiles for K, Q, V and one bulk copy of the
+// record).
 __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
-    const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
-    const float* __restrict__ S0g, const int32_t* __restrict__ cu_seqlens,
-    const int32_t* __restrict__ choff, int64_t T_total, int H_qk, int H_v,
-    const uint8_t* __restrict__ rec, bf16* __restrict__ o, float* __restrict__ Sfg, int* status) {
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+    const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ S0g,
+    const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict__ choff, int64_t T_total,
+    int H_qk, int H_v, const uint8_t* __restrict__ rec, bf16* __restrict__ o,
+    float* __restrict__ Sfg, int* status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + CS_BAR);
-    uint64_t* empty = full + kRing;
-    uint64_t* mbar = full + 2 * kRing;
+    uint64_t* mbar = full + kRing;      // chain MMA completions
+    uint64_t* obar = full + kRing + 1;  // a chunk's output accumulators complete
+    uint64_t* ofree = full + kRing + 2; // output accumulators read (one arrive per output warp)
+    uint64_t* dbar = full + kRing + 3;  // drain of in-flight MMAs after an error
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + CS_TMEM);
     volatile int* s_err = reinterpret_cast<volatile int*>(sm + CS_ERR);       // chain warps
-    volatile int* s_lerr = reinterpret_cast<volatile int*>(sm + CS_ERR + 4);  // loader warp
+    volatile int* s_lerr = reinterpret_cast<volatile int*>(sm + CS_ERR + 4);  // output warps
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -581,11 +601,11 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < kRing; ++i) {
-            mbar_init(&full[i], 33);  // 32 loader lanes (cp.async) + the expect_tx arrive
-            mbar_init(&empty[i], 1);
-        }
+        for (int i = 0; i < kRing; ++i) mbar_init(&full[i], 1);
         mbar_init(mbar, 1);
+        mbar_init(obar, 1);
+        mbar_init(ofree, 4);
+        mbar_init(dbar, 1);
         *s_err = 0;
         *s_lerr = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -600,56 +620,96 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
             *reinterpret_cast<uint4*>(sm + CS_ID + sw128_off(row, ch)) = w;
         }
         fence_proxy_async_smem();
+    } else if (warp == 8 && lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
 
-    if (warp == 8) {
-        // ================================ loader =======================================
-        int issued = 0;
+    // chunk c of this sequence -> its ring slot (issued by one lane)
+    auto issue_loads = [&](int c) {
+        const int st = c % kRing;
+        uint8_t* slot = sm + st * kSlotBytes;
+        const int32_t t0 = (int32_t)(s0 + (int64_t)c * kC);
+        mbar_arrive_expect_tx(&full[st], kSlotTx);
+        tma_load_3d(slot + SLOT_KQ, &tm_k, 0, j, t0, &full[st]);
+        tma_load_3d(slot + SLOT_KQ + 16384, &tm_k, 64, j, t0, &full[st]);
+        tma_load_3d(slot + SLOT_KQ + 8192, &tm_q, 0, j, t0, &full[st]);
+        tma_load_3d(slot + SLOT_KQ + 16384 + 8192, &tm_q, 64, j, t0, &full[st]);
+        tma_load_3d(slot + SLOT_V, &tm_v, 0, h, t0, &full[st]);
+        tma_load_3d(slot + SLOT_V + 8192, &tm_v, 64, h, t0, &full[st]);
+        bulk_g2s(slot + SLOT_REC, rec + ((size_t)(cg0 + c) * H_v + h) * kRecBytes, kRecBytes,
+                 &full[st]);
+    };
+
+    if (warp >= 8) {
+        // ============================ output + loads ===================================
+        const int qo = warp & 3;
+        const int row = qo * 32 + lane;
+        const uint32_t ctl = tmem + ((uint32_t)(qo * 32) << 16);
+        int issued = nchunks < kRing ? nchunks : kRing;
+        if (warp == 8 && lane == 0)
+            for (int c = 0; c < issued; ++c) issue_loads(c);
+        __syncwarp();
 #pragma unroll 1
         for (int c = 0; c < nchunks; ++c) {
-            const int st = c % kRing;
-            bool ok = true;
-            if (c >= kRing)
-                ok = mbar_wait_bounded(&empty[st], ((c / kRing) - 1) & 1, kWaitCycles);
+            const bool ok = mbar_wait_bounded(obar, c & 1, kWaitCycles);
             if (!ok) *s_lerr = 1;
-            if (__any_sync(0xffffffffu, !ok || *s_err != 0)) break;  // uniform over the warp
-            uint8_t* slot = sm + st * kSlotBytes;
+            if (named_bar_any(2, kOut, !ok || *s_err != 0)) break;
+            tc_fence_after();
+            const float* rg = reinterpret_cast<const float*>(sm + (c % kRing) * kSlotBytes +
+                                                             SLOT_REC + REC_G);
+            const float4* eg4 = reinterpret_cast<const float4*>(rg + RG_EGQ);
+            float ov[64];
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                float xq[32], xi[32];
+                tmem_ld32x2_sync(ctl + TM_D1Q + 32 * hf, ctl + TM_D4 + 32 * hf, xq, xi);
+#pragma unroll
+                for (int e4 = 0; e4 < 8; ++e4) {
+                    const float4 w = eg4[8 * hf + e4];
+                    const int e = 4 * e4;
+                    ov[32 * hf + e] = fmaf(w.x, xq[e], xi[e]);
+                    ov[32 * hf + e + 1] = fmaf(w.y, xq[e + 1], xi[e + 1]);
+                    ov[32 * hf + e + 2] = fmaf(w.z, xq[e + 2], xi[e + 2]);
+                    ov[32 * hf + e + 3] = fmaf(w.w, xq[e + 3], xi[e + 3]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(ofree);  // the accumulators may be overwritten
+            // o[t][i] pairs: lanes 2m, 2m+1 (rows i, i+1) swap one value per token pair
+            // so the even lane stores row pair (t, i..i+1) and the odd one (t+1, i..i+1).
             const int64_t t0 = s0 + (int64_t)c * kC;
             const int L = (int)min((int64_t)kC, s1 - t0);
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&full[st], kRecBytes);
-                bulk_g2s(slot + SLOT_REC, rec + ((size_t)(cg0 + c) * H_v + h) * kRecBytes,
-                         kRecBytes, &full[st]);
+            const bool odd = (lane & 1) != 0;
+            bf16* obase = o + ((size_t)t0 * H_v + h) * kD + (row & ~1);
+#pragma unroll
+            for (int tp = 0; tp < 32; ++tp) {
+                const float a0 = ov[2 * tp], a1 = ov[2 * tp + 1];
+                const float recv = __shfl_xor_sync(0xffffffffu, odd ? a0 : a1, 1);
+                const uint32_t w = odd ? pack_bf16x2(recv, a1) : pack_bf16x2(a0, recv);
+                const int t = 2 * tp + (odd ? 1 : 0);
+                if (t < L)
+                    *reinterpret_cast<uint32_t*>(obase + (size_t)t * H_v * kD) = w;
             }
-#pragma unroll 4
-            for (int it = 0; it < 32; ++it) {
-                const int idx = lane + 32 * it;  // 0 .. 1023
-                const int rr = idx >> 4, ch = idx & 15;
-                const bool live = rr < L;
-                const int64_t tok = live ? t0 + rr : 0;
-                const size_t rowk = ((size_t)tok * H_qk + j) * kD + ch * 8;
-                const uint32_t off = (uint32_t)(ch >> 3) * 16384u;
-                cp_async_16(slot + SLOT_KQ + off + sw128_off(rr, ch & 7), k + rowk, live ? 16u : 0u);
-                cp_async_16(slot + SLOT_KQ + off + sw128_off(rr + 64, ch & 7), q + rowk,
-                            live ? 16u : 0u);
-                cp_async_16(slot + SLOT_V + (uint32_t)(ch >> 3) * 8192u + sw128_off(rr, ch & 7),
-                            v + ((size_t)tok * H_v + h) * kD + ch * 8, live ? 16u : 0u);
+            named_bar_sync(2, kOut);  // every output warp is done with this slot
+            if (warp == 8 && lane == 0 && c + kRing < nchunks) {
+                issue_loads(c + kRing);
+                issued = c + kRing + 1;
             }
-            cp_async_mbar_arrive_noinc(&full[st]);
-            issued = c + 1;
+            __syncwarp();
         }
-        cp_async_commit();
-        cp_async_wait<0>();
-        // Drain the record copies: the last phase of each slot has completed (at
-        // once on the normal path, where the chain consumed it) before the block
-        // may leave with nothing in flight into its shared memory.
-        if (lane == 0) {
+        // Leave nothing in flight into shared memory (loads the chain did not
+        // consume are only possible after an error).
+        if (warp == 8 && lane == 0) {
             for (int c = issued - 1; c >= 0 && c >= issued - kRing; --c)
-                if (!mbar_wait_bounded(&full[c % kRing], (c / kRing) & 1, kWaitCycles)) *s_lerr = 1;
+                if (!mbar_wait_bounded(&full[c % kRing], (c / kRing) & 1, kWaitCycles))
+                    *s_lerr = 1;
         }
         __syncwarp();
     } else {
@@ -678,29 +738,53 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
         tmem_wait_st();
 
         uint32_t mphase = 0;
-        auto mma_wait = [&]() -> bool {
+        auto wait_mma = [&]() -> bool {
             const bool ok = mbar_wait_bounded(mbar, mphase, kWaitCycles);
             mphase ^= 1u;
             if (!ok) *s_err = 1;
-            const bool bad = named_bar_any(1, kChain, !ok);
             tc_fence_after();
-            return !bad;
+            return ok;
         };
 
 #pragma unroll 1
         for (int c = 0; c < nchunks; ++c) {
             const int st = c % kRing;
-            const bool ok = mbar_wait_bounded(&full[st], (c / kRing) & 1, kWaitCycles);
-            if (!ok) *s_err = 1;
-            fence_proxy_async_smem();  // the loader's cp.async rows -> tensor core reads
-            if (named_bar_any(1, kChain, !ok)) break;
             uint8_t* slot = sm + st * kSlotBytes;
             const float* rg = reinterpret_cast<const float*>(slot + SLOT_REC + REC_G);
             const uint32_t kq = smem_u32(slot + SLOT_KQ);
             const int64_t t0 = s0 + (int64_t)c * kC;
             const int L = (int)min((int64_t)kC, s1 - t0);
 
-            // ---- state: bf16 copy (A operand of the first MMA) ----------------------
+            // ---- the previous state update and this chunk's data ---------------------
+            bool ok = c > 0 ? wait_mma() : true;
+            if (!mbar_wait_bounded(&full[st], (c / kRing) & 1, kWaitCycles)) {
+                ok = false;
+                *s_err = 1;
+            }
+            if (L < kC) {
+                // rows past the sequence's end hold the next sequence's tokens: zero them
+                const int nz = (kC - L) * 8;  // 16-byte chunks per 64-column tile
+                for (int idx = tid; idx < 6 * nz; idx += kChain) {
+                    const int tile = idx / nz, r = L + (idx % nz) / 8, ch = idx & 7;
+                    const uint32_t base = tile < 4 ? SLOT_KQ + (tile >> 1) * 16384u + (tile & 1) * 8192u
+                                                   : SLOT_V + (tile - 4) * 8192u;
+                    *reinterpret_cast<uint4*>(slot + base + r * 128 + ch * 16) =
+                        make_uint4(0u, 0u, 0u, 0u);
+                }
+                fence_proxy_async_smem();
+                named_bar_sync(1, kChain);
+            }
+            if (warp == 0) {  // V^T: no dependence on the state, runs under the S step
+                __syncwarp();
+                constexpr uint32_t id_v = idesc_bf16_f32(128, 64, 1, 0);
+                const uint32_t vt = smem_u32(slot + SLOT_V), idt = smem_u32(sm + CS_ID);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16_ss_warp(tmem + TM_DV, smem_desc_sw128(vt + ks * 2048, 8192, 1024),
+                                     smem_desc_sw128(idt + ks * 32, 16, 1024), id_v, ks > 0);
+            }
+
+            // ---- state: bf16 copy (A operand of S0 K^T and S0 Q^T) ----------------------
             float sx[32], sy[32];
             tmem_ld32x2_sync(ctl + TM_S + 64 * hh, ctl + TM_S + 64 * hh + 32, sx, sy);
             {
@@ -714,26 +798,29 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
             }
             tmem_wait_st();
             tc_fence_before();
-            named_bar_sync(1, kChain);
+            if (named_bar_any(1, kChain, !ok)) break;
             tc_fence_after();
-            if (tid == 0) {
-                constexpr uint32_t id_d1 = idesc_bf16_f32(128, 128, 0, 0);
-                constexpr uint32_t id_v = idesc_bf16_f32(128, 64, 1, 0);
+            if (warp == 0) {
+                constexpr uint32_t id64 = idesc_bf16_f32(128, 64, 0, 0);
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t off = (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u;
-                    mma_bf16_ts(tmem + TM_D1, tmem + TM_S0B + 8 * ks,
-                                smem_desc_sw128(kq + off, 16, 1024), id_d1, ks > 0);
+                    mma_bf16_ts_warp(tmem + TM_D1K, tmem + TM_S0B + 8 * ks,
+                                     smem_desc_sw128(kq + off, 16, 1024), id64, ks > 0);
                 }
-                const uint32_t vt = smem_u32(slot + SLOT_V), idt = smem_u32(sm + CS_ID);
+                mma_commit_warp(mbar);
+                // S0 Q^T overwrites the accumulator the output warps read for chunk c-1
+                if (c > 0 && !mbar_wait_bounded(ofree, (c - 1) & 1, kWaitCycles)) *s_err = 1;
+                __syncwarp();
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ss(tmem + TM_DV, smem_desc_sw128(vt + ks * 2048, 8192, 1024),
-                                smem_desc_sw128(idt + ks * 32, 16, 1024), id_v, ks > 0);
-                mma_commit(mbar);
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t off =
+                        8192u + (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u;
+                    mma_bf16_ts_warp(tmem + TM_D1Q, tmem + TM_S0B + 8 * ks,
+                                     smem_desc_sw128(kq + off, 16, 1024), id64, ks > 0);
+                }
             }
-            // S <- e^{G_L} S while the MMAs run (they read only the bf16 copy)
-            {
+            {  // S <- e^{G_L} S while the MMAs run (they read only the bf16 copy)
                 const float gamma = rg[RG_GAMMA];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
@@ -743,13 +830,13 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
                 tmem_st32(ctl + TM_S + 64 * hh, sx);
                 tmem_st32(ctl + TM_S + 64 * hh + 32, sy);
             }
-            if (!mma_wait()) break;
 
-            // ---- Y^T = beta (V - e^G rk X)^T for this thread's 32 tokens -> TMEM -------
+            // ---- Y^T = beta (V - e^G rk X)^T for this thread's 32 tokens --------------
+            ok = wait_mma();  // S0 K^T and V^T
             {
                 const float4* bbe = reinterpret_cast<const float4*>(rg + RG_BBE) + 16 * hh;
                 float x[32], vv[32];
-                tmem_ld32x2_sync(ctl + TM_D1 + 32 * hh, ctl + TM_DV + 32 * hh, x, vv);
+                tmem_ld32x2_sync(ctl + TM_D1K + 32 * hh, ctl + TM_DV + 32 * hh, x, vv);
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
@@ -757,28 +844,28 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
                     pk[e] = pack_bf16x2(fmaf(f.x, vv[2 * e], -f.y * x[2 * e]),
                                         fmaf(f.z, vv[2 * e + 1], -f.w * x[2 * e + 1]));
                 }
-                tmem_st16(ctl + TM_S0B + 16 * hh, pk);  // the bf16 state copy is consumed
+                tmem_st16(ctl + TM_DV + 32 * hh, pk);  // over the V^T columns just read
             }
             tmem_wait_st();
             tc_fence_before();
-            named_bar_sync(1, kChain);
+            if (named_bar_any(1, kChain, !ok)) break;
             tc_fence_after();
-            if (tid == 0) {
+            if (warp == 0) {
                 constexpr uint32_t id = idesc_bf16_f32(128, 64, 0, 0);
                 const uint32_t tt = smem_u32(slot + SLOT_REC + REC_T);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ts(tmem + TM_D34, tmem + TM_S0B + 8 * ks,
-                                smem_desc_sw128(tt + ks * 32, 16, 1024), id, ks > 0);
-                mma_commit(mbar);
+                    mma_bf16_ts_warp(tmem + TM_D3, tmem + TM_DV + split_pairs_col(ks),
+                                     smem_desc_sw128(tt + ks * 32, 16, 1024), id, ks > 0);
+                mma_commit_warp(mbar);
             }
-            if (!mma_wait()) break;
 
-            // ---- Vn^T -> bf16 pairs in TMEM, and the decay-scaled copy ---------------
+            // ---- Vn^T -> bf16 pairs (for P Vn) and decay-scaled pairs (state update) --
+            ok = wait_mma();  // Vn^T (and S0 Q^T)
             {
                 const float4* egl4 = reinterpret_cast<const float4*>(rg + RG_EGL) + 8 * hh;
                 float x[32];
-                tmem_ld32_sync(ctl + TM_D34 + 32 * hh, x);
+                tmem_ld32_sync(ctl + TM_D3 + 32 * hh, x);
                 uint32_t pk[16], ps[16];
 #pragma unroll
                 for (int e4 = 0; e4 < 8; ++e4) {
@@ -788,63 +875,32 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
                     ps[2 * e4] = pack_bf16x2(x[4 * e4] * w.x, x[4 * e4 + 1] * w.y);
                     ps[2 * e4 + 1] = pack_bf16x2(x[4 * e4 + 2] * w.z, x[4 * e4 + 3] * w.w);
                 }
-                tmem_st16(ctl + TM_DV + 16 * hh, pk);
-                tmem_st16(ctl + TM_DV + 32 + 16 * hh, ps);
+                tmem_st16(ctl + TM_D3 + 32 * hh, pk);   // over the Vn^T columns just read
+                tmem_st16(ctl + TM_S0B + 16 * hh, ps);  // the bf16 state is consumed
             }
             tmem_wait_st();  // also covers the rescaled state stored above
             tc_fence_before();
-            named_bar_sync(1, kChain);
+            if (named_bar_any(1, kChain, !ok)) break;
             tc_fence_after();
-            if (tid == 0) {
-                constexpr uint32_t id_o = idesc_bf16_f32(128, 64, 0, 0);
+            if (warp == 0) {
                 constexpr uint32_t id_s = idesc_bf16_f32(128, 128, 0, 1);
+                constexpr uint32_t id_o = idesc_bf16_f32(128, 64, 0, 0);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16_ts_warp(tmem + TM_S, tmem + TM_S0B + 8 * ks,
+                                     smem_desc_sw128(kq + ks * 2048, 16384, 1024), id_s, 1);
+                mma_commit_warp(mbar);
                 const uint32_t ptile = smem_u32(slot + SLOT_REC + REC_P);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ts(tmem + TM_D34, tmem + TM_DV + 8 * ks,
-                                smem_desc_sw128(ptile + ks * 32, 16, 1024), id_o, ks > 0);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ts(tmem + TM_S, tmem + TM_DV + 32 + 8 * ks,
-                                smem_desc_sw128(kq + ks * 2048, 16384, 1024), id_s, 1);
-                mma_commit(mbar);
-            }
-            if (!mma_wait()) break;
-
-            // ---- O = e^G rq (Q S0^T) + P Vn: staged as [t][i] rows, 16-byte stores ----
-            uint16_t* Ost = reinterpret_cast<uint16_t*>(sm + CS_O);
-            {
-                const float4* eg4 = reinterpret_cast<const float4*>(rg + RG_EGQ) + 8 * hh;
-                float xq[32], xi[32];
-                tmem_ld32x2_sync(ctl + TM_D1 + 64 + 32 * hh, ctl + TM_D34 + 32 * hh, xq, xi);
-#pragma unroll
-                for (int e4 = 0; e4 < 8; ++e4) {
-                    const float4 w = eg4[e4];
-                    const int e = 4 * e4;
-                    uint16_t* dst = Ost + (32 * hh + e) * kD + row;
-                    const __nv_bfloat162 o01 = __floats2bfloat162_rn(fmaf(w.x, xq[e], xi[e]),
-                                                                     fmaf(w.y, xq[e + 1], xi[e + 1]));
-                    const __nv_bfloat162 o23 = __floats2bfloat162_rn(fmaf(w.z, xq[e + 2], xi[e + 2]),
-                                                                     fmaf(w.w, xq[e + 3], xi[e + 3]));
-                    dst[0] = __bfloat16_as_ushort(o01.x);
-                    dst[kD] = __bfloat16_as_ushort(o01.y);
-                    dst[2 * kD] = __bfloat16_as_ushort(o23.x);
-                    dst[3 * kD] = __bfloat16_as_ushort(o23.y);
-                }
-            }
-            named_bar_sync(1, kChain);
-            // the slot is no longer read (the last MMA on it has completed): release it
-            if (tid == 0) mbar_arrive(&empty[st]);
-#pragma unroll
-            for (int it = 0; it < 4; ++it) {
-                const int idx = tid + kChain * it;  // 0 .. 1023
-                const int t = idx >> 4, ch = idx & 15;
-                if (t < L)
-                    *reinterpret_cast<uint4*>(o + ((size_t)(t0 + t) * H_v + h) * kD + ch * 8) =
-                        *reinterpret_cast<const uint4*>(Ost + t * kD + ch * 8);
+                    mma_bf16_ts_warp(tmem + TM_D4, tmem + TM_D3 + split_pairs_col(ks),
+                                     smem_desc_sw128(ptile + ks * 32, 16, 1024), id_o, ks > 0);
+                mma_commit_warp(obar);
             }
         }
-        if (!*s_err && Sfg) {
+        bool fin = !*s_err;
+        if (fin && nchunks > 0) fin = wait_mma();  // the last state update
+        if (fin && Sfg) {
             float* dst = Sfg + sbase;
 #pragma unroll 1
             for (int cb = 0; cb < 2; ++cb) {
@@ -856,6 +912,14 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
                     d4[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
             }
         }
+        // After an error: no MMA may still run when the tensor memory is freed, and
+        // the output warps are woken to see the error and leave.
+        const bool err = __any_sync(0xffffffffu, *s_err != 0);
+        if (warp == 0 && err) {
+            mma_commit_warp(dbar);
+            (void)mbar_wait_bounded(dbar, 0, kWaitCycles);
+        }
+        if (tid == 0 && err) mbar_arrive(obar);
     }
 
     tc_fence_before();
@@ -876,14 +940,56 @@ size_t prefill_tc_workspace_bytes(int32_t N, int64_t T, int32_t H_v) {
 
 bool prefill_tc_supported(int32_t H_qk, int32_t H_v) { return H_v / H_qk <= kMaxGroup; }
 
+namespace {
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+// [T][heads][128] bf16 rows as a 3-D tensor (d, head, token); boxes of 64 d x 1
+// head x 64 tokens land as 64 rows of 128 bytes in the 128-byte swizzle. Tokens
+// past T read as zeros.
+bool make_rows_map(CUtensorMap* m, const void* base, int heads, int64_t T) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)heads, (cuuint64_t)(T > 0 ? T : 1)};
+    const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)heads * kD * 2};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)kC};
+    const cuuint32_t estride[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+              estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+}  // namespace
+
 cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const float* a,
                               const float* b, const float* A_log, const float* dt_bias,
                               const float* S0, const int32_t* cu_seqlens, int32_t N, int64_t T,
                               int32_t H_qk, int32_t H_v, float scale, void* o, float* S_final,
                               void* workspace, int* status, cudaStream_t s) {
     if (N == 0) return cudaSuccess;
+    if (T > (int64_t)0x7FFFFFFF - kC) return cudaErrorInvalidValue;  // TMA token coordinates
     int32_t* choff = static_cast<int32_t*>(workspace);
     uint8_t* rec = static_cast<uint8_t*>(workspace) + align256((size_t)(N + 1) * sizeof(int32_t));
+    // With no tokens the maps are never read; any aligned device address will do.
+    CUtensorMap tm_q, tm_k, tm_v;
+    if (!make_rows_map(&tm_q, T > 0 ? q : workspace, H_qk, T) ||
+        !make_rows_map(&tm_k, T > 0 ? k : workspace, H_qk, T) ||
+        !make_rows_map(&tm_v, T > 0 ? v : workspace, H_v, T))
+        return cudaErrorInvalidValue;
     int dev = 0, num_sms = 0;
     cudaGetDevice(&dev);
     if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
@@ -910,8 +1016,8 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
     }
     const int64_t blocks = (int64_t)N * H_v;
     chain_kernel<<<(unsigned)blocks, kChainThreads, kChainSmem, s>>>(
-        static_cast<const bf16*>(q), static_cast<const bf16*>(k), static_cast<const bf16*>(v), S0,
-        cu_seqlens, choff, T, H_qk, H_v, rec, static_cast<bf16*>(o), S_final, status);
+        tm_q, tm_k, tm_v, S0, cu_seqlens, choff, T, H_qk, H_v, rec, static_cast<bf16*>(o),
+        S_final, status);
     return cudaGetLastError();
 }
 
