@@ -538,7 +538,8 @@ constexpr uint32_t SLOT_REC = 49152;   // the (chunk, V head) record: T, P, fact
 constexpr uint32_t kSlotBytes = 67584;
 constexpr uint32_t kSlotTx = 6 * 8192 + kRecBytes;  // six 64x64 tiles + the record
 constexpr uint32_t CS_ID = kRing * kSlotBytes;      // [64][128 B] bf16 identity, sw128
-constexpr uint32_t CS_BAR = CS_ID + 8192;           // full[3], mma, out, ofree, drain
+constexpr uint32_t CS_OST = CS_ID + 8192;           // [2 col blocks][64 t][128 B] o, sw128
+constexpr uint32_t CS_BAR = CS_OST + 16384;         // full[3], mma, out, ofree, drain
 constexpr uint32_t CS_TMEM = CS_BAR + 64;
 constexpr uint32_t CS_ERR = CS_BAR + 68;
 constexpr size_t kChainSmem = CS_BAR + 128 + 1024;
@@ -569,7 +570,8 @@ __device__ __forceinline__ uint32_t split_pairs_col(int ks) {
 // record).
 __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-    const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ S0g,
+    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+    const float* __restrict__ S0g,
     const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict__ choff, int64_t T_total,
     int H_qk, int H_v, const uint8_t* __restrict__ rec, bf16* __restrict__ o,
     float* __restrict__ Sfg, int* status) {
@@ -624,6 +626,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_o);
     }
     tc_fence_before();
     __syncthreads();
@@ -655,10 +658,16 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
         if (warp == 8 && lane == 0)
             for (int c = 0; c < issued; ++c) issue_loads(c);
         __syncwarp();
+        uint8_t* ost = sm + CS_OST;
+        // this thread's element (t, i) of the staged o tile: block i / 64, 16-byte
+        // chunk (i % 64) / 8 swizzled with t % 8, halfword i % 8
+        const uint32_t o_row = (uint32_t)(row >> 6) * 8192u + (uint32_t)(row & 7) * 2u;
+        const uint32_t o_chk = (uint32_t)((row & 63) >> 3);
 #pragma unroll 1
         for (int c = 0; c < nchunks; ++c) {
             const bool ok = mbar_wait_bounded(obar, c & 1, kWaitCycles);
             if (!ok) *s_lerr = 1;
+            if (warp == 8 && lane == 0) bulk_wait_group_read<0>();  // staging free again
             if (named_bar_any(2, kOut, !ok || *s_err != 0)) break;
             tc_fence_after();
             const float* rg = reinterpret_cast<const float*>(sm + (c % kRing) * kSlotBytes +
@@ -682,28 +691,39 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(ofree);  // the accumulators may be overwritten
-            // o[t][i] pairs: lanes 2m, 2m+1 (rows i, i+1) swap one value per token pair
-            // so the even lane stores row pair (t, i..i+1) and the odd one (t+1, i..i+1).
+#pragma unroll
+            for (int t = 0; t < kC; ++t)
+                *reinterpret_cast<bf16*>(ost + o_row + (uint32_t)t * 128u +
+                                         ((o_chk ^ (uint32_t)(t & 7)) << 4)) =
+                    __float2bfloat16_rn(ov[t]);
+            fence_proxy_async_smem();
+            named_bar_sync(2, kOut);  // staged; every output warp is done with this slot
             const int64_t t0 = s0 + (int64_t)c * kC;
             const int L = (int)min((int64_t)kC, s1 - t0);
-            const bool odd = (lane & 1) != 0;
-            bf16* obase = o + ((size_t)t0 * H_v + h) * kD + (row & ~1);
-#pragma unroll
-            for (int tp = 0; tp < 32; ++tp) {
-                const float a0 = ov[2 * tp], a1 = ov[2 * tp + 1];
-                const float recv = __shfl_xor_sync(0xffffffffu, odd ? a0 : a1, 1);
-                const uint32_t w = odd ? pack_bf16x2(recv, a1) : pack_bf16x2(a0, recv);
-                const int t = 2 * tp + (odd ? 1 : 0);
-                if (t < L)
-                    *reinterpret_cast<uint32_t*>(obase + (size_t)t * H_v * kD) = w;
+            if (L == kC) {
+                if (warp == 8 && lane == 0) {
+                    tma_store_3d(&tm_o, 0, h, (int32_t)t0, ost);
+                    tma_store_3d(&tm_o, 64, h, (int32_t)t0, ost + 8192);
+                    bulk_commit_group();
+                }
+            } else {
+                // the sequence's last rows only: plain 16-byte stores
+                for (int idx = tid - kChain; idx < L * 16; idx += kOut) {
+                    const int r = idx >> 4, ch = idx & 15;
+                    const uint4 w = *reinterpret_cast<const uint4*>(
+                        ost + (uint32_t)(ch >> 3) * 8192u + (uint32_t)r * 128u +
+                        ((uint32_t)((ch & 7) ^ (r & 7)) << 4));
+                    *reinterpret_cast<uint4*>(o + ((size_t)(t0 + r) * H_v + h) * kD + ch * 8) = w;
+                }
+                named_bar_sync(2, kOut);
             }
-            named_bar_sync(2, kOut);  // every output warp is done with this slot
             if (warp == 8 && lane == 0 && c + kRing < nchunks) {
                 issue_loads(c + kRing);
                 issued = c + kRing + 1;
             }
             __syncwarp();
         }
+        if (warp == 8 && lane == 0) bulk_wait_group<0>();  // o stores complete
         // Leave nothing in flight into shared memory (loads the chain did not
         // consume are only possible after an error).
         if (warp == 8 && lane == 0) {
@@ -960,8 +980,8 @@ EncodeTiledFn encode_tiled() {
 }
 
 // [T][heads][128] bf16 rows as a 3-D tensor (d, head, token); boxes of 64 d x 1
-// head x 64 tokens land as 64 rows of 128 bytes in the 128-byte swizzle. Tokens
-// past T read as zeros.
+// head x 64 tokens move as 64 rows of 128 bytes in the 128-byte swizzle. Tokens
+// past T read as zeros and are not written.
 bool make_rows_map(CUtensorMap* m, const void* base, int heads, int64_t T) {
     EncodeTiledFn fn = encode_tiled();
     if (!fn) return false;
@@ -985,10 +1005,11 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
     int32_t* choff = static_cast<int32_t*>(workspace);
     uint8_t* rec = static_cast<uint8_t*>(workspace) + align256((size_t)(N + 1) * sizeof(int32_t));
     // With no tokens the maps are never read; any aligned device address will do.
-    CUtensorMap tm_q, tm_k, tm_v;
+    CUtensorMap tm_q, tm_k, tm_v, tm_o;
     if (!make_rows_map(&tm_q, T > 0 ? q : workspace, H_qk, T) ||
         !make_rows_map(&tm_k, T > 0 ? k : workspace, H_qk, T) ||
-        !make_rows_map(&tm_v, T > 0 ? v : workspace, H_v, T))
+        !make_rows_map(&tm_v, T > 0 ? v : workspace, H_v, T) ||
+        !make_rows_map(&tm_o, T > 0 ? o : workspace, H_v, T))
         return cudaErrorInvalidValue;
     int dev = 0, num_sms = 0;
     cudaGetDevice(&dev);
@@ -1016,7 +1037,7 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
     }
     const int64_t blocks = (int64_t)N * H_v;
     chain_kernel<<<(unsigned)blocks, kChainThreads, kChainSmem, s>>>(
-        tm_q, tm_k, tm_v, S0, cu_seqlens, choff, T, H_qk, H_v, rec, static_cast<bf16*>(o),
+        tm_q, tm_k, tm_v, tm_o, S0, cu_seqlens, choff, T, H_qk, H_v, rec, static_cast<bf16*>(o),
         S_final, status);
     return cudaGetLastError();
 }
