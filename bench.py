@@ -2,8 +2,8 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One JSON line on rank 0. A "step" is one gdn_prefill call (gate prologue + chunk
-kernel) on the 35B-A3B GDN layer shape: B=1, T=4096, 16 QK / 32 V heads,
+One JSON line on rank 0. A "step" is one gdn_prefill call (chunk offsets, prep
+and chain kernels of the tensor-core path) on the 35B-A3B GDN layer shape: B=1, T=4096, 16 QK / 32 V heads,
 d=128, bf16 q/k/v/o, fp32 gates and state, zero initial state, final state
 written. `value` is prefill tokens/s over the whole job (all ranks; each rank
 runs its own copy of the workload, so scaling is weak). The same line carries
@@ -16,6 +16,14 @@ the launching stream; a barrier and a device synchronise on both sides of the
 timed region; the max over ranks. `e2e` repeats the prefill through the public
 Python API from pinned host buffers, host<->device copies inside the timing.
 The CPU baseline is the fp64 oracle (test infrastructure) timed on this host.
+
+`roofline` is that of the dominant kernel (the chain): its duration comes from
+the library's kernel timing (CUDA events recorded around each launch on the
+launching stream, every timed step), its algorithmic bytes are those it must
+move (q, k, v read, o and the final state written); `traffic` is the DRAM bytes
+per launch from the committed ncu summary of that kernel, null when the summary
+was taken on another build of it. `roofline.step` gives the whole call against
+the slower of the HBM and tensor roofs.
 """
 from __future__ import annotations
 
@@ -52,6 +60,37 @@ def prefill_bytes(T, N, H_qk, H_v, d, io_bytes, with_initial):
     b = 2 * T * H_qk * d * io_bytes + 2 * T * H_v * d * io_bytes + 2 * T * H_v * 4
     b += N * H_v * d * d * 4 * (2 if with_initial else 1)
     return b
+
+
+def chain_bytes(T, N, H_qk, H_v, d, io_bytes, with_initial):
+    """Algorithmic HBM bytes of the chain kernel: q, k, v read, o written, the
+    final state written (and the initial state read if given)."""
+    return prefill_bytes(T, N, H_qk, H_v, d, io_bytes, with_initial) - 2 * T * H_v * 4
+
+
+CHAIN_PROFILE = os.path.join(ROOT, "profiles", "chain_kernel_prefill35b.md")
+
+
+def _chain_traffic():
+    """(DRAM bytes per launch, kernel build id) from the ncu summary of the chain kernel."""
+    try:
+        vals = {}
+        with open(CHAIN_PROFILE) as f:
+            for line in f:
+                if ":" in line and line.strip().startswith(("traffic_bytes_per_launch",
+                                                            "kernel_source_sha1")):
+                    k_, v_ = line.split(":", 1)
+                    vals[k_.strip().lstrip("-* ")] = v_.strip().strip("`")
+        return int(vals["traffic_bytes_per_launch"]), vals.get("kernel_source_sha1")
+    except Exception:
+        return None, None
+
+
+def _chain_source_sha1():
+    import hashlib
+    src = os.path.join(ROOT, "linear_attention_sequence_delta_b200", "csrc", "gdn_prefill_tc.cu")
+    with open(src, "rb") as f:
+        return hashlib.sha1(f.read()).hexdigest()
 
 
 def prefill_flops(T, N, H_qk, H_v, d, C=64):
@@ -168,6 +207,8 @@ def run_ours(args):
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
     clocks = Clocks(local)
+    kernel_ms = {}  # kernel name -> [ms per timed step]
+    prev_timing = gdn.set_kernel_timing(True)
     _barrier(ws)
     torch.cuda.synchronize()
     with clocks:
@@ -176,6 +217,9 @@ def run_ours(args):
             ev[i][0].record(stream)
             step()
             ev[i][1].record(stream)
+            for name, kms in gdn.last_prefill_kernel_times():  # waits for this step only
+                kernel_ms.setdefault(name, []).append(kms)
+        gdn.set_kernel_timing(prev_timing)
         torch.cuda.synchronize()
         _barrier(ws)
         # ---- decode: 1000 consecutive steps on the 397B-A17B GDN shape ----
@@ -218,6 +262,13 @@ def run_ours(args):
     flops = prefill_flops(T, N, H_qk, H_v, d)
     achieved = byts / (ms / 1e3) / 1e9
     t_roof = max(byts / (hbm * 1e9), flops / (tc_burst * 1e12))
+    mean_k = {n_: _max_over_ranks(sum(v_) / len(v_), ws, dev) for n_, v_ in kernel_ms.items()}
+    dom = max(mean_k, key=mean_k.get)
+    dom_ms = mean_k[dom]
+    dom_bytes = chain_bytes(T, N, H_qk, H_v, d, 2, with_initial=False)
+    traffic, traffic_src = _chain_traffic()
+    if dom != "chain" or traffic_src != _chain_source_sha1():
+        traffic = None  # the counters were taken on another build of the kernel
 
     e2e = None
     if not args.no_e2e:
@@ -232,16 +283,20 @@ def run_ours(args):
                                "fp32 gates/state, zero initial state, final state written",
                    "global_batch": ws, "seq_len": T, "parallelism": f"replicas x{ws}",
                    "l2": "flushed (512 MiB write) before every timed step"},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": None, "algorithmic_bytes": byts,
-                     "kernel": "gdn_prefill (gate prologue + chunk kernel)",
-                     "peak_source": peak_src,
-                     "tensor": {"algorithmic_flops": flops, "achieved_tflops":
-                                flops / (ms / 1e3) / 1e12, "peak_tflops": tc_burst,
-                                "frac": flops / (ms / 1e3) / 1e12 / tc_burst},
-                     "frac_of_slower_roof": t_roof / (ms / 1e3)},
+        "roofline": {"bound": "hbm", "achieved": dom_bytes / (dom_ms / 1e3) / 1e9, "peak": hbm,
+                     "unit": "GB/s", "frac": dom_bytes / (dom_ms / 1e3) / 1e9 / hbm,
+                     "traffic": traffic, "kernel": dom, "algorithmic_bytes": dom_bytes,
+                     "kernel_ms": dom_ms, "peak_source": peak_src,
+                     "kernels_ms": mean_k,
+                     "step": {"algorithmic_bytes": byts, "achieved_gbs": achieved,
+                              "frac_hbm": achieved / hbm, "algorithmic_flops": flops,
+                              "achieved_tflops": flops / (ms / 1e3) / 1e12,
+                              "peak_tflops": tc_burst,
+                              "frac_tensor": flops / (ms / 1e3) / 1e12 / tc_burst,
+                              "frac_of_slower_roof": t_roof / (ms / 1e3)}},
         "e2e": e2e,
-        "gpu_launches": 2 * args.steps + (args.decode_steps if dec else 0),
+        "gpu_launches": sum(len(v_) for v_ in kernel_ms.values())
+                        + (args.decode_steps if dec else 0),
         "clocks": clocks.summary(),
         "decode": dec,
     }

@@ -184,6 +184,29 @@ int gdn_prefill_noalloc(const void* q, const void* k, const void* v, int32_t io_
                         void* o, float* final_state, void* stream);
 
 /*
+ * Kernel timing of gdn_prefill -- a measurement aid; the pages have no
+ * counterpart. While enabled (gdn_set_kernel_timing(1)), every gdn_prefill call
+ * records a CUDA event before and after each kernel it launches, on the call's
+ * stream (at most 4 kernels per call; the library owns the events).
+ *   gdn_set_kernel_timing   enable (nonzero) or disable; returns the previous
+ *                           setting.
+ *   gdn_last_prefill_kernel_ms
+ *                           waits for the events of the most recent timed call
+ *                           and writes the duration of its first
+ *                           min(count, max_kernels) kernels, in milliseconds, to
+ *                           ms (host array); returns the kernel count, or
+ *                           -GDN_ERR_INVALID_ARG / -GDN_ERR_CUDA.
+ *   gdn_last_prefill_kernel_name
+ *                           name of kernel i of that call ("chunk_offsets",
+ *                           "prep", "chain" on the tensor-core path; "gates",
+ *                           "prefill_simt" on the CUDA-core path), or NULL.
+ * The timing state is process-wide: time from one host thread at a time.
+ */
+int gdn_set_kernel_timing(int32_t enable);
+int gdn_last_prefill_kernel_ms(float* ms, int32_t max_kernels);
+const char* gdn_last_prefill_kernel_name(int32_t i);
+
+/*
  * Synchronise `stream`, then return and clear the device status word of the
  * current device (GDN_OK, GDN_ERR_BAD_SEQLENS or GDN_ERR_TIMEOUT), or
  * GDN_ERR_CUDA if the synchronisation itself failed.

@@ -35,7 +35,51 @@ int check_heads(int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v) {
 }
 
 size_t gate_bytes(int64_t T, int32_t H_v) { return align_up((size_t)T * H_v * sizeof(float), 256); }
+// Kernel timing state (process-wide; meant for one measuring thread at a time).
+constexpr int kMaxTimed = 4;
+std::atomic<int> g_ktiming{0};
+struct KernelTimer {
+    cudaEvent_t ev[2 * kMaxTimed] = {};
+    const char* name[kMaxTimed] = {};
+    int n = 0;
+    int dev = -1;
+    bool open = false;  // an event pair is half recorded
+};
+KernelTimer g_kt;
+
+bool ktimer_ready() {
+    if (!g_ktiming.load(std::memory_order_relaxed)) return false;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    if (g_kt.dev != dev) {
+        for (cudaEvent_t& e : g_kt.ev) {
+            if (e) cudaEventDestroy(e);
+            e = nullptr;
+        }
+        for (cudaEvent_t& e : g_kt.ev)
+            if (cudaEventCreate(&e) != cudaSuccess) return false;
+        g_kt.dev = dev;
+        g_kt.n = 0;
+    }
+    return true;
+}
 }  // namespace
+
+void ktimer_reset() {
+    if (ktimer_ready()) g_kt.n = 0;
+}
+
+void ktimer_before(cudaStream_t s) {
+    if (!ktimer_ready() || g_kt.n >= kMaxTimed) return;
+    g_kt.open = cudaEventRecord(g_kt.ev[2 * g_kt.n], s) == cudaSuccess;
+}
+
+void ktimer_after(cudaStream_t s, const char* kernel) {
+    if (!ktimer_ready() || g_kt.n >= kMaxTimed || !g_kt.open) return;
+    g_kt.open = false;
+    if (cudaEventRecord(g_kt.ev[2 * g_kt.n + 1], s) != cudaSuccess) return;
+    g_kt.name[g_kt.n++] = kernel;
+}
 
 int* device_status_ptr() {
     int dev = 0;
@@ -132,6 +176,7 @@ int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
     int* st = device_status_ptr();
     if (!st) return GDN_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
+    ktimer_reset();
     if (tc_ok && impl != GDN_IMPL_CUDA_CORE) {
         return to_status(launch_prefill_tc(q, k, v, a, b, A_log, dt_bias, initial_state,
                                            cu_seqlens, num_seqs, total_tokens, H_qk, H_v, scale,
@@ -141,13 +186,18 @@ int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
     float* beta = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                            gate_bytes(total_tokens, H_v));
     if (total_tokens > 0) {
+        ktimer_before(s);
         cudaError_t e = launch_gates(a, b, A_log, dt_bias, cu_seqlens, num_seqs, total_tokens,
                                      H_v, G, nullptr, beta, st, s);
         if (e != cudaSuccess) return GDN_ERR_CUDA;
+        ktimer_after(s, "gates");
     }
-    return to_status(launch_prefill_simt(q, k, v, io_dtype, G, beta, initial_state, cu_seqlens,
-                                         num_seqs, total_tokens, H_qk, H_v, d_k, scale, o,
-                                         final_state, st, s));
+    ktimer_before(s);
+    const int rs = to_status(launch_prefill_simt(q, k, v, io_dtype, G, beta, initial_state,
+                                                 cu_seqlens, num_seqs, total_tokens, H_qk, H_v,
+                                                 d_k, scale, o, final_state, st, s));
+    ktimer_after(s, "prefill_simt");
+    return rs;
 }
 
 int gdn_decode_step(const void* q, const void* k, const void* v, int32_t io_dtype,
@@ -175,6 +225,25 @@ int gdn_set_prefill_impl(int32_t impl) {
     if (impl != GDN_IMPL_AUTO && impl != GDN_IMPL_CUDA_CORE && impl != GDN_IMPL_TENSOR_CORE)
         return -GDN_ERR_INVALID_ARG;
     return g_prefill_impl.exchange(impl);
+}
+
+int gdn_set_kernel_timing(int32_t enable) {
+    return g_ktiming.exchange(enable ? 1 : 0);
+}
+
+int gdn_last_prefill_kernel_ms(float* ms, int32_t max_kernels) {
+    if (!ms || max_kernels < 0) return -GDN_ERR_INVALID_ARG;
+    const int n = g_kt.n < max_kernels ? g_kt.n : max_kernels;
+    for (int i = 0; i < n; ++i) {
+        if (cudaEventSynchronize(g_kt.ev[2 * i + 1]) != cudaSuccess ||
+            cudaEventElapsedTime(&ms[i], g_kt.ev[2 * i], g_kt.ev[2 * i + 1]) != cudaSuccess)
+            return -GDN_ERR_CUDA;
+    }
+    return g_kt.n;
+}
+
+const char* gdn_last_prefill_kernel_name(int32_t i) {
+    return (i >= 0 && i < g_kt.n) ? g_kt.name[i] : nullptr;
 }
 
 int gdn_sync_status(void* stream) {

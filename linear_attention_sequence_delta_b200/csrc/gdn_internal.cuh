@@ -71,6 +71,13 @@ __device__ __forceinline__ void set_status(int* status, int code) {
 // Status word of the current device (a __device__ int of this library).
 int* device_status_ptr();
 
+// ---- optional per-kernel timing of gdn_prefill (see gdn_set_kernel_timing) ----
+// While timing is enabled, every kernel launch of gdn_prefill is bracketed by two
+// CUDA events recorded on the launch stream; otherwise these do nothing.
+void ktimer_reset();
+void ktimer_before(cudaStream_t s);
+void ktimer_after(cudaStream_t s, const char* kernel);
+
 cudaError_t launch_gates(const float* a, const float* b, const float* A_log,
                          const float* dt_bias, const int32_t* cu_seqlens, int32_t num_seqs,
                          int64_t total_tokens, int32_t H_v, float* G, float* g, float* beta,

@@ -1022,24 +1022,31 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
     e = cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kChainSmem);
     if (e != cudaSuccess) return e;
+    ktimer_before(s);
     chunk_offsets_kernel<<<1, 256, 0, s>>>(cu_seqlens, N, T, choff, status);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    ktimer_after(s, "chunk_offsets");
     const int64_t unit_bound = (((T + kC - 1) / kC) + N) * (int64_t)H_qk;
     const int64_t grid_cap = (int64_t)2 * num_sms;
     const int prep_grid = (int)(unit_bound < grid_cap ? unit_bound : grid_cap);
     if (prep_grid > 0) {
+        ktimer_before(s);
         prep_kernel<<<prep_grid, kPrepThreads, kPrepSmem, s>>>(
             static_cast<const bf16*>(q), static_cast<const bf16*>(k), a, b, A_log, dt_bias,
             cu_seqlens, choff, N, H_qk, H_v, scale, rec, status);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
+        ktimer_after(s, "prep");
     }
     const int64_t blocks = (int64_t)N * H_v;
+    ktimer_before(s);
     chain_kernel<<<(unsigned)blocks, kChainThreads, kChainSmem, s>>>(
         tm_q, tm_k, tm_v, tm_o, S0, cu_seqlens, choff, T, H_qk, H_v, rec, static_cast<bf16*>(o),
         S_final, status);
-    return cudaGetLastError();
+    e = cudaGetLastError();
+    if (e == cudaSuccess) ktimer_after(s, "chain");
+    return e;
 }
 
 }  // namespace gdn

@@ -29,7 +29,8 @@ _STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "
 # Every symbol include/gdn.h declares (the tests check the library exports them all).
 EXPORTS = ["gdn_status_string", "gdn_version", "gdn_prefill_workspace_size", "gdn_gates",
            "gdn_prefill", "gdn_decode_step", "gdn_sync_status", "gdn_prefill_noalloc",
-           "gdn_set_prefill_impl"]
+           "gdn_set_prefill_impl", "gdn_set_kernel_timing", "gdn_last_prefill_kernel_ms",
+           "gdn_last_prefill_kernel_name"]
 GDN_IMPL_AUTO, GDN_IMPL_CUDA_CORE, GDN_IMPL_TENSOR_CORE = 0, 1, 2
 
 
@@ -70,6 +71,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gdn_sync_status.argtypes = [P]
     lib.gdn_set_prefill_impl.restype = ctypes.c_int
     lib.gdn_set_prefill_impl.argtypes = [i32]
+    lib.gdn_set_kernel_timing.restype = ctypes.c_int
+    lib.gdn_set_kernel_timing.argtypes = [i32]
+    lib.gdn_last_prefill_kernel_ms.restype = ctypes.c_int
+    lib.gdn_last_prefill_kernel_ms.argtypes = [P, i32]
+    lib.gdn_last_prefill_kernel_name.restype = ctypes.c_char_p
+    lib.gdn_last_prefill_kernel_name.argtypes = [i32]
     _lib = lib
     return lib
 
@@ -188,3 +195,20 @@ def gdn_sync_status(device=None) -> int:
     """Synchronise the current stream and return (and clear) the device status word."""
     lib = load_library()
     return int(lib.gdn_sync_status(_stream(device)))
+
+
+def set_kernel_timing(enable: bool) -> bool:
+    """Record CUDA events around every kernel of later gdn_prefill calls; returns the
+    previous setting."""
+    return bool(load_library().gdn_set_kernel_timing(1 if enable else 0))
+
+
+def last_prefill_kernel_times() -> list:
+    """[(kernel name, milliseconds)] of the most recent gdn_prefill call made while
+    kernel timing was enabled (waits for its events)."""
+    lib = load_library()
+    ms = (ctypes.c_float * 4)()
+    n = int(lib.gdn_last_prefill_kernel_ms(ms, 4))
+    if n < 0:
+        raise GDNError(-n, "gdn_last_prefill_kernel_ms")
+    return [(lib.gdn_last_prefill_kernel_name(i).decode(), float(ms[i])) for i in range(min(n, 4))]

@@ -163,3 +163,14 @@ def test_set_prefill_impl(lib):
     assert lib.gdn_set_prefill_impl(2) == 1
     assert lib.gdn_set_prefill_impl(7) == -1      # invalid: unchanged
     assert lib.gdn_set_prefill_impl(0) == 2
+
+
+def test_kernel_timing_switch(lib):
+    prev = lib.gdn_set_kernel_timing(1)
+    assert lib.gdn_set_kernel_timing(0) == 1
+    lib.gdn_set_kernel_timing(prev)
+    assert lib.gdn_last_prefill_kernel_ms(None, 4) == -1
+    ms = (ctypes.c_float * 4)()
+    assert lib.gdn_last_prefill_kernel_ms(ms, -1) == -1
+    assert lib.gdn_last_prefill_kernel_name(-1) is None
+    assert lib.gdn_last_prefill_kernel_name(99) is None

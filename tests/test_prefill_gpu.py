@@ -202,3 +202,19 @@ def test_tensor_core_rejects_fp32(impl_switch):
     P = make_prefill_inputs([64], H_qk=1, H_v=1, d_k=128, d_v=128, io_dtype=torch.float32)
     with pytest.raises(g.GDNError):
         _run(P)
+
+
+def test_kernel_timing_names_and_durations(impl_switch):
+    g = impl_switch
+    P = make_prefill_inputs([300, 77], H_qk=2, H_v=4, d_k=128, d_v=128, seed=31)
+    prev = g.set_kernel_timing(True)
+    try:
+        for impl, names in ((g.GDN_IMPL_TENSOR_CORE, ["chunk_offsets", "prep", "chain"]),
+                            (g.GDN_IMPL_CUDA_CORE, ["gates", "prefill_simt"])):
+            g.set_prefill_impl(impl)
+            _run(P)
+            times = g.last_prefill_kernel_times()
+            assert [n for n, _ in times] == names
+            assert all(0.0 < ms < 1000.0 for _, ms in times)
+    finally:
+        g.set_kernel_timing(prev)
