@@ -66,10 +66,10 @@ constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 2 GHz
 constexpr int kMaxGroup = 16;                    // V heads per QK head handled by prep
 
 // ---- workspace record of one (chunk, V head), written by prep, bulk-copied by chain
-constexpr uint32_t REC_T = 0;        // [64][128 B] T, bf16, sw128 image
+constexpr uint32_t REC_T = 0;        // [64][128 B] T diag(beta), bf16, sw128 image
 constexpr uint32_t REC_P = 8192;     // [64][128 B] P, bf16, sw128 image
 constexpr uint32_t REC_G = 16384;    // factors (floats):
-constexpr int RG_BBE = 0;            //   [64] x (beta_t, beta_t e^{G_t} rk_t)
+constexpr int RG_FK = 0;             //   [64] e^{G_t} rk_t
 constexpr int RG_EGQ = 128;          //   [64] e^{G_t} rq_t
 constexpr int RG_EGL = 192;          //   [64] e^{G_L - G_t} rk_t
 constexpr int RG_GAMMA = 256;        //   e^{G_L}
@@ -346,8 +346,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
             const float G_last = sG[kC - 1];  // = G_{L-1}: tokens past L add g = 0
             if (tid < kC) {
                 const float eg = __expf(sG[tid]);
-                const float bt = sBeta[tid];
-                reinterpret_cast<float2*>(rg + RG_BBE)[tid] = make_float2(bt, bt * eg * rk[tid]);
+                rg[RG_FK + tid] = eg * rk[tid];
                 rg[RG_EGQ + tid] = eg * rq[tid];
                 rg[RG_EGL + tid] = __expf(G_last - sG[tid]) * rk[tid];
             }
@@ -508,11 +507,13 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
                 const int row = idx >> 3, ch = idx & 7;
                 const float4 f0 = *reinterpret_cast<const float4*>(Ts + row * kTsStride + ch * 8);
                 const float4 f1 = *reinterpret_cast<const float4*>(Ts + row * kTsStride + ch * 8 + 4);
-                uint4 w;
-                w.x = pack_bf16x2(f0.x, f0.y);
-                w.y = pack_bf16x2(f0.z, f0.w);
-                w.z = pack_bf16x2(f1.x, f1.y);
-                w.w = pack_bf16x2(f1.z, f1.w);
+                const float4 b0 = *reinterpret_cast<const float4*>(sBeta + ch * 8);
+                const float4 b1 = *reinterpret_cast<const float4*>(sBeta + ch * 8 + 4);
+                uint4 w;  // column s of T times beta_s
+                w.x = pack_bf16x2(f0.x * b0.x, f0.y * b0.y);
+                w.y = pack_bf16x2(f0.z * b0.z, f0.w * b0.w);
+                w.z = pack_bf16x2(f1.x * b1.x, f1.y * b1.y);
+                w.w = pack_bf16x2(f1.z * b1.z, f1.w * b1.w);
                 *reinterpret_cast<uint4*>(R + REC_T + sw128_off(row, ch)) = w;
             }
             __syncthreads();  // Ts, As, Xs and the head scratch are reused
@@ -527,31 +528,33 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
 }
 
 // ==================================== chain =======================================
-constexpr int kChainThreads = 384;  // warps 0-7 state chain, warps 8-11 output and loads
+constexpr int kChainThreads = 416;  // warps 0-7 state, warp 8 MMA issue, warps 9-12 output + loads
 constexpr int kChain = 256;
 constexpr int kOut = 128;
+constexpr int kIssueWarp = 8;
+constexpr int kLoadWarp = 9;
 constexpr int kRing = 3;
 // shared memory map (bytes from a 1024-byte aligned base)
 constexpr uint32_t SLOT_KQ = 0;        // [2 col blocks][K rows 0-63, Q rows 64-127][128 B], sw128
 constexpr uint32_t SLOT_V = 32768;     // [2 col blocks][64 rows][128 B] V, sw128
-constexpr uint32_t SLOT_REC = 49152;   // the (chunk, V head) record: T, P, factors
+constexpr uint32_t SLOT_REC = 49152;   // the (chunk, V head) record: T diag(beta), P, factors
 constexpr uint32_t kSlotBytes = 67584;
 constexpr uint32_t kSlotTx = 6 * 8192 + kRecBytes;  // six 64x64 tiles + the record
-constexpr uint32_t CS_ID = kRing * kSlotBytes;      // [64][128 B] bf16 identity, sw128
-constexpr uint32_t CS_OST = CS_ID + 8192;           // [2 col blocks][64 t][128 B] o, sw128
-constexpr uint32_t CS_BAR = CS_OST + 16384;         // full[3], mma, out, ofree, drain
-constexpr uint32_t CS_TMEM = CS_BAR + 64;
-constexpr uint32_t CS_ERR = CS_BAR + 68;
-constexpr size_t kChainSmem = CS_BAR + 128 + 1024;
+constexpr uint32_t CS_OST = kRing * kSlotBytes;     // [2 col blocks][64 t][128 B] o, sw128
+constexpr uint32_t CS_BAR = CS_OST + 16384;         // barriers (see below)
+constexpr uint32_t CS_TMEM = CS_BAR + 128;
+constexpr uint32_t CS_ERR = CS_BAR + 132;
+constexpr size_t kChainSmem = CS_BAR + 256 + 1024;
 
 // tensor memory columns (512 allocated)
 constexpr uint32_t TM_S = 0;      // 128: state, fp32
-constexpr uint32_t TM_S0B = 128;  // 64: state as bf16 pairs; later the decay-scaled Vn^T pairs
-constexpr uint32_t TM_D1K = 192;  // 64: S0 K^T
-constexpr uint32_t TM_D1Q = 256;  // 64: S0 Q^T
-constexpr uint32_t TM_DV = 320;   // 64: V^T; Y^T pairs overwrite columns 0-15 and 32-47
-constexpr uint32_t TM_D3 = 384;   // 64: Vn^T; Vn^T pairs overwrite columns 0-15 and 32-47
-constexpr uint32_t TM_D4 = 448;   // 64: (P Vn)^T
+constexpr uint32_t TM_S0B = 128;  // 64: state as bf16 pairs
+constexpr uint32_t TM_D1K = 192;  // 64: S0 K^T; Z^T pairs overwrite columns 0-15 and 32-47,
+                                  //     then the decay-scaled Vn^T pairs columns 0-31
+constexpr uint32_t TM_D1Q0 = 256; // 64: S0 Q^T of even chunks
+constexpr uint32_t TM_D3 = 320;   // 64: Vn^T; Vn^T pairs overwrite columns 0-15 and 32-47
+constexpr uint32_t TM_D1Q1 = 384; // 64: S0 Q^T of odd chunks
+constexpr uint32_t TM_D4 = 448;   // 64: Vn^T P^T
 constexpr uint32_t kTmemCols = 512;
 
 // Column (in 32-bit words) of the K=16 slice ks of a 64-token bf16 operand that
@@ -561,31 +564,42 @@ __device__ __forceinline__ uint32_t split_pairs_col(int ks) {
     return (uint32_t)((ks >> 1) * 32 + (ks & 1) * 8);
 }
 
-// One block per (sequence, V head). Warps 0-7 carry the state: two warps share
-// each TMEM lane quarter, warp w owning value rows 32 (w & 3) .. + 31 and, of
-// every 64- or 128-column quantity of those rows, the half w >> 2; warp 0 also
-// issues the MMAs. Warps 8-11 (one per lane quarter) turn each chunk's output
-// accumulators into o and, once a chunk's ring slot is no longer read, load the
-// chunk three ahead into it (TMA tiles for K, Q, V and one bulk copy of the
-// record).
+// Byte offset of element (row t, column i) of a [2 col blocks][64 rows][128 B]
+// bf16 tile in the 128-byte swizzle.
+__device__ __forceinline__ uint32_t tile64_off(int t, int i) {
+    return (uint32_t)(i >> 6) * 8192u + (uint32_t)t * 128u +
+           ((uint32_t)(((i & 63) >> 3) ^ (t & 7)) << 4) + (uint32_t)(i & 7) * 2u;
+}
+
+// One block per (sequence, V head).
+//   warps 0-7   the state: two warps share each TMEM lane quarter, warp w owning
+//               value rows 32 (w & 3) .. + 31 and, of every 64- or 128-column
+//               quantity of those rows, the half w >> 2. After each step's TMEM
+//               stores they arrive on `rdy` (one lane per warp) and go on.
+//   warp 8      issues every MMA (elect.sync), each group once its inputs are
+//               ready, and commits them to mbarriers; it does nothing else, so a
+//               full tensor-core queue never holds up the state warps.
+//   warps 9-12  (one per lane quarter) turn each chunk's output accumulators into o
+//               (S0 Q^T alternates between two accumulators) and, once a chunk's
+//               ring slot is no longer read, load the chunk three ahead into it
+//               (TMA tiles for K, Q, V and one bulk copy of the record).
 __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-    const float* __restrict__ S0g,
-    const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict__ choff, int64_t T_total,
-    int H_qk, int H_v, const uint8_t* __restrict__ rec, bf16* __restrict__ o,
-    float* __restrict__ Sfg, int* status) {
+    const float* __restrict__ S0g, const int32_t* __restrict__ cu_seqlens,
+    const int32_t* __restrict__ choff, int64_t T_total, int H_qk, int H_v,
+    const uint8_t* __restrict__ rec, bf16* __restrict__ o, float* __restrict__ Sfg, int* status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(sm + CS_BAR);
-    uint64_t* mbar = full + kRing;      // chain MMA completions
-    uint64_t* obar = full + kRing + 1;  // a chunk's output accumulators complete
-    uint64_t* ofree = full + kRing + 2; // output accumulators read (one arrive per output warp)
-    uint64_t* dbar = full + kRing + 3;  // drain of in-flight MMAs after an error
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + CS_BAR);  // [3] slot landed
+    uint64_t* mbar = full + kRing;         // chain MMA completions
+    uint64_t* obar = mbar + 1;             // [2] chunk parity b: output accumulators complete
+    uint64_t* ofree = mbar + 3;            // [2] chunk parity b: output accumulators read
+    uint64_t* rdy = mbar + 5;              // a state step's TMEM operands written (8 arrivals)
+    uint64_t* dbar = mbar + 6;             // drain of in-flight MMAs before the exit
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + CS_TMEM);
-    volatile int* s_err = reinterpret_cast<volatile int*>(sm + CS_ERR);       // chain warps
-    volatile int* s_lerr = reinterpret_cast<volatile int*>(sm + CS_ERR + 4);  // output warps
+    volatile int* s_err = reinterpret_cast<volatile int*>(sm + CS_ERR);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -605,24 +619,16 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
     if (tid == 0) {
         for (int i = 0; i < kRing; ++i) mbar_init(&full[i], 1);
         mbar_init(mbar, 1);
-        mbar_init(obar, 1);
-        mbar_init(ofree, 4);
+        mbar_init(&obar[0], 1);
+        mbar_init(&obar[1], 1);
+        mbar_init(&ofree[0], 4);
+        mbar_init(&ofree[1], 4);
+        mbar_init(rdy, 8);
         mbar_init(dbar, 1);
         *s_err = 0;
-        *s_lerr = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp < 8) {  // the 64x64 bf16 identity (B operand of the V^T MMA)
-#pragma unroll
-        for (int it = 0; it < 2; ++it) {
-            const int idx = tid + kChain * it;  // 0..511
-            const int row = idx >> 3, ch = idx & 7;
-            uint4 w = make_uint4(0u, 0u, 0u, 0u);
-            if ((row >> 3) == ch) (&w.x)[(row & 7) >> 1] = 0x3F80u << (16 * (row & 1));
-            *reinterpret_cast<uint4*>(sm + CS_ID + sw128_off(row, ch)) = w;
-        }
-        fence_proxy_async_smem();
-    } else if (warp == 8 && lane == 0) {
+    if (warp == kLoadWarp && lane == 0) {
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
@@ -649,91 +655,186 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
                  &full[st]);
     };
 
-    if (warp >= 8) {
+    if (warp > kIssueWarp) {
         // ============================ output + loads ===================================
         const int qo = warp & 3;
         const int row = qo * 32 + lane;
+        const int to = tid - (kIssueWarp + 1) * 32;  // 0..127
         const uint32_t ctl = tmem + ((uint32_t)(qo * 32) << 16);
+        uint8_t* ost = sm + CS_OST;
+        const bool loader = warp == kLoadWarp && lane == 0;
         int issued = nchunks < kRing ? nchunks : kRing;
-        if (warp == 8 && lane == 0)
+        if (loader)
             for (int c = 0; c < issued; ++c) issue_loads(c);
         __syncwarp();
-        uint8_t* ost = sm + CS_OST;
-        // this thread's element (t, i) of the staged o tile: block i / 64, 16-byte
-        // chunk (i % 64) / 8 swizzled with t % 8, halfword i % 8
-        const uint32_t o_row = (uint32_t)(row >> 6) * 8192u + (uint32_t)(row & 7) * 2u;
-        const uint32_t o_chk = (uint32_t)((row & 63) >> 3);
 #pragma unroll 1
-        for (int c = 0; c < nchunks; ++c) {
-            const bool ok = mbar_wait_bounded(obar, c & 1, kWaitCycles);
-            if (!ok) *s_lerr = 1;
-            if (warp == 8 && lane == 0) bulk_wait_group_read<0>();  // staging free again
+        for (int cp = 0; cp < nchunks; ++cp) {
+            const int b = cp & 1;
+            const bool ok = mbar_wait_bounded(&obar[b], (cp >> 1) & 1, kWaitCycles);
+            if (!ok) *s_err = 1;
+            if (loader) bulk_wait_group_read<0>();  // staging free again
             if (named_bar_any(2, kOut, !ok || *s_err != 0)) break;
             tc_fence_after();
-            const float* rg = reinterpret_cast<const float*>(sm + (c % kRing) * kSlotBytes +
-                                                             SLOT_REC + REC_G);
-            const float4* eg4 = reinterpret_cast<const float4*>(rg + RG_EGQ);
-            float ov[64];
+            const float4* eg4 = reinterpret_cast<const float4*>(
+                sm + (cp % kRing) * kSlotBytes + SLOT_REC + REC_G + 4 * RG_EGQ);
+            const uint32_t qacc = ctl + (b ? TM_D1Q1 : TM_D1Q0);
+            // this thread's column of the staged tile; laundered so that the 64 element
+            // addresses are formed per chunk rather than held in registers across chunks
+            uint32_t ocol = smem_u32(ost) + (uint32_t)(row >> 6) * 8192u + (uint32_t)(row & 7) * 2u;
+            uint32_t ochk = (uint32_t)((row & 63) >> 3);
+            asm volatile("" : "+r"(ocol), "+r"(ochk));
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 float xq[32], xi[32];
-                tmem_ld32x2_sync(ctl + TM_D1Q + 32 * hf, ctl + TM_D4 + 32 * hf, xq, xi);
+                tmem_ld32x2_sync(qacc + 32 * hf, ctl + TM_D4 + 32 * hf, xq, xi);
+                if (hf == 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&ofree[b]);  // the accumulators may be overwritten
+                }
 #pragma unroll
                 for (int e4 = 0; e4 < 8; ++e4) {
                     const float4 w = eg4[8 * hf + e4];
-                    const int e = 4 * e4;
-                    ov[32 * hf + e] = fmaf(w.x, xq[e], xi[e]);
-                    ov[32 * hf + e + 1] = fmaf(w.y, xq[e + 1], xi[e + 1]);
-                    ov[32 * hf + e + 2] = fmaf(w.z, xq[e + 2], xi[e + 2]);
-                    ov[32 * hf + e + 3] = fmaf(w.w, xq[e + 3], xi[e + 3]);
+                    const float wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int t = 32 * hf + 4 * e4 + u, e = 4 * e4 + u;
+                        const uint32_t a = ocol + (uint32_t)t * 128u + ((ochk ^ (uint32_t)(t & 7)) << 4);
+                        const bf16 v = __float2bfloat16_rn(fmaf(wv[u], xq[e], xi[e]));
+                        asm volatile("st.shared.b16 [%0], %1;" ::"r"(a),
+                                     "h"(*reinterpret_cast<const unsigned short*>(&v))
+                                     : "memory");
+                    }
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(ofree);  // the accumulators may be overwritten
-#pragma unroll
-            for (int t = 0; t < kC; ++t)
-                *reinterpret_cast<bf16*>(ost + o_row + (uint32_t)t * 128u +
-                                         ((o_chk ^ (uint32_t)(t & 7)) << 4)) =
-                    __float2bfloat16_rn(ov[t]);
             fence_proxy_async_smem();
-            named_bar_sync(2, kOut);  // staged; every output warp is done with this slot
-            const int64_t t0 = s0 + (int64_t)c * kC;
+            named_bar_sync(2, kOut);  // staged; every output warp is done with the slot
+            const int64_t t0 = s0 + (int64_t)cp * kC;
             const int L = (int)min((int64_t)kC, s1 - t0);
             if (L == kC) {
-                if (warp == 8 && lane == 0) {
+                if (loader) {
                     tma_store_3d(&tm_o, 0, h, (int32_t)t0, ost);
                     tma_store_3d(&tm_o, 64, h, (int32_t)t0, ost + 8192);
                     bulk_commit_group();
                 }
             } else {
                 // the sequence's last rows only: plain 16-byte stores
-                for (int idx = tid - kChain; idx < L * 16; idx += kOut) {
+                for (int idx = to; idx < L * 16; idx += kOut) {
                     const int r = idx >> 4, ch = idx & 15;
-                    const uint4 w = *reinterpret_cast<const uint4*>(
-                        ost + (uint32_t)(ch >> 3) * 8192u + (uint32_t)r * 128u +
-                        ((uint32_t)((ch & 7) ^ (r & 7)) << 4));
+                    const uint4 w = *reinterpret_cast<const uint4*>(ost + tile64_off(r, ch * 8));
                     *reinterpret_cast<uint4*>(o + ((size_t)(t0 + r) * H_v + h) * kD + ch * 8) = w;
                 }
                 named_bar_sync(2, kOut);
             }
-            if (warp == 8 && lane == 0 && c + kRing < nchunks) {
-                issue_loads(c + kRing);
-                issued = c + kRing + 1;
+            if (loader && cp + kRing < nchunks) {
+                issue_loads(cp + kRing);
+                issued = cp + kRing + 1;
             }
             __syncwarp();
         }
-        if (warp == 8 && lane == 0) bulk_wait_group<0>();  // o stores complete
-        // Leave nothing in flight into shared memory (loads the chain did not
-        // consume are only possible after an error).
-        if (warp == 8 && lane == 0) {
+        if (loader) {
+            bulk_wait_group<0>();  // o stores complete
+            // Leave nothing in flight into shared memory (loads the chain did not
+            // consume are only possible after an error).
             for (int c = issued - 1; c >= 0 && c >= issued - kRing; --c)
                 if (!mbar_wait_bounded(&full[c % kRing], (c / kRing) & 1, kWaitCycles))
-                    *s_lerr = 1;
+                    *s_err = 1;
+        }
+        __syncwarp();
+    } else if (warp == kIssueWarp) {
+        // ================================ MMA issue =====================================
+        uint32_t rphase = 0;
+        auto wait_rdy = [&]() -> bool {
+            const bool ok = mbar_wait_bounded(rdy, rphase, kWaitCycles);
+            rphase ^= 1u;
+            tc_fence_after();
+            __syncwarp();
+            return ok;
+        };
+        constexpr uint32_t id64 = idesc_bf16_f32(128, 64, 0, 0);
+#pragma unroll 1
+        for (int c = 0; c < nchunks; ++c) {
+            const int st = c % kRing;
+            uint8_t* slot = sm + st * kSlotBytes;
+            const uint32_t kq = smem_u32(slot + SLOT_KQ);
+            const uint32_t vt = smem_u32(slot + SLOT_V);
+            const uint32_t tt = smem_u32(slot + SLOT_REC + REC_T);
+            const uint32_t ptile = smem_u32(slot + SLOT_REC + REC_P);
+            bool ok = mbar_wait_bounded(&full[st], (c / kRing) & 1, kWaitCycles);
+            // (1) the bf16 state is written: S0 K^T, then V^T (T diag(beta))^T
+            ok = wait_rdy() && ok;
+            if (!ok || *s_err) { *s_err = 1; break; }
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t off = (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u;
+                mma_bf16_ts_warp(tmem + TM_D1K, tmem + TM_S0B + 8 * ks,
+                                 smem_desc_sw128(kq + off, 16, 1024), id64, ks > 0);
+            }
+            mma_commit_warp(mbar);
+            {
+                constexpr uint32_t id_v = idesc_bf16_f32(128, 64, 1, 0);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16_ss_warp(tmem + TM_D3, smem_desc_sw128(vt + ks * 2048, 8192, 1024),
+                                     smem_desc_sw128(tt + ks * 32, 16, 1024), id_v, ks > 0);
+            }
+            // (2) Z^T is written: Vn^T += Z^T (T diag(beta))^T; then S0 Q^T
+            if (!wait_rdy() || *s_err) { *s_err = 1; break; }
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16_ts_warp(tmem + TM_D3, tmem + TM_D1K + split_pairs_col(ks),
+                                 smem_desc_sw128(tt + ks * 32, 16, 1024), id64, 1);
+            mma_commit_warp(mbar);
+            if (c >= 2 && !mbar_wait_bounded(&ofree[c & 1], ((c - 2) >> 1) & 1, kWaitCycles)) {
+                *s_err = 1;
+                break;
+            }
+            __syncwarp();
+            {
+                const uint32_t qacc = tmem + ((c & 1) ? TM_D1Q1 : TM_D1Q0);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t off =
+                        8192u + (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u;
+                    mma_bf16_ts_warp(qacc, tmem + TM_S0B + 8 * ks,
+                                     smem_desc_sw128(kq + off, 16, 1024), id64, ks > 0);
+                }
+            }
+            // (3) the Vn^T pairs are written: the state update, then Vn^T P^T
+            if (!wait_rdy() || *s_err) { *s_err = 1; break; }
+            {
+                constexpr uint32_t id_s = idesc_bf16_f32(128, 128, 0, 1);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16_ts_warp(tmem + TM_S, tmem + TM_D1K + 8 * ks,
+                                     smem_desc_sw128(kq + ks * 2048, 16384, 1024), id_s, 1);
+            }
+            mma_commit_warp(mbar);
+            if (c >= 1 &&
+                !mbar_wait_bounded(&ofree[(c - 1) & 1], ((c - 1) >> 1) & 1, kWaitCycles)) {
+                *s_err = 1;
+                break;
+            }
+            __syncwarp();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16_ts_warp(tmem + TM_D4, tmem + TM_D3 + split_pairs_col(ks),
+                                 smem_desc_sw128(ptile + ks * 32, 16, 1024), id64, ks > 0);
+            mma_commit_warp(&obar[c & 1]);
+        }
+        __syncwarp();
+        // no MMA may still run when the tensor memory is freed
+        mma_commit_warp(dbar);
+        (void)mbar_wait_bounded(dbar, 0, kWaitCycles);
+        if (*s_err) {  // wake the output warps so they see the error and leave
+            if (lane == 0) {
+                mbar_arrive(&obar[0]);
+                mbar_arrive(&obar[1]);
+            }
         }
         __syncwarp();
     } else {
-        // ================================ chain ========================================
+        // ================================ state ========================================
         const int qd = warp & 3;              // TMEM lane quarter
         const int hh = warp >> 2;             // column half
         const int row = qd * 32 + lane;       // value row i = TMEM lane
@@ -758,12 +859,21 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
         tmem_wait_st();
 
         uint32_t mphase = 0;
-        auto wait_mma = [&]() -> bool {
-            const bool ok = mbar_wait_bounded(mbar, mphase, kWaitCycles);
+        auto wait_mma = [&]() -> bool {  // warp-uniform
+            bool ok = mbar_wait_bounded(mbar, mphase, kWaitCycles);
             mphase ^= 1u;
+            ok = !__any_sync(0xffffffffu, !ok || *s_err != 0);
             if (!ok) *s_err = 1;
             tc_fence_after();
             return ok;
+        };
+        // this warp's TMEM operands of the step are written (and, before that, any
+        // shared-memory writes fenced): one arrival for the issuing warp
+        auto signal_rdy = [&]() {
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(rdy);
         };
 
 #pragma unroll 1
@@ -771,18 +881,21 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
             const int st = c % kRing;
             uint8_t* slot = sm + st * kSlotBytes;
             const float* rg = reinterpret_cast<const float*>(slot + SLOT_REC + REC_G);
-            const uint32_t kq = smem_u32(slot + SLOT_KQ);
             const int64_t t0 = s0 + (int64_t)c * kC;
             const int L = (int)min((int64_t)kC, s1 - t0);
 
             // ---- the previous state update and this chunk's data ---------------------
-            bool ok = c > 0 ? wait_mma() : true;
-            if (!mbar_wait_bounded(&full[st], (c / kRing) & 1, kWaitCycles)) {
-                ok = false;
-                *s_err = 1;
+            if (c > 0 && !wait_mma()) break;
+            {
+                const bool okf = mbar_wait_bounded(&full[st], (c / kRing) & 1, kWaitCycles);
+                if (__any_sync(0xffffffffu, !okf)) {
+                    *s_err = 1;
+                    break;
+                }
             }
             if (L < kC) {
-                // rows past the sequence's end hold the next sequence's tokens: zero them
+                // rows past the sequence's end hold the next sequence's tokens (or TMA
+                // zero fill): zero them
                 const int nz = (kC - L) * 8;  // 16-byte chunks per 64-column tile
                 for (int idx = tid; idx < 6 * nz; idx += kChain) {
                     const int tile = idx / nz, r = L + (idx % nz) / 8, ch = idx & 7;
@@ -792,96 +905,50 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
                         make_uint4(0u, 0u, 0u, 0u);
                 }
                 fence_proxy_async_smem();
-                named_bar_sync(1, kChain);
-            }
-            if (warp == 0) {  // V^T: no dependence on the state, runs under the S step
-                __syncwarp();
-                constexpr uint32_t id_v = idesc_bf16_f32(128, 64, 1, 0);
-                const uint32_t vt = smem_u32(slot + SLOT_V), idt = smem_u32(sm + CS_ID);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ss_warp(tmem + TM_DV, smem_desc_sw128(vt + ks * 2048, 8192, 1024),
-                                     smem_desc_sw128(idt + ks * 32, 16, 1024), id_v, ks > 0);
             }
 
             // ---- state: bf16 copy (A operand of S0 K^T and S0 Q^T) ----------------------
-            float sx[32], sy[32];
-            tmem_ld32x2_sync(ctl + TM_S + 64 * hh, ctl + TM_S + 64 * hh + 32, sx, sy);
-            {
+#pragma unroll
+            for (int cb = 0; cb < 2; ++cb) {
+                float x[32];
+                tmem_ld32_sync(ctl + TM_S + 64 * hh + 32 * cb, x);
                 uint32_t pk[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(sx[2 * e], sx[2 * e + 1]);
-                tmem_st16(ctl + TM_S0B + 32 * hh, pk);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(sy[2 * e], sy[2 * e + 1]);
-                tmem_st16(ctl + TM_S0B + 32 * hh + 16, pk);
+                for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
+                tmem_st16(ctl + TM_S0B + 32 * hh + 16 * cb, pk);
             }
-            tmem_wait_st();
-            tc_fence_before();
-            if (named_bar_any(1, kChain, !ok)) break;
-            tc_fence_after();
-            if (warp == 0) {
-                constexpr uint32_t id64 = idesc_bf16_f32(128, 64, 0, 0);
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t off = (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u;
-                    mma_bf16_ts_warp(tmem + TM_D1K, tmem + TM_S0B + 8 * ks,
-                                     smem_desc_sw128(kq + off, 16, 1024), id64, ks > 0);
-                }
-                mma_commit_warp(mbar);
-                // S0 Q^T overwrites the accumulator the output warps read for chunk c-1
-                if (c > 0 && !mbar_wait_bounded(ofree, (c - 1) & 1, kWaitCycles)) *s_err = 1;
-                __syncwarp();
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t off =
-                        8192u + (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u;
-                    mma_bf16_ts_warp(tmem + TM_D1Q, tmem + TM_S0B + 8 * ks,
-                                     smem_desc_sw128(kq + off, 16, 1024), id64, ks > 0);
-                }
-            }
+            signal_rdy();
             {  // S <- e^{G_L} S while the MMAs run (they read only the bf16 copy)
                 const float gamma = rg[RG_GAMMA];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    sx[e] *= gamma;
-                    sy[e] *= gamma;
+                for (int cb = 0; cb < 2; ++cb) {
+                    float x[32];
+                    tmem_ld32_sync(ctl + TM_S + 64 * hh + 32 * cb, x);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) x[e] *= gamma;
+                    tmem_st32(ctl + TM_S + 64 * hh + 32 * cb, x);
                 }
-                tmem_st32(ctl + TM_S + 64 * hh, sx);
-                tmem_st32(ctl + TM_S + 64 * hh + 32, sy);
             }
 
-            // ---- Y^T = beta (V - e^G rk X)^T for this thread's 32 tokens --------------
-            ok = wait_mma();  // S0 K^T and V^T
+            // ---- Z^T = -(e^G rk) (S0 K^T) for this thread's 32 tokens, in place ----------
+            if (!wait_mma()) break;  // S0 K^T
             {
-                const float4* bbe = reinterpret_cast<const float4*>(rg + RG_BBE) + 16 * hh;
-                float x[32], vv[32];
-                tmem_ld32x2_sync(ctl + TM_D1K + 32 * hh, ctl + TM_DV + 32 * hh, x, vv);
+                const float4* fk4 = reinterpret_cast<const float4*>(rg + RG_FK) + 8 * hh;
+                float x[32];
+                tmem_ld32_sync(ctl + TM_D1K + 32 * hh, x);
                 uint32_t pk[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float4 f = bbe[e];
-                    pk[e] = pack_bf16x2(fmaf(f.x, vv[2 * e], -f.y * x[2 * e]),
-                                        fmaf(f.z, vv[2 * e + 1], -f.w * x[2 * e + 1]));
+                for (int e4 = 0; e4 < 8; ++e4) {
+                    const float4 f = fk4[e4];
+                    pk[2 * e4] = pack_bf16x2(-f.x * x[4 * e4], -f.y * x[4 * e4 + 1]);
+                    pk[2 * e4 + 1] = pack_bf16x2(-f.z * x[4 * e4 + 2], -f.w * x[4 * e4 + 3]);
                 }
-                tmem_st16(ctl + TM_DV + 32 * hh, pk);  // over the V^T columns just read
+                tmem_st16(ctl + TM_D1K + 32 * hh, pk);  // over the columns just read
             }
-            tmem_wait_st();
-            tc_fence_before();
-            if (named_bar_any(1, kChain, !ok)) break;
-            tc_fence_after();
-            if (warp == 0) {
-                constexpr uint32_t id = idesc_bf16_f32(128, 64, 0, 0);
-                const uint32_t tt = smem_u32(slot + SLOT_REC + REC_T);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ts_warp(tmem + TM_D3, tmem + TM_DV + split_pairs_col(ks),
-                                     smem_desc_sw128(tt + ks * 32, 16, 1024), id, ks > 0);
-                mma_commit_warp(mbar);
-            }
+            signal_rdy();  // (its wait also covers the rescaled state)
 
             // ---- Vn^T -> bf16 pairs (for P Vn) and decay-scaled pairs (state update) --
-            ok = wait_mma();  // Vn^T (and S0 Q^T)
+            if (!wait_mma()) break;  // Vn^T
             {
                 const float4* egl4 = reinterpret_cast<const float4*>(rg + RG_EGL) + 8 * hh;
                 float x[32];
@@ -896,27 +963,9 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
                     ps[2 * e4 + 1] = pack_bf16x2(x[4 * e4 + 2] * w.z, x[4 * e4 + 3] * w.w);
                 }
                 tmem_st16(ctl + TM_D3 + 32 * hh, pk);   // over the Vn^T columns just read
-                tmem_st16(ctl + TM_S0B + 16 * hh, ps);  // the bf16 state is consumed
+                tmem_st16(ctl + TM_D1K + 16 * hh, ps);  // Z^T there has been consumed
             }
-            tmem_wait_st();  // also covers the rescaled state stored above
-            tc_fence_before();
-            if (named_bar_any(1, kChain, !ok)) break;
-            tc_fence_after();
-            if (warp == 0) {
-                constexpr uint32_t id_s = idesc_bf16_f32(128, 128, 0, 1);
-                constexpr uint32_t id_o = idesc_bf16_f32(128, 64, 0, 0);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ts_warp(tmem + TM_S, tmem + TM_S0B + 8 * ks,
-                                     smem_desc_sw128(kq + ks * 2048, 16384, 1024), id_s, 1);
-                mma_commit_warp(mbar);
-                const uint32_t ptile = smem_u32(slot + SLOT_REC + REC_P);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ts_warp(tmem + TM_D4, tmem + TM_D3 + split_pairs_col(ks),
-                                     smem_desc_sw128(ptile + ks * 32, 16, 1024), id_o, ks > 0);
-                mma_commit_warp(obar);
-            }
+            signal_rdy();
         }
         bool fin = !*s_err;
         if (fin && nchunks > 0) fin = wait_mma();  // the last state update
@@ -932,20 +981,12 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
                     d4[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
             }
         }
-        // After an error: no MMA may still run when the tensor memory is freed, and
-        // the output warps are woken to see the error and leave.
-        const bool err = __any_sync(0xffffffffu, *s_err != 0);
-        if (warp == 0 && err) {
-            mma_commit_warp(dbar);
-            (void)mbar_wait_bounded(dbar, 0, kWaitCycles);
-        }
-        if (tid == 0 && err) mbar_arrive(obar);
     }
 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (tid == 0 && (*s_err || *s_lerr)) set_status(status, kStatusTimeout);
+    if (tid == 0 && *s_err) set_status(status, kStatusTimeout);
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
