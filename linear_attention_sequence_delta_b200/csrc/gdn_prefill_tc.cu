@@ -547,7 +547,7 @@ constexpr uint32_t CS_ERR = CS_BAR + 132;
 constexpr size_t kChainSmem = CS_BAR + 256 + 1024;
 
 // tensor memory columns (512 allocated)
-constexpr uint32_t TM_S = 0;      // 128: state, fp32
+constexpr uint32_t TM_U = 0;      // 128: the chunk's state increment (scaled Vn^T) K, fp32
 constexpr uint32_t TM_S0B = 128;  // 64: state as bf16 pairs
 constexpr uint32_t TM_D1K = 192;  // 64: S0 K^T; Z^T pairs overwrite columns 0-15 and 32-47,
                                   //     then the decay-scaled Vn^T pairs columns 0-31
@@ -572,10 +572,11 @@ __device__ __forceinline__ uint32_t tile64_off(int t, int i) {
 }
 
 // One block per (sequence, V head).
-//   warps 0-7   the state: two warps share each TMEM lane quarter, warp w owning
-//               value rows 32 (w & 3) .. + 31 and, of every 64- or 128-column
-//               quantity of those rows, the half w >> 2. After each step's TMEM
-//               stores they arrive on `rdy` (one lane per warp) and go on.
+//   warps 0-7   the state, fp32 in registers: two warps share each TMEM lane
+//               quarter, warp w owning value rows 32 (w & 3) .. + 31 and, of every
+//               64- or 128-column quantity of those rows (the state included), the
+//               half w >> 2. After each step's TMEM stores they arrive on `rdy`
+//               (one lane per warp) and go on.
 //   warp 8      issues every MMA (elect.sync), each group once its inputs are
 //               ready, and commits them to mbarriers; it does nothing else, so a
 //               full tensor-core queue never holds up the state warps.
@@ -800,14 +801,14 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
                                      smem_desc_sw128(kq + off, 16, 1024), id64, ks > 0);
                 }
             }
-            // (3) the Vn^T pairs are written: the state update, then Vn^T P^T
+            // (3) the Vn^T pairs are written: the state increment, then Vn^T P^T
             if (!wait_rdy() || *s_err) { *s_err = 1; break; }
             {
                 constexpr uint32_t id_s = idesc_bf16_f32(128, 128, 0, 1);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ts_warp(tmem + TM_S, tmem + TM_D1K + 8 * ks,
-                                     smem_desc_sw128(kq + ks * 2048, 16384, 1024), id_s, 1);
+                    mma_bf16_ts_warp(tmem + TM_U, tmem + TM_D1K + 8 * ks,
+                                     smem_desc_sw128(kq + ks * 2048, 16384, 1024), id_s, ks > 0);
             }
             mma_commit_warp(mbar);
             if (c >= 1 &&
@@ -840,23 +841,18 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
         const int row = qd * 32 + lane;       // value row i = TMEM lane
         const uint32_t ctl = tmem + ((uint32_t)(qd * 32) << 16);
         const size_t sbase = ((size_t)n * H_v + h) * kD * kD + (size_t)row * kD + 64 * hh;
-#pragma unroll 1
-        for (int cb = 0; cb < 2; ++cb) {  // initial state -> TMEM (this thread's 64 columns)
-            float x[32];
-            if (S0g) {
-                const float4* src = reinterpret_cast<const float4*>(S0g + sbase + 32 * cb);
+        float S[64];  // S[i][64 hh + e]
+        if (S0g) {
+            const float4* src = reinterpret_cast<const float4*>(S0g + sbase);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float4 f = src[e];
-                    x[4 * e] = f.x; x[4 * e + 1] = f.y; x[4 * e + 2] = f.z; x[4 * e + 3] = f.w;
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < 32; ++e) x[e] = 0.f;
+            for (int e = 0; e < 16; ++e) {
+                const float4 f = src[e];
+                S[4 * e] = f.x; S[4 * e + 1] = f.y; S[4 * e + 2] = f.z; S[4 * e + 3] = f.w;
             }
-            tmem_st32(ctl + TM_S + 64 * hh + 32 * cb, x);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 64; ++e) S[e] = 0.f;
         }
-        tmem_wait_st();
 
         uint32_t mphase = 0;
         auto wait_mma = [&]() -> bool {  // warp-uniform
@@ -875,7 +871,19 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
             __syncwarp();
             if (lane == 0) mbar_arrive(rdy);
         };
+        // S <- gamma S + U (the previous chunk's decay and increment)
+        auto apply_update = [&](float gamma) {
+#pragma unroll
+            for (int cb = 0; cb < 2; ++cb) {
+                float u[32];
+                tmem_ld32_sync(ctl + TM_U + 64 * hh + 32 * cb, u);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) S[32 * cb + e] = fmaf(gamma, S[32 * cb + e], u[e]);
+            }
+        };
 
+        float gamma = 1.f;
+        bool done = true;
 #pragma unroll 1
         for (int c = 0; c < nchunks; ++c) {
             const int st = c % kRing;
@@ -884,12 +892,16 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
             const int64_t t0 = s0 + (int64_t)c * kC;
             const int L = (int)min((int64_t)kC, s1 - t0);
 
-            // ---- the previous state update and this chunk's data ---------------------
-            if (c > 0 && !wait_mma()) break;
+            // ---- the previous chunk's state update and this chunk's data -------------
+            if (c > 0) {
+                if (!wait_mma()) { done = false; break; }
+                apply_update(gamma);
+            }
             {
                 const bool okf = mbar_wait_bounded(&full[st], (c / kRing) & 1, kWaitCycles);
                 if (__any_sync(0xffffffffu, !okf)) {
                     *s_err = 1;
+                    done = false;
                     break;
                 }
             }
@@ -910,76 +922,65 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
             // ---- state: bf16 copy (A operand of S0 K^T and S0 Q^T) ----------------------
 #pragma unroll
             for (int cb = 0; cb < 2; ++cb) {
-                float x[32];
-                tmem_ld32_sync(ctl + TM_S + 64 * hh + 32 * cb, x);
                 uint32_t pk[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
+                for (int e = 0; e < 16; ++e)
+                    pk[e] = pack_bf16x2(S[32 * cb + 2 * e], S[32 * cb + 2 * e + 1]);
                 tmem_st16(ctl + TM_S0B + 32 * hh + 16 * cb, pk);
             }
             signal_rdy();
-            {  // S <- e^{G_L} S while the MMAs run (they read only the bf16 copy)
-                const float gamma = rg[RG_GAMMA];
-#pragma unroll
-                for (int cb = 0; cb < 2; ++cb) {
-                    float x[32];
-                    tmem_ld32_sync(ctl + TM_S + 64 * hh + 32 * cb, x);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) x[e] *= gamma;
-                    tmem_st32(ctl + TM_S + 64 * hh + 32 * cb, x);
-                }
-            }
+            gamma = rg[RG_GAMMA];
 
             // ---- Z^T = -(e^G rk) (S0 K^T) for this thread's 32 tokens, in place ----------
-            if (!wait_mma()) break;  // S0 K^T
-            {
-                const float4* fk4 = reinterpret_cast<const float4*>(rg + RG_FK) + 8 * hh;
-                float x[32];
-                tmem_ld32_sync(ctl + TM_D1K + 32 * hh, x);
-                uint32_t pk[16];
+            if (!wait_mma()) { done = false; break; }  // S0 K^T
 #pragma unroll
-                for (int e4 = 0; e4 < 8; ++e4) {
+            for (int q = 0; q < 2; ++q) {  // 16 tokens at a time
+                const float4* fk4 = reinterpret_cast<const float4*>(rg + RG_FK) + 8 * hh + 4 * q;
+                float x[16];
+                tmem_ld16_sync(ctl + TM_D1K + 32 * hh + 16 * q, x);
+                uint32_t pk[8];
+#pragma unroll
+                for (int e4 = 0; e4 < 4; ++e4) {
                     const float4 f = fk4[e4];
                     pk[2 * e4] = pack_bf16x2(-f.x * x[4 * e4], -f.y * x[4 * e4 + 1]);
                     pk[2 * e4 + 1] = pack_bf16x2(-f.z * x[4 * e4 + 2], -f.w * x[4 * e4 + 3]);
                 }
-                tmem_st16(ctl + TM_D1K + 32 * hh, pk);  // over the columns just read
+                // over columns this thread has read (the second half's loads precede
+                // nothing of the first half's stores in the same 16 columns)
+                tmem_st8(ctl + TM_D1K + 32 * hh + 8 * q, pk);
             }
-            signal_rdy();  // (its wait also covers the rescaled state)
+            signal_rdy();
 
             // ---- Vn^T -> bf16 pairs (for P Vn) and decay-scaled pairs (state update) --
-            if (!wait_mma()) break;  // Vn^T
-            {
-                const float4* egl4 = reinterpret_cast<const float4*>(rg + RG_EGL) + 8 * hh;
-                float x[32];
-                tmem_ld32_sync(ctl + TM_D3 + 32 * hh, x);
-                uint32_t pk[16], ps[16];
+            if (!wait_mma()) { done = false; break; }  // Vn^T
 #pragma unroll
-                for (int e4 = 0; e4 < 8; ++e4) {
+            for (int q = 0; q < 2; ++q) {
+                const float4* egl4 = reinterpret_cast<const float4*>(rg + RG_EGL) + 8 * hh + 4 * q;
+                float x[16];
+                tmem_ld16_sync(ctl + TM_D3 + 32 * hh + 16 * q, x);
+                uint32_t pk[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) pk[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
+                tmem_st8(ctl + TM_D3 + 32 * hh + 8 * q, pk);  // over Vn^T columns read
+#pragma unroll
+                for (int e4 = 0; e4 < 4; ++e4) {
                     const float4 w = egl4[e4];
-                    pk[2 * e4] = pack_bf16x2(x[4 * e4], x[4 * e4 + 1]);
-                    pk[2 * e4 + 1] = pack_bf16x2(x[4 * e4 + 2], x[4 * e4 + 3]);
-                    ps[2 * e4] = pack_bf16x2(x[4 * e4] * w.x, x[4 * e4 + 1] * w.y);
-                    ps[2 * e4 + 1] = pack_bf16x2(x[4 * e4 + 2] * w.z, x[4 * e4 + 3] * w.w);
+                    pk[2 * e4] = pack_bf16x2(x[4 * e4] * w.x, x[4 * e4 + 1] * w.y);
+                    pk[2 * e4 + 1] = pack_bf16x2(x[4 * e4 + 2] * w.z, x[4 * e4 + 3] * w.w);
                 }
-                tmem_st16(ctl + TM_D3 + 32 * hh, pk);   // over the Vn^T columns just read
-                tmem_st16(ctl + TM_D1K + 16 * hh, ps);  // Z^T there has been consumed
+                tmem_st8(ctl + TM_D1K + 16 * hh + 8 * q, pk);  // Z^T there is consumed
             }
             signal_rdy();
         }
-        bool fin = !*s_err;
-        if (fin && nchunks > 0) fin = wait_mma();  // the last state update
-        if (fin && Sfg) {
-            float* dst = Sfg + sbase;
-#pragma unroll 1
-            for (int cb = 0; cb < 2; ++cb) {
-                float x[32];
-                tmem_ld32_sync(ctl + TM_S + 64 * hh + 32 * cb, x);
-                float4* d4 = reinterpret_cast<float4*>(dst + 32 * cb);
+        if (done && nchunks > 0) {  // the last chunk's state update
+            done = wait_mma();
+            if (done) apply_update(gamma);
+        }
+        if (done && Sfg) {
+            float4* d4 = reinterpret_cast<float4*>(Sfg + sbase);
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    d4[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
-            }
+            for (int e = 0; e < 16; ++e)
+                d4[e] = make_float4(S[4 * e], S[4 * e + 1], S[4 * e + 2], S[4 * e + 3]);
         }
     }
 
