@@ -129,6 +129,51 @@ __global__ void __launch_bounds__(256) chunk_offsets_kernel(const int32_t* __res
     }
 }
 
+// ---- warp-level tf32 MMA (m16n8k8, fp32 accumulate) for the small products of
+// the triangular solve. Fragment layouts (lane = 4 g + t): A rows g and g + 8,
+// columns t and t + 4; B rows t and t + 4, column g; C rows g and g + 8, columns
+// 2 t and 2 t + 1.
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4],
+                                                const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// d (16 x 8 tile at rows r0, columns c0 of the product) += M1[r0.., k0..k0+kn) M2[k0.., c0..)
+// with M1, M2 row-major fp32 in shared memory (row strides s1, s2), kn a multiple of 8.
+__device__ __forceinline__ void tile_mma_tf32(float (&d)[4], const float* M1, int s1,
+                                              const float* M2, int s2, int r0, int c0, int k0,
+                                              int kn, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    for (int k = k0; k < k0 + kn; k += 8) {
+        const uint32_t a[4] = {to_tf32(M1[(r0 + g) * s1 + k + t]),
+                               to_tf32(M1[(r0 + g + 8) * s1 + k + t]),
+                               to_tf32(M1[(r0 + g) * s1 + k + t + 4]),
+                               to_tf32(M1[(r0 + g + 8) * s1 + k + t + 4])};
+        const uint32_t b[2] = {to_tf32(M2[(k + t) * s2 + c0 + g]),
+                               to_tf32(M2[(k + t + 4) * s2 + c0 + g])};
+        mma_tf32_16x8x8(d, a, b);
+    }
+}
+
+// Store a 16 x 8 C fragment (times `scale`) at rows r0, columns c0 of a row-major matrix.
+__device__ __forceinline__ void tile_store(float* M, int s, int r0, int c0, const float (&d)[4],
+                                           float scale, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    *reinterpret_cast<float2*>(M + (r0 + g) * s + c0 + 2 * t) = make_float2(scale * d[0], scale * d[1]);
+    *reinterpret_cast<float2*>(M + (r0 + g + 8) * s + c0 + 2 * t) =
+        make_float2(scale * d[2], scale * d[3]);
+}
+
 // ==================================== prep ========================================
 constexpr int kPrepThreads = 256;
 constexpr int kTsStride = 68;
@@ -137,13 +182,13 @@ constexpr int kAsStride = 68;
 constexpr uint32_t PS_KQ = 0;        // [2 col blocks][128 rows][128 B], raw K then Q, sw128
 constexpr uint32_t PS_TS = 32768;    // [64][68] fp32 T
 constexpr uint32_t PS_AS = 50176;    // [64][68] fp32 A (strictly-lower part used)
-constexpr uint32_t PS_XS = 67584;    // [1024] fp32 merge scratch
-constexpr uint32_t PS_AB = 71680;    // [2][kMaxGroup][64] fp32 a, b
-constexpr uint32_t PS_HS = 79872;    // per-head scratch: G, beta, Gp [64 each], U [4][64]
-constexpr uint32_t PS_RK = 82304;    // [64] rk, [64] rq (rq includes the scale)
-constexpr uint32_t PS_BAR = 82816;   // mbarrier (MMA)
-constexpr uint32_t PS_TMEM = 82824;
-constexpr size_t kPrepSmem = 82832 + 1024;
+constexpr uint32_t PS_XS = 67584;    // [1152] fp32 merge scratch
+constexpr uint32_t PS_AB = 72192;    // [2][kMaxGroup][64] fp32 a, b
+constexpr uint32_t PS_HS = 80384;    // per-head scratch: G, beta, Gp [64 each], U [4][64]
+constexpr uint32_t PS_RK = 82816;    // [64] rk, [64] rq (rq includes the scale)
+constexpr uint32_t PS_BAR = 83328;   // mbarrier (MMA)
+constexpr uint32_t PS_TMEM = 83336;
+constexpr size_t kPrepSmem = 83344 + 1024;
 
 // Half a row (32 columns starting at 32 H) of A (row i < 64) or of P (row t =
 // i - 64) from the matching half row x of [K; Q] K^T. Columns left of the row's
@@ -432,71 +477,41 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
                 Ts[(a0 + 8 + rr) * kTsStride + a0 + cc] = -t1;
             }
             __syncthreads();
-            // ---- doubling 16 -> 32: T_10 and T_32 ------------------------------------
+            // ---- doubling 16 -> 32 (two 32-blocks) and 32 -> 64, tf32 tensor cores ----
+            // T_10 = -T_11 (A_10 T_00): X = A_10 T_00 goes through Xs (row stride 40)
+            constexpr int kXs = 36;
             {
-                const int which = tid >> 7;
-                const int q7 = tid & 127;
-                const int rr = q7 >> 3, c0 = (q7 & 7) * 2;
-                const int cb = which ? 32 : 0;
-                const int rb = which ? 48 : 16;
-                const float* Arow = As + (rb + rr) * kAsStride + cb;
-                float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    const float am = Arow[m];
-                    const float2 d = *reinterpret_cast<const float2*>(Ts + (cb + m) * kTsStride + cb + c0);
-                    acc.x = fmaf(am, d.x, acc.x);
-                    acc.y = fmaf(am, d.y, acc.y);
+                // 16 -> 32: warp w < 4: block b = w >> 1 (rows 32 b + 16 ..), column tile w & 1
+                if (warp < 4) {
+                    const int b = warp >> 1, nt = warp & 1;
+                    const int R = 32 * b;
+                    float d[4] = {0.f, 0.f, 0.f, 0.f};
+                    tile_mma_tf32(d, As, kAsStride, Ts, kTsStride, R + 16, R + 8 * nt, R, 16, lane);
+                    tile_store(Xs + b * 16 * kXs, kXs, 0, 8 * nt, d, 1.f, lane);
                 }
-                *reinterpret_cast<float2*>(Xs + which * 256 + rr * 16 + c0) = acc;
                 __syncthreads();
-                const float* Drow = Ts + (rb + rr) * kTsStride + rb;
-                float2 t2 = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    const float dm = Drow[m];
-                    const float2 xv = *reinterpret_cast<const float2*>(Xs + which * 256 + m * 16 + c0);
-                    t2.x = fmaf(dm, xv.x, t2.x);
-                    t2.y = fmaf(dm, xv.y, t2.y);
+                if (warp < 4) {
+                    const int b = warp >> 1, nt = warp & 1;
+                    const int R = 32 * b;
+                    float d[4] = {0.f, 0.f, 0.f, 0.f};
+                    // rows R+16.. of T (its 16-block, columns R+16..R+31) times X (16 x 16)
+                    tile_mma_tf32(d, Ts + R + 16, kTsStride, Xs + b * 16 * kXs, kXs, R + 16,
+                                  8 * nt, 0, 16, lane);
+                    tile_store(Ts, kTsStride, R + 16, R + 8 * nt, d, -1.f, lane);
                 }
-                *reinterpret_cast<float2*>(Ts + (rb + rr) * kTsStride + cb + c0) =
-                    make_float2(-t2.x, -t2.y);
             }
             __syncthreads();
-            // ---- doubling 32 -> 64: T[32:64, 0:32] -----------------------------------
             {
-                const int rr = tid >> 3, c0 = (tid & 7) * 4;
-                const float* Arow = As + (32 + rr) * kAsStride;
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f), acc2 = acc;
-#pragma unroll
-                for (int m = 0; m < 32; m += 2) {
-                    const float4 am = *reinterpret_cast<const float4*>(Arow + (m & ~3));
-                    const float a_0 = (m & 2) ? am.z : am.x, a_1 = (m & 2) ? am.w : am.y;
-                    const float4 d = *reinterpret_cast<const float4*>(Ts + m * kTsStride + c0);
-                    const float4 e = *reinterpret_cast<const float4*>(Ts + (m + 1) * kTsStride + c0);
-                    acc.x = fmaf(a_0, d.x, acc.x); acc.y = fmaf(a_0, d.y, acc.y);
-                    acc.z = fmaf(a_0, d.z, acc.z); acc.w = fmaf(a_0, d.w, acc.w);
-                    acc2.x = fmaf(a_1, e.x, acc2.x); acc2.y = fmaf(a_1, e.y, acc2.y);
-                    acc2.z = fmaf(a_1, e.z, acc2.z); acc2.w = fmaf(a_1, e.w, acc2.w);
-                }
-                *reinterpret_cast<float4*>(Xs + rr * 32 + c0) =
-                    make_float4(acc.x + acc2.x, acc.y + acc2.y, acc.z + acc2.z, acc.w + acc2.w);
+                // 32 -> 64: X (32 x 32) = A[32:64, 0:32] T[0:32, 0:32]; warp w: tile (w >> 2, w & 3)
+                const int mt = warp >> 2, nt = warp & 3;
+                float d[4] = {0.f, 0.f, 0.f, 0.f};
+                tile_mma_tf32(d, As, kAsStride, Ts, kTsStride, 32 + 16 * mt, 8 * nt, 0, 32, lane);
+                tile_store(Xs, kXs, 16 * mt, 8 * nt, d, 1.f, lane);
                 __syncthreads();
-                const float* Drow = Ts + (32 + rr) * kTsStride + 32;
-                float4 t4 = make_float4(0.f, 0.f, 0.f, 0.f), t5 = t4;
-#pragma unroll
-                for (int m = 0; m < 32; m += 2) {
-                    const float4 dm = *reinterpret_cast<const float4*>(Drow + (m & ~3));
-                    const float d_0 = (m & 2) ? dm.z : dm.x, d_1 = (m & 2) ? dm.w : dm.y;
-                    const float4 xv = *reinterpret_cast<const float4*>(Xs + m * 32 + c0);
-                    const float4 xw = *reinterpret_cast<const float4*>(Xs + (m + 1) * 32 + c0);
-                    t4.x = fmaf(d_0, xv.x, t4.x); t4.y = fmaf(d_0, xv.y, t4.y);
-                    t4.z = fmaf(d_0, xv.z, t4.z); t4.w = fmaf(d_0, xv.w, t4.w);
-                    t5.x = fmaf(d_1, xw.x, t5.x); t5.y = fmaf(d_1, xw.y, t5.y);
-                    t5.z = fmaf(d_1, xw.z, t5.z); t5.w = fmaf(d_1, xw.w, t5.w);
-                }
-                *reinterpret_cast<float4*>(Ts + (32 + rr) * kTsStride + c0) =
-                    make_float4(-(t4.x + t5.x), -(t4.y + t5.y), -(t4.z + t5.z), -(t4.w + t5.w));
+                float e[4] = {0.f, 0.f, 0.f, 0.f};
+                // T[32:64, 0:32] = -T[32:64, 32:64] X
+                tile_mma_tf32(e, Ts + 32, kTsStride, Xs, kXs, 32 + 16 * mt, 8 * nt, 0, 32, lane);
+                tile_store(Ts, kTsStride, 32 + 16 * mt, 8 * nt, e, -1.f, lane);
             }
             __syncthreads();
 
