@@ -184,11 +184,14 @@ constexpr uint32_t PS_TS = 32768;    // [64][68] fp32 T
 constexpr uint32_t PS_AS = 50176;    // [64][68] fp32 A (strictly-lower part used)
 constexpr uint32_t PS_XS = 67584;    // [1152] fp32 merge scratch
 constexpr uint32_t PS_AB = 72192;    // [2][kMaxGroup][64] fp32 a, b
-constexpr uint32_t PS_HS = 80384;    // per-head scratch: G, beta, Gp [64 each], U [4][64]
+constexpr uint32_t PS_HS = 80384;    // per-head scratch: U [4][64]
 constexpr uint32_t PS_RK = 82816;    // [64] rk, [64] rq (rq includes the scale)
-constexpr uint32_t PS_BAR = 83328;   // mbarrier (MMA)
-constexpr uint32_t PS_TMEM = 83336;
-constexpr size_t kPrepSmem = 83344 + 1024;
+constexpr uint32_t PS_GA = 83328;    // [kMaxGroup][64] G of every V head of the unit
+constexpr uint32_t PS_BA = 87424;    // [kMaxGroup][64] beta of every V head of the unit
+constexpr uint32_t PS_PAR = 91520;   // [2][kMaxGroup] A_log, dt_bias of those heads
+constexpr uint32_t PS_BAR = 91648;   // mbarrier (MMA)
+constexpr uint32_t PS_TMEM = 91656;
+constexpr size_t kPrepSmem = 91664 + 1024;
 
 // Half a row (32 columns starting at 32 H) of A (row i < 64) or of P (row t =
 // i - 64) from the matching half row x of [K; Q] K^T. Columns left of the row's
@@ -252,11 +255,11 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
     float* As = reinterpret_cast<float*>(sm + PS_AS);
     float* Xs = reinterpret_cast<float*>(sm + PS_XS);
     float* AB = reinterpret_cast<float*>(sm + PS_AB);
-    float* sG = reinterpret_cast<float*>(sm + PS_HS);
-    float* sBeta = sG + 64;
-    float* Gp = sG + 128;
-    float* sU = sG + 192;
+    float* sU = reinterpret_cast<float*>(sm + PS_HS);  // [4][64] per-head exp table
     float* rk = reinterpret_cast<float*>(sm + PS_RK);
+    float* sGall = reinterpret_cast<float*>(sm + PS_GA);
+    float* sBall = reinterpret_cast<float*>(sm + PS_BA);
+    float* sPar = reinterpret_cast<float*>(sm + PS_PAR);
     float* rq = rk + 64;
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + PS_BAR);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + PS_TMEM);
@@ -320,6 +323,11 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
             const float* src = (which ? b : a) + (size_t)tok * H_v + j * r + hr;
             cp_async_4(AB + (which * kMaxGroup + hr) * kC + t, src, live ? 4u : 0u);
         }
+        if (tid < 2 * r) {
+            const int hr = tid >> 1;
+            cp_async_4(sPar + (tid & 1) * kMaxGroup + hr, ((tid & 1) ? dt_bias : A_log) + j * r + hr,
+                       4u);
+        }
         cp_async_commit();
         cp_async_wait<0>();
         fence_proxy_async_smem();
@@ -349,6 +357,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
                 else rq[row - 64] = inv * scale;
             }
         }
+        __syncthreads();  // rk, rq
         if (tid == 0) {
             const uint32_t kq = smem_u32(KQ);
             constexpr uint32_t id_kq = idesc_bf16_f32(128, 64, 0, 0);
@@ -359,6 +368,36 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
                             smem_desc_sw128(kq + off, 16, 1024), id_kq, ks > 0);
             }
             mma_commit(bar);
+        }
+        // ---- gates of every V head of the group: one warp per head, two tokens a lane:
+        // g, beta, the in-chunk inclusive cumsum G, and the record's per-token factors
+        for (int hr = warp; hr < r; hr += kPrepThreads / 32) {
+            const int h = j * r + hr;
+            const float A_l = sPar[hr], dtb = sPar[kMaxGroup + hr];
+            const int ta = 2 * lane, tb = 2 * lane + 1;
+            const float ga = ta < L ? gate_g(AB[hr * kC + ta], A_l, dtb) : 0.f;
+            const float gb = tb < L ? gate_g(AB[hr * kC + tb], A_l, dtb) : 0.f;
+            const float ba = ta < L ? gate_beta(AB[(kMaxGroup + hr) * kC + ta]) : 0.f;
+            const float bb = tb < L ? gate_beta(AB[(kMaxGroup + hr) * kC + tb]) : 0.f;
+            float sc = ga + gb;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, sc, off);
+                if (lane >= off) sc += y;
+            }
+            const float Gb = sc, Ga = sc - gb;  // G_{L-1} = G of the last lane (g = 0 past L)
+            const float G_last = __shfl_sync(0xffffffffu, sc, 31);
+            *reinterpret_cast<float2*>(sGall + hr * kC + ta) = make_float2(Ga, Gb);
+            *reinterpret_cast<float2*>(sBall + hr * kC + ta) = make_float2(ba, bb);
+            float* rg = reinterpret_cast<float*>(rec + ((size_t)cg * H_v + h) * kRecBytes + REC_G);
+            const float ea = __expf(Ga), eb = __expf(Gb);
+            const float2 rk2 = *reinterpret_cast<const float2*>(rk + ta);
+            const float2 rq2 = *reinterpret_cast<const float2*>(rq + ta);
+            *reinterpret_cast<float2*>(rg + RG_FK + ta) = make_float2(ea * rk2.x, eb * rk2.y);
+            *reinterpret_cast<float2*>(rg + RG_EGQ + ta) = make_float2(ea * rq2.x, eb * rq2.y);
+            *reinterpret_cast<float2*>(rg + RG_EGL + ta) =
+                make_float2(__expf(G_last - Ga) * rk2.x, __expf(G_last - Gb) * rk2.y);
+            if (lane == 0) rg[RG_GAMMA] = __expf(G_last);
         }
         const bool ok = mbar_wait_bounded(bar, mphase, kWaitCycles);
         mphase ^= 1u;
@@ -372,43 +411,21 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
         for (int hr = 0; hr < r; ++hr) {
             const int h = j * r + hr;
             uint8_t* R = rec + ((size_t)cg * H_v + h) * kRecBytes;
-            float* rg = reinterpret_cast<float*>(R + REC_G);
-            // ---- gates: g, beta, in-chunk inclusive cumsum ----------------------------
-            if (tid < kC) {
-                const bool live = tid < L;
-                float g = live ? gate_g(AB[hr * kC + tid], A_log[h], dt_bias[h]) : 0.f;
-                sBeta[tid] = live ? gate_beta(AB[(kMaxGroup + hr) * kC + tid]) : 0.f;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, g, off);
-                    if (lane >= off) g += y;
-                }
-                Gp[tid] = g;
-            }
-            __syncthreads();
-            if (tid < kC) sG[tid] = Gp[tid] + (tid >= 32 ? Gp[31] : 0.f);
-            __syncthreads();
-            const float G_last = sG[kC - 1];  // = G_{L-1}: tokens past L add g = 0
-            if (tid < kC) {
-                const float eg = __expf(sG[tid]);
-                rg[RG_FK + tid] = eg * rk[tid];
-                rg[RG_EGQ + tid] = eg * rq[tid];
-                rg[RG_EGL + tid] = __expf(G_last - sG[tid]) * rk[tid];
-            }
-            {
+            const float* hG = sGall + hr * kC;     // this head's G
+            const float* hBeta = sBall + hr * kC;  // and beta
+            {  // U[a][j] = exp(G_{16 a} - G_j) for j < 16 a (both factors of a long gap <= 1)
                 const int ab4 = tid >> 6, jj = tid & 63;
-                sU[tid] = (jj < 16 * ab4) ? __expf(sG[16 * ab4] - sG[jj]) : 0.f;
+                sU[tid] = (jj < 16 * ab4) ? __expf(hG[16 * ab4] - hG[jj]) : 0.f;
             }
-            if (tid == 0) rg[RG_GAMMA] = __expf(G_last);
             __syncthreads();
 
             // ---- A rows 0-63 -> As (fp32); P rows 64-127 -> record (bf16 image) --------
             {
                 float val[32];
                 const int i = trow & 63;
-                const float rowf = trow < 64 ? sBeta[i] * rk[i] : rq[i];
-                if (hh == 0) ap_half_row<0>(x, trow, sG, sU, rk, rowf, val);
-                else         ap_half_row<1>(x, trow, sG, sU, rk, rowf, val);
+                const float rowf = trow < 64 ? hBeta[i] * rk[i] : rq[i];
+                if (hh == 0) ap_half_row<0>(x, trow, hG, sU, rk, rowf, val);
+                else         ap_half_row<1>(x, trow, hG, sU, rk, rowf, val);
                 if (trow < 64) {
                     float4* Arow = reinterpret_cast<float4*>(As + i * kAsStride + 32 * hh);
 #pragma unroll
@@ -522,8 +539,8 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
                 const int row = idx >> 3, ch = idx & 7;
                 const float4 f0 = *reinterpret_cast<const float4*>(Ts + row * kTsStride + ch * 8);
                 const float4 f1 = *reinterpret_cast<const float4*>(Ts + row * kTsStride + ch * 8 + 4);
-                const float4 b0 = *reinterpret_cast<const float4*>(sBeta + ch * 8);
-                const float4 b1 = *reinterpret_cast<const float4*>(sBeta + ch * 8 + 4);
+                const float4 b0 = *reinterpret_cast<const float4*>(hBeta + ch * 8);
+                const float4 b1 = *reinterpret_cast<const float4*>(hBeta + ch * 8 + 4);
                 uint4 w;  // column s of T times beta_s
                 w.x = pack_bf16x2(f0.x * b0.x, f0.y * b0.y);
                 w.y = pack_bf16x2(f0.z * b0.z, f0.w * b0.w);
