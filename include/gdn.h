@@ -71,11 +71,12 @@ int gdn_version(void);
 
 /*
  * Bytes of device workspace gdn_prefill needs for these sizes. For d = 128 it
- * covers the tensor-core path: the chunk offsets of the sequences plus one
- * 17,664-byte record (the chunk's T and P matrices and per-token factors) per
- * (64-token chunk, V head), i.e. about 276 bytes per token and V head (with one
- * extra chunk per sequence); for d = 64 (CUDA-core path) it is the per-token G
- * and beta, fp32 [T, H_v] each. Returns 0 for invalid sizes.
+ * covers the tensor-core path: the chunk offsets of the sequences, then per
+ * (64-token chunk, V head) a 4-byte ready flag and a 17,664-byte record (the
+ * chunk's T diag(beta) and P matrices and per-token factors), i.e. about 276
+ * bytes per token and V head (with one extra chunk per sequence), each part
+ * rounded up to 256 bytes; for d = 64 (CUDA-core path) it is the per-token G and
+ * beta, fp32 [T, H_v] each. Returns 0 for invalid sizes (and for num_seqs = 0).
  */
 size_t gdn_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t H_qk,
                                   int32_t H_v, int32_t d_k, int32_t d_v);
@@ -132,11 +133,21 @@ int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
  *                         kernel otherwise (fp32 I/O, d = 64);
  *   GDN_IMPL_CUDA_CORE    the fp32 CUDA-core kernel for every call;
  *   GDN_IMPL_TENSOR_CORE  tensor cores only; gdn_prefill then returns
- *                         GDN_ERR_UNSUPPORTED for shapes/types they do not cover.
+ *                         GDN_ERR_UNSUPPORTED for shapes/types they do not cover;
+ *   GDN_IMPL_TENSOR_CORE_SPLIT
+ *                         tensor cores with the state-free preparation and the
+ *                         chunk chain as separate launches (the default runs them
+ *                         in one cooperative launch, overlapped, where the device
+ *                         supports it).
  * Returns the previous setting, or -GDN_ERR_INVALID_ARG for an unknown value.
  * Not synchronised with calls in flight on other host threads.
  */
-enum { GDN_IMPL_AUTO = 0, GDN_IMPL_CUDA_CORE = 1, GDN_IMPL_TENSOR_CORE = 2 };
+enum {
+    GDN_IMPL_AUTO = 0,
+    GDN_IMPL_CUDA_CORE = 1,
+    GDN_IMPL_TENSOR_CORE = 2,
+    GDN_IMPL_TENSOR_CORE_SPLIT = 3
+};
 int gdn_set_prefill_impl(int32_t impl);
 
 /*

@@ -172,7 +172,8 @@ int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
     const int impl = g_prefill_impl.load(std::memory_order_relaxed);
     const bool tc_ok =
         io_dtype == GDN_BF16 && d_k == 128 && prefill_tc_supported(H_qk, H_v);
-    if (impl == GDN_IMPL_TENSOR_CORE && !tc_ok) return GDN_ERR_UNSUPPORTED;
+    if ((impl == GDN_IMPL_TENSOR_CORE || impl == GDN_IMPL_TENSOR_CORE_SPLIT) && !tc_ok)
+        return GDN_ERR_UNSUPPORTED;
     int* st = device_status_ptr();
     if (!st) return GDN_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
@@ -180,7 +181,8 @@ int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
     if (tc_ok && impl != GDN_IMPL_CUDA_CORE) {
         return to_status(launch_prefill_tc(q, k, v, a, b, A_log, dt_bias, initial_state,
                                            cu_seqlens, num_seqs, total_tokens, H_qk, H_v, scale,
-                                           o, final_state, workspace, st, s));
+                                           o, final_state, workspace,
+                                           impl != GDN_IMPL_TENSOR_CORE_SPLIT, st, s));
     }
     float* G = static_cast<float*>(workspace);
     float* beta = reinterpret_cast<float*>(static_cast<char*>(workspace) +
@@ -222,7 +224,8 @@ int gdn_decode_step(const void* q, const void* k, const void* v, int32_t io_dtyp
 }
 
 int gdn_set_prefill_impl(int32_t impl) {
-    if (impl != GDN_IMPL_AUTO && impl != GDN_IMPL_CUDA_CORE && impl != GDN_IMPL_TENSOR_CORE)
+    if (impl != GDN_IMPL_AUTO && impl != GDN_IMPL_CUDA_CORE && impl != GDN_IMPL_TENSOR_CORE &&
+        impl != GDN_IMPL_TENSOR_CORE_SPLIT)
         return -GDN_ERR_INVALID_ARG;
     return g_prefill_impl.exchange(impl);
 }

@@ -103,6 +103,6 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
                               const float* b, const float* A_log, const float* dt_bias,
                               const float* S0, const int32_t* cu_seqlens, int32_t N, int64_t T,
                               int32_t H_qk, int32_t H_v, float scale, void* o, float* S_final,
-                              void* workspace, int* status, cudaStream_t s);
+                              void* workspace, bool fused, int* status, cudaStream_t s);
 
 }  // namespace gdn

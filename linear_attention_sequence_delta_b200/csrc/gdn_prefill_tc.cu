@@ -241,15 +241,22 @@ __device__ __forceinline__ void ap_half_row(const float (&x)[32], int row, const
     }
 }
 
-__global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
+// Record (chunk cg, V head h) is complete: publish it to the chain (release).
+__device__ __forceinline__ void publish_record(int* flags, size_t idx) {
+    __threadfence();
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flags + idx), "r"(1) : "memory");
+}
+
+// One prep worker of kPrepThreads threads (tid 0 .. 255, synchronised by the named
+// barrier bar_id) walks the (chunk, QK head) units worker, worker + nworkers, ...
+// and writes their records; with `flags`, each finished record is published.
+__device__ __forceinline__ void prep_worker(
     const bf16* __restrict__ q, const bf16* __restrict__ k, const float* __restrict__ a,
     const float* __restrict__ b, const float* __restrict__ A_log,
     const float* __restrict__ dt_bias, const int32_t* __restrict__ cu_seqlens,
     const int32_t* __restrict__ choff, int32_t N, int H_qk, int H_v, float scale,
-    uint8_t* __restrict__ rec, int* status) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* __restrict__ rec, int* status, int* flags, uint8_t* sm, const int tid,
+    const int bar_id, const int worker, const int nworkers, const bool relinquish) {
     uint8_t* KQ = sm + PS_KQ;
     float* Ts = reinterpret_cast<float*>(sm + PS_TS);
     float* As = reinterpret_cast<float*>(sm + PS_AS);
@@ -264,14 +271,13 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + PS_BAR);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + PS_TMEM);
 
-    const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int r = H_v / H_qk;
     const int total_units = choff[N] * H_qk;
 
     if (warp == 0) {
         tmem_alloc(s_tmem, 64);
-        tmem_relinquish();
+        if (relinquish) tmem_relinquish();
     }
     if (tid == 0) {
         mbar_init(bar, 1);
@@ -280,7 +286,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
     // entries of T above its diagonal blocks are never written: zero them once
     for (int idx = tid; idx < 64 * kTsStride; idx += kPrepThreads) Ts[idx] = 0.f;
     tc_fence_before();
-    __syncthreads();
+    named_bar_sync(bar_id, kPrepThreads);
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
     const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
@@ -290,7 +296,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
     bool failed = false;
 
 #pragma unroll 1
-    for (int unit = blockIdx.x; unit < total_units; unit += gridDim.x) {
+    for (int unit = worker; unit < total_units; unit += nworkers) {
         const int cg = unit / H_qk;
         const int j = unit - cg * H_qk;
         int lo = 0, hi = N;  // sequence n with choff[n] <= cg < choff[n+1]
@@ -331,7 +337,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
         cp_async_commit();
         cp_async_wait<0>();
         fence_proxy_async_smem();
-        __syncthreads();
+        named_bar_sync(bar_id, kPrepThreads);
 
         // ---- inverse row norms (two threads per row), then Dkq = [K; Q] K^T ---------
         {
@@ -357,7 +363,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
                 else rq[row - 64] = inv * scale;
             }
         }
-        __syncthreads();  // rk, rq
+        named_bar_sync(bar_id, kPrepThreads);  // rk, rq
         if (tid == 0) {
             const uint32_t kq = smem_u32(KQ);
             constexpr uint32_t id_kq = idesc_bf16_f32(128, 64, 0, 0);
@@ -402,7 +408,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
         const bool ok = mbar_wait_bounded(bar, mphase, kWaitCycles);
         mphase ^= 1u;
         if (!ok) failed = true;
-        if (__syncthreads_or(failed)) { failed = true; break; }
+        if (named_bar_any(bar_id, kPrepThreads, failed)) { failed = true; break; }
         tc_fence_after();
         float x[32];  // this thread's half row of [K; Q] K^T, shared by the r V heads
         tmem_ld32_sync(tl + 32 * hh, x);
@@ -417,7 +423,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
                 const int ab4 = tid >> 6, jj = tid & 63;
                 sU[tid] = (jj < 16 * ab4) ? __expf(hG[16 * ab4] - hG[jj]) : 0.f;
             }
-            __syncthreads();
+            named_bar_sync(bar_id, kPrepThreads);
 
             // ---- A rows 0-63 -> As (fp32); P rows 64-127 -> record (bf16 image) --------
             {
@@ -445,7 +451,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
                     }
                 }
             }
-            __syncthreads();
+            named_bar_sync(bar_id, kPrepThreads);
 
             // ---- 8x8 diagonal blocks of T: forward substitution in registers -------
             // rows 0-31 from warp 0 (columns 0-31), rows 32-63 from warp 5 (32-63)
@@ -474,7 +480,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
 #pragma unroll
                 for (int r2 = 0; r2 < 8; ++r2) Trow[r2] = r2 < rr ? -Rr[r2] : (r2 == rr ? 1.f : 0.f);
             }
-            __syncthreads();
+            named_bar_sync(bar_id, kPrepThreads);
 
             // ---- doubling 8 -> 16: T_{hi,lo} = -D_hi (A_{hi,lo} D_lo) in each 16-block
             {
@@ -485,7 +491,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
 #pragma unroll
                 for (int m = 0; m < 8; ++m) acc = fmaf(Arow[m], Ts[(a0 + m) * kTsStride + a0 + cc], acc);
                 Xs[tid] = acc;
-                __syncthreads();
+                named_bar_sync(bar_id, kPrepThreads);
                 const float* Drow = Ts + (a0 + 8 + rr) * kTsStride + a0 + 8;
                 const float* Xb = Xs + (tid & ~63);
                 float t1 = 0.f;
@@ -493,7 +499,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
                 for (int m = 0; m < 8; ++m) t1 = fmaf(Drow[m], Xb[m * 8 + cc], t1);
                 Ts[(a0 + 8 + rr) * kTsStride + a0 + cc] = -t1;
             }
-            __syncthreads();
+            named_bar_sync(bar_id, kPrepThreads);
             // ---- doubling 16 -> 32 (two 32-blocks) and 32 -> 64, tf32 tensor cores ----
             // T_10 = -T_11 (A_10 T_00): X = A_10 T_00 goes through Xs (row stride 40)
             constexpr int kXs = 36;
@@ -506,7 +512,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
                     tile_mma_tf32(d, As, kAsStride, Ts, kTsStride, R + 16, R + 8 * nt, R, 16, lane);
                     tile_store(Xs + b * 16 * kXs, kXs, 0, 8 * nt, d, 1.f, lane);
                 }
-                __syncthreads();
+                named_bar_sync(bar_id, kPrepThreads);
                 if (warp < 4) {
                     const int b = warp >> 1, nt = warp & 1;
                     const int R = 32 * b;
@@ -517,20 +523,20 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
                     tile_store(Ts, kTsStride, R + 16, R + 8 * nt, d, -1.f, lane);
                 }
             }
-            __syncthreads();
+            named_bar_sync(bar_id, kPrepThreads);
             {
                 // 32 -> 64: X (32 x 32) = A[32:64, 0:32] T[0:32, 0:32]; warp w: tile (w >> 2, w & 3)
                 const int mt = warp >> 2, nt = warp & 3;
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
                 tile_mma_tf32(d, As, kAsStride, Ts, kTsStride, 32 + 16 * mt, 8 * nt, 0, 32, lane);
                 tile_store(Xs, kXs, 16 * mt, 8 * nt, d, 1.f, lane);
-                __syncthreads();
+                named_bar_sync(bar_id, kPrepThreads);
                 float e[4] = {0.f, 0.f, 0.f, 0.f};
                 // T[32:64, 0:32] = -T[32:64, 32:64] X
                 tile_mma_tf32(e, Ts + 32, kTsStride, Xs, kXs, 32 + 16 * mt, 8 * nt, 0, 32, lane);
                 tile_store(Ts, kTsStride, 32 + 16 * mt, 8 * nt, e, -1.f, lane);
             }
-            __syncthreads();
+            named_bar_sync(bar_id, kPrepThreads);
 
             // ---- T -> record (bf16 sw128 image) ----------------------------------------
 #pragma unroll
@@ -548,15 +554,29 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
                 w.w = pack_bf16x2(f1.z * b1.z, f1.w * b1.w);
                 *reinterpret_cast<uint4*>(R + REC_T + sw128_off(row, ch)) = w;
             }
-            __syncthreads();  // Ts, As, Xs and the head scratch are reused
+            named_bar_sync(bar_id, kPrepThreads);  // Ts, As, Xs and the head scratch are reused
+            if (flags && tid == 0) publish_record(flags, (size_t)cg * H_v + h);
         }
         tc_fence_before();  // this unit's TMEM reads precede the next unit's MMA
     }
     tc_fence_before();
-    __syncthreads();
+    named_bar_sync(bar_id, kPrepThreads);
     tc_fence_after();
     if (failed && tid == 0) set_status(status, kStatusTimeout);
     if (warp == 0) tmem_dealloc(tmem, 64);
+}
+
+__global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
+    const bf16* __restrict__ q, const bf16* __restrict__ k, const float* __restrict__ a,
+    const float* __restrict__ b, const float* __restrict__ A_log,
+    const float* __restrict__ dt_bias, const int32_t* __restrict__ cu_seqlens,
+    const int32_t* __restrict__ choff, int32_t N, int H_qk, int H_v, float scale,
+    uint8_t* __restrict__ rec, int* status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    prep_worker(q, k, a, b, A_log, dt_bias, cu_seqlens, choff, N, H_qk, H_v, scale, rec, status,
+                nullptr, sm, threadIdx.x, 1, blockIdx.x, gridDim.x, true);
 }
 
 // ==================================== chain =======================================
@@ -616,28 +636,40 @@ __device__ __forceinline__ uint32_t tile64_off(int t, int i) {
 //               (S0 Q^T alternates between two accumulators) and, once a chunk's
 //               ring slot is no longer read, load the chunk three ahead into it
 //               (TMA tiles for K, Q, V and one bulk copy of the record).
-__global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
-    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-    const float* __restrict__ S0g, const int32_t* __restrict__ cu_seqlens,
+// Waits (bounded) until a record is published by a prep worker (acquire).
+__device__ __forceinline__ bool wait_record(const int* flag, long long max_cycles) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    if (v) return true;
+    const long long t0 = clock64();
+    do {
+        __nanosleep(64);
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+        if (v) return true;
+    } while (clock64() - t0 < max_cycles);
+    return false;
+}
+
+// The whole chunk chain of one (sequence n, V head h), run by the kChainThreads
+// threads of a block (tid 0 .. 415, synchronised by the named barrier sync_id) on
+// the tensor memory `tmem` (512 columns). With `flags`, a chunk's record is
+// copied only once a prep worker has published it.
+__device__ __forceinline__ void chain_unit(
+    const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+    const CUtensorMap& tm_o, const float* __restrict__ S0g, const int32_t* __restrict__ cu_seqlens,
     const int32_t* __restrict__ choff, int64_t T_total, int H_qk, int H_v,
-    const uint8_t* __restrict__ rec, bf16* __restrict__ o, float* __restrict__ Sfg, int* status) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint8_t* __restrict__ rec, bf16* __restrict__ o, float* __restrict__ Sfg, int* status,
+    const int* flags, uint8_t* sm, const int tid, const int n, const int h, const uint32_t tmem,
+    const int sync_id) {
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + CS_BAR);  // [3] slot landed
     uint64_t* mbar = full + kRing;         // chain MMA completions
     uint64_t* obar = mbar + 1;             // [2] chunk parity b: output accumulators complete
     uint64_t* ofree = mbar + 3;            // [2] chunk parity b: output accumulators read
     uint64_t* rdy = mbar + 5;              // a state step's TMEM operands written (8 arrivals)
     uint64_t* dbar = mbar + 6;             // drain of in-flight MMAs before the exit
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + CS_TMEM);
     volatile int* s_err = reinterpret_cast<volatile int*>(sm + CS_ERR);
 
-    const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const int h = blockIdx.x % H_v;
-    const int n = blockIdx.x / H_v;
     const int j = h / (H_v / H_qk);
     const int64_t s0 = cu_seqlens[n];
     const int64_t s1 = cu_seqlens[n + 1];
@@ -645,10 +677,6 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
     const int nchunks = (int)((s1 - s0 + kC - 1) / kC);
     const int cg0 = choff[n];
 
-    if (warp == 0) {
-        tmem_alloc(s_tmem, kTmemCols);
-        tmem_relinquish();
-    }
     if (tid == 0) {
         for (int i = 0; i < kRing; ++i) mbar_init(&full[i], 1);
         mbar_init(mbar, 1);
@@ -668,15 +696,21 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
         tma_prefetch_desc(&tm_o);
     }
     tc_fence_before();
-    __syncthreads();
+    named_bar_sync(sync_id, kChainThreads);
     tc_fence_after();
-    const uint32_t tmem = *s_tmem;
 
     // chunk c of this sequence -> its ring slot (issued by one lane)
-    auto issue_loads = [&](int c) {
+    auto issue_loads = [&](int c) -> bool {
         const int st = c % kRing;
         uint8_t* slot = sm + st * kSlotBytes;
         const int32_t t0 = (int32_t)(s0 + (int64_t)c * kC);
+        if (flags) {
+            if (!wait_record(flags + (size_t)(cg0 + c) * H_v + h, kWaitCycles)) {
+                *s_err = 1;
+                return false;
+            }
+            asm volatile("fence.proxy.async.global;" ::: "memory");  // the record, read by TMA
+        }
         mbar_arrive_expect_tx(&full[st], kSlotTx);
         tma_load_3d(slot + SLOT_KQ, &tm_k, 0, j, t0, &full[st]);
         tma_load_3d(slot + SLOT_KQ + 16384, &tm_k, 64, j, t0, &full[st]);
@@ -686,6 +720,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
         tma_load_3d(slot + SLOT_V + 8192, &tm_v, 64, h, t0, &full[st]);
         bulk_g2s(slot + SLOT_REC, rec + ((size_t)(cg0 + c) * H_v + h) * kRecBytes, kRecBytes,
                  &full[st]);
+        return true;
     };
 
     if (warp > kIssueWarp) {
@@ -696,9 +731,12 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
         const uint32_t ctl = tmem + ((uint32_t)(qo * 32) << 16);
         uint8_t* ost = sm + CS_OST;
         const bool loader = warp == kLoadWarp && lane == 0;
-        int issued = nchunks < kRing ? nchunks : kRing;
+        int issued = 0;
         if (loader)
-            for (int c = 0; c < issued; ++c) issue_loads(c);
+            for (int c = 0; c < kRing && c < nchunks; ++c) {
+                if (!issue_loads(c)) break;
+                issued = c + 1;
+            }
         __syncwarp();
 #pragma unroll 1
         for (int cp = 0; cp < nchunks; ++cp) {
@@ -759,9 +797,8 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
                 }
                 named_bar_sync(2, kOut);
             }
-            if (loader && cp + kRing < nchunks) {
-                issue_loads(cp + kRing);
-                issued = cp + kRing + 1;
+            if (loader && cp + kRing < nchunks && issued == cp + kRing) {
+                if (issue_loads(cp + kRing)) issued = cp + kRing + 1;
             }
             __syncwarp();
         }
@@ -1017,19 +1054,122 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
     }
 
     tc_fence_before();
-    __syncthreads();
+    named_bar_sync(sync_id, kChainThreads);
     tc_fence_after();
     if (tid == 0 && *s_err) set_status(status, kStatusTimeout);
+}
+
+__global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+    const float* __restrict__ S0g, const int32_t* __restrict__ cu_seqlens,
+    const int32_t* __restrict__ choff, int64_t T_total, int H_qk, int H_v,
+    const uint8_t* __restrict__ rec, bf16* __restrict__ o, float* __restrict__ Sfg, int* status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + CS_TMEM);
+    const int warp = threadIdx.x >> 5;
+    if (warp == 0) {
+        tmem_alloc(s_tmem, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+    chain_unit(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v, rec, o, Sfg,
+               status, nullptr, sm, threadIdx.x, blockIdx.x / H_v, blockIdx.x % H_v, tmem, 1);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ==================================== fused =======================================
+// Prep and chain in one cooperative launch (every block resident at once), so the
+// chain of the first sequences runs while prep workers produce the later records.
+// Blocks 0 .. c0-1 start on the chain units; the others run two prep workers each
+// (256 threads, their own 90 KB of shared memory and 64 TMEM columns), then join
+// the chain. Chain units are handed out in (sequence, V head) order by an atomic
+// counter; a chain's loader waits (bounded) for each record's flag before its bulk
+// copy, and prep workers never wait on chains, so every wait ends.
+constexpr int kFusedThreads = 512;
+constexpr uint32_t kPrepRegion = 92160;
+static_assert(kPrepRegion + 1024 >= kPrepSmem, "prep worker region too small");
+constexpr size_t kFusedSmem =
+    kChainSmem > 2 * (size_t)kPrepRegion + 1024 ? kChainSmem : 2 * (size_t)kPrepRegion + 1024;
+constexpr int kChainSync = 5;  // named barrier of the chain threads in the fused kernel
+
+__global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+    const bf16* __restrict__ q, const bf16* __restrict__ k, const float* __restrict__ a,
+    const float* __restrict__ b, const float* __restrict__ A_log,
+    const float* __restrict__ dt_bias, const float* __restrict__ S0g,
+    const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict__ choff, int32_t N,
+    int64_t T_total, int H_qk, int H_v, float scale, uint8_t* __restrict__ rec,
+    bf16* __restrict__ o, float* __restrict__ Sfg, int* status, int* flags, int* counter,
+    int chain_units, int c0) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x;
+    if ((int)blockIdx.x >= c0) {
+        const int sub = tid >> 8;
+        prep_worker(q, k, a, b, A_log, dt_bias, cu_seqlens, choff, N, H_qk, H_v, scale, rec,
+                    status, flags, sm + sub * kPrepRegion, tid & 255, 3 + sub,
+                    2 * ((int)blockIdx.x - c0) + sub, 2 * ((int)gridDim.x - c0), false);
+        __syncthreads();  // both workers are done and have freed their TMEM
+    }
+    if (tid >= kChainThreads) return;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + CS_TMEM);
+    volatile int* s_unit = reinterpret_cast<volatile int*>(sm + CS_ERR + 8);
+    if ((tid >> 5) == 0) {
+        tmem_alloc(s_tmem, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    named_bar_sync(kChainSync, kChainThreads);
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+#pragma unroll 1
+    for (;;) {
+        if (tid == 0) *s_unit = atomicAdd(counter, 1);
+        named_bar_sync(kChainSync, kChainThreads);
+        const int u = *s_unit;
+        named_bar_sync(kChainSync, kChainThreads);
+        if (u >= chain_units) break;
+        chain_unit(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v, rec, o,
+                   Sfg, status, flags, sm, tid, u / H_v, u % H_v, tmem, kChainSync);
+    }
+    tc_fence_before();
+    named_bar_sync(kChainSync, kChainThreads);
+    tc_fence_after();
+    if ((tid >> 5) == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
+// Workspace: chunk offsets [N + 1] | record flags [records] | counter | records.
+struct TcWorkspace {
+    size_t off_flags, off_counter, off_rec, total;
+};
+
+TcWorkspace tc_workspace_layout(int32_t N, int64_t T, int32_t H_v) {
+    const size_t records = ((size_t)((T + kC - 1) / kC) + (size_t)N) * H_v;
+    TcWorkspace w;
+    w.off_flags = align256((size_t)(N + 1) * sizeof(int32_t));
+    w.off_counter = w.off_flags + align256(records * sizeof(int32_t));
+    w.off_rec = w.off_counter + 256;
+    w.total = w.off_rec + records * kRecBytes;
+    return w;
+}
+
 }  // namespace
 
 size_t prefill_tc_workspace_bytes(int32_t N, int64_t T, int32_t H_v) {
-    const size_t chunk_bound = (size_t)((T + kC - 1) / kC) + (size_t)N;
-    return align256((size_t)(N + 1) * sizeof(int32_t)) + chunk_bound * H_v * kRecBytes;
+    return tc_workspace_layout(N, T, H_v).total;
 }
 
 bool prefill_tc_supported(int32_t H_qk, int32_t H_v) { return H_v / H_qk <= kMaxGroup; }
@@ -1073,11 +1213,15 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
                               const float* b, const float* A_log, const float* dt_bias,
                               const float* S0, const int32_t* cu_seqlens, int32_t N, int64_t T,
                               int32_t H_qk, int32_t H_v, float scale, void* o, float* S_final,
-                              void* workspace, int* status, cudaStream_t s) {
+                              void* workspace, bool fused, int* status, cudaStream_t s) {
     if (N == 0) return cudaSuccess;
     if (T > (int64_t)0x7FFFFFFF - kC) return cudaErrorInvalidValue;  // TMA token coordinates
-    int32_t* choff = static_cast<int32_t*>(workspace);
-    uint8_t* rec = static_cast<uint8_t*>(workspace) + align256((size_t)(N + 1) * sizeof(int32_t));
+    const TcWorkspace ws = tc_workspace_layout(N, T, H_v);
+    uint8_t* wb = static_cast<uint8_t*>(workspace);
+    int32_t* choff = reinterpret_cast<int32_t*>(wb);
+    int* flags = reinterpret_cast<int*>(wb + ws.off_flags);
+    int* counter = reinterpret_cast<int*>(wb + ws.off_counter);
+    uint8_t* rec = wb + ws.off_rec;
     // With no tokens the maps are never read; any aligned device address will do.
     CUtensorMap tm_q, tm_k, tm_v, tm_o;
     if (!make_rows_map(&tm_q, T > 0 ? q : workspace, H_qk, T) ||
@@ -1085,13 +1229,51 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
         !make_rows_map(&tm_v, T > 0 ? v : workspace, H_v, T) ||
         !make_rows_map(&tm_o, T > 0 ? o : workspace, H_v, T))
         return cudaErrorInvalidValue;
-    int dev = 0, num_sms = 0;
+    int dev = 0, num_sms = 0, coop = 0;
     cudaGetDevice(&dev);
     if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         num_sms <= 0)
         num_sms = 148;
-    cudaError_t e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kPrepSmem);
+    if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess) coop = 0;
+    cudaError_t e;
+    const int64_t chain_units = (int64_t)N * H_v;
+
+    if (fused && coop) {
+        e = cudaFuncSetAttribute(fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kFusedSmem);
+        if (e != cudaSuccess) return e;
+        int per_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fused_kernel, kFusedThreads,
+                                                          kFusedSmem);
+        if (e != cudaSuccess) return e;
+        const int grid = per_sm >= 1 ? num_sms : 0;
+        if (grid >= 2 && chain_units < ((int64_t)1 << 30)) {
+            const int c0 = (int)(chain_units < grid / 2 ? chain_units : grid / 2);
+            e = cudaMemsetAsync(wb + ws.off_flags, 0, ws.off_rec - ws.off_flags, s);
+            if (e != cudaSuccess) return e;
+            ktimer_before(s);
+            chunk_offsets_kernel<<<1, 256, 0, s>>>(cu_seqlens, N, T, choff, status);
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+            ktimer_after(s, "chunk_offsets");
+            const bf16* qb = static_cast<const bf16*>(q);
+            const bf16* kb = static_cast<const bf16*>(k);
+            bf16* ob = static_cast<bf16*>(o);
+            int units = (int)chain_units;
+            int c0v = c0;
+            void* args[] = {&tm_q, &tm_k, &tm_v, &tm_o, &qb, &kb, &a, &b, &A_log, &dt_bias, &S0,
+                            &cu_seqlens, &choff, &N, &T, &H_qk, &H_v, &scale, &rec, &ob,
+                            &S_final, &status, &flags, &counter, &units, &c0v};
+            ktimer_before(s);
+            e = cudaLaunchCooperativeKernel((const void*)fused_kernel, dim3(grid),
+                                            dim3(kFusedThreads), args, kFusedSmem, s);
+            if (e == cudaSuccess) ktimer_after(s, "fused");
+            return e;
+        }
+    }
+
+    e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kPrepSmem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kChainSmem);
@@ -1113,9 +1295,8 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
         if (e != cudaSuccess) return e;
         ktimer_after(s, "prep");
     }
-    const int64_t blocks = (int64_t)N * H_v;
     ktimer_before(s);
-    chain_kernel<<<(unsigned)blocks, kChainThreads, kChainSmem, s>>>(
+    chain_kernel<<<(unsigned)chain_units, kChainThreads, kChainSmem, s>>>(
         tm_q, tm_k, tm_v, tm_o, S0, cu_seqlens, choff, T, H_qk, H_v, rec, static_cast<bf16*>(o),
         S_final, status);
     e = cudaGetLastError();

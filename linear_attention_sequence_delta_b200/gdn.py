@@ -31,7 +31,7 @@ EXPORTS = ["gdn_status_string", "gdn_version", "gdn_prefill_workspace_size", "gd
            "gdn_prefill", "gdn_decode_step", "gdn_sync_status", "gdn_prefill_noalloc",
            "gdn_set_prefill_impl", "gdn_set_kernel_timing", "gdn_last_prefill_kernel_ms",
            "gdn_last_prefill_kernel_name"]
-GDN_IMPL_AUTO, GDN_IMPL_CUDA_CORE, GDN_IMPL_TENSOR_CORE = 0, 1, 2
+GDN_IMPL_AUTO, GDN_IMPL_CUDA_CORE, GDN_IMPL_TENSOR_CORE, GDN_IMPL_TENSOR_CORE_SPLIT = 0, 1, 2, 3
 
 
 class GDNError(RuntimeError):

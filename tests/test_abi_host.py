@@ -44,10 +44,11 @@ def test_status_strings(lib):
 def test_workspace_size(lib):
     ws = lib.gdn_prefill_workspace_size
     a256 = lambda x: (x + 255) // 256 * 256
-    # d = 128: chunk offsets (N + 1 int32) + one 17,664-byte record per (chunk, V head),
-    # with at most ceil(T / 64) + N chunks over all sequences
-    assert ws(1, 4096, 16, 32, 128, 128) == a256(2 * 4) + (64 + 1) * 32 * 17664
-    assert ws(4, 4 * 16384, 16, 64, 128, 128) == a256(5 * 4) + (1024 + 4) * 64 * 17664
+    # d = 128: chunk offsets (N + 1 int32), a flag per record, a counter block, and one
+    # 17,664-byte record per (chunk, V head), with at most ceil(T / 64) + N chunks
+    tc = lambda N, recs: a256((N + 1) * 4) + a256(recs * 4) + 256 + recs * 17664
+    assert ws(1, 4096, 16, 32, 128, 128) == tc(1, (64 + 1) * 32)
+    assert ws(4, 4 * 16384, 16, 64, 128, 128) == tc(4, (1024 + 4) * 64)
     # never below the CUDA-core path's need (G and beta, fp32 [T, H_v] each)
     assert ws(1, 3, 1, 1, 128, 128) >= 2 * 256
     assert ws(1, 3, 1, 1, 64, 64) == 2 * 256  # each part rounded up to 256 bytes
@@ -161,8 +162,9 @@ def test_binding_fails_loudly_without_library(tmp_path):
 def test_set_prefill_impl(lib):
     assert lib.gdn_set_prefill_impl(1) == 0
     assert lib.gdn_set_prefill_impl(2) == 1
+    assert lib.gdn_set_prefill_impl(3) == 2
     assert lib.gdn_set_prefill_impl(7) == -1      # invalid: unchanged
-    assert lib.gdn_set_prefill_impl(0) == 2
+    assert lib.gdn_set_prefill_impl(0) == 3
 
 
 def test_kernel_timing_switch(lib):

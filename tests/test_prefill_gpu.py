@@ -174,11 +174,15 @@ def impl_switch():
     gdn.set_prefill_impl(prev)
 
 
-@pytest.mark.parametrize("impl", ["cuda_core", "tensor_core"])
+IMPLS = {"cuda_core": "GDN_IMPL_CUDA_CORE", "tensor_core": "GDN_IMPL_TENSOR_CORE",
+         "tensor_core_split": "GDN_IMPL_TENSOR_CORE_SPLIT"}
+
+
+@pytest.mark.parametrize("impl", list(IMPLS))
 @pytest.mark.parametrize("lengths", [[1], [63], [64], [65], [127], [200], [5, 0, 130, 64]])
-def test_bf16_both_implementations(impl_switch, impl, lengths):
+def test_bf16_every_implementation(impl_switch, impl, lengths):
     g = impl_switch
-    g.set_prefill_impl(g.GDN_IMPL_CUDA_CORE if impl == "cuda_core" else g.GDN_IMPL_TENSOR_CORE)
+    g.set_prefill_impl(getattr(g, IMPLS[impl]))
     P = make_prefill_inputs(lengths, H_qk=2, H_v=4, d_k=128, d_v=128, state_std=0.05,
                             seed=sum(lengths) + 7)
     _check(P, TOL_BF16)
@@ -209,7 +213,8 @@ def test_kernel_timing_names_and_durations(impl_switch):
     P = make_prefill_inputs([300, 77], H_qk=2, H_v=4, d_k=128, d_v=128, seed=31)
     prev = g.set_kernel_timing(True)
     try:
-        for impl, names in ((g.GDN_IMPL_TENSOR_CORE, ["chunk_offsets", "prep", "chain"]),
+        for impl, names in ((g.GDN_IMPL_TENSOR_CORE, ["chunk_offsets", "fused"]),
+                            (g.GDN_IMPL_TENSOR_CORE_SPLIT, ["chunk_offsets", "prep", "chain"]),
                             (g.GDN_IMPL_CUDA_CORE, ["gates", "prefill_simt"])):
             g.set_prefill_impl(impl)
             _run(P)
@@ -218,3 +223,22 @@ def test_kernel_timing_names_and_durations(impl_switch):
             assert all(0.0 < ms < 1000.0 for _, ms in times)
     finally:
         g.set_kernel_timing(prev)
+
+
+@pytest.mark.parametrize("wl", ["prefill_35b", "varlen_64"])
+def test_fused_equals_split(impl_switch, wl):
+    """The overlapped single launch and the separate launches compute the same thing
+    (same arithmetic, different scheduling): outputs agree to the last bit."""
+    g = impl_switch
+    W = dict(WORKLOADS[wl])
+    if wl == "varlen_64":
+        W["num_seqs"] = 12
+    P = make_prefill_inputs(**W, seed=3, device="cuda")
+    outs = []
+    for impl in (g.GDN_IMPL_TENSOR_CORE, g.GDN_IMPL_TENSOR_CORE_SPLIT):
+        g.set_prefill_impl(impl)
+        o, Sf = gdn_prefill(P.q, P.k, P.v, P.a, P.b, P.A_log, P.dt_bias, P.cu_seqlens,
+                            P.initial_state)
+        assert gdn_sync_status() == 0
+        outs.append((o, Sf))
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
