@@ -2,8 +2,9 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One JSON line on rank 0. A "step" is one gdn_prefill call (chunk offsets, prep
-and chain kernels of the tensor-core path) on the 35B-A3B GDN layer shape: B=1, T=4096, 16 QK / 32 V heads,
+One JSON line on rank 0. A "step" is one gdn_prefill call (the chunk-offsets
+kernel and the fused prep + chunk-chain kernel of the tensor-core path) on the
+35B-A3B GDN layer shape: B=1, T=4096, 16 QK / 32 V heads,
 d=128, bf16 q/k/v/o, fp32 gates and state, zero initial state, final state
 written. `value` is prefill tokens/s over the whole job (all ranks; each rank
 runs its own copy of the workload, so scaling is weak). The same line carries
@@ -17,12 +18,13 @@ timed region; the max over ranks. `e2e` repeats the prefill through the public
 Python API from pinned host buffers, host<->device copies inside the timing.
 The CPU baseline is the fp64 oracle (test infrastructure) timed on this host.
 
-`roofline` is that of the dominant kernel (the chain): its duration comes from
-the library's kernel timing (CUDA events recorded around each launch on the
-launching stream, every timed step), its algorithmic bytes are those it must
-move (q, k, v read, o and the final state written); `traffic` is the DRAM bytes
-per launch from the committed ncu summary of that kernel, null when the summary
-was taken on another build of it. `roofline.step` gives the whole call against
+`roofline` is that of the dominant kernel (the fused prep + chain kernel): its
+duration comes from the library's kernel timing (CUDA events recorded around
+each launch on the launching stream, every timed step), its algorithmic bytes
+are those of the whole path (q, k, v, a, b read, o and the final state
+written), all of which it moves; `traffic` is the DRAM bytes per launch from
+the committed ncu summary of that kernel, null when the summary was taken on
+another build of it. `roofline.step` gives the whole call against
 the slower of the HBM and tensor roofs.
 """
 from __future__ import annotations
@@ -68,14 +70,14 @@ def chain_bytes(T, N, H_qk, H_v, d, io_bytes, with_initial):
     return prefill_bytes(T, N, H_qk, H_v, d, io_bytes, with_initial) - 2 * T * H_v * 4
 
 
-CHAIN_PROFILE = os.path.join(ROOT, "profiles", "chain_kernel_prefill35b.md")
+KERNEL_PROFILE = os.path.join(ROOT, "profiles", "fused_kernel_prefill35b.md")
 
 
-def _chain_traffic():
-    """(DRAM bytes per launch, kernel build id) from the ncu summary of the chain kernel."""
+def _kernel_traffic():
+    """(DRAM bytes per launch, kernel build id) from the ncu summary of the dominant kernel."""
     try:
         vals = {}
-        with open(CHAIN_PROFILE) as f:
+        with open(KERNEL_PROFILE) as f:
             for line in f:
                 if ":" in line and line.strip().startswith(("traffic_bytes_per_launch",
                                                             "kernel_source_sha1")):
@@ -86,7 +88,7 @@ def _chain_traffic():
         return None, None
 
 
-def _chain_source_sha1():
+def _kernel_source_sha1():
     import hashlib
     src = os.path.join(ROOT, "linear_attention_sequence_delta_b200", "csrc", "gdn_prefill_tc.cu")
     with open(src, "rb") as f:
@@ -265,9 +267,10 @@ def run_ours(args):
     mean_k = {n_: _max_over_ranks(sum(v_) / len(v_), ws, dev) for n_, v_ in kernel_ms.items()}
     dom = max(mean_k, key=mean_k.get)
     dom_ms = mean_k[dom]
-    dom_bytes = chain_bytes(T, N, H_qk, H_v, d, 2, with_initial=False)
-    traffic, traffic_src = _chain_traffic()
-    if dom != "chain" or traffic_src != _chain_source_sha1():
+    dom_bytes = (chain_bytes(T, N, H_qk, H_v, d, 2, with_initial=False) if dom == "chain"
+                 else byts)
+    traffic, traffic_src = _kernel_traffic()
+    if dom != "fused" or traffic_src != _kernel_source_sha1():
         traffic = None  # the counters were taken on another build of the kernel
 
     e2e = None
