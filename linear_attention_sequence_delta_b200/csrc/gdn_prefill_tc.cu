@@ -584,6 +584,8 @@ constexpr int kChainThreads = 416;  // warps 0-7 state, warp 8 MMA issue, warps 
 constexpr int kChain = 256;
 constexpr int kOut = 128;
 constexpr int kIssueWarp = 8;
+constexpr int kRdyBar = 6;     // named barrier: state threads arrive, the issuing warp waits
+constexpr int kRdyCount = 288;
 constexpr int kLoadWarp = 9;
 constexpr int kRing = 3;
 // shared memory map (bytes from a 1024-byte aligned base)
@@ -627,11 +629,12 @@ __device__ __forceinline__ uint32_t tile64_off(int t, int i) {
 //   warps 0-7   the state, fp32 in registers: two warps share each TMEM lane
 //               quarter, warp w owning value rows 32 (w & 3) .. + 31 and, of every
 //               64- or 128-column quantity of those rows (the state included), the
-//               half w >> 2. After each step's TMEM stores they arrive on `rdy`
-//               (one lane per warp) and go on.
+//               half w >> 2. After each step's TMEM stores they arrive on a named
+//               barrier that the issuing warp waits on, and go on.
 //   warp 8      issues every MMA (elect.sync), each group once its inputs are
 //               ready, and commits them to mbarriers; it does nothing else, so a
-//               full tensor-core queue never holds up the state warps.
+//               full tensor-core queue never holds up the state warps. Both sides
+//               take exactly three barrier steps per chunk, errors included.
 //   warps 9-12  (one per lane quarter) turn each chunk's output accumulators into o
 //               (S0 Q^T alternates between two accumulators) and, once a chunk's
 //               ring slot is no longer read, load the chunk three ahead into it
@@ -665,8 +668,7 @@ __device__ __forceinline__ void chain_unit(
     uint64_t* mbar = full + kRing;         // chain MMA completions
     uint64_t* obar = mbar + 1;             // [2] chunk parity b: output accumulators complete
     uint64_t* ofree = mbar + 3;            // [2] chunk parity b: output accumulators read
-    uint64_t* rdy = mbar + 5;              // a state step's TMEM operands written (8 arrivals)
-    uint64_t* dbar = mbar + 6;             // drain of in-flight MMAs before the exit
+    uint64_t* dbar = mbar + 5;             // drain of in-flight MMAs before the exit
     volatile int* s_err = reinterpret_cast<volatile int*>(sm + CS_ERR);
 
     const int warp = tid >> 5, lane = tid & 31;
@@ -684,7 +686,6 @@ __device__ __forceinline__ void chain_unit(
         mbar_init(&obar[1], 1);
         mbar_init(&ofree[0], 4);
         mbar_init(&ofree[1], 4);
-        mbar_init(rdy, 8);
         mbar_init(dbar, 1);
         *s_err = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -813,15 +814,30 @@ __device__ __forceinline__ void chain_unit(
         __syncwarp();
     } else if (warp == kIssueWarp) {
         // ================================ MMA issue =====================================
-        uint32_t rphase = 0;
-        auto wait_rdy = [&]() -> bool {
-            const bool ok = mbar_wait_bounded(rdy, rphase, kWaitCycles);
-            rphase ^= 1u;
+        // Three waits per chunk on the state threads' barrier, always (after an error
+        // the MMAs are skipped but the waits stay, so every arrival is consumed).
+        auto wait_rdy = [&]() {
+            named_bar_sync(kRdyBar, kRdyCount);
             tc_fence_after();
-            __syncwarp();
-            return ok;
         };
+        bool dead = false;
         constexpr uint32_t id64 = idesc_bf16_f32(128, 64, 0, 0);
+        constexpr uint32_t id_v = idesc_bf16_f32(128, 64, 1, 0);
+        constexpr uint32_t id_s = idesc_bf16_f32(128, 128, 0, 1);
+        // TMEM A operands (fixed for the whole unit)
+        uint32_t aS0[4], aS1[4], aZ[4], aU[4], aN[4];
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            aS0[ks] = tmem + TM_S0B + 8 * ks;
+            aS1[ks] = tmem + TM_S0B + 8 * (ks + 4);
+            aZ[ks] = tmem + TM_D1K + split_pairs_col(ks);
+            aU[ks] = tmem + TM_D1K + 8 * ks;
+            aN[ks] = tmem + TM_D3 + split_pairs_col(ks);
+        }
+        auto check = [&](bool ok) {  // warp-uniform: stop issuing after any failure
+            dead = __any_sync(0xffffffffu, dead || !ok || *s_err != 0);
+            if (dead) *s_err = 1;
+        };
 #pragma unroll 1
         for (int c = 0; c < nchunks; ++c) {
             const int st = c % kRing;
@@ -830,67 +846,58 @@ __device__ __forceinline__ void chain_unit(
             const uint32_t vt = smem_u32(slot + SLOT_V);
             const uint32_t tt = smem_u32(slot + SLOT_REC + REC_T);
             const uint32_t ptile = smem_u32(slot + SLOT_REC + REC_P);
-            bool ok = mbar_wait_bounded(&full[st], (c / kRing) & 1, kWaitCycles);
+            // shared-memory descriptors of this chunk's operands, formed while waiting
+            uint64_t dK0[4], dK1[4], dQ0[4], dQ1[4], dV[4], dT[4], dKm[4], dP[4];
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                dK0[ks] = smem_desc_sw128(kq + ks * 32u, 16, 1024);
+                dK1[ks] = smem_desc_sw128(kq + 16384u + ks * 32u, 16, 1024);
+                dQ0[ks] = smem_desc_sw128(kq + 8192u + ks * 32u, 16, 1024);
+                dQ1[ks] = smem_desc_sw128(kq + 16384u + 8192u + ks * 32u, 16, 1024);
+                dV[ks] = smem_desc_sw128(vt + ks * 2048u, 8192, 1024);
+                dT[ks] = smem_desc_sw128(tt + ks * 32u, 16, 1024);
+                dKm[ks] = smem_desc_sw128(kq + ks * 2048u, 16384, 1024);
+                dP[ks] = smem_desc_sw128(ptile + ks * 32u, 16, 1024);
+            }
+            if (!dead) check(mbar_wait_bounded(&full[st], (c / kRing) & 1, kWaitCycles));
             // (1) the bf16 state is written: S0 K^T, then V^T (T diag(beta))^T
-            ok = wait_rdy() && ok;
-            if (!ok || *s_err) { *s_err = 1; break; }
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t off = (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u;
-                mma_bf16_ts_warp(tmem + TM_D1K, tmem + TM_S0B + 8 * ks,
-                                 smem_desc_sw128(kq + off, 16, 1024), id64, ks > 0);
+            wait_rdy();
+            check(true);
+            if (!dead) {
+                mma_ts_group4(tmem + TM_D1K, aS0, dK0, id64, 0);
+                mma_ts_group4(tmem + TM_D1K, aS1, dK1, id64, 1);
+                mma_commit_warp(mbar);
+                mma_ss_group4(tmem + TM_D3, dV, dT, id_v, 0);
             }
-            mma_commit_warp(mbar);
-            {
-                constexpr uint32_t id_v = idesc_bf16_f32(128, 64, 1, 0);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ss_warp(tmem + TM_D3, smem_desc_sw128(vt + ks * 2048, 8192, 1024),
-                                     smem_desc_sw128(tt + ks * 32, 16, 1024), id_v, ks > 0);
+            // (2) Z^T is written: Vn^T += Z^T (T diag(beta))^T; then S0 Q^T into the
+            // accumulator of parity c & 1, last read for chunk c - 2
+            wait_rdy();
+            check(true);
+            if (!dead) {
+                mma_ts_group4(tmem + TM_D3, aZ, dT, id64, 1);
+                mma_commit_warp(mbar);
+                if (c >= 2)
+                    check(mbar_wait_bounded(&ofree[c & 1], ((c - 2) >> 1) & 1, kWaitCycles));
             }
-            // (2) Z^T is written: Vn^T += Z^T (T diag(beta))^T; then S0 Q^T
-            if (!wait_rdy() || *s_err) { *s_err = 1; break; }
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16_ts_warp(tmem + TM_D3, tmem + TM_D1K + split_pairs_col(ks),
-                                 smem_desc_sw128(tt + ks * 32, 16, 1024), id64, 1);
-            mma_commit_warp(mbar);
-            if (c >= 2 && !mbar_wait_bounded(&ofree[c & 1], ((c - 2) >> 1) & 1, kWaitCycles)) {
-                *s_err = 1;
-                break;
-            }
-            __syncwarp();
-            {
+            if (!dead) {
                 const uint32_t qacc = tmem + ((c & 1) ? TM_D1Q1 : TM_D1Q0);
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t off =
-                        8192u + (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u;
-                    mma_bf16_ts_warp(qacc, tmem + TM_S0B + 8 * ks,
-                                     smem_desc_sw128(kq + off, 16, 1024), id64, ks > 0);
-                }
+                mma_ts_group4(qacc, aS0, dQ0, id64, 0);
+                mma_ts_group4(qacc, aS1, dQ1, id64, 1);
             }
             // (3) the Vn^T pairs are written: the state increment, then Vn^T P^T
-            if (!wait_rdy() || *s_err) { *s_err = 1; break; }
-            {
-                constexpr uint32_t id_s = idesc_bf16_f32(128, 128, 0, 1);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ts_warp(tmem + TM_U, tmem + TM_D1K + 8 * ks,
-                                     smem_desc_sw128(kq + ks * 2048, 16384, 1024), id_s, ks > 0);
+            wait_rdy();
+            check(true);
+            if (!dead) {
+                mma_ts_group4(tmem + TM_U, aU, dKm, id_s, 0);
+                mma_commit_warp(mbar);
+                if (c >= 1)
+                    check(mbar_wait_bounded(&ofree[(c - 1) & 1], ((c - 1) >> 1) & 1,
+                                            kWaitCycles));
             }
-            mma_commit_warp(mbar);
-            if (c >= 1 &&
-                !mbar_wait_bounded(&ofree[(c - 1) & 1], ((c - 1) >> 1) & 1, kWaitCycles)) {
-                *s_err = 1;
-                break;
+            if (!dead) {
+                mma_ts_group4(tmem + TM_D4, aN, dP, id64, 0);
+                mma_commit_warp(&obar[c & 1]);
             }
-            __syncwarp();
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16_ts_warp(tmem + TM_D4, tmem + TM_D3 + split_pairs_col(ks),
-                                 smem_desc_sw128(ptile + ks * 32, 16, 1024), id64, ks > 0);
-            mma_commit_warp(&obar[c & 1]);
         }
         __syncwarp();
         // no MMA may still run when the tensor memory is freed
@@ -924,21 +931,24 @@ __device__ __forceinline__ void chain_unit(
         }
 
         uint32_t mphase = 0;
-        auto wait_mma = [&]() -> bool {  // warp-uniform
-            bool ok = mbar_wait_bounded(mbar, mphase, kWaitCycles);
+        bool dead = false;  // warp-uniform: after an error only the barrier arrivals remain
+        auto wait_mma = [&]() {
+            if (dead) return;
+            bool ok = *s_err == 0 && mbar_wait_bounded(mbar, mphase, kWaitCycles);
             mphase ^= 1u;
-            ok = !__any_sync(0xffffffffu, !ok || *s_err != 0);
-            if (!ok) *s_err = 1;
+            dead = __any_sync(0xffffffffu, !ok || *s_err != 0);
+            if (dead) *s_err = 1;
             tc_fence_after();
-            return ok;
         };
         // this warp's TMEM operands of the step are written (and, before that, any
-        // shared-memory writes fenced): one arrival for the issuing warp
+        // shared-memory writes fenced): arrive for the issuing warp, always. After an
+        // error the arrival waits for the barrier to complete, so that no thread can
+        // run a barrier generation ahead of the issuing warp.
         auto signal_rdy = [&]() {
-            tmem_wait_st();
+            if (!dead) tmem_wait_st();
             tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(rdy);
+            if (dead) named_bar_sync(kRdyBar, kRdyCount);
+            else named_bar_arrive(kRdyBar, kRdyCount);
         };
         // S <- gamma S + U (the previous chunk's decay and increment)
         auto apply_update = [&](float gamma) {
@@ -952,7 +962,6 @@ __device__ __forceinline__ void chain_unit(
         };
 
         float gamma = 1.f;
-        bool done = true;
 #pragma unroll 1
         for (int c = 0; c < nchunks; ++c) {
             const int st = c % kRing;
@@ -963,18 +972,16 @@ __device__ __forceinline__ void chain_unit(
 
             // ---- the previous chunk's state update and this chunk's data -------------
             if (c > 0) {
-                if (!wait_mma()) { done = false; break; }
-                apply_update(gamma);
+                wait_mma();
+                if (!dead) apply_update(gamma);
             }
-            {
-                const bool okf = mbar_wait_bounded(&full[st], (c / kRing) & 1, kWaitCycles);
-                if (__any_sync(0xffffffffu, !okf)) {
-                    *s_err = 1;
-                    done = false;
-                    break;
-                }
+            if (!dead) {
+                const bool okf =
+                    *s_err == 0 && mbar_wait_bounded(&full[st], (c / kRing) & 1, kWaitCycles);
+                dead = __any_sync(0xffffffffu, !okf || *s_err != 0);
+                if (dead) *s_err = 1;
             }
-            if (L < kC) {
+            if (!dead && L < kC) {
                 // rows past the sequence's end hold the next sequence's tokens (or TMA
                 // zero fill): zero them
                 const int nz = (kC - L) * 8;  // 16-byte chunks per 64-column tile
@@ -989,60 +996,68 @@ __device__ __forceinline__ void chain_unit(
             }
 
             // ---- state: bf16 copy (A operand of S0 K^T and S0 Q^T) ----------------------
+            if (!dead) {
 #pragma unroll
-            for (int cb = 0; cb < 2; ++cb) {
-                uint32_t pk[16];
+                for (int cb = 0; cb < 2; ++cb) {
+                    uint32_t pk[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    pk[e] = pack_bf16x2(S[32 * cb + 2 * e], S[32 * cb + 2 * e + 1]);
-                tmem_st16(ctl + TM_S0B + 32 * hh + 16 * cb, pk);
+                    for (int e = 0; e < 16; ++e)
+                        pk[e] = pack_bf16x2(S[32 * cb + 2 * e], S[32 * cb + 2 * e + 1]);
+                    tmem_st16(ctl + TM_S0B + 32 * hh + 16 * cb, pk);
+                }
             }
             signal_rdy();
-            gamma = rg[RG_GAMMA];
+            if (!dead) gamma = rg[RG_GAMMA];
 
             // ---- Z^T = -(e^G rk) (S0 K^T) for this thread's 32 tokens, in place ----------
-            if (!wait_mma()) { done = false; break; }  // S0 K^T
+            wait_mma();  // S0 K^T
+            if (!dead) {
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {  // 16 tokens at a time
-                const float4* fk4 = reinterpret_cast<const float4*>(rg + RG_FK) + 8 * hh + 4 * q;
-                float x[16];
-                tmem_ld16_sync(ctl + TM_D1K + 32 * hh + 16 * q, x);
-                uint32_t pk[8];
+                for (int q = 0; q < 2; ++q) {  // 16 tokens at a time
+                    const float4* fk4 = reinterpret_cast<const float4*>(rg + RG_FK) + 8 * hh + 4 * q;
+                    float x[16];
+                    tmem_ld16_sync(ctl + TM_D1K + 32 * hh + 16 * q, x);
+                    uint32_t pk[8];
 #pragma unroll
-                for (int e4 = 0; e4 < 4; ++e4) {
-                    const float4 f = fk4[e4];
-                    pk[2 * e4] = pack_bf16x2(-f.x * x[4 * e4], -f.y * x[4 * e4 + 1]);
-                    pk[2 * e4 + 1] = pack_bf16x2(-f.z * x[4 * e4 + 2], -f.w * x[4 * e4 + 3]);
+                    for (int e4 = 0; e4 < 4; ++e4) {
+                        const float4 f = fk4[e4];
+                        pk[2 * e4] = pack_bf16x2(-f.x * x[4 * e4], -f.y * x[4 * e4 + 1]);
+                        pk[2 * e4 + 1] = pack_bf16x2(-f.z * x[4 * e4 + 2], -f.w * x[4 * e4 + 3]);
+                    }
+                    // over columns this thread has already read
+                    tmem_st8(ctl + TM_D1K + 32 * hh + 8 * q, pk);
                 }
-                // over columns this thread has read (the second half's loads precede
-                // nothing of the first half's stores in the same 16 columns)
-                tmem_st8(ctl + TM_D1K + 32 * hh + 8 * q, pk);
             }
             signal_rdy();
 
             // ---- Vn^T -> bf16 pairs (for P Vn) and decay-scaled pairs (state update) --
-            if (!wait_mma()) { done = false; break; }  // Vn^T
+            wait_mma();  // Vn^T
+            if (!dead) {
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                const float4* egl4 = reinterpret_cast<const float4*>(rg + RG_EGL) + 8 * hh + 4 * q;
-                float x[16];
-                tmem_ld16_sync(ctl + TM_D3 + 32 * hh + 16 * q, x);
-                uint32_t pk[8];
+                for (int q = 0; q < 2; ++q) {
+                    const float4* egl4 =
+                        reinterpret_cast<const float4*>(rg + RG_EGL) + 8 * hh + 4 * q;
+                    float x[16];
+                    tmem_ld16_sync(ctl + TM_D3 + 32 * hh + 16 * q, x);
+                    uint32_t pk[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) pk[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
-                tmem_st8(ctl + TM_D3 + 32 * hh + 8 * q, pk);  // over Vn^T columns read
+                    for (int e = 0; e < 8; ++e) pk[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
+                    tmem_st8(ctl + TM_D3 + 32 * hh + 8 * q, pk);  // over Vn^T columns read
 #pragma unroll
-                for (int e4 = 0; e4 < 4; ++e4) {
-                    const float4 w = egl4[e4];
-                    pk[2 * e4] = pack_bf16x2(x[4 * e4] * w.x, x[4 * e4 + 1] * w.y);
-                    pk[2 * e4 + 1] = pack_bf16x2(x[4 * e4 + 2] * w.z, x[4 * e4 + 3] * w.w);
+                    for (int e4 = 0; e4 < 4; ++e4) {
+                        const float4 w = egl4[e4];
+                        pk[2 * e4] = pack_bf16x2(x[4 * e4] * w.x, x[4 * e4 + 1] * w.y);
+                        pk[2 * e4 + 1] = pack_bf16x2(x[4 * e4 + 2] * w.z, x[4 * e4 + 3] * w.w);
+                    }
+                    tmem_st8(ctl + TM_D1K + 16 * hh + 8 * q, pk);  // Z^T there is consumed
                 }
-                tmem_st8(ctl + TM_D1K + 16 * hh + 8 * q, pk);  // Z^T there is consumed
             }
             signal_rdy();
         }
+        bool done = !dead;
         if (done && nchunks > 0) {  // the last chunk's state update
-            done = wait_mma();
+            wait_mma();
+            done = !dead;
             if (done) apply_update(gamma);
         }
         if (done && Sfg) {

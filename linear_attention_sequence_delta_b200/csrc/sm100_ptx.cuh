@@ -34,8 +34,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Wait for the phase with the given parity to complete; give up after
 // `max_cycles` SM clocks (returns false).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   long long max_cycles) {
+    if (mbar_test_wait(bar, parity)) return true;  // already complete: no suspend
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
@@ -232,6 +245,45 @@ __device__ __forceinline__ void mma_bf16_ts_warp(uint32_t d_tmem, uint32_t a_tme
         : "memory");
 }
 
+// A group of 4 or 8 MMAs into one accumulator issued by one elected lane of a
+// converged warp: A from TMEM (a[i]) or shared memory (descriptor ad[i]), B
+// descriptors b[i]; the first accumulates into D only if `acc_first`, the rest
+// always. Operands are formed before the call so the issue itself is a short
+// run of MMA instructions.
+__device__ __forceinline__ void mma_ts_group4(uint32_t d, const uint32_t (&a)[4],
+                                              const uint64_t (&b)[4], uint32_t idesc,
+                                              uint32_t acc_first) {
+    asm volatile(
+        "{\n\t.reg .pred e, p0, p1;\n\t"
+        "setp.ne.b32 p0, %10, 0;\n\t"
+        "setp.eq.b32 p1, %10, %10;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %5, %9, p0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %6, %9, p1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %7, %9, p1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %8, %9, p1;\n\t}"
+        ::"r"(d), "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]),
+        "l"(b[3]), "r"(idesc), "r"(acc_first)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_ss_group4(uint32_t d, const uint64_t (&a)[4],
+                                              const uint64_t (&b)[4], uint32_t idesc,
+                                              uint32_t acc_first) {
+    asm volatile(
+        "{\n\t.reg .pred e, p0, p1;\n\t"
+        "setp.ne.b32 p0, %10, 0;\n\t"
+        "setp.eq.b32 p1, %10, %10;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %5, %9, p0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %6, %9, p1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %7, %9, p1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %8, %9, p1;\n\t}"
+        ::"r"(d), "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]),
+        "l"(b[3]), "r"(idesc), "r"(acc_first)
+        : "memory");
+}
+
 __device__ __forceinline__ void mma_commit_warp(uint64_t* bar) {
     asm volatile(
         "{\n\t.reg .pred e;\n\t"
@@ -399,6 +451,11 @@ __device__ __forceinline__ void tmem_wait_st() {
 // Named barrier over `nthreads` threads (a multiple of 32) with id 1..15.
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Producer side of a named barrier: mark arrival and go on (no wait).
+__device__ __forceinline__ void named_bar_arrive(int id, int nthreads) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // Named barrier that also ORs a predicate over the participating threads: every
