@@ -136,9 +136,10 @@ int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
  *                         GDN_ERR_UNSUPPORTED for shapes/types they do not cover;
  *   GDN_IMPL_TENSOR_CORE_SPLIT
  *                         tensor cores with the state-free preparation and the
- *                         chunk chain as separate launches (the default runs them
- *                         in one cooperative launch, overlapped, where the device
- *                         supports it).
+ *                         chunk chain as separate launches always (by default
+ *                         they run in one cooperative launch, overlapped, when
+ *                         the device supports it and there are at most half as
+ *                         many (sequence, V head) chains as SMs).
  * Returns the previous setting, or -GDN_ERR_INVALID_ARG for an unknown value.
  * Not synchronised with calls in flight on other host threads.
  */

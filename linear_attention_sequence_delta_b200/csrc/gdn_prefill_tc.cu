@@ -1262,8 +1262,11 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
                                                           kFusedSmem);
         if (e != cudaSuccess) return e;
         const int grid = per_sm >= 1 ? num_sms : 0;
-        if (grid >= 2 && chain_units < ((int64_t)1 << 30)) {
-            const int c0 = (int)(chain_units < grid / 2 ? chain_units : grid / 2);
+        // Overlap pays when the chains are few (latency-bound: each holds one SM for
+        // its whole sequence); with many chains the separate launches keep both
+        // phases at full occupancy.
+        if (grid >= 2 && 2 * chain_units <= grid) {
+            const int c0 = (int)chain_units;
             e = cudaMemsetAsync(wb + ws.off_flags, 0, ws.off_rec - ws.off_flags, s);
             if (e != cudaSuccess) return e;
             ktimer_before(s);

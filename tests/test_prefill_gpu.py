@@ -213,7 +213,7 @@ def test_kernel_timing_names_and_durations(impl_switch):
     P = make_prefill_inputs([300, 77], H_qk=2, H_v=4, d_k=128, d_v=128, seed=31)
     prev = g.set_kernel_timing(True)
     try:
-        for impl, names in ((g.GDN_IMPL_TENSOR_CORE, ["chunk_offsets", "fused"]),
+        for impl, names in ((g.GDN_IMPL_TENSOR_CORE, ["chunk_offsets", "fused"]),  # 2 x 4 chains
                             (g.GDN_IMPL_TENSOR_CORE_SPLIT, ["chunk_offsets", "prep", "chain"]),
                             (g.GDN_IMPL_CUDA_CORE, ["gates", "prefill_simt"])):
             g.set_prefill_impl(impl)
@@ -232,13 +232,33 @@ def test_fused_equals_split(impl_switch, wl):
     g = impl_switch
     W = dict(WORKLOADS[wl])
     if wl == "varlen_64":
-        W["num_seqs"] = 12
+        W["num_seqs"] = 2  # 64 chains: few enough for the overlapped launch
     P = make_prefill_inputs(**W, seed=3, device="cuda")
     outs = []
-    for impl in (g.GDN_IMPL_TENSOR_CORE, g.GDN_IMPL_TENSOR_CORE_SPLIT):
-        g.set_prefill_impl(impl)
-        o, Sf = gdn_prefill(P.q, P.k, P.v, P.a, P.b, P.A_log, P.dt_bias, P.cu_seqlens,
-                            P.initial_state)
-        assert gdn_sync_status() == 0
-        outs.append((o, Sf))
+    prev = g.set_kernel_timing(True)
+    try:
+        for impl, kernel in ((g.GDN_IMPL_TENSOR_CORE, "fused"),
+                             (g.GDN_IMPL_TENSOR_CORE_SPLIT, "chain")):
+            g.set_prefill_impl(impl)
+            o, Sf = gdn_prefill(P.q, P.k, P.v, P.a, P.b, P.A_log, P.dt_bias, P.cu_seqlens,
+                                P.initial_state)
+            assert gdn_sync_status() == 0
+            assert kernel in [n for n, _ in g.last_prefill_kernel_times()]
+            outs.append((o, Sf))
+    finally:
+        g.set_kernel_timing(prev)
     assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+
+
+def test_many_chains_use_separate_launches(impl_switch):
+    """With more (sequence, V head) chains than half the SMs the default path runs the
+    preparation and the chains as separate launches."""
+    g = impl_switch
+    g.set_prefill_impl(g.GDN_IMPL_AUTO)
+    P = make_prefill_inputs([100] * 8, H_qk=16, H_v=32, d_k=128, d_v=128, seed=4)
+    prev = g.set_kernel_timing(True)
+    try:
+        _check(P, TOL_BF16)
+        assert [n for n, _ in g.last_prefill_kernel_times()] == ["chunk_offsets", "prep", "chain"]
+    finally:
+        g.set_kernel_timing(prev)
