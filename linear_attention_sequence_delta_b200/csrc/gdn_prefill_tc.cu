@@ -1115,6 +1115,7 @@ static_assert(kPrepRegion + 1024 >= kPrepSmem, "prep worker region too small");
 constexpr size_t kFusedSmem =
     kChainSmem > 2 * (size_t)kPrepRegion + 1024 ? kChainSmem : 2 * (size_t)kPrepRegion + 1024;
 constexpr int kChainSync = 5;  // named barrier of the chain threads in the fused kernel
+constexpr int kFusedMaxSeqs = 255;  // the fused kernel computes the chunk offsets itself
 
 __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -1122,14 +1123,47 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
     const bf16* __restrict__ q, const bf16* __restrict__ k, const float* __restrict__ a,
     const float* __restrict__ b, const float* __restrict__ A_log,
     const float* __restrict__ dt_bias, const float* __restrict__ S0g,
-    const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict__ choff, int32_t N,
+    const int32_t* __restrict__ cu_seqlens, const int32_t* choff, int32_t N,
     int64_t T_total, int H_qk, int H_v, float scale, uint8_t* __restrict__ rec,
     bf16* __restrict__ o, float* __restrict__ Sfg, int* status, int* flags, int* counter,
     int chain_units, int c0) {
     extern __shared__ uint8_t smem_raw[];
+    __shared__ int32_t s_choff[kFusedMaxSeqs + 1];
+    __shared__ int s_bad;
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x;
+    // chunk offsets of the sequences (prefix sum of ceil(len / 64)), by one warp
+    if (tid < 32) {
+        int32_t carry = 0;
+        bool bad = false;
+        for (int base = 0; base < N; base += 32) {
+            const int n = base + tid;
+            int32_t nc = 0;
+            if (n < N) {
+                const int64_t s0 = cu_seqlens[n], s1 = cu_seqlens[n + 1];
+                if (bad_seq(s0, s1, T_total, n)) bad = true;
+                else nc = (int32_t)((s1 - s0 + kC - 1) / kC);
+            }
+            int32_t x = nc;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int32_t y = __shfl_up_sync(0xffffffffu, x, off);
+                if (tid >= off) x += y;
+            }
+            if (n < N) s_choff[n] = carry + x - nc;
+            carry += __shfl_sync(0xffffffffu, x, 31);
+        }
+        bad = __any_sync(0xffffffffu, bad);
+        if (tid == 0) {
+            s_choff[N] = carry;
+            s_bad = bad ? 1 : 0;
+            if (bad && blockIdx.x == 0) set_status(status, kStatusBadSeqlens);
+        }
+    }
+    __syncthreads();
+    if (s_bad) return;  // reported; nothing is computed
+    choff = s_choff;
     if ((int)blockIdx.x >= c0) {
         const int sub = tid >> 8;
         prep_worker(q, k, a, b, A_log, dt_bias, cu_seqlens, choff, N, H_qk, H_v, scale, rec,
@@ -1265,15 +1299,10 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
         // Overlap pays when the chains are few (latency-bound: each holds one SM for
         // its whole sequence); with many chains the separate launches keep both
         // phases at full occupancy.
-        if (grid >= 2 && 2 * chain_units <= grid) {
+        if (grid >= 2 && 2 * chain_units <= grid && N <= kFusedMaxSeqs) {
             const int c0 = (int)chain_units;
             e = cudaMemsetAsync(wb + ws.off_flags, 0, ws.off_rec - ws.off_flags, s);
             if (e != cudaSuccess) return e;
-            ktimer_before(s);
-            chunk_offsets_kernel<<<1, 256, 0, s>>>(cu_seqlens, N, T, choff, status);
-            e = cudaGetLastError();
-            if (e != cudaSuccess) return e;
-            ktimer_after(s, "chunk_offsets");
             const bf16* qb = static_cast<const bf16*>(q);
             const bf16* kb = static_cast<const bf16*>(k);
             bf16* ob = static_cast<bf16*>(o);

@@ -213,7 +213,7 @@ def test_kernel_timing_names_and_durations(impl_switch):
     P = make_prefill_inputs([300, 77], H_qk=2, H_v=4, d_k=128, d_v=128, seed=31)
     prev = g.set_kernel_timing(True)
     try:
-        for impl, names in ((g.GDN_IMPL_TENSOR_CORE, ["chunk_offsets", "fused"]),  # 2 x 4 chains
+        for impl, names in ((g.GDN_IMPL_TENSOR_CORE, ["fused"]),  # 2 x 4 chains: overlapped
                             (g.GDN_IMPL_TENSOR_CORE_SPLIT, ["chunk_offsets", "prep", "chain"]),
                             (g.GDN_IMPL_CUDA_CORE, ["gates", "prefill_simt"])):
             g.set_prefill_impl(impl)
