@@ -189,9 +189,11 @@ constexpr uint32_t PS_RK = 82816;    // [64] rk, [64] rq (rq includes the scale)
 constexpr uint32_t PS_GA = 83328;    // [kMaxGroup][64] G of every V head of the unit
 constexpr uint32_t PS_BA = 87424;    // [kMaxGroup][64] beta of every V head of the unit
 constexpr uint32_t PS_PAR = 91520;   // [2][kMaxGroup] A_log, dt_bias of those heads
-constexpr uint32_t PS_BAR = 91648;   // mbarrier (MMA)
-constexpr uint32_t PS_TMEM = 91656;
-constexpr size_t kPrepSmem = 91664 + 1024;
+constexpr uint32_t PS_E = 91648;     // per head: [4][16][16] exp(G_i - G_j) inside 16-blocks
+constexpr uint32_t PS_CI = 95744;    // per head: [64] exp(G_i - G_{16-block start of i})
+constexpr uint32_t PS_BAR = 96000;   // mbarrier (MMA)
+constexpr uint32_t PS_TMEM = 96008;
+constexpr size_t kPrepSmem = 96016 + 1024;
 
 // Half a row (32 columns starting at 32 H) of A (row i < 64) or of P (row t =
 // i - 64) from the matching half row x of [K; Q] K^T. Columns left of the row's
@@ -199,45 +201,45 @@ constexpr size_t kPrepSmem = 91664 + 1024;
 // most 16 columns inside the block take their own exponential; columns right of
 // the row are zero. rowf = beta_i rk_i (A) or rq_t (P); rk gives the column factor.
 template <int H>
-__device__ __forceinline__ void ap_half_row(const float (&x)[32], int row, const float* G,
-                                            const float* U, const float* rk, float rowf,
-                                            float (&val)[32]) {
+__device__ __forceinline__ void ap_half_row(const float (&x)[32], int row, const float* U,
+                                            const float* E, const float* CI, const float* rk,
+                                            float rowf, float (&val)[32]) {
     const int i = row & 63;
     const int a0 = i & ~15;
-    const float Gi = G[i];
-    const float ci = __expf(Gi - G[a0]);
-    const float* Urow = U + (a0 >> 4) * 64 + 32 * H;
-    const float* Gc = G + 32 * H;
     const float4* rk4 = reinterpret_cast<const float4*>(rk + 32 * H);
     float cf[32];
 #pragma unroll
     for (int e4 = 0; e4 < 8; ++e4) {
         const float4 r4 = rk4[e4];
-        cf[4 * e4] = r4.x * x[4 * e4];
-        cf[4 * e4 + 1] = r4.y * x[4 * e4 + 1];
-        cf[4 * e4 + 2] = r4.z * x[4 * e4 + 2];
-        cf[4 * e4 + 3] = r4.w * x[4 * e4 + 3];
+        cf[4 * e4] = rowf * r4.x * x[4 * e4];
+        cf[4 * e4 + 1] = rowf * r4.y * x[4 * e4 + 1];
+        cf[4 * e4 + 2] = rowf * r4.z * x[4 * e4 + 2];
+        cf[4 * e4 + 3] = rowf * r4.w * x[4 * e4 + 3];
     }
-    if (a0 >= 32 * H + 32) {
-        const float f = rowf * ci;
+    // The half's two 16-column groups each lie wholly left of the row's 16-block
+    // (exp(G_i - G_j) = ci U_j, both factors <= 1), on it (the block's own table, zero
+    // right of the diagonal) or right of it (zero).
 #pragma unroll
-        for (int e = 0; e < 32; ++e) val[e] = f * Urow[e] * cf[e];
-    } else if (a0 == 32 * H + 16) {
-        const float f = rowf * ci;
+    for (int g = 0; g < 2; ++g) {
+        const int c0 = 32 * H + 16 * g;
+        const float4* t4;
+        float f;
+        if (c0 < a0) {
+            t4 = reinterpret_cast<const float4*>(U + (a0 >> 4) * 64 + c0);
+            f = CI[i];
+        } else {
+            t4 = reinterpret_cast<const float4*>(E + (a0 >> 4) * 256 + (i - a0) * 16);
+            f = c0 == a0 ? 1.f : 0.f;
+        }
 #pragma unroll
-        for (int e = 0; e < 16; ++e) val[e] = f * Urow[e] * cf[e];
-#pragma unroll
-        for (int e = 16; e < 32; ++e)
-            val[e] = (32 * H + e <= i) ? rowf * __expf(Gi - Gc[e]) * cf[e] : 0.f;
-    } else if (a0 == 32 * H) {
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-            val[e] = (32 * H + e <= i) ? rowf * __expf(Gi - Gc[e]) * cf[e] : 0.f;
-#pragma unroll
-        for (int e = 16; e < 32; ++e) val[e] = 0.f;
-    } else {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) val[e] = 0.f;
+        for (int e4 = 0; e4 < 4; ++e4) {
+            const float4 u = t4[e4];
+            const int e = 16 * g + 4 * e4;
+            val[e] = f * u.x * cf[e];
+            val[e + 1] = f * u.y * cf[e + 1];
+            val[e + 2] = f * u.z * cf[e + 2];
+            val[e + 3] = f * u.w * cf[e + 3];
+        }
     }
 }
 
@@ -267,6 +269,8 @@ __device__ __forceinline__ void prep_worker(
     float* sGall = reinterpret_cast<float*>(sm + PS_GA);
     float* sBall = reinterpret_cast<float*>(sm + PS_BA);
     float* sPar = reinterpret_cast<float*>(sm + PS_PAR);
+    float* sE = reinterpret_cast<float*>(sm + PS_E);
+    float* sCI = reinterpret_cast<float*>(sm + PS_CI);
     float* rq = rk + 64;
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + PS_BAR);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + PS_TMEM);
@@ -422,6 +426,14 @@ __device__ __forceinline__ void prep_worker(
             {  // U[a][j] = exp(G_{16 a} - G_j) for j < 16 a (both factors of a long gap <= 1)
                 const int ab4 = tid >> 6, jj = tid & 63;
                 sU[tid] = (jj < 16 * ab4) ? __expf(hG[16 * ab4] - hG[jj]) : 0.f;
+                // E[b][ii][jj] = exp(G_{16b+ii} - G_{16b+jj}) for jj <= ii, else 0
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const int idx = tid + kPrepThreads * q4;  // 0..1023
+                    const int bb = idx >> 8, ii = (idx >> 4) & 15, jb = idx & 15;
+                    sE[idx] = jb <= ii ? __expf(hG[16 * bb + ii] - hG[16 * bb + jb]) : 0.f;
+                }
+                if (tid < kC) sCI[tid] = __expf(hG[tid] - hG[tid & ~15]);
             }
             named_bar_sync(bar_id, kPrepThreads);
 
@@ -430,8 +442,8 @@ __device__ __forceinline__ void prep_worker(
                 float val[32];
                 const int i = trow & 63;
                 const float rowf = trow < 64 ? hBeta[i] * rk[i] : rq[i];
-                if (hh == 0) ap_half_row<0>(x, trow, hG, sU, rk, rowf, val);
-                else         ap_half_row<1>(x, trow, hG, sU, rk, rowf, val);
+                if (hh == 0) ap_half_row<0>(x, trow, sU, sE, sCI, rk, rowf, val);
+                else         ap_half_row<1>(x, trow, sU, sE, sCI, rk, rowf, val);
                 if (trow < 64) {
                     float4* Arow = reinterpret_cast<float4*>(As + i * kAsStride + 32 * hh);
 #pragma unroll
@@ -1110,7 +1122,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
 // counter; a chain's loader waits (bounded) for each record's flag before its bulk
 // copy, and prep workers never wait on chains, so every wait ends.
 constexpr int kFusedThreads = 512;
-constexpr uint32_t kPrepRegion = 92160;
+constexpr uint32_t kPrepRegion = 96256;
 static_assert(kPrepRegion + 1024 >= kPrepSmem, "prep worker region too small");
 constexpr size_t kFusedSmem =
     kChainSmem > 2 * (size_t)kPrepRegion + 1024 ? kChainSmem : 2 * (size_t)kPrepRegion + 1024;
