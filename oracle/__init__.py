@@ -19,6 +19,10 @@ Functions and the passages they follow:
   forward          -- gates followed by the recurrence
   decode_step      -- one token per sequence from a stored state (the same
                       recurrence with a length-1 sequence per slot)
+  conv1d_silu      -- causal depthwise convolution + SiLU over the q/k/v channels,
+                      with the per-sequence conv cache in and out (``mixer_oracle.c``;
+                      "Qwen3.5-MoE-35B-A3B architecture teardown", 3.3 phase 2)
+  rmsnorm_gated    -- RMSNorm(o) * w * SiLU(z) per row (3.3 phase 4)
 """
 from __future__ import annotations
 
@@ -30,6 +34,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "gdn_oracle.c")
+_SRCS = [_SRC, os.path.join(_HERE, "mixer_oracle.c")]
 _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 _lib = None
 
@@ -37,13 +42,13 @@ CHUNK = 64
 
 
 def build(force: bool = False) -> str:
-    """Compile gdn_oracle.c into liboracle.so next to it (gcc, OpenMP)."""
-    if force or not os.path.exists(_LIB_PATH) or (
-        os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)
+    """Compile the oracle's C sources into liboracle.so next to them (gcc, OpenMP)."""
+    if force or not os.path.exists(_LIB_PATH) or any(
+        os.path.getmtime(_LIB_PATH) < os.path.getmtime(src) for src in _SRCS
     ):
         tmp = _LIB_PATH + f".tmp{os.getpid()}"
         subprocess.check_call(
-            ["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", _SRC, "-o", tmp, "-lm"]
+            ["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", *_SRCS, "-o", tmp, "-lm"]
         )
         os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
@@ -65,6 +70,8 @@ def _load():
             P, P, P, P, P, P, P, P, P, i32, i64, i32, i32, i32, i32, f64, i32, P, P
         ]
         lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_conv1d_silu.argtypes = [P, P, P, P, P, i32, i32, i32, P, P]
+        lib.oracle_rmsnorm_gated.argtypes = [P, P, P, f64, i64, i32, P]
         _lib = lib
     return _lib
 
@@ -163,3 +170,35 @@ def decode_step(q, k, v, a, b, A_log, dt_bias, state, scale: float = 1.0):
     N = _f64(q).shape[0]
     cu = np.arange(N + 1, dtype=np.int64)
     return forward(q, k, v, a, b, A_log, dt_bias, cu, initial_state=state, scale=scale)
+
+
+def conv1d_silu(x, weight, bias, cu_seqlens, state_in=None, want_state: bool = True):
+    """Causal depthwise convolution + SiLU. Returns (y [T, C], state_out [N, K-1, C] or None).
+
+    x [T, C]; weight [C, K] (weight[:, K-1] multiplies the current token); bias [C] or
+    None; state_in [N, K-1, C] (the K-1 positions before each sequence, oldest first) or
+    None for zeros.
+    """
+    lib = _load()
+    x, w, bias, state_in = _f64(x), _f64(weight), _f64(bias), _f64(state_in)
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    T, C = x.shape
+    K = w.shape[1]
+    N = len(cu) - 1
+    assert w.shape[0] == C and cu[0] == 0 and cu[-1] == T
+    y = np.empty_like(x)
+    so = np.empty((N, K - 1, C)) if want_state else None
+    lib.oracle_conv1d_silu(_ptr(x), _ptr(w), _ptr(bias), _ptr(state_in), _ptr(cu), N, C, K,
+                           _ptr(y), _ptr(so))
+    return y, so
+
+
+def rmsnorm_gated(o, z, weight, eps: float = 1e-6):
+    """y = o / sqrt(mean(o^2) + eps) * weight * silu(z) over the last axis (length d)."""
+    lib = _load()
+    o, z, w = _f64(o), _f64(z), _f64(weight)
+    d = o.shape[-1]
+    rows = o.size // d
+    y = np.empty_like(o)
+    lib.oracle_rmsnorm_gated(_ptr(o), _ptr(z), _ptr(w), float(eps), rows, d, _ptr(y))
+    return y

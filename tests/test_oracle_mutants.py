@@ -16,6 +16,7 @@ import oracle
 from tests import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "gdn_oracle.c")
+MIXER_SRC = os.path.join(os.path.dirname(oracle.__file__), "mixer_oracle.c")
 
 MUTANTS = {
     # the P5 reading: read with the undecayed state (decay applied after)
@@ -71,14 +72,14 @@ def _mutate(src, name):
     return src
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_catch_mutant(name, tmp_path):
-    src = _mutate(open(SRC).read(), name)
+def _run_pins_on(tmp_path, gdn_src, mixer_src, pins_to_run, name):
     cpath = tmp_path / "m.c"
-    cpath.write_text(src)
+    cpath.write_text(gdn_src)
+    mpath = tmp_path / "mx.c"
+    mpath.write_text(mixer_src)
     so = tmp_path / "libm.so"
-    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", str(cpath), "-o",
-                           str(so), "-lm"])
+    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", str(cpath), str(mpath),
+                           "-o", str(so), "-lm"])
     saved_lib, saved_path = oracle._lib, oracle._LIB_PATH
     try:
         oracle._lib = None
@@ -87,7 +88,7 @@ def test_pins_catch_mutant(name, tmp_path):
         real_build = oracle.build
         oracle.build = lambda force=False: str(so)
         caught = 0
-        for pin in PINS:
+        for pin in pins_to_run:
             try:
                 pin()
             except AssertionError:
@@ -96,3 +97,35 @@ def test_pins_catch_mutant(name, tmp_path):
     finally:
         oracle.build = real_build
         oracle._lib, oracle._LIB_PATH = saved_lib, saved_path
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, tmp_path):
+    _run_pins_on(tmp_path, _mutate(open(SRC).read(), name), open(MIXER_SRC).read(), PINS, name)
+
+
+# planted slips in the convolution / gated-RMSNorm oracle, against its own pins
+MIXER_MUTANTS = {
+    "conv_taps_reversed": ("acc += w[(int64_t)c * K + i] * XAT(t - (K - 1) + i);",
+                           "acc += w[(int64_t)c * K + (K - 1 - i)] * XAT(t - (K - 1) + i);"),
+    "conv_window_off_by_one": ("acc += w[(int64_t)c * K + i] * XAT(t - (K - 1) + i);",
+                               "acc += w[(int64_t)c * K + i] * XAT(t - K + i);"),
+    "conv_cache_newest_first": ("state_in[((int64_t)n * W + (W + (p))) * C + c]",
+                                "state_in[((int64_t)n * W + (-1 - (p))) * C + c]"),
+    "conv_no_activation": ("y[(s0 + t) * C + c] = oracle_silu(acc);",
+                           "y[(s0 + t) * C + c] = acc;"),
+    "rms_sum_not_mean": ("const double inv = 1.0 / sqrt(ss / d + eps);",
+                         "const double inv = 1.0 / sqrt(ss + eps);"),
+    "rms_gate_sigmoid": ("y[r * d + e] = o[r * d + e] * inv * w[e] * oracle_silu(z[r * d + e]);",
+                         "y[r * d + e] = o[r * d + e] * inv * w[e] / (1.0 + exp(-z[r * d + e]));"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MIXER_MUTANTS))
+def test_mixer_pins_catch_mutant(name, tmp_path):
+    from tests import test_mixer_oracle_pins as mp
+    a, b = MIXER_MUTANTS[name]
+    src = open(MIXER_SRC).read()
+    assert a in src, name
+    mixer_pins = [getattr(mp, f) for f in dir(mp) if f.startswith("test_")]
+    _run_pins_on(tmp_path, open(SRC).read(), src.replace(a, b, 1), mixer_pins, name)
