@@ -107,6 +107,84 @@ def decode_bytes(N, H_qk, H_v, d, io_bytes):
     return 2 * N * H_v * d * d * 4 + N * (2 * H_qk * d + 2 * H_v * d) * io_bytes + 2 * N * H_v * 4
 
 
+def mixer_bytes(T, N, C, K, rows, d, io_bytes, N_dec, C_dec):
+    """Algorithmic HBM bytes of the steps around the delta rule: the conv reads x and
+    writes y (plus the taps and, per sequence, the K-1 cached positions written out);
+    the conv decode reads x, the taps and the cache and writes y and the slid cache; the
+    gated norm reads o and z and writes y (plus the d-long weight)."""
+    conv = 2 * T * C * io_bytes + C * K * 4 + N * (K - 1) * C * io_bytes
+    conv_dec = 2 * N_dec * C_dec * io_bytes + C_dec * K * 4 + 2 * N_dec * (K - 1) * C_dec * io_bytes
+    norm = 3 * rows * d * io_bytes + d * 4
+    return conv, conv_dec, norm
+
+
+def _time_op(fn, iters, flush, stream):
+    """Mean device time of fn() over iters launches, the L2 flushed before each."""
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(iters)]
+    for i in range(iters):
+        flush.fill_(i & 0xFF)
+        evs[i][0].record(stream)
+        fn()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in evs) / iters
+
+
+def run_mixer(rank, dev, flush, stream, hbm, peak_src, iters):
+    """The convolution in front of the delta rule and the gated norm after it, on the
+    35B-A3B layer (T=4096, conv_dim=8192, 32 V heads x 128) and the conv decode step on
+    the 397B-A17B decode batch (256 sequences, conv_dim=12288)."""
+    from linear_attention_sequence_delta_b200 import gdn
+    from linear_attention_sequence_delta_b200.inputs import make_mixer_inputs
+    M = make_mixer_inputs(num_seqs=1, seq_len=4096, H_qk=16, H_v=32, d_k=128, d_v=128,
+                          seed=rank, device=dev)
+    Md = make_mixer_inputs([1] * 256, H_qk=16, H_v=64, d_k=128, d_v=128, seed=rank,
+                           device=dev)
+    T, C = M.x.shape
+    K = M.conv_weight.shape[1]
+    y = torch.empty_like(M.x)
+    cst = torch.empty_like(M.conv_state)
+    yn = torch.empty_like(M.o)
+    yd = torch.empty_like(Md.x)
+    st_d = Md.conv_state.clone()
+    conv_ms = _time_op(lambda: gdn.gdn_conv1d_silu(M.x, M.conv_weight, None, M.cu_seqlens, None,
+                                                   out=y, conv_state_out=cst),
+                       iters, flush, stream)
+    dec_ms = _time_op(lambda: gdn.gdn_conv1d_silu_decode(Md.x, Md.conv_weight, None, st_d,
+                                                         out=yd),
+                      iters, flush, stream)
+    norm_ms = _time_op(lambda: gdn.gdn_rmsnorm_gated(M.o, M.z, M.norm_weight, 1e-6, out=yn),
+                       iters, flush, stream)
+    rows, d = M.o.shape[0] * M.o.shape[1], M.o.shape[2]
+    b_conv, b_dec, b_norm = mixer_bytes(T, 1, C, K, rows, d, 2, Md.x.shape[0], Md.x.shape[1])
+
+    def roof(b, ms_):
+        gbs = b / (ms_ / 1e3) / 1e9
+        return {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                "algorithmic_bytes": b, "kernel_ms": ms_, "peak_source": peak_src}
+
+    out = {
+        "conv1d_silu": {"workload": f"T={T}, conv_dim={C}, K={K}, bf16, zero cache in, "
+                                    "cache out", "tokens_per_s": T / (conv_ms / 1e3),
+                        "roofline": roof(b_conv, conv_ms), "launches_per_call": 2},
+        "conv1d_silu_decode": {"workload": f"{Md.x.shape[0]} seqs x 1 token, "
+                                           f"conv_dim={Md.x.shape[1]}, K={K}, bf16, "
+                                           "cache in place",
+                               "us_per_step": dec_ms * 1e3, "roofline": roof(b_dec, dec_ms),
+                               "launches_per_call": 1},
+        "rmsnorm_gated": {"workload": f"{T} tokens x {M.o.shape[1]} V heads x {d}, bf16",
+                          "tokens_per_s": T / (norm_ms / 1e3), "roofline": roof(b_norm, norm_ms),
+                          "launches_per_call": 1},
+        "l2": "flushed (512 MiB write) before every timed launch",
+        "iters": iters,
+    }
+    return out, iters * 4
+
+
 class Clocks:
     """nvidia-smi sampled every 200 ms while the timed region runs."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -257,6 +335,10 @@ def run_ours(args):
                                 "algorithmic_bytes": db, "peak_source": peak_src},
                    "gpu_launches": args.decode_steps}
             del D
+        mixer, mixer_launches = None, 0
+        if not args.no_mixer:
+            mixer, mixer_launches = run_mixer(rank, dev, flush, stream, hbm, peak_src,
+                                              args.mixer_iters)
     kern_ms = [a.elapsed_time(b) for a, b in ev]
     ms = _max_over_ranks(sum(kern_ms) / len(kern_ms), ws, dev)
     tok_s = ws * T / (ms / 1e3)
@@ -299,9 +381,10 @@ def run_ours(args):
                               "frac_of_slower_roof": t_roof / (ms / 1e3)}},
         "e2e": e2e,
         "gpu_launches": sum(len(v_) for v_ in kernel_ms.values())
-                        + (args.decode_steps if dec else 0),
+                        + (args.decode_steps if dec else 0) + mixer_launches,
         "clocks": clocks.summary(),
         "decode": dec,
+        "mixer": mixer,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(P)
@@ -447,6 +530,9 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-mixer", action="store_true",
+                    help="skip the conv1d / gated-norm measurements")
+    ap.add_argument("--mixer-iters", type=int, default=20)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -219,6 +219,62 @@ int gdn_last_prefill_kernel_ms(float* ms, int32_t max_kernels);
 const char* gdn_last_prefill_kernel_name(int32_t i);
 
 /*
+ * The steps around the delta rule in the GDN token mixer ("Qwen3.5-MoE-35B-A3B
+ * architecture teardown", section 3.3 phase 2 and phase 4, section 3.4 for the
+ * conv cache; "Qwen3.5 observation notes", "Qwen3_5MoeGatedDeltaNet": a causal
+ * depthwise conv1d with SiLU over the concatenated q/k/v channels, and
+ * RMSNormGated on the mixer output).
+ *
+ * gdn_conv1d_silu -- causal depthwise convolution + SiLU over a packed batch:
+ *   y[t][c] = silu(bias[c] + sum_{i<K} weight[c][i] * x[t-(K-1)+i][c])
+ * where positions before a sequence's first token come from conv_state_in
+ * (zeros when it is NULL): the last tap multiplies the current token.
+ *   x               [T, conv_dim] io_dtype                               (in)
+ *   weight          [conv_dim, K] fp32 (16-byte aligned)                 (in)
+ *   bias            [conv_dim] fp32, or NULL (no bias)                   (in)
+ *   conv_state_in   [N, K-1, conv_dim] io_dtype, oldest position first,
+ *                   or NULL (zeros)                                      (in)
+ *   cu_seqlens      [N+1] int32, device                                  (in)
+ *   y               [T, conv_dim] io_dtype; must not be x               (out)
+ *   conv_state_out  [N, K-1, conv_dim] io_dtype, or NULL: the K-1 inputs
+ *                   ending at each sequence's last token (older cache
+ *                   entries where the sequence is shorter than K-1; an
+ *                   empty sequence keeps its cache). May be conv_state_in
+ *                   (updated in place).                                 (out)
+ * K = kernel_size in {2, 3, 4} (the pages' models use 4); conv_dim a multiple
+ * of 8. Arithmetic in fp32; y rounded once to io_dtype; the cache holds the
+ * inputs unchanged. Bad cu_seqlens contents set GDN_ERR_BAD_SEQLENS in the
+ * device status word.
+ */
+int gdn_conv1d_silu(const void* x, int32_t io_dtype, const float* weight, const float* bias,
+                    const void* conv_state_in, const int32_t* cu_seqlens, int32_t num_seqs,
+                    int64_t total_tokens, int32_t conv_dim, int32_t kernel_size, void* y,
+                    void* conv_state_out, void* stream);
+
+/*
+ * gdn_conv1d_silu_decode -- the same convolution for one token of each of N
+ * sequences, the cache slid by one position in place:
+ *   x [N, conv_dim] io_dtype (in); conv_state [N, K-1, conv_dim] io_dtype
+ *   (in/out); y [N, conv_dim] io_dtype (out); weight, bias as above.
+ * Equal to gdn_conv1d_silu on N one-token sequences with conv_state_in =
+ * conv_state_out = conv_state.
+ */
+int gdn_conv1d_silu_decode(const void* x, int32_t io_dtype, const float* weight,
+                           const float* bias, void* conv_state, int32_t num_seqs,
+                           int32_t conv_dim, int32_t kernel_size, void* y, void* stream);
+
+/*
+ * gdn_rmsnorm_gated -- the mixer's output norm, per row of d values:
+ *   y[r][:] = o[r][:] / sqrt(mean(o[r][:]^2) + eps) * weight[:] * silu(z[r][:])
+ *   o, z   [rows, d] io_dtype (rows = tokens x V heads)                  (in)
+ *   weight [d] fp32, 16-byte aligned, shared by all heads                (in)
+ *   y      [rows, d] io_dtype; may be o or z                            (out)
+ * d in {64, 128}; eps >= 0 (the pages' models use 1e-6). Arithmetic in fp32.
+ */
+int gdn_rmsnorm_gated(const void* o, const void* z, int32_t io_dtype, const float* weight,
+                      float eps, int64_t rows, int32_t d, void* y, void* stream);
+
+/*
  * Synchronise `stream`, then return and clear the device status word of the
  * current device (GDN_OK, GDN_ERR_BAD_SEQLENS or GDN_ERR_TIMEOUT), or
  * GDN_ERR_CUDA if the synchronisation itself failed.

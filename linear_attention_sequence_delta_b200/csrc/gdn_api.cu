@@ -223,6 +223,59 @@ int gdn_decode_step(const void* q, const void* k, const void* v, int32_t io_dtyp
                                    H_qk, H_v, d_k, scale, o, (cudaStream_t)stream));
 }
 
+int gdn_conv1d_silu(const void* x, int32_t io_dtype, const float* weight, const float* bias,
+                    const void* conv_state_in, const int32_t* cu_seqlens, int32_t num_seqs,
+                    int64_t total_tokens, int32_t conv_dim, int32_t kernel_size, void* y,
+                    void* conv_state_out, void* stream) {
+    if (io_dtype != GDN_BF16 && io_dtype != GDN_FP32) return GDN_ERR_INVALID_ARG;
+    if (num_seqs < 0 || total_tokens < 0 || conv_dim <= 0) return GDN_ERR_INVALID_ARG;
+    if (kernel_size < 2 || kernel_size > 4 || conv_dim % 8 != 0) return GDN_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return total_tokens == 0 ? GDN_OK : GDN_ERR_INVALID_ARG;
+    if (total_tokens == 0 && !conv_state_out) return GDN_OK;
+    if (!x || !weight || !cu_seqlens || (total_tokens > 0 && !y)) return GDN_ERR_INVALID_ARG;
+    const void* ptrs16[] = {x, y, weight, conv_state_in, conv_state_out};
+    for (const void* p : ptrs16)
+        if (p && !aligned(p, 16)) return GDN_ERR_INVALID_ARG;
+    if (bias && !aligned(bias, 4)) return GDN_ERR_INVALID_ARG;
+    if (!aligned(cu_seqlens, 4)) return GDN_ERR_INVALID_ARG;
+    if (x == y) return GDN_ERR_INVALID_ARG;  // the window reads neighbouring tokens
+    return to_status(launch_conv1d_silu(x, io_dtype, weight, bias, conv_state_in, cu_seqlens,
+                                        num_seqs, total_tokens, conv_dim, kernel_size, y,
+                                        conv_state_out, device_status_ptr(),
+                                        (cudaStream_t)stream));
+}
+
+int gdn_conv1d_silu_decode(const void* x, int32_t io_dtype, const float* weight,
+                           const float* bias, void* conv_state, int32_t num_seqs,
+                           int32_t conv_dim, int32_t kernel_size, void* y, void* stream) {
+    if (io_dtype != GDN_BF16 && io_dtype != GDN_FP32) return GDN_ERR_INVALID_ARG;
+    if (num_seqs < 0 || conv_dim <= 0) return GDN_ERR_INVALID_ARG;
+    if (kernel_size < 2 || kernel_size > 4 || conv_dim % 8 != 0) return GDN_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return GDN_OK;
+    if (!x || !weight || !conv_state || !y) return GDN_ERR_INVALID_ARG;
+    const void* ptrs16[] = {x, y, weight, conv_state};
+    for (const void* p : ptrs16)
+        if (!aligned(p, 16)) return GDN_ERR_INVALID_ARG;
+    if (bias && !aligned(bias, 4)) return GDN_ERR_INVALID_ARG;
+    return to_status(launch_conv1d_silu_decode(x, io_dtype, weight, bias, conv_state, num_seqs,
+                                               conv_dim, kernel_size, y,
+                                               (cudaStream_t)stream));
+}
+
+int gdn_rmsnorm_gated(const void* o, const void* z, int32_t io_dtype, const float* weight,
+                      float eps, int64_t rows, int32_t d, void* y, void* stream) {
+    if (io_dtype != GDN_BF16 && io_dtype != GDN_FP32) return GDN_ERR_INVALID_ARG;
+    if (rows < 0 || !(eps >= 0.f) || !isfinite(eps)) return GDN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return GDN_ERR_UNSUPPORTED;
+    if (rows == 0) return GDN_OK;
+    if (!o || !z || !weight || !y) return GDN_ERR_INVALID_ARG;
+    const void* ptrs16[] = {o, z, weight, y};
+    for (const void* p : ptrs16)
+        if (!aligned(p, 16)) return GDN_ERR_INVALID_ARG;
+    return to_status(
+        launch_rmsnorm_gated(o, z, io_dtype, weight, eps, rows, d, y, (cudaStream_t)stream));
+}
+
 int gdn_set_prefill_impl(int32_t impl) {
     if (impl != GDN_IMPL_AUTO && impl != GDN_IMPL_CUDA_CORE && impl != GDN_IMPL_TENSOR_CORE &&
         impl != GDN_IMPL_TENSOR_CORE_SPLIT)

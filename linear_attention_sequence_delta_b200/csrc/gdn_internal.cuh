@@ -105,4 +105,15 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
                               int32_t H_qk, int32_t H_v, float scale, void* o, float* S_final,
                               void* workspace, bool fused, int* status, cudaStream_t s);
 
+// Steps around the delta rule (gdn_mixer.cu): causal depthwise conv1d + SiLU with
+// the per-sequence conv cache, its single-token decode form, and the gated RMSNorm.
+cudaError_t launch_conv1d_silu(const void* x, int io_dtype, const float* w, const float* bias,
+                               const void* state_in, const int32_t* cu, int N, int64_t T, int C,
+                               int K, void* y, void* state_out, int* status, cudaStream_t s);
+cudaError_t launch_conv1d_silu_decode(const void* x, int io_dtype, const float* w,
+                                      const float* bias, void* state, int N, int C, int K,
+                                      void* y, cudaStream_t s);
+cudaError_t launch_rmsnorm_gated(const void* o, const void* z, int io_dtype, const float* w,
+                                 float eps, int64_t rows, int d, void* y, cudaStream_t s);
+
 }  // namespace gdn

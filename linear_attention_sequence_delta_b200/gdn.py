@@ -6,10 +6,14 @@ passes raw pointers and the current CUDA stream across the C ABI declared in
 include/gdn.h. There is no fallback: if the library is missing or cannot be
 loaded, every call raises.
 
-The three calls keep the C names:
+The calls keep the C names:
   gdn_gates(a, b, A_log, dt_bias, cu_seqlens, ...)
   gdn_prefill(q, k, v, a, b, A_log, dt_bias, cu_seqlens, initial_state=None, ...)
   gdn_decode_step(q, k, v, a, b, A_log, dt_bias, state, ...)
+and the steps around the delta rule in the mixer:
+  gdn_conv1d_silu(x, weight, bias, cu_seqlens, conv_state_in=None, ...)
+  gdn_conv1d_silu_decode(x, weight, bias, conv_state, ...)
+  gdn_rmsnorm_gated(o, z, weight, eps=1e-6, ...)
 """
 from __future__ import annotations
 
@@ -30,7 +34,8 @@ _STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "
 EXPORTS = ["gdn_status_string", "gdn_version", "gdn_prefill_workspace_size", "gdn_gates",
            "gdn_prefill", "gdn_decode_step", "gdn_sync_status", "gdn_prefill_noalloc",
            "gdn_set_prefill_impl", "gdn_set_kernel_timing", "gdn_last_prefill_kernel_ms",
-           "gdn_last_prefill_kernel_name"]
+           "gdn_last_prefill_kernel_name", "gdn_conv1d_silu", "gdn_conv1d_silu_decode",
+           "gdn_rmsnorm_gated"]
 GDN_IMPL_AUTO, GDN_IMPL_CUDA_CORE, GDN_IMPL_TENSOR_CORE, GDN_IMPL_TENSOR_CORE_SPLIT = 0, 1, 2, 3
 
 
@@ -77,6 +82,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gdn_last_prefill_kernel_ms.argtypes = [P, i32]
     lib.gdn_last_prefill_kernel_name.restype = ctypes.c_char_p
     lib.gdn_last_prefill_kernel_name.argtypes = [i32]
+    lib.gdn_conv1d_silu.restype = ctypes.c_int
+    lib.gdn_conv1d_silu.argtypes = [P, i32, P, P, P, P, i32, i64, i32, i32, P, P, P]
+    lib.gdn_conv1d_silu_decode.restype = ctypes.c_int
+    lib.gdn_conv1d_silu_decode.argtypes = [P, i32, P, P, P, i32, i32, i32, P, P]
+    lib.gdn_rmsnorm_gated.restype = ctypes.c_int
+    lib.gdn_rmsnorm_gated.argtypes = [P, P, i32, P, f32, i64, i32, P, P]
     _lib = lib
     return lib
 
@@ -212,3 +223,59 @@ def last_prefill_kernel_times() -> list:
     if n < 0:
         raise GDNError(-n, "gdn_last_prefill_kernel_ms")
     return [(lib.gdn_last_prefill_kernel_name(i).decode(), float(ms[i])) for i in range(min(n, 4))]
+
+
+def gdn_conv1d_silu(x, weight, bias, cu_seqlens, conv_state_in=None, *, want_state=True,
+                    out=None, conv_state_out=None):
+    """Causal depthwise conv1d + SiLU over a packed batch. Returns (y, conv_state_out or None).
+
+    x [T, C] (bf16 or fp32); weight [C, K] fp32; bias [C] fp32 or None; cu_seqlens int32
+    [N+1]; conv_state_in [N, K-1, C] (x's dtype) or None (zeros). conv_state_out may be
+    conv_state_in (updated in place).
+    """
+    lib = load_library()
+    _need_cuda(x, weight, bias, cu_seqlens, conv_state_in, out, conv_state_out)
+    io = _io_dtype(x)
+    T, C = x.shape
+    K = weight.shape[1]
+    N = cu_seqlens.numel() - 1
+    y = out if out is not None else torch.empty_like(x)
+    if want_state and conv_state_out is None:
+        conv_state_out = torch.empty((N, K - 1, C), device=x.device, dtype=x.dtype)
+    if not want_state:
+        conv_state_out = None
+    st = lib.gdn_conv1d_silu(_ptr(x), io, _ptr(weight), _ptr(bias), _ptr(conv_state_in),
+                             _ptr(cu_seqlens), N, T, C, K, _ptr(y), _ptr(conv_state_out),
+                             _stream(x.device))
+    _check(st, "gdn_conv1d_silu")
+    return y, conv_state_out
+
+
+def gdn_conv1d_silu_decode(x, weight, bias, conv_state, *, out=None):
+    """One token per sequence: x [N, C]; conv_state [N, K-1, C] slides in place. Returns y."""
+    lib = load_library()
+    _need_cuda(x, weight, bias, conv_state, out)
+    io = _io_dtype(x)
+    N, C = x.shape
+    K = weight.shape[1]
+    y = out if out is not None else torch.empty_like(x)
+    st = lib.gdn_conv1d_silu_decode(_ptr(x), io, _ptr(weight), _ptr(bias), _ptr(conv_state), N,
+                                    C, K, _ptr(y), _stream(x.device))
+    _check(st, "gdn_conv1d_silu_decode")
+    return y
+
+
+def gdn_rmsnorm_gated(o, z, weight, eps: float = 1e-6, *, out=None):
+    """o / rms(o) * weight * silu(z) over the last dimension d (64 or 128); o and z of the
+    same shape and dtype, weight [d] fp32. Returns y (may be passed as o or z via `out`)."""
+    lib = load_library()
+    _need_cuda(o, z, weight, out)
+    if o.shape != z.shape or o.dtype != z.dtype:
+        raise ValueError("o and z must share shape and dtype")
+    io = _io_dtype(o)
+    d = o.shape[-1]
+    y = out if out is not None else torch.empty_like(o)
+    st = lib.gdn_rmsnorm_gated(_ptr(o), _ptr(z), io, _ptr(weight), float(eps), o.numel() // d, d,
+                               _ptr(y), _stream(o.device))
+    _check(st, "gdn_rmsnorm_gated")
+    return y

@@ -12,6 +12,15 @@ made on, drawn in this fixed order):
   3. a, b  [T, H_v] ~ N(0, 1), fp32;
   4. A_log [H_v] ~ U(0, ln 16), dt_bias [H_v] ~ U(-1, 1), fp32;
   5. initial state [N, H_v, d_v, d_k] ~ N(0, state_std^2), fp32 (when asked for).
+For the steps around the delta rule (make_mixer_inputs, drawn in this order):
+  1. sequence lengths as above;
+  2. x [T, C] ~ N(0, 1) (C = conv_dim = 2 H_qk d_k + H_v d_v, the concatenated
+     q/k/v channels), rounded to the I/O type;
+  3. conv weight [C, K] ~ U(-1/sqrt(K), 1/sqrt(K)), conv bias [C] ~ N(0, 0.1^2)
+     (used only where a test asks for a bias), fp32;
+  4. conv cache [N, K-1, C] ~ N(0, 1), rounded to the I/O type;
+  5. o, z [T, H_v, d_v] ~ N(0, 1), rounded to the I/O type; norm weight
+     [d_v] ~ U(0.5, 1.5), fp32.
 The shapes follow the Qwen3.5 GDN layers: 16 QK heads, 32 (35B-A3B) or 64
 (397B-A17B) V heads, head dim 128. The CPU and CUDA generators produce
 different streams; a given test always draws on one device.
@@ -124,6 +133,53 @@ def make_decode_inputs(*, steps: int, num_seqs: int = 256, H_qk: int = 16, H_v: 
     dt_bias = torch.rand((H_v,), generator=g, device=device, dtype=f32) * 2.0 - 1.0
     state = torch.randn((N, H_v, d_v, d_k), generator=g, device=device, dtype=f32) * state_std
     return DecodeInputs(q, k, v, a, b, A_log, dt_bias, state)
+
+
+@dataclass
+class MixerInputs:
+    x: torch.Tensor            # [T, C]
+    conv_weight: torch.Tensor  # [C, K] fp32
+    conv_bias: torch.Tensor    # [C] fp32
+    conv_state: torch.Tensor   # [N, K-1, C]
+    o: torch.Tensor            # [T, H_v, d_v]
+    z: torch.Tensor            # [T, H_v, d_v]
+    norm_weight: torch.Tensor  # [d_v] fp32
+    cu_seqlens: torch.Tensor   # int32 [N+1]
+
+    def to(self, device) -> "MixerInputs":
+        return MixerInputs(*(getattr(self, f).to(device) for f in self.__dataclass_fields__))
+
+
+def make_mixer_inputs(lengths=None, *, num_seqs: int = 1, seq_len: int = 256,
+                      len_lo: int = 128, len_hi: int = 8192, H_qk: int = 16, H_v: int = 32,
+                      d_k: int = 128, d_v: int = 128, kernel_size: int = 4,
+                      io_dtype: torch.dtype = torch.bfloat16, seed: int = 0,
+                      device="cpu") -> MixerInputs:
+    """Inputs of the convolution in front of the delta rule and of the gated norm after it."""
+    g = _gen(device, seed)
+    if isinstance(lengths, str) and lengths == "random":
+        lens = torch.randint(len_lo, len_hi + 1, (num_seqs,), generator=g, device=device)
+        lens = [int(x) for x in lens.cpu()]
+    elif lengths is None:
+        lens = [seq_len] * num_seqs
+    else:
+        lens = [int(x) for x in lengths]
+    cu = [0]
+    for n in lens:
+        cu.append(cu[-1] + n)
+    T, N, K = cu[-1], len(lens), kernel_size
+    C = 2 * H_qk * d_k + H_v * d_v
+    f32 = torch.float32
+    x = torch.randn((T, C), generator=g, device=device, dtype=f32).to(io_dtype)
+    bound = 1.0 / math.sqrt(K)
+    w = (torch.rand((C, K), generator=g, device=device, dtype=f32) * 2.0 - 1.0) * bound
+    bias = torch.randn((C,), generator=g, device=device, dtype=f32) * 0.1
+    st = torch.randn((N, K - 1, C), generator=g, device=device, dtype=f32).to(io_dtype)
+    o = torch.randn((T, H_v, d_v), generator=g, device=device, dtype=f32).to(io_dtype)
+    z = torch.randn((T, H_v, d_v), generator=g, device=device, dtype=f32).to(io_dtype)
+    nw = torch.rand((d_v,), generator=g, device=device, dtype=f32) + 0.5
+    cu_t = torch.tensor(cu, dtype=torch.int32, device=device)
+    return MixerInputs(x, w, bias, st, o, z, nw, cu_t)
 
 
 # The five workloads, by name. Sizes are those of the Qwen3.5 GDN layers.

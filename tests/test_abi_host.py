@@ -24,7 +24,7 @@ def lib():
 def _declared():
     src = open(os.path.join(ROOT, "include", "gdn.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(gdn_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(gdn_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_exports_every_declared_symbol(lib):
@@ -147,6 +147,65 @@ def test_gates_rejects(lib):
     assert g(v(F + 2), v(F), v(F), v(F), v(F), 1, 4, 4, v(F), None, None, None) == 1
     # nothing asked for: success without a launch
     assert g(v(F), v(F), v(F), v(F), v(F), 1, 4, 4, None, None, None, None) == 0
+
+
+def _call_conv(lib, **over):
+    a = dict(x=F, io=gdn.GDN_BF16, w=F + 0x1000, bias=None, sin=None, cu=F + 0x2000, N=2, T=64,
+             C=256, K=4, y=F + 0x8000, sout=None, stream=None)
+    a.update(over)
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.gdn_conv1d_silu(v(a["x"]), a["io"], v(a["w"]), v(a["bias"]), v(a["sin"]),
+                               v(a["cu"]), a["N"], a["T"], a["C"], a["K"], v(a["y"]),
+                               v(a["sout"]), v(a["stream"]))
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(io=3), 1), (dict(N=-1), 1), (dict(T=-1), 1), (dict(C=0), 1), (dict(N=0, T=8), 1),
+    (dict(K=1), 2), (dict(K=5), 2), (dict(C=260), 2),
+    (dict(x=None), 1), (dict(w=None), 1), (dict(cu=None), 1), (dict(y=None), 1),
+    (dict(x=F + 8), 1), (dict(y=F + 4), 1), (dict(w=F + 4), 1), (dict(sin=F + 2), 1),
+    (dict(sout=F + 8), 1), (dict(bias=F + 2), 1), (dict(cu=F + 2), 1),
+    (dict(y=F), 1),                     # in place is refused: the window reads neighbours
+])
+def test_conv1d_rejects(lib, over, code):
+    assert _call_conv(lib, **over) == code
+
+
+def test_conv1d_noops(lib):
+    assert _call_conv(lib, N=0, T=0, x=None, y=None) == 0
+    assert _call_conv(lib, T=0, y=None) == 0          # no tokens, no cache asked for
+
+
+def test_conv1d_decode_rejects(lib):
+    v = ctypes.c_void_p
+    d = lib.gdn_conv1d_silu_decode
+    ok = lambda **o: dict(dict(x=F, io=0, w=F + 0x1000, b=None, st=F + 0x2000, N=4, C=64, K=4,
+                               y=F + 0x3000), **o)
+    call = lambda a: d(v(a["x"]) if a["x"] else None, a["io"], v(a["w"]) if a["w"] else None,
+                       v(a["b"]) if a["b"] else None, v(a["st"]) if a["st"] else None, a["N"],
+                       a["C"], a["K"], v(a["y"]) if a["y"] else None, None)
+    assert call(ok(io=2)) == 1
+    assert call(ok(N=-1)) == 1
+    assert call(ok(K=6)) == 2
+    assert call(ok(C=12)) == 2
+    assert call(ok(st=None)) == 1
+    assert call(ok(st=F + 0x2004)) == 1
+    assert call(ok(b=F + 1)) == 1
+    assert call(ok(N=0)) == 0
+
+
+def test_rmsnorm_gated_rejects(lib):
+    v = ctypes.c_void_p
+    r = lib.gdn_rmsnorm_gated
+    assert r(v(F), v(F + 0x100), 5, v(F + 0x200), 1e-6, 4, 128, v(F + 0x300), None) == 1
+    assert r(v(F), v(F + 0x100), 0, v(F + 0x200), 1e-6, -1, 128, v(F + 0x300), None) == 1
+    assert r(v(F), v(F + 0x100), 0, v(F + 0x200), -1.0, 4, 128, v(F + 0x300), None) == 1
+    assert r(v(F), v(F + 0x100), 0, v(F + 0x200), math.nan, 4, 128, v(F + 0x300), None) == 1
+    assert r(v(F), v(F + 0x100), 0, v(F + 0x200), 1e-6, 4, 96, v(F + 0x300), None) == 2
+    assert r(None, v(F + 0x100), 0, v(F + 0x200), 1e-6, 4, 128, v(F + 0x300), None) == 1
+    assert r(v(F), v(F + 0x100), 0, v(F + 0x204), 1e-6, 4, 128, v(F + 0x300), None) == 1
+    assert r(v(F + 8), v(F + 0x100), 0, v(F + 0x200), 1e-6, 4, 128, v(F + 0x300), None) == 1
+    assert r(None, None, 0, None, 1e-6, 0, 128, None, None) == 0
 
 
 def test_binding_fails_loudly_without_library(tmp_path):
