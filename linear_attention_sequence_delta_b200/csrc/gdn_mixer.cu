@@ -13,8 +13,7 @@ namespace gdn {
 namespace {
 
 constexpr int kVec = 8;        // channels per thread (one 16-byte bf16 vector)
-constexpr int kConvTile = 16;  // tokens per thread in the prefill convolution
-constexpr int kConvBatch = 8;  // tokens loaded ahead within a tile
+constexpr int kDecSeqs = 2;    // sequences per thread in the decode convolution
 constexpr int kMaxK = 4;
 
 template <typename IO>
@@ -66,7 +65,18 @@ struct Vec8<float> {
     }
 };
 
-__device__ __forceinline__ float silu_f32(float x) { return x / (1.f + __expf(-x)); }
+// x * sigmoid(x) with the fast exponential and division: two SFU operations per value
+// (an IEEE division costs several times more and made the convolution compute-bound).
+// Relative error a few fp32 ulp; for x < -88 the exponential overflows to inf and the
+// result is 0, where the exact value is below 1e-36 in magnitude.
+__device__ __forceinline__ float silu_f32(float x) { return __fdividef(x, 1.f + __expf(-x)); }
+
+// Tokens per thread in the prefill convolution: all of a tile's inputs are loaded
+// before any is used (16 x 16 bytes for bf16, 8 x 32 bytes for fp32).
+template <typename IO>
+struct ConvTile {
+    static constexpr int value = sizeof(IO) == 2 ? 16 : 8;
+};
 
 // sequence n with cu[n] <= t < cu[n + 1] (the last such n for empty sequences)
 __device__ __forceinline__ int find_seq(const int32_t* cu, int N, int64_t t) {
@@ -98,12 +108,12 @@ __device__ __forceinline__ void load_taps(const float* __restrict__ w,
     for (int e = 0; e < kVec; ++e) bs[e] = bias ? __ldg(bias + c0 + e) : 0.f;
 }
 
-// y for kConvTile consecutive tokens x kVec channels per thread; consecutive threads
-// take consecutive channel vectors of the same token tile. The window of the last
-// K-1 inputs is carried in registers; at a sequence's start it comes from the cache
-// (or zeros). Tiles inside one sequence load kConvBatch tokens ahead.
+// y for kTile consecutive tokens x kVec channels per thread; consecutive threads take
+// consecutive channel vectors of the same token tile. The window of the last K-1
+// inputs is carried in registers; at a sequence's start it comes from the cache (or
+// zeros). A tile inside one sequence loads all its inputs up front.
 template <typename IO, int K>
-__global__ void __launch_bounds__(256) conv1d_silu_kernel(
+__global__ void __launch_bounds__(128) conv1d_silu_kernel(
     const IO* __restrict__ x, const float* __restrict__ w, const float* __restrict__ bias,
     const IO* __restrict__ state_in, const int32_t* __restrict__ cu, int N, int64_t T, int C,
     IO* __restrict__ y, int* status) {
@@ -111,8 +121,23 @@ __global__ void __launch_bounds__(256) conv1d_silu_kernel(
     const int64_t gidx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t tile = gidx / nv;
     const int c0 = (int)(gidx - tile * nv) * kVec;
-    const int64_t t0 = tile * kConvTile;
+    constexpr int kTile = ConvTile<IO>::value;
+    const int64_t t0 = tile * kTile;
     if (t0 >= T) return;
+    // Let the cache kernel that follows start its loads (it waits before storing).
+    asm volatile("griddepcontrol.launch_dependents;");
+    // Loads that need no sequence bounds go first, so that they overlap the lookup in
+    // cu_seqlens: the tile's tokens (index clamped to T-1) and the K-1 positions before
+    // it (clamped to 0).
+    typename Vec8<IO>::Raw xb[kTile], wb[K - 1];
+#pragma unroll
+    for (int i = 0; i < kTile; ++i)
+        xb[i] = Vec8<IO>::load_raw(x + (size_t)(t0 + i < T ? t0 + i : T - 1) * C + c0);
+#pragma unroll
+    for (int j = 0; j < K - 1; ++j) {
+        const int64_t p = t0 - (K - 1) + j;
+        wb[j] = Vec8<IO>::load_raw(x + (size_t)(p > 0 ? p : 0) * C + c0);
+    }
     float wt[K][kVec], bs[kVec];
     load_taps<K>(w, bias, c0, wt, bs);
     int n = find_seq(cu, N, t0);
@@ -155,24 +180,30 @@ __global__ void __launch_bounds__(256) conv1d_silu_kernel(
 #pragma unroll
         for (int e = 0; e < kVec; ++e) win[K - 2][e] = xt[e];
     };
-    fill_window(t0);
-    if (t0 + kConvTile <= s1) {  // the whole tile in one sequence
-#pragma unroll 1
-        for (int b = 0; b < kConvTile; b += kConvBatch) {
-            typename Vec8<IO>::Raw xb[kConvBatch];
+    if (t0 + kTile <= s1) {  // the whole tile in one sequence
 #pragma unroll
-            for (int i = 0; i < kConvBatch; ++i)
-                xb[i] = Vec8<IO>::load_raw(x + (size_t)(t0 + b + i) * C + c0);
+        for (int j = 0; j < K - 1; ++j) {
+            const int64_t p = t0 - (K - 1) + j;
+            if (p >= s0) {
+                Vec8<IO>::unpack(wb[j], win[j]);
+            } else if (state_in) {
+                Vec8<IO>::load(state_in + ((size_t)n * (K - 1) + (K - 1) + (p - s0)) * C + c0,
+                               win[j]);
+            } else {
 #pragma unroll
-            for (int i = 0; i < kConvBatch; ++i) {
-                float xt[kVec];
-                Vec8<IO>::unpack(xb[i], xt);
-                step(xt, t0 + b + i);
+                for (int e = 0; e < kVec; ++e) win[j][e] = 0.f;
             }
+        }
+#pragma unroll
+        for (int i = 0; i < kTile; ++i) {
+            float xt[kVec];
+            Vec8<IO>::unpack(xb[i], xt);
+            step(xt, t0 + i);
         }
         return;
     }
-    const int64_t t_end = t0 + kConvTile < T ? t0 + kConvTile : T;
+    fill_window(t0);
+    const int64_t t_end = t0 + kTile < T ? t0 + kTile : T;
     for (int64_t t = t0; t < t_end; ++t) {
         if (t >= s1) {  // the next non-empty sequence starts here
             while (t >= s1) {
@@ -229,42 +260,61 @@ __global__ void __launch_bounds__(256) conv_state_kernel(const IO* __restrict__ 
             for (int e = 0; e < kVec; ++e) v[j][e] = 0.f;
         }
     }
+    // Launched as a programmatic dependent of the convolution: everything above only
+    // reads; the stores wait for the convolution grid (which may read state_in == state_out)
+    // to finish. Without that launch attribute the wait returns at once.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 #pragma unroll
     for (int j = 0; j < K - 1; ++j)
         Vec8<IO>::store(state_out + ((size_t)n * (K - 1) + j) * C + c0, v[j]);
 }
 
 // One token per sequence: y = silu(bias + w . [cache, x]); the cache slides by one.
+// A thread takes one channel vector of kDecSeqs sequences (the taps loaded once) and
+// loads all their inputs before using any.
 template <typename IO, int K>
-__global__ void __launch_bounds__(256) conv_decode_kernel(const IO* __restrict__ x,
+__global__ void __launch_bounds__(128) conv_decode_kernel(const IO* __restrict__ x,
                                                           const float* __restrict__ w,
                                                           const float* __restrict__ bias,
                                                           IO* state, int N, int C,
                                                           IO* __restrict__ y) {
     const int nv = C / kVec;
     const int64_t gidx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t n = gidx / nv;
-    const int c0 = (int)(gidx - n * nv) * kVec;
-    if (n >= N) return;
+    const int64_t grp = gidx / nv;
+    const int c0 = (int)(gidx - grp * nv) * kVec;
+    const int64_t n0 = grp * kDecSeqs;
+    if (n0 >= N) return;
+    typename Vec8<IO>::Raw raw[kDecSeqs][K];
+#pragma unroll
+    for (int q = 0; q < kDecSeqs; ++q) {
+        const int64_t n = n0 + q < N ? n0 + q : n0;  // a missing last sequence re-reads n0
+#pragma unroll
+        for (int j = 0; j < K - 1; ++j)
+            raw[q][j] = Vec8<IO>::load_raw(state + ((size_t)n * (K - 1) + j) * C + c0);
+        raw[q][K - 1] = Vec8<IO>::load_raw(x + (size_t)n * C + c0);
+    }
     float wt[K][kVec], bs[kVec];
     load_taps<K>(w, bias, c0, wt, bs);
-    float win[kMaxK][kVec];
 #pragma unroll
-    for (int j = 0; j < K - 1; ++j)
-        Vec8<IO>::load(state + ((size_t)n * (K - 1) + j) * C + c0, win[j]);
-    Vec8<IO>::load(x + (size_t)n * C + c0, win[K - 1]);
-    float out[kVec];
+    for (int q = 0; q < kDecSeqs; ++q) {
+        const int64_t n = n0 + q;
+        if (n >= N) break;
+        float out[kVec];
+        float win[K][kVec];
 #pragma unroll
-    for (int e = 0; e < kVec; ++e) {
-        float acc = bs[e];
+        for (int j = 0; j < K; ++j) Vec8<IO>::unpack(raw[q][j], win[j]);
 #pragma unroll
-        for (int i = 0; i < K; ++i) acc = fmaf(wt[i][e], win[i][e], acc);
-        out[e] = silu_f32(acc);
+        for (int e = 0; e < kVec; ++e) {
+            float acc = bs[e];
+#pragma unroll
+            for (int i = 0; i < K; ++i) acc = fmaf(wt[i][e], win[i][e], acc);
+            out[e] = silu_f32(acc);
+        }
+        Vec8<IO>::store(y + (size_t)n * C + c0, out);
+#pragma unroll
+        for (int j = 0; j < K - 1; ++j)
+            Vec8<IO>::store(state + ((size_t)n * (K - 1) + j) * C + c0, win[j + 1]);
     }
-    Vec8<IO>::store(y + (size_t)n * C + c0, out);
-#pragma unroll
-    for (int j = 0; j < K - 1; ++j)
-        Vec8<IO>::store(state + ((size_t)n * (K - 1) + j) * C + c0, win[j + 1]);
 }
 
 // Rows of D (64 or 128) values, D/8 lanes per row, each lane 8 consecutive values.
@@ -309,10 +359,11 @@ template <typename IO, int K>
 cudaError_t conv_launch(const void* x, const float* w, const float* bias, const void* state_in,
                         const int32_t* cu, int N, int64_t T, int C, void* y, void* state_out,
                         int* status, cudaStream_t s) {
-    const int threads = 256;
     const int64_t nv = C / kVec;
     if (T > 0) {
-        const int64_t tiles = (T + kConvTile - 1) / kConvTile;
+        const int threads = 128;
+        constexpr int kTile = ConvTile<IO>::value;
+        const int64_t tiles = (T + kTile - 1) / kTile;
         conv1d_silu_kernel<IO, K><<<blocks_for(tiles * nv, threads), threads, 0, s>>>(
             static_cast<const IO*>(x), w, bias, static_cast<const IO*>(state_in), cu, N, T, C,
             static_cast<IO*>(y), status);
@@ -320,10 +371,19 @@ cudaError_t conv_launch(const void* x, const float* w, const float* bias, const 
         if (e != cudaSuccess) return e;
     }
     if (state_out && N > 0) {
-        conv_state_kernel<IO, K><<<blocks_for((int64_t)N * nv, threads), threads, 0, s>>>(
-            static_cast<const IO*>(x), static_cast<const IO*>(state_in), cu, N, T, C,
-            static_cast<IO*>(state_out));
-        return cudaGetLastError();
+        // programmatic dependent launch: its loads overlap the convolution's tail
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = T > 0 ? 1 : 0;
+        cfg.gridDim = dim3(blocks_for((int64_t)N * nv, 256));
+        cfg.blockDim = dim3(256);
+        cfg.stream = s;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, conv_state_kernel<IO, K>, static_cast<const IO*>(x),
+                                  static_cast<const IO*>(state_in), cu, N, T, C,
+                                  static_cast<IO*>(state_out));
     }
     return cudaSuccess;
 }
@@ -331,8 +391,9 @@ cudaError_t conv_launch(const void* x, const float* w, const float* bias, const 
 template <typename IO, int K>
 cudaError_t conv_decode_launch(const void* x, const float* w, const float* bias, void* state,
                                int N, int C, void* y, cudaStream_t s) {
-    const int threads = 256;
-    conv_decode_kernel<IO, K><<<blocks_for((int64_t)N * (C / kVec), threads), threads, 0, s>>>(
+    const int threads = 128;
+    const int64_t groups = (N + kDecSeqs - 1) / kDecSeqs;
+    conv_decode_kernel<IO, K><<<blocks_for(groups * (C / kVec), threads), threads, 0, s>>>(
         static_cast<const IO*>(x), w, bias, static_cast<IO*>(state), N, C, static_cast<IO*>(y));
     return cudaGetLastError();
 }
