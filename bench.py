@@ -185,6 +185,42 @@ def run_mixer(rank, dev, flush, stream, hbm, peak_src, iters):
     return out, iters * 4
 
 
+def run_decode_variants(rank, dev, flush, stream, hbm, peak_src, iters):
+    """gdn_decode_slots on the 397B-A17B decode shape (256 sequences, 64 V heads, d=128):
+    L = 1 with the states scattered over a pool of 512 slots (continuous batching), and
+    L = 2 (a token plus one MTP draft) with the per-token states written out."""
+    from linear_attention_sequence_delta_b200 import gdn
+    from linear_attention_sequence_delta_b200.inputs import make_decode_inputs
+    N, pool_n, H_qk, H_v, d = 256, 512, 16, 64, 128
+    D = make_decode_inputs(steps=2, num_seqs=pool_n, H_qk=H_qk, H_v=H_v, d_k=d, d_v=d,
+                           seed=rank, device=dev)
+    g = torch.Generator(device="cpu").manual_seed(rank)
+    slots = torch.randperm(pool_n, generator=g)[:N].to(torch.int32).to(dev)
+    tok = lambda x, L: x[:L, :N].transpose(0, 1).contiguous()
+    out = {}
+    for L, inter in ((1, False), (2, True)):
+        q, k, v, a, b = (tok(x, L) for x in (D.q, D.k, D.v, D.a, D.b))
+        o = torch.empty((N, L, H_v, d), device=dev, dtype=q.dtype)
+        I = torch.empty((N, L, H_v, d, d), device=dev, dtype=torch.float32) if inter else None
+        ms = _time_op(lambda: gdn.gdn_decode_slots(q, k, v, a, b, D.A_log, D.dt_bias, D.state,
+                                                   slots, out=o, intermediate_states=I),
+                      iters, flush, stream)
+        byts = (2 + (L if inter else 0)) * N * H_v * d * d * 4 \
+            + N * L * (2 * H_qk * d + 2 * H_v * d) * 2 + 2 * N * L * H_v * 4 + N * 4
+        gbs = byts / (ms / 1e3) / 1e9
+        out[f"L{L}" + ("_intermediates" if inter else "")] = {
+            "workload": f"{N} seqs x {L} token(s), states in a pool of {pool_n} slots, "
+                        f"H_qk={H_qk}, H_v={H_v}, d={d}, bf16"
+                        + (", state after every token written" if inter else ""),
+            "us_per_call": ms * 1e3, "tokens_per_s": N * L / (ms / 1e3),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                         "frac": gbs / hbm, "algorithmic_bytes": byts, "kernel_ms": ms,
+                         "peak_source": peak_src}}
+    out["l2"] = "flushed (512 MiB write) before every timed launch"
+    out["iters"] = iters
+    return out, 2 * iters
+
+
 class Clocks:
     """nvidia-smi sampled every 200 ms while the timed region runs."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -339,6 +375,10 @@ def run_ours(args):
         if not args.no_mixer:
             mixer, mixer_launches = run_mixer(rank, dev, flush, stream, hbm, peak_src,
                                               args.mixer_iters)
+        dvar, dvar_launches = None, 0
+        if not args.no_decode:
+            dvar, dvar_launches = run_decode_variants(rank, dev, flush, stream, hbm, peak_src,
+                                                      args.mixer_iters)
     kern_ms = [a.elapsed_time(b) for a, b in ev]
     ms = _max_over_ranks(sum(kern_ms) / len(kern_ms), ws, dev)
     tok_s = ws * T / (ms / 1e3)
@@ -381,9 +421,11 @@ def run_ours(args):
                               "frac_of_slower_roof": t_roof / (ms / 1e3)}},
         "e2e": e2e,
         "gpu_launches": sum(len(v_) for v_ in kernel_ms.values())
-                        + (args.decode_steps if dec else 0) + mixer_launches,
+                        + (args.decode_steps if dec else 0) + mixer_launches
+                        + dvar_launches,
         "clocks": clocks.summary(),
         "decode": dec,
+        "decode_slots": dvar,
         "mixer": mixer,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:

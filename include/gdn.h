@@ -58,7 +58,8 @@ typedef enum {
     GDN_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required        */
     GDN_ERR_CUDA = 4,        /* a CUDA runtime call failed (launch, attribute)    */
     GDN_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out                */
-    GDN_ERR_BAD_SEQLENS = 6  /* cu_seqlens not non-decreasing / out of range      */
+    GDN_ERR_BAD_SEQLENS = 6, /* cu_seqlens not non-decreasing / out of range      */
+    GDN_ERR_BAD_SLOT = 7     /* a state / cache slot index >= the pool size       */
 } gdn_status;
 
 typedef enum { GDN_BF16 = 0, GDN_FP32 = 1 } gdn_dtype;
@@ -165,6 +166,35 @@ int gdn_decode_step(const void* q, const void* k, const void* v, int32_t io_dtyp
                     const float* a, const float* b, const float* A_log, const float* dt_bias,
                     float* state, int32_t num_seqs, int32_t H_qk, int32_t H_v, int32_t d_k,
                     int32_t d_v, float scale, void* o, void* stream);
+
+/*
+ * gdn_decode_slots -- L tokens for each of N sequences whose states live in a pool
+ * of cache slots ("Qwen3.5 observation notes", section "Cache": a request keeps
+ * one batch index of the cache for its whole life, so a serving loop keeps states
+ * in fixed slots; "Qwen3.5-MoE-35B-A3B architecture teardown", section 6.2: an MTP
+ * draft is verified by running the main model on several tokens at once).
+ *   q, k   [N, L, H_qk, d_k] io_dtype     v [N, L, H_v, d_v] io_dtype     (in)
+ *   a, b   [N, L, H_v] fp32               A_log, dt_bias [H_v] fp32        (in)
+ *   state_pool   [num_slots, H_v, d_v, d_k] fp32                      (in/out)
+ *   state_slots  [N] int32, device, or NULL (sequence n uses slot n; then
+ *                num_slots >= N). Slot < 0: a padding entry -- its outputs
+ *                are written as zeros and no state is touched. Slot >=
+ *                num_slots sets GDN_ERR_BAD_SLOT in the device status word
+ *                and that sequence is skipped. Two sequences of one call must
+ *                not share a slot (their updates would race).
+ *   o      [N, L, H_v, d_v] io_dtype                                      (out)
+ *   intermediate_states  [N, L, H_v, d_v, d_k] fp32, or NULL: the state after
+ *                every token (entry L-1 equals the new pool state), so a
+ *                caller can roll back to the last accepted draft token.   (out)
+ * 1 <= L <= 16 (tokens_per_seq). The tokens of a sequence are applied in order,
+ * exactly as L calls of gdn_decode_step; the state is read and written once.
+ */
+int gdn_decode_slots(const void* q, const void* k, const void* v, int32_t io_dtype,
+                     const float* a, const float* b, const float* A_log, const float* dt_bias,
+                     float* state_pool, const int32_t* state_slots, int32_t num_slots,
+                     int32_t num_seqs, int32_t tokens_per_seq, int32_t H_qk, int32_t H_v,
+                     int32_t d_k, int32_t d_v, float scale, void* o,
+                     float* intermediate_states, void* stream);
 
 /*
  * gdn_prefill_noalloc -- gdn_prefill for callers that cannot allocate device
@@ -276,7 +306,7 @@ int gdn_rmsnorm_gated(const void* o, const void* z, int32_t io_dtype, const floa
 
 /*
  * Synchronise `stream`, then return and clear the device status word of the
- * current device (GDN_OK, GDN_ERR_BAD_SEQLENS or GDN_ERR_TIMEOUT), or
+ * current device (GDN_OK, GDN_ERR_BAD_SEQLENS, GDN_ERR_BAD_SLOT or GDN_ERR_TIMEOUT), or
  * GDN_ERR_CUDA if the synchronisation itself failed.
  */
 int gdn_sync_status(void* stream);

@@ -112,6 +112,7 @@ const char* gdn_status_string(int status) {
         case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
         case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
         case GDN_ERR_BAD_SEQLENS: return "GDN_ERR_BAD_SEQLENS";
+        case GDN_ERR_BAD_SLOT: return "GDN_ERR_BAD_SLOT";
         default: return "GDN_ERR_UNKNOWN";
     }
 }
@@ -221,6 +222,34 @@ int gdn_decode_step(const void* q, const void* k, const void* v, int32_t io_dtyp
     if (!aligned(a, 4) || !aligned(b, 4)) return GDN_ERR_INVALID_ARG;
     return to_status(launch_decode(q, k, v, io_dtype, a, b, A_log, dt_bias, state, num_seqs,
                                    H_qk, H_v, d_k, scale, o, (cudaStream_t)stream));
+}
+
+int gdn_decode_slots(const void* q, const void* k, const void* v, int32_t io_dtype,
+                     const float* a, const float* b, const float* A_log, const float* dt_bias,
+                     float* state_pool, const int32_t* state_slots, int32_t num_slots,
+                     int32_t num_seqs, int32_t tokens_per_seq, int32_t H_qk, int32_t H_v,
+                     int32_t d_k, int32_t d_v, float scale, void* o,
+                     float* intermediate_states, void* stream) {
+    if (io_dtype != GDN_BF16 && io_dtype != GDN_FP32) return GDN_ERR_INVALID_ARG;
+    if (num_seqs < 0 || num_slots < 0) return GDN_ERR_INVALID_ARG;
+    if (tokens_per_seq < 1 || tokens_per_seq > kMaxDecodeTokens) return GDN_ERR_UNSUPPORTED;
+    int hs = check_heads(H_qk, H_v, d_k, d_v);
+    if (hs != GDN_OK) return hs;
+    if (!isfinite(scale)) return GDN_ERR_INVALID_ARG;
+    if (!state_slots && num_slots < num_seqs) return GDN_ERR_INVALID_ARG;
+    if (num_seqs == 0) return GDN_OK;
+    if ((int64_t)num_seqs * H_v >= (int64_t)1 << 31) return GDN_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !a || !b || !A_log || !dt_bias || !o) return GDN_ERR_INVALID_ARG;
+    if (!state_pool && num_slots > 0) return GDN_ERR_INVALID_ARG;
+    const void* ptrs16[] = {q, k, v, o, state_pool, intermediate_states};
+    for (const void* p : ptrs16)
+        if (p && !aligned(p, 16)) return GDN_ERR_INVALID_ARG;
+    if (!aligned(a, 4) || !aligned(b, 4) || (state_slots && !aligned(state_slots, 4)))
+        return GDN_ERR_INVALID_ARG;
+    return to_status(launch_decode_multi(q, k, v, io_dtype, a, b, A_log, dt_bias, state_pool,
+                                         state_slots, num_slots, num_seqs, tokens_per_seq, H_qk,
+                                         H_v, d_k, scale, o, intermediate_states,
+                                         device_status_ptr(), (cudaStream_t)stream));
 }
 
 int gdn_conv1d_silu(const void* x, int32_t io_dtype, const float* weight, const float* bias,

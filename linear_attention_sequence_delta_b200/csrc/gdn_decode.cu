@@ -165,7 +165,177 @@ cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const f
     return cudaGetLastError();
 }
 
+// Decode of L tokens per sequence from a state pool ("Qwen3.5 observation notes",
+// section "Cache": a request keeps one batch index of the cache for its whole life;
+// "Qwen3.5-MoE-35B-A3B architecture teardown", section 6.2: the main model checks an MTP
+// draft token in the same forward pass, i.e. several tokens per step). The
+// state of sequence n lives in pool slot slots[n] (n without slots). Each block owns one
+// (sequence, V head); its rows stay in registers across the L tokens, so the state is
+// read and written once per call whatever L is. Normalised q, k, the values and the gates
+// of the L tokens are staged in shared memory first. With `inter`, the state after every
+// token is also written out (for rolling back rejected drafts).
+template <typename IO, int D>
+__global__ void __launch_bounds__(128) decode_multi_kernel(
+    const IO* __restrict__ q, const IO* __restrict__ k, const IO* __restrict__ v,
+    const float* __restrict__ a, const float* __restrict__ b, const float* __restrict__ A_log,
+    const float* __restrict__ dt_bias, float* __restrict__ pool,
+    const int32_t* __restrict__ slots, int num_slots, int L, int H_qk, int H_v, float scale,
+    IO* __restrict__ o, float* __restrict__ inter, int* status) {
+    constexpr int NV = D / 32;
+    constexpr int ROWS_PER_WARP = D / 4;
+    constexpr int ITERS = ROWS_PER_WARP / 4;
+    extern __shared__ float4 dm_smem[];
+    float* qs = reinterpret_cast<float*>(dm_smem);  // [L][D] normalised, scaled q
+    float* ks = qs + L * D;                          // [L][D] normalised k
+    float* vs = ks + L * D;                          // [L][D] values
+    float* par = vs + L * D;                         // [L][4]: alpha, beta, k.q
+
+    const int unit = blockIdx.x;  // n * H_v + h
+    const int n = unit / H_v;
+    const int h = unit - n * H_v;
+    const int j = h / (H_v / H_qk);
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int slot = slots ? slots[n] : n;
+    if (slot < 0) {  // a padding entry: zero outputs, no state touched
+        for (int idx = threadIdx.x; idx < L * D; idx += blockDim.x) {
+            const int t = idx / D, i = idx - t * D;
+            o[(((size_t)n * L + t) * H_v + h) * D + i] = from_f32<IO>(0.f);
+        }
+        return;
+    }
+    if (slot >= num_slots) {
+        if (threadIdx.x == 0) set_status(status, kStatusBadSlot);
+        return;
+    }
+    // stage the L tokens: one warp per token, lane owns columns lane + 32 m
+    for (int t = warp; t < L; t += 4) {
+        const size_t tok = (size_t)n * L + t;
+        const IO* qp = q + (tok * H_qk + j) * D;
+        const IO* kp = k + (tok * H_qk + j) * D;
+        const IO* vp = v + (tok * H_v + h) * D;
+        float qv[NV], kv[NV];
+        float sq = 0.f, sk = 0.f;
+#pragma unroll
+        for (int m = 0; m < NV; ++m) {
+            qv[m] = to_f32(qp[lane + 32 * m]);
+            kv[m] = to_f32(kp[lane + 32 * m]);
+            vs[t * D + lane + 32 * m] = to_f32(vp[lane + 32 * m]);
+            sq = fmaf(qv[m], qv[m], sq);
+            sk = fmaf(kv[m], kv[m], sk);
+        }
+        sq = warp_sum(sq);
+        sk = warp_sum(sk);
+        const float rq = scale / sqrtf(sq + kL2Eps);
+        const float rk = 1.f / sqrtf(sk + kL2Eps);
+        float kq = 0.f;
+#pragma unroll
+        for (int m = 0; m < NV; ++m) {
+            qv[m] *= rq;
+            kv[m] *= rk;
+            kq = fmaf(kv[m], qv[m], kq);
+            qs[t * D + lane + 32 * m] = qv[m];
+            ks[t * D + lane + 32 * m] = kv[m];
+        }
+        kq = warp_sum(kq);
+        if (lane == 0) {
+            const size_t gi = tok * H_v + h;
+            par[4 * t + 0] = expf(gate_g(a[gi], A_log[h], dt_bias[h]));
+            par[4 * t + 1] = gate_beta(b[gi]);
+            par[4 * t + 2] = kq;
+        }
+    }
+    __syncthreads();
+
+    const int p = lane & 7;
+    const int rg = lane >> 3;
+    float* S = pool + ((size_t)slot * H_v + h) * D * D;
+#pragma unroll 1
+    for (int it = 0; it < ITERS; ++it) {
+        const int row = warp * ROWS_PER_WARP + it * 4 + rg;
+        float4 sr[NV];
+        const float* rp = S + (size_t)row * D + 4 * p;
+#pragma unroll
+        for (int m = 0; m < NV; ++m) sr[m] = __ldcs(reinterpret_cast<const float4*>(rp + 32 * m));
+#pragma unroll 1
+        for (int t = 0; t < L; ++t) {
+            const float alpha = par[4 * t], beta = par[4 * t + 1], kq = par[4 * t + 2];
+            float4 kr[NV], qr[NV];
+#pragma unroll
+            for (int m = 0; m < NV; ++m) {
+                kr[m] = *reinterpret_cast<const float4*>(ks + t * D + 4 * p + 32 * m);
+                qr[m] = *reinterpret_cast<const float4*>(qs + t * D + 4 * p + 32 * m);
+            }
+            float dk = 0.f, dq = 0.f;
+#pragma unroll
+            for (int m = 0; m < NV; ++m) {
+                dk = fmaf(sr[m].x, kr[m].x, dk); dq = fmaf(sr[m].x, qr[m].x, dq);
+                dk = fmaf(sr[m].y, kr[m].y, dk); dq = fmaf(sr[m].y, qr[m].y, dq);
+                dk = fmaf(sr[m].z, kr[m].z, dk); dq = fmaf(sr[m].z, qr[m].z, dq);
+                dk = fmaf(sr[m].w, kr[m].w, dk); dq = fmaf(sr[m].w, qr[m].w, dq);
+            }
+#pragma unroll
+            for (int x = 1; x < 8; x <<= 1) {
+                dk += __shfl_xor_sync(0xffffffffu, dk, x);
+                dq += __shfl_xor_sync(0xffffffffu, dq, x);
+            }
+            const float delta = beta * (vs[t * D + row] - alpha * dk);
+#pragma unroll
+            for (int m = 0; m < NV; ++m) {
+                sr[m].x = fmaf(alpha, sr[m].x, delta * kr[m].x);
+                sr[m].y = fmaf(alpha, sr[m].y, delta * kr[m].y);
+                sr[m].z = fmaf(alpha, sr[m].z, delta * kr[m].z);
+                sr[m].w = fmaf(alpha, sr[m].w, delta * kr[m].w);
+            }
+            const size_t tok = (size_t)n * L + t;
+            if (p == 0) o[(tok * H_v + h) * D + row] = from_f32<IO>(fmaf(alpha, dq, delta * kq));
+            if (inter) {
+                float* ip = inter + (tok * H_v + h) * D * D + (size_t)row * D + 4 * p;
+#pragma unroll
+                for (int m = 0; m < NV; ++m) __stcs(reinterpret_cast<float4*>(ip + 32 * m), sr[m]);
+            }
+        }
+        float* wp = S + (size_t)row * D + 4 * p;
+#pragma unroll
+        for (int m = 0; m < NV; ++m) __stcs(reinterpret_cast<float4*>(wp + 32 * m), sr[m]);
+    }
+}
+
+template <typename IO, int D>
+cudaError_t launch_decode_multi_t(const void* q, const void* k, const void* v, const float* a,
+                                  const float* b, const float* A_log, const float* dt_bias,
+                                  float* pool, const int32_t* slots, int32_t num_slots,
+                                  int32_t N, int32_t L, int32_t H_qk, int32_t H_v, float scale,
+                                  void* o, float* inter, int* status, cudaStream_t s) {
+    const int64_t units = (int64_t)N * H_v;
+    if (units == 0) return cudaSuccess;
+    const size_t smem = (size_t)L * (3 * D + 4) * sizeof(float);
+    decode_multi_kernel<IO, D><<<(unsigned)units, 128, smem, s>>>(
+        static_cast<const IO*>(q), static_cast<const IO*>(k), static_cast<const IO*>(v), a, b,
+        A_log, dt_bias, pool, slots, num_slots, L, H_qk, H_v, scale, static_cast<IO*>(o), inter,
+        status);
+    return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_decode_multi(const void* q, const void* k, const void* v, int io_dtype,
+                                const float* a, const float* b, const float* A_log,
+                                const float* dt_bias, float* pool, const int32_t* slots,
+                                int32_t num_slots, int32_t N, int32_t L, int32_t H_qk,
+                                int32_t H_v, int32_t d, float scale, void* o, float* inter,
+                                int* status, cudaStream_t s) {
+#define GDN_DM(IO, D)                                                                          \
+    return launch_decode_multi_t<IO, D>(q, k, v, a, b, A_log, dt_bias, pool, slots, num_slots, \
+                                        N, L, H_qk, H_v, scale, o, inter, status, s)
+    if (io_dtype == GDN_BF16) {
+        if (d == 128) GDN_DM(__nv_bfloat16, 128);
+        GDN_DM(__nv_bfloat16, 64);
+    }
+    if (d == 128) GDN_DM(float, 128);
+    GDN_DM(float, 64);
+#undef GDN_DM
+}
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, int io_dtype,
                           const float* a, const float* b, const float* A_log,

@@ -21,6 +21,7 @@ constexpr float kMinLogDecay = -128.f;
 // Device status word values (written by kernels, read by gdn_sync_status).
 constexpr int kStatusBadSeqlens = GDN_ERR_BAD_SEQLENS;
 constexpr int kStatusTimeout = GDN_ERR_TIMEOUT;
+constexpr int kStatusBadSlot = GDN_ERR_BAD_SLOT;
 
 // ---- small device helpers ---------------------------------------------------
 
@@ -87,6 +88,16 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, int io_dt
                           const float* a, const float* b, const float* A_log,
                           const float* dt_bias, float* state, int32_t N, int32_t H_qk,
                           int32_t H_v, int32_t d, float scale, void* o, cudaStream_t s);
+
+// L tokens per sequence from a state pool indexed by slots (NULL: slot n), optional
+// per-token states; at most kMaxDecodeTokens tokens.
+constexpr int kMaxDecodeTokens = 16;
+cudaError_t launch_decode_multi(const void* q, const void* k, const void* v, int io_dtype,
+                                const float* a, const float* b, const float* A_log,
+                                const float* dt_bias, float* pool, const int32_t* slots,
+                                int32_t num_slots, int32_t N, int32_t L, int32_t H_qk,
+                                int32_t H_v, int32_t d, float scale, void* o, float* inter,
+                                int* status, cudaStream_t s);
 
 cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, int io_dtype,
                                 const float* G, const float* beta, const float* S0,

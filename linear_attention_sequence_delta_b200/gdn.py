@@ -28,14 +28,15 @@ LIB_PATH = os.path.join(_HERE, "libgdn.so")
 
 GDN_BF16, GDN_FP32 = 0, 1
 _STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "GDN_ERR_WORKSPACE",
-           4: "GDN_ERR_CUDA", 5: "GDN_ERR_TIMEOUT", 6: "GDN_ERR_BAD_SEQLENS"}
+           4: "GDN_ERR_CUDA", 5: "GDN_ERR_TIMEOUT", 6: "GDN_ERR_BAD_SEQLENS",
+           7: "GDN_ERR_BAD_SLOT"}
 
 # Every symbol include/gdn.h declares (the tests check the library exports them all).
 EXPORTS = ["gdn_status_string", "gdn_version", "gdn_prefill_workspace_size", "gdn_gates",
            "gdn_prefill", "gdn_decode_step", "gdn_sync_status", "gdn_prefill_noalloc",
            "gdn_set_prefill_impl", "gdn_set_kernel_timing", "gdn_last_prefill_kernel_ms",
            "gdn_last_prefill_kernel_name", "gdn_conv1d_silu", "gdn_conv1d_silu_decode",
-           "gdn_rmsnorm_gated"]
+           "gdn_rmsnorm_gated", "gdn_decode_slots"]
 GDN_IMPL_AUTO, GDN_IMPL_CUDA_CORE, GDN_IMPL_TENSOR_CORE, GDN_IMPL_TENSOR_CORE_SPLIT = 0, 1, 2, 3
 
 
@@ -86,6 +87,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gdn_conv1d_silu.argtypes = [P, i32, P, P, P, P, i32, i64, i32, i32, P, P, P]
     lib.gdn_conv1d_silu_decode.restype = ctypes.c_int
     lib.gdn_conv1d_silu_decode.argtypes = [P, i32, P, P, P, i32, i32, i32, P, P]
+    lib.gdn_decode_slots.restype = ctypes.c_int
+    lib.gdn_decode_slots.argtypes = [P, P, P, i32, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32,
+                                     i32, f32, P, P, P]
     lib.gdn_rmsnorm_gated.restype = ctypes.c_int
     lib.gdn_rmsnorm_gated.argtypes = [P, P, i32, P, f32, i64, i32, P, P]
     _lib = lib
@@ -192,6 +196,36 @@ def gdn_decode_step(q, k, v, a, b, A_log, dt_bias, state, *, scale: float = 1.0,
                              _ptr(o), _stream(q.device))
     _check(st, "gdn_decode_step")
     return o
+
+
+def gdn_decode_slots(q, k, v, a, b, A_log, dt_bias, state_pool, state_slots=None, *,
+                     scale: float = 1.0, out=None, intermediate_states=None,
+                     want_intermediate: bool = False):
+    """L tokens per sequence from a pool of states; the pool is updated in place.
+
+    q, k [N, L, H_qk, d_k]; v [N, L, H_v, d_v]; a, b [N, L, H_v] fp32;
+    state_pool [num_slots, H_v, d_v, d_k] fp32; state_slots int32 [N] or None (slot n).
+    Returns (o [N, L, H_v, d_v], intermediate states [N, L, H_v, d_v, d_k] or None).
+    """
+    lib = load_library()
+    _need_cuda(q, k, v, a, b, A_log, dt_bias, state_pool, state_slots, out, intermediate_states)
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k and v must share one dtype")
+    if state_slots is not None and state_slots.dtype != torch.int32:
+        raise TypeError("state_slots must be int32")
+    io = _io_dtype(q)
+    N, L, H_qk, d_k = q.shape
+    H_v, d_v = v.shape[2], v.shape[3]
+    o = out if out is not None else torch.empty((N, L, H_v, d_v), device=q.device, dtype=q.dtype)
+    if want_intermediate and intermediate_states is None:
+        intermediate_states = torch.empty((N, L, H_v, d_v, d_k), device=q.device,
+                                          dtype=torch.float32)
+    st = lib.gdn_decode_slots(_ptr(q), _ptr(k), _ptr(v), io, _ptr(a), _ptr(b), _ptr(A_log),
+                              _ptr(dt_bias), _ptr(state_pool), _ptr(state_slots),
+                              state_pool.shape[0], N, L, H_qk, H_v, d_k, d_v, float(scale),
+                              _ptr(o), _ptr(intermediate_states), _stream(q.device))
+    _check(st, "gdn_decode_slots")
+    return o, intermediate_states
 
 
 def set_prefill_impl(impl: int) -> int:

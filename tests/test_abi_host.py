@@ -208,6 +208,34 @@ def test_rmsnorm_gated_rejects(lib):
     assert r(None, None, 0, None, 1e-6, 0, 128, None, None) == 0
 
 
+def _call_slots(lib, **over):
+    a = dict(q=F, k=F + 0x1000, v=F + 0x2000, io=gdn.GDN_BF16, a=F + 0x3000, b=F + 0x4000,
+             A_log=F + 0x5000, dt_bias=F + 0x6000, pool=F + 0x10000, slots=F + 0x7000, ns=8,
+             N=4, L=2, H_qk=2, H_v=4, d_k=128, d_v=128, scale=1.0, o=F + 0x8000, inter=None)
+    a.update(over)
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.gdn_decode_slots(v(a["q"]), v(a["k"]), v(a["v"]), a["io"], v(a["a"]), v(a["b"]),
+                                v(a["A_log"]), v(a["dt_bias"]), v(a["pool"]), v(a["slots"]),
+                                a["ns"], a["N"], a["L"], a["H_qk"], a["H_v"], a["d_k"], a["d_v"],
+                                a["scale"], v(a["o"]), v(a["inter"]), None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(io=2), 1), (dict(N=-1), 1), (dict(ns=-1), 1), (dict(L=0), 2), (dict(L=17), 2),
+    (dict(H_v=5), 1), (dict(d_k=32, d_v=32), 2), (dict(scale=math.inf), 1),
+    (dict(slots=None, ns=3), 1),        # identity slots need a pool of at least N states
+    (dict(q=None), 1), (dict(o=None), 1), (dict(pool=None), 1),
+    (dict(pool=F + 8), 1), (dict(inter=F + 4), 1), (dict(slots=F + 2), 1), (dict(a=F + 1), 1),
+])
+def test_decode_slots_rejects(lib, over, code):
+    assert _call_slots(lib, **over) == code
+
+
+def test_decode_slots_noop(lib):
+    assert _call_slots(lib, N=0) == 0
+    assert _call_slots(lib, N=0, slots=None, ns=0, pool=None) == 0
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     saved = gdn._lib
     try:
