@@ -283,15 +283,21 @@ int gdn_conv1d_silu(const void* x, int32_t io_dtype, const float* weight, const 
 
 /*
  * gdn_conv1d_silu_decode -- the same convolution for one token of each of N
- * sequences, the cache slid by one position in place:
- *   x [N, conv_dim] io_dtype (in); conv_state [N, K-1, conv_dim] io_dtype
- *   (in/out); y [N, conv_dim] io_dtype (out); weight, bias as above.
- * Equal to gdn_conv1d_silu on N one-token sequences with conv_state_in =
- * conv_state_out = conv_state.
+ * sequences, each sequence's cache slid by one position in place:
+ *   x [N, conv_dim] io_dtype (in); y [N, conv_dim] io_dtype (out);
+ *   conv_state [num_slots, K-1, conv_dim] io_dtype, a pool of caches (in/out);
+ *   cache_slots [N] int32, device, or NULL (sequence n uses entry n; then
+ *   num_slots >= N). Slot < 0: a padding entry (y written as zeros, no cache
+ *   touched); slot >= num_slots sets GDN_ERR_BAD_SLOT in the device status word
+ *   and that sequence is skipped. Two sequences must not share a slot.
+ *   weight, bias as above.
+ * With identity slots it equals gdn_conv1d_silu on N one-token sequences with
+ * conv_state_in = conv_state_out = conv_state.
  */
 int gdn_conv1d_silu_decode(const void* x, int32_t io_dtype, const float* weight,
-                           const float* bias, void* conv_state, int32_t num_seqs,
-                           int32_t conv_dim, int32_t kernel_size, void* y, void* stream);
+                           const float* bias, void* conv_state, const int32_t* cache_slots,
+                           int32_t num_slots, int32_t num_seqs, int32_t conv_dim,
+                           int32_t kernel_size, void* y, void* stream);
 
 /*
  * gdn_rmsnorm_gated -- the mixer's output norm, per row of d values:

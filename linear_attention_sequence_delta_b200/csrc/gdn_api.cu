@@ -275,19 +275,23 @@ int gdn_conv1d_silu(const void* x, int32_t io_dtype, const float* weight, const 
 }
 
 int gdn_conv1d_silu_decode(const void* x, int32_t io_dtype, const float* weight,
-                           const float* bias, void* conv_state, int32_t num_seqs,
-                           int32_t conv_dim, int32_t kernel_size, void* y, void* stream) {
+                           const float* bias, void* conv_state, const int32_t* cache_slots,
+                           int32_t num_slots, int32_t num_seqs, int32_t conv_dim,
+                           int32_t kernel_size, void* y, void* stream) {
     if (io_dtype != GDN_BF16 && io_dtype != GDN_FP32) return GDN_ERR_INVALID_ARG;
-    if (num_seqs < 0 || conv_dim <= 0) return GDN_ERR_INVALID_ARG;
+    if (num_seqs < 0 || num_slots < 0 || conv_dim <= 0) return GDN_ERR_INVALID_ARG;
     if (kernel_size < 2 || kernel_size > 4 || conv_dim % 8 != 0) return GDN_ERR_UNSUPPORTED;
+    if (!cache_slots && num_slots < num_seqs) return GDN_ERR_INVALID_ARG;
     if (num_seqs == 0) return GDN_OK;
-    if (!x || !weight || !conv_state || !y) return GDN_ERR_INVALID_ARG;
+    if (!x || !weight || !y || (!conv_state && num_slots > 0)) return GDN_ERR_INVALID_ARG;
     const void* ptrs16[] = {x, y, weight, conv_state};
     for (const void* p : ptrs16)
-        if (!aligned(p, 16)) return GDN_ERR_INVALID_ARG;
+        if (p && !aligned(p, 16)) return GDN_ERR_INVALID_ARG;
     if (bias && !aligned(bias, 4)) return GDN_ERR_INVALID_ARG;
-    return to_status(launch_conv1d_silu_decode(x, io_dtype, weight, bias, conv_state, num_seqs,
-                                               conv_dim, kernel_size, y,
+    if (cache_slots && !aligned(cache_slots, 4)) return GDN_ERR_INVALID_ARG;
+    return to_status(launch_conv1d_silu_decode(x, io_dtype, weight, bias, conv_state,
+                                               cache_slots, num_slots, num_seqs, conv_dim,
+                                               kernel_size, y, device_status_ptr(),
                                                (cudaStream_t)stream));
 }
 

@@ -122,8 +122,9 @@ cudaError_t launch_conv1d_silu(const void* x, int io_dtype, const float* w, cons
                                const void* state_in, const int32_t* cu, int N, int64_t T, int C,
                                int K, void* y, void* state_out, int* status, cudaStream_t s);
 cudaError_t launch_conv1d_silu_decode(const void* x, int io_dtype, const float* w,
-                                      const float* bias, void* state, int N, int C, int K,
-                                      void* y, cudaStream_t s);
+                                      const float* bias, void* state, const int32_t* slots,
+                                      int num_slots, int N, int C, int K, void* y, int* status,
+                                      cudaStream_t s);
 cudaError_t launch_rmsnorm_gated(const void* o, const void* z, int io_dtype, const float* w,
                                  float eps, int64_t rows, int d, void* y, cudaStream_t s);
 

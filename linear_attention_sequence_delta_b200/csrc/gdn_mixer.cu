@@ -270,27 +270,35 @@ __global__ void __launch_bounds__(256) conv_state_kernel(const IO* __restrict__ 
 }
 
 // One token per sequence: y = silu(bias + w . [cache, x]); the cache slides by one.
-// A thread takes one channel vector of kDecSeqs sequences (the taps loaded once) and
-// loads all their inputs before using any.
+// The cache of sequence n is pool entry slots[n] (n without slots): a slot < 0 is a
+// padding entry (y zeroed, no cache touched), a slot >= num_slots is reported. A thread
+// takes one channel vector of kDecSeqs sequences (the taps loaded once) and loads all
+// their inputs before using any.
 template <typename IO, int K>
 __global__ void __launch_bounds__(128) conv_decode_kernel(const IO* __restrict__ x,
                                                           const float* __restrict__ w,
                                                           const float* __restrict__ bias,
-                                                          IO* state, int N, int C,
-                                                          IO* __restrict__ y) {
+                                                          IO* state,
+                                                          const int32_t* __restrict__ slots,
+                                                          int num_slots, int N, int C,
+                                                          IO* __restrict__ y, int* status) {
     const int nv = C / kVec;
     const int64_t gidx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t grp = gidx / nv;
     const int c0 = (int)(gidx - grp * nv) * kVec;
     const int64_t n0 = grp * kDecSeqs;
     if (n0 >= N) return;
+    int64_t slot[kDecSeqs];
     typename Vec8<IO>::Raw raw[kDecSeqs][K];
 #pragma unroll
     for (int q = 0; q < kDecSeqs; ++q) {
         const int64_t n = n0 + q < N ? n0 + q : n0;  // a missing last sequence re-reads n0
+        slot[q] = slots ? slots[n] : n;
+        const bool ok = slot[q] >= 0 && slot[q] < num_slots;
 #pragma unroll
         for (int j = 0; j < K - 1; ++j)
-            raw[q][j] = Vec8<IO>::load_raw(state + ((size_t)n * (K - 1) + j) * C + c0);
+            raw[q][j] = Vec8<IO>::load_raw(state + ((size_t)(ok ? slot[q] : 0) * (K - 1) + j) * C
+                                           + c0);
         raw[q][K - 1] = Vec8<IO>::load_raw(x + (size_t)n * C + c0);
     }
     float wt[K][kVec], bs[kVec];
@@ -300,6 +308,16 @@ __global__ void __launch_bounds__(128) conv_decode_kernel(const IO* __restrict__
         const int64_t n = n0 + q;
         if (n >= N) break;
         float out[kVec];
+        if (slot[q] < 0) {
+#pragma unroll
+            for (int e = 0; e < kVec; ++e) out[e] = 0.f;
+            Vec8<IO>::store(y + (size_t)n * C + c0, out);
+            continue;
+        }
+        if (slot[q] >= num_slots) {
+            set_status(status, kStatusBadSlot);
+            continue;
+        }
         float win[K][kVec];
 #pragma unroll
         for (int j = 0; j < K; ++j) Vec8<IO>::unpack(raw[q][j], win[j]);
@@ -313,7 +331,7 @@ __global__ void __launch_bounds__(128) conv_decode_kernel(const IO* __restrict__
         Vec8<IO>::store(y + (size_t)n * C + c0, out);
 #pragma unroll
         for (int j = 0; j < K - 1; ++j)
-            Vec8<IO>::store(state + ((size_t)n * (K - 1) + j) * C + c0, win[j + 1]);
+            Vec8<IO>::store(state + ((size_t)slot[q] * (K - 1) + j) * C + c0, win[j + 1]);
     }
 }
 
@@ -390,11 +408,13 @@ cudaError_t conv_launch(const void* x, const float* w, const float* bias, const 
 
 template <typename IO, int K>
 cudaError_t conv_decode_launch(const void* x, const float* w, const float* bias, void* state,
-                               int N, int C, void* y, cudaStream_t s) {
+                               const int32_t* slots, int num_slots, int N, int C, void* y,
+                               int* status, cudaStream_t s) {
     const int threads = 128;
     const int64_t groups = (N + kDecSeqs - 1) / kDecSeqs;
     conv_decode_kernel<IO, K><<<blocks_for(groups * (C / kVec), threads), threads, 0, s>>>(
-        static_cast<const IO*>(x), w, bias, static_cast<IO*>(state), N, C, static_cast<IO*>(y));
+        static_cast<const IO*>(x), w, bias, static_cast<IO*>(state), slots, num_slots, N, C,
+        static_cast<IO*>(y), status);
     return cudaGetLastError();
 }
 
@@ -411,11 +431,12 @@ cudaError_t conv_dispatch_k(int K, const void* x, const float* w, const float* b
 
 template <typename IO>
 cudaError_t conv_decode_dispatch_k(int K, const void* x, const float* w, const float* bias,
-                                   void* state, int N, int C, void* y, cudaStream_t s) {
+                                   void* state, const int32_t* slots, int num_slots, int N,
+                                   int C, void* y, int* status, cudaStream_t s) {
     switch (K) {
-        case 2: return conv_decode_launch<IO, 2>(x, w, bias, state, N, C, y, s);
-        case 3: return conv_decode_launch<IO, 3>(x, w, bias, state, N, C, y, s);
-        default: return conv_decode_launch<IO, 4>(x, w, bias, state, N, C, y, s);
+        case 2: return conv_decode_launch<IO, 2>(x, w, bias, state, slots, num_slots, N, C, y, status, s);
+        case 3: return conv_decode_launch<IO, 3>(x, w, bias, state, slots, num_slots, N, C, y, status, s);
+        default: return conv_decode_launch<IO, 4>(x, w, bias, state, slots, num_slots, N, C, y, status, s);
     }
 }
 
@@ -440,11 +461,14 @@ cudaError_t launch_conv1d_silu(const void* x, int io_dtype, const float* w, cons
 }
 
 cudaError_t launch_conv1d_silu_decode(const void* x, int io_dtype, const float* w,
-                                      const float* bias, void* state, int N, int C, int K,
-                                      void* y, cudaStream_t s) {
+                                      const float* bias, void* state, const int32_t* slots,
+                                      int num_slots, int N, int C, int K, void* y, int* status,
+                                      cudaStream_t s) {
     if (io_dtype == GDN_BF16)
-        return conv_decode_dispatch_k<__nv_bfloat16>(K, x, w, bias, state, N, C, y, s);
-    return conv_decode_dispatch_k<float>(K, x, w, bias, state, N, C, y, s);
+        return conv_decode_dispatch_k<__nv_bfloat16>(K, x, w, bias, state, slots, num_slots, N,
+                                                     C, y, status, s);
+    return conv_decode_dispatch_k<float>(K, x, w, bias, state, slots, num_slots, N, C, y,
+                                         status, s);
 }
 
 cudaError_t launch_rmsnorm_gated(const void* o, const void* z, int io_dtype, const float* w,

@@ -86,7 +86,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gdn_conv1d_silu.restype = ctypes.c_int
     lib.gdn_conv1d_silu.argtypes = [P, i32, P, P, P, P, i32, i64, i32, i32, P, P, P]
     lib.gdn_conv1d_silu_decode.restype = ctypes.c_int
-    lib.gdn_conv1d_silu_decode.argtypes = [P, i32, P, P, P, i32, i32, i32, P, P]
+    lib.gdn_conv1d_silu_decode.argtypes = [P, i32, P, P, P, P, i32, i32, i32, i32, P, P]
     lib.gdn_decode_slots.restype = ctypes.c_int
     lib.gdn_decode_slots.argtypes = [P, P, P, i32, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32,
                                      i32, f32, P, P, P]
@@ -285,16 +285,20 @@ def gdn_conv1d_silu(x, weight, bias, cu_seqlens, conv_state_in=None, *, want_sta
     return y, conv_state_out
 
 
-def gdn_conv1d_silu_decode(x, weight, bias, conv_state, *, out=None):
-    """One token per sequence: x [N, C]; conv_state [N, K-1, C] slides in place. Returns y."""
+def gdn_conv1d_silu_decode(x, weight, bias, conv_state, cache_slots=None, *, out=None):
+    """One token per sequence: x [N, C]; conv_state [num_slots, K-1, C] (a pool of caches)
+    slides in place; cache_slots int32 [N] or None (entry n). Returns y [N, C]."""
     lib = load_library()
-    _need_cuda(x, weight, bias, conv_state, out)
+    _need_cuda(x, weight, bias, conv_state, cache_slots, out)
+    if cache_slots is not None and cache_slots.dtype != torch.int32:
+        raise TypeError("cache_slots must be int32")
     io = _io_dtype(x)
     N, C = x.shape
     K = weight.shape[1]
     y = out if out is not None else torch.empty_like(x)
-    st = lib.gdn_conv1d_silu_decode(_ptr(x), io, _ptr(weight), _ptr(bias), _ptr(conv_state), N,
-                                    C, K, _ptr(y), _stream(x.device))
+    st = lib.gdn_conv1d_silu_decode(_ptr(x), io, _ptr(weight), _ptr(bias), _ptr(conv_state),
+                                    _ptr(cache_slots), conv_state.shape[0], N, C, K, _ptr(y),
+                                    _stream(x.device))
     _check(st, "gdn_conv1d_silu_decode")
     return y
 

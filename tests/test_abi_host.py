@@ -179,18 +179,21 @@ def test_conv1d_noops(lib):
 def test_conv1d_decode_rejects(lib):
     v = ctypes.c_void_p
     d = lib.gdn_conv1d_silu_decode
-    ok = lambda **o: dict(dict(x=F, io=0, w=F + 0x1000, b=None, st=F + 0x2000, N=4, C=64, K=4,
-                               y=F + 0x3000), **o)
-    call = lambda a: d(v(a["x"]) if a["x"] else None, a["io"], v(a["w"]) if a["w"] else None,
-                       v(a["b"]) if a["b"] else None, v(a["st"]) if a["st"] else None, a["N"],
-                       a["C"], a["K"], v(a["y"]) if a["y"] else None, None)
+    ok = lambda **o: dict(dict(x=F, io=0, w=F + 0x1000, b=None, st=F + 0x2000, sl=None, ns=4,
+                               N=4, C=64, K=4, y=F + 0x3000), **o)
+    p = lambda x: v(x) if x else None
+    call = lambda a: d(p(a["x"]), a["io"], p(a["w"]), p(a["b"]), p(a["st"]), p(a["sl"]),
+                       a["ns"], a["N"], a["C"], a["K"], p(a["y"]), None)
     assert call(ok(io=2)) == 1
     assert call(ok(N=-1)) == 1
+    assert call(ok(ns=-1)) == 1
+    assert call(ok(ns=3)) == 1            # identity slots need N cache entries
     assert call(ok(K=6)) == 2
     assert call(ok(C=12)) == 2
     assert call(ok(st=None)) == 1
     assert call(ok(st=F + 0x2004)) == 1
     assert call(ok(b=F + 1)) == 1
+    assert call(ok(sl=F + 0x4002, ns=2)) == 1
     assert call(ok(N=0)) == 0
 
 

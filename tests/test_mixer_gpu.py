@@ -155,6 +155,32 @@ def test_conv_decode_fp32_k3():
     np.testing.assert_array_equal(_np(st), so_ref)
 
 
+def test_conv_decode_cache_slots():
+    """Caches in a pool of slots: each sequence slides its own entry; a padding entry
+    (slot -1) gives zeros and touches nothing; unnamed entries come back bit for bit; a
+    slot past the pool is reported."""
+    N, pool_n = 5, 9
+    M = make_mixer_inputs([1] * pool_n, H_qk=2, H_v=4, d_k=64, d_v=64, seed=13)
+    slots = torch.tensor([7, 0, -1, 3, 8], dtype=torch.int32)
+    Md = M.to("cuda")
+    pool = Md.conv_state.clone()
+    x = Md.x[:N].contiguous()
+    y = gdn_conv1d_silu_decode(x, Md.conv_weight, Md.conv_bias, pool, slots.cuda())
+    assert gdn_sync_status() == 0
+    live = [n for n in range(N) if slots[n] >= 0]
+    sl = [int(slots[n]) for n in live]
+    y_ref, st_ref = oracle.conv1d_silu(M.x[live], M.conv_weight, M.conv_bias,
+                                       np.arange(len(live) + 1), M.conv_state[sl])
+    _close(y[live], y_ref, torch.bfloat16)
+    np.testing.assert_array_equal(_np(pool[sl]), st_ref)
+    assert torch.all(y[2] == 0)
+    rest = sorted(set(range(pool_n)) - set(sl))
+    assert torch.equal(pool[rest].cpu(), M.conv_state[rest])
+    bad = torch.tensor([1, 9], dtype=torch.int32, device="cuda")
+    gdn_conv1d_silu_decode(x[:2].contiguous(), Md.conv_weight, None, pool, bad)
+    assert gdn_sync_status() == 7
+
+
 def test_conv_bad_seqlens_reported():
     M = make_mixer_inputs(num_seqs=1, seq_len=40, H_qk=2, H_v=4, d_k=64, d_v=64, seed=8)
     Md = M.to("cuda")
