@@ -216,9 +216,24 @@ def run_decode_variants(rank, dev, flush, stream, hbm, peak_src, iters):
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
                          "frac": gbs / hbm, "algorithmic_bytes": byts, "kernel_ms": ms,
                          "peak_source": peak_src}}
+    # the single-token step with the state stored in bf16 (half the state bytes)
+    S16 = D.state[:N].to(torch.bfloat16)
+    q, k, v, a, b = (x[0, :N].contiguous() for x in (D.q, D.k, D.v, D.a, D.b))
+    o1 = torch.empty((N, H_v, d), device=dev, dtype=q.dtype)
+    ms = _time_op(lambda: gdn.gdn_decode_step_bf16_state(q, k, v, a, b, D.A_log, D.dt_bias, S16,
+                                                         out=o1), iters, flush, stream)
+    byts = 2 * N * H_v * d * d * 2 + N * (2 * H_qk * d + 2 * H_v * d) * 2 + 2 * N * H_v * 4
+    gbs = byts / (ms / 1e3) / 1e9
+    out["L1_bf16_state"] = {
+        "workload": f"{N} seqs x 1 token, H_qk={H_qk}, H_v={H_v}, d={d}, bf16 q/k/v/o, "
+                    "bf16 state in place (dense, no slots)",
+        "us_per_call": ms * 1e3, "tokens_per_s": N / (ms / 1e3),
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                     "frac": gbs / hbm, "algorithmic_bytes": byts, "kernel_ms": ms,
+                     "peak_source": peak_src}}
     out["l2"] = "flushed (512 MiB write) before every timed launch"
     out["iters"] = iters
-    return out, 2 * iters
+    return out, 3 * iters
 
 
 class Clocks:

@@ -168,6 +168,23 @@ int gdn_decode_step(const void* q, const void* k, const void* v, int32_t io_dtyp
                     int32_t d_v, float scale, void* o, void* stream);
 
 /*
+ * gdn_decode_step_bf16_state -- gdn_decode_step with the state stored in bf16
+ * ("Qwen3.5-MoE-35B-A3B architecture teardown", section 9.4: moving the fp32
+ * state to bf16 halves its memory; for decode it also halves the bytes moved).
+ *   state  [N, H_v, d_v, d_k] bf16, value-major, updated in place      (in/out)
+ *   everything else as gdn_decode_step.
+ * The state is widened to fp32, updated as in gdn_decode_step and rounded to bf16
+ * (round to nearest even) when written back, so each step adds a relative error
+ * of up to 2^-9 to the state; the decay keeps the sum of these errors bounded.
+ * Callers convert a prefill's fp32 final state to bf16 themselves.
+ */
+int gdn_decode_step_bf16_state(const void* q, const void* k, const void* v, int32_t io_dtype,
+                               const float* a, const float* b, const float* A_log,
+                               const float* dt_bias, void* state, int32_t num_seqs,
+                               int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v, float scale,
+                               void* o, void* stream);
+
+/*
  * gdn_decode_slots -- L tokens for each of N sequences whose states live in a pool
  * of cache slots ("Qwen3.5 observation notes", section "Cache": a request keeps
  * one batch index of the cache for its whole life, so a serving loop keeps states

@@ -224,6 +224,29 @@ int gdn_decode_step(const void* q, const void* k, const void* v, int32_t io_dtyp
                                    H_qk, H_v, d_k, scale, o, (cudaStream_t)stream));
 }
 
+int gdn_decode_step_bf16_state(const void* q, const void* k, const void* v, int32_t io_dtype,
+                               const float* a, const float* b, const float* A_log,
+                               const float* dt_bias, void* state, int32_t num_seqs,
+                               int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v, float scale,
+                               void* o, void* stream) {
+    if (io_dtype != GDN_BF16 && io_dtype != GDN_FP32) return GDN_ERR_INVALID_ARG;
+    if (num_seqs < 0) return GDN_ERR_INVALID_ARG;
+    int hs = check_heads(H_qk, H_v, d_k, d_v);
+    if (hs != GDN_OK) return hs;
+    if (!isfinite(scale)) return GDN_ERR_INVALID_ARG;
+    if (num_seqs == 0) return GDN_OK;
+    if ((int64_t)num_seqs * H_v >= (int64_t)1 << 31) return GDN_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !a || !b || !A_log || !dt_bias || !state || !o)
+        return GDN_ERR_INVALID_ARG;
+    const void* ptrs16[] = {q, k, v, o, state};
+    for (const void* p : ptrs16)
+        if (!aligned(p, 16)) return GDN_ERR_INVALID_ARG;
+    if (!aligned(a, 4) || !aligned(b, 4)) return GDN_ERR_INVALID_ARG;
+    return to_status(launch_decode_bf16_state(q, k, v, io_dtype, a, b, A_log, dt_bias, state,
+                                              num_seqs, H_qk, H_v, d_k, scale, o,
+                                              (cudaStream_t)stream));
+}
+
 int gdn_decode_slots(const void* q, const void* k, const void* v, int32_t io_dtype,
                      const float* a, const float* b, const float* A_log, const float* dt_bias,
                      float* state_pool, const int32_t* state_slots, int32_t num_slots,

@@ -165,6 +165,158 @@ cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const f
     return cudaGetLastError();
 }
 
+// The same step with the state stored in bf16 ("Qwen3.5-MoE-35B-A3B architecture
+// teardown", section 9.4: the fp32 state could move to bf16 to save half of its
+// memory; for decode that is also half the traffic): the state is read as bf16, updated in fp32 and
+// rounded to bf16 (round to nearest even) when written back. A lane holds 8
+// consecutive columns per 16-byte access (columns 8p + 64m), so every load and store
+// is 16 bytes as in the fp32 kernel.
+template <typename IO, int D>
+__global__ void __launch_bounds__(128, 5) decode_bf16_state_kernel(
+    const IO* __restrict__ q, const IO* __restrict__ k, const IO* __restrict__ v,
+    const float* __restrict__ a, const float* __restrict__ b,
+    const float* __restrict__ A_log, const float* __restrict__ dt_bias,
+    __nv_bfloat16* __restrict__ state, int H_qk, int H_v, float scale, IO* __restrict__ o) {
+    constexpr int NV = D / 64;               // 16-byte chunks of 8 columns per lane per row
+    constexpr int ROWS_PER_WARP = D / 4;
+    constexpr int ITERS = ROWS_PER_WARP / 4;
+    constexpr int B = 2 * kRowGroupsInFlight;  // half the bytes per row: twice the rows
+    static_assert(ITERS % B == 0, "row groups must tile the warp's rows");
+    // Each warp keeps its own copy of the normalised q and k in shared memory (read back
+    // as 16-byte broadcasts), which leaves registers for 8 blocks per SM.
+    __shared__ __align__(16) float qk_s[4][2][D];
+
+    const int unit = blockIdx.x;
+    const int n = unit / H_v;
+    const int h = unit - n * H_v;
+    const int j = h / (H_v / H_qk);
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int p = lane & 7;
+    const int rg = lane >> 3;
+
+    __nv_bfloat16* S = state + (size_t)unit * D * D;
+    const IO* vp = v + (size_t)unit * D;
+    IO* op = o + (size_t)unit * D;
+
+    // the first row groups' state loads go out before the q/k work they do not need
+    uint4 raw[B][NV];
+    float vi[B];
+    auto load_groups = [&](int it0) {
+#pragma unroll
+        for (int bb = 0; bb < B; ++bb) {
+            const int row = warp * ROWS_PER_WARP + (it0 + bb) * 4 + rg;
+            const __nv_bfloat16* rp = S + (size_t)row * D + 8 * p;
+#pragma unroll
+            for (int m = 0; m < NV; ++m) raw[bb][m] = __ldcs(reinterpret_cast<const uint4*>(rp + 64 * m));
+            vi[bb] = to_f32(vp[row]);
+        }
+    };
+    load_groups(0);
+
+    // normalised q and k (lane owns columns lane + 32 m), written to this warp's copy
+    const IO* qp = q + ((size_t)n * H_qk + j) * D;
+    const IO* kp = k + ((size_t)n * H_qk + j) * D;
+    float qv[D / 32], kv[D / 32];
+    float sq = 0.f, sk = 0.f;
+#pragma unroll
+    for (int m = 0; m < D / 32; ++m) {
+        qv[m] = to_f32(qp[lane + 32 * m]);
+        kv[m] = to_f32(kp[lane + 32 * m]);
+        sq = fmaf(qv[m], qv[m], sq);
+        sk = fmaf(kv[m], kv[m], sk);
+    }
+    sq = warp_sum(sq);
+    sk = warp_sum(sk);
+    const float rq = scale / sqrtf(sq + kL2Eps);
+    const float rk = 1.f / sqrtf(sk + kL2Eps);
+    float kq = 0.f;
+#pragma unroll
+    for (int m = 0; m < D / 32; ++m) {
+        qv[m] *= rq;
+        kv[m] *= rk;
+        kq = fmaf(kv[m], qv[m], kq);
+        qk_s[warp][0][lane + 32 * m] = qv[m];
+        qk_s[warp][1][lane + 32 * m] = kv[m];
+    }
+    kq = warp_sum(kq);
+    __syncwarp();
+    const float alpha = expf(gate_g(a[unit], A_log[h], dt_bias[h]));
+    const float beta = gate_beta(b[unit]);
+    const float* qs = qk_s[warp][0];
+    const float* ks = qk_s[warp][1];
+
+#pragma unroll 1
+    for (int it0 = 0; it0 < ITERS; it0 += B) {
+        if (it0 > 0) load_groups(it0);
+#pragma unroll
+        for (int bb = 0; bb < B; ++bb) {
+            const int row = warp * ROWS_PER_WARP + (it0 + bb) * 4 + rg;
+            float sv[NV][8];
+#pragma unroll
+            for (int m = 0; m < NV; ++m) {
+                const __nv_bfloat162* hp = reinterpret_cast<const __nv_bfloat162*>(&raw[bb][m]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(hp[e]);
+                    sv[m][2 * e] = f.x;
+                    sv[m][2 * e + 1] = f.y;
+                }
+            }
+            float dk = 0.f, dq = 0.f;
+#pragma unroll
+            for (int m = 0; m < NV; ++m)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const float4 k4 = *reinterpret_cast<const float4*>(ks + 8 * p + 64 * m + 4 * hh);
+                    const float4 q4 = *reinterpret_cast<const float4*>(qs + 8 * p + 64 * m + 4 * hh);
+                    const float* sp = sv[m] + 4 * hh;
+                    dk = fmaf(sp[0], k4.x, dk); dq = fmaf(sp[0], q4.x, dq);
+                    dk = fmaf(sp[1], k4.y, dk); dq = fmaf(sp[1], q4.y, dq);
+                    dk = fmaf(sp[2], k4.z, dk); dq = fmaf(sp[2], q4.z, dq);
+                    dk = fmaf(sp[3], k4.w, dk); dq = fmaf(sp[3], q4.w, dq);
+                }
+#pragma unroll
+            for (int x = 1; x < 8; x <<= 1) {
+                dk += __shfl_xor_sync(0xffffffffu, dk, x);
+                dq += __shfl_xor_sync(0xffffffffu, dq, x);
+            }
+            const float delta = beta * (vi[bb] - alpha * dk);
+            __nv_bfloat16* rp = S + (size_t)row * D + 8 * p;
+#pragma unroll
+            for (int m = 0; m < NV; ++m) {
+                const float4 k0 = *reinterpret_cast<const float4*>(ks + 8 * p + 64 * m);
+                const float4 k1 = *reinterpret_cast<const float4*>(ks + 8 * p + 64 * m + 4);
+                const float kk[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+                uint4 w;
+                __nv_bfloat162* wh = reinterpret_cast<__nv_bfloat162*>(&w);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    wh[e] = __floats2bfloat162_rn(fmaf(alpha, sv[m][2 * e], delta * kk[2 * e]),
+                                                  fmaf(alpha, sv[m][2 * e + 1],
+                                                       delta * kk[2 * e + 1]));
+                __stcs(reinterpret_cast<uint4*>(rp + 64 * m), w);
+            }
+            if (p == 0) op[row] = from_f32<IO>(fmaf(alpha, dq, delta * kq));
+        }
+    }
+}
+
+template <typename IO, int D>
+cudaError_t launch_decode_bf16_state_t(const void* q, const void* k, const void* v,
+                                       const float* a, const float* b, const float* A_log,
+                                       const float* dt_bias, void* state, int32_t N,
+                                       int32_t H_qk, int32_t H_v, float scale, void* o,
+                                       cudaStream_t s) {
+    const int64_t units = (int64_t)N * H_v;
+    if (units == 0) return cudaSuccess;
+    decode_bf16_state_kernel<IO, D><<<(unsigned)units, 128, 0, s>>>(
+        static_cast<const IO*>(q), static_cast<const IO*>(k), static_cast<const IO*>(v), a, b,
+        A_log, dt_bias, static_cast<__nv_bfloat16*>(state), H_qk, H_v, scale,
+        static_cast<IO*>(o));
+    return cudaGetLastError();
+}
+
 // Decode of L tokens per sequence from a state pool ("Qwen3.5 observation notes",
 // section "Cache": a request keeps one batch index of the cache for its whole life;
 // "Qwen3.5-MoE-35B-A3B architecture teardown", section 6.2: the main model checks an MTP
@@ -335,6 +487,23 @@ cudaError_t launch_decode_multi(const void* q, const void* k, const void* v, int
     if (d == 128) GDN_DM(float, 128);
     GDN_DM(float, 64);
 #undef GDN_DM
+}
+
+cudaError_t launch_decode_bf16_state(const void* q, const void* k, const void* v,
+                                     int io_dtype, const float* a, const float* b,
+                                     const float* A_log, const float* dt_bias, void* state,
+                                     int32_t N, int32_t H_qk, int32_t H_v, int32_t d,
+                                     float scale, void* o, cudaStream_t s) {
+#define GDN_DB(IO, D)                                                                       \
+    return launch_decode_bf16_state_t<IO, D>(q, k, v, a, b, A_log, dt_bias, state, N, H_qk, \
+                                             H_v, scale, o, s)
+    if (io_dtype == GDN_BF16) {
+        if (d == 128) GDN_DB(__nv_bfloat16, 128);
+        GDN_DB(__nv_bfloat16, 64);
+    }
+    if (d == 128) GDN_DB(float, 128);
+    GDN_DB(float, 64);
+#undef GDN_DB
 }
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, int io_dtype,

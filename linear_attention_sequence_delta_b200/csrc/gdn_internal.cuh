@@ -89,6 +89,13 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, int io_dt
                           const float* dt_bias, float* state, int32_t N, int32_t H_qk,
                           int32_t H_v, int32_t d, float scale, void* o, cudaStream_t s);
 
+// Single-token decode with a bf16 state [N, H_v, d_v, d_k], updated in place.
+cudaError_t launch_decode_bf16_state(const void* q, const void* k, const void* v,
+                                     int io_dtype, const float* a, const float* b,
+                                     const float* A_log, const float* dt_bias, void* state,
+                                     int32_t N, int32_t H_qk, int32_t H_v, int32_t d,
+                                     float scale, void* o, cudaStream_t s);
+
 // L tokens per sequence from a state pool indexed by slots (NULL: slot n), optional
 // per-token states; at most kMaxDecodeTokens tokens.
 constexpr int kMaxDecodeTokens = 16;

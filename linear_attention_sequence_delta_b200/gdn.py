@@ -36,7 +36,7 @@ EXPORTS = ["gdn_status_string", "gdn_version", "gdn_prefill_workspace_size", "gd
            "gdn_prefill", "gdn_decode_step", "gdn_sync_status", "gdn_prefill_noalloc",
            "gdn_set_prefill_impl", "gdn_set_kernel_timing", "gdn_last_prefill_kernel_ms",
            "gdn_last_prefill_kernel_name", "gdn_conv1d_silu", "gdn_conv1d_silu_decode",
-           "gdn_rmsnorm_gated", "gdn_decode_slots"]
+           "gdn_rmsnorm_gated", "gdn_decode_slots", "gdn_decode_step_bf16_state"]
 GDN_IMPL_AUTO, GDN_IMPL_CUDA_CORE, GDN_IMPL_TENSOR_CORE, GDN_IMPL_TENSOR_CORE_SPLIT = 0, 1, 2, 3
 
 
@@ -87,6 +87,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gdn_conv1d_silu.argtypes = [P, i32, P, P, P, P, i32, i64, i32, i32, P, P, P]
     lib.gdn_conv1d_silu_decode.restype = ctypes.c_int
     lib.gdn_conv1d_silu_decode.argtypes = [P, i32, P, P, P, P, i32, i32, i32, i32, P, P]
+    lib.gdn_decode_step_bf16_state.restype = ctypes.c_int
+    lib.gdn_decode_step_bf16_state.argtypes = [P, P, P, i32, P, P, P, P, P, i32, i32, i32, i32,
+                                               i32, f32, P, P]
     lib.gdn_decode_slots.restype = ctypes.c_int
     lib.gdn_decode_slots.argtypes = [P, P, P, i32, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32,
                                      i32, f32, P, P, P]
@@ -195,6 +198,24 @@ def gdn_decode_step(q, k, v, a, b, A_log, dt_bias, state, *, scale: float = 1.0,
                              _ptr(dt_bias), _ptr(state), N, H_qk, H_v, d_k, d_v, float(scale),
                              _ptr(o), _stream(q.device))
     _check(st, "gdn_decode_step")
+    return o
+
+
+def gdn_decode_step_bf16_state(q, k, v, a, b, A_log, dt_bias, state, *, scale: float = 1.0,
+                               out=None):
+    """gdn_decode_step with a bf16 state [N, H_v, d_v, d_k] updated in place. Returns o."""
+    lib = load_library()
+    _need_cuda(q, k, v, a, b, A_log, dt_bias, state, out)
+    if state.dtype != torch.bfloat16:
+        raise TypeError("state must be bfloat16")
+    io = _io_dtype(q)
+    N, H_qk, d_k = q.shape
+    _, H_v, d_v = v.shape
+    o = out if out is not None else torch.empty((N, H_v, d_v), device=q.device, dtype=q.dtype)
+    st = lib.gdn_decode_step_bf16_state(_ptr(q), _ptr(k), _ptr(v), io, _ptr(a), _ptr(b),
+                                        _ptr(A_log), _ptr(dt_bias), _ptr(state), N, H_qk, H_v,
+                                        d_k, d_v, float(scale), _ptr(o), _stream(q.device))
+    _check(st, "gdn_decode_step_bf16_state")
     return o
 
 

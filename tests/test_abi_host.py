@@ -134,6 +134,25 @@ def test_decode_rejects(lib, over, code):
     assert _call_decode(lib, **over) == code
 
 
+def test_decode_bf16_state_rejects(lib):
+    v = ctypes.c_void_p
+    f = lib.gdn_decode_step_bf16_state
+    args = lambda **o: dict(dict(q=F, k=F + 0x1000, vv=F + 0x2000, io=0, a=F + 0x3000,
+                                 b=F + 0x4000, al=F + 0x5000, dt=F + 0x6000, S=F + 0x10000, N=8,
+                                 hq=2, hv=4, dk=128, dv=128, sc=1.0, o=F + 0x8000), **o)
+    p = lambda x: v(x) if x else None
+    call = lambda a: f(p(a["q"]), p(a["k"]), p(a["vv"]), a["io"], p(a["a"]), p(a["b"]),
+                       p(a["al"]), p(a["dt"]), p(a["S"]), a["N"], a["hq"], a["hv"], a["dk"],
+                       a["dv"], a["sc"], p(a["o"]), None)
+    assert call(args(io=3)) == 1
+    assert call(args(hv=5)) == 1
+    assert call(args(dk=96, dv=96)) == 2
+    assert call(args(S=None)) == 1
+    assert call(args(S=F + 0x10008)) == 1
+    assert call(args(sc=math.nan)) == 1
+    assert call(args(N=0)) == 0
+
+
 def test_decode_zero_sequences_is_noop(lib):
     assert _call_decode(lib, N=0) == 0
 
