@@ -73,11 +73,13 @@ int gdn_version(void);
 /*
  * Bytes of device workspace gdn_prefill needs for these sizes. For d = 128 it
  * covers the tensor-core path: the chunk offsets of the sequences, then per
- * (64-token chunk, V head) a 4-byte ready flag and a 17,664-byte record (the
+ * (64-token chunk, V head) an 8-byte ready flag and a 17,664-byte record (the
  * chunk's T diag(beta) and P matrices and per-token factors), i.e. about 276
  * bytes per token and V head (with one extra chunk per sequence), each part
  * rounded up to 256 bytes; for d = 64 (CUDA-core path) it is the per-token G and
  * beta, fp32 [T, H_v] each. Returns 0 for invalid sizes (and for num_seqs = 0).
+ * The workspace needs no initialisation: a ready flag holds the number of the
+ * call that wrote it, and call numbers grow within the process.
  */
 size_t gdn_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t H_qk,
                                   int32_t H_v, int32_t d_k, int32_t d_v);

@@ -50,6 +50,8 @@
 // word, leaves its loops, drains its copies, frees its tensor memory and exits.
 #include <cuda.h>
 
+#include <atomic>
+
 #include "gdn_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -243,10 +245,13 @@ __device__ __forceinline__ void ap_half_row(const float (&x)[32], int row, const
     }
 }
 
-// Record (chunk cg, V head h) is complete: publish it to the chain (release).
-__device__ __forceinline__ void publish_record(int* flags, size_t idx) {
+// Record (chunk cg, V head h) is complete: publish it to the chain (release). A flag
+// holds the number of the call that wrote it last; call numbers only grow within a
+// process, so flags left by earlier calls never read as ready and need no reset.
+__device__ __forceinline__ void publish_record(unsigned long long* flags, size_t idx,
+                                               unsigned long long epoch) {
     __threadfence();
-    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flags + idx), "r"(1) : "memory");
+    asm volatile("st.release.gpu.global.b64 [%0], %1;" ::"l"(flags + idx), "l"(epoch) : "memory");
 }
 
 // One prep worker of kPrepThreads threads (tid 0 .. 255, synchronised by the named
@@ -257,8 +262,9 @@ __device__ __forceinline__ void prep_worker(
     const float* __restrict__ b, const float* __restrict__ A_log,
     const float* __restrict__ dt_bias, const int32_t* __restrict__ cu_seqlens,
     const int32_t* __restrict__ choff, int32_t N, int H_qk, int H_v, float scale,
-    uint8_t* __restrict__ rec, int* status, int* flags, uint8_t* sm, const int tid,
-    const int bar_id, const int worker, const int nworkers, const bool relinquish) {
+    uint8_t* __restrict__ rec, int* status, unsigned long long* flags,
+    unsigned long long epoch, uint8_t* sm, const int tid, const int bar_id, const int worker,
+    const int nworkers, const bool relinquish) {
     uint8_t* KQ = sm + PS_KQ;
     float* Ts = reinterpret_cast<float*>(sm + PS_TS);
     float* As = reinterpret_cast<float*>(sm + PS_AS);
@@ -567,7 +573,7 @@ __device__ __forceinline__ void prep_worker(
                 *reinterpret_cast<uint4*>(R + REC_T + sw128_off(row, ch)) = w;
             }
             named_bar_sync(bar_id, kPrepThreads);  // Ts, As, Xs and the head scratch are reused
-            if (flags && tid == 0) publish_record(flags, (size_t)cg * H_v + h);
+            if (flags && tid == 0) publish_record(flags, (size_t)cg * H_v + h, epoch);
         }
         tc_fence_before();  // this unit's TMEM reads precede the next unit's MMA
     }
@@ -588,7 +594,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     prep_worker(q, k, a, b, A_log, dt_bias, cu_seqlens, choff, N, H_qk, H_v, scale, rec, status,
-                nullptr, sm, threadIdx.x, 1, blockIdx.x, gridDim.x, true);
+                nullptr, 0, sm, threadIdx.x, 1, blockIdx.x, gridDim.x, true);
 }
 
 // ==================================== chain =======================================
@@ -610,7 +616,8 @@ constexpr uint32_t CS_OST = kRing * kSlotBytes;     // [2 col blocks][64 t][128 
 constexpr uint32_t CS_BAR = CS_OST + 16384;         // barriers (see below)
 constexpr uint32_t CS_TMEM = CS_BAR + 128;
 constexpr uint32_t CS_ERR = CS_BAR + 132;
-constexpr size_t kChainSmem = CS_BAR + 256 + 1024;
+constexpr uint32_t CS_EGQ = CS_BAR + 256;           // [64] fp32: the chunk's output row factors
+constexpr size_t kChainSmem = CS_EGQ + 256 + 1024;
 
 // tensor memory columns (512 allocated)
 constexpr uint32_t TM_U = 0;      // 128: the chunk's state increment (scaled Vn^T) K, fp32
@@ -651,16 +658,17 @@ __device__ __forceinline__ uint32_t tile64_off(int t, int i) {
 //               (S0 Q^T alternates between two accumulators) and, once a chunk's
 //               ring slot is no longer read, load the chunk three ahead into it
 //               (TMA tiles for K, Q, V and one bulk copy of the record).
-// Waits (bounded) until a record is published by a prep worker (acquire).
-__device__ __forceinline__ bool wait_record(const int* flag, long long max_cycles) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
-    if (v) return true;
+// Waits (bounded) until a prep worker publishes a record in this call (acquire).
+__device__ __forceinline__ bool wait_record(const unsigned long long* flag,
+                                            unsigned long long epoch, long long max_cycles) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(flag) : "memory");
+    if (v == epoch) return true;
     const long long t0 = clock64();
     do {
         __nanosleep(64);
-        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
-        if (v) return true;
+        asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(flag) : "memory");
+        if (v == epoch) return true;
     } while (clock64() - t0 < max_cycles);
     return false;
 }
@@ -674,7 +682,8 @@ __device__ __forceinline__ void chain_unit(
     const CUtensorMap& tm_o, const float* __restrict__ S0g, const int32_t* __restrict__ cu_seqlens,
     const int32_t* __restrict__ choff, int64_t T_total, int H_qk, int H_v,
     const uint8_t* __restrict__ rec, bf16* __restrict__ o, float* __restrict__ Sfg, int* status,
-    const int* flags, uint8_t* sm, const int tid, const int n, const int h, const uint32_t tmem,
+    const unsigned long long* flags, unsigned long long epoch, uint8_t* sm, const int tid,
+    const int n, const int h, const uint32_t tmem,
     const int sync_id) {
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + CS_BAR);  // [3] slot landed
     uint64_t* mbar = full + kRing;         // chain MMA completions
@@ -712,18 +721,13 @@ __device__ __forceinline__ void chain_unit(
     named_bar_sync(sync_id, kChainThreads);
     tc_fence_after();
 
-    // chunk c of this sequence -> its ring slot (issued by one lane)
-    auto issue_loads = [&](int c) -> bool {
+    // chunk c of this sequence -> its ring slot (issued by one lane). The K, Q, V tiles
+    // need nothing from the prep workers and go first; the record follows once its
+    // flag is seen (the slot's barrier expects both).
+    auto load_tiles = [&](int c) {
         const int st = c % kRing;
         uint8_t* slot = sm + st * kSlotBytes;
         const int32_t t0 = (int32_t)(s0 + (int64_t)c * kC);
-        if (flags) {
-            if (!wait_record(flags + (size_t)(cg0 + c) * H_v + h, kWaitCycles)) {
-                *s_err = 1;
-                return false;
-            }
-            asm volatile("fence.proxy.async.global;" ::: "memory");  // the record, read by TMA
-        }
         mbar_arrive_expect_tx(&full[st], kSlotTx);
         tma_load_3d(slot + SLOT_KQ, &tm_k, 0, j, t0, &full[st]);
         tma_load_3d(slot + SLOT_KQ + 16384, &tm_k, 64, j, t0, &full[st]);
@@ -731,9 +735,22 @@ __device__ __forceinline__ void chain_unit(
         tma_load_3d(slot + SLOT_KQ + 16384 + 8192, &tm_q, 64, j, t0, &full[st]);
         tma_load_3d(slot + SLOT_V, &tm_v, 0, h, t0, &full[st]);
         tma_load_3d(slot + SLOT_V + 8192, &tm_v, 64, h, t0, &full[st]);
-        bulk_g2s(slot + SLOT_REC, rec + ((size_t)(cg0 + c) * H_v + h) * kRecBytes, kRecBytes,
-                 &full[st]);
+    };
+    // After a wait that ran out the record is copied all the same (valid memory, the
+    // results are discarded), so that the slot's barrier completes and no copy is left
+    // in flight when the block exits.
+    auto record_ready = [&](int c) -> bool {
+        if (flags && !wait_record(flags + (size_t)(cg0 + c) * H_v + h, epoch, kWaitCycles)) {
+            *s_err = 1;
+            return false;
+        }
         return true;
+    };
+    auto load_record = [&](int c) {
+        const int st = c % kRing;
+        if (flags) asm volatile("fence.proxy.async.global;" ::: "memory");  // read by TMA
+        bulk_g2s(sm + st * kSlotBytes + SLOT_REC, rec + ((size_t)(cg0 + c) * H_v + h) * kRecBytes,
+                 kRecBytes, &full[st]);
     };
 
     if (warp > kIssueWarp) {
@@ -744,23 +761,39 @@ __device__ __forceinline__ void chain_unit(
         const uint32_t ctl = tmem + ((uint32_t)(qo * 32) << 16);
         uint8_t* ost = sm + CS_OST;
         const bool loader = warp == kLoadWarp && lane == 0;
-        int issued = 0;
-        if (loader)
+        float* egq = reinterpret_cast<float*>(sm + CS_EGQ);
+        int issued = 0;   // chunks whose tiles and record were issued
+        if (loader) {
+            for (int c = 0; c < kRing && c < nchunks; ++c) load_tiles(c);
             for (int c = 0; c < kRing && c < nchunks; ++c) {
-                if (!issue_loads(c)) break;
+                record_ready(c);
+                load_record(c);
                 issued = c + 1;
             }
+        }
         __syncwarp();
 #pragma unroll 1
         for (int cp = 0; cp < nchunks; ++cp) {
             const int b = cp & 1;
+            const int cn = cp + kRing;  // the chunk that will reuse this chunk's slot
+            // its record's flag is checked while this chunk's MMAs still run
+            const bool next = loader && cn < nchunks && issued == cn;
+            if (next) record_ready(cn);
             const bool ok = mbar_wait_bounded(&obar[b], (cp >> 1) & 1, kWaitCycles);
             if (!ok) *s_err = 1;
             if (loader) bulk_wait_group_read<0>();  // staging free again
+            // the slot's only remaining reader is this copy of the row factors
+            if (ok && to < 16)
+                reinterpret_cast<float4*>(egq)[to] = reinterpret_cast<const float4*>(
+                    sm + (cp % kRing) * kSlotBytes + SLOT_REC + REC_G + 4 * RG_EGQ)[to];
             if (named_bar_any(2, kOut, !ok || *s_err != 0)) break;
+            if (next) {  // the slot is free: refill it now, two chunks before it is needed
+                load_tiles(cn);
+                load_record(cn);
+                issued = cn + 1;
+            }
             tc_fence_after();
-            const float4* eg4 = reinterpret_cast<const float4*>(
-                sm + (cp % kRing) * kSlotBytes + SLOT_REC + REC_G + 4 * RG_EGQ);
+            const float4* eg4 = reinterpret_cast<const float4*>(egq);
             const uint32_t qacc = ctl + (b ? TM_D1Q1 : TM_D1Q0);
             // this thread's column of the staged tile; laundered so that the 64 element
             // addresses are formed per chunk rather than held in registers across chunks
@@ -809,9 +842,6 @@ __device__ __forceinline__ void chain_unit(
                     *reinterpret_cast<uint4*>(o + ((size_t)(t0 + r) * H_v + h) * kD + ch * 8) = w;
                 }
                 named_bar_sync(2, kOut);
-            }
-            if (loader && cp + kRing < nchunks && issued == cp + kRing) {
-                if (issue_loads(cp + kRing)) issued = cp + kRing + 1;
             }
             __syncwarp();
         }
@@ -1106,7 +1136,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
     chain_unit(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v, rec, o, Sfg,
-               status, nullptr, sm, threadIdx.x, blockIdx.x / H_v, blockIdx.x % H_v, tmem, 1);
+               status, nullptr, 0, sm, threadIdx.x, blockIdx.x / H_v, blockIdx.x % H_v, tmem, 1);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1116,11 +1146,11 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
 // ==================================== fused =======================================
 // Prep and chain in one cooperative launch (every block resident at once), so the
 // chain of the first sequences runs while prep workers produce the later records.
-// Blocks 0 .. c0-1 start on the chain units; the others run two prep workers each
-// (256 threads, their own 90 KB of shared memory and 64 TMEM columns), then join
-// the chain. Chain units are handed out in (sequence, V head) order by an atomic
-// counter; a chain's loader waits (bounded) for each record's flag before its bulk
-// copy, and prep workers never wait on chains, so every wait ends.
+// Block u < c0 runs chain unit u (sequence u / H_v, V head u % H_v); the others run
+// two prep workers each (256 threads, their own 90 KB of shared memory and 64 TMEM
+// columns). A chain's loader waits (bounded) for each record's flag to carry this
+// call's number before its bulk copy, and prep workers never wait on chains, so
+// every wait ends. Nothing in the workspace needs clearing between calls.
 constexpr int kFusedThreads = 512;
 constexpr uint32_t kPrepRegion = 96256;
 static_assert(kPrepRegion + 1024 >= kPrepSmem, "prep worker region too small");
@@ -1137,8 +1167,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
     const float* __restrict__ dt_bias, const float* __restrict__ S0g,
     const int32_t* __restrict__ cu_seqlens, const int32_t* choff, int32_t N,
     int64_t T_total, int H_qk, int H_v, float scale, uint8_t* __restrict__ rec,
-    bf16* __restrict__ o, float* __restrict__ Sfg, int* status, int* flags, int* counter,
-    int chain_units, int c0) {
+    bf16* __restrict__ o, float* __restrict__ Sfg, int* status, unsigned long long* flags,
+    unsigned long long epoch, int c0) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ int32_t s_choff[kFusedMaxSeqs + 1];
     __shared__ int s_bad;
@@ -1179,13 +1209,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
     if ((int)blockIdx.x >= c0) {
         const int sub = tid >> 8;
         prep_worker(q, k, a, b, A_log, dt_bias, cu_seqlens, choff, N, H_qk, H_v, scale, rec,
-                    status, flags, sm + sub * kPrepRegion, tid & 255, 3 + sub,
+                    status, flags, epoch, sm + sub * kPrepRegion, tid & 255, 3 + sub,
                     2 * ((int)blockIdx.x - c0) + sub, 2 * ((int)gridDim.x - c0), false);
-        __syncthreads();  // both workers are done and have freed their TMEM
+        return;
     }
     if (tid >= kChainThreads) return;
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + CS_TMEM);
-    volatile int* s_unit = reinterpret_cast<volatile int*>(sm + CS_ERR + 8);
     if ((tid >> 5) == 0) {
         tmem_alloc(s_tmem, kTmemCols);
         tmem_relinquish();
@@ -1194,16 +1223,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
     named_bar_sync(kChainSync, kChainThreads);
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
-#pragma unroll 1
-    for (;;) {
-        if (tid == 0) *s_unit = atomicAdd(counter, 1);
-        named_bar_sync(kChainSync, kChainThreads);
-        const int u = *s_unit;
-        named_bar_sync(kChainSync, kChainThreads);
-        if (u >= chain_units) break;
-        chain_unit(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v, rec, o,
-                   Sfg, status, flags, sm, tid, u / H_v, u % H_v, tmem, kChainSync);
-    }
+    const int u = (int)blockIdx.x;
+    chain_unit(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v, rec, o, Sfg,
+               status, flags, epoch, sm, tid, u / H_v, u % H_v, tmem, kChainSync);
     tc_fence_before();
     named_bar_sync(kChainSync, kChainThreads);
     tc_fence_after();
@@ -1212,17 +1234,16 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-// Workspace: chunk offsets [N + 1] | record flags [records] | counter | records.
+// Workspace: chunk offsets [N + 1] | record flags [records] (64-bit call numbers) | records.
 struct TcWorkspace {
-    size_t off_flags, off_counter, off_rec, total;
+    size_t off_flags, off_rec, total;
 };
 
 TcWorkspace tc_workspace_layout(int32_t N, int64_t T, int32_t H_v) {
     const size_t records = ((size_t)((T + kC - 1) / kC) + (size_t)N) * H_v;
     TcWorkspace w;
     w.off_flags = align256((size_t)(N + 1) * sizeof(int32_t));
-    w.off_counter = w.off_flags + align256(records * sizeof(int32_t));
-    w.off_rec = w.off_counter + 256;
+    w.off_rec = w.off_flags + align256(records * sizeof(unsigned long long));
     w.total = w.off_rec + records * kRecBytes;
     return w;
 }
@@ -1280,8 +1301,7 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
     const TcWorkspace ws = tc_workspace_layout(N, T, H_v);
     uint8_t* wb = static_cast<uint8_t*>(workspace);
     int32_t* choff = reinterpret_cast<int32_t*>(wb);
-    int* flags = reinterpret_cast<int*>(wb + ws.off_flags);
-    int* counter = reinterpret_cast<int*>(wb + ws.off_counter);
+    unsigned long long* flags = reinterpret_cast<unsigned long long*>(wb + ws.off_flags);
     uint8_t* rec = wb + ws.off_rec;
     // With no tokens the maps are never read; any aligned device address will do.
     CUtensorMap tm_q, tm_k, tm_v, tm_o;
@@ -1313,16 +1333,16 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
         // phases at full occupancy.
         if (grid >= 2 && 2 * chain_units <= grid && N <= kFusedMaxSeqs) {
             const int c0 = (int)chain_units;
-            e = cudaMemsetAsync(wb + ws.off_flags, 0, ws.off_rec - ws.off_flags, s);
-            if (e != cudaSuccess) return e;
+            // this call's number: above every number an earlier call wrote
+            static std::atomic<unsigned long long> call_number{0};
+            unsigned long long epoch = call_number.fetch_add(1) + 1;
             const bf16* qb = static_cast<const bf16*>(q);
             const bf16* kb = static_cast<const bf16*>(k);
             bf16* ob = static_cast<bf16*>(o);
-            int units = (int)chain_units;
             int c0v = c0;
             void* args[] = {&tm_q, &tm_k, &tm_v, &tm_o, &qb, &kb, &a, &b, &A_log, &dt_bias, &S0,
                             &cu_seqlens, &choff, &N, &T, &H_qk, &H_v, &scale, &rec, &ob,
-                            &S_final, &status, &flags, &counter, &units, &c0v};
+                            &S_final, &status, &flags, &epoch, &c0v};
             ktimer_before(s);
             e = cudaLaunchCooperativeKernel((const void*)fused_kernel, dim3(grid),
                                             dim3(kFusedThreads), args, kFusedSmem, s);

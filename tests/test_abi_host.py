@@ -44,9 +44,9 @@ def test_status_strings(lib):
 def test_workspace_size(lib):
     ws = lib.gdn_prefill_workspace_size
     a256 = lambda x: (x + 255) // 256 * 256
-    # d = 128: chunk offsets (N + 1 int32), a flag per record, a counter block, and one
+    # d = 128: chunk offsets (N + 1 int32), an 8-byte flag per record, and one
     # 17,664-byte record per (chunk, V head), with at most ceil(T / 64) + N chunks
-    tc = lambda N, recs: a256((N + 1) * 4) + a256(recs * 4) + 256 + recs * 17664
+    tc = lambda N, recs: a256((N + 1) * 4) + a256(recs * 8) + recs * 17664
     assert ws(1, 4096, 16, 32, 128, 128) == tc(1, (64 + 1) * 32)
     assert ws(4, 4 * 16384, 16, 64, 128, 128) == tc(4, (1024 + 4) * 64)
     # never below the CUDA-core path's need (G and beta, fp32 [T, H_v] each)
