@@ -79,6 +79,19 @@ def test_conv_varlen_cache_bias(K, dtype):
     np.testing.assert_array_equal(_np(so), so_ref)
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_conv_narrow_channels(dtype):
+    """conv_dim = 24 (three 8-channel vectors): one warp spans several token tiles and the
+    grid's last block is partly empty (bf16 and fp32)."""
+    lens = [70, 0, 2, 33]
+    M = make_mixer_inputs(lens, H_qk=1, H_v=1, d_k=8, d_v=8, io_dtype=dtype, seed=14)
+    assert M.x.shape[1] == 24
+    y, so = _conv(M, bias=True)
+    y_ref, so_ref = _conv_ref(M, bias=True)
+    _close(y, y_ref, dtype)
+    np.testing.assert_array_equal(_np(so), so_ref)
+
+
 def test_conv_no_state_out_and_zero_cache():
     M = make_mixer_inputs([7, 300, 1], H_qk=2, H_v=4, d_k=64, d_v=64, seed=3)
     y, so = _conv(M, cache=False, want_state=False)
