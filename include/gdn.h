@@ -142,7 +142,12 @@ int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
  *                         chunk chain as separate launches always (by default
  *                         they run in one cooperative launch, overlapped, when
  *                         the device supports it and there are at most half as
- *                         many (sequence, V head) chains as SMs).
+ *                         many (sequence, V head) chains as SMs; with at most a
+ *                         quarter as many, each chain is split over two blocks
+ *                         that own 64 value rows each);
+ *   GDN_IMPL_TENSOR_CORE_WHOLE_ROWS
+ *                         the one-launch schedule whenever it applies, but never
+ *                         with half-row chain blocks.
  * Returns the previous setting, or -GDN_ERR_INVALID_ARG for an unknown value.
  * Not synchronised with calls in flight on other host threads.
  */
@@ -150,7 +155,8 @@ enum {
     GDN_IMPL_AUTO = 0,
     GDN_IMPL_CUDA_CORE = 1,
     GDN_IMPL_TENSOR_CORE = 2,
-    GDN_IMPL_TENSOR_CORE_SPLIT = 3
+    GDN_IMPL_TENSOR_CORE_SPLIT = 3,
+    GDN_IMPL_TENSOR_CORE_WHOLE_ROWS = 4
 };
 int gdn_set_prefill_impl(int32_t impl);
 

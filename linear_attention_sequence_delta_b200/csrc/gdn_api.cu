@@ -173,7 +173,8 @@ int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
     const int impl = g_prefill_impl.load(std::memory_order_relaxed);
     const bool tc_ok =
         io_dtype == GDN_BF16 && d_k == 128 && prefill_tc_supported(H_qk, H_v);
-    if ((impl == GDN_IMPL_TENSOR_CORE || impl == GDN_IMPL_TENSOR_CORE_SPLIT) && !tc_ok)
+    if ((impl == GDN_IMPL_TENSOR_CORE || impl == GDN_IMPL_TENSOR_CORE_SPLIT ||
+         impl == GDN_IMPL_TENSOR_CORE_WHOLE_ROWS) && !tc_ok)
         return GDN_ERR_UNSUPPORTED;
     int* st = device_status_ptr();
     if (!st) return GDN_ERR_CUDA;
@@ -183,7 +184,9 @@ int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
         return to_status(launch_prefill_tc(q, k, v, a, b, A_log, dt_bias, initial_state,
                                            cu_seqlens, num_seqs, total_tokens, H_qk, H_v, scale,
                                            o, final_state, workspace,
-                                           impl != GDN_IMPL_TENSOR_CORE_SPLIT, st, s));
+                                           impl == GDN_IMPL_TENSOR_CORE_SPLIT ? 0
+                                           : impl == GDN_IMPL_TENSOR_CORE_WHOLE_ROWS ? 1 : 2,
+                                           st, s));
     }
     float* G = static_cast<float*>(workspace);
     float* beta = reinterpret_cast<float*>(static_cast<char*>(workspace) +
@@ -334,7 +337,7 @@ int gdn_rmsnorm_gated(const void* o, const void* z, int32_t io_dtype, const floa
 
 int gdn_set_prefill_impl(int32_t impl) {
     if (impl != GDN_IMPL_AUTO && impl != GDN_IMPL_CUDA_CORE && impl != GDN_IMPL_TENSOR_CORE &&
-        impl != GDN_IMPL_TENSOR_CORE_SPLIT)
+        impl != GDN_IMPL_TENSOR_CORE_SPLIT && impl != GDN_IMPL_TENSOR_CORE_WHOLE_ROWS)
         return -GDN_ERR_INVALID_ARG;
     return g_prefill_impl.exchange(impl);
 }

@@ -113,7 +113,9 @@ cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, int
                                 int* status, cudaStream_t s);
 
 // Tensor-core prefill (bf16 I/O, d = 128): chunk offsets, the state-independent
-// prep kernel, then the chain kernel. The workspace holds the chunk offsets and
+// prep kernel, then the chain kernel. schedule: 0 = always separate launches, 1 = one
+// cooperative launch where it pays (whole-row chain blocks), 2 = the same with half-row
+// chain blocks when the chains are few enough. The workspace holds the chunk offsets and
 // one record (T, P and per-token factors) per (chunk, V head).
 size_t prefill_tc_workspace_bytes(int32_t N, int64_t T, int32_t H_v);
 bool prefill_tc_supported(int32_t H_qk, int32_t H_v);
@@ -121,7 +123,7 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
                               const float* b, const float* A_log, const float* dt_bias,
                               const float* S0, const int32_t* cu_seqlens, int32_t N, int64_t T,
                               int32_t H_qk, int32_t H_v, float scale, void* o, float* S_final,
-                              void* workspace, bool fused, int* status, cudaStream_t s);
+                              void* workspace, int schedule, int* status, cudaStream_t s);
 
 // Steps around the delta rule (gdn_mixer.cu): causal depthwise conv1d + SiLU with
 // the per-sequence conv cache, its single-token decode form, and the gated RMSNorm.

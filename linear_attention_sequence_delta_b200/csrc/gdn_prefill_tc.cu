@@ -677,14 +677,16 @@ __device__ __forceinline__ bool wait_record(const unsigned long long* flag,
 // threads of a block (tid 0 .. 415, synchronised by the named barrier sync_id) on
 // the tensor memory `tmem` (512 columns). With `flags`, a chunk's record is
 // copied only once a prep worker has published it.
+template <int kM>
 __device__ __forceinline__ void chain_unit(
     const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
     const CUtensorMap& tm_o, const float* __restrict__ S0g, const int32_t* __restrict__ cu_seqlens,
     const int32_t* __restrict__ choff, int64_t T_total, int H_qk, int H_v,
     const uint8_t* __restrict__ rec, bf16* __restrict__ o, float* __restrict__ Sfg, int* status,
     const unsigned long long* flags, unsigned long long epoch, uint8_t* sm, const int tid,
-    const int n, const int h, const uint32_t tmem,
+    const int n, const int h, const int hv, const uint32_t tmem,
     const int sync_id) {
+    static_assert(kM == 128 || kM == 64, "a chain block owns all 128 value rows or one half");
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + CS_BAR);  // [3] slot landed
     uint64_t* mbar = full + kRing;         // chain MMA completions
     uint64_t* obar = mbar + 1;             // [2] chunk parity b: output accumulators complete
@@ -795,30 +797,56 @@ __device__ __forceinline__ void chain_unit(
             tc_fence_after();
             const float4* eg4 = reinterpret_cast<const float4*>(egq);
             const uint32_t qacc = ctl + (b ? TM_D1Q1 : TM_D1Q0);
-            // this thread's column of the staged tile; laundered so that the 64 element
-            // addresses are formed per chunk rather than held in registers across chunks
-            uint32_t ocol = smem_u32(ost) + (uint32_t)(row >> 6) * 8192u + (uint32_t)(row & 7) * 2u;
-            uint32_t ochk = (uint32_t)((row & 63) >> 3);
-            asm volatile("" : "+r"(ocol), "+r"(ochk));
+            if constexpr (kM == 128) {
+                // this thread's column of the staged tile; laundered so that the 64 element
+                // addresses are formed per chunk rather than held in registers across chunks
+                uint32_t ocol = smem_u32(ost) + (uint32_t)(row >> 6) * 8192u + (uint32_t)(row & 7) * 2u;
+                uint32_t ochk = (uint32_t)((row & 63) >> 3);
+                asm volatile("" : "+r"(ocol), "+r"(ochk));
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                float xq[32], xi[32];
-                tmem_ld32x2_sync(qacc + 32 * hf, ctl + TM_D4 + 32 * hf, xq, xi);
-                if (hf == 1) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&ofree[b]);  // the accumulators may be overwritten
+                for (int hf = 0; hf < 2; ++hf) {
+                    float xq[32], xi[32];
+                    tmem_ld32x2_sync(qacc + 32 * hf, ctl + TM_D4 + 32 * hf, xq, xi);
+                    if (hf == 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&ofree[b]);  // the accumulators may be overwritten
+                    }
+#pragma unroll
+                    for (int e4 = 0; e4 < 8; ++e4) {
+                        const float4 w = eg4[8 * hf + e4];
+                        const float wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int t = 32 * hf + 4 * e4 + u, e = 4 * e4 + u;
+                            const uint32_t a = ocol + (uint32_t)t * 128u + ((ochk ^ (uint32_t)(t & 7)) << 4);
+                            const bf16 v = __float2bfloat16_rn(fmaf(wv[u], xq[e], xi[e]));
+                            asm volatile("st.shared.b16 [%0], %1;" ::"r"(a),
+                                         "h"(*reinterpret_cast<const unsigned short*>(&v))
+                                         : "memory");
+                        }
+                    }
                 }
+            } else {
+                // value rows r0 = 16 qo + lane / 4 and r0 + 8 of this block's half; tokens
+                // 8 j + 2 (lane % 4) and + 1 (16-lane accumulator layout)
+                float xq[32], xi[32];
+                tmem_ld16r_x8x2_sync(qacc, ctl + TM_D4, xq, xi);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ofree[b]);  // the accumulators may be overwritten
+                const int r0 = qo * 16 + (lane >> 2), tp = 2 * (lane & 3);
+                uint32_t obase = smem_u32(ost);
+                asm volatile("" : "+r"(obase));
 #pragma unroll
-                for (int e4 = 0; e4 < 8; ++e4) {
-                    const float4 w = eg4[8 * hf + e4];
-                    const float wv[4] = {w.x, w.y, w.z, w.w};
+                for (int jj = 0; jj < 8; ++jj) {
+                    const float2 w = reinterpret_cast<const float2*>(egq)[4 * jj + (lane & 3)];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int t = 32 * hf + 4 * e4 + u, e = 4 * e4 + u;
-                        const uint32_t a = ocol + (uint32_t)t * 128u + ((ochk ^ (uint32_t)(t & 7)) << 4);
-                        const bf16 v = __float2bfloat16_rn(fmaf(wv[u], xq[e], xi[e]));
-                        asm volatile("st.shared.b16 [%0], %1;" ::"r"(a),
+                    for (int e = 0; e < 4; ++e) {
+                        const int t = 8 * jj + tp + (e & 1), r = r0 + 8 * (e >> 1);
+                        const float wt = (e & 1) ? w.y : w.x;
+                        const bf16 v = __float2bfloat16_rn(fmaf(wt, xq[4 * jj + e], xi[4 * jj + e]));
+                        asm volatile("st.shared.b16 [%0], %1;" ::"r"(obase + tile64_off(t, r)),
                                      "h"(*reinterpret_cast<const unsigned short*>(&v))
                                      : "memory");
                     }
@@ -828,18 +856,24 @@ __device__ __forceinline__ void chain_unit(
             named_bar_sync(2, kOut);  // staged; every output warp is done with the slot
             const int64_t t0 = s0 + (int64_t)cp * kC;
             const int L = (int)min((int64_t)kC, s1 - t0);
+            constexpr int kOutCh = kM / 8;  // 16-byte chunks per staged row
             if (L == kC) {
                 if (loader) {
-                    tma_store_3d(&tm_o, 0, h, (int32_t)t0, ost);
-                    tma_store_3d(&tm_o, 64, h, (int32_t)t0, ost + 8192);
+                    if constexpr (kM == 128) {
+                        tma_store_3d(&tm_o, 0, h, (int32_t)t0, ost);
+                        tma_store_3d(&tm_o, 64, h, (int32_t)t0, ost + 8192);
+                    } else {
+                        tma_store_3d(&tm_o, 64 * hv, h, (int32_t)t0, ost);
+                    }
                     bulk_commit_group();
                 }
             } else {
                 // the sequence's last rows only: plain 16-byte stores
-                for (int idx = to; idx < L * 16; idx += kOut) {
-                    const int r = idx >> 4, ch = idx & 15;
+                for (int idx = to; idx < L * kOutCh; idx += kOut) {
+                    const int r = idx / kOutCh, ch = idx % kOutCh;
                     const uint4 w = *reinterpret_cast<const uint4*>(ost + tile64_off(r, ch * 8));
-                    *reinterpret_cast<uint4*>(o + ((size_t)(t0 + r) * H_v + h) * kD + ch * 8) = w;
+                    *reinterpret_cast<uint4*>(o + ((size_t)(t0 + r) * H_v + h) * kD +
+                                              (kM == 64 ? 64 * hv : 0) + ch * 8) = w;
                 }
                 named_bar_sync(2, kOut);
             }
@@ -863,9 +897,9 @@ __device__ __forceinline__ void chain_unit(
             tc_fence_after();
         };
         bool dead = false;
-        constexpr uint32_t id64 = idesc_bf16_f32(128, 64, 0, 0);
-        constexpr uint32_t id_v = idesc_bf16_f32(128, 64, 1, 0);
-        constexpr uint32_t id_s = idesc_bf16_f32(128, 128, 0, 1);
+        constexpr uint32_t id64 = idesc_bf16_f32(kM, 64, 0, 0);
+        constexpr uint32_t id_v = idesc_bf16_f32(kM, 64, 1, 0);
+        constexpr uint32_t id_s = idesc_bf16_f32(kM, 128, 0, 1);
         // TMEM A operands (fixed for the whole unit)
         uint32_t aS0[4], aS1[4], aZ[4], aU[4], aN[4];
 #pragma unroll
@@ -896,7 +930,8 @@ __device__ __forceinline__ void chain_unit(
                 dK1[ks] = smem_desc_sw128(kq + 16384u + ks * 32u, 16, 1024);
                 dQ0[ks] = smem_desc_sw128(kq + 8192u + ks * 32u, 16, 1024);
                 dQ1[ks] = smem_desc_sw128(kq + 16384u + 8192u + ks * 32u, 16, 1024);
-                dV[ks] = smem_desc_sw128(vt + ks * 2048u, 8192, 1024);
+                // V^T rows = value rows: this block's half of them when kM = 64
+                dV[ks] = smem_desc_sw128(vt + (kM == 64 ? 8192u * hv : 0u) + ks * 2048u, 8192, 1024);
                 dT[ks] = smem_desc_sw128(tt + ks * 32u, 16, 1024);
                 dKm[ks] = smem_desc_sw128(kq + ks * 2048u, 16384, 1024);
                 dP[ks] = smem_desc_sw128(ptile + ks * 32u, 16, 1024);
@@ -953,160 +988,313 @@ __device__ __forceinline__ void chain_unit(
         }
         __syncwarp();
     } else {
-        // ================================ state ========================================
-        const int qd = warp & 3;              // TMEM lane quarter
-        const int hh = warp >> 2;             // column half
-        const int row = qd * 32 + lane;       // value row i = TMEM lane
-        const uint32_t ctl = tmem + ((uint32_t)(qd * 32) << 16);
-        const size_t sbase = ((size_t)n * H_v + h) * kD * kD + (size_t)row * kD + 64 * hh;
-        float S[64];  // S[i][64 hh + e]
-        if (S0g) {
-            const float4* src = reinterpret_cast<const float4*>(S0g + sbase);
+        if constexpr (kM == 128) {
+            // ================================ state ========================================
+            const int qd = warp & 3;              // TMEM lane quarter
+            const int hh = warp >> 2;             // column half
+            const int row = qd * 32 + lane;       // value row i = TMEM lane
+            const uint32_t ctl = tmem + ((uint32_t)(qd * 32) << 16);
+            const size_t sbase = ((size_t)n * H_v + h) * kD * kD + (size_t)row * kD + 64 * hh;
+            float S[64];  // S[i][64 hh + e]
+            if (S0g) {
+                const float4* src = reinterpret_cast<const float4*>(S0g + sbase);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const float4 f = src[e];
-                S[4 * e] = f.x; S[4 * e + 1] = f.y; S[4 * e + 2] = f.z; S[4 * e + 3] = f.w;
-            }
-        } else {
-#pragma unroll
-            for (int e = 0; e < 64; ++e) S[e] = 0.f;
-        }
-
-        uint32_t mphase = 0;
-        bool dead = false;  // warp-uniform: after an error only the barrier arrivals remain
-        auto wait_mma = [&]() {
-            if (dead) return;
-            bool ok = *s_err == 0 && mbar_wait_bounded(mbar, mphase, kWaitCycles);
-            mphase ^= 1u;
-            dead = __any_sync(0xffffffffu, !ok || *s_err != 0);
-            if (dead) *s_err = 1;
-            tc_fence_after();
-        };
-        // this warp's TMEM operands of the step are written (and, before that, any
-        // shared-memory writes fenced): arrive for the issuing warp, always. After an
-        // error the arrival waits for the barrier to complete, so that no thread can
-        // run a barrier generation ahead of the issuing warp.
-        auto signal_rdy = [&]() {
-            if (!dead) tmem_wait_st();
-            tc_fence_before();
-            if (dead) named_bar_sync(kRdyBar, kRdyCount);
-            else named_bar_arrive(kRdyBar, kRdyCount);
-        };
-        // S <- gamma S + U (the previous chunk's decay and increment)
-        auto apply_update = [&](float gamma) {
-#pragma unroll
-            for (int cb = 0; cb < 2; ++cb) {
-                float u[32];
-                tmem_ld32_sync(ctl + TM_U + 64 * hh + 32 * cb, u);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) S[32 * cb + e] = fmaf(gamma, S[32 * cb + e], u[e]);
-            }
-        };
-
-        float gamma = 1.f;
-#pragma unroll 1
-        for (int c = 0; c < nchunks; ++c) {
-            const int st = c % kRing;
-            uint8_t* slot = sm + st * kSlotBytes;
-            const float* rg = reinterpret_cast<const float*>(slot + SLOT_REC + REC_G);
-            const int64_t t0 = s0 + (int64_t)c * kC;
-            const int L = (int)min((int64_t)kC, s1 - t0);
-
-            // ---- the previous chunk's state update and this chunk's data -------------
-            if (c > 0) {
-                wait_mma();
-                if (!dead) apply_update(gamma);
-            }
-            if (!dead) {
-                const bool okf =
-                    *s_err == 0 && mbar_wait_bounded(&full[st], (c / kRing) & 1, kWaitCycles);
-                dead = __any_sync(0xffffffffu, !okf || *s_err != 0);
-                if (dead) *s_err = 1;
-            }
-            if (!dead && L < kC) {
-                // rows past the sequence's end hold the next sequence's tokens (or TMA
-                // zero fill): zero them
-                const int nz = (kC - L) * 8;  // 16-byte chunks per 64-column tile
-                for (int idx = tid; idx < 6 * nz; idx += kChain) {
-                    const int tile = idx / nz, r = L + (idx % nz) / 8, ch = idx & 7;
-                    const uint32_t base = tile < 4 ? SLOT_KQ + (tile >> 1) * 16384u + (tile & 1) * 8192u
-                                                   : SLOT_V + (tile - 4) * 8192u;
-                    *reinterpret_cast<uint4*>(slot + base + r * 128 + ch * 16) =
-                        make_uint4(0u, 0u, 0u, 0u);
+                for (int e = 0; e < 16; ++e) {
+                    const float4 f = src[e];
+                    S[4 * e] = f.x; S[4 * e + 1] = f.y; S[4 * e + 2] = f.z; S[4 * e + 3] = f.w;
                 }
-                fence_proxy_async_smem();
+            } else {
+#pragma unroll
+                for (int e = 0; e < 64; ++e) S[e] = 0.f;
             }
 
-            // ---- state: bf16 copy (A operand of S0 K^T and S0 Q^T) ----------------------
-            if (!dead) {
+            uint32_t mphase = 0;
+            bool dead = false;  // warp-uniform: after an error only the barrier arrivals remain
+            auto wait_mma = [&]() {
+                if (dead) return;
+                bool ok = *s_err == 0 && mbar_wait_bounded(mbar, mphase, kWaitCycles);
+                mphase ^= 1u;
+                dead = __any_sync(0xffffffffu, !ok || *s_err != 0);
+                if (dead) *s_err = 1;
+                tc_fence_after();
+            };
+            // this warp's TMEM operands of the step are written (and, before that, any
+            // shared-memory writes fenced): arrive for the issuing warp, always. After an
+            // error the arrival waits for the barrier to complete, so that no thread can
+            // run a barrier generation ahead of the issuing warp.
+            auto signal_rdy = [&]() {
+                if (!dead) tmem_wait_st();
+                tc_fence_before();
+                if (dead) named_bar_sync(kRdyBar, kRdyCount);
+                else named_bar_arrive(kRdyBar, kRdyCount);
+            };
+            // S <- gamma S + U (the previous chunk's decay and increment)
+            auto apply_update = [&](float gamma) {
 #pragma unroll
                 for (int cb = 0; cb < 2; ++cb) {
+                    float u[32];
+                    tmem_ld32_sync(ctl + TM_U + 64 * hh + 32 * cb, u);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) S[32 * cb + e] = fmaf(gamma, S[32 * cb + e], u[e]);
+                }
+            };
+
+            float gamma = 1.f;
+#pragma unroll 1
+            for (int c = 0; c < nchunks; ++c) {
+                const int st = c % kRing;
+                uint8_t* slot = sm + st * kSlotBytes;
+                const float* rg = reinterpret_cast<const float*>(slot + SLOT_REC + REC_G);
+                const int64_t t0 = s0 + (int64_t)c * kC;
+                const int L = (int)min((int64_t)kC, s1 - t0);
+
+                // ---- the previous chunk's state update and this chunk's data -------------
+                if (c > 0) {
+                    wait_mma();
+                    if (!dead) apply_update(gamma);
+                }
+                if (!dead) {
+                    const bool okf =
+                        *s_err == 0 && mbar_wait_bounded(&full[st], (c / kRing) & 1, kWaitCycles);
+                    dead = __any_sync(0xffffffffu, !okf || *s_err != 0);
+                    if (dead) *s_err = 1;
+                }
+                if (!dead && L < kC) {
+                    // rows past the sequence's end hold the next sequence's tokens (or TMA
+                    // zero fill): zero them
+                    const int nz = (kC - L) * 8;  // 16-byte chunks per 64-column tile
+                    for (int idx = tid; idx < 6 * nz; idx += kChain) {
+                        const int tile = idx / nz, r = L + (idx % nz) / 8, ch = idx & 7;
+                        const uint32_t base = tile < 4 ? SLOT_KQ + (tile >> 1) * 16384u + (tile & 1) * 8192u
+                                                       : SLOT_V + (tile - 4) * 8192u;
+                        *reinterpret_cast<uint4*>(slot + base + r * 128 + ch * 16) =
+                            make_uint4(0u, 0u, 0u, 0u);
+                    }
+                    fence_proxy_async_smem();
+                }
+
+                // ---- state: bf16 copy (A operand of S0 K^T and S0 Q^T) ----------------------
+                if (!dead) {
+#pragma unroll
+                    for (int cb = 0; cb < 2; ++cb) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            pk[e] = pack_bf16x2(S[32 * cb + 2 * e], S[32 * cb + 2 * e + 1]);
+                        tmem_st16(ctl + TM_S0B + 32 * hh + 16 * cb, pk);
+                    }
+                }
+                signal_rdy();
+                if (!dead) gamma = rg[RG_GAMMA];
+
+                // ---- Z^T = -(e^G rk) (S0 K^T) for this thread's 32 tokens, in place ----------
+                wait_mma();  // S0 K^T
+                if (!dead) {
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {  // 16 tokens at a time
+                        const float4* fk4 = reinterpret_cast<const float4*>(rg + RG_FK) + 8 * hh + 4 * q;
+                        float x[16];
+                        tmem_ld16_sync(ctl + TM_D1K + 32 * hh + 16 * q, x);
+                        uint32_t pk[8];
+#pragma unroll
+                        for (int e4 = 0; e4 < 4; ++e4) {
+                            const float4 f = fk4[e4];
+                            pk[2 * e4] = pack_bf16x2(-f.x * x[4 * e4], -f.y * x[4 * e4 + 1]);
+                            pk[2 * e4 + 1] = pack_bf16x2(-f.z * x[4 * e4 + 2], -f.w * x[4 * e4 + 3]);
+                        }
+                        // over columns this thread has already read
+                        tmem_st8(ctl + TM_D1K + 32 * hh + 8 * q, pk);
+                    }
+                }
+                signal_rdy();
+
+                // ---- Vn^T -> bf16 pairs (for P Vn) and decay-scaled pairs (state update) --
+                wait_mma();  // Vn^T
+                if (!dead) {
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const float4* egl4 =
+                            reinterpret_cast<const float4*>(rg + RG_EGL) + 8 * hh + 4 * q;
+                        float x[16];
+                        tmem_ld16_sync(ctl + TM_D3 + 32 * hh + 16 * q, x);
+                        uint32_t pk[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) pk[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
+                        tmem_st8(ctl + TM_D3 + 32 * hh + 8 * q, pk);  // over Vn^T columns read
+#pragma unroll
+                        for (int e4 = 0; e4 < 4; ++e4) {
+                            const float4 w = egl4[e4];
+                            pk[2 * e4] = pack_bf16x2(x[4 * e4] * w.x, x[4 * e4 + 1] * w.y);
+                            pk[2 * e4 + 1] = pack_bf16x2(x[4 * e4 + 2] * w.z, x[4 * e4 + 3] * w.w);
+                        }
+                        tmem_st8(ctl + TM_D1K + 16 * hh + 8 * q, pk);  // Z^T there is consumed
+                    }
+                }
+                signal_rdy();
+            }
+            bool done = !dead;
+            if (done && nchunks > 0) {  // the last chunk's state update
+                wait_mma();
+                done = !dead;
+                if (done) apply_update(gamma);
+            }
+            if (done && Sfg) {
+                float4* d4 = reinterpret_cast<float4*>(Sfg + sbase);
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    d4[e] = make_float4(S[4 * e], S[4 * e + 1], S[4 * e + 2], S[4 * e + 3]);
+            }
+        } else {
+            // ======================= state, one half of the value rows =======================
+            // The block's 64 value rows 64 hv .. 64 hv + 63 sit in TMEM lanes 0-15 of each lane
+            // quarter (M = 64 layout): warp w takes quarter qd = w & 3 (rows 16 qd ..) and the
+            // column half hh = w >> 2 of every quantity; a thread holds rows r0 and r0 + 8 and,
+            // of each 8-column group, the column pair 2 (lane % 4), + 1 (16-lane accesses).
+            const int qd = warp & 3;
+            const int hh = warp >> 2;
+            const int r0 = 64 * hv + qd * 16 + (lane >> 2);  // value row of registers e = 0, 1
+            const int cp2 = 2 * (lane & 3);
+            const uint32_t ctl = tmem + ((uint32_t)(qd * 32) << 16);
+            const size_t hbase = ((size_t)n * H_v + h) * kD * kD;
+            float S[32];  // S[4 j + e]: row r0 + 8 (e >> 1), column 64 hh + 8 j + cp2 + (e & 1)
+            if (S0g) {
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    const int col = 64 * hh + 8 * jj + cp2;
+                    const float2 f0 = *reinterpret_cast<const float2*>(S0g + hbase + (size_t)r0 * kD + col);
+                    const float2 f1 =
+                        *reinterpret_cast<const float2*>(S0g + hbase + (size_t)(r0 + 8) * kD + col);
+                    S[4 * jj] = f0.x; S[4 * jj + 1] = f0.y; S[4 * jj + 2] = f1.x; S[4 * jj + 3] = f1.y;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) S[e] = 0.f;
+            }
+
+            uint32_t mphase = 0;
+            bool dead = false;  // warp-uniform: after an error only the barrier arrivals remain
+            auto wait_mma = [&]() {
+                if (dead) return;
+                bool ok = *s_err == 0 && mbar_wait_bounded(mbar, mphase, kWaitCycles);
+                mphase ^= 1u;
+                dead = __any_sync(0xffffffffu, !ok || *s_err != 0);
+                if (dead) *s_err = 1;
+                tc_fence_after();
+            };
+            // as in the full-row variant: arrive for the issuing warp, always
+            auto signal_rdy = [&]() {
+                if (!dead) tmem_wait_st();
+                tc_fence_before();
+                if (dead) named_bar_sync(kRdyBar, kRdyCount);
+                else named_bar_arrive(kRdyBar, kRdyCount);
+            };
+            // S <- gamma S + U (the previous chunk's decay and increment)
+            auto apply_update = [&](float gamma) {
+                float u[32];
+                tmem_ld16r_x8_sync(ctl + TM_U + 64 * hh, u);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) S[e] = fmaf(gamma, S[e], u[e]);
+            };
+
+            float gamma = 1.f;
+#pragma unroll 1
+            for (int c = 0; c < nchunks; ++c) {
+                const int st = c % kRing;
+                uint8_t* slot = sm + st * kSlotBytes;
+                const float* rg = reinterpret_cast<const float*>(slot + SLOT_REC + REC_G);
+                const int64_t t0 = s0 + (int64_t)c * kC;
+                const int L = (int)min((int64_t)kC, s1 - t0);
+
+                // ---- the previous chunk's state update and this chunk's data -------------
+                if (c > 0) {
+                    wait_mma();
+                    if (!dead) apply_update(gamma);
+                }
+                if (!dead) {
+                    const bool okf =
+                        *s_err == 0 && mbar_wait_bounded(&full[st], (c / kRing) & 1, kWaitCycles);
+                    dead = __any_sync(0xffffffffu, !okf || *s_err != 0);
+                    if (dead) *s_err = 1;
+                }
+                if (!dead && L < kC) {
+                    // rows past the sequence's end hold the next sequence's tokens (or TMA
+                    // zero fill): zero them
+                    const int nz = (kC - L) * 8;  // 16-byte chunks per 64-column tile
+                    for (int idx = tid; idx < 6 * nz; idx += kChain) {
+                        const int tile = idx / nz, r = L + (idx % nz) / 8, ch = idx & 7;
+                        const uint32_t base = tile < 4 ? SLOT_KQ + (tile >> 1) * 16384u + (tile & 1) * 8192u
+                                                       : SLOT_V + (tile - 4) * 8192u;
+                        *reinterpret_cast<uint4*>(slot + base + r * 128 + ch * 16) =
+                            make_uint4(0u, 0u, 0u, 0u);
+                    }
+                    fence_proxy_async_smem();
+                }
+
+                // ---- state: bf16 pairs (A operand of S0 K^T and S0 Q^T), key k at column k/2
+                if (!dead) {
                     uint32_t pk[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        pk[e] = pack_bf16x2(S[32 * cb + 2 * e], S[32 * cb + 2 * e + 1]);
-                    tmem_st16(ctl + TM_S0B + 32 * hh + 16 * cb, pk);
+                    for (int jj = 0; jj < 8; ++jj) {
+                        pk[2 * jj] = pack_bf16x2(S[4 * jj], S[4 * jj + 1]);
+                        pk[2 * jj + 1] = pack_bf16x2(S[4 * jj + 2], S[4 * jj + 3]);
+                    }
+                    tmem_st16r_x8(ctl + TM_S0B + 32 * hh, pk);
                 }
-            }
-            signal_rdy();
-            if (!dead) gamma = rg[RG_GAMMA];
+                signal_rdy();
+                if (!dead) gamma = rg[RG_GAMMA];
 
-            // ---- Z^T = -(e^G rk) (S0 K^T) for this thread's 32 tokens, in place ----------
-            wait_mma();  // S0 K^T
-            if (!dead) {
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {  // 16 tokens at a time
-                    const float4* fk4 = reinterpret_cast<const float4*>(rg + RG_FK) + 8 * hh + 4 * q;
+                // ---- Z^T = -(e^G rk) (S0 K^T) for this thread's tokens 32 hh + 8 j + cp2, + 1
+                wait_mma();  // S0 K^T
+                if (!dead) {
                     float x[16];
-                    tmem_ld16_sync(ctl + TM_D1K + 32 * hh + 16 * q, x);
+                    tmem_ld16r_x4_sync(ctl + TM_D1K + 32 * hh, x);
                     uint32_t pk[8];
 #pragma unroll
-                    for (int e4 = 0; e4 < 4; ++e4) {
-                        const float4 f = fk4[e4];
-                        pk[2 * e4] = pack_bf16x2(-f.x * x[4 * e4], -f.y * x[4 * e4 + 1]);
-                        pk[2 * e4 + 1] = pack_bf16x2(-f.z * x[4 * e4 + 2], -f.w * x[4 * e4 + 3]);
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const float2 f = *reinterpret_cast<const float2*>(rg + RG_FK + 32 * hh + 8 * jj + cp2);
+                        pk[2 * jj] = pack_bf16x2(-f.x * x[4 * jj], -f.y * x[4 * jj + 1]);
+                        pk[2 * jj + 1] = pack_bf16x2(-f.x * x[4 * jj + 2], -f.y * x[4 * jj + 3]);
                     }
-                    // over columns this thread has already read
-                    tmem_st8(ctl + TM_D1K + 32 * hh + 8 * q, pk);
+                    // over the columns just read: pairs of tokens 32 hh + 16 q .. at 32 hh + 8 q
+                    tmem_st16r_x4(ctl + TM_D1K + 32 * hh, pk);
                 }
-            }
-            signal_rdy();
+                signal_rdy();
 
-            // ---- Vn^T -> bf16 pairs (for P Vn) and decay-scaled pairs (state update) --
-            wait_mma();  // Vn^T
-            if (!dead) {
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const float4* egl4 =
-                        reinterpret_cast<const float4*>(rg + RG_EGL) + 8 * hh + 4 * q;
+                // ---- Vn^T -> bf16 pairs (for P Vn) and decay-scaled pairs (state update) --
+                wait_mma();  // Vn^T
+                if (!dead) {
                     float x[16];
-                    tmem_ld16_sync(ctl + TM_D3 + 32 * hh + 16 * q, x);
-                    uint32_t pk[8];
+                    tmem_ld16r_x4_sync(ctl + TM_D3 + 32 * hh, x);
+                    uint32_t pk[8], pw[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) pk[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
-                    tmem_st8(ctl + TM_D3 + 32 * hh + 8 * q, pk);  // over Vn^T columns read
-#pragma unroll
-                    for (int e4 = 0; e4 < 4; ++e4) {
-                        const float4 w = egl4[e4];
-                        pk[2 * e4] = pack_bf16x2(x[4 * e4] * w.x, x[4 * e4 + 1] * w.y);
-                        pk[2 * e4 + 1] = pack_bf16x2(x[4 * e4 + 2] * w.z, x[4 * e4 + 3] * w.w);
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const float2 w = *reinterpret_cast<const float2*>(rg + RG_EGL + 32 * hh + 8 * jj + cp2);
+                        pk[2 * jj] = pack_bf16x2(x[4 * jj], x[4 * jj + 1]);
+                        pk[2 * jj + 1] = pack_bf16x2(x[4 * jj + 2], x[4 * jj + 3]);
+                        pw[2 * jj] = pack_bf16x2(x[4 * jj] * w.x, x[4 * jj + 1] * w.y);
+                        pw[2 * jj + 1] = pack_bf16x2(x[4 * jj + 2] * w.x, x[4 * jj + 3] * w.y);
                     }
-                    tmem_st8(ctl + TM_D1K + 16 * hh + 8 * q, pk);  // Z^T there is consumed
+                    tmem_st16r_x4(ctl + TM_D3 + 32 * hh, pk);   // over Vn^T columns read
+                    tmem_st16r_x4(ctl + TM_D1K + 16 * hh, pw);  // Z^T there is consumed
+                }
+                signal_rdy();
+            }
+            bool done = !dead;
+            if (done && nchunks > 0) {  // the last chunk's state update
+                wait_mma();
+                done = !dead;
+                if (done) apply_update(gamma);
+            }
+            if (done && Sfg) {
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    const int col = 64 * hh + 8 * jj + cp2;
+                    *reinterpret_cast<float2*>(Sfg + hbase + (size_t)r0 * kD + col) =
+                        make_float2(S[4 * jj], S[4 * jj + 1]);
+                    *reinterpret_cast<float2*>(Sfg + hbase + (size_t)(r0 + 8) * kD + col) =
+                        make_float2(S[4 * jj + 2], S[4 * jj + 3]);
                 }
             }
-            signal_rdy();
-        }
-        bool done = !dead;
-        if (done && nchunks > 0) {  // the last chunk's state update
-            wait_mma();
-            done = !dead;
-            if (done) apply_update(gamma);
-        }
-        if (done && Sfg) {
-            float4* d4 = reinterpret_cast<float4*>(Sfg + sbase);
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-                d4[e] = make_float4(S[4 * e], S[4 * e + 1], S[4 * e + 2], S[4 * e + 3]);
         }
     }
 
@@ -1135,8 +1323,9 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
-    chain_unit(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v, rec, o, Sfg,
-               status, nullptr, 0, sm, threadIdx.x, blockIdx.x / H_v, blockIdx.x % H_v, tmem, 1);
+    chain_unit<128>(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v, rec, o,
+                    Sfg, status, nullptr, 0, sm, threadIdx.x, blockIdx.x / H_v, blockIdx.x % H_v,
+                    0, tmem, 1);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1159,6 +1348,7 @@ constexpr size_t kFusedSmem =
 constexpr int kChainSync = 5;  // named barrier of the chain threads in the fused kernel
 constexpr int kFusedMaxSeqs = 255;  // the fused kernel computes the chunk offsets itself
 
+template <int kM>
 __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -1223,9 +1413,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
     named_bar_sync(kChainSync, kChainThreads);
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
-    const int u = (int)blockIdx.x;
-    chain_unit(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v, rec, o, Sfg,
-               status, flags, epoch, sm, tid, u / H_v, u % H_v, tmem, kChainSync);
+    // block u: (sequence, V head) u, or with half-row blocks its half u & 1 of unit u >> 1
+    const int u = kM == 64 ? (int)blockIdx.x >> 1 : (int)blockIdx.x;
+    const int hv = kM == 64 ? (int)blockIdx.x & 1 : 0;
+    chain_unit<kM>(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v, rec, o,
+                   Sfg, status, flags, epoch, sm, tid, u / H_v, u % H_v, hv, tmem, kChainSync);
     tc_fence_before();
     named_bar_sync(kChainSync, kChainThreads);
     tc_fence_after();
@@ -1295,7 +1487,7 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
                               const float* b, const float* A_log, const float* dt_bias,
                               const float* S0, const int32_t* cu_seqlens, int32_t N, int64_t T,
                               int32_t H_qk, int32_t H_v, float scale, void* o, float* S_final,
-                              void* workspace, bool fused, int* status, cudaStream_t s) {
+                              void* workspace, int schedule, int* status, cudaStream_t s) {
     if (N == 0) return cudaSuccess;
     if (T > (int64_t)0x7FFFFFFF - kC) return cudaErrorInvalidValue;  // TMA token coordinates
     const TcWorkspace ws = tc_workspace_layout(N, T, H_v);
@@ -1319,34 +1511,38 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
     cudaError_t e;
     const int64_t chain_units = (int64_t)N * H_v;
 
-    if (fused && coop) {
-        e = cudaFuncSetAttribute(fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (schedule > 0 && coop) {
+        // Overlap pays when the chains are few (latency-bound: each holds one SM for
+        // its whole sequence); with many chains the separate launches keep both
+        // phases at full occupancy. With at most a quarter as many chains as SMs each
+        // chain runs as two blocks of 64 value rows (half the per-thread state work on
+        // the critical path).
+        const bool half = schedule == 2 && 4 * chain_units <= num_sms;
+        const void* kfn = half ? (const void*)fused_kernel<64> : (const void*)fused_kernel<128>;
+        e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kFusedSmem);
         if (e != cudaSuccess) return e;
         int per_sm = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fused_kernel, kFusedThreads,
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kfn, kFusedThreads,
                                                           kFusedSmem);
         if (e != cudaSuccess) return e;
         const int grid = per_sm >= 1 ? num_sms : 0;
-        // Overlap pays when the chains are few (latency-bound: each holds one SM for
-        // its whole sequence); with many chains the separate launches keep both
-        // phases at full occupancy.
-        if (grid >= 2 && 2 * chain_units <= grid && N <= kFusedMaxSeqs) {
-            const int c0 = (int)chain_units;
+        const int64_t chain_blocks = (half ? 2 : 1) * chain_units;
+        if (grid >= 2 && 2 * chain_blocks <= grid && N <= kFusedMaxSeqs) {
             // this call's number: above every number an earlier call wrote
             static std::atomic<unsigned long long> call_number{0};
             unsigned long long epoch = call_number.fetch_add(1) + 1;
             const bf16* qb = static_cast<const bf16*>(q);
             const bf16* kb = static_cast<const bf16*>(k);
             bf16* ob = static_cast<bf16*>(o);
-            int c0v = c0;
+            int c0v = (int)chain_blocks;
             void* args[] = {&tm_q, &tm_k, &tm_v, &tm_o, &qb, &kb, &a, &b, &A_log, &dt_bias, &S0,
                             &cu_seqlens, &choff, &N, &T, &H_qk, &H_v, &scale, &rec, &ob,
                             &S_final, &status, &flags, &epoch, &c0v};
             ktimer_before(s);
-            e = cudaLaunchCooperativeKernel((const void*)fused_kernel, dim3(grid),
-                                            dim3(kFusedThreads), args, kFusedSmem, s);
-            if (e == cudaSuccess) ktimer_after(s, "fused");
+            e = cudaLaunchCooperativeKernel(kfn, dim3(grid), dim3(kFusedThreads), args, kFusedSmem,
+                                            s);
+            if (e == cudaSuccess) ktimer_after(s, half ? "fused_half_rows" : "fused");
             return e;
         }
     }

@@ -38,6 +38,7 @@ EXPORTS = ["gdn_status_string", "gdn_version", "gdn_prefill_workspace_size", "gd
            "gdn_last_prefill_kernel_name", "gdn_conv1d_silu", "gdn_conv1d_silu_decode",
            "gdn_rmsnorm_gated", "gdn_decode_slots", "gdn_decode_step_bf16_state"]
 GDN_IMPL_AUTO, GDN_IMPL_CUDA_CORE, GDN_IMPL_TENSOR_CORE, GDN_IMPL_TENSOR_CORE_SPLIT = 0, 1, 2, 3
+GDN_IMPL_TENSOR_CORE_WHOLE_ROWS = 4
 
 
 class GDNError(RuntimeError):

@@ -272,8 +272,9 @@ def test_set_prefill_impl(lib):
     assert lib.gdn_set_prefill_impl(1) == 0
     assert lib.gdn_set_prefill_impl(2) == 1
     assert lib.gdn_set_prefill_impl(3) == 2
+    assert lib.gdn_set_prefill_impl(4) == 3
     assert lib.gdn_set_prefill_impl(7) == -1      # invalid: unchanged
-    assert lib.gdn_set_prefill_impl(0) == 3
+    assert lib.gdn_set_prefill_impl(0) == 4
 
 
 def test_kernel_timing_switch(lib):

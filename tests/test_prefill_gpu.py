@@ -175,7 +175,8 @@ def impl_switch():
 
 
 IMPLS = {"cuda_core": "GDN_IMPL_CUDA_CORE", "tensor_core": "GDN_IMPL_TENSOR_CORE",
-         "tensor_core_split": "GDN_IMPL_TENSOR_CORE_SPLIT"}
+         "tensor_core_split": "GDN_IMPL_TENSOR_CORE_SPLIT",
+         "tensor_core_whole_rows": "GDN_IMPL_TENSOR_CORE_WHOLE_ROWS"}
 
 
 @pytest.mark.parametrize("impl", list(IMPLS))
@@ -213,7 +214,8 @@ def test_kernel_timing_names_and_durations(impl_switch):
     P = make_prefill_inputs([300, 77], H_qk=2, H_v=4, d_k=128, d_v=128, seed=31)
     prev = g.set_kernel_timing(True)
     try:
-        for impl, names in ((g.GDN_IMPL_TENSOR_CORE, ["fused"]),  # 2 x 4 chains: overlapped
+        for impl, names in ((g.GDN_IMPL_TENSOR_CORE, ["fused_half_rows"]),  # 8 chains
+                            (g.GDN_IMPL_TENSOR_CORE_WHOLE_ROWS, ["fused"]),
                             (g.GDN_IMPL_TENSOR_CORE_SPLIT, ["chunk_offsets", "prep", "chain"]),
                             (g.GDN_IMPL_CUDA_CORE, ["gates", "prefill_simt"])):
             g.set_prefill_impl(impl)
@@ -227,17 +229,20 @@ def test_kernel_timing_names_and_durations(impl_switch):
 
 @pytest.mark.parametrize("wl", ["prefill_35b", "varlen_64"])
 def test_fused_equals_split(impl_switch, wl):
-    """The overlapped single launch and the separate launches compute the same thing
-    (same arithmetic, different scheduling): outputs agree to the last bit."""
+    """The overlapped single launch (half-row chain blocks for the 35B layer's 32 chains,
+    whole-row blocks for 64 chains) and the separate launches compute the same thing
+    (same arithmetic per element, different scheduling): outputs agree to the last bit."""
     g = impl_switch
     W = dict(WORKLOADS[wl])
     if wl == "varlen_64":
         W["num_seqs"] = 2  # 64 chains: few enough for the overlapped launch
     P = make_prefill_inputs(**W, seed=3, device="cuda")
+    fused = "fused_half_rows" if wl == "prefill_35b" else "fused"
     outs = []
     prev = g.set_kernel_timing(True)
     try:
-        for impl, kernel in ((g.GDN_IMPL_TENSOR_CORE, "fused"),
+        for impl, kernel in ((g.GDN_IMPL_TENSOR_CORE, fused),
+                             (g.GDN_IMPL_TENSOR_CORE_WHOLE_ROWS, "fused"),
                              (g.GDN_IMPL_TENSOR_CORE_SPLIT, "chain")):
             g.set_prefill_impl(impl)
             o, Sf = gdn_prefill(P.q, P.k, P.v, P.a, P.b, P.A_log, P.dt_bias, P.cu_seqlens,
@@ -247,7 +252,8 @@ def test_fused_equals_split(impl_switch, wl):
             outs.append((o, Sf))
     finally:
         g.set_kernel_timing(prev)
-    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    for o_, S_ in outs[1:]:
+        assert torch.equal(outs[0][0], o_) and torch.equal(outs[0][1], S_)
 
 
 def test_many_chains_use_separate_launches(impl_switch):
