@@ -222,6 +222,29 @@ int gdn_decode_slots(const void* q, const void* k, const void* v, int32_t io_dty
                      float* intermediate_states, void* stream);
 
 /*
+ * gdn_prefill_slots -- gdn_prefill with the states in a pool of cache slots, the
+ * pool of gdn_decode_slots ("Qwen3.5 observation notes", section "Cache": a request
+ * keeps one batch index of the cache for its whole life).
+ *   state_pool         [num_slots, H_v, d_v, d_k] fp32                    (in/out)
+ *   state_slots        [N] int32, device: sequence n's slot. Its initial state is
+ *                      pool[slot] where has_initial_state is NULL or
+ *                      has_initial_state[n] != 0 (else zeros, a new request); its
+ *                      final state is written to pool[slot] (in place). Slot < 0:
+ *                      zeros in, nothing written (outputs still computed). Slot >=
+ *                      num_slots: the same, and GDN_ERR_BAD_SLOT in the device
+ *                      status word. Two sequences must not share a slot.
+ *   has_initial_state  [N] int32, device, or NULL (every sequence continues).
+ * Everything else as gdn_prefill (same workspace size).
+ */
+int gdn_prefill_slots(const void* q, const void* k, const void* v, int32_t io_dtype,
+                      const float* a, const float* b, const float* A_log, const float* dt_bias,
+                      float* state_pool, const int32_t* state_slots,
+                      const int32_t* has_initial_state, int32_t num_slots,
+                      const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                      int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v, float scale, void* o,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * gdn_prefill_noalloc -- gdn_prefill for callers that cannot allocate device
  * memory. The pages have no counterpart: this is a deployment variant.
  *

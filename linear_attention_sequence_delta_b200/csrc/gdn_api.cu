@@ -146,12 +146,17 @@ int gdn_gates(const float* a, const float* b, const float* A_log, const float* d
                                   g_chunk_cumsum, g, beta, st, (cudaStream_t)stream));
 }
 
-int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
-                const float* a, const float* b, const float* A_log, const float* dt_bias,
-                const float* initial_state, const int32_t* cu_seqlens, int32_t num_seqs,
-                int64_t total_tokens, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
-                float scale, void* o, float* final_state, void* workspace,
-                size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+// gdn_prefill and gdn_prefill_slots: the same path, the states addressed per sequence or
+// through pool slots
+int prefill_common(const void* q, const void* k, const void* v, int32_t io_dtype,
+                   const float* a, const float* b, const float* A_log, const float* dt_bias,
+                   const float* initial_state, const int32_t* cu_seqlens, int32_t num_seqs,
+                   int64_t total_tokens, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
+                   float scale, void* o, float* final_state, StateIndex sref, void* workspace,
+                   size_t workspace_bytes, void* stream) {
     if (io_dtype != GDN_BF16 && io_dtype != GDN_FP32) return GDN_ERR_INVALID_ARG;
     if (num_seqs < 0 || total_tokens < 0) return GDN_ERR_INVALID_ARG;
     if (num_seqs == 0 && total_tokens != 0) return GDN_ERR_INVALID_ARG;
@@ -183,7 +188,7 @@ int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
     if (tc_ok && impl != GDN_IMPL_CUDA_CORE) {
         return to_status(launch_prefill_tc(q, k, v, a, b, A_log, dt_bias, initial_state,
                                            cu_seqlens, num_seqs, total_tokens, H_qk, H_v, scale,
-                                           o, final_state, workspace,
+                                           o, final_state, sref, workspace,
                                            impl == GDN_IMPL_TENSOR_CORE_SPLIT ? 0
                                            : impl == GDN_IMPL_TENSOR_CORE_WHOLE_ROWS ? 1 : 2,
                                            st, s));
@@ -201,9 +206,44 @@ int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
     ktimer_before(s);
     const int rs = to_status(launch_prefill_simt(q, k, v, io_dtype, G, beta, initial_state,
                                                  cu_seqlens, num_seqs, total_tokens, H_qk, H_v,
-                                                 d_k, scale, o, final_state, st, s));
+                                                 d_k, scale, o, final_state, sref, st, s));
     ktimer_after(s, "prefill_simt");
     return rs;
+}
+}  // namespace
+
+extern "C" {
+
+int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
+                const float* a, const float* b, const float* A_log, const float* dt_bias,
+                const float* initial_state, const int32_t* cu_seqlens, int32_t num_seqs,
+                int64_t total_tokens, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
+                float scale, void* o, float* final_state, void* workspace,
+                size_t workspace_bytes, void* stream) {
+    return prefill_common(q, k, v, io_dtype, a, b, A_log, dt_bias, initial_state, cu_seqlens,
+                          num_seqs, total_tokens, H_qk, H_v, d_k, d_v, scale, o, final_state,
+                          StateIndex{}, workspace, workspace_bytes, stream);
+}
+
+int gdn_prefill_slots(const void* q, const void* k, const void* v, int32_t io_dtype,
+                      const float* a, const float* b, const float* A_log, const float* dt_bias,
+                      float* state_pool, const int32_t* state_slots,
+                      const int32_t* has_initial_state, int32_t num_slots,
+                      const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                      int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v, float scale, void* o,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+    if (num_seqs > 0 && (!state_slots || !state_pool)) return GDN_ERR_INVALID_ARG;
+    if (num_slots < 0) return GDN_ERR_INVALID_ARG;
+    if ((state_slots && !aligned(state_slots, 4)) ||
+        (has_initial_state && !aligned(has_initial_state, 4)))
+        return GDN_ERR_INVALID_ARG;
+    StateIndex sref;
+    sref.slots = state_slots;
+    sref.has_init = has_initial_state;
+    sref.num_slots = num_slots;
+    return prefill_common(q, k, v, io_dtype, a, b, A_log, dt_bias, state_pool, cu_seqlens,
+                          num_seqs, total_tokens, H_qk, H_v, d_k, d_v, scale, o, state_pool, sref,
+                          workspace, workspace_bytes, stream);
 }
 
 int gdn_decode_step(const void* q, const void* k, const void* v, int32_t io_dtype,

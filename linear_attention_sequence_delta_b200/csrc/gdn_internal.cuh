@@ -67,6 +67,29 @@ __device__ __forceinline__ void set_status(int* status, int code) {
     if (status) atomicCAS(status, 0, code);
 }
 
+// Where each sequence's initial and final states live. Without slots sequence n uses
+// state n of the initial / final arrays. With slots it uses entry slots[n] of one pool,
+// read only where has_init is null or has_init[n] != 0 (else it starts from zeros) and
+// written at the end; slot < 0 starts from zeros and writes nothing; a slot >= num_slots
+// is reported (GDN_ERR_BAD_SLOT) and treated like slot < 0.
+struct StateIndex {
+    const int32_t* slots = nullptr;
+    const int32_t* has_init = nullptr;
+    int num_slots = 0;
+    __device__ __forceinline__ int resolve(int n, bool& read, bool& write, int* status) const {
+        read = write = true;
+        if (!slots) return n;
+        const int s = slots[n];
+        if (s < 0 || s >= num_slots) {
+            if (s >= num_slots) set_status(status, GDN_ERR_BAD_SLOT);
+            read = write = false;
+            return 0;
+        }
+        read = !has_init || has_init[n] != 0;
+        return s;
+    }
+};
+
 // ---- host launchers (one per kernel family) ----------------------------------
 
 // Status word of the current device (a __device__ int of this library).
@@ -110,7 +133,7 @@ cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, int
                                 const float* G, const float* beta, const float* S0,
                                 const int32_t* cu_seqlens, int32_t N, int64_t T, int32_t H_qk,
                                 int32_t H_v, int32_t d, float scale, void* o, float* S_final,
-                                int* status, cudaStream_t s);
+                                StateIndex sref, int* status, cudaStream_t s);
 
 // Tensor-core prefill (bf16 I/O, d = 128): chunk offsets, the state-independent
 // prep kernel, then the chain kernel. schedule: 0 = always separate launches, 1 = one
@@ -123,7 +146,8 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
                               const float* b, const float* A_log, const float* dt_bias,
                               const float* S0, const int32_t* cu_seqlens, int32_t N, int64_t T,
                               int32_t H_qk, int32_t H_v, float scale, void* o, float* S_final,
-                              void* workspace, int schedule, int* status, cudaStream_t s);
+                              StateIndex sref, void* workspace, int schedule, int* status,
+                              cudaStream_t s);
 
 // Steps around the delta rule (gdn_mixer.cu): causal depthwise conv1d + SiLU with
 // the per-sequence conv cache, its single-token decode form, and the gated RMSNorm.

@@ -105,7 +105,8 @@ extern "C" int gdn_prefill_noalloc(const void* q, const void* k, const void* v, 
             return GDN_ERR_CUDA;
     }
     return launch_prefill_simt(q, k, v, io_dtype, G, beta, initial_state, cu_seqlens, num_seqs,
-                               total_tokens, H_qk, H_v, d_k, scale, o, final_state, st, s) ==
+                               total_tokens, H_qk, H_v, d_k, scale, o, final_state, StateIndex{},
+                               st, s) ==
                    cudaSuccess
                ? GDN_OK
                : GDN_ERR_CUDA;

@@ -55,8 +55,8 @@ template <typename IO, int D, int DVS>
 __global__ void __launch_bounds__(kThreads, 1) prefill_simt_kernel(
     const IO* __restrict__ q, const IO* __restrict__ k, const IO* __restrict__ v,
     const float* __restrict__ Gcs, const float* __restrict__ beta,
-    const float* __restrict__ S0, const int32_t* __restrict__ cu_seqlens, int64_t T_total,
-    int H_qk, int H_v, float scale, IO* __restrict__ o, float* __restrict__ S_final,
+    const float* S0, const int32_t* __restrict__ cu_seqlens, int64_t T_total,
+    int H_qk, int H_v, float scale, IO* __restrict__ o, float* S_final, StateIndex sref,
     int* status) {
     using L = SimtSmem<D, DVS>;
     constexpr int KP = L::KP, CP = L::CP;
@@ -91,11 +91,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_simt_kernel(
         return;
     }
 
-    // state slice: rows dv0 .. dv0+DVS-1 of the d_v x d_k value-major state
-    const size_t sbase = ((size_t)n * H_v + h) * D * D + (size_t)dv0 * D;
+    // state slice: rows dv0 .. dv0+DVS-1 of the d_v x d_k value-major state (of the
+    // sequence's state, or of its pool slot); read completely before anything is written
+    bool rd, wr;
+    const int sidx = sref.resolve(n, rd, wr, tid == 0 ? status : nullptr);
+    const float* S0s = rd ? S0 : nullptr;
+    float* Sfs = wr ? S_final : nullptr;
+    const size_t sbase = ((size_t)sidx * H_v + h) * D * D + (size_t)dv0 * D;
     for (int idx = tid; idx < DVS * D; idx += kThreads) {
         const int c = idx / D, kk = idx % D;
-        Ss[c * KP + kk] = S0 ? S0[sbase + idx] : 0.f;
+        Ss[c * KP + kk] = S0s ? S0s[sbase + idx] : 0.f;
     }
 
     for (int64_t t0 = s0; t0 < s1; t0 += kC) {
@@ -332,10 +337,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_simt_kernel(
         }
     }
     __syncthreads();
-    if (S_final) {
+    if (Sfs) {
         for (int idx = tid; idx < DVS * D; idx += kThreads) {
             const int c = idx / D, kk = idx % D;
-            S_final[sbase + idx] = Ss[c * KP + kk];
+            Sfs[sbase + idx] = Ss[c * KP + kk];
         }
     }
 }
@@ -344,7 +349,7 @@ template <typename IO, int D, int DVS>
 cudaError_t launch_simt_t(const void* q, const void* k, const void* v, const float* G,
                           const float* beta, const float* S0, const int32_t* cu, int32_t N,
                           int64_t T, int32_t H_qk, int32_t H_v, float scale, void* o,
-                          float* S_final, int* status, cudaStream_t s) {
+                          float* S_final, StateIndex sref, int* status, cudaStream_t s) {
     using L = SimtSmem<D, DVS>;
     auto kern = prefill_simt_kernel<IO, D, DVS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -354,7 +359,7 @@ cudaError_t launch_simt_t(const void* q, const void* k, const void* v, const flo
     if (blocks == 0) return cudaSuccess;
     kern<<<(unsigned)blocks, kThreads, L::bytes, s>>>(
         static_cast<const IO*>(q), static_cast<const IO*>(k), static_cast<const IO*>(v), G, beta,
-        S0, cu, T, H_qk, H_v, scale, static_cast<IO*>(o), S_final, status);
+        S0, cu, T, H_qk, H_v, scale, static_cast<IO*>(o), S_final, sref, status);
     return cudaGetLastError();
 }
 
@@ -364,19 +369,17 @@ cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, int
                                 const float* G, const float* beta, const float* S0,
                                 const int32_t* cu_seqlens, int32_t N, int64_t T, int32_t H_qk,
                                 int32_t H_v, int32_t d, float scale, void* o, float* S_final,
-                                int* status, cudaStream_t s) {
+                                StateIndex sref, int* status, cudaStream_t s) {
+#define GDN_SIMT(IO, D)                                                                      \
+    return launch_simt_t<IO, D, 32>(q, k, v, G, beta, S0, cu_seqlens, N, T, H_qk, H_v, scale, \
+                                    o, S_final, sref, status, s)
     if (io_dtype == GDN_BF16) {
-        if (d == 128)
-            return launch_simt_t<__nv_bfloat16, 128, 32>(q, k, v, G, beta, S0, cu_seqlens, N, T,
-                                                         H_qk, H_v, scale, o, S_final, status, s);
-        return launch_simt_t<__nv_bfloat16, 64, 32>(q, k, v, G, beta, S0, cu_seqlens, N, T, H_qk,
-                                                    H_v, scale, o, S_final, status, s);
+        if (d == 128) GDN_SIMT(__nv_bfloat16, 128);
+        GDN_SIMT(__nv_bfloat16, 64);
     }
-    if (d == 128)
-        return launch_simt_t<float, 128, 32>(q, k, v, G, beta, S0, cu_seqlens, N, T, H_qk, H_v,
-                                             scale, o, S_final, status, s);
-    return launch_simt_t<float, 64, 32>(q, k, v, G, beta, S0, cu_seqlens, N, T, H_qk, H_v, scale,
-                                        o, S_final, status, s);
+    if (d == 128) GDN_SIMT(float, 128);
+    GDN_SIMT(float, 64);
+#undef GDN_SIMT
 }
 
 }  // namespace gdn

@@ -680,9 +680,10 @@ __device__ __forceinline__ bool wait_record(const unsigned long long* flag,
 template <int kM>
 __device__ __forceinline__ void chain_unit(
     const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-    const CUtensorMap& tm_o, const float* __restrict__ S0g, const int32_t* __restrict__ cu_seqlens,
+    const CUtensorMap& tm_o, const float* S0g, const int32_t* __restrict__ cu_seqlens,
     const int32_t* __restrict__ choff, int64_t T_total, int H_qk, int H_v,
-    const uint8_t* __restrict__ rec, bf16* __restrict__ o, float* __restrict__ Sfg, int* status,
+    const uint8_t* __restrict__ rec, bf16* __restrict__ o, float* Sfg, const StateIndex sref,
+    int* status,
     const unsigned long long* flags, unsigned long long epoch, uint8_t* sm, const int tid,
     const int n, const int h, const int hv, const uint32_t tmem,
     const int sync_id) {
@@ -994,10 +995,14 @@ __device__ __forceinline__ void chain_unit(
             const int hh = warp >> 2;             // column half
             const int row = qd * 32 + lane;       // value row i = TMEM lane
             const uint32_t ctl = tmem + ((uint32_t)(qd * 32) << 16);
-            const size_t sbase = ((size_t)n * H_v + h) * kD * kD + (size_t)row * kD + 64 * hh;
+            bool rd, wr;  // the sequence's state (or pool slot): read at the start, written at the end
+            const int sidx = sref.resolve(n, rd, wr, tid == 0 ? status : nullptr);
+            const float* S0s = rd ? S0g : nullptr;
+            float* Sfs = wr ? Sfg : nullptr;
+            const size_t sbase = ((size_t)sidx * H_v + h) * kD * kD + (size_t)row * kD + 64 * hh;
             float S[64];  // S[i][64 hh + e]
-            if (S0g) {
-                const float4* src = reinterpret_cast<const float4*>(S0g + sbase);
+            if (S0s) {
+                const float4* src = reinterpret_cast<const float4*>(S0s + sbase);
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const float4 f = src[e];
@@ -1138,8 +1143,8 @@ __device__ __forceinline__ void chain_unit(
                 done = !dead;
                 if (done) apply_update(gamma);
             }
-            if (done && Sfg) {
-                float4* d4 = reinterpret_cast<float4*>(Sfg + sbase);
+            if (done && Sfs) {
+                float4* d4 = reinterpret_cast<float4*>(Sfs + sbase);
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
                     d4[e] = make_float4(S[4 * e], S[4 * e + 1], S[4 * e + 2], S[4 * e + 3]);
@@ -1155,15 +1160,19 @@ __device__ __forceinline__ void chain_unit(
             const int r0 = 64 * hv + qd * 16 + (lane >> 2);  // value row of registers e = 0, 1
             const int cp2 = 2 * (lane & 3);
             const uint32_t ctl = tmem + ((uint32_t)(qd * 32) << 16);
-            const size_t hbase = ((size_t)n * H_v + h) * kD * kD;
+            bool rd, wr;  // the sequence's state (or pool slot): read at the start, written at the end
+            const int sidx = sref.resolve(n, rd, wr, tid == 0 ? status : nullptr);
+            const float* S0s = rd ? S0g : nullptr;
+            float* Sfs = wr ? Sfg : nullptr;
+            const size_t hbase = ((size_t)sidx * H_v + h) * kD * kD;
             float S[32];  // S[4 j + e]: row r0 + 8 (e >> 1), column 64 hh + 8 j + cp2 + (e & 1)
-            if (S0g) {
+            if (S0s) {
 #pragma unroll
                 for (int jj = 0; jj < 8; ++jj) {
                     const int col = 64 * hh + 8 * jj + cp2;
-                    const float2 f0 = *reinterpret_cast<const float2*>(S0g + hbase + (size_t)r0 * kD + col);
+                    const float2 f0 = *reinterpret_cast<const float2*>(S0s + hbase + (size_t)r0 * kD + col);
                     const float2 f1 =
-                        *reinterpret_cast<const float2*>(S0g + hbase + (size_t)(r0 + 8) * kD + col);
+                        *reinterpret_cast<const float2*>(S0s + hbase + (size_t)(r0 + 8) * kD + col);
                     S[4 * jj] = f0.x; S[4 * jj + 1] = f0.y; S[4 * jj + 2] = f1.x; S[4 * jj + 3] = f1.y;
                 }
             } else {
@@ -1285,13 +1294,13 @@ __device__ __forceinline__ void chain_unit(
                 done = !dead;
                 if (done) apply_update(gamma);
             }
-            if (done && Sfg) {
+            if (done && Sfs) {
 #pragma unroll
                 for (int jj = 0; jj < 8; ++jj) {
                     const int col = 64 * hh + 8 * jj + cp2;
-                    *reinterpret_cast<float2*>(Sfg + hbase + (size_t)r0 * kD + col) =
+                    *reinterpret_cast<float2*>(Sfs + hbase + (size_t)r0 * kD + col) =
                         make_float2(S[4 * jj], S[4 * jj + 1]);
-                    *reinterpret_cast<float2*>(Sfg + hbase + (size_t)(r0 + 8) * kD + col) =
+                    *reinterpret_cast<float2*>(Sfs + hbase + (size_t)(r0 + 8) * kD + col) =
                         make_float2(S[4 * jj + 2], S[4 * jj + 3]);
                 }
             }
@@ -1307,9 +1316,10 @@ __device__ __forceinline__ void chain_unit(
 __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-    const float* __restrict__ S0g, const int32_t* __restrict__ cu_seqlens,
+    const float* S0g, const int32_t* __restrict__ cu_seqlens,
     const int32_t* __restrict__ choff, int64_t T_total, int H_qk, int H_v,
-    const uint8_t* __restrict__ rec, bf16* __restrict__ o, float* __restrict__ Sfg, int* status) {
+    const uint8_t* __restrict__ rec, bf16* __restrict__ o, float* Sfg, const StateIndex sref,
+    int* status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1324,8 +1334,8 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
     chain_unit<128>(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v, rec, o,
-                    Sfg, status, nullptr, 0, sm, threadIdx.x, blockIdx.x / H_v, blockIdx.x % H_v,
-                    0, tmem, 1);
+                    Sfg, sref, status, nullptr, 0, sm, threadIdx.x, blockIdx.x / H_v,
+                    blockIdx.x % H_v, 0, tmem, 1);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1354,10 +1364,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
     const bf16* __restrict__ q, const bf16* __restrict__ k, const float* __restrict__ a,
     const float* __restrict__ b, const float* __restrict__ A_log,
-    const float* __restrict__ dt_bias, const float* __restrict__ S0g,
+    const float* __restrict__ dt_bias, const float* S0g,
     const int32_t* __restrict__ cu_seqlens, const int32_t* choff, int32_t N,
     int64_t T_total, int H_qk, int H_v, float scale, uint8_t* __restrict__ rec,
-    bf16* __restrict__ o, float* __restrict__ Sfg, int* status, unsigned long long* flags,
+    bf16* __restrict__ o, float* Sfg, const StateIndex sref, int* status,
+    unsigned long long* flags,
     unsigned long long epoch, int c0) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ int32_t s_choff[kFusedMaxSeqs + 1];
@@ -1417,7 +1428,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
     const int u = kM == 64 ? (int)blockIdx.x >> 1 : (int)blockIdx.x;
     const int hv = kM == 64 ? (int)blockIdx.x & 1 : 0;
     chain_unit<kM>(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v, rec, o,
-                   Sfg, status, flags, epoch, sm, tid, u / H_v, u % H_v, hv, tmem, kChainSync);
+                   Sfg, sref, status, flags, epoch, sm, tid, u / H_v, u % H_v, hv, tmem,
+                   kChainSync);
     tc_fence_before();
     named_bar_sync(kChainSync, kChainThreads);
     tc_fence_after();
@@ -1487,7 +1499,8 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
                               const float* b, const float* A_log, const float* dt_bias,
                               const float* S0, const int32_t* cu_seqlens, int32_t N, int64_t T,
                               int32_t H_qk, int32_t H_v, float scale, void* o, float* S_final,
-                              void* workspace, int schedule, int* status, cudaStream_t s) {
+                              StateIndex sref, void* workspace, int schedule, int* status,
+                              cudaStream_t s) {
     if (N == 0) return cudaSuccess;
     if (T > (int64_t)0x7FFFFFFF - kC) return cudaErrorInvalidValue;  // TMA token coordinates
     const TcWorkspace ws = tc_workspace_layout(N, T, H_v);
@@ -1538,7 +1551,7 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
             int c0v = (int)chain_blocks;
             void* args[] = {&tm_q, &tm_k, &tm_v, &tm_o, &qb, &kb, &a, &b, &A_log, &dt_bias, &S0,
                             &cu_seqlens, &choff, &N, &T, &H_qk, &H_v, &scale, &rec, &ob,
-                            &S_final, &status, &flags, &epoch, &c0v};
+                            &S_final, &sref, &status, &flags, &epoch, &c0v};
             ktimer_before(s);
             e = cudaLaunchCooperativeKernel(kfn, dim3(grid), dim3(kFusedThreads), args, kFusedSmem,
                                             s);
@@ -1573,7 +1586,7 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
     ktimer_before(s);
     chain_kernel<<<(unsigned)chain_units, kChainThreads, kChainSmem, s>>>(
         tm_q, tm_k, tm_v, tm_o, S0, cu_seqlens, choff, T, H_qk, H_v, rec, static_cast<bf16*>(o),
-        S_final, status);
+        S_final, sref, status);
     e = cudaGetLastError();
     if (e == cudaSuccess) ktimer_after(s, "chain");
     return e;

@@ -36,7 +36,8 @@ EXPORTS = ["gdn_status_string", "gdn_version", "gdn_prefill_workspace_size", "gd
            "gdn_prefill", "gdn_decode_step", "gdn_sync_status", "gdn_prefill_noalloc",
            "gdn_set_prefill_impl", "gdn_set_kernel_timing", "gdn_last_prefill_kernel_ms",
            "gdn_last_prefill_kernel_name", "gdn_conv1d_silu", "gdn_conv1d_silu_decode",
-           "gdn_rmsnorm_gated", "gdn_decode_slots", "gdn_decode_step_bf16_state"]
+           "gdn_rmsnorm_gated", "gdn_decode_slots", "gdn_decode_step_bf16_state",
+           "gdn_prefill_slots"]
 GDN_IMPL_AUTO, GDN_IMPL_CUDA_CORE, GDN_IMPL_TENSOR_CORE, GDN_IMPL_TENSOR_CORE_SPLIT = 0, 1, 2, 3
 GDN_IMPL_TENSOR_CORE_WHOLE_ROWS = 4
 
@@ -88,6 +89,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gdn_conv1d_silu.argtypes = [P, i32, P, P, P, P, i32, i64, i32, i32, P, P, P]
     lib.gdn_conv1d_silu_decode.restype = ctypes.c_int
     lib.gdn_conv1d_silu_decode.argtypes = [P, i32, P, P, P, P, i32, i32, i32, i32, P, P]
+    lib.gdn_prefill_slots.restype = ctypes.c_int
+    lib.gdn_prefill_slots.argtypes = [P, P, P, i32, P, P, P, P, P, P, P, i32, P, i32, i64, i32,
+                                      i32, i32, i32, f32, P, P, sz, P]
     lib.gdn_decode_step_bf16_state.restype = ctypes.c_int
     lib.gdn_decode_step_bf16_state.argtypes = [P, P, P, i32, P, P, P, P, P, i32, i32, i32, i32,
                                                i32, f32, P, P]
@@ -182,6 +186,36 @@ def gdn_prefill(q, k, v, a, b, A_log, dt_bias, cu_seqlens, initial_state=None, *
                          workspace.numel(), _stream(q.device))
     _check(st, "gdn_prefill")
     return o, final_state
+
+
+def gdn_prefill_slots(q, k, v, a, b, A_log, dt_bias, cu_seqlens, state_pool, state_slots,
+                      has_initial_state=None, *, scale: float = 1.0, out=None, workspace=None):
+    """gdn_prefill with the states in a pool: sequence n starts from state_pool[slot]
+    (or zeros where has_initial_state[n] == 0) and its final state replaces it.
+    state_pool [num_slots, H_v, d_v, d_k] fp32; state_slots, has_initial_state int32 [N]."""
+    lib = load_library()
+    _need_cuda(q, k, v, a, b, A_log, dt_bias, cu_seqlens, state_pool, state_slots,
+               has_initial_state, out, workspace)
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k and v must share one dtype")
+    for t in (state_slots, has_initial_state):
+        if t is not None and t.dtype != torch.int32:
+            raise TypeError("state_slots and has_initial_state must be int32")
+    io = _io_dtype(q)
+    T, H_qk, d_k = q.shape
+    _, H_v, d_v = v.shape
+    N = cu_seqlens.numel() - 1
+    o = out if out is not None else torch.empty((T, H_v, d_v), device=q.device, dtype=q.dtype)
+    need = lib.gdn_prefill_workspace_size(N, T, H_qk, H_v, d_k, d_v)
+    if workspace is None:
+        workspace = torch.empty((max(int(need), 1),), device=q.device, dtype=torch.uint8)
+    st = lib.gdn_prefill_slots(_ptr(q), _ptr(k), _ptr(v), io, _ptr(a), _ptr(b), _ptr(A_log),
+                               _ptr(dt_bias), _ptr(state_pool), _ptr(state_slots),
+                               _ptr(has_initial_state), state_pool.shape[0], _ptr(cu_seqlens), N,
+                               T, H_qk, H_v, d_k, d_v, float(scale), _ptr(o), _ptr(workspace),
+                               workspace.numel(), _stream(q.device))
+    _check(st, "gdn_prefill_slots")
+    return o
 
 
 def gdn_decode_step(q, k, v, a, b, A_log, dt_bias, state, *, scale: float = 1.0, out=None):

@@ -253,6 +253,30 @@ def test_decode_slots_rejects(lib, over, code):
     assert _call_slots(lib, **over) == code
 
 
+def test_prefill_slots_rejects(lib):
+    v = ctypes.c_void_p
+    f = lib.gdn_prefill_slots
+    base = dict(q=F, k=F + 0x1000, vv=F + 0x2000, io=0, a=F + 0x3000, b=F + 0x4000,
+                al=F + 0x5000, dt=F + 0x6000, pool=F + 0x10000, sl=F + 0x7000, hi=None, ns=4,
+                cu=F + 0x7100, N=2, T=128, hq=2, hv=4, dk=128, dv=128, sc=1.0, o=F + 0x8000,
+                ws=F + 0x100000, wsb=1 << 30)
+    p = lambda x: v(x) if x else None
+    call = lambda **o: (lambda a: f(p(a["q"]), p(a["k"]), p(a["vv"]), a["io"], p(a["a"]),
+                                    p(a["b"]), p(a["al"]), p(a["dt"]), p(a["pool"]), p(a["sl"]),
+                                    p(a["hi"]), a["ns"], p(a["cu"]), a["N"], a["T"], a["hq"],
+                                    a["hv"], a["dk"], a["dv"], a["sc"], p(a["o"]), p(a["ws"]),
+                                    a["wsb"], None))(dict(base, **o))
+    assert call(sl=None) == 1
+    assert call(pool=None) == 1
+    assert call(ns=-1) == 1
+    assert call(sl=F + 0x7002) == 1
+    assert call(hi=F + 0x7203) == 1
+    assert call(pool=F + 0x10004) == 1   # the pool is the initial / final state array
+    assert call(io=5) == 1
+    assert call(wsb=10) == 3
+    assert call(N=0, T=0, sl=None, pool=None) == 0
+
+
 def test_decode_slots_noop(lib):
     assert _call_slots(lib, N=0) == 0
     assert _call_slots(lib, N=0, slots=None, ns=0, pool=None) == 0

@@ -128,3 +128,84 @@ def test_bad_slot_reported_and_skipped():
     assert gdn_sync_status() == 7
     assert torch.equal(pool_d[[0, 2]].cpu(), pool[[0, 2]])
     assert gdn_sync_status() == 0
+
+
+# ------------------------------------------------------------ prefill into the pool --
+
+PREFILL_IMPLS = ["GDN_IMPL_AUTO", "GDN_IMPL_TENSOR_CORE_WHOLE_ROWS", "GDN_IMPL_TENSOR_CORE_SPLIT",
+                 "GDN_IMPL_CUDA_CORE"]
+
+
+@pytest.mark.parametrize("impl", PREFILL_IMPLS)
+def test_prefill_slots_against_oracle(impl):
+    """Sequences start from their slot (or zeros where has_initial_state is 0, or for slot
+    -1), write their final state back in place; unnamed slots come back bit for bit."""
+    from linear_attention_sequence_delta_b200 import gdn, gdn_prefill_slots
+    from linear_attention_sequence_delta_b200.inputs import make_prefill_inputs
+    lens = [70, 0, 130, 64, 1]
+    P = make_prefill_inputs(lens, H_qk=2, H_v=4, d_k=128, d_v=128, seed=21)
+    D = make_decode_inputs(steps=1, num_seqs=9, H_qk=2, H_v=4, d_k=128, d_v=128, seed=22)
+    pool = D.state.contiguous()
+    slots = torch.tensor([6, 2, -1, 0, 8], dtype=torch.int32)
+    has_init = torch.tensor([1, 0, 1, 1, 0], dtype=torch.int32)
+    prev = gdn.set_prefill_impl(getattr(gdn, impl))
+    try:
+        Pd = P.to("cuda")
+        pool_d = pool.cuda()
+        o = gdn_prefill_slots(Pd.q, Pd.k, Pd.v, Pd.a, Pd.b, Pd.A_log, Pd.dt_bias, Pd.cu_seqlens,
+                              pool_d, slots.cuda(), has_init.cuda())
+        assert gdn_sync_status() == 0
+    finally:
+        gdn.set_prefill_impl(prev)
+    cu = P.cu_seqlens.tolist()
+    for n in range(len(lens)):
+        s, use = int(slots[n]), bool(has_init[n]) and int(slots[n]) >= 0
+        S0 = pool[s:s + 1].unsqueeze(0)[0] if use else torch.zeros(1, 4, 128, 128)
+        o_ref, S_ref = oracle.forward(P.q[cu[n]:cu[n + 1]], P.k[cu[n]:cu[n + 1]],
+                                      P.v[cu[n]:cu[n + 1]], P.a[cu[n]:cu[n + 1]],
+                                      P.b[cu[n]:cu[n + 1]], P.A_log, P.dt_bias, [0, lens[n]], S0)
+        if lens[n]:
+            assert rel_err(o[cu[n]:cu[n + 1]], o_ref) <= TOL_BF16, n
+        if s >= 0:
+            assert rel_err(pool_d[s], S_ref[0]) <= TOL_BF16, n
+    named = {int(x) for x in slots if x >= 0}
+    rest = [i for i in range(9) if i not in named]
+    assert torch.equal(pool_d[rest].cpu(), pool[rest])
+
+
+def test_prefill_slots_then_decode_slots_equals_one_prefill():
+    """A prefill into the pool followed by decode steps from it equals one longer prefill."""
+    from linear_attention_sequence_delta_b200 import gdn_prefill, gdn_prefill_slots
+    from linear_attention_sequence_delta_b200.inputs import make_prefill_inputs
+    L0, steps = 100, 3
+    P = make_prefill_inputs([L0 + steps] * 2, H_qk=2, H_v=4, d_k=128, d_v=128, seed=23)
+    Pd = P.to("cuda")
+    o_all, S_all = gdn_prefill(Pd.q, Pd.k, Pd.v, Pd.a, Pd.b, Pd.A_log, Pd.dt_bias, Pd.cu_seqlens,
+                               None)
+    idx = torch.cat([torch.arange(n * (L0 + steps), n * (L0 + steps) + L0) for n in range(2)])
+    sub = lambda x: x[idx.cuda()].contiguous()
+    cu = torch.tensor([0, L0, 2 * L0], dtype=torch.int32, device="cuda")
+    pool = torch.zeros(4, 4, 128, 128, device="cuda")
+    slots = torch.tensor([3, 1], dtype=torch.int32, device="cuda")
+    gdn_prefill_slots(sub(Pd.q), sub(Pd.k), sub(Pd.v), sub(Pd.a), sub(Pd.b), Pd.A_log, Pd.dt_bias,
+                      cu, pool, slots, torch.zeros(2, dtype=torch.int32, device="cuda"))
+    tok = torch.tensor([[n * (L0 + steps) + L0 + s for s in range(steps)] for n in range(2)],
+                       device="cuda")
+    g = lambda x: x[tok].contiguous()
+    o_d, _ = gdn_decode_slots(g(Pd.q), g(Pd.k), g(Pd.v), g(Pd.a), g(Pd.b), Pd.A_log, Pd.dt_bias,
+                              pool, slots)
+    assert gdn_sync_status() == 0
+    assert rel_err(o_d, o_all[tok].cpu().float().numpy()) <= TOL_BF16
+    assert rel_err(pool[slots.long()], S_all.cpu().numpy()) <= TOL_BF16
+
+
+def test_prefill_bad_slot_reported():
+    from linear_attention_sequence_delta_b200 import gdn_prefill_slots
+    from linear_attention_sequence_delta_b200.inputs import make_prefill_inputs
+    P = make_prefill_inputs([40, 20], H_qk=1, H_v=2, d_k=128, d_v=128, seed=24).to("cuda")
+    pool = torch.zeros(2, 2, 128, 128, device="cuda")
+    gdn_prefill_slots(P.q, P.k, P.v, P.a, P.b, P.A_log, P.dt_bias, P.cu_seqlens, pool,
+                      torch.tensor([0, 5], dtype=torch.int32, device="cuda"))
+    assert gdn_sync_status() == 7
+    assert torch.all(pool[1] == 0)
+    assert gdn_sync_status() == 0
