@@ -71,12 +71,12 @@ struct Vec8<float> {
 // result is 0, where the exact value is below 1e-36 in magnitude.
 __device__ __forceinline__ float silu_f32(float x) { return __fdividef(x, 1.f + __expf(-x)); }
 
-// Tokens per thread in the prefill convolution: all of a tile's inputs are loaded
-// before any is used (16 x 16 bytes for bf16, 8 x 32 bytes for fp32).
-template <typename IO>
-struct ConvTile {
-    static constexpr int value = sizeof(IO) == 2 ? 16 : 8;
-};
+// The prefill convolution: a thread walks kConvRange consecutive tokens of one channel
+// vector, kConvGroup tokens at a time, and issues the next group's loads before it
+// computes the current one; the window of the last K-1 inputs stays in registers, so
+// each input is read once (plus K-1 positions per range).
+constexpr int kConvRange = 32;
+constexpr int kConvGroup = 4;
 
 // sequence n with cu[n] <= t < cu[n + 1] (the last such n for empty sequences)
 __device__ __forceinline__ int find_seq(const int32_t* cu, int N, int64_t t) {
@@ -108,60 +108,60 @@ __device__ __forceinline__ void load_taps(const float* __restrict__ w,
     for (int e = 0; e < kVec; ++e) bs[e] = bias ? __ldg(bias + c0 + e) : 0.f;
 }
 
-// y for kTile consecutive tokens x kVec channels per thread; consecutive threads take
-// consecutive channel vectors of the same token tile. The window of the last K-1
-// inputs is carried in registers; at a sequence's start it comes from the cache (or
-// zeros). A tile inside one sequence loads all its inputs up front.
+// y for kConvRange consecutive tokens x kVec channels per thread; consecutive threads
+// take consecutive channel vectors of the same token range. At a sequence's start the
+// window comes from the cache (or zeros).
 template <typename IO, int K>
 __global__ void __launch_bounds__(128) conv1d_silu_kernel(
     const IO* __restrict__ x, const float* __restrict__ w, const float* __restrict__ bias,
     const IO* __restrict__ state_in, const int32_t* __restrict__ cu, int N, int64_t T, int C,
     IO* __restrict__ y, int* status) {
+    using V = Vec8<IO>;
     const int nv = C / kVec;
     const int64_t gidx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t tile = gidx / nv;
-    const int c0 = (int)(gidx - tile * nv) * kVec;
-    constexpr int kTile = ConvTile<IO>::value;
-    const int64_t t0 = tile * kTile;
-    if (t0 >= T) return;
+    const int64_t range = gidx / nv;
+    const int c0 = (int)(gidx - range * nv) * kVec;
+    const int64_t tb = range * kConvRange;
+    if (tb >= T) return;
+    const int64_t te = tb + kConvRange < T ? tb + kConvRange : T;
     // Let the cache kernel that follows start its loads (it waits before storing).
     asm volatile("griddepcontrol.launch_dependents;");
     // Loads that need no sequence bounds go first, so that they overlap the lookup in
-    // cu_seqlens: the tile's tokens (index clamped to T-1) and the K-1 positions before
-    // it (clamped to 0).
-    typename Vec8<IO>::Raw xb[kTile], wb[K - 1];
+    // cu_seqlens: the first group (index clamped to the range) and the K-1 positions
+    // before the range (clamped to 0).
+    typename V::Raw cur[kConvGroup], wb[K - 1];
 #pragma unroll
-    for (int i = 0; i < kTile; ++i)
-        xb[i] = Vec8<IO>::load_raw(x + (size_t)(t0 + i < T ? t0 + i : T - 1) * C + c0);
+    for (int i = 0; i < kConvGroup; ++i)
+        cur[i] = V::load_raw(x + (size_t)(tb + i < te ? tb + i : te - 1) * C + c0);
 #pragma unroll
     for (int j = 0; j < K - 1; ++j) {
-        const int64_t p = t0 - (K - 1) + j;
-        wb[j] = Vec8<IO>::load_raw(x + (size_t)(p > 0 ? p : 0) * C + c0);
+        const int64_t p = tb - (K - 1) + j;
+        wb[j] = V::load_raw(x + (size_t)(p > 0 ? p : 0) * C + c0);
     }
     float wt[K][kVec], bs[kVec];
     load_taps<K>(w, bias, c0, wt, bs);
-    int n = find_seq(cu, N, t0);
+    int n = find_seq(cu, N, tb);
     int64_t s0 = cu[n], s1 = cu[n + 1];
-    if (s0 < 0 || t0 < s0 || s1 < s0 || s1 > T) {
+    if (s0 < 0 || tb < s0 || s1 < s0 || s1 > T) {
         set_status(status, kStatusBadSeqlens);
         return;
     }
     float win[kMaxK - 1][kVec];  // win[K-2] is the newest
-    auto fill_window = [&](int64_t t) {  // positions t-(K-1) .. t-1 of sequence n
+    // positions t-(K-1) .. t-1 of sequence n, those before its start from the cache
+    auto window_entry = [&](int64_t p, float (&v)[kVec]) {
+        if (state_in) {
+            V::load(state_in + ((size_t)n * (K - 1) + (K - 1) + (p - s0)) * C + c0, v);
+        } else {
 #pragma unroll
-        for (int j = 0; j < K - 1; ++j) {
-            const int64_t p = t - (K - 1) + j;
-            if (p >= s0) {
-                Vec8<IO>::load(x + (size_t)p * C + c0, win[j]);
-            } else if (state_in) {
-                Vec8<IO>::load(state_in + ((size_t)n * (K - 1) + (K - 1) + (p - s0)) * C + c0,
-                               win[j]);
-            } else {
-#pragma unroll
-                for (int e = 0; e < kVec; ++e) win[j][e] = 0.f;
-            }
+            for (int e = 0; e < kVec; ++e) v[e] = 0.f;
         }
     };
+#pragma unroll
+    for (int j = 0; j < K - 1; ++j) {
+        const int64_t p = tb - (K - 1) + j;
+        if (p >= s0) V::unpack(wb[j], win[j]);
+        else window_entry(p, win[j]);
+    }
     auto step = [&](const float (&xt)[kVec], int64_t t) {
         float out[kVec];
 #pragma unroll
@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(128) conv1d_silu_kernel(
             acc = fmaf(wt[K - 1][e], xt[e], acc);
             out[e] = silu_f32(acc);
         }
-        Vec8<IO>::store(y + (size_t)t * C + c0, out);
+        V::store(y + (size_t)t * C + c0, out);
 #pragma unroll
         for (int j = 0; j + 1 < K - 1; ++j)
 #pragma unroll
@@ -180,54 +180,52 @@ __global__ void __launch_bounds__(128) conv1d_silu_kernel(
 #pragma unroll
         for (int e = 0; e < kVec; ++e) win[K - 2][e] = xt[e];
     };
-    if (t0 + kTile <= s1) {  // the whole tile in one sequence
+#pragma unroll 1
+    for (int64_t g0 = tb; g0 < te; g0 += kConvGroup) {
+        const bool more = g0 + kConvGroup < te;
+        typename V::Raw nxt[kConvGroup];
+        if (more) {
 #pragma unroll
-        for (int j = 0; j < K - 1; ++j) {
-            const int64_t p = t0 - (K - 1) + j;
-            if (p >= s0) {
-                Vec8<IO>::unpack(wb[j], win[j]);
-            } else if (state_in) {
-                Vec8<IO>::load(state_in + ((size_t)n * (K - 1) + (K - 1) + (p - s0)) * C + c0,
-                               win[j]);
-            } else {
-#pragma unroll
-                for (int e = 0; e < kVec; ++e) win[j][e] = 0.f;
+            for (int i = 0; i < kConvGroup; ++i) {
+                const int64_t t = g0 + kConvGroup + i;
+                nxt[i] = V::load_raw(x + (size_t)(t < te ? t : te - 1) * C + c0);
             }
         }
 #pragma unroll
-        for (int i = 0; i < kTile; ++i) {
-            float xt[kVec];
-            Vec8<IO>::unpack(xb[i], xt);
-            step(xt, t0 + i);
-        }
-        return;
-    }
-    fill_window(t0);
-    const int64_t t_end = t0 + kTile < T ? t0 + kTile : T;
-    for (int64_t t = t0; t < t_end; ++t) {
-        if (t >= s1) {  // the next non-empty sequence starts here
-            while (t >= s1) {
-                if (n + 1 >= N) {  // tokens past cu[N]
-                    set_status(status, kStatusBadSeqlens);
-                    return;
+        for (int i = 0; i < kConvGroup; ++i) {
+            const int64_t t = g0 + i;
+            if (t < te) {
+                if (t >= s1) {  // the next non-empty sequence starts here
+                    while (t >= s1) {
+                        if (n + 1 >= N) {  // tokens past cu[N]
+                            set_status(status, kStatusBadSeqlens);
+                            return;
+                        }
+                        ++n;
+                        s0 = s1;
+                        s1 = cu[n + 1];
+                        if (s1 < s0) {
+                            set_status(status, kStatusBadSeqlens);
+                            return;
+                        }
+                    }
+                    if (s1 > T) {
+                        set_status(status, kStatusBadSeqlens);
+                        return;
+                    }
+                    // t == s0: the whole window precedes the sequence
+#pragma unroll
+                    for (int j = 0; j < K - 1; ++j) window_entry(t - (K - 1) + j, win[j]);
                 }
-                ++n;
-                s0 = s1;
-                s1 = cu[n + 1];
-                if (s1 < s0) {
-                    set_status(status, kStatusBadSeqlens);
-                    return;
-                }
+                float xt[kVec];
+                V::unpack(cur[i], xt);
+                step(xt, t);
             }
-            if (s1 > T || s0 < 0) {
-                set_status(status, kStatusBadSeqlens);
-                return;
-            }
-            fill_window(t);
         }
-        float xt[kVec];
-        Vec8<IO>::load(x + (size_t)t * C + c0, xt);
-        step(xt, t);
+        if (more) {
+#pragma unroll
+            for (int i = 0; i < kConvGroup; ++i) cur[i] = nxt[i];
+        }
     }
 }
 
@@ -380,9 +378,8 @@ cudaError_t conv_launch(const void* x, const float* w, const float* bias, const 
     const int64_t nv = C / kVec;
     if (T > 0) {
         const int threads = 128;
-        constexpr int kTile = ConvTile<IO>::value;
-        const int64_t tiles = (T + kTile - 1) / kTile;
-        conv1d_silu_kernel<IO, K><<<blocks_for(tiles * nv, threads), threads, 0, s>>>(
+        const int64_t ranges = (T + kConvRange - 1) / kConvRange;
+        conv1d_silu_kernel<IO, K><<<blocks_for(ranges * nv, threads), threads, 0, s>>>(
             static_cast<const IO*>(x), w, bias, static_cast<const IO*>(state_in), cu, N, T, C,
             static_cast<IO*>(y), status);
         const cudaError_t e = cudaGetLastError();
