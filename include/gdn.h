@@ -75,8 +75,11 @@ int gdn_version(void);
  * covers the tensor-core path: the chunk offsets of the sequences, then per
  * (64-token chunk, V head) an 8-byte ready flag and a 17,664-byte record (the
  * chunk's T diag(beta) and P matrices and per-token factors), i.e. about 276
- * bytes per token and V head (with one extra chunk per sequence), each part
- * rounded up to 256 bytes; for d = 64 (CUDA-core path) it is the per-token G and
+ * bytes per token and V head (with one extra chunk per sequence), the first two
+ * parts rounded up to 256 bytes; while GDN_IMPL_TENSOR_CORE_GRAM is selected, also
+ * an 8,192-byte tile per (chunk, QK head) (the cross-chunk key Gram matrix), so a
+ * workspace sized under another setting is too small for that one (the call then
+ * returns GDN_ERR_WORKSPACE); for d = 64 (CUDA-core path) it is the per-token G and
  * beta, fp32 [T, H_v] each. Returns 0 for invalid sizes (and for num_seqs = 0).
  * The workspace needs no initialisation: a ready flag holds the number of the
  * call that wrote it, and call numbers grow within the process.
@@ -147,7 +150,15 @@ int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
  *                         that own 64 value rows each);
  *   GDN_IMPL_TENSOR_CORE_WHOLE_ROWS
  *                         the one-launch schedule whenever it applies, but never
- *                         with half-row chain blocks.
+ *                         with half-row chain blocks;
+ *   GDN_IMPL_TENSOR_CORE_GRAM
+ *                         as GDN_IMPL_TENSOR_CORE, but half-row chain blocks form
+ *                         S_c K_c^T as e^{G_L} S_{c-1} K_c^T + W_{c-1} (K_{c-1} K_c^T)
+ *                         with the cross-chunk key Gram matrix from the
+ *                         preparation, which takes the state update off the path
+ *                         from one chunk to the next (the same mathematics with a
+ *                         different bf16 rounding, so not bit-identical to the
+ *                         other schedules).
  * Returns the previous setting, or -GDN_ERR_INVALID_ARG for an unknown value.
  * Not synchronised with calls in flight on other host threads.
  */
@@ -156,7 +167,8 @@ enum {
     GDN_IMPL_CUDA_CORE = 1,
     GDN_IMPL_TENSOR_CORE = 2,
     GDN_IMPL_TENSOR_CORE_SPLIT = 3,
-    GDN_IMPL_TENSOR_CORE_WHOLE_ROWS = 4
+    GDN_IMPL_TENSOR_CORE_WHOLE_ROWS = 4,
+    GDN_IMPL_TENSOR_CORE_GRAM = 5
 };
 int gdn_set_prefill_impl(int32_t impl);
 

@@ -126,7 +126,8 @@ size_t gdn_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_
     if (num_seqs == 0) return 0;  // an empty batch launches nothing
     const size_t simt = 2 * gate_bytes(total_tokens, H_v);
     if (d_k != 128) return simt;
-    const size_t tc = prefill_tc_workspace_bytes(num_seqs, total_tokens, H_v);
+    const bool gram = g_prefill_impl.load(std::memory_order_relaxed) == GDN_IMPL_TENSOR_CORE_GRAM;
+    const size_t tc = prefill_tc_workspace_bytes(num_seqs, total_tokens, H_qk, H_v, gram);
     return tc > simt ? tc : simt;
 }
 
@@ -179,7 +180,7 @@ int prefill_common(const void* q, const void* k, const void* v, int32_t io_dtype
     const bool tc_ok =
         io_dtype == GDN_BF16 && d_k == 128 && prefill_tc_supported(H_qk, H_v);
     if ((impl == GDN_IMPL_TENSOR_CORE || impl == GDN_IMPL_TENSOR_CORE_SPLIT ||
-         impl == GDN_IMPL_TENSOR_CORE_WHOLE_ROWS) && !tc_ok)
+         impl == GDN_IMPL_TENSOR_CORE_WHOLE_ROWS || impl == GDN_IMPL_TENSOR_CORE_GRAM) && !tc_ok)
         return GDN_ERR_UNSUPPORTED;
     int* st = device_status_ptr();
     if (!st) return GDN_ERR_CUDA;
@@ -190,7 +191,8 @@ int prefill_common(const void* q, const void* k, const void* v, int32_t io_dtype
                                            cu_seqlens, num_seqs, total_tokens, H_qk, H_v, scale,
                                            o, final_state, sref, workspace,
                                            impl == GDN_IMPL_TENSOR_CORE_SPLIT ? 0
-                                           : impl == GDN_IMPL_TENSOR_CORE_WHOLE_ROWS ? 1 : 2,
+                                           : impl == GDN_IMPL_TENSOR_CORE_WHOLE_ROWS ? 1
+                                           : impl == GDN_IMPL_TENSOR_CORE_GRAM ? 3 : 2,
                                            st, s));
     }
     float* G = static_cast<float*>(workspace);
@@ -377,7 +379,8 @@ int gdn_rmsnorm_gated(const void* o, const void* z, int32_t io_dtype, const floa
 
 int gdn_set_prefill_impl(int32_t impl) {
     if (impl != GDN_IMPL_AUTO && impl != GDN_IMPL_CUDA_CORE && impl != GDN_IMPL_TENSOR_CORE &&
-        impl != GDN_IMPL_TENSOR_CORE_SPLIT && impl != GDN_IMPL_TENSOR_CORE_WHOLE_ROWS)
+        impl != GDN_IMPL_TENSOR_CORE_SPLIT && impl != GDN_IMPL_TENSOR_CORE_WHOLE_ROWS &&
+        impl != GDN_IMPL_TENSOR_CORE_GRAM)
         return -GDN_ERR_INVALID_ARG;
     return g_prefill_impl.exchange(impl);
 }

@@ -140,7 +140,8 @@ cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, int
 // cooperative launch where it pays (whole-row chain blocks), 2 = the same with half-row
 // chain blocks when the chains are few enough. The workspace holds the chunk offsets and
 // one record (T, P and per-token factors) per (chunk, V head).
-size_t prefill_tc_workspace_bytes(int32_t N, int64_t T, int32_t H_v);
+// `gram`: room for the cross-chunk Gram tiles of the Gram-matrix schedule (schedule 3)
+size_t prefill_tc_workspace_bytes(int32_t N, int64_t T, int32_t H_qk, int32_t H_v, bool gram);
 bool prefill_tc_supported(int32_t H_qk, int32_t H_v);
 cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const float* a,
                               const float* b, const float* A_log, const float* dt_bias,

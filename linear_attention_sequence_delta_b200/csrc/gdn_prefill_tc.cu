@@ -76,6 +76,10 @@ constexpr int RG_EGQ = 128;          //   [64] e^{G_t} rq_t
 constexpr int RG_EGL = 192;          //   [64] e^{G_L - G_t} rk_t
 constexpr int RG_GAMMA = 256;        //   e^{G_L}
 constexpr uint32_t kRecBytes = 17664;  // 69 x 256
+// Cross-chunk key Gram matrix of (chunk c, QK head): K_c K_{c-1}^T of the raw bf16 rows,
+// row n = token n of chunk c, column m = token m of chunk c-1, as a bf16 sw128 image
+// (zero for a sequence's first chunk).
+constexpr uint32_t kGramBytes = 8192;
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -256,15 +260,18 @@ __device__ __forceinline__ void publish_record(unsigned long long* flags, size_t
 
 // One prep worker of kPrepThreads threads (tid 0 .. 255, synchronised by the named
 // barrier bar_id) walks the (chunk, QK head) units worker, worker + nworkers, ...
-// and writes their records; with `flags`, each finished record is published.
+// and writes their records; with `flags`, each finished record is published. With
+// `gram`, it also writes each unit's cross-chunk key Gram matrix K_c K_{c-1}^T (the
+// previous chunk's raw K rows staged where A is built later; a second MMA beside
+// K K^T into TMEM columns 64-127) before the unit's first record is published.
 __device__ __forceinline__ void prep_worker(
     const bf16* __restrict__ q, const bf16* __restrict__ k, const float* __restrict__ a,
     const float* __restrict__ b, const float* __restrict__ A_log,
     const float* __restrict__ dt_bias, const int32_t* __restrict__ cu_seqlens,
     const int32_t* __restrict__ choff, int32_t N, int H_qk, int H_v, float scale,
-    uint8_t* __restrict__ rec, int* status, unsigned long long* flags,
-    unsigned long long epoch, uint8_t* sm, const int tid, const int bar_id, const int worker,
-    const int nworkers, const bool relinquish) {
+    uint8_t* __restrict__ rec, uint8_t* __restrict__ gram, int* status,
+    unsigned long long* flags, unsigned long long epoch, uint8_t* sm, const int tid,
+    const int bar_id, const int worker, const int nworkers, const bool relinquish) {
     uint8_t* KQ = sm + PS_KQ;
     float* Ts = reinterpret_cast<float*>(sm + PS_TS);
     float* As = reinterpret_cast<float*>(sm + PS_AS);
@@ -285,8 +292,9 @@ __device__ __forceinline__ void prep_worker(
     const int r = H_v / H_qk;
     const int total_units = choff[N] * H_qk;
 
+    const uint32_t tcols = gram ? 128u : 64u;
     if (warp == 0) {
-        tmem_alloc(s_tmem, 64);
+        tmem_alloc(s_tmem, tcols);
         if (relinquish) tmem_relinquish();
     }
     if (tid == 0) {
@@ -329,6 +337,13 @@ __device__ __forceinline__ void prep_worker(
             const uint32_t off = (uint32_t)(ch >> 3) * 16384u;
             cp_async_16(KQ + off + sw128_off(rr, ch & 7), k + rowk, live ? 16u : 0u);
             cp_async_16(KQ + off + sw128_off(rr + 64, ch & 7), q + rowk, live ? 16u : 0u);
+            if (gram) {  // the previous chunk's K rows (zeros before the sequence's start)
+                const bool prev = cg > choff[n];
+                const size_t rowp = ((size_t)(prev ? t0 - kC + rr : 0) * H_qk + j) * kD + ch * 8;
+                cp_async_16(reinterpret_cast<uint8_t*>(As) + (uint32_t)(ch >> 3) * 8192u +
+                                sw128_off(rr, ch & 7),
+                            k + rowp, prev ? 16u : 0u);
+            }
         }
         for (int idx = tid; idx < 2 * r * kC; idx += kPrepThreads) {
             const int which = idx / (r * kC);            // 0: a, 1: b
@@ -383,6 +398,16 @@ __device__ __forceinline__ void prep_worker(
                 mma_bf16_ss(tmem, smem_desc_sw128(kq + off, 16, 1024),
                             smem_desc_sw128(kq + off, 16, 1024), id_kq, ks > 0);
             }
+            if (gram) {  // [K; Q] K_{c-1}^T: rows 0-63 are the Gram matrix
+                const uint32_t kp = smem_u32(As);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t off = (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u;
+                    const uint32_t offp = (uint32_t)(ks >> 2) * 8192u + (uint32_t)(ks & 3) * 32u;
+                    mma_bf16_ss(tmem + 64, smem_desc_sw128(kq + off, 16, 1024),
+                                smem_desc_sw128(kp + offp, 16, 1024), id_kq, ks > 0);
+                }
+            }
             mma_commit(bar);
         }
         // ---- gates of every V head of the group: one warp per head, two tokens a lane:
@@ -422,6 +447,20 @@ __device__ __forceinline__ void prep_worker(
         tc_fence_after();
         float x[32];  // this thread's half row of [K; Q] K^T, shared by the r V heads
         tmem_ld32_sync(tl + 32 * hh, x);
+        if (gram && trow < 64) {  // Gram row trow, columns 32 hh .. + 31 -> bf16 image
+            float gv[32];
+            tmem_ld32_sync(tl + 64 + 32 * hh, gv);
+            uint8_t* G = gram + ((size_t)cg * H_qk + j) * kGramBytes;
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                uint4 w;
+                w.x = pack_bf16x2(gv[8 * q4 + 0], gv[8 * q4 + 1]);
+                w.y = pack_bf16x2(gv[8 * q4 + 2], gv[8 * q4 + 3]);
+                w.z = pack_bf16x2(gv[8 * q4 + 4], gv[8 * q4 + 5]);
+                w.w = pack_bf16x2(gv[8 * q4 + 6], gv[8 * q4 + 7]);
+                *reinterpret_cast<uint4*>(G + sw128_off((uint32_t)trow, 4 * hh + q4)) = w;
+            }
+        }
 
 #pragma unroll 1
         for (int hr = 0; hr < r; ++hr) {
@@ -581,7 +620,7 @@ __device__ __forceinline__ void prep_worker(
     named_bar_sync(bar_id, kPrepThreads);
     tc_fence_after();
     if (failed && tid == 0) set_status(status, kStatusTimeout);
-    if (warp == 0) tmem_dealloc(tmem, 64);
+    if (warp == 0) tmem_dealloc(tmem, tcols);
 }
 
 __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
@@ -593,8 +632,8 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    prep_worker(q, k, a, b, A_log, dt_bias, cu_seqlens, choff, N, H_qk, H_v, scale, rec, status,
-                nullptr, 0, sm, threadIdx.x, 1, blockIdx.x, gridDim.x, true);
+    prep_worker(q, k, a, b, A_log, dt_bias, cu_seqlens, choff, N, H_qk, H_v, scale, rec, nullptr,
+                status, nullptr, 0, sm, threadIdx.x, 1, blockIdx.x, gridDim.x, true);
 }
 
 // ==================================== chain =======================================
@@ -603,6 +642,11 @@ constexpr int kChain = 256;
 constexpr int kOut = 128;
 constexpr int kIssueWarp = 8;
 constexpr int kRdyBar = 6;     // named barrier: state threads arrive, the issuing warp waits
+// The Gram-matrix schedule gives each of its three steps its own barrier (6, 7, 8): its
+// state warps may arrive for step 2 before the issuing warp has passed step 1 (nothing
+// between the two waits for the issuing warp), and a barrier must not be arrived at
+// twice before it completes.
+constexpr int kRdyBarZ = 6, kRdyBarS = 7, kRdyBarV = 8;
 constexpr int kRdyCount = 288;
 constexpr int kLoadWarp = 9;
 constexpr int kRing = 3;
@@ -619,6 +663,10 @@ constexpr uint32_t CS_ERR = CS_BAR + 132;
 constexpr uint32_t CS_EGQ = CS_BAR + 256;           // [64] fp32: the chunk's output row factors
 constexpr size_t kChainSmem = CS_EGQ + 256 + 1024;
 
+// Slot of the Gram-matrix schedule (half rows): the block's half of V at SLOT_V, the
+// chunk's Gram tile in the other half's place.
+constexpr uint32_t SLOT_GRAM = SLOT_V + 8192;
+
 // tensor memory columns (512 allocated)
 constexpr uint32_t TM_U = 0;      // 128: the chunk's state increment (scaled Vn^T) K, fp32
 constexpr uint32_t TM_S0B = 128;  // 64: state as bf16 pairs
@@ -629,6 +677,14 @@ constexpr uint32_t TM_D3 = 320;   // 64: Vn^T; Vn^T pairs overwrite columns 0-15
 constexpr uint32_t TM_D1Q1 = 384; // 64: S0 Q^T of odd chunks
 constexpr uint32_t TM_D4 = 448;   // 64: Vn^T P^T
 constexpr uint32_t kTmemCols = 512;
+// ... and of the Gram-matrix schedule: U 0-127 as above, then
+constexpr uint32_t TG_S0B = 128;  // 64: S_c as bf16 pairs (A operand of S_c Q_c^T)
+constexpr uint32_t TG_GS = 192;   // 64: e^{G_L} S_c as bf16 pairs (of S_c K_{c+1}^T)
+constexpr uint32_t TG_R = 256;    // 64: S_c K_c^T; Z^T pairs overwrite columns 0-15, 32-47
+constexpr uint32_t TG_D3 = 320;   // 64: Vn^T; Vn^T pairs overwrite columns 0-15, 32-47 and
+                                  //     the decay-scaled pairs columns 16-31, 48-63
+constexpr uint32_t TG_D1Q = 384;  // 64: S_c Q_c^T (one accumulator)
+constexpr uint32_t TG_D4 = 448;   // 64: Vn^T P^T
 
 // Column (in 32-bit words) of the K=16 slice ks of a 64-token bf16 operand that
 // two warps wrote in place over the fp32 columns they had read: tokens 0-31 at
@@ -677,22 +733,25 @@ __device__ __forceinline__ bool wait_record(const unsigned long long* flag,
 // threads of a block (tid 0 .. 415, synchronised by the named barrier sync_id) on
 // the tensor memory `tmem` (512 columns). With `flags`, a chunk's record is
 // copied only once a prep worker has published it.
-template <int kM>
+template <int kM, bool kGram>
 __device__ __forceinline__ void chain_unit(
     const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
     const CUtensorMap& tm_o, const float* S0g, const int32_t* __restrict__ cu_seqlens,
     const int32_t* __restrict__ choff, int64_t T_total, int H_qk, int H_v,
-    const uint8_t* __restrict__ rec, bf16* __restrict__ o, float* Sfg, const StateIndex sref,
-    int* status,
+    const uint8_t* __restrict__ rec, const uint8_t* __restrict__ gram, bf16* __restrict__ o,
+    float* Sfg, const StateIndex sref, int* status,
     const unsigned long long* flags, unsigned long long epoch, uint8_t* sm, const int tid,
     const int n, const int h, const int hv, const uint32_t tmem,
     const int sync_id) {
     static_assert(kM == 128 || kM == 64, "a chain block owns all 128 value rows or one half");
+    static_assert(!kGram || kM == 64, "the Gram-matrix schedule runs on half rows");
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + CS_BAR);  // [3] slot landed
     uint64_t* mbar = full + kRing;         // chain MMA completions
     uint64_t* obar = mbar + 1;             // [2] chunk parity b: output accumulators complete
     uint64_t* ofree = mbar + 3;            // [2] chunk parity b: output accumulators read
     uint64_t* dbar = mbar + 5;             // drain of in-flight MMAs before the exit
+    uint64_t* kbar = mbar + 6;             // Gram schedule: S_c K_c^T complete (mbar: Vn^T)
+    uint64_t* ubar = mbar + 7;             // Gram schedule: the state increment complete
     volatile int* s_err = reinterpret_cast<volatile int*>(sm + CS_ERR);
 
     const int warp = tid >> 5, lane = tid & 31;
@@ -711,6 +770,8 @@ __device__ __forceinline__ void chain_unit(
         mbar_init(&ofree[0], 4);
         mbar_init(&ofree[1], 4);
         mbar_init(dbar, 1);
+        mbar_init(kbar, 1);
+        mbar_init(ubar, 1);
         *s_err = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -736,8 +797,12 @@ __device__ __forceinline__ void chain_unit(
         tma_load_3d(slot + SLOT_KQ + 16384, &tm_k, 64, j, t0, &full[st]);
         tma_load_3d(slot + SLOT_KQ + 8192, &tm_q, 0, j, t0, &full[st]);
         tma_load_3d(slot + SLOT_KQ + 16384 + 8192, &tm_q, 64, j, t0, &full[st]);
-        tma_load_3d(slot + SLOT_V, &tm_v, 0, h, t0, &full[st]);
-        tma_load_3d(slot + SLOT_V + 8192, &tm_v, 64, h, t0, &full[st]);
+        if constexpr (kGram) {
+            tma_load_3d(slot + SLOT_V, &tm_v, 64 * hv, h, t0, &full[st]);
+        } else {
+            tma_load_3d(slot + SLOT_V, &tm_v, 0, h, t0, &full[st]);
+            tma_load_3d(slot + SLOT_V + 8192, &tm_v, 64, h, t0, &full[st]);
+        }
     };
     // After a wait that ran out the record is copied all the same (valid memory, the
     // results are discarded), so that the slot's barrier completes and no copy is left
@@ -754,6 +819,9 @@ __device__ __forceinline__ void chain_unit(
         if (flags) asm volatile("fence.proxy.async.global;" ::: "memory");  // read by TMA
         bulk_g2s(sm + st * kSlotBytes + SLOT_REC, rec + ((size_t)(cg0 + c) * H_v + h) * kRecBytes,
                  kRecBytes, &full[st]);
+        if constexpr (kGram)  // written before the record was published
+            bulk_g2s(sm + st * kSlotBytes + SLOT_GRAM,
+                     gram + ((size_t)(cg0 + c) * H_qk + j) * kGramBytes, kGramBytes, &full[st]);
     };
 
     if (warp > kIssueWarp) {
@@ -781,7 +849,6 @@ __device__ __forceinline__ void chain_unit(
             const int cn = cp + kRing;  // the chunk that will reuse this chunk's slot
             // its record's flag is checked while this chunk's MMAs still run
             const bool next = loader && cn < nchunks && issued == cn;
-            if (next) record_ready(cn);
             const bool ok = mbar_wait_bounded(&obar[b], (cp >> 1) & 1, kWaitCycles);
             if (!ok) *s_err = 1;
             if (loader) bulk_wait_group_read<0>();  // staging free again
@@ -790,14 +857,9 @@ __device__ __forceinline__ void chain_unit(
                 reinterpret_cast<float4*>(egq)[to] = reinterpret_cast<const float4*>(
                     sm + (cp % kRing) * kSlotBytes + SLOT_REC + REC_G + 4 * RG_EGQ)[to];
             if (named_bar_any(2, kOut, !ok || *s_err != 0)) break;
-            if (next) {  // the slot is free: refill it now, two chunks before it is needed
-                load_tiles(cn);
-                load_record(cn);
-                issued = cn + 1;
-            }
             tc_fence_after();
             const float4* eg4 = reinterpret_cast<const float4*>(egq);
-            const uint32_t qacc = ctl + (b ? TM_D1Q1 : TM_D1Q0);
+            const uint32_t qacc = ctl + (kGram ? TG_D1Q : b ? TM_D1Q1 : TM_D1Q0);
             if constexpr (kM == 128) {
                 // this thread's column of the staged tile; laundered so that the 64 element
                 // addresses are formed per chunk rather than held in registers across chunks
@@ -853,6 +915,16 @@ __device__ __forceinline__ void chain_unit(
                     }
                 }
             }
+            // The slot is free: refill it with the chunk three ahead. Its record's flag is
+            // checked only now, after the accumulators were read (an acquire load of the
+            // flag is an L2 round trip; before the read it delayed every chunk's output).
+            if (next) {
+                record_ready(cn);
+                load_tiles(cn);
+                load_record(cn);
+                issued = cn + 1;
+            }
+            __syncwarp();
             fence_proxy_async_smem();
             named_bar_sync(2, kOut);  // staged; every output warp is done with the slot
             const int64_t t0 = s0 + (int64_t)cp * kC;
@@ -893,8 +965,8 @@ __device__ __forceinline__ void chain_unit(
         // ================================ MMA issue =====================================
         // Three waits per chunk on the state threads' barrier, always (after an error
         // the MMAs are skipped but the waits stay, so every arrival is consumed).
-        auto wait_rdy = [&]() {
-            named_bar_sync(kRdyBar, kRdyCount);
+        auto wait_rdy = [&](int id = kRdyBar) {
+            named_bar_sync(id, kRdyCount);
             tc_fence_after();
         };
         bool dead = false;
@@ -915,66 +987,181 @@ __device__ __forceinline__ void chain_unit(
             dead = __any_sync(0xffffffffu, dead || !ok || *s_err != 0);
             if (dead) *s_err = 1;
         };
-#pragma unroll 1
-        for (int c = 0; c < nchunks; ++c) {
-            const int st = c % kRing;
-            uint8_t* slot = sm + st * kSlotBytes;
-            const uint32_t kq = smem_u32(slot + SLOT_KQ);
-            const uint32_t vt = smem_u32(slot + SLOT_V);
-            const uint32_t tt = smem_u32(slot + SLOT_REC + REC_T);
-            const uint32_t ptile = smem_u32(slot + SLOT_REC + REC_P);
-            // shared-memory descriptors of this chunk's operands, formed while waiting
-            uint64_t dK0[4], dK1[4], dQ0[4], dQ1[4], dV[4], dT[4], dKm[4], dP[4];
+        if constexpr (kGram) {
+            // Per chunk c: (1) Z_c written -> Vn_c += Z_c (T diag(beta))^T; (2) S_c and
+            // e^{G_L} S_c written -> chunk c+1's S_{c+1} K_{c+1}^T begins as
+            // e^{G_L} S_c K_{c+1}^T; (3) the Vn_c and decay-scaled pairs W_c written ->
+            // S_{c+1} K_{c+1}^T += W_c (K_c K_{c+1}^T) (the Gram tile; it completes the
+            // product, since S_{c+1} = e^{G_L} S_c + W_c K_c), the increment W_c K_c,
+            // S_c Q_c^T, Vn_c P_c^T, and chunk c+1's V^T (T diag(beta))^T. MMAs run in issue
+            // order, so an accumulator is overwritten only after the MMAs that read it before.
+            uint32_t aS0[4], aS1[4], aG0[4], aG1[4], aZ[4], aW[4], aN[4];
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
-                dK0[ks] = smem_desc_sw128(kq + ks * 32u, 16, 1024);
-                dK1[ks] = smem_desc_sw128(kq + 16384u + ks * 32u, 16, 1024);
-                dQ0[ks] = smem_desc_sw128(kq + 8192u + ks * 32u, 16, 1024);
-                dQ1[ks] = smem_desc_sw128(kq + 16384u + 8192u + ks * 32u, 16, 1024);
-                // V^T rows = value rows: this block's half of them when kM = 64
-                dV[ks] = smem_desc_sw128(vt + (kM == 64 ? 8192u * hv : 0u) + ks * 2048u, 8192, 1024);
-                dT[ks] = smem_desc_sw128(tt + ks * 32u, 16, 1024);
-                dKm[ks] = smem_desc_sw128(kq + ks * 2048u, 16384, 1024);
-                dP[ks] = smem_desc_sw128(ptile + ks * 32u, 16, 1024);
+                aS0[ks] = tmem + TG_S0B + 8 * ks;
+                aS1[ks] = tmem + TG_S0B + 8 * (ks + 4);
+                aG0[ks] = tmem + TG_GS + 8 * ks;
+                aG1[ks] = tmem + TG_GS + 8 * (ks + 4);
+                aZ[ks] = tmem + TG_R + split_pairs_col(ks);
+                aN[ks] = tmem + TG_D3 + split_pairs_col(ks);
+                aW[ks] = tmem + TG_D3 + 16 + split_pairs_col(ks);
             }
-            if (!dead) check(mbar_wait_bounded(&full[st], (c / kRing) & 1, kWaitCycles));
-            // (1) the bf16 state is written: S0 K^T, then V^T (T diag(beta))^T
-            wait_rdy();
-            check(true);
-            if (!dead) {
-                mma_ts_group4(tmem + TM_D1K, aS0, dK0, id64, 0);
-                mma_ts_group4(tmem + TM_D1K, aS1, dK1, id64, 1);
-                mma_commit_warp(mbar);
-                mma_ss_group4(tmem + TM_D3, dV, dT, id_v, 0);
+            // S K^T of the chunk in slot st (K rows as B, K-major), then its V^T
+            // (T diag(beta))^T
+            auto issue_sk = [&](int st) {
+                const uint32_t kq = smem_u32(sm + st * kSlotBytes + SLOT_KQ);
+                uint64_t d0[4], d1[4];
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    d0[ks] = smem_desc_sw128(kq + ks * 32u, 16, 1024);
+                    d1[ks] = smem_desc_sw128(kq + 16384u + ks * 32u, 16, 1024);
+                }
+                mma_ts_group4(tmem + TG_R, aG0, d0, id64, 0);
+                mma_ts_group4(tmem + TG_R, aG1, d1, id64, 1);
+            };
+            auto issue_vpart = [&](int st) {
+                uint8_t* slot = sm + st * kSlotBytes;
+                const uint32_t vt = smem_u32(slot + SLOT_V);
+                const uint32_t tt = smem_u32(slot + SLOT_REC + REC_T);
+                uint64_t dV[4], dT[4];
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    dV[ks] = smem_desc_sw128(vt + ks * 2048u, 8192, 1024);
+                    dT[ks] = smem_desc_sw128(tt + ks * 32u, 16, 1024);
+                }
+                mma_ss_group4(tmem + TG_D3, dV, dT, id_v, 0);
+            };
+            // chunk 0: S_0 K_0^T from the initial state (written to TG_GS by the state warps)
+            if (nchunks > 0) {
+                if (!dead) check(mbar_wait_bounded(&full[0], 0, kWaitCycles));
+                wait_rdy(kRdyBarZ);
+                check(true);
+                if (!dead) {
+                    issue_sk(0);
+                    mma_commit_warp(kbar);
+                    issue_vpart(0);
+                }
             }
-            // (2) Z^T is written: Vn^T += Z^T (T diag(beta))^T; then S0 Q^T into the
-            // accumulator of parity c & 1, last read for chunk c - 2
-            wait_rdy();
-            check(true);
-            if (!dead) {
-                mma_ts_group4(tmem + TM_D3, aZ, dT, id64, 1);
-                mma_commit_warp(mbar);
-                if (c >= 2)
-                    check(mbar_wait_bounded(&ofree[c & 1], ((c - 2) >> 1) & 1, kWaitCycles));
+#pragma unroll 1
+            for (int c = 0; c < nchunks; ++c) {
+                const int st = c % kRing;
+                const int sn = (c + 1) % kRing;
+                const bool more = c + 1 < nchunks;
+                uint8_t* slot = sm + st * kSlotBytes;
+                const uint32_t kq = smem_u32(slot + SLOT_KQ);
+                const uint32_t tt = smem_u32(slot + SLOT_REC + REC_T);
+                const uint32_t ptile = smem_u32(slot + SLOT_REC + REC_P);
+                const uint32_t gt = smem_u32(sm + sn * kSlotBytes + SLOT_GRAM);
+                uint64_t dQ0[4], dQ1[4], dT[4], dKm[4], dP[4], dG[4];
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    dQ0[ks] = smem_desc_sw128(kq + 8192u + ks * 32u, 16, 1024);
+                    dQ1[ks] = smem_desc_sw128(kq + 16384u + 8192u + ks * 32u, 16, 1024);
+                    dT[ks] = smem_desc_sw128(tt + ks * 32u, 16, 1024);
+                    dKm[ks] = smem_desc_sw128(kq + ks * 2048u, 16384, 1024);
+                    dP[ks] = smem_desc_sw128(ptile + ks * 32u, 16, 1024);
+                    dG[ks] = smem_desc_sw128(gt + ks * 32u, 16, 1024);
+                }
+                // (1) Z_c
+                wait_rdy(kRdyBarZ);
+                check(true);
+                if (!dead) {
+                    mma_ts_group4(tmem + TG_D3, aZ, dT, id64, 1);
+                    mma_commit_warp(mbar);
+                }
+                // (2) S_c, e^{G_L} S_c: chunk c+1's S K^T begins
+                wait_rdy(kRdyBarS);
+                check(true);
+                if (!dead && more)
+                    check(mbar_wait_bounded(&full[sn], ((c + 1) / kRing) & 1, kWaitCycles));
+                if (!dead && more) issue_sk(sn);
+                // (3) Vn_c pairs and W_c pairs. The path to the next chunk goes first; S_c Q_c^T
+                // waits until the output accumulators were read for chunk c - 1, and the
+                // increment's commit follows it (the state warps rewrite S_c's pairs only
+                // after that commit).
+                wait_rdy(kRdyBarV);
+                check(true);
+                if (!dead) {
+                    if (more) {
+                        mma_ts_group4(tmem + TG_R, aW, dG, id64, 1);
+                        mma_commit_warp(kbar);
+                    }
+                    mma_ts_group4(tmem + TM_U, aW, dKm, id_s, 0);
+                    if (c >= 1)
+                        check(mbar_wait_bounded(&ofree[(c - 1) & 1], ((c - 1) >> 1) & 1,
+                                                kWaitCycles));
+                }
+                if (!dead) {
+                    mma_ts_group4(tmem + TG_D1Q, aS0, dQ0, id64, 0);
+                    mma_ts_group4(tmem + TG_D1Q, aS1, dQ1, id64, 1);
+                    mma_commit_warp(ubar);
+                    mma_ts_group4(tmem + TG_D4, aN, dP, id64, 0);
+                    mma_commit_warp(&obar[c & 1]);
+                    if (more) issue_vpart(sn);
+                }
             }
-            if (!dead) {
-                const uint32_t qacc = tmem + ((c & 1) ? TM_D1Q1 : TM_D1Q0);
-                mma_ts_group4(qacc, aS0, dQ0, id64, 0);
-                mma_ts_group4(qacc, aS1, dQ1, id64, 1);
-            }
-            // (3) the Vn^T pairs are written: the state increment, then Vn^T P^T
-            wait_rdy();
-            check(true);
-            if (!dead) {
-                mma_ts_group4(tmem + TM_U, aU, dKm, id_s, 0);
-                mma_commit_warp(mbar);
-                if (c >= 1)
-                    check(mbar_wait_bounded(&ofree[(c - 1) & 1], ((c - 1) >> 1) & 1,
-                                            kWaitCycles));
-            }
-            if (!dead) {
-                mma_ts_group4(tmem + TM_D4, aN, dP, id64, 0);
-                mma_commit_warp(&obar[c & 1]);
+        } else {
+    #pragma unroll 1
+            for (int c = 0; c < nchunks; ++c) {
+                const int st = c % kRing;
+                uint8_t* slot = sm + st * kSlotBytes;
+                const uint32_t kq = smem_u32(slot + SLOT_KQ);
+                const uint32_t vt = smem_u32(slot + SLOT_V);
+                const uint32_t tt = smem_u32(slot + SLOT_REC + REC_T);
+                const uint32_t ptile = smem_u32(slot + SLOT_REC + REC_P);
+                // shared-memory descriptors of this chunk's operands, formed while waiting
+                uint64_t dK0[4], dK1[4], dQ0[4], dQ1[4], dV[4], dT[4], dKm[4], dP[4];
+    #pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    dK0[ks] = smem_desc_sw128(kq + ks * 32u, 16, 1024);
+                    dK1[ks] = smem_desc_sw128(kq + 16384u + ks * 32u, 16, 1024);
+                    dQ0[ks] = smem_desc_sw128(kq + 8192u + ks * 32u, 16, 1024);
+                    dQ1[ks] = smem_desc_sw128(kq + 16384u + 8192u + ks * 32u, 16, 1024);
+                    // V^T rows = value rows: this block's half of them when kM = 64
+                    dV[ks] = smem_desc_sw128(vt + (kM == 64 ? 8192u * hv : 0u) + ks * 2048u, 8192, 1024);
+                    dT[ks] = smem_desc_sw128(tt + ks * 32u, 16, 1024);
+                    dKm[ks] = smem_desc_sw128(kq + ks * 2048u, 16384, 1024);
+                    dP[ks] = smem_desc_sw128(ptile + ks * 32u, 16, 1024);
+                }
+                if (!dead) check(mbar_wait_bounded(&full[st], (c / kRing) & 1, kWaitCycles));
+                // (1) the bf16 state is written: S0 K^T, then V^T (T diag(beta))^T
+                wait_rdy();
+                check(true);
+                if (!dead) {
+                    mma_ts_group4(tmem + TM_D1K, aS0, dK0, id64, 0);
+                    mma_ts_group4(tmem + TM_D1K, aS1, dK1, id64, 1);
+                    mma_commit_warp(mbar);
+                    mma_ss_group4(tmem + TM_D3, dV, dT, id_v, 0);
+                }
+                // (2) Z^T is written: Vn^T += Z^T (T diag(beta))^T; then S0 Q^T into the
+                // accumulator of parity c & 1, last read for chunk c - 2
+                wait_rdy();
+                check(true);
+                if (!dead) {
+                    mma_ts_group4(tmem + TM_D3, aZ, dT, id64, 1);
+                    mma_commit_warp(mbar);
+                    if (c >= 2)
+                        check(mbar_wait_bounded(&ofree[c & 1], ((c - 2) >> 1) & 1, kWaitCycles));
+                }
+                if (!dead) {
+                    const uint32_t qacc = tmem + ((c & 1) ? TM_D1Q1 : TM_D1Q0);
+                    mma_ts_group4(qacc, aS0, dQ0, id64, 0);
+                    mma_ts_group4(qacc, aS1, dQ1, id64, 1);
+                }
+                // (3) the Vn^T pairs are written: the state increment, then Vn^T P^T
+                wait_rdy();
+                check(true);
+                if (!dead) {
+                    mma_ts_group4(tmem + TM_U, aU, dKm, id_s, 0);
+                    mma_commit_warp(mbar);
+                    if (c >= 1)
+                        check(mbar_wait_bounded(&ofree[(c - 1) & 1], ((c - 1) >> 1) & 1,
+                                                kWaitCycles));
+                }
+                if (!dead) {
+                    mma_ts_group4(tmem + TM_D4, aN, dP, id64, 0);
+                    mma_commit_warp(&obar[c & 1]);
+                }
             }
         }
         __syncwarp();
@@ -1149,7 +1336,7 @@ __device__ __forceinline__ void chain_unit(
                 for (int e = 0; e < 16; ++e)
                     d4[e] = make_float4(S[4 * e], S[4 * e + 1], S[4 * e + 2], S[4 * e + 3]);
             }
-        } else {
+        } else if constexpr (!kGram) {
             // ======================= state, one half of the value rows =======================
             // The block's 64 value rows 64 hv .. 64 hv + 63 sit in TMEM lanes 0-15 of each lane
             // quarter (M = 64 layout): warp w takes quarter qd = w & 3 (rows 16 qd ..) and the
@@ -1304,6 +1491,173 @@ __device__ __forceinline__ void chain_unit(
                         make_float2(S[4 * jj + 2], S[4 * jj + 3]);
                 }
             }
+        } else {
+            // ============ state, one half of the value rows, Gram-matrix schedule ============
+            // Layout as in the half-row schedule above (rows r0, r0 + 8; column pairs cp2).
+            // Per chunk c: (A) S_c K_c^T complete -> Z_c; (B) S_c = e^{G_L} S_{c-1} + U_{c-1},
+            // then S_c and e^{G_L} S_c as bf16 pairs; (C) Vn_c complete -> Vn_c pairs and the
+            // decay-scaled pairs. Only (A) and (C) are on the path from chunk to chunk.
+            const int qd = warp & 3;
+            const int hh = warp >> 2;
+            const int r0 = 64 * hv + qd * 16 + (lane >> 2);
+            const int cp2 = 2 * (lane & 3);
+            const uint32_t ctl = tmem + ((uint32_t)(qd * 32) << 16);
+            bool rd, wr;
+            const int sidx = sref.resolve(n, rd, wr, tid == 0 ? status : nullptr);
+            const float* S0s = rd ? S0g : nullptr;
+            float* Sfs = wr ? Sfg : nullptr;
+            const size_t hbase = ((size_t)sidx * H_v + h) * kD * kD;
+            float S[32];  // S[4 j + e]: row r0 + 8 (e >> 1), column 64 hh + 8 j + cp2 + (e & 1)
+            if (S0s) {
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    const int col = 64 * hh + 8 * jj + cp2;
+                    const float2 f0 = *reinterpret_cast<const float2*>(S0s + hbase + (size_t)r0 * kD + col);
+                    const float2 f1 =
+                        *reinterpret_cast<const float2*>(S0s + hbase + (size_t)(r0 + 8) * kD + col);
+                    S[4 * jj] = f0.x; S[4 * jj + 1] = f0.y; S[4 * jj + 2] = f1.x; S[4 * jj + 3] = f1.y;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) S[e] = 0.f;
+            }
+
+            uint32_t kph = 0, uph = 0, vph = 0;
+            bool dead = false;  // warp-uniform: after an error only the barrier arrivals remain
+            auto wait_bar = [&](uint64_t* bar, uint32_t& ph) {
+                if (dead) return;
+                bool ok = *s_err == 0 && mbar_wait_bounded(bar, ph, kWaitCycles);
+                ph ^= 1u;
+                dead = __any_sync(0xffffffffu, !ok || *s_err != 0);
+                if (dead) *s_err = 1;
+                tc_fence_after();
+            };
+            auto wait_full = [&](int c) {  // chunk c's slot landed (its record is read here)
+                if (dead) return;
+                const bool okf =
+                    *s_err == 0 && mbar_wait_bounded(&full[c % kRing], (c / kRing) & 1, kWaitCycles);
+                dead = __any_sync(0xffffffffu, !okf || *s_err != 0);
+                if (dead) *s_err = 1;
+            };
+            auto signal_rdy = [&](int id) {
+                if (!dead) tmem_wait_st();
+                tc_fence_before();
+                if (dead) named_bar_sync(id, kRdyCount);
+                else named_bar_arrive(id, kRdyCount);
+            };
+            // A sequence's last chunk: rows past its end (the next sequence's tokens, or TMA
+            // zero fill) in chunk c's K, Q and V tiles are zeroed before any MMA reads them.
+            auto zero_tail = [&](int c) {
+                const int L = (int)min((int64_t)kC, s1 - (s0 + (int64_t)c * kC));
+                if (L >= kC) return;
+                wait_full(c);
+                if (dead) return;
+                uint8_t* slot = sm + (c % kRing) * kSlotBytes;
+                const int nz = (kC - L) * 8;  // 16-byte chunks per 64-column tile
+                for (int idx = tid; idx < 5 * nz; idx += kChain) {
+                    const int tile = idx / nz, r = L + (idx % nz) / 8, ch = idx & 7;
+                    const uint32_t base =
+                        tile < 4 ? SLOT_KQ + (tile >> 1) * 16384u + (tile & 1) * 8192u : SLOT_V;
+                    *reinterpret_cast<uint4*>(slot + base + r * 128 + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
+                }
+                fence_proxy_async_smem();
+            };
+            // bf16 pairs of scale * S (key k at column k / 2 of this block's rows)
+            auto pack_state = [&](uint32_t col, float scale) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    pk[2 * jj] = pack_bf16x2(scale * S[4 * jj], scale * S[4 * jj + 1]);
+                    pk[2 * jj + 1] = pack_bf16x2(scale * S[4 * jj + 2], scale * S[4 * jj + 3]);
+                }
+                tmem_st16r_x8(ctl + col + 32 * hh, pk);
+            };
+            auto apply_update = [&](float gamma) {
+                float u[32];
+                tmem_ld16r_x8_sync(ctl + TM_U + 64 * hh, u);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) S[e] = fmaf(gamma, S[e], u[e]);
+            };
+
+            // chunk 0's S K^T reads the initial state
+            if (nchunks > 0) {
+                if (!dead) {
+                    zero_tail(0);
+                    if (!dead) pack_state(TG_GS, 1.f);
+                }
+                signal_rdy(kRdyBarZ);
+            }
+            float gamma = 1.f;  // e^{G_L} of the chunk before
+#pragma unroll 1
+            for (int c = 0; c < nchunks; ++c) {
+                const float* rg =
+                    reinterpret_cast<const float*>(sm + (c % kRing) * kSlotBytes + SLOT_REC + REC_G);
+                const bool more = c + 1 < nchunks;
+                // ---- (A) Z^T = -(e^G rk) (S_c K_c^T), tokens 32 hh + 8 j + cp2, + 1 --------
+                wait_bar(kbar, kph);
+                wait_full(c);
+                if (!dead) {
+                    float x[16];
+                    tmem_ld16r_x4_sync(ctl + TG_R + 32 * hh, x);
+                    uint32_t pk[8];
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const float2 f = *reinterpret_cast<const float2*>(rg + RG_FK + 32 * hh + 8 * jj + cp2);
+                        pk[2 * jj] = pack_bf16x2(-f.x * x[4 * jj], -f.y * x[4 * jj + 1]);
+                        pk[2 * jj + 1] = pack_bf16x2(-f.x * x[4 * jj + 2], -f.y * x[4 * jj + 3]);
+                    }
+                    tmem_st16r_x4(ctl + TG_R + 32 * hh, pk);
+                }
+                signal_rdy(kRdyBarZ);
+                // ---- (B) the state of this chunk, its bf16 copies --------------------------
+                if (c > 0) {
+                    wait_bar(ubar, uph);
+                    if (!dead) apply_update(gamma);
+                }
+                if (!dead) {
+                    gamma = rg[RG_GAMMA];
+                    if (more) zero_tail(c + 1);
+                }
+                if (!dead) {
+                    pack_state(TG_S0B, 1.f);
+                    if (more) pack_state(TG_GS, gamma);
+                }
+                signal_rdy(kRdyBarS);
+                // ---- (C) Vn^T -> bf16 pairs (for P Vn) and decay-scaled pairs ---------------
+                wait_bar(mbar, vph);
+                if (!dead) {
+                    float x[16];
+                    tmem_ld16r_x4_sync(ctl + TG_D3 + 32 * hh, x);
+                    uint32_t pk[8], pw[8];
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const float2 w = *reinterpret_cast<const float2*>(rg + RG_EGL + 32 * hh + 8 * jj + cp2);
+                        pk[2 * jj] = pack_bf16x2(x[4 * jj], x[4 * jj + 1]);
+                        pk[2 * jj + 1] = pack_bf16x2(x[4 * jj + 2], x[4 * jj + 3]);
+                        pw[2 * jj] = pack_bf16x2(x[4 * jj] * w.x, x[4 * jj + 1] * w.y);
+                        pw[2 * jj + 1] = pack_bf16x2(x[4 * jj + 2] * w.x, x[4 * jj + 3] * w.y);
+                    }
+                    tmem_st16r_x4(ctl + TG_D3 + 32 * hh, pk);
+                    tmem_st16r_x4(ctl + TG_D3 + 32 * hh + 16, pw);
+                }
+                signal_rdy(kRdyBarV);
+            }
+            bool done = !dead;
+            if (done && nchunks > 0) {  // the last chunk's state update
+                wait_bar(ubar, uph);
+                done = !dead;
+                if (done) apply_update(gamma);
+            }
+            if (done && Sfs) {
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    const int col = 64 * hh + 8 * jj + cp2;
+                    *reinterpret_cast<float2*>(Sfs + hbase + (size_t)r0 * kD + col) =
+                        make_float2(S[4 * jj], S[4 * jj + 1]);
+                    *reinterpret_cast<float2*>(Sfs + hbase + (size_t)(r0 + 8) * kD + col) =
+                        make_float2(S[4 * jj + 2], S[4 * jj + 3]);
+                }
+            }
         }
     }
 
@@ -1333,9 +1687,9 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
-    chain_unit<128>(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v, rec, o,
-                    Sfg, sref, status, nullptr, 0, sm, threadIdx.x, blockIdx.x / H_v,
-                    blockIdx.x % H_v, 0, tmem, 1);
+    chain_unit<128, false>(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v,
+                           rec, nullptr, o, Sfg, sref, status, nullptr, 0, sm, threadIdx.x,
+                           blockIdx.x / H_v, blockIdx.x % H_v, 0, tmem, 1);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1358,7 +1712,7 @@ constexpr size_t kFusedSmem =
 constexpr int kChainSync = 5;  // named barrier of the chain threads in the fused kernel
 constexpr int kFusedMaxSeqs = 255;  // the fused kernel computes the chunk offsets itself
 
-template <int kM>
+template <int kM, bool kGram>
 __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -1367,9 +1721,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
     const float* __restrict__ dt_bias, const float* S0g,
     const int32_t* __restrict__ cu_seqlens, const int32_t* choff, int32_t N,
     int64_t T_total, int H_qk, int H_v, float scale, uint8_t* __restrict__ rec,
-    bf16* __restrict__ o, float* Sfg, const StateIndex sref, int* status,
-    unsigned long long* flags,
-    unsigned long long epoch, int c0) {
+    uint8_t* __restrict__ gram, bf16* __restrict__ o, float* Sfg, const StateIndex sref,
+    int* status, unsigned long long* flags, unsigned long long epoch, int c0) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ int32_t s_choff[kFusedMaxSeqs + 1];
     __shared__ int s_bad;
@@ -1410,8 +1763,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
     if ((int)blockIdx.x >= c0) {
         const int sub = tid >> 8;
         prep_worker(q, k, a, b, A_log, dt_bias, cu_seqlens, choff, N, H_qk, H_v, scale, rec,
-                    status, flags, epoch, sm + sub * kPrepRegion, tid & 255, 3 + sub,
-                    2 * ((int)blockIdx.x - c0) + sub, 2 * ((int)gridDim.x - c0), false);
+                    kGram ? gram : nullptr, status, flags, epoch, sm + sub * kPrepRegion,
+                    tid & 255, 3 + sub, 2 * ((int)blockIdx.x - c0) + sub,
+                    2 * ((int)gridDim.x - c0), false);
         return;
     }
     if (tid >= kChainThreads) return;
@@ -1427,9 +1781,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
     // block u: (sequence, V head) u, or with half-row blocks its half u & 1 of unit u >> 1
     const int u = kM == 64 ? (int)blockIdx.x >> 1 : (int)blockIdx.x;
     const int hv = kM == 64 ? (int)blockIdx.x & 1 : 0;
-    chain_unit<kM>(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v, rec, o,
-                   Sfg, sref, status, flags, epoch, sm, tid, u / H_v, u % H_v, hv, tmem,
-                   kChainSync);
+    chain_unit<kM, kGram>(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v,
+                          rec, gram, o, Sfg, sref, status, flags, epoch, sm, tid, u / H_v,
+                          u % H_v, hv, tmem, kChainSync);
     tc_fence_before();
     named_bar_sync(kChainSync, kChainThreads);
     tc_fence_after();
@@ -1438,24 +1792,27 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-// Workspace: chunk offsets [N + 1] | record flags [records] (64-bit call numbers) | records.
 struct TcWorkspace {
-    size_t off_flags, off_rec, total;
+    size_t off_flags, off_rec, off_gram, total;
 };
 
-TcWorkspace tc_workspace_layout(int32_t N, int64_t T, int32_t H_v) {
-    const size_t records = ((size_t)((T + kC - 1) / kC) + (size_t)N) * H_v;
+// Workspace: chunk offsets [N + 1] | record flags [records] (64-bit call numbers) |
+// records [chunks][H_v] | with the Gram-matrix schedule, Gram tiles [chunks][H_qk].
+TcWorkspace tc_workspace_layout(int32_t N, int64_t T, int32_t H_qk, int32_t H_v, bool gram) {
+    const size_t chunks = (size_t)((T + kC - 1) / kC) + (size_t)N;
+    const size_t records = chunks * H_v;
     TcWorkspace w;
     w.off_flags = align256((size_t)(N + 1) * sizeof(int32_t));
     w.off_rec = w.off_flags + align256(records * sizeof(unsigned long long));
-    w.total = w.off_rec + records * kRecBytes;
+    w.off_gram = w.off_rec + records * kRecBytes;
+    w.total = w.off_gram + (gram ? chunks * H_qk * kGramBytes : 0);
     return w;
 }
 
 }  // namespace
 
-size_t prefill_tc_workspace_bytes(int32_t N, int64_t T, int32_t H_v) {
-    return tc_workspace_layout(N, T, H_v).total;
+size_t prefill_tc_workspace_bytes(int32_t N, int64_t T, int32_t H_qk, int32_t H_v, bool gram) {
+    return tc_workspace_layout(N, T, H_qk, H_v, gram).total;
 }
 
 bool prefill_tc_supported(int32_t H_qk, int32_t H_v) { return H_v / H_qk <= kMaxGroup; }
@@ -1503,11 +1860,12 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
                               cudaStream_t s) {
     if (N == 0) return cudaSuccess;
     if (T > (int64_t)0x7FFFFFFF - kC) return cudaErrorInvalidValue;  // TMA token coordinates
-    const TcWorkspace ws = tc_workspace_layout(N, T, H_v);
+    const TcWorkspace ws = tc_workspace_layout(N, T, H_qk, H_v, schedule == 3);
     uint8_t* wb = static_cast<uint8_t*>(workspace);
     int32_t* choff = reinterpret_cast<int32_t*>(wb);
     unsigned long long* flags = reinterpret_cast<unsigned long long*>(wb + ws.off_flags);
     uint8_t* rec = wb + ws.off_rec;
+    uint8_t* gram = wb + ws.off_gram;
     // With no tokens the maps are never read; any aligned device address will do.
     CUtensorMap tm_q, tm_k, tm_v, tm_o;
     if (!make_rows_map(&tm_q, T > 0 ? q : workspace, H_qk, T) ||
@@ -1530,8 +1888,11 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
         // phases at full occupancy. With at most a quarter as many chains as SMs each
         // chain runs as two blocks of 64 value rows (half the per-thread state work on
         // the critical path).
-        const bool half = schedule == 2 && 4 * chain_units <= num_sms;
-        const void* kfn = half ? (const void*)fused_kernel<64> : (const void*)fused_kernel<128>;
+        const bool half = schedule >= 2 && 4 * chain_units <= num_sms;
+        const bool gram_sched = half && schedule == 3;
+        const void* kfn = gram_sched ? (const void*)fused_kernel<64, true>
+                          : half     ? (const void*)fused_kernel<64, false>
+                                     : (const void*)fused_kernel<128, false>;
         e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kFusedSmem);
         if (e != cudaSuccess) return e;
@@ -1550,12 +1911,13 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
             bf16* ob = static_cast<bf16*>(o);
             int c0v = (int)chain_blocks;
             void* args[] = {&tm_q, &tm_k, &tm_v, &tm_o, &qb, &kb, &a, &b, &A_log, &dt_bias, &S0,
-                            &cu_seqlens, &choff, &N, &T, &H_qk, &H_v, &scale, &rec, &ob,
+                            &cu_seqlens, &choff, &N, &T, &H_qk, &H_v, &scale, &rec, &gram, &ob,
                             &S_final, &sref, &status, &flags, &epoch, &c0v};
             ktimer_before(s);
             e = cudaLaunchCooperativeKernel(kfn, dim3(grid), dim3(kFusedThreads), args, kFusedSmem,
                                             s);
-            if (e == cudaSuccess) ktimer_after(s, half ? "fused_half_rows" : "fused");
+            if (e == cudaSuccess)
+                ktimer_after(s, gram_sched ? "fused_half_rows_gram" : half ? "fused_half_rows" : "fused");
             return e;
         }
     }

@@ -40,6 +40,7 @@ EXPORTS = ["gdn_status_string", "gdn_version", "gdn_prefill_workspace_size", "gd
            "gdn_prefill_slots"]
 GDN_IMPL_AUTO, GDN_IMPL_CUDA_CORE, GDN_IMPL_TENSOR_CORE, GDN_IMPL_TENSOR_CORE_SPLIT = 0, 1, 2, 3
 GDN_IMPL_TENSOR_CORE_WHOLE_ROWS = 4
+GDN_IMPL_TENSOR_CORE_GRAM = 5
 
 
 class GDNError(RuntimeError):

@@ -44,11 +44,17 @@ def test_status_strings(lib):
 def test_workspace_size(lib):
     ws = lib.gdn_prefill_workspace_size
     a256 = lambda x: (x + 255) // 256 * 256
-    # d = 128: chunk offsets (N + 1 int32), an 8-byte flag per record, and one
+    # d = 128: chunk offsets (N + 1 int32), an 8-byte flag per record and one
     # 17,664-byte record per (chunk, V head), with at most ceil(T / 64) + N chunks
-    tc = lambda N, recs: a256((N + 1) * 4) + a256(recs * 8) + recs * 17664
-    assert ws(1, 4096, 16, 32, 128, 128) == tc(1, (64 + 1) * 32)
-    assert ws(4, 4 * 16384, 16, 64, 128, 128) == tc(4, (1024 + 4) * 64)
+    tc = lambda N, ch, hv: a256((N + 1) * 4) + a256(ch * hv * 8) + ch * hv * 17664
+    assert ws(1, 4096, 16, 32, 128, 128) == tc(1, 64 + 1, 32)
+    assert ws(4, 4 * 16384, 16, 64, 128, 128) == tc(4, 1024 + 4, 64)
+    # the Gram-matrix schedule adds one 8,192-byte tile per (chunk, QK head)
+    prev = lib.gdn_set_prefill_impl(5)
+    try:
+        assert ws(1, 4096, 16, 32, 128, 128) == tc(1, 64 + 1, 32) + 65 * 16 * 8192
+    finally:
+        lib.gdn_set_prefill_impl(prev)
     # never below the CUDA-core path's need (G and beta, fp32 [T, H_v] each)
     assert ws(1, 3, 1, 1, 128, 128) >= 2 * 256
     assert ws(1, 3, 1, 1, 64, 64) == 2 * 256  # each part rounded up to 256 bytes
@@ -297,8 +303,9 @@ def test_set_prefill_impl(lib):
     assert lib.gdn_set_prefill_impl(2) == 1
     assert lib.gdn_set_prefill_impl(3) == 2
     assert lib.gdn_set_prefill_impl(4) == 3
+    assert lib.gdn_set_prefill_impl(5) == 4
     assert lib.gdn_set_prefill_impl(7) == -1      # invalid: unchanged
-    assert lib.gdn_set_prefill_impl(0) == 4
+    assert lib.gdn_set_prefill_impl(0) == 5
 
 
 def test_kernel_timing_switch(lib):

@@ -176,7 +176,8 @@ def impl_switch():
 
 IMPLS = {"cuda_core": "GDN_IMPL_CUDA_CORE", "tensor_core": "GDN_IMPL_TENSOR_CORE",
          "tensor_core_split": "GDN_IMPL_TENSOR_CORE_SPLIT",
-         "tensor_core_whole_rows": "GDN_IMPL_TENSOR_CORE_WHOLE_ROWS"}
+         "tensor_core_whole_rows": "GDN_IMPL_TENSOR_CORE_WHOLE_ROWS",
+         "tensor_core_gram": "GDN_IMPL_TENSOR_CORE_GRAM"}
 
 
 @pytest.mark.parametrize("impl", list(IMPLS))
@@ -189,10 +190,11 @@ def test_bf16_every_implementation(impl_switch, impl, lengths):
     _check(P, TOL_BF16)
 
 
-def test_tensor_core_stress_gates(impl_switch):
+@pytest.mark.parametrize("impl", ["GDN_IMPL_TENSOR_CORE", "GDN_IMPL_TENSOR_CORE_GRAM"])
+def test_tensor_core_stress_gates(impl_switch, impl):
     """Slow decay, strong writes and extreme gates through the tensor-core path."""
     g = impl_switch
-    g.set_prefill_impl(g.GDN_IMPL_TENSOR_CORE)
+    g.set_prefill_impl(getattr(g, impl))
     P = make_prefill_inputs([500], H_qk=1, H_v=4, d_k=128, d_v=128, state_std=0.1, seed=12)
     P.A_log[0] = -4.0                 # alpha near 0.98: long carry across chunks
     P.b[:, 1] = 4.0                   # beta near 1
@@ -215,6 +217,7 @@ def test_kernel_timing_names_and_durations(impl_switch):
     prev = g.set_kernel_timing(True)
     try:
         for impl, names in ((g.GDN_IMPL_TENSOR_CORE, ["fused_half_rows"]),  # 8 chains
+                            (g.GDN_IMPL_TENSOR_CORE_GRAM, ["fused_half_rows_gram"]),
                             (g.GDN_IMPL_TENSOR_CORE_WHOLE_ROWS, ["fused"]),
                             (g.GDN_IMPL_TENSOR_CORE_SPLIT, ["chunk_offsets", "prep", "chain"]),
                             (g.GDN_IMPL_CUDA_CORE, ["gates", "prefill_simt"])):
@@ -254,6 +257,37 @@ def test_fused_equals_split(impl_switch, wl):
         g.set_kernel_timing(prev)
     for o_, S_ in outs[1:]:
         assert torch.equal(outs[0][0], o_) and torch.equal(outs[0][1], S_)
+
+
+@pytest.mark.parametrize("lengths,H_qk,H_v", [([4096], 4, 8), ([1000, 300, 64, 2000, 1], 2, 4)])
+def test_gram_schedule(impl_switch, lengths, H_qk, H_v):
+    """The cross-chunk Gram-matrix schedule (half-row blocks; S_c K_c^T built from the
+    previous chunk's bf16 state and the key Gram matrix) against the oracle, every output,
+    and against the default schedule: the same mathematics with another bf16 rounding."""
+    g = impl_switch
+    P = make_prefill_inputs(lengths, H_qk=H_qk, H_v=H_v, d_k=128, d_v=128, state_std=0.05,
+                            seed=len(lengths) + 40)
+    prev = g.set_kernel_timing(True)
+    try:
+        g.set_prefill_impl(g.GDN_IMPL_TENSOR_CORE_GRAM)
+        o, Sf = _run(P)
+        assert [n for n, _ in g.last_prefill_kernel_times()] == ["fused_half_rows_gram"]
+        g.set_prefill_impl(g.GDN_IMPL_TENSOR_CORE)
+        o_d, S_d = _run(P)
+    finally:
+        g.set_kernel_timing(prev)
+    o_ref, S_ref = _full_oracle(P)
+    assert rel_err(o, o_ref) <= TOL_BF16 and rel_err(Sf, S_ref) <= TOL_BF16
+    # both schedules sit well inside the tolerance and close to each other
+    assert rel_err(o, o_d.float().cpu().numpy()) <= TOL_BF16 / 2
+    assert rel_err(Sf, S_d.cpu().numpy()) <= TOL_BF16 / 2
+
+
+def test_gram_schedule_35b_layer_full(impl_switch):
+    g = impl_switch
+    g.set_prefill_impl(g.GDN_IMPL_TENSOR_CORE_GRAM)
+    P = make_prefill_inputs(**WORKLOADS["prefill_35b"], seed=0)
+    _check(P, TOL_BF16)
 
 
 def test_many_chains_use_separate_launches(impl_switch):
