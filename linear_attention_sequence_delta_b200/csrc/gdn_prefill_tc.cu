@@ -21,30 +21,30 @@
 // (directly, or as a product of two factors that are both <= 1), so nothing
 // overflows however strong the decay.
 //
-// Three launches:
-//   chunk offsets  first global chunk index of every sequence (and the check of
-//                  cu_seqlens);
-//   prep           everything that does not depend on the state, for all
-//                  chunks at once: a persistent grid walks (chunk, QK head)
-//                  units; each forms K K^T / Q K^T once, then for each V head
-//                  sharing that QK head the gates, A, P and T = (I + A)^-1 in
-//                  fp32 (8x8 diagonal blocks by forward substitution in
-//                  registers, lanes exchanging finished rows by shuffles, then
-//                  three doubling steps 8 -> 16 -> 32 -> 64, each block pair
-//                  merged as T_10 = -D_1 A_10 D_0). T, P and the per-token
-//                  factors go to the workspace as images of the chain's shared
-//                  memory tiles;
-//   chain          one block per (sequence, V head) walks its chunks in order
-//                  with the 128x128 fp32 state resident in tensor memory (lane
-//                  i = value row i). A loader warp fills a 3-deep ring with the
-//                  raw K/Q/V rows (cp.async) and the prepared T/P/factors (one
-//                  bulk copy); eight warps (two per lane quarter, each owning
-//                  half the columns of its rows) run the state-dependent steps,
-//                  the state's decay rescale overlapping the first MMA. Every
-//                  A operand (the bf16 state, Y^T, Vn^T and the decay-scaled
-//                  Vn^T) is written to tensor memory by the threads owning
-//                  those rows, and V^T itself is produced in tensor memory by
-//                  one MMA against an identity tile.
+// Two stages:
+//   prep           everything that does not depend on the state, for all chunks:
+//                  workers walk (chunk, QK head) units; each forms K K^T / Q K^T once
+//                  (one MMA into TMEM), then for each V head sharing that QK head the
+//                  gates, A, P and T = (I + A)^-1 in fp32 (8x8 diagonal blocks by
+//                  forward substitution in registers, then doubling steps 8 -> 16 ->
+//                  32 -> 64 with T_10 = -D_1 A_10 D_0, the last two on tf32 tensor
+//                  cores). T diag(beta), P and the per-token factors go to the
+//                  workspace as a record per (chunk, V head): images of the chain's
+//                  shared-memory tiles.
+//   chain          one (sequence, V head) walks its chunks in order. The fp32 state
+//                  lives in the registers of eight state warps; every A operand they
+//                  produce (the bf16 state, Z^T, Vn^T and its decay-scaled copy) goes to
+//                  TMEM, one warp issues the MMAs, four warps turn the output
+//                  accumulators into o (TMA stores) and refill a 3-deep ring of K, Q,
+//                  V tiles (TMA) and records (bulk copies).
+// Launches: with few chains (at most half as many as SMs) both stages run in one
+// cooperative launch (fused_kernel), chain blocks consuming records as prep blocks
+// publish them (per-record flags holding the call's number); with at most a quarter
+// as many chains as SMs each chain is split over two blocks of 64 value rows (M = 64
+// MMAs). Otherwise three launches: chunk offsets, prep_kernel, chain_kernel. An
+// opt-in schedule (kGram) forms S_c K_c^T from the previous chunk's state and the
+// cross-chunk key Gram matrix K_{c-1} K_c^T that prep provides, taking the state
+// update off the path from one chunk to the next.
 //
 // Every wait is bounded; on expiry a block records GDN_ERR_TIMEOUT in the status
 // word, leaves its loops, drains its copies, frees its tensor memory and exits.
