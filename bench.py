@@ -79,10 +79,10 @@ def _kernel_traffic():
         vals = {}
         with open(KERNEL_PROFILE) as f:
             for line in f:
-                if ":" in line and line.strip().startswith(("traffic_bytes_per_launch",
-                                                            "kernel_source_sha1")):
-                    k_, v_ = line.split(":", 1)
-                    vals[k_.strip().lstrip("-* ")] = v_.strip().strip("`")
+                t = line.strip().lstrip("-* ")  # list markers before the key are allowed
+                if ":" in t and t.startswith(("traffic_bytes_per_launch", "kernel_source_sha1")):
+                    k_, v_ = t.split(":", 1)
+                    vals[k_.strip()] = v_.strip().strip("`")
         return int(vals["traffic_bytes_per_launch"]), vals.get("kernel_source_sha1")
     except Exception:
         return None, None

@@ -272,8 +272,10 @@ __global__ void __launch_bounds__(256) conv_state_kernel(const IO* __restrict__ 
 // padding entry (y zeroed, no cache touched), a slot >= num_slots is reported. A thread
 // takes one channel vector of kDecSeqs sequences (the taps loaded once) and loads all
 // their inputs before using any.
+constexpr int kDecThreads = 64;  // small blocks: 17.7 -> 16.7 us on 256 x 12288 (vs 128)
+
 template <typename IO, int K>
-__global__ void __launch_bounds__(128) conv_decode_kernel(const IO* __restrict__ x,
+__global__ void __launch_bounds__(kDecThreads) conv_decode_kernel(const IO* __restrict__ x,
                                                           const float* __restrict__ w,
                                                           const float* __restrict__ bias,
                                                           IO* state,
@@ -407,7 +409,7 @@ template <typename IO, int K>
 cudaError_t conv_decode_launch(const void* x, const float* w, const float* bias, void* state,
                                const int32_t* slots, int num_slots, int N, int C, void* y,
                                int* status, cudaStream_t s) {
-    const int threads = 128;
+    const int threads = kDecThreads;
     const int64_t groups = (N + kDecSeqs - 1) / kDecSeqs;
     conv_decode_kernel<IO, K><<<blocks_for(groups * (C / kVec), threads), threads, 0, s>>>(
         static_cast<const IO*>(x), w, bias, static_cast<IO*>(state), slots, num_slots, N, C,

@@ -64,3 +64,14 @@ def test_single_rank_helpers_need_no_process_group():
     import bench
     assert bench._max_over_ranks(2.5, 1, "cpu") == 2.5
     bench._barrier(1)
+
+
+def test_kernel_profile_lines_parse():
+    """bench.py reads the dominant kernel's DRAM traffic and the source hash it was taken on
+    from the committed ncu summary (list-marked lines)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    traffic, sha = bench._kernel_traffic()
+    assert isinstance(traffic, int) and 10**7 < traffic < 10**9
+    assert isinstance(sha, str) and len(sha) == 40 and all(c in "0123456789abcdef" for c in sha)
+    assert len(bench._kernel_source_sha1()) == 40
