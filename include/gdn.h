@@ -54,7 +54,7 @@ extern "C" {
 typedef enum {
     GDN_OK = 0,
     GDN_ERR_INVALID_ARG = 1, /* null / misaligned pointer, bad size or count       */
-    GDN_ERR_UNSUPPORTED = 2, /* a shape or type this build does not implement     */
+    GDN_ERR_UNSUPPORTED = 2, /* a shape or type the library does not implement    */
     GDN_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required        */
     GDN_ERR_CUDA = 4,        /* a CUDA runtime call failed (launch, attribute)    */
     GDN_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out                */
