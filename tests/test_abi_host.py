@@ -113,6 +113,20 @@ def test_prefill_rejects(lib, over, code):
     assert _call_prefill(lib, **over) == code
 
 
+def test_gram_schedule_needs_its_workspace(lib):
+    """A workspace sized while another schedule was selected is too small for the
+    Gram-matrix schedule (its tiles are counted only while it is selected): the call is
+    rejected on the host before anything is launched."""
+    dims = dict(N=1, T=4096, H_qk=16, H_v=32, d_k=128, d_v=128)
+    size_default = lib.gdn_prefill_workspace_size(1, 4096, 16, 32, 128, 128)
+    prev = lib.gdn_set_prefill_impl(5)
+    try:
+        assert lib.gdn_prefill_workspace_size(1, 4096, 16, 32, 128, 128) > size_default
+        assert _call_prefill(lib, ws_bytes=size_default, **dims) == 3
+    finally:
+        lib.gdn_set_prefill_impl(prev)
+
+
 def test_prefill_empty_batch_is_noop(lib):
     # N = 0, T = 0: nothing to do, no CUDA call, success
     assert _call_prefill(lib, N=0, T=0, q=None, k=None, v=None, o=None, ws=None,
