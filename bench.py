@@ -236,6 +236,57 @@ def run_decode_variants(rank, dev, flush, stream, hbm, peak_src, iters):
     return out, 3 * iters
 
 
+def run_other_prefill(rank, dev, flush, stream, hbm, tc_burst, peak_src, iters):
+    """gdn_prefill on the two workloads with many (sequence, V head) chains: the 397B-A17B
+    long prefill (4 x 16384 tokens, 16 QK / 64 V heads) and the packed batch of 64
+    sequences of random length (32 V heads, initial states in, final states out). Each
+    call's kernels are timed by the library's kernel timing; the call itself with CUDA
+    events around it, the L2 flushed before each call (the inputs exceed L2 as well)."""
+    from linear_attention_sequence_delta_b200 import gdn
+    from linear_attention_sequence_delta_b200.inputs import WORKLOADS, make_prefill_inputs
+    out, launches = {}, 0
+    for name in ("prefill_397b_long", "varlen_64"):
+        P = make_prefill_inputs(**WORKLOADS[name], seed=rank, device=dev)
+        T, H_qk, d = P.q.shape
+        H_v, N = P.v.shape[1], P.num_seqs
+        o = torch.empty((T, H_v, d), device=dev, dtype=P.q.dtype)
+        Sf = torch.empty((N, H_v, d, d), device=dev, dtype=torch.float32)
+        work = torch.empty((max(gdn.workspace_size(N, T, H_qk, H_v, d, d), 1),), device=dev,
+                           dtype=torch.uint8)
+        call = lambda: gdn.gdn_prefill(P.q, P.k, P.v, P.a, P.b, P.A_log, P.dt_bias,
+                                       P.cu_seqlens, P.initial_state, out=o, final_state=Sf,
+                                       workspace=work)
+        ms = _time_op(call, iters, flush, stream)
+        prev = gdn.set_kernel_timing(True)
+        kms = {}
+        for i in range(iters):
+            flush.fill_(i & 0xFF)
+            call()
+            for kn, t_ in gdn.last_prefill_kernel_times():
+                kms.setdefault(kn, []).append(t_)
+        gdn.set_kernel_timing(prev)
+        torch.cuda.synchronize()
+        launches += 2 * iters * len(kms)  # the event-timed calls and the kernel-timed ones
+        byts = prefill_bytes(T, N, H_qk, H_v, d, 2, with_initial=P.initial_state is not None)
+        flops = prefill_flops(T, N, H_qk, H_v, d)
+        t_roof = max(byts / (hbm * 1e9), flops / (tc_burst * 1e12))
+        out[name] = {
+            "workload": f"N={N}, T_total={T}, H_qk={H_qk}, H_v={H_v}, d={d}, bf16 q/k/v/o"
+                        + (", initial states in" if P.initial_state is not None else "")
+                        + ", final states out",
+            "ms_per_call": ms, "tokens_per_s": T / (ms / 1e3),
+            "kernels_ms": {kn: sum(v_) / len(v_) for kn, v_ in kms.items()},
+            "algorithmic_bytes": byts, "algorithmic_flops": flops,
+            "achieved_gbs": byts / (ms / 1e3) / 1e9,
+            "frac_hbm": byts / (ms / 1e3) / 1e9 / hbm,
+            "frac_tensor": flops / (ms / 1e3) / 1e12 / tc_burst,
+            "frac_of_slower_roof": t_roof / (ms / 1e3), "peak_source": peak_src}
+        del P, o, Sf, work
+    out["l2"] = "flushed (512 MiB write) before every timed call"
+    out["iters"] = iters
+    return out, launches
+
+
 class Clocks:
     """nvidia-smi sampled every 200 ms while the timed region runs."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -394,6 +445,10 @@ def run_ours(args):
         if not args.no_decode:
             dvar, dvar_launches = run_decode_variants(rank, dev, flush, stream, hbm, peak_src,
                                                       args.mixer_iters)
+        other, other_launches = None, 0
+        if not args.no_other_prefill:
+            other, other_launches = run_other_prefill(rank, dev, flush, stream, hbm, tc_burst,
+                                                      peak_src, args.other_iters)
     kern_ms = [a.elapsed_time(b) for a, b in ev]
     ms = _max_over_ranks(sum(kern_ms) / len(kern_ms), ws, dev)
     tok_s = ws * T / (ms / 1e3)
@@ -437,11 +492,12 @@ def run_ours(args):
         "e2e": e2e,
         "gpu_launches": sum(len(v_) for v_ in kernel_ms.values())
                         + (args.decode_steps if dec else 0) + mixer_launches
-                        + dvar_launches,
+                        + dvar_launches + other_launches,
         "clocks": clocks.summary(),
         "decode": dec,
         "decode_slots": dvar,
         "mixer": mixer,
+        "prefill_many_chains": other,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(P)
@@ -597,6 +653,9 @@ def main():
     ap.add_argument("--no-mixer", action="store_true",
                     help="skip the conv1d / gated-norm measurements")
     ap.add_argument("--mixer-iters", type=int, default=20)
+    ap.add_argument("--no-other-prefill", action="store_true",
+                    help="skip the 397B-A17B long and varlen_64 prefill measurements")
+    ap.add_argument("--other-iters", type=int, default=5)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
