@@ -9,7 +9,9 @@ d=128, bf16 q/k/v/o, fp32 gates and state, zero initial state, final state
 written. `value` is prefill tokens/s over the whole job (all ranks; each rank
 runs its own copy of the workload, so scaling is weak). The same line carries
 the decode measurement (256 sequences x 64 V heads, 1000 consecutive in-place
-steps of gdn_decode_step) under "decode".
+steps of gdn_decode_step) under "decode", and the prefill of the workloads with
+many (sequence, V head) chains (397B-A17B long prefill, 64 packed sequences of
+random length) under "prefill_many_chains".
 
 Timing: W untimed warm-up steps; then K steps, each preceded by an L2 flush
 (a 512 MiB write, outside the timed window) and bracketed by CUDA events on
