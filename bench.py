@@ -238,7 +238,8 @@ def run_decode_variants(rank, dev, flush, stream, hbm, peak_src, iters):
     return out, 3 * iters
 
 
-def run_other_prefill(rank, dev, flush, stream, hbm, tc_burst, peak_src, iters):
+def run_other_prefill(rank, dev, flush, stream, hbm, tc_burst, peak_src, iters,
+                      names=("prefill_397b_long", "varlen_64"), num_seqs=None):
     """gdn_prefill on the two workloads with many (sequence, V head) chains: the 397B-A17B
     long prefill (4 x 16384 tokens, 16 QK / 64 V heads) and the packed batch of 64
     sequences of random length (32 V heads, initial states in, final states out). Each
@@ -247,8 +248,9 @@ def run_other_prefill(rank, dev, flush, stream, hbm, tc_burst, peak_src, iters):
     from linear_attention_sequence_delta_b200 import gdn
     from linear_attention_sequence_delta_b200.inputs import WORKLOADS, make_prefill_inputs
     out, launches = {}, 0
-    for name in ("prefill_397b_long", "varlen_64"):
-        P = make_prefill_inputs(**WORKLOADS[name], seed=rank, device=dev)
+    for name in names:
+        wl = dict(WORKLOADS[name], **({"num_seqs": num_seqs} if num_seqs else {}))
+        P = make_prefill_inputs(**wl, seed=rank, device=dev)
         T, H_qk, d = P.q.shape
         H_v, N = P.v.shape[1], P.num_seqs
         o = torch.empty((T, H_v, d), device=dev, dtype=P.q.dtype)
@@ -450,7 +452,9 @@ def run_ours(args):
         other, other_launches = None, 0
         if not args.no_other_prefill:
             other, other_launches = run_other_prefill(rank, dev, flush, stream, hbm, tc_burst,
-                                                      peak_src, args.other_iters)
+                                                      peak_src, args.other_iters,
+                                                      args.many_chains.split(","),
+                                                      args.many_chains_seqs)
     kern_ms = [a.elapsed_time(b) for a, b in ev]
     ms = _max_over_ranks(sum(kern_ms) / len(kern_ms), ws, dev)
     tok_s = ws * T / (ms / 1e3)
@@ -658,6 +662,11 @@ def main():
     ap.add_argument("--no-other-prefill", action="store_true",
                     help="skip the 397B-A17B long and varlen_64 prefill measurements")
     ap.add_argument("--other-iters", type=int, default=5)
+    ap.add_argument("--many-chains", default="prefill_397b_long,varlen_64",
+                    help="comma-separated workloads of the many-chain prefill block")
+    ap.add_argument("--many-chains-seqs", type=int, default=None,
+                    help="sequences per many-chain workload (default: the workload's own; "
+                         "smaller values only for profiling captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
