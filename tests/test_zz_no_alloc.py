@@ -6,8 +6,9 @@ input and output buffers), so they cannot hand gdn_prefill a workspace. This
 entry point keeps that scratch in a fixed array inside the library. The test
 calls it through the C ABI, twice in a row on different inputs (the array keeps
 the previous call's contents), and checks each result against gdn_prefill's
-within the parity tolerance. It also checks that a call larger than the built-in
-scratch is refused before anything is launched.
+within the parity tolerance. It also checks, on the host, that a call larger than
+the built-in scratch and calls with bad arguments are refused before anything is
+launched.
 
 This file is named so that pytest collects it last.
 """
@@ -55,6 +56,30 @@ def test_refuses_more_than_the_builtin_scratch():
     st = _fn()(v(F), v(F), v(F), 0, v(F), v(F), v(F), v(F), None, v(F), 1, T, 16, H_v, 128, 128,
                1.0, v(F), None, None)
     assert st == 3  # GDN_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(io=7), 1),                       # not a dtype
+    (dict(d=96), 2),                       # head size the library does not implement
+    (dict(H_v=24), 1),                     # H_v not a multiple of H_qk
+    (dict(N=-1), 1),
+    (dict(N=0), 1),                        # tokens but no sequence
+    (dict(scale=float("inf")), 1),
+    (dict(cu=None), 1),
+    (dict(q=0x7F0000000008), 1),           # not 16-byte aligned
+    (dict(Sf=0x7F0000000004), 1),
+    (dict(N=0, T=0), 0),                   # nothing to do: success, nothing launched
+])
+def test_host_checks(over, code):
+    # Every case is decided on the host before any CUDA call, so no GPU is needed.
+    F = 0x7F0000000000
+    a = dict(io=0, N=1, T=256, H_qk=16, H_v=32, d=128, scale=1.0, cu=F, q=F, Sf=None)
+    a.update(over)
+    v = lambda p: None if p is None else ctypes.c_void_p(p)
+    st = _fn()(v(a["q"]), v(F), v(F), a["io"], v(F), v(F), v(F), v(F), None, v(a["cu"]),
+               a["N"], a["T"], a["H_qk"], a["H_v"], a["d"], a["d"], a["scale"], v(F),
+               v(a["Sf"]), None)
+    assert st == code
 
 
 @pytest.mark.gpu
