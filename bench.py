@@ -2,36 +2,37 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One JSON line on rank 0. A "step" is one gdn_prefill call (the chunk-offsets
-kernel and the fused prep + chunk-chain kernel of the tensor-core path) on the
-35B-A3B GDN layer shape: B=1, T=4096, 16 QK / 32 V heads,
-d=128, bf16 q/k/v/o, fp32 gates and state, zero initial state, final state
-written. `value` is prefill tokens/s over the whole job (all ranks; each rank
-runs its own copy of the workload, so scaling is weak). The same line carries
-the decode measurement (256 sequences x 64 V heads, 1000 consecutive in-place
-steps of gdn_decode_step) under "decode", and the prefill of the workloads with
-many (sequence, V head) chains (397B-A17B long prefill, 64 packed sequences of
-random length) under "prefill_many_chains".
+One JSON line on rank 0. A "step" is one gdn_prefill call on the largest single-GPU
+workload, the packed varlen batch: 64 sequences with lengths ~ U[128, 8192] (274,156
+tokens with seed 0), 16 QK / 32 V heads, d=128, bf16 q/k/v/o, fp32 gates, initial
+states ~ N(0, 0.02^2) in, final states out. `value` is prefill tokens/s over the
+whole job (all ranks; each rank runs its own copy of the workload, so scaling is
+weak). The same line carries the other prefill workloads (the 35B-A3B layer, B=1,
+T=4096, 32 V heads; the 397B-A17B long prefill, 4 x 16384 tokens, 64 V heads) under
+"prefill_other_configs", the decode measurement (256 sequences x 64 V heads, 1000
+consecutive in-place steps of gdn_decode_step) under "decode", the decode variants
+and the steps around the delta rule.
 
-Timing: W untimed warm-up steps; then K steps, each preceded by an L2 flush
-(a 512 MiB write, outside the timed window) and bracketed by CUDA events on
-the launching stream; a barrier and a device synchronise on both sides of the
-timed region; the max over ranks. `e2e` repeats the prefill through the public
-Python API from pinned host buffers, host<->device copies inside the timing.
-The CPU baseline is the fp64 oracle (test infrastructure) timed on this host.
+Timing: W untimed warm-up steps; then K steps, each preceded by an L2 flush (a 512
+MiB write, outside the timed window; the inputs, 4.7 GB, exceed L2 as well) and
+bracketed by CUDA events on the launching stream; a barrier and a device synchronise
+on both sides of the timed region; the max over ranks. `e2e` repeats the headline
+prefill through the public Python API from pinned host buffers, host<->device copies
+inside the timing. The CPU baseline is the fp64 oracle (test infrastructure) timed on
+this host on a bounded sample of the same workload.
 
-`roofline` is that of the dominant kernel (the fused prep + chain kernel): its
-duration comes from the library's kernel timing (CUDA events recorded around
-each launch on the launching stream, every timed step), its algorithmic bytes
-are those of the whole path (q, k, v, a, b read, o and the final state
-written), all of which it moves; `traffic` is the DRAM bytes per launch from
-the committed ncu summary of that kernel, null when the summary was taken on
-another build of it. `roofline.step` gives the whole call against
-the slower of the HBM and tensor roofs.
+`roofline` is that of the dominant kernel of the step (the longest of the call's
+launches): its duration comes from a kernel timer (CUDA events recorded around each
+launch on the launching stream, every timed step), its algorithmic bytes are the
+ones that kernel must move (see kernel_bytes), `traffic` is the DRAM bytes per launch
+from the committed ncu record (profiles/roofline_traffic.json), null when that record
+was taken on another build of the kernel. `roofline.step` gives the whole call
+against the slower of the HBM and tensor roofs.
 """
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -44,8 +45,15 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-WORKLOAD = "prefill_35b"
+WORKLOAD = "varlen_64"
+WORKLOAD_DESC = ("varlen_64: 64 sequences, lengths ~ U[128, 8192] packed via cu_seqlens, "
+                 "H_qk=16, H_v=32, d=128, bf16 q/k/v/o, fp32 gates, initial states "
+                 "~N(0, 0.02^2) in, final states out")
+OTHER_PREFILL = ("prefill_35b", "prefill_397b_long")
 METRIC = "GDN prefill tokens/s and decode steps/s on 1 B200, % of roofline"
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "roofline_traffic.json")
+TC_SOURCE = os.path.join(ROOT, "linear_attention_sequence_delta_b200", "csrc",
+                         "gdn_prefill_tc.cu")
 
 
 def _peaks():
@@ -66,43 +74,44 @@ def prefill_bytes(T, N, H_qk, H_v, d, io_bytes, with_initial):
     return b
 
 
-def chain_bytes(T, N, H_qk, H_v, d, io_bytes, with_initial):
-    """Algorithmic HBM bytes of the chain kernel: q, k, v read, o written, the
-    final state written (and the initial state read if given)."""
-    return prefill_bytes(T, N, H_qk, H_v, d, io_bytes, with_initial) - 2 * T * H_v * 4
-
-
-KERNEL_PROFILE = os.path.join(ROOT, "profiles", "fused_kernel_prefill35b.md")
-
-
-def _kernel_traffic():
-    """(DRAM bytes per launch, kernel build id) from the ncu summary of the dominant kernel."""
-    try:
-        vals = {}
-        with open(KERNEL_PROFILE) as f:
-            for line in f:
-                t = line.strip().lstrip("-* ")  # list markers before the key are allowed
-                if ":" in t and t.startswith(("traffic_bytes_per_launch", "kernel_source_sha1")):
-                    k_, v_ = t.split(":", 1)
-                    vals[k_.strip()] = v_.strip().strip("`")
-        return int(vals["traffic_bytes_per_launch"]), vals.get("kernel_source_sha1")
-    except Exception:
-        return None, None
-
-
-def _kernel_source_sha1():
-    import hashlib
-    src = os.path.join(ROOT, "linear_attention_sequence_delta_b200", "csrc", "gdn_prefill_tc.cu")
-    with open(src, "rb") as f:
-        return hashlib.sha1(f.read()).hexdigest()
+def kernel_bytes(kernel, T, N, H_qk, H_v, d, io_bytes, with_initial):
+    """Algorithmic HBM bytes of one launch of a kernel of the tensor-core prefill:
+    the one-launch kernels move the whole call's; the chain reads q, k, v, writes o
+    and the final states (and reads the initial ones); the prep reads q, k, a and b
+    (its records are intermediates, not algorithmic bytes)."""
+    if kernel.startswith("fused"):
+        return prefill_bytes(T, N, H_qk, H_v, d, io_bytes, with_initial)
+    if kernel == "chain":
+        return prefill_bytes(T, N, H_qk, H_v, d, io_bytes, with_initial) - 2 * T * H_v * 4
+    if kernel == "prep":
+        return 2 * T * H_qk * d * io_bytes + 2 * T * H_v * 4
+    return 4 * (N + 1)
 
 
 def prefill_flops(T, N, H_qk, H_v, d, C=64):
-    """Algorithmic tensor flops: the in-chunk products QK^T and KK^T per QK head,
-    and per V head the solve-applied T Y (C^2 d), the intra-chunk P Vnew (C^2 d),
-    and the state products K S^T, Q S^T and the state update (3 x 2 C d^2 per
-    chunk)."""
-    return T * (H_qk * 4 * C * d + H_v * (4 * C * d + 6 * d * d))
+    """Algorithmic tensor flops of the chunk form per token: the in-chunk products
+    K K^T and Q K^T once per QK head (4 C d), and per V head the solve-applied value
+    update (2 C d), the intra-chunk P V_new and S0 [K; Q]^T products (4 C d) and the
+    state's three chunk products (6 d^2)."""
+    return T * (H_qk * 4 * C * d + H_v * (2 * C * d + 4 * C * d + 6 * d * d))
+
+
+def _source_sha1(path=TC_SOURCE):
+    with open(path, "rb") as f:
+        return hashlib.sha1(f.read()).hexdigest()
+
+
+def kernel_traffic(kernel, workload):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu record,
+    or None (no record, or one taken on another build of the kernel source)."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)[f"{kernel}@{workload}"]
+        if rec["kernel_source_sha1"] != _source_sha1():
+            return None
+        return int(rec["traffic_bytes_per_launch"])
+    except Exception:
+        return None
 
 
 def decode_bytes(N, H_qk, H_v, d, io_bytes):
@@ -239,16 +248,19 @@ def run_decode_variants(rank, dev, flush, stream, hbm, peak_src, iters):
 
 
 def run_other_prefill(rank, dev, flush, stream, hbm, tc_burst, peak_src, iters,
-                      names=("prefill_397b_long", "varlen_64"), num_seqs=None):
-    """gdn_prefill on the two workloads with many (sequence, V head) chains: the 397B-A17B
-    long prefill (4 x 16384 tokens, 16 QK / 64 V heads) and the packed batch of 64
-    sequences of random length (32 V heads, initial states in, final states out). Each
-    call's kernels are timed by the library's kernel timing; the call itself with CUDA
-    events around it, the L2 flushed before each call (the inputs exceed L2 as well)."""
+                      names=OTHER_PREFILL, num_seqs=None):
+    """gdn_prefill on the other prefill workloads: the 35B-A3B layer (B=1, T=4096,
+    16 QK / 32 V heads; 32 chains, one overlapped launch) and the 397B-A17B long
+    prefill (4 x 16384 tokens, 16 QK / 64 V heads; 256 chains, separate launches).
+    Each call's kernels are timed by a kernel timer; the call itself with CUDA events
+    around it, the L2 flushed before each call."""
     from linear_attention_sequence_delta_b200 import gdn
     from linear_attention_sequence_delta_b200.inputs import WORKLOADS, make_prefill_inputs
     out, launches = {}, 0
+    timer = gdn.Timer()
     for name in names:
+        if not name:
+            continue
         wl = dict(WORKLOADS[name], **({"num_seqs": num_seqs} if num_seqs else {}))
         P = make_prefill_inputs(**wl, seed=rank, device=dev)
         T, H_qk, d = P.q.shape
@@ -257,35 +269,43 @@ def run_other_prefill(rank, dev, flush, stream, hbm, tc_burst, peak_src, iters,
         Sf = torch.empty((N, H_v, d, d), device=dev, dtype=torch.float32)
         work = torch.empty((max(gdn.workspace_size(N, T, H_qk, H_v, d, d), 1),), device=dev,
                            dtype=torch.uint8)
-        call = lambda: gdn.gdn_prefill(P.q, P.k, P.v, P.a, P.b, P.A_log, P.dt_bias,
-                                       P.cu_seqlens, P.initial_state, out=o, final_state=Sf,
-                                       workspace=work)
+        call = lambda tm=None: gdn.gdn_prefill(P.q, P.k, P.v, P.a, P.b, P.A_log, P.dt_bias,
+                                               P.cu_seqlens, P.initial_state, out=o,
+                                               final_state=Sf, workspace=work, timer=tm)
         ms = _time_op(call, iters, flush, stream)
-        prev = gdn.set_kernel_timing(True)
         kms = {}
         for i in range(iters):
             flush.fill_(i & 0xFF)
-            call()
-            for kn, t_ in gdn.last_prefill_kernel_times():
+            call(timer)
+            for kn, t_ in timer.times():
                 kms.setdefault(kn, []).append(t_)
-        gdn.set_kernel_timing(prev)
         torch.cuda.synchronize()
-        launches += 2 * iters * len(kms)  # the event-timed calls and the kernel-timed ones
-        byts = prefill_bytes(T, N, H_qk, H_v, d, 2, with_initial=P.initial_state is not None)
+        launches += (iters + 3) * len(kms) + iters * len(kms)
+        with_init = P.initial_state is not None
+        byts = prefill_bytes(T, N, H_qk, H_v, d, 2, with_initial=with_init)
         flops = prefill_flops(T, N, H_qk, H_v, d)
         t_roof = max(byts / (hbm * 1e9), flops / (tc_burst * 1e12))
+        mean_k = {kn: sum(v_) / len(v_) for kn, v_ in kms.items()}
+        dom = max(mean_k, key=mean_k.get)
+        dom_b = kernel_bytes(dom, T, N, H_qk, H_v, d, 2, with_init)
         out[name] = {
             "workload": f"N={N}, T_total={T}, H_qk={H_qk}, H_v={H_v}, d={d}, bf16 q/k/v/o"
-                        + (", initial states in" if P.initial_state is not None else "")
+                        + (", initial states in" if with_init else "")
                         + ", final states out",
             "ms_per_call": ms, "tokens_per_s": T / (ms / 1e3),
-            "kernels_ms": {kn: sum(v_) / len(v_) for kn, v_ in kms.items()},
+            "kernels_ms": mean_k,
             "algorithmic_bytes": byts, "algorithmic_flops": flops,
             "achieved_gbs": byts / (ms / 1e3) / 1e9,
             "frac_hbm": byts / (ms / 1e3) / 1e9 / hbm,
             "frac_tensor": flops / (ms / 1e3) / 1e12 / tc_burst,
-            "frac_of_slower_roof": t_roof / (ms / 1e3), "peak_source": peak_src}
+            "frac_of_slower_roof": t_roof / (ms / 1e3),
+            "dominant_kernel": {"kernel": dom, "kernel_ms": mean_k[dom],
+                                "algorithmic_bytes": dom_b,
+                                "frac_hbm": dom_b / (mean_k[dom] / 1e3) / 1e9 / hbm,
+                                "traffic": kernel_traffic(dom, name)},
+            "peak_source": peak_src}
         del P, o, Sf, work
+    timer.close()
     out["l2"] = "flushed (512 MiB write) before every timed call"
     out["iters"] = iters
     return out, launches
@@ -371,7 +391,7 @@ def run_ours(args):
                                 device_id=dev)
     gdn.load_library()
     hbm, tc_burst, tc_sust, peak_src = _peaks()
-    W = WORKLOADS[WORKLOAD]
+    W = dict(WORKLOADS[WORKLOAD], **({"num_seqs": args.seqs} if args.seqs else {}))
     P = make_prefill_inputs(**W, seed=rank, device=dev)
     T, H_qk, d = P.q.shape
     H_v = P.v.shape[1]
@@ -382,10 +402,11 @@ def run_ours(args):
     work = torch.empty((max(wsz, 1),), device=dev, dtype=torch.uint8)
     flush = torch.empty((512 << 20,), device=dev, dtype=torch.uint8)
     stream = torch.cuda.current_stream(dev)
+    timer = gdn.Timer()
 
-    def step():
-        gdn.gdn_prefill(P.q, P.k, P.v, P.a, P.b, P.A_log, P.dt_bias, P.cu_seqlens, None,
-                        out=o, final_state=Sf, workspace=work)
+    def step(tm=None):
+        gdn.gdn_prefill(P.q, P.k, P.v, P.a, P.b, P.A_log, P.dt_bias, P.cu_seqlens,
+                        P.initial_state, out=o, final_state=Sf, workspace=work, timer=tm)
 
     for _ in range(args.warmup):
         step()
@@ -394,18 +415,16 @@ def run_ours(args):
           for _ in range(args.steps)]
     clocks = Clocks(local)
     kernel_ms = {}  # kernel name -> [ms per timed step]
-    prev_timing = gdn.set_kernel_timing(True)
     _barrier(ws)
     torch.cuda.synchronize()
     with clocks:
         for i in range(args.steps):
             flush.fill_(i & 0xFF)  # L2 flush, outside the events
             ev[i][0].record(stream)
-            step()
+            step(timer)
             ev[i][1].record(stream)
-            for name, kms in gdn.last_prefill_kernel_times():  # waits for this step only
+            for name, kms in timer.times():  # waits for this step only
                 kernel_ms.setdefault(name, []).append(kms)
-        gdn.set_kernel_timing(prev_timing)
         torch.cuda.synchronize()
         _barrier(ws)
         # ---- decode: 1000 consecutive steps on the 397B-A17B GDN shape ----
@@ -453,23 +472,20 @@ def run_ours(args):
         if not args.no_other_prefill:
             other, other_launches = run_other_prefill(rank, dev, flush, stream, hbm, tc_burst,
                                                       peak_src, args.other_iters,
-                                                      args.many_chains.split(","),
-                                                      args.many_chains_seqs)
+                                                      args.other_prefill.split(","),
+                                                      args.other_prefill_seqs)
     kern_ms = [a.elapsed_time(b) for a, b in ev]
     ms = _max_over_ranks(sum(kern_ms) / len(kern_ms), ws, dev)
     tok_s = ws * T / (ms / 1e3)
-    byts = prefill_bytes(T, N, H_qk, H_v, d, 2, with_initial=False)
+    with_init = P.initial_state is not None
+    byts = prefill_bytes(T, N, H_qk, H_v, d, 2, with_initial=with_init)
     flops = prefill_flops(T, N, H_qk, H_v, d)
     achieved = byts / (ms / 1e3) / 1e9
     t_roof = max(byts / (hbm * 1e9), flops / (tc_burst * 1e12))
     mean_k = {n_: _max_over_ranks(sum(v_) / len(v_), ws, dev) for n_, v_ in kernel_ms.items()}
     dom = max(mean_k, key=mean_k.get)
     dom_ms = mean_k[dom]
-    dom_bytes = (chain_bytes(T, N, H_qk, H_v, d, 2, with_initial=False) if dom == "chain"
-                 else byts)
-    traffic, traffic_src = _kernel_traffic()
-    if not dom.startswith("fused") or traffic_src != _kernel_source_sha1():
-        traffic = None  # the counters were taken on another build of the kernel
+    dom_bytes = kernel_bytes(dom, T, N, H_qk, H_v, d, 2, with_init)
 
     e2e = None
     if not args.no_e2e:
@@ -480,15 +496,14 @@ def run_ours(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": "prefill_35b: B=1, T=4096, H_qk=16, H_v=32, d=128, bf16 q/k/v/o, "
-                               "fp32 gates/state, zero initial state, final state written",
-                   "global_batch": ws, "seq_len": T, "parallelism": f"replicas x{ws}",
-                   "l2": "flushed (512 MiB write) before every timed step"},
+        "config": {"workload": WORKLOAD_DESC + f" ({N} sequences, {T} tokens per rank)",
+                   "global_batch": ws * N, "seq_len": T, "parallelism": f"replicas x{ws}",
+                   "l2": "flushed (512 MiB write) before every timed step; inputs exceed L2"},
         "roofline": {"bound": "hbm", "achieved": dom_bytes / (dom_ms / 1e3) / 1e9, "peak": hbm,
                      "unit": "GB/s", "frac": dom_bytes / (dom_ms / 1e3) / 1e9 / hbm,
-                     "traffic": traffic, "kernel": dom, "algorithmic_bytes": dom_bytes,
-                     "kernel_ms": dom_ms, "peak_source": peak_src,
-                     "kernels_ms": mean_k,
+                     "traffic": kernel_traffic(dom, WORKLOAD), "kernel": dom,
+                     "algorithmic_bytes": dom_bytes, "kernel_ms": dom_ms,
+                     "peak_source": peak_src, "kernels_ms": mean_k,
                      "step": {"algorithmic_bytes": byts, "achieved_gbs": achieved,
                               "frac_hbm": achieved / hbm, "algorithmic_flops": flops,
                               "achieved_tflops": flops / (ms / 1e3) / 1e12,
@@ -496,17 +511,17 @@ def run_ours(args):
                               "frac_tensor": flops / (ms / 1e3) / 1e12 / tc_burst,
                               "frac_of_slower_roof": t_roof / (ms / 1e3)}},
         "e2e": e2e,
-        "gpu_launches": sum(len(v_) for v_ in kernel_ms.values())
-                        + (args.decode_steps if dec else 0) + mixer_launches
-                        + dvar_launches + other_launches,
+        "gpu_launches": sum(len(v_) for v_ in kernel_ms.values()),
+        "gpu_launches_other_blocks": (args.decode_steps if dec else 0) + mixer_launches
+                                     + dvar_launches + other_launches,
         "clocks": clocks.summary(),
+        "prefill_other_configs": other,
         "decode": dec,
         "decode_slots": dvar,
         "mixer": mixer,
-        "prefill_many_chains": other,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(P)
+        line["cpu_baseline"] = cpu_baseline()
     if ws > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -522,8 +537,9 @@ def _e2e(args, P, o, Sf, ws, dev, stream):
     step's upload overlap the current call, as a serving loop would run them."""
     from linear_attention_sequence_delta_b200 import gdn
     T = P.q.shape[0]
-    names = ("q", "k", "v", "a", "b", "A_log", "dt_bias", "cu_seqlens")
-    host = {k_: getattr(P, k_).cpu().pin_memory() for k_ in names}
+    names = ("q", "k", "v", "a", "b", "A_log", "dt_bias", "cu_seqlens", "initial_state")
+    host = {k_: getattr(P, k_).cpu().pin_memory() for k_ in names
+            if getattr(P, k_) is not None}
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = o.numel() * o.element_size() + Sf.numel() * Sf.element_size()
     up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
@@ -552,7 +568,8 @@ def _e2e(args, P, o, Sf, ws, dev, stream):
         stream.wait_event(b_["out_free"])  # step i-2's outputs have been read back
         dv = b_["dev"]
         gdn.gdn_prefill(dv["q"], dv["k"], dv["v"], dv["a"], dv["b"], dv["A_log"],
-                        dv["dt_bias"], dv["cu_seqlens"], None, out=b_["o"], final_state=b_["S"],
+                        dv["dt_bias"], dv["cu_seqlens"], dv.get("initial_state"), out=b_["o"],
+                        final_state=b_["S"],
                         workspace=work)
         b_["in_free"].record(stream)
         b_["out_ready"].record(stream)
@@ -582,61 +599,77 @@ def _e2e(args, P, o, Sf, ws, dev, stream):
             "copy_streams": 2}
 
 
-def cpu_baseline(P, heads=None, min_seconds=10.0):
-    """The fp64 oracle on this host's cores, on a bounded sample of the workload."""
-    import numpy as np
-
-    import oracle
-    H_v = P.v.shape[1]
-    heads = heads or H_v
-    r = H_v // P.q.shape[1]
-    Q = P.q.cpu()
-    K = P.k.cpu()
-    hs = list(range(heads))
-    js = sorted({h // r for h in hs})
-    args = (Q[:, js[0]:js[-1] + 1], K[:, js[0]:js[-1] + 1], P.v[:, :heads].cpu(),
-            P.a[:, :heads].cpu(), P.b[:, :heads].cpu(), P.A_log[:heads].cpu(),
-            P.dt_bias[:heads].cpu(), P.cu_seqlens.cpu().numpy().astype(np.int64))
-    # repeat the sample until about 10 s of host time have passed (at most 60 passes)
-    reps, t0 = 0, time.perf_counter()
-    while True:
-        oracle.forward(*args)
-        reps += 1
-        dt = time.perf_counter() - t0
-        if dt >= min_seconds or reps >= 60:
+def _reference_sample(seed=0, min_tokens=8192):
+    """A bounded sample of the headline workload for the oracle: the workload's first
+    sequence lengths (drawn on the host with the workload's recipe) until at least
+    min_tokens tokens, all V heads, inputs drawn on the host with the same recipe."""
+    from linear_attention_sequence_delta_b200.inputs import WORKLOADS, make_prefill_inputs
+    W = dict(WORKLOADS[WORKLOAD])
+    g = torch.Generator().manual_seed(seed)
+    lens = [int(x) for x in torch.randint(W["len_lo"], W["len_hi"] + 1, (W["num_seqs"],),
+                                          generator=g)]
+    take = []
+    for n in lens:
+        take.append(n)
+        if sum(take) >= min_tokens:
             break
-    T = P.q.shape[0]
-    return {"value": reps * T * heads / H_v / dt, "unit": "tokens/s",
-            "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{heads} of {H_v} V heads x {T} tokens, {reps} passes ({dt:.1f} s), "
-                      "scaled to all heads"}
+    for k_ in ("lengths", "num_seqs", "len_lo", "len_hi"):
+        W.pop(k_, None)
+    return make_prefill_inputs(take, seed=seed, **W)
+
+
+def _oracle_pass(P):
+    """One oracle pass over a whole packed batch (all sequences, all V heads)."""
+    import oracle
+    t0 = time.perf_counter()
+    oracle.forward(P.q, P.k, P.v, P.a, P.b, P.A_log, P.dt_bias,
+                   P.cu_seqlens.numpy().astype("int64"), P.initial_state)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(min_seconds=10.0):
+    """The fp64 oracle on this host's cores, on a bounded sample of the headline
+    workload (its first sequences, all V heads), repeated for about min_seconds."""
+    import oracle
+    P = _reference_sample()
+    T, H_v = P.q.shape[0], P.v.shape[1]
+    reps, total = 0, 0.0
+    while total < min_seconds and reps < 60:
+        total += _oracle_pass(P)
+        reps += 1
+    return {"value": reps * T / total, "unit": "tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{WORKLOAD}: first {P.num_seqs} sequences ({T} tokens), all {H_v} V "
+                      f"heads, {reps} passes ({total:.1f} s)"}
 
 
 def run_reference(args):
-    """The oracle (a plain sequential fp64 CPU program) as the reference arm."""
+    """The oracle (a plain sequential fp64 CPU program) as the reference arm: each step
+    is one pass over a bounded sample of the headline workload (its first sequences,
+    all V heads), timed as it runs."""
     ws, rank, _ = _dist()
     if rank != 0:
         return
-    from linear_attention_sequence_delta_b200.inputs import WORKLOADS, make_prefill_inputs
-    P = make_prefill_inputs(**WORKLOADS[WORKLOAD], seed=0)
-    heads = 8
+    import oracle
+    P = _reference_sample()
+    T, H_v = P.q.shape[0], P.v.shape[1]
     for _ in range(args.warmup):
-        cpu_baseline(P, heads=2, min_seconds=0.0)  # untimed warm-up (page in library, inputs)
-    vals = []
-    for _ in range(args.steps):
-        vals.append(cpu_baseline(P, heads=heads, min_seconds=0.0))  # one pass per step
-    v = statistics.median(x["value"] for x in vals)
-    T = P.q.shape[0]
+        _oracle_pass(P)
+    secs = [_oracle_pass(P) for _ in range(args.steps)]
+    ms = 1e3 * sum(secs) / len(secs)
+    v = T / (ms / 1e3)
+    sample = (f"{WORKLOAD}: first {P.num_seqs} sequences ({T} tokens), all {H_v} V heads, "
+              "one pass per step")
     line = {
         "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": T / v * 1e3, "higher_is_better": True,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "impl": "reference",
-        "config": {"workload": "prefill_35b: B=1, T=4096, H_qk=16, H_v=32, d=128, bf16 q/k/v "
-                               "(upcast exactly), fp64 arithmetic", "global_batch": 1,
-                   "seq_len": T, "parallelism": "host cores (OpenMP)"},
+        "config": {"workload": WORKLOAD_DESC + "; bf16 q/k/v upcast exactly, fp64 arithmetic",
+                   "global_batch": P.num_seqs, "seq_len": T,
+                   "parallelism": "host cores (OpenMP over (sequence, V head) units)"},
         "cpu_baseline": {"value": v, "unit": "tokens/s", "kind": "oracle",
-                         "cores": vals[0]["cores"], "sample": vals[0]["sample"]},
+                         "cores": oracle.num_threads(), "sample": sample},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -653,6 +686,9 @@ def main():
     ap.add_argument("--decode-seqs", type=int, default=256,
                     help="sequences per decode step (256 = the decode workload; smaller values "
                          "only for profiling captures)")
+    ap.add_argument("--seqs", type=int, default=None,
+                    help="sequences of the headline workload (default: its own 64; smaller "
+                         "values only for profiling captures)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -660,13 +696,13 @@ def main():
                     help="skip the conv1d / gated-norm measurements")
     ap.add_argument("--mixer-iters", type=int, default=20)
     ap.add_argument("--no-other-prefill", action="store_true",
-                    help="skip the 397B-A17B long and varlen_64 prefill measurements")
-    ap.add_argument("--other-iters", type=int, default=5)
-    ap.add_argument("--many-chains", default="prefill_397b_long,varlen_64",
-                    help="comma-separated workloads of the many-chain prefill block")
-    ap.add_argument("--many-chains-seqs", type=int, default=None,
-                    help="sequences per many-chain workload (default: the workload's own; "
-                         "smaller values only for profiling captures)")
+                    help="skip the 35B-A3B layer and 397B-A17B long prefill measurements")
+    ap.add_argument("--other-iters", type=int, default=10)
+    ap.add_argument("--other-prefill", default=",".join(OTHER_PREFILL),
+                    help="comma-separated workloads of the other-prefill block")
+    ap.add_argument("--other-prefill-seqs", type=int, default=None,
+                    help="sequences per other-prefill workload (default: the workload's "
+                         "own; smaller values only for profiling captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

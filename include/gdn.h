@@ -76,13 +76,15 @@ int gdn_version(void);
  * (64-token chunk, V head) an 8-byte ready flag and a 17,664-byte record (the
  * chunk's T diag(beta) and P matrices and per-token factors), i.e. about 276
  * bytes per token and V head (with one extra chunk per sequence), the first two
- * parts rounded up to 256 bytes; while GDN_IMPL_TENSOR_CORE_GRAM is selected, also
- * an 8,192-byte tile per (chunk, QK head) (the cross-chunk key Gram matrix), so a
- * workspace sized under another setting is too small for that one (the call then
- * returns GDN_ERR_WORKSPACE); for d = 64 (CUDA-core path) it is the per-token G and
- * beta, fp32 [T, H_v] each. Returns 0 for invalid sizes (and for num_seqs = 0).
- * The workspace needs no initialisation: a ready flag holds the number of the
- * call that wrote it, and call numbers grow within the process.
+ * parts rounded up to 256 bytes; for d = 64 (CUDA-core path) it is the per-token
+ * G and beta, fp32 [T, H_v] each. Returns 0 for invalid sizes (and for
+ * num_seqs = 0).
+ * The workspace needs no initialisation and may hold anything (earlier calls'
+ * records and flags, unrelated data): each call publishes its records under a
+ * 64-bit number that no earlier call of the process used (a random per-process
+ * base with the top bit set, plus a call counter), and a record counts as ready
+ * only when its flag equals that number. Stale words of any other origin equal
+ * it only by chance (probability 2^-64 per flag).
  */
 size_t gdn_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t H_qk,
                                   int32_t H_v, int32_t d_k, int32_t d_v);
@@ -132,45 +134,82 @@ int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
                 size_t workspace_bytes, void* stream);
 
 /*
- * Process-wide choice of the gdn_prefill implementation (for A/B comparison and
- * tests; the default is GDN_IMPL_AUTO):
- *   GDN_IMPL_AUTO         tensor cores (tcgen05) for bf16 I/O with d = 128 and at
- *                         most 16 V heads per QK head, the fp32 CUDA-core
- *                         kernel otherwise (fp32 I/O, d = 64);
- *   GDN_IMPL_CUDA_CORE    the fp32 CUDA-core kernel for every call;
- *   GDN_IMPL_TENSOR_CORE  tensor cores only; gdn_prefill then returns
- *                         GDN_ERR_UNSUPPORTED for shapes/types they do not cover;
- *   GDN_IMPL_TENSOR_CORE_SPLIT
- *                         tensor cores with the state-free preparation and the
- *                         chunk chain as separate launches always (by default
- *                         they run in one cooperative launch, overlapped, when
- *                         the device supports it and there are at most half as
- *                         many (sequence, V head) chains as SMs; with at most a
- *                         quarter as many, each chain is split over two blocks
- *                         that own 64 value rows each);
- *   GDN_IMPL_TENSOR_CORE_WHOLE_ROWS
- *                         the one-launch schedule whenever it applies, but never
- *                         with half-row chain blocks;
- *   GDN_IMPL_TENSOR_CORE_GRAM
- *                         as GDN_IMPL_TENSOR_CORE, but half-row chain blocks form
- *                         S_c K_c^T as e^{G_L} S_{c-1} K_c^T + W_{c-1} (K_{c-1} K_c^T)
- *                         with the cross-chunk key Gram matrix from the
- *                         preparation, which takes the state update off the path
- *                         from one chunk to the next (the same mathematics with a
- *                         different bf16 rounding, so not bit-identical to the
- *                         other schedules).
- * Returns the previous setting, or -GDN_ERR_INVALID_ARG for an unknown value.
- * Not synchronised with calls in flight on other host threads.
+ * gdn_prefill_ex / gdn_prefill_slots_ex -- gdn_prefill / gdn_prefill_slots with
+ * per-call options, for A/B comparison, measurement and tests of the failure
+ * paths (the pages have no counterpart). A NULL options pointer, or all fields
+ * zero, is exactly gdn_prefill / gdn_prefill_slots. Nothing here is process-wide
+ * state: every option applies to this call only.
+ *   impl               which implementation runs:
+ *     GDN_IMPL_AUTO         tensor cores (tcgen05) for bf16 I/O with d = 128 and at
+ *                           most 16 V heads per QK head, the fp32 CUDA-core kernel
+ *                           otherwise (fp32 I/O, d = 64). On the tensor-core path,
+ *                           with at most half as many (sequence, V head) chains as
+ *                           SMs, preparation and chains run overlapped in one
+ *                           cooperative launch (with at most a quarter as many,
+ *                           each chain is split over two blocks of 64 value rows);
+ *                           otherwise as separate launches.
+ *     GDN_IMPL_CUDA_CORE    the fp32 CUDA-core kernel for every shape.
+ *     GDN_IMPL_TENSOR_CORE  tensor cores only (GDN_ERR_UNSUPPORTED for shapes and
+ *                           types they do not cover), scheduled as AUTO.
+ *     GDN_IMPL_TENSOR_CORE_SPLIT       tensor cores, always separate launches.
+ *     GDN_IMPL_TENSOR_CORE_WHOLE_ROWS  tensor cores, never half-row chain blocks.
+ *   fault              GDN_FAULT_NONE, or GDN_FAULT_WITHHOLD_RECORDS: in the
+ *                      overlapped launch the preparation publishes no record, so
+ *                      every chain's bounded wait for its first record runs out;
+ *                      the call then ends with GDN_ERR_TIMEOUT in the device
+ *                      status word (outputs undefined) and the context stays
+ *                      usable. Nothing faults. Other launches ignore it.
+ *   wait_limit_cycles  limit of every bounded device-side wait of the tensor-core
+ *                      path, in SM clock cycles; 0 = the default (4e9, about 2 s).
+ *   timer              NULL, or a timer from gdn_timer_create: CUDA events are
+ *                      recorded on `stream` around each kernel the call launches.
  */
 enum {
     GDN_IMPL_AUTO = 0,
     GDN_IMPL_CUDA_CORE = 1,
     GDN_IMPL_TENSOR_CORE = 2,
     GDN_IMPL_TENSOR_CORE_SPLIT = 3,
-    GDN_IMPL_TENSOR_CORE_WHOLE_ROWS = 4,
-    GDN_IMPL_TENSOR_CORE_GRAM = 5
+    GDN_IMPL_TENSOR_CORE_WHOLE_ROWS = 4
 };
-int gdn_set_prefill_impl(int32_t impl);
+enum { GDN_FAULT_NONE = 0, GDN_FAULT_WITHHOLD_RECORDS = 1 };
+
+typedef struct gdn_timer gdn_timer;
+
+typedef struct {
+    int32_t impl;
+    int32_t fault;
+    int64_t wait_limit_cycles;
+    gdn_timer* timer;
+} gdn_prefill_options;
+
+int gdn_prefill_ex(const void* q, const void* k, const void* v, int32_t io_dtype,
+                   const float* a, const float* b, const float* A_log, const float* dt_bias,
+                   const float* initial_state, const int32_t* cu_seqlens, int32_t num_seqs,
+                   int64_t total_tokens, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
+                   float scale, void* o, float* final_state, void* workspace,
+                   size_t workspace_bytes, const gdn_prefill_options* options, void* stream);
+
+/*
+ * Kernel timing of gdn_prefill_ex -- a measurement aid; the pages have no
+ * counterpart. A timer owns 8 CUDA events of the device current at creation (it
+ * is the only object of this library that allocates, and only here).
+ *   gdn_timer_create      returns a timer, or NULL if the events cannot be made.
+ *   gdn_timer_destroy     frees it (NULL is ignored).
+ *   gdn_timer_read        waits for the events of the most recent call that used
+ *                         the timer and writes the durations of its first
+ *                         min(count, max_kernels) kernels, in milliseconds, to ms
+ *                         (host array); returns the kernel count (at most 4), or
+ *                         -GDN_ERR_INVALID_ARG / -GDN_ERR_CUDA.
+ *   gdn_timer_kernel_name name of kernel i of that call ("chunk_offsets", "prep",
+ *                         "chain", "fused", "fused_half_rows" on the tensor-core
+ *                         path; "gates", "prefill_simt" on the CUDA-core path), or
+ *                         NULL.
+ * A timer may be used by one call at a time.
+ */
+gdn_timer* gdn_timer_create(void);
+void gdn_timer_destroy(gdn_timer* timer);
+int gdn_timer_read(gdn_timer* timer, float* ms, int32_t max_kernels);
+const char* gdn_timer_kernel_name(const gdn_timer* timer, int32_t i);
 
 /*
  * gdn_decode_step -- one token for each of N sequences, the state updated in
@@ -255,23 +294,42 @@ int gdn_prefill_slots(const void* q, const void* k, const void* v, int32_t io_dt
                       const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
                       int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v, float scale, void* o,
                       void* workspace, size_t workspace_bytes, void* stream);
+int gdn_prefill_slots_ex(const void* q, const void* k, const void* v, int32_t io_dtype,
+                         const float* a, const float* b, const float* A_log,
+                         const float* dt_bias, float* state_pool, const int32_t* state_slots,
+                         const int32_t* has_initial_state, int32_t num_slots,
+                         const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                         int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v, float scale,
+                         void* o, void* workspace, size_t workspace_bytes,
+                         const gdn_prefill_options* options, void* stream);
 
 /*
  * gdn_prefill_noalloc -- gdn_prefill for callers that cannot allocate device
  * memory. The pages have no counterpart: this is a deployment variant.
  *
- * gdn_prefill asks the caller for a workspace (the per-token gates G and beta).
- * Callers that cannot call cudaMalloc -- code running under CUDA graph stream
- * capture, runtimes whose device memory belongs to a pool they must not touch,
- * plugins that are handed only their input and output buffers -- use this call
- * instead: the same computation and the same arguments minus the workspace, with
- * the scratch kept in a fixed array inside the library.
+ * gdn_prefill asks the caller for a workspace. Some callers cannot call
+ * cudaMalloc or any allocator at the point where they run the mixer: a runtime
+ * whose device memory is owned by a pool it must not touch, a plugin that is
+ * handed only its input and output buffers, code that runs where an allocation
+ * would block or synchronise the device. This call takes the same arguments minus
+ * the workspace and keeps its scratch (the per-token G and beta) in a fixed
+ * array inside the library.
+ *   - It always runs the fp32 CUDA-core chunk kernel (the gate kernel, then the
+ *     CUDA-core prefill), whatever the shape and type: the tensor-core path needs
+ *     a workspace proportional to the tokens (about 276 bytes per token and V
+ *     head), which a fixed array cannot hold for useful sizes. The results agree
+ *     with gdn_prefill within the same tolerances; for bf16 with d = 128 the call
+ *     is much slower (on the 35B-A3B layer shape, T = 4096 with 32 V heads: about
+ *     3.5 ms against about 0.14 ms for gdn_prefill).
  *   - Capacity: total_tokens * H_v <= GDN_NOALLOC_MAX_GATE_ELEMS; larger calls
  *     return GDN_ERR_WORKSPACE and launch nothing (use gdn_prefill for them).
  *     The array (8 MiB) is held on every GPU that loads the library until the
  *     process exits.
  *   - The first call on each device looks up the array's device address (with
- *     that device current); make that first call before any stream capture.
+ *     that device current) and caches it; make that first call before any
+ *     stream capture. The cached address is not renewed: after cudaDeviceReset
+ *     (or anything else that destroys the device's primary context) the library
+ *     must be reloaded before this call is used again.
  *   - Every call shares the one array: calls that overlap on the GPU (two
  *     streams, or two host threads on one device) race and give wrong results.
  *     Serialise them (one stream) or use gdn_prefill with separate workspaces.
@@ -284,29 +342,6 @@ int gdn_prefill_noalloc(const void* q, const void* k, const void* v, int32_t io_
                         const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
                         int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v, float scale,
                         void* o, float* final_state, void* stream);
-
-/*
- * Kernel timing of gdn_prefill -- a measurement aid; the pages have no
- * counterpart. While enabled (gdn_set_kernel_timing(1)), every gdn_prefill call
- * records a CUDA event before and after each kernel it launches, on the call's
- * stream (at most 4 kernels per call; the library owns the events).
- *   gdn_set_kernel_timing   enable (nonzero) or disable; returns the previous
- *                           setting.
- *   gdn_last_prefill_kernel_ms
- *                           waits for the events of the most recent timed call
- *                           and writes the duration of its first
- *                           min(count, max_kernels) kernels, in milliseconds, to
- *                           ms (host array); returns the kernel count, or
- *                           -GDN_ERR_INVALID_ARG / -GDN_ERR_CUDA.
- *   gdn_last_prefill_kernel_name
- *                           name of kernel i of that call ("chunk_offsets",
- *                           "prep", "chain" on the tensor-core path; "gates",
- *                           "prefill_simt" on the CUDA-core path), or NULL.
- * The timing state is process-wide: time from one host thread at a time.
- */
-int gdn_set_kernel_timing(int32_t enable);
-int gdn_last_prefill_kernel_ms(float* ms, int32_t max_kernels);
-const char* gdn_last_prefill_kernel_name(int32_t i);
 
 /*
  * The steps around the delta rule in the GDN token mixer ("Qwen3.5-MoE-35B-A3B

@@ -4,6 +4,7 @@
 
 #include <atomic>
 #include <mutex>
+#include <new>
 
 #include "gdn_internal.cuh"
 
@@ -15,7 +16,6 @@ __device__ int g_status_word;
 
 namespace {
 constexpr int kMaxDevices = 64;
-std::atomic<int> g_prefill_impl{GDN_IMPL_AUTO};
 std::atomic<int*> g_status_ptr[kMaxDevices];
 std::mutex g_status_mu;
 
@@ -35,50 +35,32 @@ int check_heads(int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v) {
 }
 
 size_t gate_bytes(int64_t T, int32_t H_v) { return align_up((size_t)T * H_v * sizeof(float), 256); }
-// Kernel timing state (process-wide; meant for one measuring thread at a time).
-constexpr int kMaxTimed = 4;
-std::atomic<int> g_ktiming{0};
-struct KernelTimer {
-    cudaEvent_t ev[2 * kMaxTimed] = {};
-    const char* name[kMaxTimed] = {};
-    int n = 0;
-    int dev = -1;
-    bool open = false;  // an event pair is half recorded
-};
-KernelTimer g_kt;
-
-bool ktimer_ready() {
-    if (!g_ktiming.load(std::memory_order_relaxed)) return false;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return false;
-    if (g_kt.dev != dev) {
-        for (cudaEvent_t& e : g_kt.ev) {
-            if (e) cudaEventDestroy(e);
-            e = nullptr;
-        }
-        for (cudaEvent_t& e : g_kt.ev)
-            if (cudaEventCreate(&e) != cudaSuccess) return false;
-        g_kt.dev = dev;
-        g_kt.n = 0;
-    }
-    return true;
-}
 }  // namespace
 
-void ktimer_reset() {
-    if (ktimer_ready()) g_kt.n = 0;
+}  // namespace gdn
+
+// A caller-owned kernel timer (gdn_timer_create): event pairs around each kernel of
+// the most recent call that used it.
+struct gdn_timer {
+    static constexpr int kMax = 4;
+    cudaEvent_t ev[2 * kMax] = {};
+    const char* name[kMax] = {};
+    int n = 0;
+    bool open = false;  // an event pair is half recorded
+};
+
+namespace gdn {
+
+void timer_before(gdn_timer* t, cudaStream_t s) {
+    if (!t || t->n >= gdn_timer::kMax) return;
+    t->open = cudaEventRecord(t->ev[2 * t->n], s) == cudaSuccess;
 }
 
-void ktimer_before(cudaStream_t s) {
-    if (!ktimer_ready() || g_kt.n >= kMaxTimed) return;
-    g_kt.open = cudaEventRecord(g_kt.ev[2 * g_kt.n], s) == cudaSuccess;
-}
-
-void ktimer_after(cudaStream_t s, const char* kernel) {
-    if (!ktimer_ready() || g_kt.n >= kMaxTimed || !g_kt.open) return;
-    g_kt.open = false;
-    if (cudaEventRecord(g_kt.ev[2 * g_kt.n + 1], s) != cudaSuccess) return;
-    g_kt.name[g_kt.n++] = kernel;
+void timer_after(gdn_timer* t, cudaStream_t s, const char* kernel) {
+    if (!t || t->n >= gdn_timer::kMax || !t->open) return;
+    t->open = false;
+    if (cudaEventRecord(t->ev[2 * t->n + 1], s) != cudaSuccess) return;
+    t->name[t->n++] = kernel;
 }
 
 int* device_status_ptr() {
@@ -126,8 +108,7 @@ size_t gdn_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_
     if (num_seqs == 0) return 0;  // an empty batch launches nothing
     const size_t simt = 2 * gate_bytes(total_tokens, H_v);
     if (d_k != 128) return simt;
-    const bool gram = g_prefill_impl.load(std::memory_order_relaxed) == GDN_IMPL_TENSOR_CORE_GRAM;
-    const size_t tc = prefill_tc_workspace_bytes(num_seqs, total_tokens, H_qk, H_v, gram);
+    const size_t tc = prefill_tc_workspace_bytes(num_seqs, total_tokens, H_v);
     return tc > simt ? tc : simt;
 }
 
@@ -150,14 +131,26 @@ int gdn_gates(const float* a, const float* b, const float* A_log, const float* d
 }  // extern "C"
 
 namespace {
-// gdn_prefill and gdn_prefill_slots: the same path, the states addressed per sequence or
-// through pool slots
+// gdn_prefill(_ex) and gdn_prefill_slots(_ex): the same path, the states addressed per
+// sequence or through pool slots
 int prefill_common(const void* q, const void* k, const void* v, int32_t io_dtype,
                    const float* a, const float* b, const float* A_log, const float* dt_bias,
                    const float* initial_state, const int32_t* cu_seqlens, int32_t num_seqs,
                    int64_t total_tokens, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
                    float scale, void* o, float* final_state, StateIndex sref, void* workspace,
-                   size_t workspace_bytes, void* stream) {
+                   size_t workspace_bytes, const gdn_prefill_options* options, void* stream) {
+    PrefillOpts opt;
+    if (options) {
+        if (options->impl < GDN_IMPL_AUTO || options->impl > GDN_IMPL_TENSOR_CORE_WHOLE_ROWS)
+            return GDN_ERR_INVALID_ARG;
+        if (options->fault != GDN_FAULT_NONE && options->fault != GDN_FAULT_WITHHOLD_RECORDS)
+            return GDN_ERR_INVALID_ARG;
+        if (options->wait_limit_cycles < 0) return GDN_ERR_INVALID_ARG;
+        opt.impl = options->impl;
+        opt.fault = options->fault;
+        if (options->wait_limit_cycles > 0) opt.wait_cycles = options->wait_limit_cycles;
+        opt.timer = options->timer;
+    }
     if (io_dtype != GDN_BF16 && io_dtype != GDN_FP32) return GDN_ERR_INVALID_ARG;
     if (num_seqs < 0 || total_tokens < 0) return GDN_ERR_INVALID_ARG;
     if (num_seqs == 0 && total_tokens != 0) return GDN_ERR_INVALID_ARG;
@@ -176,41 +169,59 @@ int prefill_common(const void* q, const void* k, const void* v, int32_t io_dtype
     if (workspace_bytes < need || (need > 0 && !workspace)) return GDN_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return GDN_ERR_WORKSPACE;
 
-    const int impl = g_prefill_impl.load(std::memory_order_relaxed);
     const bool tc_ok =
         io_dtype == GDN_BF16 && d_k == 128 && prefill_tc_supported(H_qk, H_v);
-    if ((impl == GDN_IMPL_TENSOR_CORE || impl == GDN_IMPL_TENSOR_CORE_SPLIT ||
-         impl == GDN_IMPL_TENSOR_CORE_WHOLE_ROWS || impl == GDN_IMPL_TENSOR_CORE_GRAM) && !tc_ok)
-        return GDN_ERR_UNSUPPORTED;
+    const bool tc_forced = opt.impl == GDN_IMPL_TENSOR_CORE ||
+                           opt.impl == GDN_IMPL_TENSOR_CORE_SPLIT ||
+                           opt.impl == GDN_IMPL_TENSOR_CORE_WHOLE_ROWS;
+    if (tc_forced && !tc_ok) return GDN_ERR_UNSUPPORTED;
     int* st = device_status_ptr();
     if (!st) return GDN_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
-    ktimer_reset();
-    if (tc_ok && impl != GDN_IMPL_CUDA_CORE) {
+    if (opt.timer) opt.timer->n = 0;
+    if (tc_ok && opt.impl != GDN_IMPL_CUDA_CORE) {
         return to_status(launch_prefill_tc(q, k, v, a, b, A_log, dt_bias, initial_state,
                                            cu_seqlens, num_seqs, total_tokens, H_qk, H_v, scale,
-                                           o, final_state, sref, workspace,
-                                           impl == GDN_IMPL_TENSOR_CORE_SPLIT ? 0
-                                           : impl == GDN_IMPL_TENSOR_CORE_WHOLE_ROWS ? 1
-                                           : impl == GDN_IMPL_TENSOR_CORE_GRAM ? 3 : 2,
-                                           st, s));
+                                           o, final_state, sref, workspace, opt, st, s));
     }
     float* G = static_cast<float*>(workspace);
     float* beta = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                            gate_bytes(total_tokens, H_v));
     if (total_tokens > 0) {
-        ktimer_before(s);
+        timer_before(opt.timer, s);
         cudaError_t e = launch_gates(a, b, A_log, dt_bias, cu_seqlens, num_seqs, total_tokens,
                                      H_v, G, nullptr, beta, st, s);
         if (e != cudaSuccess) return GDN_ERR_CUDA;
-        ktimer_after(s, "gates");
+        timer_after(opt.timer, s, "gates");
     }
-    ktimer_before(s);
+    timer_before(opt.timer, s);
     const int rs = to_status(launch_prefill_simt(q, k, v, io_dtype, G, beta, initial_state,
                                                  cu_seqlens, num_seqs, total_tokens, H_qk, H_v,
                                                  d_k, scale, o, final_state, sref, st, s));
-    ktimer_after(s, "prefill_simt");
+    timer_after(opt.timer, s, "prefill_simt");
     return rs;
+}
+
+int prefill_slots_common(const void* q, const void* k, const void* v, int32_t io_dtype,
+                         const float* a, const float* b, const float* A_log,
+                         const float* dt_bias, float* state_pool, const int32_t* state_slots,
+                         const int32_t* has_initial_state, int32_t num_slots,
+                         const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                         int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v, float scale,
+                         void* o, void* workspace, size_t workspace_bytes,
+                         const gdn_prefill_options* options, void* stream) {
+    if (num_seqs > 0 && (!state_slots || !state_pool)) return GDN_ERR_INVALID_ARG;
+    if (num_slots < 0) return GDN_ERR_INVALID_ARG;
+    if ((state_slots && !aligned(state_slots, 4)) ||
+        (has_initial_state && !aligned(has_initial_state, 4)))
+        return GDN_ERR_INVALID_ARG;
+    StateIndex sref;
+    sref.slots = state_slots;
+    sref.has_init = has_initial_state;
+    sref.num_slots = num_slots;
+    return prefill_common(q, k, v, io_dtype, a, b, A_log, dt_bias, state_pool, cu_seqlens,
+                          num_seqs, total_tokens, H_qk, H_v, d_k, d_v, scale, o, state_pool, sref,
+                          workspace, workspace_bytes, options, stream);
 }
 }  // namespace
 
@@ -224,7 +235,18 @@ int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
                 size_t workspace_bytes, void* stream) {
     return prefill_common(q, k, v, io_dtype, a, b, A_log, dt_bias, initial_state, cu_seqlens,
                           num_seqs, total_tokens, H_qk, H_v, d_k, d_v, scale, o, final_state,
-                          StateIndex{}, workspace, workspace_bytes, stream);
+                          StateIndex{}, workspace, workspace_bytes, nullptr, stream);
+}
+
+int gdn_prefill_ex(const void* q, const void* k, const void* v, int32_t io_dtype,
+                   const float* a, const float* b, const float* A_log, const float* dt_bias,
+                   const float* initial_state, const int32_t* cu_seqlens, int32_t num_seqs,
+                   int64_t total_tokens, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
+                   float scale, void* o, float* final_state, void* workspace,
+                   size_t workspace_bytes, const gdn_prefill_options* options, void* stream) {
+    return prefill_common(q, k, v, io_dtype, a, b, A_log, dt_bias, initial_state, cu_seqlens,
+                          num_seqs, total_tokens, H_qk, H_v, d_k, d_v, scale, o, final_state,
+                          StateIndex{}, workspace, workspace_bytes, options, stream);
 }
 
 int gdn_prefill_slots(const void* q, const void* k, const void* v, int32_t io_dtype,
@@ -234,18 +256,24 @@ int gdn_prefill_slots(const void* q, const void* k, const void* v, int32_t io_dt
                       const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
                       int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v, float scale, void* o,
                       void* workspace, size_t workspace_bytes, void* stream) {
-    if (num_seqs > 0 && (!state_slots || !state_pool)) return GDN_ERR_INVALID_ARG;
-    if (num_slots < 0) return GDN_ERR_INVALID_ARG;
-    if ((state_slots && !aligned(state_slots, 4)) ||
-        (has_initial_state && !aligned(has_initial_state, 4)))
-        return GDN_ERR_INVALID_ARG;
-    StateIndex sref;
-    sref.slots = state_slots;
-    sref.has_init = has_initial_state;
-    sref.num_slots = num_slots;
-    return prefill_common(q, k, v, io_dtype, a, b, A_log, dt_bias, state_pool, cu_seqlens,
-                          num_seqs, total_tokens, H_qk, H_v, d_k, d_v, scale, o, state_pool, sref,
-                          workspace, workspace_bytes, stream);
+    return prefill_slots_common(q, k, v, io_dtype, a, b, A_log, dt_bias, state_pool,
+                                state_slots, has_initial_state, num_slots, cu_seqlens, num_seqs,
+                                total_tokens, H_qk, H_v, d_k, d_v, scale, o, workspace,
+                                workspace_bytes, nullptr, stream);
+}
+
+int gdn_prefill_slots_ex(const void* q, const void* k, const void* v, int32_t io_dtype,
+                         const float* a, const float* b, const float* A_log,
+                         const float* dt_bias, float* state_pool, const int32_t* state_slots,
+                         const int32_t* has_initial_state, int32_t num_slots,
+                         const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                         int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v, float scale,
+                         void* o, void* workspace, size_t workspace_bytes,
+                         const gdn_prefill_options* options, void* stream) {
+    return prefill_slots_common(q, k, v, io_dtype, a, b, A_log, dt_bias, state_pool,
+                                state_slots, has_initial_state, num_slots, cu_seqlens, num_seqs,
+                                total_tokens, H_qk, H_v, d_k, d_v, scale, o, workspace,
+                                workspace_bytes, options, stream);
 }
 
 int gdn_decode_step(const void* q, const void* k, const void* v, int32_t io_dtype,
@@ -377,31 +405,39 @@ int gdn_rmsnorm_gated(const void* o, const void* z, int32_t io_dtype, const floa
         launch_rmsnorm_gated(o, z, io_dtype, weight, eps, rows, d, y, (cudaStream_t)stream));
 }
 
-int gdn_set_prefill_impl(int32_t impl) {
-    if (impl != GDN_IMPL_AUTO && impl != GDN_IMPL_CUDA_CORE && impl != GDN_IMPL_TENSOR_CORE &&
-        impl != GDN_IMPL_TENSOR_CORE_SPLIT && impl != GDN_IMPL_TENSOR_CORE_WHOLE_ROWS &&
-        impl != GDN_IMPL_TENSOR_CORE_GRAM)
-        return -GDN_ERR_INVALID_ARG;
-    return g_prefill_impl.exchange(impl);
+gdn_timer* gdn_timer_create(void) {
+    gdn_timer* t = new (std::nothrow) gdn_timer();
+    if (!t) return nullptr;
+    for (cudaEvent_t& e : t->ev) {
+        if (cudaEventCreate(&e) != cudaSuccess) {
+            e = nullptr;
+            gdn_timer_destroy(t);
+            return nullptr;
+        }
+    }
+    return t;
 }
 
-int gdn_set_kernel_timing(int32_t enable) {
-    return g_ktiming.exchange(enable ? 1 : 0);
+void gdn_timer_destroy(gdn_timer* t) {
+    if (!t) return;
+    for (cudaEvent_t e : t->ev)
+        if (e) cudaEventDestroy(e);
+    delete t;
 }
 
-int gdn_last_prefill_kernel_ms(float* ms, int32_t max_kernels) {
-    if (!ms || max_kernels < 0) return -GDN_ERR_INVALID_ARG;
-    const int n = g_kt.n < max_kernels ? g_kt.n : max_kernels;
+int gdn_timer_read(gdn_timer* t, float* ms, int32_t max_kernels) {
+    if (!t || !ms || max_kernels < 0) return -GDN_ERR_INVALID_ARG;
+    const int n = t->n < max_kernels ? t->n : max_kernels;
     for (int i = 0; i < n; ++i) {
-        if (cudaEventSynchronize(g_kt.ev[2 * i + 1]) != cudaSuccess ||
-            cudaEventElapsedTime(&ms[i], g_kt.ev[2 * i], g_kt.ev[2 * i + 1]) != cudaSuccess)
+        if (cudaEventSynchronize(t->ev[2 * i + 1]) != cudaSuccess ||
+            cudaEventElapsedTime(&ms[i], t->ev[2 * i], t->ev[2 * i + 1]) != cudaSuccess)
             return -GDN_ERR_CUDA;
     }
-    return g_kt.n;
+    return t->n;
 }
 
-const char* gdn_last_prefill_kernel_name(int32_t i) {
-    return (i >= 0 && i < g_kt.n) ? g_kt.name[i] : nullptr;
+const char* gdn_timer_kernel_name(const gdn_timer* t, int32_t i) {
+    return (t && i >= 0 && i < t->n) ? t->name[i] : nullptr;
 }
 
 int gdn_sync_status(void* stream) {

@@ -95,12 +95,19 @@ struct StateIndex {
 // Status word of the current device (a __device__ int of this library).
 int* device_status_ptr();
 
-// ---- optional per-kernel timing of gdn_prefill (see gdn_set_kernel_timing) ----
-// While timing is enabled, every kernel launch of gdn_prefill is bracketed by two
-// CUDA events recorded on the launch stream; otherwise these do nothing.
-void ktimer_reset();
-void ktimer_before(cudaStream_t s);
-void ktimer_after(cudaStream_t s, const char* kernel);
+// ---- per-call options of the prefill (gdn_prefill_ex) ----
+// Default limit of a bounded device-side wait: about 2 s at 2 GHz.
+constexpr long long kDefaultWaitCycles = 4000000000LL;
+struct PrefillOpts {
+    int impl = GDN_IMPL_AUTO;
+    int fault = GDN_FAULT_NONE;
+    long long wait_cycles = kDefaultWaitCycles;
+    gdn_timer* timer = nullptr;
+};
+// With a timer, every kernel launch of the call is bracketed by two CUDA events
+// recorded on the launch stream; with NULL these do nothing.
+void timer_before(gdn_timer* t, cudaStream_t s);
+void timer_after(gdn_timer* t, cudaStream_t s, const char* kernel);
 
 cudaError_t launch_gates(const float* a, const float* b, const float* A_log,
                          const float* dt_bias, const int32_t* cu_seqlens, int32_t num_seqs,
@@ -136,19 +143,18 @@ cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, int
                                 StateIndex sref, int* status, cudaStream_t s);
 
 // Tensor-core prefill (bf16 I/O, d = 128): chunk offsets, the state-independent
-// prep kernel, then the chain kernel. schedule: 0 = always separate launches, 1 = one
-// cooperative launch where it pays (whole-row chain blocks), 2 = the same with half-row
-// chain blocks when the chains are few enough. The workspace holds the chunk offsets and
-// one record (T, P and per-token factors) per (chunk, V head).
-// `gram`: room for the cross-chunk Gram tiles of the Gram-matrix schedule (schedule 3)
-size_t prefill_tc_workspace_bytes(int32_t N, int64_t T, int32_t H_qk, int32_t H_v, bool gram);
+// prep kernel, then the chain kernel, or both stages in one cooperative launch where
+// that pays (opt.impl: GDN_IMPL_TENSOR_CORE_SPLIT forces separate launches,
+// GDN_IMPL_TENSOR_CORE_WHOLE_ROWS forbids half-row chain blocks). The workspace holds
+// the chunk offsets and one record (T, P and per-token factors) per (chunk, V head).
+size_t prefill_tc_workspace_bytes(int32_t N, int64_t T, int32_t H_v);
 bool prefill_tc_supported(int32_t H_qk, int32_t H_v);
 cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const float* a,
                               const float* b, const float* A_log, const float* dt_bias,
                               const float* S0, const int32_t* cu_seqlens, int32_t N, int64_t T,
                               int32_t H_qk, int32_t H_v, float scale, void* o, float* S_final,
-                              StateIndex sref, void* workspace, int schedule, int* status,
-                              cudaStream_t s);
+                              StateIndex sref, void* workspace, const PrefillOpts& opt,
+                              int* status, cudaStream_t s);
 
 // Steps around the delta rule (gdn_mixer.cu): causal depthwise conv1d + SiLU with
 // the per-sequence conv cache, its single-token decode form, and the gated RMSNorm.

@@ -1,13 +1,15 @@
 // gdn_prefill_noalloc: the chunked prefill for callers that cannot allocate
 // device memory.
 //
-// gdn_prefill needs a caller-provided workspace for the per-token gates (the
-// chunk-cumulative log-decay G and beta). Some callers cannot provide one: code
-// running while a CUDA graph is being captured, where a cudaMalloc would break
-// the capture; runtimes whose device memory is fully owned by a pool they must
-// not disturb; plugins handed only input and output buffers. This entry point
-// keeps that scratch in a fixed array inside the library instead, so the caller
-// passes only inputs and outputs and nothing is allocated on any call.
+// gdn_prefill needs a caller-provided workspace. Some callers cannot provide one:
+// a runtime whose device memory is fully owned by a pool it must not disturb, a
+// plugin handed only input and output buffers, code that runs where an allocation
+// would block or synchronise the device. This entry point keeps its scratch (the
+// chunk-cumulative log-decay G and beta of every token) in a fixed array inside
+// the library instead, so the caller passes only inputs and outputs and nothing is
+// allocated on any call. It always runs the fp32 CUDA-core chunk kernel: the
+// tensor-core path's workspace grows with the tokens (about 276 bytes per token and
+// V head), which a fixed array cannot hold for useful sizes.
 //
 // The array is a file-scope __device__ variable: every GPU that loads this
 // library holds it (kNoallocScratchBytes) until the process exits. In host code

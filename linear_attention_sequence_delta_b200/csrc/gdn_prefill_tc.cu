@@ -41,16 +41,17 @@
 // cooperative launch (fused_kernel), chain blocks consuming records as prep blocks
 // publish them (per-record flags holding the call's number); with at most a quarter
 // as many chains as SMs each chain is split over two blocks of 64 value rows (M = 64
-// MMAs). Otherwise three launches: chunk offsets, prep_kernel, chain_kernel. An
-// opt-in schedule (kGram) forms S_c K_c^T from the previous chunk's state and the
-// cross-chunk key Gram matrix K_{c-1} K_c^T that prep provides, taking the state
-// update off the path from one chunk to the next.
+// MMAs). Otherwise three launches: chunk offsets, prep_kernel, chain_kernel.
 //
 // Every wait is bounded; on expiry a block records GDN_ERR_TIMEOUT in the status
 // word, leaves its loops, drains its copies, frees its tensor memory and exits.
 #include <cuda.h>
 
+#include <unistd.h>
+
 #include <atomic>
+#include <chrono>
+#include <random>
 
 #include "gdn_internal.cuh"
 #include "sm100_ptx.cuh"
@@ -64,7 +65,6 @@ using bf16 = __nv_bfloat16;
 
 constexpr int kD = 128;
 constexpr int kC = kChunk;  // 64
-constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 2 GHz
 constexpr int kMaxGroup = 16;                    // V heads per QK head handled by prep
 
 // ---- workspace record of one (chunk, V head), written by prep, bulk-copied by chain
@@ -76,10 +76,6 @@ constexpr int RG_EGQ = 128;          //   [64] e^{G_t} rq_t
 constexpr int RG_EGL = 192;          //   [64] e^{G_L - G_t} rk_t
 constexpr int RG_GAMMA = 256;        //   e^{G_L}
 constexpr uint32_t kRecBytes = 17664;  // 69 x 256
-// Cross-chunk key Gram matrix of (chunk c, QK head): K_c K_{c-1}^T of the raw bf16 rows,
-// row n = token n of chunk c, column m = token m of chunk c-1, as a bf16 sw128 image
-// (zero for a sequence's first chunk).
-constexpr uint32_t kGramBytes = 8192;
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -260,18 +256,16 @@ __device__ __forceinline__ void publish_record(unsigned long long* flags, size_t
 
 // One prep worker of kPrepThreads threads (tid 0 .. 255, synchronised by the named
 // barrier bar_id) walks the (chunk, QK head) units worker, worker + nworkers, ...
-// and writes their records; with `flags`, each finished record is published. With
-// `gram`, it also writes each unit's cross-chunk key Gram matrix K_c K_{c-1}^T (the
-// previous chunk's raw K rows staged where A is built later; a second MMA beside
-// K K^T into TMEM columns 64-127) before the unit's first record is published.
+// and writes their records; with `flags`, each finished record is published.
 __device__ __forceinline__ void prep_worker(
     const bf16* __restrict__ q, const bf16* __restrict__ k, const float* __restrict__ a,
     const float* __restrict__ b, const float* __restrict__ A_log,
     const float* __restrict__ dt_bias, const int32_t* __restrict__ cu_seqlens,
     const int32_t* __restrict__ choff, int32_t N, int H_qk, int H_v, float scale,
-    uint8_t* __restrict__ rec, uint8_t* __restrict__ gram, int* status,
+    uint8_t* __restrict__ rec, int* status,
     unsigned long long* flags, unsigned long long epoch, uint8_t* sm, const int tid,
-    const int bar_id, const int worker, const int nworkers, const bool relinquish) {
+    const int bar_id, const int worker, const int nworkers, const bool relinquish,
+    const long long wait_cycles) {
     uint8_t* KQ = sm + PS_KQ;
     float* Ts = reinterpret_cast<float*>(sm + PS_TS);
     float* As = reinterpret_cast<float*>(sm + PS_AS);
@@ -292,7 +286,7 @@ __device__ __forceinline__ void prep_worker(
     const int r = H_v / H_qk;
     const int total_units = choff[N] * H_qk;
 
-    const uint32_t tcols = gram ? 128u : 64u;
+    constexpr uint32_t tcols = 64u;
     if (warp == 0) {
         tmem_alloc(s_tmem, tcols);
         if (relinquish) tmem_relinquish();
@@ -337,13 +331,6 @@ __device__ __forceinline__ void prep_worker(
             const uint32_t off = (uint32_t)(ch >> 3) * 16384u;
             cp_async_16(KQ + off + sw128_off(rr, ch & 7), k + rowk, live ? 16u : 0u);
             cp_async_16(KQ + off + sw128_off(rr + 64, ch & 7), q + rowk, live ? 16u : 0u);
-            if (gram) {  // the previous chunk's K rows (zeros before the sequence's start)
-                const bool prev = cg > choff[n];
-                const size_t rowp = ((size_t)(prev ? t0 - kC + rr : 0) * H_qk + j) * kD + ch * 8;
-                cp_async_16(reinterpret_cast<uint8_t*>(As) + (uint32_t)(ch >> 3) * 8192u +
-                                sw128_off(rr, ch & 7),
-                            k + rowp, prev ? 16u : 0u);
-            }
         }
         for (int idx = tid; idx < 2 * r * kC; idx += kPrepThreads) {
             const int which = idx / (r * kC);            // 0: a, 1: b
@@ -398,16 +385,6 @@ __device__ __forceinline__ void prep_worker(
                 mma_bf16_ss(tmem, smem_desc_sw128(kq + off, 16, 1024),
                             smem_desc_sw128(kq + off, 16, 1024), id_kq, ks > 0);
             }
-            if (gram) {  // [K; Q] K_{c-1}^T: rows 0-63 are the Gram matrix
-                const uint32_t kp = smem_u32(As);
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t off = (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u;
-                    const uint32_t offp = (uint32_t)(ks >> 2) * 8192u + (uint32_t)(ks & 3) * 32u;
-                    mma_bf16_ss(tmem + 64, smem_desc_sw128(kq + off, 16, 1024),
-                                smem_desc_sw128(kp + offp, 16, 1024), id_kq, ks > 0);
-                }
-            }
             mma_commit(bar);
         }
         // ---- gates of every V head of the group: one warp per head, two tokens a lane:
@@ -440,27 +417,13 @@ __device__ __forceinline__ void prep_worker(
                 make_float2(__expf(G_last - Ga) * rk2.x, __expf(G_last - Gb) * rk2.y);
             if (lane == 0) rg[RG_GAMMA] = __expf(G_last);
         }
-        const bool ok = mbar_wait_bounded(bar, mphase, kWaitCycles);
+        const bool ok = mbar_wait_bounded(bar, mphase, wait_cycles);
         mphase ^= 1u;
         if (!ok) failed = true;
         if (named_bar_any(bar_id, kPrepThreads, failed)) { failed = true; break; }
         tc_fence_after();
         float x[32];  // this thread's half row of [K; Q] K^T, shared by the r V heads
         tmem_ld32_sync(tl + 32 * hh, x);
-        if (gram && trow < 64) {  // Gram row trow, columns 32 hh .. + 31 -> bf16 image
-            float gv[32];
-            tmem_ld32_sync(tl + 64 + 32 * hh, gv);
-            uint8_t* G = gram + ((size_t)cg * H_qk + j) * kGramBytes;
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                uint4 w;
-                w.x = pack_bf16x2(gv[8 * q4 + 0], gv[8 * q4 + 1]);
-                w.y = pack_bf16x2(gv[8 * q4 + 2], gv[8 * q4 + 3]);
-                w.z = pack_bf16x2(gv[8 * q4 + 4], gv[8 * q4 + 5]);
-                w.w = pack_bf16x2(gv[8 * q4 + 6], gv[8 * q4 + 7]);
-                *reinterpret_cast<uint4*>(G + sw128_off((uint32_t)trow, 4 * hh + q4)) = w;
-            }
-        }
 
 #pragma unroll 1
         for (int hr = 0; hr < r; ++hr) {
@@ -628,12 +591,12 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
     const float* __restrict__ b, const float* __restrict__ A_log,
     const float* __restrict__ dt_bias, const int32_t* __restrict__ cu_seqlens,
     const int32_t* __restrict__ choff, int32_t N, int H_qk, int H_v, float scale,
-    uint8_t* __restrict__ rec, int* status) {
+    uint8_t* __restrict__ rec, int* status, long long wait_cycles) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    prep_worker(q, k, a, b, A_log, dt_bias, cu_seqlens, choff, N, H_qk, H_v, scale, rec, nullptr,
-                status, nullptr, 0, sm, threadIdx.x, 1, blockIdx.x, gridDim.x, true);
+    prep_worker(q, k, a, b, A_log, dt_bias, cu_seqlens, choff, N, H_qk, H_v, scale, rec, status,
+                nullptr, 0, sm, threadIdx.x, 1, blockIdx.x, gridDim.x, true, wait_cycles);
 }
 
 // ==================================== chain =======================================
@@ -642,11 +605,6 @@ constexpr int kChain = 256;
 constexpr int kOut = 128;
 constexpr int kIssueWarp = 8;
 constexpr int kRdyBar = 6;     // named barrier: state threads arrive, the issuing warp waits
-// The Gram-matrix schedule gives each of its three steps its own barrier (6, 7, 8): its
-// state warps may arrive for step 2 before the issuing warp has passed step 1 (nothing
-// between the two waits for the issuing warp), and a barrier must not be arrived at
-// twice before it completes.
-constexpr int kRdyBarZ = 6, kRdyBarS = 7, kRdyBarV = 8;
 constexpr int kRdyCount = 288;
 constexpr int kLoadWarp = 9;
 constexpr int kRing = 3;
@@ -663,10 +621,6 @@ constexpr uint32_t CS_ERR = CS_BAR + 132;
 constexpr uint32_t CS_EGQ = CS_BAR + 256;           // [64] fp32: the chunk's output row factors
 constexpr size_t kChainSmem = CS_EGQ + 256 + 1024;
 
-// Slot of the Gram-matrix schedule (half rows): the block's half of V at SLOT_V, the
-// chunk's Gram tile in the other half's place.
-constexpr uint32_t SLOT_GRAM = SLOT_V + 8192;
-
 // tensor memory columns (512 allocated)
 constexpr uint32_t TM_U = 0;      // 128: the chunk's state increment (scaled Vn^T) K, fp32
 constexpr uint32_t TM_S0B = 128;  // 64: state as bf16 pairs
@@ -677,14 +631,6 @@ constexpr uint32_t TM_D3 = 320;   // 64: Vn^T; Vn^T pairs overwrite columns 0-15
 constexpr uint32_t TM_D1Q1 = 384; // 64: S0 Q^T of odd chunks
 constexpr uint32_t TM_D4 = 448;   // 64: Vn^T P^T
 constexpr uint32_t kTmemCols = 512;
-// ... and of the Gram-matrix schedule: U 0-127 as above, then
-constexpr uint32_t TG_S0B = 128;  // 64: S_c as bf16 pairs (A operand of S_c Q_c^T)
-constexpr uint32_t TG_GS = 192;   // 64: e^{G_L} S_c as bf16 pairs (of S_c K_{c+1}^T)
-constexpr uint32_t TG_R = 256;    // 64: S_c K_c^T; Z^T pairs overwrite columns 0-15, 32-47
-constexpr uint32_t TG_D3 = 320;   // 64: Vn^T; Vn^T pairs overwrite columns 0-15, 32-47 and
-                                  //     the decay-scaled pairs columns 16-31, 48-63
-constexpr uint32_t TG_D1Q = 384;  // 64: S_c Q_c^T (one accumulator)
-constexpr uint32_t TG_D4 = 448;   // 64: Vn^T P^T
 
 // Column (in 32-bit words) of the K=16 slice ks of a 64-token bf16 operand that
 // two warps wrote in place over the fp32 columns they had read: tokens 0-31 at
@@ -733,25 +679,22 @@ __device__ __forceinline__ bool wait_record(const unsigned long long* flag,
 // threads of a block (tid 0 .. 415, synchronised by the named barrier sync_id) on
 // the tensor memory `tmem` (512 columns). With `flags`, a chunk's record is
 // copied only once a prep worker has published it.
-template <int kM, bool kGram>
+template <int kM>
 __device__ __forceinline__ void chain_unit(
     const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
     const CUtensorMap& tm_o, const float* S0g, const int32_t* __restrict__ cu_seqlens,
     const int32_t* __restrict__ choff, int64_t T_total, int H_qk, int H_v,
-    const uint8_t* __restrict__ rec, const uint8_t* __restrict__ gram, bf16* __restrict__ o,
+    const uint8_t* __restrict__ rec, bf16* __restrict__ o,
     float* Sfg, const StateIndex sref, int* status,
     const unsigned long long* flags, unsigned long long epoch, uint8_t* sm, const int tid,
     const int n, const int h, const int hv, const uint32_t tmem,
-    const int sync_id) {
+    const int sync_id, const long long wait_cycles) {
     static_assert(kM == 128 || kM == 64, "a chain block owns all 128 value rows or one half");
-    static_assert(!kGram || kM == 64, "the Gram-matrix schedule runs on half rows");
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + CS_BAR);  // [3] slot landed
     uint64_t* mbar = full + kRing;         // chain MMA completions
     uint64_t* obar = mbar + 1;             // [2] chunk parity b: output accumulators complete
     uint64_t* ofree = mbar + 3;            // [2] chunk parity b: output accumulators read
     uint64_t* dbar = mbar + 5;             // drain of in-flight MMAs before the exit
-    uint64_t* kbar = mbar + 6;             // Gram schedule: S_c K_c^T complete (mbar: Vn^T)
-    uint64_t* ubar = mbar + 7;             // Gram schedule: the state increment complete
     volatile int* s_err = reinterpret_cast<volatile int*>(sm + CS_ERR);
 
     const int warp = tid >> 5, lane = tid & 31;
@@ -770,8 +713,6 @@ __device__ __forceinline__ void chain_unit(
         mbar_init(&ofree[0], 4);
         mbar_init(&ofree[1], 4);
         mbar_init(dbar, 1);
-        mbar_init(kbar, 1);
-        mbar_init(ubar, 1);
         *s_err = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -797,18 +738,14 @@ __device__ __forceinline__ void chain_unit(
         tma_load_3d(slot + SLOT_KQ + 16384, &tm_k, 64, j, t0, &full[st]);
         tma_load_3d(slot + SLOT_KQ + 8192, &tm_q, 0, j, t0, &full[st]);
         tma_load_3d(slot + SLOT_KQ + 16384 + 8192, &tm_q, 64, j, t0, &full[st]);
-        if constexpr (kGram) {
-            tma_load_3d(slot + SLOT_V, &tm_v, 64 * hv, h, t0, &full[st]);
-        } else {
-            tma_load_3d(slot + SLOT_V, &tm_v, 0, h, t0, &full[st]);
-            tma_load_3d(slot + SLOT_V + 8192, &tm_v, 64, h, t0, &full[st]);
-        }
+        tma_load_3d(slot + SLOT_V, &tm_v, 0, h, t0, &full[st]);
+        tma_load_3d(slot + SLOT_V + 8192, &tm_v, 64, h, t0, &full[st]);
     };
     // After a wait that ran out the record is copied all the same (valid memory, the
     // results are discarded), so that the slot's barrier completes and no copy is left
     // in flight when the block exits.
     auto record_ready = [&](int c) -> bool {
-        if (flags && !wait_record(flags + (size_t)(cg0 + c) * H_v + h, epoch, kWaitCycles)) {
+        if (flags && !wait_record(flags + (size_t)(cg0 + c) * H_v + h, epoch, wait_cycles)) {
             *s_err = 1;
             return false;
         }
@@ -819,9 +756,6 @@ __device__ __forceinline__ void chain_unit(
         if (flags) asm volatile("fence.proxy.async.global;" ::: "memory");  // read by TMA
         bulk_g2s(sm + st * kSlotBytes + SLOT_REC, rec + ((size_t)(cg0 + c) * H_v + h) * kRecBytes,
                  kRecBytes, &full[st]);
-        if constexpr (kGram)  // written before the record was published
-            bulk_g2s(sm + st * kSlotBytes + SLOT_GRAM,
-                     gram + ((size_t)(cg0 + c) * H_qk + j) * kGramBytes, kGramBytes, &full[st]);
     };
 
     if (warp > kIssueWarp) {
@@ -849,7 +783,7 @@ __device__ __forceinline__ void chain_unit(
             const int cn = cp + kRing;  // the chunk that will reuse this chunk's slot
             // its record's flag is checked while this chunk's MMAs still run
             const bool next = loader && cn < nchunks && issued == cn;
-            const bool ok = mbar_wait_bounded(&obar[b], (cp >> 1) & 1, kWaitCycles);
+            const bool ok = mbar_wait_bounded(&obar[b], (cp >> 1) & 1, wait_cycles);
             if (!ok) *s_err = 1;
             if (loader) bulk_wait_group_read<0>();  // staging free again
             // the slot's only remaining reader is this copy of the row factors
@@ -859,7 +793,7 @@ __device__ __forceinline__ void chain_unit(
             if (named_bar_any(2, kOut, !ok || *s_err != 0)) break;
             tc_fence_after();
             const float4* eg4 = reinterpret_cast<const float4*>(egq);
-            const uint32_t qacc = ctl + (kGram ? TG_D1Q : b ? TM_D1Q1 : TM_D1Q0);
+            const uint32_t qacc = ctl + (b ? TM_D1Q1 : TM_D1Q0);
             if constexpr (kM == 128) {
                 // this thread's column of the staged tile; laundered so that the 64 element
                 // addresses are formed per chunk rather than held in registers across chunks
@@ -957,7 +891,7 @@ __device__ __forceinline__ void chain_unit(
             // Leave nothing in flight into shared memory (loads the chain did not
             // consume are only possible after an error).
             for (int c = issued - 1; c >= 0 && c >= issued - kRing; --c)
-                if (!mbar_wait_bounded(&full[c % kRing], (c / kRing) & 1, kWaitCycles))
+                if (!mbar_wait_bounded(&full[c % kRing], (c / kRing) & 1, wait_cycles))
                     *s_err = 1;
         }
         __syncwarp();
@@ -987,187 +921,72 @@ __device__ __forceinline__ void chain_unit(
             dead = __any_sync(0xffffffffu, dead || !ok || *s_err != 0);
             if (dead) *s_err = 1;
         };
-        if constexpr (kGram) {
-            // Per chunk c: (1) Z_c written -> Vn_c += Z_c (T diag(beta))^T; (2) S_c and
-            // e^{G_L} S_c written -> chunk c+1's S_{c+1} K_{c+1}^T begins as
-            // e^{G_L} S_c K_{c+1}^T; (3) the Vn_c and decay-scaled pairs W_c written ->
-            // S_{c+1} K_{c+1}^T += W_c (K_c K_{c+1}^T) (the Gram tile; it completes the
-            // product, since S_{c+1} = e^{G_L} S_c + W_c K_c), the increment W_c K_c,
-            // S_c Q_c^T, Vn_c P_c^T, and chunk c+1's V^T (T diag(beta))^T. MMAs run in issue
-            // order, so an accumulator is overwritten only after the MMAs that read it before.
-            uint32_t aS0[4], aS1[4], aG0[4], aG1[4], aZ[4], aW[4], aN[4];
+#pragma unroll 1
+        for (int c = 0; c < nchunks; ++c) {
+            const int st = c % kRing;
+            uint8_t* slot = sm + st * kSlotBytes;
+            const uint32_t kq = smem_u32(slot + SLOT_KQ);
+            const uint32_t vt = smem_u32(slot + SLOT_V);
+            const uint32_t tt = smem_u32(slot + SLOT_REC + REC_T);
+            const uint32_t ptile = smem_u32(slot + SLOT_REC + REC_P);
+            // shared-memory descriptors of this chunk's operands, formed while waiting
+            uint64_t dK0[4], dK1[4], dQ0[4], dQ1[4], dV[4], dT[4], dKm[4], dP[4];
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
-                aS0[ks] = tmem + TG_S0B + 8 * ks;
-                aS1[ks] = tmem + TG_S0B + 8 * (ks + 4);
-                aG0[ks] = tmem + TG_GS + 8 * ks;
-                aG1[ks] = tmem + TG_GS + 8 * (ks + 4);
-                aZ[ks] = tmem + TG_R + split_pairs_col(ks);
-                aN[ks] = tmem + TG_D3 + split_pairs_col(ks);
-                aW[ks] = tmem + TG_D3 + 16 + split_pairs_col(ks);
+                dK0[ks] = smem_desc_sw128(kq + ks * 32u, 16, 1024);
+                dK1[ks] = smem_desc_sw128(kq + 16384u + ks * 32u, 16, 1024);
+                dQ0[ks] = smem_desc_sw128(kq + 8192u + ks * 32u, 16, 1024);
+                dQ1[ks] = smem_desc_sw128(kq + 16384u + 8192u + ks * 32u, 16, 1024);
+                // V^T rows = value rows: this block's half of them when kM = 64
+                dV[ks] = smem_desc_sw128(vt + (kM == 64 ? 8192u * hv : 0u) + ks * 2048u, 8192, 1024);
+                dT[ks] = smem_desc_sw128(tt + ks * 32u, 16, 1024);
+                dKm[ks] = smem_desc_sw128(kq + ks * 2048u, 16384, 1024);
+                dP[ks] = smem_desc_sw128(ptile + ks * 32u, 16, 1024);
             }
-            // S K^T of the chunk in slot st (K rows as B, K-major), then its V^T
-            // (T diag(beta))^T
-            auto issue_sk = [&](int st) {
-                const uint32_t kq = smem_u32(sm + st * kSlotBytes + SLOT_KQ);
-                uint64_t d0[4], d1[4];
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    d0[ks] = smem_desc_sw128(kq + ks * 32u, 16, 1024);
-                    d1[ks] = smem_desc_sw128(kq + 16384u + ks * 32u, 16, 1024);
-                }
-                mma_ts_group4(tmem + TG_R, aG0, d0, id64, 0);
-                mma_ts_group4(tmem + TG_R, aG1, d1, id64, 1);
-            };
-            auto issue_vpart = [&](int st) {
-                uint8_t* slot = sm + st * kSlotBytes;
-                const uint32_t vt = smem_u32(slot + SLOT_V);
-                const uint32_t tt = smem_u32(slot + SLOT_REC + REC_T);
-                uint64_t dV[4], dT[4];
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    dV[ks] = smem_desc_sw128(vt + ks * 2048u, 8192, 1024);
-                    dT[ks] = smem_desc_sw128(tt + ks * 32u, 16, 1024);
-                }
-                mma_ss_group4(tmem + TG_D3, dV, dT, id_v, 0);
-            };
-            // chunk 0: S_0 K_0^T from the initial state (written to TG_GS by the state warps)
-            if (nchunks > 0) {
-                if (!dead) check(mbar_wait_bounded(&full[0], 0, kWaitCycles));
-                wait_rdy(kRdyBarZ);
-                check(true);
-                if (!dead) {
-                    issue_sk(0);
-                    mma_commit_warp(kbar);
-                    issue_vpart(0);
-                }
+            if (!dead) check(mbar_wait_bounded(&full[st], (c / kRing) & 1, wait_cycles));
+            // (1) the bf16 state is written: S0 K^T, then V^T (T diag(beta))^T
+            wait_rdy();
+            check(true);
+            if (!dead) {
+                mma_ts_group4(tmem + TM_D1K, aS0, dK0, id64, 0);
+                mma_ts_group4(tmem + TM_D1K, aS1, dK1, id64, 1);
+                mma_commit_warp(mbar);
+                mma_ss_group4(tmem + TM_D3, dV, dT, id_v, 0);
             }
-#pragma unroll 1
-            for (int c = 0; c < nchunks; ++c) {
-                const int st = c % kRing;
-                const int sn = (c + 1) % kRing;
-                const bool more = c + 1 < nchunks;
-                uint8_t* slot = sm + st * kSlotBytes;
-                const uint32_t kq = smem_u32(slot + SLOT_KQ);
-                const uint32_t tt = smem_u32(slot + SLOT_REC + REC_T);
-                const uint32_t ptile = smem_u32(slot + SLOT_REC + REC_P);
-                const uint32_t gt = smem_u32(sm + sn * kSlotBytes + SLOT_GRAM);
-                uint64_t dQ0[4], dQ1[4], dT[4], dKm[4], dP[4], dG[4];
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    dQ0[ks] = smem_desc_sw128(kq + 8192u + ks * 32u, 16, 1024);
-                    dQ1[ks] = smem_desc_sw128(kq + 16384u + 8192u + ks * 32u, 16, 1024);
-                    dT[ks] = smem_desc_sw128(tt + ks * 32u, 16, 1024);
-                    dKm[ks] = smem_desc_sw128(kq + ks * 2048u, 16384, 1024);
-                    dP[ks] = smem_desc_sw128(ptile + ks * 32u, 16, 1024);
-                    dG[ks] = smem_desc_sw128(gt + ks * 32u, 16, 1024);
-                }
-                // (1) Z_c
-                wait_rdy(kRdyBarZ);
-                check(true);
-                if (!dead) {
-                    mma_ts_group4(tmem + TG_D3, aZ, dT, id64, 1);
-                    mma_commit_warp(mbar);
-                }
-                // (2) S_c, e^{G_L} S_c: chunk c+1's S K^T begins
-                wait_rdy(kRdyBarS);
-                check(true);
-                if (!dead && more)
-                    check(mbar_wait_bounded(&full[sn], ((c + 1) / kRing) & 1, kWaitCycles));
-                if (!dead && more) issue_sk(sn);
-                // (3) Vn_c pairs and W_c pairs. The path to the next chunk goes first; S_c Q_c^T
-                // waits until the output accumulators were read for chunk c - 1, and the
-                // increment's commit follows it (the state warps rewrite S_c's pairs only
-                // after that commit).
-                wait_rdy(kRdyBarV);
-                check(true);
-                if (!dead) {
-                    if (more) {
-                        mma_ts_group4(tmem + TG_R, aW, dG, id64, 1);
-                        mma_commit_warp(kbar);
-                    }
-                    mma_ts_group4(tmem + TM_U, aW, dKm, id_s, 0);
-                    if (c >= 1)
-                        check(mbar_wait_bounded(&ofree[(c - 1) & 1], ((c - 1) >> 1) & 1,
-                                                kWaitCycles));
-                }
-                if (!dead) {
-                    mma_ts_group4(tmem + TG_D1Q, aS0, dQ0, id64, 0);
-                    mma_ts_group4(tmem + TG_D1Q, aS1, dQ1, id64, 1);
-                    mma_commit_warp(ubar);
-                    mma_ts_group4(tmem + TG_D4, aN, dP, id64, 0);
-                    mma_commit_warp(&obar[c & 1]);
-                    if (more) issue_vpart(sn);
-                }
+            // (2) Z^T is written: Vn^T += Z^T (T diag(beta))^T; then S0 Q^T into the
+            // accumulator of parity c & 1, last read for chunk c - 2
+            wait_rdy();
+            check(true);
+            if (!dead) {
+                mma_ts_group4(tmem + TM_D3, aZ, dT, id64, 1);
+                mma_commit_warp(mbar);
+                if (c >= 2)
+                    check(mbar_wait_bounded(&ofree[c & 1], ((c - 2) >> 1) & 1, wait_cycles));
             }
-        } else {
-    #pragma unroll 1
-            for (int c = 0; c < nchunks; ++c) {
-                const int st = c % kRing;
-                uint8_t* slot = sm + st * kSlotBytes;
-                const uint32_t kq = smem_u32(slot + SLOT_KQ);
-                const uint32_t vt = smem_u32(slot + SLOT_V);
-                const uint32_t tt = smem_u32(slot + SLOT_REC + REC_T);
-                const uint32_t ptile = smem_u32(slot + SLOT_REC + REC_P);
-                // shared-memory descriptors of this chunk's operands, formed while waiting
-                uint64_t dK0[4], dK1[4], dQ0[4], dQ1[4], dV[4], dT[4], dKm[4], dP[4];
-    #pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    dK0[ks] = smem_desc_sw128(kq + ks * 32u, 16, 1024);
-                    dK1[ks] = smem_desc_sw128(kq + 16384u + ks * 32u, 16, 1024);
-                    dQ0[ks] = smem_desc_sw128(kq + 8192u + ks * 32u, 16, 1024);
-                    dQ1[ks] = smem_desc_sw128(kq + 16384u + 8192u + ks * 32u, 16, 1024);
-                    // V^T rows = value rows: this block's half of them when kM = 64
-                    dV[ks] = smem_desc_sw128(vt + (kM == 64 ? 8192u * hv : 0u) + ks * 2048u, 8192, 1024);
-                    dT[ks] = smem_desc_sw128(tt + ks * 32u, 16, 1024);
-                    dKm[ks] = smem_desc_sw128(kq + ks * 2048u, 16384, 1024);
-                    dP[ks] = smem_desc_sw128(ptile + ks * 32u, 16, 1024);
-                }
-                if (!dead) check(mbar_wait_bounded(&full[st], (c / kRing) & 1, kWaitCycles));
-                // (1) the bf16 state is written: S0 K^T, then V^T (T diag(beta))^T
-                wait_rdy();
-                check(true);
-                if (!dead) {
-                    mma_ts_group4(tmem + TM_D1K, aS0, dK0, id64, 0);
-                    mma_ts_group4(tmem + TM_D1K, aS1, dK1, id64, 1);
-                    mma_commit_warp(mbar);
-                    mma_ss_group4(tmem + TM_D3, dV, dT, id_v, 0);
-                }
-                // (2) Z^T is written: Vn^T += Z^T (T diag(beta))^T; then S0 Q^T into the
-                // accumulator of parity c & 1, last read for chunk c - 2
-                wait_rdy();
-                check(true);
-                if (!dead) {
-                    mma_ts_group4(tmem + TM_D3, aZ, dT, id64, 1);
-                    mma_commit_warp(mbar);
-                    if (c >= 2)
-                        check(mbar_wait_bounded(&ofree[c & 1], ((c - 2) >> 1) & 1, kWaitCycles));
-                }
-                if (!dead) {
-                    const uint32_t qacc = tmem + ((c & 1) ? TM_D1Q1 : TM_D1Q0);
-                    mma_ts_group4(qacc, aS0, dQ0, id64, 0);
-                    mma_ts_group4(qacc, aS1, dQ1, id64, 1);
-                }
-                // (3) the Vn^T pairs are written: the state increment, then Vn^T P^T
-                wait_rdy();
-                check(true);
-                if (!dead) {
-                    mma_ts_group4(tmem + TM_U, aU, dKm, id_s, 0);
-                    mma_commit_warp(mbar);
-                    if (c >= 1)
-                        check(mbar_wait_bounded(&ofree[(c - 1) & 1], ((c - 1) >> 1) & 1,
-                                                kWaitCycles));
-                }
-                if (!dead) {
-                    mma_ts_group4(tmem + TM_D4, aN, dP, id64, 0);
-                    mma_commit_warp(&obar[c & 1]);
-                }
+            if (!dead) {
+                const uint32_t qacc = tmem + ((c & 1) ? TM_D1Q1 : TM_D1Q0);
+                mma_ts_group4(qacc, aS0, dQ0, id64, 0);
+                mma_ts_group4(qacc, aS1, dQ1, id64, 1);
+            }
+            // (3) the Vn^T pairs are written: the state increment, then Vn^T P^T
+            wait_rdy();
+            check(true);
+            if (!dead) {
+                mma_ts_group4(tmem + TM_U, aU, dKm, id_s, 0);
+                mma_commit_warp(mbar);
+                if (c >= 1)
+                    check(mbar_wait_bounded(&ofree[(c - 1) & 1], ((c - 1) >> 1) & 1,
+                                            wait_cycles));
+            }
+            if (!dead) {
+                mma_ts_group4(tmem + TM_D4, aN, dP, id64, 0);
+                mma_commit_warp(&obar[c & 1]);
             }
         }
         __syncwarp();
         // no MMA may still run when the tensor memory is freed
         mma_commit_warp(dbar);
-        (void)mbar_wait_bounded(dbar, 0, kWaitCycles);
+        (void)mbar_wait_bounded(dbar, 0, wait_cycles);
         if (*s_err) {  // wake the output warps so they see the error and leave
             if (lane == 0) {
                 mbar_arrive(&obar[0]);
@@ -1204,7 +1023,7 @@ __device__ __forceinline__ void chain_unit(
             bool dead = false;  // warp-uniform: after an error only the barrier arrivals remain
             auto wait_mma = [&]() {
                 if (dead) return;
-                bool ok = *s_err == 0 && mbar_wait_bounded(mbar, mphase, kWaitCycles);
+                bool ok = *s_err == 0 && mbar_wait_bounded(mbar, mphase, wait_cycles);
                 mphase ^= 1u;
                 dead = __any_sync(0xffffffffu, !ok || *s_err != 0);
                 if (dead) *s_err = 1;
@@ -1247,7 +1066,7 @@ __device__ __forceinline__ void chain_unit(
                 }
                 if (!dead) {
                     const bool okf =
-                        *s_err == 0 && mbar_wait_bounded(&full[st], (c / kRing) & 1, kWaitCycles);
+                        *s_err == 0 && mbar_wait_bounded(&full[st], (c / kRing) & 1, wait_cycles);
                     dead = __any_sync(0xffffffffu, !okf || *s_err != 0);
                     if (dead) *s_err = 1;
                 }
@@ -1336,7 +1155,7 @@ __device__ __forceinline__ void chain_unit(
                 for (int e = 0; e < 16; ++e)
                     d4[e] = make_float4(S[4 * e], S[4 * e + 1], S[4 * e + 2], S[4 * e + 3]);
             }
-        } else if constexpr (!kGram) {
+        } else {
             // ======================= state, one half of the value rows =======================
             // The block's 64 value rows 64 hv .. 64 hv + 63 sit in TMEM lanes 0-15 of each lane
             // quarter (M = 64 layout): warp w takes quarter qd = w & 3 (rows 16 qd ..) and the
@@ -1371,7 +1190,7 @@ __device__ __forceinline__ void chain_unit(
             bool dead = false;  // warp-uniform: after an error only the barrier arrivals remain
             auto wait_mma = [&]() {
                 if (dead) return;
-                bool ok = *s_err == 0 && mbar_wait_bounded(mbar, mphase, kWaitCycles);
+                bool ok = *s_err == 0 && mbar_wait_bounded(mbar, mphase, wait_cycles);
                 mphase ^= 1u;
                 dead = __any_sync(0xffffffffu, !ok || *s_err != 0);
                 if (dead) *s_err = 1;
@@ -1408,7 +1227,7 @@ __device__ __forceinline__ void chain_unit(
                 }
                 if (!dead) {
                     const bool okf =
-                        *s_err == 0 && mbar_wait_bounded(&full[st], (c / kRing) & 1, kWaitCycles);
+                        *s_err == 0 && mbar_wait_bounded(&full[st], (c / kRing) & 1, wait_cycles);
                     dead = __any_sync(0xffffffffu, !okf || *s_err != 0);
                     if (dead) *s_err = 1;
                 }
@@ -1491,173 +1310,6 @@ __device__ __forceinline__ void chain_unit(
                         make_float2(S[4 * jj + 2], S[4 * jj + 3]);
                 }
             }
-        } else {
-            // ============ state, one half of the value rows, Gram-matrix schedule ============
-            // Layout as in the half-row schedule above (rows r0, r0 + 8; column pairs cp2).
-            // Per chunk c: (A) S_c K_c^T complete -> Z_c; (B) S_c = e^{G_L} S_{c-1} + U_{c-1},
-            // then S_c and e^{G_L} S_c as bf16 pairs; (C) Vn_c complete -> Vn_c pairs and the
-            // decay-scaled pairs. Only (A) and (C) are on the path from chunk to chunk.
-            const int qd = warp & 3;
-            const int hh = warp >> 2;
-            const int r0 = 64 * hv + qd * 16 + (lane >> 2);
-            const int cp2 = 2 * (lane & 3);
-            const uint32_t ctl = tmem + ((uint32_t)(qd * 32) << 16);
-            bool rd, wr;
-            const int sidx = sref.resolve(n, rd, wr, tid == 0 ? status : nullptr);
-            const float* S0s = rd ? S0g : nullptr;
-            float* Sfs = wr ? Sfg : nullptr;
-            const size_t hbase = ((size_t)sidx * H_v + h) * kD * kD;
-            float S[32];  // S[4 j + e]: row r0 + 8 (e >> 1), column 64 hh + 8 j + cp2 + (e & 1)
-            if (S0s) {
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
-                    const int col = 64 * hh + 8 * jj + cp2;
-                    const float2 f0 = *reinterpret_cast<const float2*>(S0s + hbase + (size_t)r0 * kD + col);
-                    const float2 f1 =
-                        *reinterpret_cast<const float2*>(S0s + hbase + (size_t)(r0 + 8) * kD + col);
-                    S[4 * jj] = f0.x; S[4 * jj + 1] = f0.y; S[4 * jj + 2] = f1.x; S[4 * jj + 3] = f1.y;
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < 32; ++e) S[e] = 0.f;
-            }
-
-            uint32_t kph = 0, uph = 0, vph = 0;
-            bool dead = false;  // warp-uniform: after an error only the barrier arrivals remain
-            auto wait_bar = [&](uint64_t* bar, uint32_t& ph) {
-                if (dead) return;
-                bool ok = *s_err == 0 && mbar_wait_bounded(bar, ph, kWaitCycles);
-                ph ^= 1u;
-                dead = __any_sync(0xffffffffu, !ok || *s_err != 0);
-                if (dead) *s_err = 1;
-                tc_fence_after();
-            };
-            auto wait_full = [&](int c) {  // chunk c's slot landed (its record is read here)
-                if (dead) return;
-                const bool okf =
-                    *s_err == 0 && mbar_wait_bounded(&full[c % kRing], (c / kRing) & 1, kWaitCycles);
-                dead = __any_sync(0xffffffffu, !okf || *s_err != 0);
-                if (dead) *s_err = 1;
-            };
-            auto signal_rdy = [&](int id) {
-                if (!dead) tmem_wait_st();
-                tc_fence_before();
-                if (dead) named_bar_sync(id, kRdyCount);
-                else named_bar_arrive(id, kRdyCount);
-            };
-            // A sequence's last chunk: rows past its end (the next sequence's tokens, or TMA
-            // zero fill) in chunk c's K, Q and V tiles are zeroed before any MMA reads them.
-            auto zero_tail = [&](int c) {
-                const int L = (int)min((int64_t)kC, s1 - (s0 + (int64_t)c * kC));
-                if (L >= kC) return;
-                wait_full(c);
-                if (dead) return;
-                uint8_t* slot = sm + (c % kRing) * kSlotBytes;
-                const int nz = (kC - L) * 8;  // 16-byte chunks per 64-column tile
-                for (int idx = tid; idx < 5 * nz; idx += kChain) {
-                    const int tile = idx / nz, r = L + (idx % nz) / 8, ch = idx & 7;
-                    const uint32_t base =
-                        tile < 4 ? SLOT_KQ + (tile >> 1) * 16384u + (tile & 1) * 8192u : SLOT_V;
-                    *reinterpret_cast<uint4*>(slot + base + r * 128 + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
-                }
-                fence_proxy_async_smem();
-            };
-            // bf16 pairs of scale * S (key k at column k / 2 of this block's rows)
-            auto pack_state = [&](uint32_t col, float scale) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
-                    pk[2 * jj] = pack_bf16x2(scale * S[4 * jj], scale * S[4 * jj + 1]);
-                    pk[2 * jj + 1] = pack_bf16x2(scale * S[4 * jj + 2], scale * S[4 * jj + 3]);
-                }
-                tmem_st16r_x8(ctl + col + 32 * hh, pk);
-            };
-            auto apply_update = [&](float gamma) {
-                float u[32];
-                tmem_ld16r_x8_sync(ctl + TM_U + 64 * hh, u);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) S[e] = fmaf(gamma, S[e], u[e]);
-            };
-
-            // chunk 0's S K^T reads the initial state
-            if (nchunks > 0) {
-                if (!dead) {
-                    zero_tail(0);
-                    if (!dead) pack_state(TG_GS, 1.f);
-                }
-                signal_rdy(kRdyBarZ);
-            }
-            float gamma = 1.f;  // e^{G_L} of the chunk before
-#pragma unroll 1
-            for (int c = 0; c < nchunks; ++c) {
-                const float* rg =
-                    reinterpret_cast<const float*>(sm + (c % kRing) * kSlotBytes + SLOT_REC + REC_G);
-                const bool more = c + 1 < nchunks;
-                // ---- (A) Z^T = -(e^G rk) (S_c K_c^T), tokens 32 hh + 8 j + cp2, + 1 --------
-                wait_bar(kbar, kph);
-                wait_full(c);
-                if (!dead) {
-                    float x[16];
-                    tmem_ld16r_x4_sync(ctl + TG_R + 32 * hh, x);
-                    uint32_t pk[8];
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        const float2 f = *reinterpret_cast<const float2*>(rg + RG_FK + 32 * hh + 8 * jj + cp2);
-                        pk[2 * jj] = pack_bf16x2(-f.x * x[4 * jj], -f.y * x[4 * jj + 1]);
-                        pk[2 * jj + 1] = pack_bf16x2(-f.x * x[4 * jj + 2], -f.y * x[4 * jj + 3]);
-                    }
-                    tmem_st16r_x4(ctl + TG_R + 32 * hh, pk);
-                }
-                signal_rdy(kRdyBarZ);
-                // ---- (B) the state of this chunk, its bf16 copies --------------------------
-                if (c > 0) {
-                    wait_bar(ubar, uph);
-                    if (!dead) apply_update(gamma);
-                }
-                if (!dead) {
-                    gamma = rg[RG_GAMMA];
-                    if (more) zero_tail(c + 1);
-                }
-                if (!dead) {
-                    pack_state(TG_S0B, 1.f);
-                    if (more) pack_state(TG_GS, gamma);
-                }
-                signal_rdy(kRdyBarS);
-                // ---- (C) Vn^T -> bf16 pairs (for P Vn) and decay-scaled pairs ---------------
-                wait_bar(mbar, vph);
-                if (!dead) {
-                    float x[16];
-                    tmem_ld16r_x4_sync(ctl + TG_D3 + 32 * hh, x);
-                    uint32_t pk[8], pw[8];
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        const float2 w = *reinterpret_cast<const float2*>(rg + RG_EGL + 32 * hh + 8 * jj + cp2);
-                        pk[2 * jj] = pack_bf16x2(x[4 * jj], x[4 * jj + 1]);
-                        pk[2 * jj + 1] = pack_bf16x2(x[4 * jj + 2], x[4 * jj + 3]);
-                        pw[2 * jj] = pack_bf16x2(x[4 * jj] * w.x, x[4 * jj + 1] * w.y);
-                        pw[2 * jj + 1] = pack_bf16x2(x[4 * jj + 2] * w.x, x[4 * jj + 3] * w.y);
-                    }
-                    tmem_st16r_x4(ctl + TG_D3 + 32 * hh, pk);
-                    tmem_st16r_x4(ctl + TG_D3 + 32 * hh + 16, pw);
-                }
-                signal_rdy(kRdyBarV);
-            }
-            bool done = !dead;
-            if (done && nchunks > 0) {  // the last chunk's state update
-                wait_bar(ubar, uph);
-                done = !dead;
-                if (done) apply_update(gamma);
-            }
-            if (done && Sfs) {
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
-                    const int col = 64 * hh + 8 * jj + cp2;
-                    *reinterpret_cast<float2*>(Sfs + hbase + (size_t)r0 * kD + col) =
-                        make_float2(S[4 * jj], S[4 * jj + 1]);
-                    *reinterpret_cast<float2*>(Sfs + hbase + (size_t)(r0 + 8) * kD + col) =
-                        make_float2(S[4 * jj + 2], S[4 * jj + 3]);
-                }
-            }
         }
     }
 
@@ -1673,7 +1325,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
     const float* S0g, const int32_t* __restrict__ cu_seqlens,
     const int32_t* __restrict__ choff, int64_t T_total, int H_qk, int H_v,
     const uint8_t* __restrict__ rec, bf16* __restrict__ o, float* Sfg, const StateIndex sref,
-    int* status) {
+    int* status, long long wait_cycles) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1687,9 +1339,9 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
-    chain_unit<128, false>(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v,
-                           rec, nullptr, o, Sfg, sref, status, nullptr, 0, sm, threadIdx.x,
-                           blockIdx.x / H_v, blockIdx.x % H_v, 0, tmem, 1);
+    chain_unit<128>(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v, rec, o,
+                    Sfg, sref, status, nullptr, 0, sm, threadIdx.x, blockIdx.x / H_v,
+                    blockIdx.x % H_v, 0, tmem, 1, wait_cycles);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1712,7 +1364,7 @@ constexpr size_t kFusedSmem =
 constexpr int kChainSync = 5;  // named barrier of the chain threads in the fused kernel
 constexpr int kFusedMaxSeqs = 255;  // the fused kernel computes the chunk offsets itself
 
-template <int kM, bool kGram>
+template <int kM>
 __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -1721,8 +1373,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
     const float* __restrict__ dt_bias, const float* S0g,
     const int32_t* __restrict__ cu_seqlens, const int32_t* choff, int32_t N,
     int64_t T_total, int H_qk, int H_v, float scale, uint8_t* __restrict__ rec,
-    uint8_t* __restrict__ gram, bf16* __restrict__ o, float* Sfg, const StateIndex sref,
-    int* status, unsigned long long* flags, unsigned long long epoch, int c0) {
+    bf16* __restrict__ o, float* Sfg, const StateIndex sref,
+    int* status, unsigned long long* flags, unsigned long long epoch, int c0,
+    long long wait_cycles, int withhold_records) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ int32_t s_choff[kFusedMaxSeqs + 1];
     __shared__ int s_bad;
@@ -1762,10 +1415,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
     choff = s_choff;
     if ((int)blockIdx.x >= c0) {
         const int sub = tid >> 8;
+        // a fault-injection call withholds every record: the chains' waits run out
         prep_worker(q, k, a, b, A_log, dt_bias, cu_seqlens, choff, N, H_qk, H_v, scale, rec,
-                    kGram ? gram : nullptr, status, flags, epoch, sm + sub * kPrepRegion,
+                    status, withhold_records ? nullptr : flags, epoch, sm + sub * kPrepRegion,
                     tid & 255, 3 + sub, 2 * ((int)blockIdx.x - c0) + sub,
-                    2 * ((int)gridDim.x - c0), false);
+                    2 * ((int)gridDim.x - c0), false, wait_cycles);
         return;
     }
     if (tid >= kChainThreads) return;
@@ -1781,9 +1435,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
     // block u: (sequence, V head) u, or with half-row blocks its half u & 1 of unit u >> 1
     const int u = kM == 64 ? (int)blockIdx.x >> 1 : (int)blockIdx.x;
     const int hv = kM == 64 ? (int)blockIdx.x & 1 : 0;
-    chain_unit<kM, kGram>(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v,
-                          rec, gram, o, Sfg, sref, status, flags, epoch, sm, tid, u / H_v,
-                          u % H_v, hv, tmem, kChainSync);
+    chain_unit<kM>(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v, rec, o,
+                   Sfg, sref, status, flags, epoch, sm, tid, u / H_v, u % H_v, hv, tmem,
+                   kChainSync, wait_cycles);
     tc_fence_before();
     named_bar_sync(kChainSync, kChainThreads);
     tc_fence_after();
@@ -1793,26 +1447,49 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct TcWorkspace {
-    size_t off_flags, off_rec, off_gram, total;
+    size_t off_flags, off_rec, total;
 };
 
 // Workspace: chunk offsets [N + 1] | record flags [records] (64-bit call numbers) |
-// records [chunks][H_v] | with the Gram-matrix schedule, Gram tiles [chunks][H_qk].
-TcWorkspace tc_workspace_layout(int32_t N, int64_t T, int32_t H_qk, int32_t H_v, bool gram) {
+// records [chunks][H_v].
+TcWorkspace tc_workspace_layout(int32_t N, int64_t T, int32_t H_v) {
     const size_t chunks = (size_t)((T + kC - 1) / kC) + (size_t)N;
     const size_t records = chunks * H_v;
     TcWorkspace w;
     w.off_flags = align256((size_t)(N + 1) * sizeof(int32_t));
     w.off_rec = w.off_flags + align256(records * sizeof(unsigned long long));
-    w.off_gram = w.off_rec + records * kRecBytes;
-    w.total = w.off_gram + (gram ? chunks * H_qk * kGramBytes : 0);
+    w.total = w.off_rec + records * kRecBytes;
     return w;
+}
+
+// The number a call publishes its records under. Flags hold the number of the call
+// that wrote them last, or whatever the workspace held before; a chain takes a record
+// as published only when its flag equals this call's number. The numbers are a random
+// 64-bit base drawn once per process (top bit set) plus a call counter, so no earlier
+// call of this process used this call's number, and stale contents of any other origin
+// (small integers, floats, another process's flags) match it only by chance, with
+// probability 2^-64 per flag.
+unsigned long long next_call_number() {
+    static const unsigned long long base = [] {
+        unsigned long long x = 0;
+        try {
+            std::random_device rd;
+            x = ((unsigned long long)rd() << 32) ^ (unsigned long long)rd();
+        } catch (...) {
+        }
+        x ^= (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count() *
+             0x9E3779B97F4A7C15ull;
+        x ^= (unsigned long long)getpid() * 0xC2B2AE3D27D4EB4Full;
+        return x | (1ull << 63);
+    }();
+    static std::atomic<unsigned long long> counter{0};
+    return base + counter.fetch_add(1) + 1;
 }
 
 }  // namespace
 
-size_t prefill_tc_workspace_bytes(int32_t N, int64_t T, int32_t H_qk, int32_t H_v, bool gram) {
-    return tc_workspace_layout(N, T, H_qk, H_v, gram).total;
+size_t prefill_tc_workspace_bytes(int32_t N, int64_t T, int32_t H_v) {
+    return tc_workspace_layout(N, T, H_v).total;
 }
 
 bool prefill_tc_supported(int32_t H_qk, int32_t H_v) { return H_v / H_qk <= kMaxGroup; }
@@ -1856,16 +1533,15 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
                               const float* b, const float* A_log, const float* dt_bias,
                               const float* S0, const int32_t* cu_seqlens, int32_t N, int64_t T,
                               int32_t H_qk, int32_t H_v, float scale, void* o, float* S_final,
-                              StateIndex sref, void* workspace, int schedule, int* status,
-                              cudaStream_t s) {
+                              StateIndex sref, void* workspace, const PrefillOpts& opt,
+                              int* status, cudaStream_t s) {
     if (N == 0) return cudaSuccess;
     if (T > (int64_t)0x7FFFFFFF - kC) return cudaErrorInvalidValue;  // TMA token coordinates
-    const TcWorkspace ws = tc_workspace_layout(N, T, H_qk, H_v, schedule == 3);
+    const TcWorkspace ws = tc_workspace_layout(N, T, H_v);
     uint8_t* wb = static_cast<uint8_t*>(workspace);
     int32_t* choff = reinterpret_cast<int32_t*>(wb);
     unsigned long long* flags = reinterpret_cast<unsigned long long*>(wb + ws.off_flags);
     uint8_t* rec = wb + ws.off_rec;
-    uint8_t* gram = wb + ws.off_gram;
     // With no tokens the maps are never read; any aligned device address will do.
     CUtensorMap tm_q, tm_k, tm_v, tm_o;
     if (!make_rows_map(&tm_q, T > 0 ? q : workspace, H_qk, T) ||
@@ -1881,18 +1557,18 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
     if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess) coop = 0;
     cudaError_t e;
     const int64_t chain_units = (int64_t)N * H_v;
+    long long wait_cycles = opt.wait_cycles;
+    const bool separate = opt.impl == GDN_IMPL_TENSOR_CORE_SPLIT;
+    const bool whole_rows = opt.impl == GDN_IMPL_TENSOR_CORE_WHOLE_ROWS;
 
-    if (schedule > 0 && coop) {
+    if (!separate && coop) {
         // Overlap pays when the chains are few (latency-bound: each holds one SM for
         // its whole sequence); with many chains the separate launches keep both
         // phases at full occupancy. With at most a quarter as many chains as SMs each
         // chain runs as two blocks of 64 value rows (half the per-thread state work on
         // the critical path).
-        const bool half = schedule >= 2 && 4 * chain_units <= num_sms;
-        const bool gram_sched = half && schedule == 3;
-        const void* kfn = gram_sched ? (const void*)fused_kernel<64, true>
-                          : half     ? (const void*)fused_kernel<64, false>
-                                     : (const void*)fused_kernel<128, false>;
+        const bool half = !whole_rows && 4 * chain_units <= num_sms;
+        const void* kfn = half ? (const void*)fused_kernel<64> : (const void*)fused_kernel<128>;
         e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kFusedSmem);
         if (e != cudaSuccess) return e;
@@ -1903,21 +1579,20 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
         const int grid = per_sm >= 1 ? num_sms : 0;
         const int64_t chain_blocks = (half ? 2 : 1) * chain_units;
         if (grid >= 2 && 2 * chain_blocks <= grid && N <= kFusedMaxSeqs) {
-            // this call's number: above every number an earlier call wrote
-            static std::atomic<unsigned long long> call_number{0};
-            unsigned long long epoch = call_number.fetch_add(1) + 1;
+            unsigned long long epoch = next_call_number();
             const bf16* qb = static_cast<const bf16*>(q);
             const bf16* kb = static_cast<const bf16*>(k);
             bf16* ob = static_cast<bf16*>(o);
             int c0v = (int)chain_blocks;
+            int withhold = opt.fault == GDN_FAULT_WITHHOLD_RECORDS ? 1 : 0;
             void* args[] = {&tm_q, &tm_k, &tm_v, &tm_o, &qb, &kb, &a, &b, &A_log, &dt_bias, &S0,
-                            &cu_seqlens, &choff, &N, &T, &H_qk, &H_v, &scale, &rec, &gram, &ob,
-                            &S_final, &sref, &status, &flags, &epoch, &c0v};
-            ktimer_before(s);
+                            &cu_seqlens, &choff, &N, &T, &H_qk, &H_v, &scale, &rec, &ob,
+                            &S_final, &sref, &status, &flags, &epoch, &c0v, &wait_cycles,
+                            &withhold};
+            timer_before(opt.timer, s);
             e = cudaLaunchCooperativeKernel(kfn, dim3(grid), dim3(kFusedThreads), args, kFusedSmem,
                                             s);
-            if (e == cudaSuccess)
-                ktimer_after(s, gram_sched ? "fused_half_rows_gram" : half ? "fused_half_rows" : "fused");
+            if (e == cudaSuccess) timer_after(opt.timer, s, half ? "fused_half_rows" : "fused");
             return e;
         }
     }
@@ -1928,29 +1603,29 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
     e = cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kChainSmem);
     if (e != cudaSuccess) return e;
-    ktimer_before(s);
+    timer_before(opt.timer, s);
     chunk_offsets_kernel<<<1, 256, 0, s>>>(cu_seqlens, N, T, choff, status);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    ktimer_after(s, "chunk_offsets");
+    timer_after(opt.timer, s, "chunk_offsets");
     const int64_t unit_bound = (((T + kC - 1) / kC) + N) * (int64_t)H_qk;
     const int64_t grid_cap = (int64_t)2 * num_sms;
     const int prep_grid = (int)(unit_bound < grid_cap ? unit_bound : grid_cap);
     if (prep_grid > 0) {
-        ktimer_before(s);
+        timer_before(opt.timer, s);
         prep_kernel<<<prep_grid, kPrepThreads, kPrepSmem, s>>>(
             static_cast<const bf16*>(q), static_cast<const bf16*>(k), a, b, A_log, dt_bias,
-            cu_seqlens, choff, N, H_qk, H_v, scale, rec, status);
+            cu_seqlens, choff, N, H_qk, H_v, scale, rec, status, wait_cycles);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
-        ktimer_after(s, "prep");
+        timer_after(opt.timer, s, "prep");
     }
-    ktimer_before(s);
+    timer_before(opt.timer, s);
     chain_kernel<<<(unsigned)chain_units, kChainThreads, kChainSmem, s>>>(
         tm_q, tm_k, tm_v, tm_o, S0, cu_seqlens, choff, T, H_qk, H_v, rec, static_cast<bf16*>(o),
-        S_final, sref, status);
+        S_final, sref, status, wait_cycles);
     e = cudaGetLastError();
-    if (e == cudaSuccess) ktimer_after(s, "chain");
+    if (e == cudaSuccess) timer_after(opt.timer, s, "chain");
     return e;
 }
 

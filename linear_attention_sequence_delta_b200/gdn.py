@@ -33,14 +33,21 @@ _STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "
 
 # Every symbol include/gdn.h declares (the tests check the library exports them all).
 EXPORTS = ["gdn_status_string", "gdn_version", "gdn_prefill_workspace_size", "gdn_gates",
-           "gdn_prefill", "gdn_decode_step", "gdn_sync_status", "gdn_prefill_noalloc",
-           "gdn_set_prefill_impl", "gdn_set_kernel_timing", "gdn_last_prefill_kernel_ms",
-           "gdn_last_prefill_kernel_name", "gdn_conv1d_silu", "gdn_conv1d_silu_decode",
+           "gdn_prefill", "gdn_prefill_ex", "gdn_decode_step", "gdn_sync_status",
+           "gdn_prefill_noalloc", "gdn_timer_create", "gdn_timer_destroy", "gdn_timer_read",
+           "gdn_timer_kernel_name", "gdn_conv1d_silu", "gdn_conv1d_silu_decode",
            "gdn_rmsnorm_gated", "gdn_decode_slots", "gdn_decode_step_bf16_state",
-           "gdn_prefill_slots"]
+           "gdn_prefill_slots", "gdn_prefill_slots_ex"]
 GDN_IMPL_AUTO, GDN_IMPL_CUDA_CORE, GDN_IMPL_TENSOR_CORE, GDN_IMPL_TENSOR_CORE_SPLIT = 0, 1, 2, 3
 GDN_IMPL_TENSOR_CORE_WHOLE_ROWS = 4
-GDN_IMPL_TENSOR_CORE_GRAM = 5
+GDN_FAULT_NONE, GDN_FAULT_WITHHOLD_RECORDS = 0, 1
+
+
+class PrefillOptions(ctypes.Structure):
+    """gdn_prefill_options of include/gdn.h (per-call implementation choice, fault
+    injection, wait limit, kernel timer)."""
+    _fields_ = [("impl", ctypes.c_int32), ("fault", ctypes.c_int32),
+                ("wait_limit_cycles", ctypes.c_int64), ("timer", ctypes.c_void_p)]
 
 
 class GDNError(RuntimeError):
@@ -78,14 +85,20 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                     P]
     lib.gdn_sync_status.restype = ctypes.c_int
     lib.gdn_sync_status.argtypes = [P]
-    lib.gdn_set_prefill_impl.restype = ctypes.c_int
-    lib.gdn_set_prefill_impl.argtypes = [i32]
-    lib.gdn_set_kernel_timing.restype = ctypes.c_int
-    lib.gdn_set_kernel_timing.argtypes = [i32]
-    lib.gdn_last_prefill_kernel_ms.restype = ctypes.c_int
-    lib.gdn_last_prefill_kernel_ms.argtypes = [P, i32]
-    lib.gdn_last_prefill_kernel_name.restype = ctypes.c_char_p
-    lib.gdn_last_prefill_kernel_name.argtypes = [i32]
+    lib.gdn_prefill_ex.restype = ctypes.c_int
+    lib.gdn_prefill_ex.argtypes = [P, P, P, i32, P, P, P, P, P, P, i32, i64, i32, i32, i32, i32,
+                                   f32, P, P, P, sz, P, P]
+    lib.gdn_prefill_slots_ex.restype = ctypes.c_int
+    lib.gdn_prefill_slots_ex.argtypes = [P, P, P, i32, P, P, P, P, P, P, P, i32, P, i32, i64,
+                                         i32, i32, i32, i32, f32, P, P, sz, P, P]
+    lib.gdn_timer_create.restype = P
+    lib.gdn_timer_create.argtypes = []
+    lib.gdn_timer_destroy.restype = None
+    lib.gdn_timer_destroy.argtypes = [P]
+    lib.gdn_timer_read.restype = ctypes.c_int
+    lib.gdn_timer_read.argtypes = [P, P, i32]
+    lib.gdn_timer_kernel_name.restype = ctypes.c_char_p
+    lib.gdn_timer_kernel_name.argtypes = [P, i32]
     lib.gdn_conv1d_silu.restype = ctypes.c_int
     lib.gdn_conv1d_silu.argtypes = [P, i32, P, P, P, P, i32, i64, i32, i32, P, P, P]
     lib.gdn_conv1d_silu_decode.restype = ctypes.c_int
@@ -155,14 +168,53 @@ def gdn_gates(a, b, A_log, dt_bias, cu_seqlens, *, want_cumsum=True, want_g=True
     return G, g, beta
 
 
+class Timer:
+    """A gdn_timer: CUDA events around every kernel of the calls it is passed to."""
+
+    def __init__(self):
+        self._lib = load_library()
+        self._t = self._lib.gdn_timer_create()
+        if not self._t:
+            raise GDNError(4, "gdn_timer_create")
+
+    def times(self) -> list:
+        """[(kernel name, milliseconds)] of the most recent call made with this timer
+        (waits for its events)."""
+        ms = (ctypes.c_float * 4)()
+        n = int(self._lib.gdn_timer_read(ctypes.c_void_p(self._t), ms, 4))
+        if n < 0:
+            raise GDNError(-n, "gdn_timer_read")
+        return [(self._lib.gdn_timer_kernel_name(ctypes.c_void_p(self._t), i).decode(),
+                 float(ms[i])) for i in range(min(n, 4))]
+
+    def close(self):
+        if getattr(self, "_t", None):
+            self._lib.gdn_timer_destroy(ctypes.c_void_p(self._t))
+            self._t = None
+
+    def __del__(self):
+        self.close()
+
+
+def _options(impl, fault, wait_limit_cycles, timer):
+    if impl == GDN_IMPL_AUTO and fault == GDN_FAULT_NONE and not wait_limit_cycles and \
+            timer is None:
+        return None
+    return ctypes.byref(PrefillOptions(int(impl), int(fault), int(wait_limit_cycles),
+                                       None if timer is None else timer._t))
+
+
 def gdn_prefill(q, k, v, a, b, A_log, dt_bias, cu_seqlens, initial_state=None, *,
                 scale: float = 1.0, output_final_state: bool = True, out=None,
-                final_state=None, workspace=None):
+                final_state=None, workspace=None, impl: int = GDN_IMPL_AUTO,
+                timer: Optional[Timer] = None, fault: int = GDN_FAULT_NONE,
+                wait_limit_cycles: int = 0):
     """Chunked prefill over a packed batch. Returns (o, final_state or None).
 
     q, k [T, H_qk, d_k]; v [T, H_v, d_v] (bf16 or fp32, all the same);
     a, b [T, H_v] fp32; A_log, dt_bias [H_v] fp32; cu_seqlens int32 [N+1];
-    initial_state [N, H_v, d_v, d_k] fp32 or None.
+    initial_state [N, H_v, d_v, d_k] fp32 or None. impl, timer, fault and
+    wait_limit_cycles are gdn_prefill_options (gdn_prefill_ex).
     """
     lib = load_library()
     _need_cuda(q, k, v, a, b, A_log, dt_bias, cu_seqlens, initial_state, out, final_state,
@@ -181,16 +233,21 @@ def gdn_prefill(q, k, v, a, b, A_log, dt_bias, cu_seqlens, initial_state=None, *
     need = lib.gdn_prefill_workspace_size(N, T, H_qk, H_v, d_k, d_v)
     if workspace is None:
         workspace = torch.empty((max(int(need), 1),), device=q.device, dtype=torch.uint8)
-    st = lib.gdn_prefill(_ptr(q), _ptr(k), _ptr(v), io, _ptr(a), _ptr(b), _ptr(A_log),
-                         _ptr(dt_bias), _ptr(initial_state), _ptr(cu_seqlens), N, T, H_qk, H_v,
-                         d_k, d_v, float(scale), _ptr(o), _ptr(final_state), _ptr(workspace),
-                         workspace.numel(), _stream(q.device))
+    opts = _options(impl, fault, wait_limit_cycles, timer)
+    args = (_ptr(q), _ptr(k), _ptr(v), io, _ptr(a), _ptr(b), _ptr(A_log), _ptr(dt_bias),
+            _ptr(initial_state), _ptr(cu_seqlens), N, T, H_qk, H_v, d_k, d_v, float(scale),
+            _ptr(o), _ptr(final_state), _ptr(workspace), workspace.numel())
+    if opts is None:
+        st = lib.gdn_prefill(*args, _stream(q.device))
+    else:
+        st = lib.gdn_prefill_ex(*args, opts, _stream(q.device))
     _check(st, "gdn_prefill")
     return o, final_state
 
 
 def gdn_prefill_slots(q, k, v, a, b, A_log, dt_bias, cu_seqlens, state_pool, state_slots,
-                      has_initial_state=None, *, scale: float = 1.0, out=None, workspace=None):
+                      has_initial_state=None, *, scale: float = 1.0, out=None, workspace=None,
+                      impl: int = GDN_IMPL_AUTO):
     """gdn_prefill with the states in a pool: sequence n starts from state_pool[slot]
     (or zeros where has_initial_state[n] == 0) and its final state replaces it.
     state_pool [num_slots, H_v, d_v, d_k] fp32; state_slots, has_initial_state int32 [N]."""
@@ -210,11 +267,15 @@ def gdn_prefill_slots(q, k, v, a, b, A_log, dt_bias, cu_seqlens, state_pool, sta
     need = lib.gdn_prefill_workspace_size(N, T, H_qk, H_v, d_k, d_v)
     if workspace is None:
         workspace = torch.empty((max(int(need), 1),), device=q.device, dtype=torch.uint8)
-    st = lib.gdn_prefill_slots(_ptr(q), _ptr(k), _ptr(v), io, _ptr(a), _ptr(b), _ptr(A_log),
-                               _ptr(dt_bias), _ptr(state_pool), _ptr(state_slots),
-                               _ptr(has_initial_state), state_pool.shape[0], _ptr(cu_seqlens), N,
-                               T, H_qk, H_v, d_k, d_v, float(scale), _ptr(o), _ptr(workspace),
-                               workspace.numel(), _stream(q.device))
+    args = (_ptr(q), _ptr(k), _ptr(v), io, _ptr(a), _ptr(b), _ptr(A_log), _ptr(dt_bias),
+            _ptr(state_pool), _ptr(state_slots), _ptr(has_initial_state), state_pool.shape[0],
+            _ptr(cu_seqlens), N, T, H_qk, H_v, d_k, d_v, float(scale), _ptr(o), _ptr(workspace),
+            workspace.numel())
+    opts = _options(impl, GDN_FAULT_NONE, 0, None)
+    if opts is None:
+        st = lib.gdn_prefill_slots(*args, _stream(q.device))
+    else:
+        st = lib.gdn_prefill_slots_ex(*args, opts, _stream(q.device))
     _check(st, "gdn_prefill_slots")
     return o
 
@@ -285,35 +346,10 @@ def gdn_decode_slots(q, k, v, a, b, A_log, dt_bias, state_pool, state_slots=None
     return o, intermediate_states
 
 
-def set_prefill_impl(impl: int) -> int:
-    """Choose the gdn_prefill implementation process-wide; returns the previous choice."""
-    prev = int(load_library().gdn_set_prefill_impl(int(impl)))
-    if prev < 0:
-        raise GDNError(-prev, "gdn_set_prefill_impl")
-    return prev
-
-
 def gdn_sync_status(device=None) -> int:
     """Synchronise the current stream and return (and clear) the device status word."""
     lib = load_library()
     return int(lib.gdn_sync_status(_stream(device)))
-
-
-def set_kernel_timing(enable: bool) -> bool:
-    """Record CUDA events around every kernel of later gdn_prefill calls; returns the
-    previous setting."""
-    return bool(load_library().gdn_set_kernel_timing(1 if enable else 0))
-
-
-def last_prefill_kernel_times() -> list:
-    """[(kernel name, milliseconds)] of the most recent gdn_prefill call made while
-    kernel timing was enabled (waits for its events)."""
-    lib = load_library()
-    ms = (ctypes.c_float * 4)()
-    n = int(lib.gdn_last_prefill_kernel_ms(ms, 4))
-    if n < 0:
-        raise GDNError(-n, "gdn_last_prefill_kernel_ms")
-    return [(lib.gdn_last_prefill_kernel_name(i).decode(), float(ms[i])) for i in range(min(n, 4))]
 
 
 def gdn_conv1d_silu(x, weight, bias, cu_seqlens, conv_state_in=None, *, want_state=True,

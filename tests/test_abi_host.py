@@ -49,12 +49,6 @@ def test_workspace_size(lib):
     tc = lambda N, ch, hv: a256((N + 1) * 4) + a256(ch * hv * 8) + ch * hv * 17664
     assert ws(1, 4096, 16, 32, 128, 128) == tc(1, 64 + 1, 32)
     assert ws(4, 4 * 16384, 16, 64, 128, 128) == tc(4, 1024 + 4, 64)
-    # the Gram-matrix schedule adds one 8,192-byte tile per (chunk, QK head)
-    prev = lib.gdn_set_prefill_impl(5)
-    try:
-        assert ws(1, 4096, 16, 32, 128, 128) == tc(1, 64 + 1, 32) + 65 * 16 * 8192
-    finally:
-        lib.gdn_set_prefill_impl(prev)
     # never below the CUDA-core path's need (G and beta, fp32 [T, H_v] each)
     assert ws(1, 3, 1, 1, 128, 128) >= 2 * 256
     assert ws(1, 3, 1, 1, 64, 64) == 2 * 256  # each part rounded up to 256 bytes
@@ -113,18 +107,38 @@ def test_prefill_rejects(lib, over, code):
     assert _call_prefill(lib, **over) == code
 
 
-def test_gram_schedule_needs_its_workspace(lib):
-    """A workspace sized while another schedule was selected is too small for the
-    Gram-matrix schedule (its tiles are counted only while it is selected): the call is
-    rejected on the host before anything is launched."""
-    dims = dict(N=1, T=4096, H_qk=16, H_v=32, d_k=128, d_v=128)
-    size_default = lib.gdn_prefill_workspace_size(1, 4096, 16, 32, 128, 128)
-    prev = lib.gdn_set_prefill_impl(5)
-    try:
-        assert lib.gdn_prefill_workspace_size(1, 4096, 16, 32, 128, 128) > size_default
-        assert _call_prefill(lib, ws_bytes=size_default, **dims) == 3
-    finally:
-        lib.gdn_set_prefill_impl(prev)
+def _call_prefill_ex(lib, opts, **over):
+    a = _prefill_args(**over)
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.gdn_prefill_ex(v(a["q"]), v(a["k"]), v(a["v"]), a["io"], v(a["a"]), v(a["b"]),
+                              v(a["A_log"]), v(a["dt_bias"]), v(a["S0"]), v(a["cu"]), a["N"],
+                              a["T"], a["H_qk"], a["H_v"], a["d_k"], a["d_v"], a["scale"],
+                              v(a["o"]), v(a["Sf"]), v(a["ws"]), a["ws_bytes"],
+                              None if opts is None else ctypes.byref(opts), v(a["stream"]))
+
+
+@pytest.mark.parametrize("opts,over,code", [
+    (dict(impl=5), {}, 1),                          # no such implementation
+    (dict(impl=-1), {}, 1),
+    (dict(fault=2), {}, 1),                         # no such fault
+    (dict(wait_limit_cycles=-1), {}, 1),
+    (dict(impl=2), {}, 2),                          # tensor cores forced, d = 64: unsupported
+    (dict(impl=3), dict(io=gdn.GDN_FP32, d_k=128, d_v=128), 2),  # fp32 I/O
+    (dict(impl=1), dict(ws_bytes=100), 3),          # the ordinary checks still apply
+    (dict(impl=0), dict(N=0, T=0, q=None, k=None, v=None, o=None, ws=None, ws_bytes=0), 0),
+])
+def test_prefill_ex_rejects(lib, opts, over, code):
+    """Per-call options are checked on the host, before any launch, like every argument."""
+    o = gdn.PrefillOptions()
+    for k_, v_ in opts.items():
+        setattr(o, k_, v_)
+    assert _call_prefill_ex(lib, o, **over) == code
+
+
+def test_prefill_ex_null_options_is_prefill(lib):
+    for over in (dict(ws_bytes=100), dict(io=7), dict(N=0, T=0, q=None, k=None, v=None, o=None,
+                                                     ws=None, ws_bytes=0)):
+        assert _call_prefill_ex(lib, None, **over) == _call_prefill(lib, **over)
 
 
 def test_prefill_empty_batch_is_noop(lib):
@@ -312,22 +326,9 @@ def test_binding_fails_loudly_without_library(tmp_path):
         gdn._lib = saved
 
 
-def test_set_prefill_impl(lib):
-    assert lib.gdn_set_prefill_impl(1) == 0
-    assert lib.gdn_set_prefill_impl(2) == 1
-    assert lib.gdn_set_prefill_impl(3) == 2
-    assert lib.gdn_set_prefill_impl(4) == 3
-    assert lib.gdn_set_prefill_impl(5) == 4
-    assert lib.gdn_set_prefill_impl(7) == -1      # invalid: unchanged
-    assert lib.gdn_set_prefill_impl(0) == 5
-
-
-def test_kernel_timing_switch(lib):
-    prev = lib.gdn_set_kernel_timing(1)
-    assert lib.gdn_set_kernel_timing(0) == 1
-    lib.gdn_set_kernel_timing(prev)
-    assert lib.gdn_last_prefill_kernel_ms(None, 4) == -1
+def test_timer_host_checks(lib):
+    """The timer calls reject null handles without touching the GPU."""
     ms = (ctypes.c_float * 4)()
-    assert lib.gdn_last_prefill_kernel_ms(ms, -1) == -1
-    assert lib.gdn_last_prefill_kernel_name(-1) is None
-    assert lib.gdn_last_prefill_kernel_name(99) is None
+    assert lib.gdn_timer_read(None, ms, 4) == -1
+    assert lib.gdn_timer_kernel_name(None, 0) is None
+    lib.gdn_timer_destroy(None)  # ignored

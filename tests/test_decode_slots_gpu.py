@@ -148,15 +148,11 @@ def test_prefill_slots_against_oracle(impl):
     pool = D.state.contiguous()
     slots = torch.tensor([6, 2, -1, 0, 8], dtype=torch.int32)
     has_init = torch.tensor([1, 0, 1, 1, 0], dtype=torch.int32)
-    prev = gdn.set_prefill_impl(getattr(gdn, impl))
-    try:
-        Pd = P.to("cuda")
-        pool_d = pool.cuda()
-        o = gdn_prefill_slots(Pd.q, Pd.k, Pd.v, Pd.a, Pd.b, Pd.A_log, Pd.dt_bias, Pd.cu_seqlens,
-                              pool_d, slots.cuda(), has_init.cuda())
-        assert gdn_sync_status() == 0
-    finally:
-        gdn.set_prefill_impl(prev)
+    Pd = P.to("cuda")
+    pool_d = pool.cuda()
+    o = gdn_prefill_slots(Pd.q, Pd.k, Pd.v, Pd.a, Pd.b, Pd.A_log, Pd.dt_bias, Pd.cu_seqlens,
+                          pool_d, slots.cuda(), has_init.cuda(), impl=getattr(gdn, impl))
+    assert gdn_sync_status() == 0
     cu = P.cu_seqlens.tolist()
     for n in range(len(lens)):
         s, use = int(slots[n]), bool(has_init[n]) and int(slots[n]) >= 0

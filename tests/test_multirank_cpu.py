@@ -66,12 +66,40 @@ def test_single_rank_helpers_need_no_process_group():
     bench._barrier(1)
 
 
-def test_kernel_profile_lines_parse():
-    """bench.py reads the dominant kernel's DRAM traffic and the source hash it was taken on
-    from the committed ncu summary (list-marked lines)."""
+def test_kernel_traffic_record(tmp_path, monkeypatch):
+    """bench.py takes a kernel's DRAM traffic per launch from the committed ncu record
+    (a JSON file), and only while the record's source hash matches the kernel source."""
+    import json
     sys.path.insert(0, ROOT)
     import bench
-    traffic, sha = bench._kernel_traffic()
-    assert isinstance(traffic, int) and 10**7 < traffic < 10**9
-    assert isinstance(sha, str) and len(sha) == 40 and all(c in "0123456789abcdef" for c in sha)
-    assert len(bench._kernel_source_sha1()) == 40
+    committed = json.load(open(bench.TRAFFIC_FILE))
+    for key, rec in committed.items():
+        kernel, workload = key.split("@")
+        assert isinstance(rec["traffic_bytes_per_launch"], int)
+        assert len(rec["kernel_source_sha1"]) == 40 and rec["command"]
+    sha = bench._source_sha1()
+    f = tmp_path / "t.json"
+    f.write_text(json.dumps({"prep@w": {"traffic_bytes_per_launch": 123,
+                                        "kernel_source_sha1": sha, "command": "x"},
+                             "chain@w": {"traffic_bytes_per_launch": 456,
+                                         "kernel_source_sha1": "0" * 40, "command": "x"}}))
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(f))
+    assert bench.kernel_traffic("prep", "w") == 123
+    assert bench.kernel_traffic("chain", "w") is None      # taken on another build
+    assert bench.kernel_traffic("fused", "w") is None      # no record
+
+
+def test_kernel_bytes_and_flops():
+    """The algorithmic accounting of the bench line, on the 35B-A3B layer shape: bytes
+    of the whole call and of each kernel, and the chunk form's tensor flops."""
+    sys.path.insert(0, ROOT)
+    import bench
+    T, N, H_qk, H_v, d = 4096, 1, 16, 32, 128
+    call = bench.prefill_bytes(T, N, H_qk, H_v, d, 2, False)
+    assert call == 103_809_024
+    assert bench.kernel_bytes("fused_half_rows", T, N, H_qk, H_v, d, 2, False) == call
+    assert bench.kernel_bytes("chain", T, N, H_qk, H_v, d, 2, False) == call - 8 * T * H_v
+    assert bench.kernel_bytes("prep", T, N, H_qk, H_v, d, 2, False) == \
+        4 * T * H_qk * d + 8 * T * H_v
+    # H_qk 4 C d + H_v (2 C d + 4 C d + 6 d^2) per token
+    assert bench.prefill_flops(T, N, H_qk, H_v, d) == 21_474_836_480

@@ -11,9 +11,9 @@ import pytest
 import torch
 
 import oracle
-from linear_attention_sequence_delta_b200 import gdn_prefill, gdn_sync_status
+from linear_attention_sequence_delta_b200 import gdn, gdn_prefill, gdn_sync_status
 from linear_attention_sequence_delta_b200.inputs import WORKLOADS, make_prefill_inputs
-from tests.parity_util import TOL_BF16, TOL_FP32, oracle_prefill_heads, rel_err
+from tests.parity_util import TOL_BF16, TOL_FP32, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -134,171 +134,230 @@ def test_prefill_35b_layer_full():
     _check(P, TOL_BF16)
 
 
-def test_prefill_397b_long_sampled():
-    """B=4, T=16384, 16 QK / 64 V heads: the full launch, sampled (sequence, head) units."""
+def _check_per_sequence(P, o, Sf):
+    """Every output and final state against the oracle, one oracle call per sequence
+    (all V heads of it at once, OpenMP over the heads): exact, since (sequence, head)
+    units are independent, and the host memory stays bounded."""
+    cu = P.cu_seqlens.cpu().tolist()
+    worst_o = worst_s = 0.0
+    for n in range(len(cu) - 1):
+        s0, s1 = cu[n], cu[n + 1]
+        S0 = None if P.initial_state is None else P.initial_state[n:n + 1].cpu()
+        o_ref, S_ref = oracle.forward(P.q[s0:s1].cpu(), P.k[s0:s1].cpu(), P.v[s0:s1].cpu(),
+                                      P.a[s0:s1].cpu(), P.b[s0:s1].cpu(), P.A_log.cpu(),
+                                      P.dt_bias.cpu(), [0, s1 - s0], S0)
+        eo, es = rel_err(o[s0:s1], o_ref), rel_err(Sf[n:n + 1], S_ref)
+        assert eo <= TOL_BF16 and es <= TOL_BF16, (n, eo, es)
+        worst_o, worst_s = max(worst_o, eo), max(worst_s, es)
+    return worst_o, worst_s
+
+
+def test_prefill_397b_long_full():
+    """B=4, T=16384, 16 QK / 64 V heads, d=128, bf16: every output and final state of
+    all 256 (sequence, head) units against the oracle."""
     P = make_prefill_inputs(**WORKLOADS["prefill_397b_long"], seed=0, device="cuda")
     o, Sf = gdn_prefill(P.q, P.k, P.v, P.a, P.b, P.A_log, P.dt_bias, P.cu_seqlens, None)
     assert gdn_sync_status() == 0
-    units = [(0, 0), (1, 17), (3, 63)]
-    ref = {}
-    for n, h in units:
-        ref.update(oracle_prefill_heads(P, [h], seqs=[n]))
-    cu = P.cu_seqlens.cpu().tolist()
-    for (n, h), (o_ref, S_ref) in ref.items():
-        assert rel_err(o[cu[n]:cu[n + 1], h], o_ref) <= TOL_BF16
-        assert rel_err(Sf[n, h], S_ref) <= TOL_BF16
-    assert torch.isfinite(o.float()).all() and torch.isfinite(Sf).all()
+    _check_per_sequence(P, o, Sf)
 
 
-def test_varlen_64_sampled():
-    """64 sequences, lengths U[128, 8192], nonzero initial states: sampled units."""
+def test_varlen_64_full():
+    """64 sequences, lengths U[128, 8192], nonzero initial states: all 2,048 units."""
     P = make_prefill_inputs(**WORKLOADS["varlen_64"], seed=0, device="cuda")
     o, Sf = gdn_prefill(P.q, P.k, P.v, P.a, P.b, P.A_log, P.dt_bias, P.cu_seqlens,
                         P.initial_state)
     assert gdn_sync_status() == 0
-    cu = P.cu_seqlens.cpu().tolist()
-    lens = np.diff(cu)
-    seqs = [int(np.argmin(lens)), int(np.argmax(lens)), 31]
-    ref = oracle_prefill_heads(P, [0, 13, 31], seqs=seqs)
-    for (n, h), (o_ref, S_ref) in ref.items():
-        assert rel_err(o[cu[n]:cu[n + 1], h], o_ref) <= TOL_BF16
-        assert rel_err(Sf[n, h], S_ref) <= TOL_BF16
-    assert torch.isfinite(o.float()).all() and torch.isfinite(Sf).all()
+    _check_per_sequence(P, o, Sf)
 
 
-@pytest.fixture
-def impl_switch():
-    from linear_attention_sequence_delta_b200 import gdn
-    prev = gdn.set_prefill_impl(gdn.GDN_IMPL_AUTO)
-    yield gdn
-    gdn.set_prefill_impl(prev)
+IMPLS = {"cuda_core": gdn.GDN_IMPL_CUDA_CORE, "tensor_core": gdn.GDN_IMPL_TENSOR_CORE,
+         "tensor_core_split": gdn.GDN_IMPL_TENSOR_CORE_SPLIT,
+         "tensor_core_whole_rows": gdn.GDN_IMPL_TENSOR_CORE_WHOLE_ROWS}
 
 
-IMPLS = {"cuda_core": "GDN_IMPL_CUDA_CORE", "tensor_core": "GDN_IMPL_TENSOR_CORE",
-         "tensor_core_split": "GDN_IMPL_TENSOR_CORE_SPLIT",
-         "tensor_core_whole_rows": "GDN_IMPL_TENSOR_CORE_WHOLE_ROWS",
-         "tensor_core_gram": "GDN_IMPL_TENSOR_CORE_GRAM"}
+def _check_impl(P, impl, tol=TOL_BF16, timer=None):
+    Pd = P.to("cuda")
+    o, Sf = gdn_prefill(Pd.q, Pd.k, Pd.v, Pd.a, Pd.b, Pd.A_log, Pd.dt_bias, Pd.cu_seqlens,
+                        Pd.initial_state, impl=impl, timer=timer)
+    assert gdn_sync_status() == 0
+    o_ref, S_ref = _full_oracle(P)
+    eo, es = rel_err(o, o_ref), rel_err(Sf, S_ref)
+    assert eo <= tol and es <= tol, (eo, es)
+    return o, Sf
 
 
 @pytest.mark.parametrize("impl", list(IMPLS))
 @pytest.mark.parametrize("lengths", [[1], [63], [64], [65], [127], [200], [5, 0, 130, 64]])
-def test_bf16_every_implementation(impl_switch, impl, lengths):
-    g = impl_switch
-    g.set_prefill_impl(getattr(g, IMPLS[impl]))
+def test_bf16_every_implementation(impl, lengths):
     P = make_prefill_inputs(lengths, H_qk=2, H_v=4, d_k=128, d_v=128, state_std=0.05,
                             seed=sum(lengths) + 7)
-    _check(P, TOL_BF16)
+    _check_impl(P, IMPLS[impl])
 
 
-@pytest.mark.parametrize("impl", ["GDN_IMPL_TENSOR_CORE", "GDN_IMPL_TENSOR_CORE_GRAM"])
-def test_tensor_core_stress_gates(impl_switch, impl):
+@pytest.mark.parametrize("impl", ["tensor_core", "tensor_core_split"])
+def test_tensor_core_stress_gates(impl):
     """Slow decay, strong writes and extreme gates through the tensor-core path."""
-    g = impl_switch
-    g.set_prefill_impl(getattr(g, impl))
     P = make_prefill_inputs([500], H_qk=1, H_v=4, d_k=128, d_v=128, state_std=0.1, seed=12)
     P.A_log[0] = -4.0                 # alpha near 0.98: long carry across chunks
     P.b[:, 1] = 4.0                   # beta near 1
     P.a[100:130, 2] = -1e30           # alpha = 1 run
     P.A_log[3] = 100.0                # alpha = 0 every token
-    _check(P, TOL_BF16)
+    _check_impl(P, IMPLS[impl])
 
 
-def test_tensor_core_rejects_fp32(impl_switch):
-    g = impl_switch
-    g.set_prefill_impl(g.GDN_IMPL_TENSOR_CORE)
+def test_tensor_core_rejects_fp32():
     P = make_prefill_inputs([64], H_qk=1, H_v=1, d_k=128, d_v=128, io_dtype=torch.float32)
-    with pytest.raises(g.GDNError):
-        _run(P)
+    with pytest.raises(gdn.GDNError):
+        _check_impl(P, gdn.GDN_IMPL_TENSOR_CORE)
 
 
-def test_kernel_timing_names_and_durations(impl_switch):
-    g = impl_switch
+def test_kernel_timing_names_and_durations():
     P = make_prefill_inputs([300, 77], H_qk=2, H_v=4, d_k=128, d_v=128, seed=31)
-    prev = g.set_kernel_timing(True)
-    try:
-        for impl, names in ((g.GDN_IMPL_TENSOR_CORE, ["fused_half_rows"]),  # 8 chains
-                            (g.GDN_IMPL_TENSOR_CORE_GRAM, ["fused_half_rows_gram"]),
-                            (g.GDN_IMPL_TENSOR_CORE_WHOLE_ROWS, ["fused"]),
-                            (g.GDN_IMPL_TENSOR_CORE_SPLIT, ["chunk_offsets", "prep", "chain"]),
-                            (g.GDN_IMPL_CUDA_CORE, ["gates", "prefill_simt"])):
-            g.set_prefill_impl(impl)
-            _run(P)
-            times = g.last_prefill_kernel_times()
-            assert [n for n, _ in times] == names
-            assert all(0.0 < ms < 1000.0 for _, ms in times)
-    finally:
-        g.set_kernel_timing(prev)
+    timer = gdn.Timer()
+    for impl, names in ((gdn.GDN_IMPL_TENSOR_CORE, ["fused_half_rows"]),  # 8 chains
+                        (gdn.GDN_IMPL_TENSOR_CORE_WHOLE_ROWS, ["fused"]),
+                        (gdn.GDN_IMPL_TENSOR_CORE_SPLIT, ["chunk_offsets", "prep", "chain"]),
+                        (gdn.GDN_IMPL_CUDA_CORE, ["gates", "prefill_simt"])):
+        _check_impl(P, impl, timer=timer)
+        times = timer.times()
+        assert [n for n, _ in times] == names
+        assert all(0.0 < ms < 1000.0 for _, ms in times)
+    # a call without the timer leaves its record alone
+    _check_impl(P, gdn.GDN_IMPL_TENSOR_CORE_SPLIT)
+    assert [n for n, _ in timer.times()] == ["gates", "prefill_simt"]
+    timer.close()
 
 
 @pytest.mark.parametrize("wl", ["prefill_35b", "varlen_64"])
-def test_fused_equals_split(impl_switch, wl):
+def test_fused_equals_split(wl):
     """The overlapped single launch (half-row chain blocks for the 35B layer's 32 chains,
     whole-row blocks for 64 chains) and the separate launches compute the same thing
     (same arithmetic per element, different scheduling): outputs agree to the last bit."""
-    g = impl_switch
     W = dict(WORKLOADS[wl])
     if wl == "varlen_64":
         W["num_seqs"] = 2  # 64 chains: few enough for the overlapped launch
     P = make_prefill_inputs(**W, seed=3, device="cuda")
     fused = "fused_half_rows" if wl == "prefill_35b" else "fused"
     outs = []
-    prev = g.set_kernel_timing(True)
-    try:
-        for impl, kernel in ((g.GDN_IMPL_TENSOR_CORE, fused),
-                             (g.GDN_IMPL_TENSOR_CORE_WHOLE_ROWS, "fused"),
-                             (g.GDN_IMPL_TENSOR_CORE_SPLIT, "chain")):
-            g.set_prefill_impl(impl)
-            o, Sf = gdn_prefill(P.q, P.k, P.v, P.a, P.b, P.A_log, P.dt_bias, P.cu_seqlens,
-                                P.initial_state)
-            assert gdn_sync_status() == 0
-            assert kernel in [n for n, _ in g.last_prefill_kernel_times()]
-            outs.append((o, Sf))
-    finally:
-        g.set_kernel_timing(prev)
+    timer = gdn.Timer()
+    for impl, kernel in ((gdn.GDN_IMPL_TENSOR_CORE, fused),
+                         (gdn.GDN_IMPL_TENSOR_CORE_WHOLE_ROWS, "fused"),
+                         (gdn.GDN_IMPL_TENSOR_CORE_SPLIT, "chain")):
+        o, Sf = gdn_prefill(P.q, P.k, P.v, P.a, P.b, P.A_log, P.dt_bias, P.cu_seqlens,
+                            P.initial_state, impl=impl, timer=timer)
+        assert gdn_sync_status() == 0
+        assert kernel in [n for n, _ in timer.times()]
+        outs.append((o, Sf))
     for o_, S_ in outs[1:]:
         assert torch.equal(outs[0][0], o_) and torch.equal(outs[0][1], S_)
 
 
-@pytest.mark.parametrize("lengths,H_qk,H_v", [([4096], 4, 8), ([1000, 300, 64, 2000, 1], 2, 4)])
-def test_gram_schedule(impl_switch, lengths, H_qk, H_v):
-    """The cross-chunk Gram-matrix schedule (half-row blocks; S_c K_c^T built from the
-    previous chunk's bf16 state and the key Gram matrix) against the oracle, every output,
-    and against the default schedule: the same mathematics with another bf16 rounding."""
-    g = impl_switch
-    P = make_prefill_inputs(lengths, H_qk=H_qk, H_v=H_v, d_k=128, d_v=128, state_std=0.05,
-                            seed=len(lengths) + 40)
-    prev = g.set_kernel_timing(True)
-    try:
-        g.set_prefill_impl(g.GDN_IMPL_TENSOR_CORE_GRAM)
-        o, Sf = _run(P)
-        assert [n for n, _ in g.last_prefill_kernel_times()] == ["fused_half_rows_gram"]
-        g.set_prefill_impl(g.GDN_IMPL_TENSOR_CORE)
-        o_d, S_d = _run(P)
-    finally:
-        g.set_kernel_timing(prev)
-    o_ref, S_ref = _full_oracle(P)
-    assert rel_err(o, o_ref) <= TOL_BF16 and rel_err(Sf, S_ref) <= TOL_BF16
-    # both schedules sit well inside the tolerance and close to each other
-    assert rel_err(o, o_d.float().cpu().numpy()) <= TOL_BF16 / 2
-    assert rel_err(Sf, S_d.cpu().numpy()) <= TOL_BF16 / 2
-
-
-def test_gram_schedule_35b_layer_full(impl_switch):
-    g = impl_switch
-    g.set_prefill_impl(g.GDN_IMPL_TENSOR_CORE_GRAM)
-    P = make_prefill_inputs(**WORKLOADS["prefill_35b"], seed=0)
-    _check(P, TOL_BF16)
-
-
-def test_many_chains_use_separate_launches(impl_switch):
+def test_many_chains_use_separate_launches():
     """With more (sequence, V head) chains than half the SMs the default path runs the
     preparation and the chains as separate launches."""
-    g = impl_switch
-    g.set_prefill_impl(g.GDN_IMPL_AUTO)
     P = make_prefill_inputs([100] * 8, H_qk=16, H_v=32, d_k=128, d_v=128, seed=4)
-    prev = g.set_kernel_timing(True)
-    try:
-        _check(P, TOL_BF16)
-        assert [n for n, _ in g.last_prefill_kernel_times()] == ["chunk_offsets", "prep", "chain"]
-    finally:
-        g.set_kernel_timing(prev)
+    timer = gdn.Timer()
+    _check_impl(P, gdn.GDN_IMPL_AUTO, timer=timer)
+    assert [n for n, _ in timer.times()] == ["chunk_offsets", "prep", "chain"]
+
+
+# ------------------------------------------------ workspace contents, failures ----
+
+def _ws_fill(work, pattern):
+    """Fill a workspace with contents a caching allocator could hand back."""
+    w64 = work[: work.numel() // 8 * 8].view(torch.int64)
+    if pattern == "small_ints":      # every small integer, in order
+        w64.copy_(torch.arange(w64.numel(), device=work.device, dtype=torch.int64))
+    elif pattern == "small_ints_rev":
+        w64.copy_(torch.arange(w64.numel(), 0, -1, device=work.device, dtype=torch.int64))
+    elif pattern == "ones":
+        w64.fill_(1)
+    elif pattern == "all_bits":
+        work.fill_(0xFF)
+    elif pattern == "top_bit":       # the form this library's call numbers take
+        w64.fill_(-(1 << 63))
+
+
+@pytest.mark.parametrize("pattern", ["small_ints", "small_ints_rev", "ones", "all_bits",
+                                     "top_bit"])
+@pytest.mark.parametrize("lengths,H_v,impl", [([700, 333], 4, gdn.GDN_IMPL_TENSOR_CORE),
+                                              ([700, 333], 4, gdn.GDN_IMPL_TENSOR_CORE_WHOLE_ROWS),
+                                              ([1000] * 20, 4, gdn.GDN_IMPL_TENSOR_CORE_SPLIT)])
+def test_workspace_contents_do_not_matter(pattern, lengths, H_v, impl):
+    """A record counts as published only when its flag equals this call's number. A
+    workspace that already holds integers (every small value, as indices or counts left
+    by other work would), all-ones bytes, or words with only the top bit set, must give
+    the same results as a fresh one, compared with the oracle on every output."""
+    P = make_prefill_inputs(lengths, H_qk=2, H_v=H_v, d_k=128, d_v=128, state_std=0.05,
+                            seed=len(lengths) + 50)
+    Pd = P.to("cuda")
+    T, N = P.q.shape[0], P.num_seqs
+    work = torch.empty(gdn.workspace_size(N, T, 2, H_v, 128, 128), dtype=torch.uint8,
+                       device="cuda")
+    o_ref, S_ref = _full_oracle(P)
+    for _ in range(2):  # refilled before each of two calls in a row
+        _ws_fill(work, pattern)
+        o, Sf = gdn_prefill(Pd.q, Pd.k, Pd.v, Pd.a, Pd.b, Pd.A_log, Pd.dt_bias, Pd.cu_seqlens,
+                            Pd.initial_state, workspace=work, impl=impl)
+        assert gdn_sync_status() == 0
+        assert rel_err(o, o_ref) <= TOL_BF16 and rel_err(Sf, S_ref) <= TOL_BF16
+
+
+@pytest.mark.parametrize("lengths,H_v", [([300, 77], 4),      # half-row chain blocks
+                                         ([200] * 12, 4)])    # whole-row chain blocks
+def test_bounded_wait_runs_out_and_context_survives(lengths, H_v):
+    """Fault injection on the host side: the overlapped launch's preparation publishes
+    no record, so every chain's bounded wait (here about 10^5 cycles) runs out. The
+    call must end by itself with GDN_ERR_TIMEOUT in the status word (nothing traps or
+    hangs: each role leaves its loops, drains its copies and frees its tensor memory),
+    and the next ordinary call on the same context must match the oracle."""
+    P = make_prefill_inputs(lengths, H_qk=2, H_v=H_v, d_k=128, d_v=128, state_std=0.05,
+                            seed=len(lengths) + 60)
+    Pd = P.to("cuda")
+    timer = gdn.Timer()
+    for _ in range(2):
+        gdn_prefill(Pd.q, Pd.k, Pd.v, Pd.a, Pd.b, Pd.A_log, Pd.dt_bias, Pd.cu_seqlens,
+                    Pd.initial_state, fault=gdn.GDN_FAULT_WITHHOLD_RECORDS,
+                    wait_limit_cycles=100_000, timer=timer)
+        assert gdn_sync_status() == 5  # GDN_ERR_TIMEOUT
+        assert gdn_sync_status() == 0  # read and cleared
+        (name, ms), = timer.times()
+        assert name.startswith("fused") and ms < 100.0  # the short limit, not the default
+    o, Sf = _check_impl(P, gdn.GDN_IMPL_AUTO)
+
+
+def _guarded(shape, dtype, guard=4096):
+    """A tensor of `shape` inside a larger buffer whose guard regions (`guard` bytes on
+    each side) hold a known pattern."""
+    n = int(np.prod(shape)) * torch.tensor([], dtype=dtype).element_size()
+    buf = torch.empty(n + 2 * guard, dtype=torch.uint8, device="cuda")
+    buf.fill_(0xA5)
+    t = buf[guard:guard + n].view(dtype).view(shape)
+    return buf, t
+
+
+def _guards_intact(buf, guard=4096):
+    return bool((buf[:guard] == 0xA5).all() and (buf[-guard:] == 0xA5).all())
+
+
+@pytest.mark.parametrize("impl,lengths,io", [
+    (gdn.GDN_IMPL_TENSOR_CORE, [70, 0, 1, 130], torch.bfloat16),
+    (gdn.GDN_IMPL_TENSOR_CORE_WHOLE_ROWS, [70, 0, 1, 130], torch.bfloat16),
+    (gdn.GDN_IMPL_TENSOR_CORE_SPLIT, [70, 0, 1, 130], torch.bfloat16),
+    (gdn.GDN_IMPL_CUDA_CORE, [70, 0, 1, 130], torch.float32)])
+def test_outputs_stay_inside_their_buffers(impl, lengths, io):
+    """Guard regions around o and the final states (a stand-in for a memory checker):
+    ragged tails, empty and one-token sequences write nothing outside the outputs."""
+    P = make_prefill_inputs(lengths, H_qk=2, H_v=4, d_k=128, d_v=128, io_dtype=io,
+                            state_std=0.05, seed=70)
+    Pd = P.to("cuda")
+    T, N = P.q.shape[0], P.num_seqs
+    ob, o = _guarded((T, 4, 128), io)
+    sb, Sf = _guarded((N, 4, 128, 128), torch.float32)
+    gdn_prefill(Pd.q, Pd.k, Pd.v, Pd.a, Pd.b, Pd.A_log, Pd.dt_bias, Pd.cu_seqlens,
+                Pd.initial_state, out=o, final_state=Sf, impl=impl)
+    assert gdn_sync_status() == 0
+    assert _guards_intact(ob) and _guards_intact(sb)
+    o_ref, S_ref = _full_oracle(P)
+    tol = TOL_BF16 if io == torch.bfloat16 else TOL_FP32
+    assert rel_err(o, o_ref) <= tol and rel_err(Sf, S_ref) <= tol

@@ -1,14 +1,15 @@
 """gdn_prefill_noalloc: the prefill for callers that cannot allocate device memory.
 
-Some callers cannot call cudaMalloc (code under CUDA graph stream capture, a
-runtime whose device memory is owned by its own pool, a plugin given only its
-input and output buffers), so they cannot hand gdn_prefill a workspace. This
-entry point keeps that scratch in a fixed array inside the library. The test
-calls it through the C ABI, twice in a row on different inputs (the array keeps
-the previous call's contents), and checks each result against gdn_prefill's
-within the parity tolerance. It also checks, on the host, that a call larger than
-the built-in scratch and calls with bad arguments are refused before anything is
-launched.
+Some callers cannot call cudaMalloc where they run the mixer (a runtime whose device
+memory is owned by its own pool, a plugin given only its input and output buffers,
+code where an allocation would block or synchronise the device), so they cannot hand
+gdn_prefill a workspace. This entry point keeps that scratch in a fixed array inside
+the library. The test calls it through the C ABI, twice in a row on different inputs
+(the array keeps the previous call's contents), and checks each result against the
+fp64 oracle and against gdn_prefill's, within the parity tolerance; once more at
+exactly the array's capacity. It also checks, on the host, that a call one element
+larger than the built-in scratch and calls with bad arguments are refused before
+anything is launched, and that a call at exactly the capacity passes the size check.
 
 This file is named so that pytest collects it last.
 """
@@ -17,6 +18,7 @@ import ctypes
 import pytest
 import torch
 
+import oracle
 from linear_attention_sequence_delta_b200 import gdn
 from linear_attention_sequence_delta_b200.inputs import make_prefill_inputs
 from tests.parity_util import TOL_BF16, TOL_FP32, rel_err
@@ -56,6 +58,19 @@ def test_refuses_more_than_the_builtin_scratch():
     st = _fn()(v(F), v(F), v(F), 0, v(F), v(F), v(F), v(F), None, v(F), 1, T, 16, H_v, 128, 128,
                1.0, v(F), None, None)
     assert st == 3  # GDN_ERR_WORKSPACE
+
+
+def test_capacity_is_inclusive():
+    # Exactly GDN_NOALLOC_MAX_GATE_ELEMS gate values pass the size check: with a
+    # misaligned q the call then stops at the pointer checks that follow it
+    # (GDN_ERR_INVALID_ARG, not GDN_ERR_WORKSPACE), still on the host.
+    F = 0x7F0000000000
+    v = ctypes.c_void_p
+    for H_v in (4, 32):
+        T = MAX_GATE_ELEMS // H_v
+        st = _fn()(v(F + 8), v(F), v(F), 0, v(F), v(F), v(F), v(F), None, v(F), 1, T, 2,
+                   H_v, 128, 128, 1.0, v(F), None, None)
+        assert st == 1, H_v
 
 
 @pytest.mark.parametrize("over,code", [
@@ -100,3 +115,26 @@ def test_noalloc_matches_gdn_prefill_twice(io):
         assert gdn.gdn_sync_status() == 0
         assert rel_err(o, o_ref.float().cpu().numpy()) <= tol
         assert rel_err(Sf, S_ref.cpu().numpy()) <= tol
+        Pc = P.to("cpu")
+        o_or, S_or = oracle.forward(Pc.q, Pc.k, Pc.v, Pc.a, Pc.b, Pc.A_log, Pc.dt_bias,
+                                    Pc.cu_seqlens.numpy(), Pc.initial_state, scale=0.7)
+        assert rel_err(o, o_or) <= tol
+        assert rel_err(Sf, S_or) <= tol
+
+
+@pytest.mark.gpu
+def test_noalloc_at_exactly_the_capacity():
+    """T * H_v == GDN_NOALLOC_MAX_GATE_ELEMS: the beta half of the array ends at its
+    last byte. 64 sequences of 4096 tokens, 4 V heads, d = 64, against the oracle."""
+    P = make_prefill_inputs([4096] * 64, H_qk=2, H_v=4, d_k=64, d_v=64, state_std=0.05,
+                            seed=33).to("cuda")
+    assert P.q.shape[0] * P.v.shape[1] == MAX_GATE_ELEMS
+    o = torch.full_like(P.v, float("nan"))
+    Sf = torch.full_like(P.initial_state, float("nan"))
+    assert _call(P, o, Sf) == 0
+    assert gdn.gdn_sync_status() == 0
+    Pc = P.to("cpu")
+    o_or, S_or = oracle.forward(Pc.q, Pc.k, Pc.v, Pc.a, Pc.b, Pc.A_log, Pc.dt_bias,
+                                Pc.cu_seqlens.numpy(), Pc.initial_state)
+    assert rel_err(o, o_or) <= TOL_BF16
+    assert rel_err(Sf, S_or) <= TOL_BF16
