@@ -178,49 +178,44 @@ __device__ __forceinline__ void tile_store(float* M, int s, int r0, int c0, cons
 
 // ==================================== prep ========================================
 constexpr int kPrepThreads = 256;
-constexpr int kTsStride = 68;
+constexpr int kTsStride = 68;  // rows of T and A: conflict-free as the A operand of the merges
 constexpr int kAsStride = 68;
-// shared memory map (bytes from a 1024-byte aligned base)
-constexpr uint32_t PS_KQ = 0;        // [2 col blocks][128 rows][128 B], raw K then Q, sw128
-constexpr uint32_t PS_TS = 32768;    // [64][68] fp32 T
-constexpr uint32_t PS_AS = 50176;    // [64][68] fp32 A (strictly-lower part used)
-constexpr uint32_t PS_XS = 67584;    // [1152] fp32 merge scratch
-constexpr uint32_t PS_AB = 72192;    // [2][kMaxGroup][64] fp32 a, b
-constexpr uint32_t PS_HS = 80384;    // per-head scratch: U [4][64]
-constexpr uint32_t PS_RK = 82816;    // [64] rk, [64] rq (rq includes the scale)
-constexpr uint32_t PS_GA = 83328;    // [kMaxGroup][64] G of every V head of the unit
-constexpr uint32_t PS_BA = 87424;    // [kMaxGroup][64] beta of every V head of the unit
-constexpr uint32_t PS_PAR = 91520;   // [2][kMaxGroup] A_log, dt_bias of those heads
-constexpr uint32_t PS_E = 91648;     // per head: [4][16][16] exp(G_i - G_j) inside 16-blocks
-constexpr uint32_t PS_CI = 95744;    // per head: [64] exp(G_i - G_{16-block start of i})
-constexpr uint32_t PS_BAR = 96000;   // mbarrier (MMA)
-constexpr uint32_t PS_TMEM = 96008;
-constexpr size_t kPrepSmem = 96016 + 1024;
+constexpr int kXsStride = 40;  // merge scratch: conflict-free as the B operand of the merges
+constexpr int kEStride = 20;   // rows of the in-block exponential table (16 used): the 8 lanes
+                               // of a 16-byte shared-memory access phase hit distinct banks
+// Shared memory map (bytes from a 1024-byte aligned base). The first 32 KB hold the raw
+// K and Q rows until the unit's MMA has read them; after that, A, the staging image of
+// P and the exponential tables of the V head being worked on.
+constexpr uint32_t PS_KQ = 0;      // [2 col blocks][128 rows][128 B], raw K then Q, sw128
+constexpr uint32_t PS_AS = 0;      // [64][68] fp32 A (strictly-lower part used)
+constexpr uint32_t PS_PST = 17408; // [64][128 B] P, bf16 sw128 image (the record's P)
+constexpr uint32_t PS_E = 25600;   // [4][16][20] exp(G_i - G_j) inside 16-blocks
+constexpr uint32_t PS_U = 30720;   // [4][64] exp(G_{16 a} - G_j)
+constexpr uint32_t PS_CI = 31744;  // [64] exp(G_i - G_{16-block start of i})
+constexpr uint32_t PS_TS = 32768;  // [64][68] fp32 T (entries above its diagonal blocks stay 0)
+constexpr uint32_t PS_XS = 50176;  // [32][40] fp32 merge scratch
+constexpr uint32_t PS_AB = 55296;  // [2][kMaxGroup][64] fp32 a, b
+constexpr uint32_t PS_GA = 63488;  // [kMaxGroup][64] G of every V head of the unit
+constexpr uint32_t PS_BA = 67584;  // [kMaxGroup][64] beta of every V head of the unit
+constexpr uint32_t PS_RK = 71680;  // [64] rk, [64] rq (rq includes the scale)
+constexpr uint32_t PS_PAR = 72192; // [2][kMaxGroup] A_log, dt_bias of those heads
+constexpr uint32_t PS_BAR = 72320; // mbarrier (MMA)
+constexpr uint32_t PS_TMEM = 72328;
+constexpr size_t kPrepSmem = 72336 + 1024;
+static_assert(PS_CI + 64 * 4 <= PS_TS, "the per-head area must fit where K and Q were");
 
-// Half a row (32 columns starting at 32 H) of A (row i < 64) or of P (row t =
-// i - 64) from the matching half row x of [K; Q] K^T. Columns left of the row's
-// 16-block use exp(G_i - G_j) = exp(G_i - G_a0) U_j (both factors <= 1); the at
-// most 16 columns inside the block take their own exponential; columns right of
-// the row are zero. rowf = beta_i rk_i (A) or rq_t (P); rk gives the column factor.
+// Half a row (32 columns from 32 H) of A (row i < 64, to the A matrix) or of P (row
+// t = i - 64, to the staging image) from the matching half row x of [K; Q] K^T, whose
+// columns are already scaled by rk. Columns left of the row's 16-block use
+// exp(G_i - G_j) = exp(G_i - G_a0) U_j (both factors <= 1); the at most 16 columns
+// inside the block take their own exponential; columns right of the row are zero.
+// rowf = beta_i rk_i (A) or rq_t (P).
 template <int H>
 __device__ __forceinline__ void ap_half_row(const float (&x)[32], int row, const float* U,
-                                            const float* E, const float* CI, const float* rk,
-                                            float rowf, float (&val)[32]) {
+                                            const float* E, const float* CI, float rowf,
+                                            float* As, uint8_t* Pst, bool live) {
     const int i = row & 63;
     const int a0 = i & ~15;
-    const float4* rk4 = reinterpret_cast<const float4*>(rk + 32 * H);
-    float cf[32];
-#pragma unroll
-    for (int e4 = 0; e4 < 8; ++e4) {
-        const float4 r4 = rk4[e4];
-        cf[4 * e4] = rowf * r4.x * x[4 * e4];
-        cf[4 * e4 + 1] = rowf * r4.y * x[4 * e4 + 1];
-        cf[4 * e4 + 2] = rowf * r4.z * x[4 * e4 + 2];
-        cf[4 * e4 + 3] = rowf * r4.w * x[4 * e4 + 3];
-    }
-    // The half's two 16-column groups each lie wholly left of the row's 16-block
-    // (exp(G_i - G_j) = ci U_j, both factors <= 1), on it (the block's own table, zero
-    // right of the diagonal) or right of it (zero).
 #pragma unroll
     for (int g = 0; g < 2; ++g) {
         const int c0 = 32 * H + 16 * g;
@@ -228,21 +223,57 @@ __device__ __forceinline__ void ap_half_row(const float (&x)[32], int row, const
         float f;
         if (c0 < a0) {
             t4 = reinterpret_cast<const float4*>(U + (a0 >> 4) * 64 + c0);
-            f = CI[i];
+            f = rowf * CI[i];
         } else {
-            t4 = reinterpret_cast<const float4*>(E + (a0 >> 4) * 256 + (i - a0) * 16);
-            f = c0 == a0 ? 1.f : 0.f;
+            t4 = reinterpret_cast<const float4*>(E + (a0 >> 4) * (16 * kEStride) +
+                                                 (i - a0) * kEStride);
+            f = c0 == a0 ? rowf : 0.f;
         }
+        float v[16];
 #pragma unroll
         for (int e4 = 0; e4 < 4; ++e4) {
             const float4 u = t4[e4];
             const int e = 16 * g + 4 * e4;
-            val[e] = f * u.x * cf[e];
-            val[e + 1] = f * u.y * cf[e + 1];
-            val[e + 2] = f * u.z * cf[e + 2];
-            val[e + 3] = f * u.w * cf[e + 3];
+            v[4 * e4] = f * u.x * x[e];
+            v[4 * e4 + 1] = f * u.y * x[e + 1];
+            v[4 * e4 + 2] = f * u.z * x[e + 2];
+            v[4 * e4 + 3] = f * u.w * x[e + 3];
+        }
+        if (row < 64) {
+            float4* Arow = reinterpret_cast<float4*>(As + i * kAsStride + c0);
+#pragma unroll
+            for (int e4 = 0; e4 < 4; ++e4)
+                Arow[e4] = make_float4(v[4 * e4], v[4 * e4 + 1], v[4 * e4 + 2], v[4 * e4 + 3]);
+        } else {
+#pragma unroll
+            for (int q2 = 0; q2 < 2; ++q2) {
+                uint4 w;
+                w.x = live ? pack_bf16x2(v[8 * q2 + 0], v[8 * q2 + 1]) : 0u;
+                w.y = live ? pack_bf16x2(v[8 * q2 + 2], v[8 * q2 + 3]) : 0u;
+                w.z = live ? pack_bf16x2(v[8 * q2 + 4], v[8 * q2 + 5]) : 0u;
+                w.w = live ? pack_bf16x2(v[8 * q2 + 6], v[8 * q2 + 7]) : 0u;
+                *reinterpret_cast<uint4*>(Pst + sw128_off((uint32_t)i, (uint32_t)(4 * H + 2 * g + q2))) = w;
+            }
         }
     }
+}
+
+// The exponential tables of one V head's G (the thread's share of them):
+//   U[a][j] = exp(G_{16 a} - G_j) for j < 16 a (both factors of a long gap are <= 1),
+//   E[b][ii][jj] = exp(G_{16 b + ii} - G_{16 b + jj}) for jj <= ii, else 0,
+//   CI[i] = exp(G_i - G_{16-block start of i}).
+__device__ __forceinline__ void exp_tables(const float* hG, float* sU, float* sE, float* sCI,
+                                           int tid) {
+    const int ab4 = tid >> 6, jj = tid & 63;
+    sU[tid] = (jj < 16 * ab4) ? __expf(hG[16 * ab4] - hG[jj]) : 0.f;
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+        const int idx = tid + kPrepThreads * q4;  // 0..1023
+        const int bb = idx >> 8, ii = (idx >> 4) & 15, jb = idx & 15;
+        sE[bb * (16 * kEStride) + ii * kEStride + jb] =
+            jb <= ii ? __expf(hG[16 * bb + ii] - hG[16 * bb + jb]) : 0.f;
+    }
+    if (tid < kC) sCI[tid] = __expf(hG[tid] - hG[tid & ~15]);
 }
 
 // Record (chunk cg, V head h) is complete: publish it to the chain (release). A flag
@@ -271,7 +302,8 @@ __device__ __forceinline__ void prep_worker(
     float* As = reinterpret_cast<float*>(sm + PS_AS);
     float* Xs = reinterpret_cast<float*>(sm + PS_XS);
     float* AB = reinterpret_cast<float*>(sm + PS_AB);
-    float* sU = reinterpret_cast<float*>(sm + PS_HS);  // [4][64] per-head exp table
+    float* sU = reinterpret_cast<float*>(sm + PS_U);   // per-head exp tables (see exp_tables)
+    uint8_t* Pst = sm + PS_PST;                        // P staging image
     float* rk = reinterpret_cast<float*>(sm + PS_RK);
     float* sGall = reinterpret_cast<float*>(sm + PS_GA);
     float* sBall = reinterpret_cast<float*>(sm + PS_BA);
@@ -422,59 +454,43 @@ __device__ __forceinline__ void prep_worker(
         if (!ok) failed = true;
         if (named_bar_any(bar_id, kPrepThreads, failed)) { failed = true; break; }
         tc_fence_after();
-        float x[32];  // this thread's half row of [K; Q] K^T, shared by the r V heads
+        // this thread's half row of [K; Q] K^T, shared by the r V heads, columns scaled
+        // by rk once for all of them
+        float x[32];
         tmem_ld32_sync(tl + 32 * hh, x);
+        {
+            const float4* rk4 = reinterpret_cast<const float4*>(rk + 32 * hh);
+#pragma unroll
+            for (int e4 = 0; e4 < 8; ++e4) {
+                const float4 r4 = rk4[e4];
+                x[4 * e4] *= r4.x;
+                x[4 * e4 + 1] *= r4.y;
+                x[4 * e4 + 2] *= r4.z;
+                x[4 * e4 + 3] *= r4.w;
+            }
+        }
+        // The K and Q rows have been read (norms, MMA): their area now takes A, the P
+        // staging image and the tables. The first head's tables get a phase of their own;
+        // every later head's are built while the head before writes its record.
+        exp_tables(sGall, sU, sE, sCI, tid);
+        named_bar_sync(bar_id, kPrepThreads);
 
 #pragma unroll 1
         for (int hr = 0; hr < r; ++hr) {
             const int h = j * r + hr;
             uint8_t* R = rec + ((size_t)cg * H_v + h) * kRecBytes;
-            const float* hG = sGall + hr * kC;     // this head's G
-            const float* hBeta = sBall + hr * kC;  // and beta
-            {  // U[a][j] = exp(G_{16 a} - G_j) for j < 16 a (both factors of a long gap <= 1)
-                const int ab4 = tid >> 6, jj = tid & 63;
-                sU[tid] = (jj < 16 * ab4) ? __expf(hG[16 * ab4] - hG[jj]) : 0.f;
-                // E[b][ii][jj] = exp(G_{16b+ii} - G_{16b+jj}) for jj <= ii, else 0
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const int idx = tid + kPrepThreads * q4;  // 0..1023
-                    const int bb = idx >> 8, ii = (idx >> 4) & 15, jb = idx & 15;
-                    sE[idx] = jb <= ii ? __expf(hG[16 * bb + ii] - hG[16 * bb + jb]) : 0.f;
-                }
-                if (tid < kC) sCI[tid] = __expf(hG[tid] - hG[tid & ~15]);
-            }
-            named_bar_sync(bar_id, kPrepThreads);
+            const float* hBeta = sBall + hr * kC;  // this head's beta
 
-            // ---- A rows 0-63 -> As (fp32); P rows 64-127 -> record (bf16 image) --------
+            // ---- A rows 0-63 -> As (fp32); P rows 64-127 -> staging (bf16 image);
+            // then the 8x8 diagonal blocks of T by forward substitution in registers,
+            // by the two warps that wrote the A rows those blocks read (rows 0-31,
+            // columns 0-31: warp 0; rows 32-63, columns 32-63: warp 5), no barrier between
             {
-                float val[32];
                 const int i = trow & 63;
                 const float rowf = trow < 64 ? hBeta[i] * rk[i] : rq[i];
-                if (hh == 0) ap_half_row<0>(x, trow, sU, sE, sCI, rk, rowf, val);
-                else         ap_half_row<1>(x, trow, sU, sE, sCI, rk, rowf, val);
-                if (trow < 64) {
-                    float4* Arow = reinterpret_cast<float4*>(As + i * kAsStride + 32 * hh);
-#pragma unroll
-                    for (int e4 = 0; e4 < 8; ++e4)
-                        Arow[e4] = make_float4(val[4 * e4], val[4 * e4 + 1], val[4 * e4 + 2],
-                                               val[4 * e4 + 3]);
-                } else {
-                    const bool live = i < L;
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        uint4 w;
-                        w.x = live ? pack_bf16x2(val[8 * q4 + 0], val[8 * q4 + 1]) : 0u;
-                        w.y = live ? pack_bf16x2(val[8 * q4 + 2], val[8 * q4 + 3]) : 0u;
-                        w.z = live ? pack_bf16x2(val[8 * q4 + 4], val[8 * q4 + 5]) : 0u;
-                        w.w = live ? pack_bf16x2(val[8 * q4 + 6], val[8 * q4 + 7]) : 0u;
-                        *reinterpret_cast<uint4*>(R + REC_P + sw128_off((uint32_t)i, 4 * hh + q4)) = w;
-                    }
-                }
+                if (hh == 0) ap_half_row<0>(x, trow, sU, sE, sCI, rowf, As, Pst, i < L);
+                else         ap_half_row<1>(x, trow, sU, sE, sCI, rowf, As, Pst, i < L);
             }
-            named_bar_sync(bar_id, kPrepThreads);
-
-            // ---- 8x8 diagonal blocks of T: forward substitution in registers -------
-            // rows 0-31 from warp 0 (columns 0-31), rows 32-63 from warp 5 (32-63)
             if (warp == 0 || warp == 5) {
                 const int i = trow;
                 const int rr = i & 7;
@@ -521,26 +537,25 @@ __device__ __forceinline__ void prep_worker(
             }
             named_bar_sync(bar_id, kPrepThreads);
             // ---- doubling 16 -> 32 (two 32-blocks) and 32 -> 64, tf32 tensor cores ----
-            // T_10 = -T_11 (A_10 T_00): X = A_10 T_00 goes through Xs (row stride 40)
-            constexpr int kXs = 36;
+            // T_10 = -T_11 (A_10 T_00): X = A_10 T_00 goes through Xs
             {
                 // 16 -> 32: warp w < 4: block b = w >> 1 (rows 32 b + 16 ..), column tile w & 1
                 if (warp < 4) {
                     const int b = warp >> 1, nt = warp & 1;
-                    const int R = 32 * b;
+                    const int Rb = 32 * b;
                     float d[4] = {0.f, 0.f, 0.f, 0.f};
-                    tile_mma_tf32(d, As, kAsStride, Ts, kTsStride, R + 16, R + 8 * nt, R, 16, lane);
-                    tile_store(Xs + b * 16 * kXs, kXs, 0, 8 * nt, d, 1.f, lane);
+                    tile_mma_tf32(d, As, kAsStride, Ts, kTsStride, Rb + 16, Rb + 8 * nt, Rb, 16, lane);
+                    tile_store(Xs + b * 16 * kXsStride, kXsStride, 0, 8 * nt, d, 1.f, lane);
                 }
                 named_bar_sync(bar_id, kPrepThreads);
                 if (warp < 4) {
                     const int b = warp >> 1, nt = warp & 1;
-                    const int R = 32 * b;
+                    const int Rb = 32 * b;
                     float d[4] = {0.f, 0.f, 0.f, 0.f};
-                    // rows R+16.. of T (its 16-block, columns R+16..R+31) times X (16 x 16)
-                    tile_mma_tf32(d, Ts + R + 16, kTsStride, Xs + b * 16 * kXs, kXs, R + 16,
-                                  8 * nt, 0, 16, lane);
-                    tile_store(Ts, kTsStride, R + 16, R + 8 * nt, d, -1.f, lane);
+                    // rows Rb+16.. of T (its 16-block, columns Rb+16..Rb+31) times X (16 x 16)
+                    tile_mma_tf32(d, Ts + Rb + 16, kTsStride, Xs + b * 16 * kXsStride, kXsStride,
+                                  Rb + 16, 8 * nt, 0, 16, lane);
+                    tile_store(Ts, kTsStride, Rb + 16, Rb + 8 * nt, d, -1.f, lane);
                 }
             }
             named_bar_sync(bar_id, kPrepThreads);
@@ -549,16 +564,17 @@ __device__ __forceinline__ void prep_worker(
                 const int mt = warp >> 2, nt = warp & 3;
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
                 tile_mma_tf32(d, As, kAsStride, Ts, kTsStride, 32 + 16 * mt, 8 * nt, 0, 32, lane);
-                tile_store(Xs, kXs, 16 * mt, 8 * nt, d, 1.f, lane);
+                tile_store(Xs, kXsStride, 16 * mt, 8 * nt, d, 1.f, lane);
                 named_bar_sync(bar_id, kPrepThreads);
                 float e[4] = {0.f, 0.f, 0.f, 0.f};
                 // T[32:64, 0:32] = -T[32:64, 32:64] X
-                tile_mma_tf32(e, Ts + 32, kTsStride, Xs, kXs, 32 + 16 * mt, 8 * nt, 0, 32, lane);
+                tile_mma_tf32(e, Ts + 32, kTsStride, Xs, kXsStride, 32 + 16 * mt, 8 * nt, 0, 32, lane);
                 tile_store(Ts, kTsStride, 32 + 16 * mt, 8 * nt, e, -1.f, lane);
             }
             named_bar_sync(bar_id, kPrepThreads);
 
-            // ---- T -> record (bf16 sw128 image) ----------------------------------------
+            // ---- T diag(beta) -> record (bf16 sw128 image), the staged P -> record, both
+            // as coalesced 16-byte stores; the next head's tables meanwhile -------------
 #pragma unroll
             for (int it = 0; it < 2; ++it) {
                 const int idx = tid + kPrepThreads * it;  // 0..511
@@ -573,8 +589,10 @@ __device__ __forceinline__ void prep_worker(
                 w.z = pack_bf16x2(f1.x * b1.x, f1.y * b1.y);
                 w.w = pack_bf16x2(f1.z * b1.z, f1.w * b1.w);
                 *reinterpret_cast<uint4*>(R + REC_T + sw128_off(row, ch)) = w;
+                reinterpret_cast<uint4*>(R + REC_P)[idx] = reinterpret_cast<const uint4*>(Pst)[idx];
             }
-            named_bar_sync(bar_id, kPrepThreads);  // Ts, As, Xs and the head scratch are reused
+            if (hr + 1 < r) exp_tables(sGall + (hr + 1) * kC, sU, sE, sCI, tid);
+            named_bar_sync(bar_id, kPrepThreads);  // Ts, As, Xs, the staging and tables are reused
             if (flags && tid == 0) publish_record(flags, (size_t)cg * H_v + h, epoch);
         }
         tc_fence_before();  // this unit's TMEM reads precede the next unit's MMA
@@ -586,7 +604,8 @@ __device__ __forceinline__ void prep_worker(
     if (warp == 0) tmem_dealloc(tmem, tcols);
 }
 
-__global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(
+constexpr int kPrepBlocksPerSm = 3;
+__global__ void __launch_bounds__(kPrepThreads, kPrepBlocksPerSm) prep_kernel(
     const bf16* __restrict__ q, const bf16* __restrict__ k, const float* __restrict__ a,
     const float* __restrict__ b, const float* __restrict__ A_log,
     const float* __restrict__ dt_bias, const int32_t* __restrict__ cu_seqlens,
@@ -1357,7 +1376,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
 // call's number before its bulk copy, and prep workers never wait on chains, so
 // every wait ends. Nothing in the workspace needs clearing between calls.
 constexpr int kFusedThreads = 512;
-constexpr uint32_t kPrepRegion = 96256;
+constexpr uint32_t kPrepRegion = 73728;
 static_assert(kPrepRegion + 1024 >= kPrepSmem, "prep worker region too small");
 constexpr size_t kFusedSmem =
     kChainSmem > 2 * (size_t)kPrepRegion + 1024 ? kChainSmem : 2 * (size_t)kPrepRegion + 1024;
@@ -1600,6 +1619,9 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
     e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kPrepSmem);
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kChainSmem);
     if (e != cudaSuccess) return e;
@@ -1608,8 +1630,11 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     timer_after(opt.timer, s, "chunk_offsets");
+    // Prep workers never wait on one another, so any grid size is safe: one wave of
+    // them at the residency the launch bounds ask for (the shared-memory carveout is
+    // set to its maximum so that it is reached).
     const int64_t unit_bound = (((T + kC - 1) / kC) + N) * (int64_t)H_qk;
-    const int64_t grid_cap = (int64_t)2 * num_sms;
+    const int64_t grid_cap = (int64_t)kPrepBlocksPerSm * num_sms;
     const int prep_grid = (int)(unit_bound < grid_cap ? unit_bound : grid_cap);
     if (prep_grid > 0) {
         timer_before(opt.timer, s);
