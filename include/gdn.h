@@ -406,6 +406,55 @@ int gdn_rmsnorm_gated(const void* o, const void* z, int32_t io_dtype, const floa
                       float eps, int64_t rows, int32_t d, void* y, void* stream);
 
 /*
+ * gdn_mixer_prefill -- the GDN token mixer's core over a packed batch in one call:
+ * the causal depthwise conv1d + SiLU over the concatenated q/k/v channels, the gated
+ * delta rule, and the gated RMSNorm of its output ("Qwen3.5-MoE-35B-A3B architecture
+ * teardown", section 3.3 phases 2-4 and 3.4 for the conv cache; "Qwen3.5 observation
+ * notes", "Qwen3_5MoeGatedDeltaNet": causal_conv1d_fn on mixed_qkv, the split into q, k,
+ * v, chunk_gated_delta_rule, then self.norm(core_attn_out, z)). It computes
+ *   [q | k | v] = gdn_conv1d_silu(x)   (q, k, v rounded to io_dtype)
+ *   o           = gdn_prefill(q, k, v, a, b, ...)
+ *   y           = gdn_rmsnorm_gated(o, z)
+ * with the same conventions as those three calls:
+ *   x               [T, conv_dim] io_dtype, conv_dim = (2 H_qk + H_v) d; channels
+ *                   q (H_qk heads of d) | k (H_qk heads) | v (H_v heads)     (in)
+ *   conv_weight     [conv_dim, K] fp32, conv_bias [conv_dim] fp32 or NULL     (in)
+ *   conv_state_in   [N, K-1, conv_dim] io_dtype or NULL (zeros)               (in)
+ *   conv_state_out  [N, K-1, conv_dim] io_dtype or NULL; may be conv_state_in (out)
+ *   kernel_size     K in {2, 3, 4}
+ *   a, b, A_log, dt_bias, initial_state, cu_seqlens, scale: as gdn_prefill
+ *   z               [T, H_v, d] io_dtype, the output gate                     (in)
+ *   norm_weight     [d] fp32; eps >= 0                                        (in)
+ *   y               [T, H_v, d] io_dtype; must not be x or z                  (out)
+ *   final_state     [N, H_v, d, d] fp32 or NULL                               (out)
+ *   workspace       >= gdn_mixer_prefill_workspace_size(...) bytes, 256-byte aligned:
+ *                   the post-conv q | k | v ([T, conv_dim] io_dtype), then the
+ *                   prefill's workspace
+ *   options         as gdn_prefill_ex, or NULL
+ * For bf16 with d = 128 (at most 16 V heads per QK head) the steps are fused into the
+ * tensor-core prefill: its preparation stage reads x (with each sequence's K-1 earlier
+ * positions from the conv cache), convolves the q and k channels it needs itself and
+ * writes all post-conv channels once for the chain stage, which applies the gated norm
+ * to each tile of o before it is stored, and writes the conv cache at the end of each
+ * sequence. The convolution's arithmetic is that of gdn_conv1d_silu (bit for bit);
+ * the norm's sum of squares is taken in another order than gdn_rmsnorm_gated's. For
+ * other shapes and types (and with GDN_IMPL_CUDA_CORE) the call runs the convolution,
+ * the CUDA-core prefill and the norm one after another on the same buffers.
+ */
+size_t gdn_mixer_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t H_qk,
+                                        int32_t H_v, int32_t d_k, int32_t d_v,
+                                        int32_t io_dtype);
+int gdn_mixer_prefill(const void* x, int32_t io_dtype, const float* conv_weight,
+                      const float* conv_bias, const void* conv_state_in, void* conv_state_out,
+                      int32_t kernel_size, const float* a, const float* b, const float* A_log,
+                      const float* dt_bias, const float* initial_state,
+                      const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                      int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v, float scale,
+                      const void* z, const float* norm_weight, float eps, void* y,
+                      float* final_state, void* workspace, size_t workspace_bytes,
+                      const gdn_prefill_options* options, void* stream);
+
+/*
  * Synchronise `stream`, then return and clear the device status word of the
  * current device (GDN_OK, GDN_ERR_BAD_SEQLENS, GDN_ERR_BAD_SLOT or GDN_ERR_TIMEOUT), or
  * GDN_ERR_CUDA if the synchronisation itself failed.

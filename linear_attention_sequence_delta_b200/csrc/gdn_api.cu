@@ -276,6 +276,130 @@ int gdn_prefill_slots_ex(const void* q, const void* k, const void* v, int32_t io
                                 workspace_bytes, options, stream);
 }
 
+size_t gdn_mixer_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t H_qk,
+                                        int32_t H_v, int32_t d_k, int32_t d_v,
+                                        int32_t io_dtype) {
+    if (io_dtype != GDN_BF16 && io_dtype != GDN_FP32) return 0;
+    const size_t pre = gdn_prefill_workspace_size(num_seqs, total_tokens, H_qk, H_v, d_k, d_v);
+    if (pre == 0) return 0;
+    const size_t conv_dim = (size_t)(2 * H_qk + H_v) * d_k;
+    const size_t s = io_dtype == GDN_BF16 ? 2 : 4;
+    return align_up((size_t)total_tokens * conv_dim * s, 256) + pre;
+}
+
+int gdn_mixer_prefill(const void* x, int32_t io_dtype, const float* conv_weight,
+                      const float* conv_bias, const void* conv_state_in, void* conv_state_out,
+                      int32_t kernel_size, const float* a, const float* b, const float* A_log,
+                      const float* dt_bias, const float* initial_state,
+                      const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                      int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v, float scale,
+                      const void* z, const float* norm_weight, float eps, void* y,
+                      float* final_state, void* workspace, size_t workspace_bytes,
+                      const gdn_prefill_options* options, void* stream) {
+    PrefillOpts opt;
+    if (options) {
+        if (options->impl < GDN_IMPL_AUTO || options->impl > GDN_IMPL_TENSOR_CORE_WHOLE_ROWS)
+            return GDN_ERR_INVALID_ARG;
+        if (options->fault != GDN_FAULT_NONE && options->fault != GDN_FAULT_WITHHOLD_RECORDS)
+            return GDN_ERR_INVALID_ARG;
+        if (options->wait_limit_cycles < 0) return GDN_ERR_INVALID_ARG;
+        opt.impl = options->impl;
+        opt.fault = options->fault;
+        if (options->wait_limit_cycles > 0) opt.wait_cycles = options->wait_limit_cycles;
+        opt.timer = options->timer;
+    }
+    if (io_dtype != GDN_BF16 && io_dtype != GDN_FP32) return GDN_ERR_INVALID_ARG;
+    if (num_seqs < 0 || total_tokens < 0) return GDN_ERR_INVALID_ARG;
+    if (num_seqs == 0 && total_tokens != 0) return GDN_ERR_INVALID_ARG;
+    int hs = check_heads(H_qk, H_v, d_k, d_v);
+    if (hs != GDN_OK) return hs;
+    if (kernel_size < 2 || kernel_size > 4) return GDN_ERR_UNSUPPORTED;
+    if (!isfinite(scale) || !(eps >= 0.f) || !isfinite(eps)) return GDN_ERR_INVALID_ARG;
+    if (num_seqs == 0) return GDN_OK;
+    if ((int64_t)num_seqs * H_v * (d_v / 32) >= (int64_t)1 << 31) return GDN_ERR_UNSUPPORTED;
+    if (!cu_seqlens || !A_log || !dt_bias || !conv_weight || !norm_weight)
+        return GDN_ERR_INVALID_ARG;
+    if (total_tokens > 0 && (!x || !a || !b || !z || !y)) return GDN_ERR_INVALID_ARG;
+    const void* ptrs16[] = {x, z, y, conv_weight, norm_weight, conv_state_in, conv_state_out,
+                            initial_state, final_state};
+    for (const void* p : ptrs16)
+        if (!aligned(p, 16)) return GDN_ERR_INVALID_ARG;
+    if (!aligned(a, 4) || !aligned(b, 4) || !aligned(conv_bias, 4)) return GDN_ERR_INVALID_ARG;
+    if (y && (y == x || y == z)) return GDN_ERR_INVALID_ARG;  // y is written while x, z are read
+    const size_t need = gdn_mixer_prefill_workspace_size(num_seqs, total_tokens, H_qk, H_v,
+                                                         d_k, d_v, io_dtype);
+    if (workspace_bytes < need || !workspace || !aligned(workspace, 256)) return GDN_ERR_WORKSPACE;
+
+    const int conv_dim = (2 * H_qk + H_v) * d_k;
+    const size_t s_io = io_dtype == GDN_BF16 ? 2 : 4;
+    uint8_t* wb = static_cast<uint8_t*>(workspace);
+    void* qkvc = wb;  // [T][conv_dim] post-conv q | k | v
+    void* pre_ws = wb + align_up((size_t)total_tokens * conv_dim * s_io, 256);
+    const bool tc_ok = io_dtype == GDN_BF16 && d_k == 128 && prefill_tc_supported(H_qk, H_v);
+    const bool tc_forced = opt.impl == GDN_IMPL_TENSOR_CORE ||
+                           opt.impl == GDN_IMPL_TENSOR_CORE_SPLIT ||
+                           opt.impl == GDN_IMPL_TENSOR_CORE_WHOLE_ROWS;
+    if (tc_forced && !tc_ok) return GDN_ERR_UNSUPPORTED;
+    int* st = device_status_ptr();
+    if (!st) return GDN_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (opt.timer) opt.timer->n = 0;
+    if (tc_ok && opt.impl != GDN_IMPL_CUDA_CORE) {
+        // one fused path: the convolution in the preparation's loads, the gated norm in
+        // the chain's output
+        MixerFusion mix;
+        mix.x = static_cast<const __nv_bfloat16*>(x);
+        mix.conv_w = conv_weight;
+        mix.conv_b = conv_bias;
+        mix.cache_in = static_cast<const __nv_bfloat16*>(conv_state_in);
+        mix.cache_out = static_cast<__nv_bfloat16*>(conv_state_out);
+        mix.qkvc = static_cast<__nv_bfloat16*>(qkvc);
+        mix.conv_dim = conv_dim;
+        mix.K = kernel_size;
+        mix.z = static_cast<const __nv_bfloat16*>(z);
+        mix.norm_w = norm_weight;
+        mix.eps = eps;
+        return to_status(launch_prefill_tc(nullptr, nullptr, nullptr, a, b, A_log, dt_bias,
+                                           initial_state, cu_seqlens, num_seqs, total_tokens,
+                                           H_qk, H_v, scale, y, final_state, StateIndex{}, pre_ws,
+                                           opt, st, s, mix));
+    }
+    // The three steps one after another: the convolution into the workspace, the
+    // CUDA-core prefill reading q, k and v there with o written to y, the norm in place.
+    timer_before(opt.timer, s);
+    if (launch_conv1d_silu(x, io_dtype, conv_weight, conv_bias, conv_state_in, cu_seqlens,
+                           num_seqs, total_tokens, conv_dim, kernel_size, qkvc, conv_state_out,
+                           st, s) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    timer_after(opt.timer, s, "conv1d_silu");
+    float* G = static_cast<float*>(pre_ws);
+    float* beta = reinterpret_cast<float*>(static_cast<char*>(pre_ws) +
+                                           gate_bytes(total_tokens, H_v));
+    if (total_tokens > 0) {
+        timer_before(opt.timer, s);
+        if (launch_gates(a, b, A_log, dt_bias, cu_seqlens, num_seqs, total_tokens, H_v, G,
+                         nullptr, beta, st, s) != cudaSuccess)
+            return GDN_ERR_CUDA;
+        timer_after(opt.timer, s, "gates");
+    }
+    const char* qc = static_cast<const char*>(qkvc);
+    timer_before(opt.timer, s);
+    if (launch_prefill_simt(qc, qc + (size_t)H_qk * d_k * s_io, qc + (size_t)2 * H_qk * d_k * s_io,
+                            io_dtype, G, beta, initial_state, cu_seqlens, num_seqs, total_tokens,
+                            H_qk, H_v, d_k, scale, y, final_state, StateIndex{}, st, s, conv_dim,
+                            conv_dim) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    timer_after(opt.timer, s, "prefill_simt");
+    if (total_tokens > 0) {
+        timer_before(opt.timer, s);
+        if (launch_rmsnorm_gated(y, z, io_dtype, norm_weight, eps, total_tokens * H_v, d_v, y, s) !=
+            cudaSuccess)
+            return GDN_ERR_CUDA;
+        timer_after(opt.timer, s, "rmsnorm_gated");
+    }
+    return GDN_OK;
+}
+
 int gdn_decode_step(const void* q, const void* k, const void* v, int32_t io_dtype,
                     const float* a, const float* b, const float* A_log, const float* dt_bias,
                     float* state, int32_t num_seqs, int32_t H_qk, int32_t H_v, int32_t d_k,

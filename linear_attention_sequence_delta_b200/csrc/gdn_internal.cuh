@@ -90,6 +90,22 @@ struct StateIndex {
     }
 };
 
+// The steps around the delta rule that gdn_mixer_prefill fuses into the tensor-core
+// prefill's kernels: the causal depthwise convolution + SiLU in the preparation's loads
+// of q, k and v (x != nullptr), and the gated RMSNorm in the chain's output (z != nullptr).
+struct MixerFusion {
+    const __nv_bfloat16* x = nullptr;         // [T][conv_dim] pre-conv, channels q | k | v
+    const float* conv_w = nullptr;            // [conv_dim][K]
+    const float* conv_b = nullptr;            // [conv_dim] or null
+    const __nv_bfloat16* cache_in = nullptr;  // [N][K-1][conv_dim] or null (zeros)
+    __nv_bfloat16* cache_out = nullptr;       // [N][K-1][conv_dim] or null
+    __nv_bfloat16* qkvc = nullptr;            // [T][conv_dim] post-conv q, k, v (workspace)
+    int conv_dim = 0, K = 0;
+    const __nv_bfloat16* z = nullptr;         // [T][H_v][d] output gate
+    const float* norm_w = nullptr;            // [d]
+    float eps = 0.f;
+};
+
 // ---- host launchers (one per kernel family) ----------------------------------
 
 // Status word of the current device (a __device__ int of this library).
@@ -136,11 +152,14 @@ cudaError_t launch_decode_multi(const void* q, const void* k, const void* v, int
                                 int32_t H_v, int32_t d, float scale, void* o, float* inter,
                                 int* status, cudaStream_t s);
 
+// qk_tok, v_tok: elements from one token's q (k) rows to the next token's, and v's
+// (H_qk d and H_v d for dense [T, H, d] tensors; larger for strided views).
 cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, int io_dtype,
                                 const float* G, const float* beta, const float* S0,
                                 const int32_t* cu_seqlens, int32_t N, int64_t T, int32_t H_qk,
                                 int32_t H_v, int32_t d, float scale, void* o, float* S_final,
-                                StateIndex sref, int* status, cudaStream_t s);
+                                StateIndex sref, int* status, cudaStream_t s,
+                                int64_t qk_tok = 0, int64_t v_tok = 0);
 
 // Tensor-core prefill (bf16 I/O, d = 128): chunk offsets, the state-independent
 // prep kernel, then the chain kernel, or both stages in one cooperative launch where
@@ -154,7 +173,7 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
                               const float* S0, const int32_t* cu_seqlens, int32_t N, int64_t T,
                               int32_t H_qk, int32_t H_v, float scale, void* o, float* S_final,
                               StateIndex sref, void* workspace, const PrefillOpts& opt,
-                              int* status, cudaStream_t s);
+                              int* status, cudaStream_t s, const MixerFusion& mix = MixerFusion{});
 
 // Steps around the delta rule (gdn_mixer.cu): causal depthwise conv1d + SiLU with
 // the per-sequence conv cache, its single-token decode form, and the gated RMSNorm.

@@ -57,7 +57,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_simt_kernel(
     const float* __restrict__ Gcs, const float* __restrict__ beta,
     const float* S0, const int32_t* __restrict__ cu_seqlens, int64_t T_total,
     int H_qk, int H_v, float scale, IO* __restrict__ o, float* S_final, StateIndex sref,
-    int* status) {
+    int* status, int64_t qk_tok, int64_t v_tok) {
     using L = SimtSmem<D, DVS>;
     constexpr int KP = L::KP, CP = L::CP;
     constexpr int NSL = D / DVS;
@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_simt_kernel(
             const int t = idx / D, c = idx % D;
             float kv = 0.f, qv = 0.f;
             if (t < Lc) {
-                const size_t gi = ((size_t)(t0 + t) * H_qk + j) * D + c;
+                const size_t gi = (size_t)(t0 + t) * qk_tok + (size_t)j * D + c;
                 kv = to_f32(k[gi]);
                 qv = to_f32(q[gi]);
             }
@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_simt_kernel(
         }
         for (int idx = tid; idx < kC * DVS; idx += kThreads) {
             const int t = idx / DVS, c = idx % DVS;
-            Vs[idx] = t < Lc ? to_f32(v[((size_t)(t0 + t) * H_v + h) * D + dv0 + c]) : 0.f;
+            Vs[idx] = t < Lc ? to_f32(v[(size_t)(t0 + t) * v_tok + (size_t)h * D + dv0 + c]) : 0.f;
         }
         if (tid < kC) {
             const bool ok = tid < Lc;
@@ -349,7 +349,8 @@ template <typename IO, int D, int DVS>
 cudaError_t launch_simt_t(const void* q, const void* k, const void* v, const float* G,
                           const float* beta, const float* S0, const int32_t* cu, int32_t N,
                           int64_t T, int32_t H_qk, int32_t H_v, float scale, void* o,
-                          float* S_final, StateIndex sref, int* status, cudaStream_t s) {
+                          float* S_final, StateIndex sref, int* status, cudaStream_t s,
+                          int64_t qk_tok, int64_t v_tok) {
     using L = SimtSmem<D, DVS>;
     auto kern = prefill_simt_kernel<IO, D, DVS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -359,7 +360,7 @@ cudaError_t launch_simt_t(const void* q, const void* k, const void* v, const flo
     if (blocks == 0) return cudaSuccess;
     kern<<<(unsigned)blocks, kThreads, L::bytes, s>>>(
         static_cast<const IO*>(q), static_cast<const IO*>(k), static_cast<const IO*>(v), G, beta,
-        S0, cu, T, H_qk, H_v, scale, static_cast<IO*>(o), S_final, sref, status);
+        S0, cu, T, H_qk, H_v, scale, static_cast<IO*>(o), S_final, sref, status, qk_tok, v_tok);
     return cudaGetLastError();
 }
 
@@ -369,10 +370,13 @@ cudaError_t launch_prefill_simt(const void* q, const void* k, const void* v, int
                                 const float* G, const float* beta, const float* S0,
                                 const int32_t* cu_seqlens, int32_t N, int64_t T, int32_t H_qk,
                                 int32_t H_v, int32_t d, float scale, void* o, float* S_final,
-                                StateIndex sref, int* status, cudaStream_t s) {
+                                StateIndex sref, int* status, cudaStream_t s, int64_t qk_tok,
+                                int64_t v_tok) {
+    if (qk_tok == 0) qk_tok = (int64_t)H_qk * d;
+    if (v_tok == 0) v_tok = (int64_t)H_v * d;
 #define GDN_SIMT(IO, D)                                                                      \
     return launch_simt_t<IO, D, 32>(q, k, v, G, beta, S0, cu_seqlens, N, T, H_qk, H_v, scale, \
-                                    o, S_final, sref, status, s)
+                                    o, S_final, sref, status, s, qk_tok, v_tok)
     if (io_dtype == GDN_BF16) {
         if (d == 128) GDN_SIMT(__nv_bfloat16, 128);
         GDN_SIMT(__nv_bfloat16, 64);

@@ -276,6 +276,109 @@ __device__ __forceinline__ void exp_tables(const float* hG, float* sU, float* sE
     if (tid < kC) sCI[tid] = __expf(hG[tid] - hG[tid & ~15]);
 }
 
+__device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.f + __expf(-x)); }
+
+// SiLU with one special-function operation: x sigmoid(x), sigmoid(x) = (1 + tanh(x/2)) / 2,
+// tanh from the hardware's approximation (relative error about 2^-11, below half a bf16 ulp).
+__device__ __forceinline__ float silu_tanh(float x) {
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+    return x * fmaf(0.5f, t, 0.5f);
+}
+
+// The causal depthwise convolution + SiLU of one unit's channels ("Qwen3.5-MoE-35B-A3B
+// architecture teardown", 3.3 phase 2: conv over the concatenated q/k/v channels, kernel
+// K, then SiLU): the q and k channels of QK head j and the v channels of its r V heads,
+// for the chunk's tokens t0 .. t0+L-1 of sequence n (which starts at s0). Positions
+// before the sequence's start come from the conv cache (zeros without one). q and k go
+// to the K/Q tile in shared memory (rows past L zero), and every channel to the post-conv
+// buffer that the chain's tile loads read. The arithmetic (bias, then the taps oldest
+// first with fused multiply-adds, then SiLU, one rounding to bf16) is that of the
+// standalone convolution kernel, so both give the same bits. A thread takes 4 channels x
+// 8 tokens at a time; consecutive threads take consecutive channel groups.
+__device__ __forceinline__ void conv_unit(const MixerFusion& mix, int n, int64_t s0, int64_t t0,
+                                          int L, int j, int r, int H_qk, uint8_t* KQ, int tid) {
+    const int C = mix.conv_dim, K = mix.K;
+    const int nv4 = 64 + 32 * r;  // 4-channel groups: q 32, k 32, v 32 per V head
+    const int items = nv4 * 8;    // x 8 segments of 8 tokens
+    // item -> (first channel, first token) and its input window: positions
+    // p = t0 + tt0 - (K-1) + s, s = 0 .. 6 + K, 4 bf16 (8 bytes) each
+    auto locate = [&](int item, int& c, int& v4, int& tt0) {
+        const int seg = item / nv4;
+        v4 = item - seg * nv4;
+        tt0 = seg * 8;
+        if (v4 < 32) c = j * kD + 4 * v4;
+        else if (v4 < 64) c = H_qk * kD + j * kD + 4 * (v4 - 32);
+        else c = 2 * H_qk * kD + (j * r + ((v4 - 64) >> 5)) * kD + 4 * ((v4 - 64) & 31);
+    };
+    auto load = [&](int c, int tt0, uint2 (&raw)[11]) {
+#pragma unroll
+        for (int s_ = 0; s_ < 11; ++s_) {
+            raw[s_] = make_uint2(0u, 0u);
+            const int64_t p = t0 + tt0 - (K - 1) + s_;
+            if (s_ < 7 + K && p < t0 + L) {
+                if (p >= s0)
+                    raw[s_] = *reinterpret_cast<const uint2*>(mix.x + (size_t)p * C + c);
+                else if (mix.cache_in)
+                    raw[s_] = *reinterpret_cast<const uint2*>(
+                        mix.cache_in + ((size_t)n * (K - 1) + (K - 1) + (p - s0)) * C + c);
+            }
+        }
+    };
+    auto compute = [&](int c, int v4, int tt0, const uint2 (&raw)[11]) {
+        float w[4][4], bs[4];  // w[e][i]: tap i (oldest first) of channel c + e
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            bs[e] = mix.conv_b ? mix.conv_b[c + e] : 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) w[e][i] = i < K ? mix.conv_w[(size_t)(c + e) * K + i] : 0.f;
+        }
+        const int cc = (v4 & 31) * 4;  // channel within the head (q, k)
+        uint8_t* kq = KQ + (uint32_t)(cc >> 6) * 16384u + (uint32_t)((cc >> 2) & 1) * 8u;
+        const int row0 = v4 < 32 ? 64 : 0;  // Q rows 64-127, K rows 0-63
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            float acc[4] = {bs[0], bs[1], bs[2], bs[3]};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                if (i < K) {
+                    const uint2 rw = raw[u + i];
+                    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&rw.x));
+                    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&rw.y));
+                    acc[0] = fmaf(w[0][i], lo.x, acc[0]);
+                    acc[1] = fmaf(w[1][i], lo.y, acc[1]);
+                    acc[2] = fmaf(w[2][i], hi.x, acc[2]);
+                    acc[3] = fmaf(w[3][i], hi.y, acc[3]);
+                }
+            }
+            const int tt = tt0 + u;
+            const bool live = tt < L;
+            uint2 out = make_uint2(0u, 0u);
+            if (live)
+                out = make_uint2(pack_bf16x2(silu_fast(acc[0]), silu_fast(acc[1])),
+                                 pack_bf16x2(silu_fast(acc[2]), silu_fast(acc[3])));
+            if (v4 < 64)
+                *reinterpret_cast<uint2*>(kq + sw128_off((uint32_t)(row0 + tt), (uint32_t)((cc & 63) >> 3))) = out;
+            if (live) *reinterpret_cast<uint2*>(mix.qkvc + (size_t)(t0 + tt) * C + c) = out;
+        }
+    };
+    // two items in flight: both windows are loaded before either is computed
+#pragma unroll 1
+    for (int item = tid; item < items; item += 2 * kPrepThreads) {
+        int ca, va, ta, cb = 0, vb = 0, tb = 0;
+        uint2 rawa[11], rawb[11];
+        const bool two = item + kPrepThreads < items;
+        locate(item, ca, va, ta);
+        load(ca, ta, rawa);
+        if (two) {
+            locate(item + kPrepThreads, cb, vb, tb);
+            load(cb, tb, rawb);
+        }
+        compute(ca, va, ta, rawa);
+        if (two) compute(cb, vb, tb, rawb);
+    }
+}
+
 // Record (chunk cg, V head h) is complete: publish it to the chain (release). A flag
 // holds the number of the call that wrote it last; call numbers only grow within a
 // process, so flags left by earlier calls never read as ready and need no reset.
@@ -288,6 +391,7 @@ __device__ __forceinline__ void publish_record(unsigned long long* flags, size_t
 // One prep worker of kPrepThreads threads (tid 0 .. 255, synchronised by the named
 // barrier bar_id) walks the (chunk, QK head) units worker, worker + nworkers, ...
 // and writes their records; with `flags`, each finished record is published.
+template <bool kConv>
 __device__ __forceinline__ void prep_worker(
     const bf16* __restrict__ q, const bf16* __restrict__ k, const float* __restrict__ a,
     const float* __restrict__ b, const float* __restrict__ A_log,
@@ -296,7 +400,7 @@ __device__ __forceinline__ void prep_worker(
     uint8_t* __restrict__ rec, int* status,
     unsigned long long* flags, unsigned long long epoch, uint8_t* sm, const int tid,
     const int bar_id, const int worker, const int nworkers, const bool relinquish,
-    const long long wait_cycles) {
+    const long long wait_cycles, const MixerFusion& mix, const int64_t qk_tok) {
     uint8_t* KQ = sm + PS_KQ;
     float* Ts = reinterpret_cast<float*>(sm + PS_TS);
     float* As = reinterpret_cast<float*>(sm + PS_AS);
@@ -352,17 +456,22 @@ __device__ __forceinline__ void prep_worker(
         const int64_t t0 = (int64_t)cu_seqlens[n] + (int64_t)(cg - choff[n]) * kC;
         const int L = (int)min((int64_t)kC, (int64_t)cu_seqlens[n + 1] - t0);
 
-        // ---- raw K and Q rows (sw128), gates of the r V heads ------------------------
+        // ---- raw K and Q rows (sw128), or the convolution that makes them; gates of
+        // the r V heads
+        if constexpr (kConv) {
+            conv_unit(mix, n, cu_seqlens[n], t0, L, j, r, H_qk, KQ, tid);
+        } else {
 #pragma unroll
-        for (int it = 0; it < 4; ++it) {
-            const int idx = tid + kPrepThreads * it;  // 0 .. 1023
-            const int rr = idx >> 4, ch = idx & 15;
-            const bool live = rr < L;
-            const int64_t tok = live ? t0 + rr : 0;
-            const size_t rowk = ((size_t)tok * H_qk + j) * kD + ch * 8;
-            const uint32_t off = (uint32_t)(ch >> 3) * 16384u;
-            cp_async_16(KQ + off + sw128_off(rr, ch & 7), k + rowk, live ? 16u : 0u);
-            cp_async_16(KQ + off + sw128_off(rr + 64, ch & 7), q + rowk, live ? 16u : 0u);
+            for (int it = 0; it < 4; ++it) {
+                const int idx = tid + kPrepThreads * it;  // 0 .. 1023
+                const int rr = idx >> 4, ch = idx & 15;
+                const bool live = rr < L;
+                const int64_t tok = live ? t0 + rr : 0;
+                const size_t rowk = (size_t)tok * qk_tok + (size_t)j * kD + ch * 8;
+                const uint32_t off = (uint32_t)(ch >> 3) * 16384u;
+                cp_async_16(KQ + off + sw128_off(rr, ch & 7), k + rowk, live ? 16u : 0u);
+                cp_async_16(KQ + off + sw128_off(rr + 64, ch & 7), q + rowk, live ? 16u : 0u);
+            }
         }
         for (int idx = tid; idx < 2 * r * kC; idx += kPrepThreads) {
             const int which = idx / (r * kC);            // 0: a, 1: b
@@ -605,17 +714,20 @@ __device__ __forceinline__ void prep_worker(
 }
 
 constexpr int kPrepBlocksPerSm = 3;
+template <bool kConv>
 __global__ void __launch_bounds__(kPrepThreads, kPrepBlocksPerSm) prep_kernel(
     const bf16* __restrict__ q, const bf16* __restrict__ k, const float* __restrict__ a,
     const float* __restrict__ b, const float* __restrict__ A_log,
     const float* __restrict__ dt_bias, const int32_t* __restrict__ cu_seqlens,
     const int32_t* __restrict__ choff, int32_t N, int H_qk, int H_v, float scale,
-    uint8_t* __restrict__ rec, int* status, long long wait_cycles) {
+    uint8_t* __restrict__ rec, int* status, long long wait_cycles, const MixerFusion mix,
+    int64_t qk_tok) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    prep_worker(q, k, a, b, A_log, dt_bias, cu_seqlens, choff, N, H_qk, H_v, scale, rec, status,
-                nullptr, 0, sm, threadIdx.x, 1, blockIdx.x, gridDim.x, true, wait_cycles);
+    prep_worker<kConv>(q, k, a, b, A_log, dt_bias, cu_seqlens, choff, N, H_qk, H_v, scale, rec,
+                       status, nullptr, 0, sm, threadIdx.x, 1, blockIdx.x, gridDim.x, true,
+                       wait_cycles, mix, qk_tok);
 }
 
 // ==================================== chain =======================================
@@ -638,7 +750,8 @@ constexpr uint32_t CS_BAR = CS_OST + 16384;         // barriers (see below)
 constexpr uint32_t CS_TMEM = CS_BAR + 128;
 constexpr uint32_t CS_ERR = CS_BAR + 132;
 constexpr uint32_t CS_EGQ = CS_BAR + 256;           // [64] fp32: the chunk's output row factors
-constexpr size_t kChainSmem = CS_EGQ + 256 + 1024;
+constexpr uint32_t CS_NW = CS_EGQ + 256;            // [128] fp32: the gated norm's weights
+constexpr size_t kChainSmem = CS_NW + 512 + 1024;
 
 // tensor memory columns (512 allocated)
 constexpr uint32_t TM_U = 0;      // 128: the chunk's state increment (scaled Vn^T) K, fp32
@@ -694,11 +807,40 @@ __device__ __forceinline__ bool wait_record(const unsigned long long* flag,
     return false;
 }
 
+// The conv cache of sequence n after it ("Qwen3.5-MoE-35B-A3B architecture teardown",
+// 3.4: conv_dim x (K-1) per sequence): the K-1 inputs ending at its last token (older
+// cache entries where the sequence is shorter), for the v channels of V head h and, with
+// `qk`, the q and k channels of QK head j. One thread per 4-channel group walks the
+// positions oldest first, so an update in place reads every old entry before it is
+// overwritten.
+__device__ __forceinline__ void write_conv_cache(const MixerFusion& mix, int n, int64_t s0,
+                                                 int64_t s1, int h, int j, bool qk, int H_qk,
+                                                 int to, int nthreads) {
+    const int C = mix.conv_dim, Km1 = mix.K - 1;
+    const int64_t len = s1 - s0;
+    const int ng = qk ? 96 : 32;
+    for (int g = to; g < ng; g += nthreads) {
+        int c;
+        if (g < 32) c = 2 * H_qk * kD + h * kD + 4 * g;
+        else if (g < 64) c = j * kD + 4 * (g - 32);
+        else c = H_qk * kD + j * kD + 4 * (g - 64);
+        for (int i = 0; i < Km1; ++i) {
+            const int64_t p = len - Km1 + i;
+            uint2 v = make_uint2(0u, 0u);
+            if (p >= 0)
+                v = *reinterpret_cast<const uint2*>(mix.x + (size_t)(s0 + p) * C + c);
+            else if (mix.cache_in)
+                v = *reinterpret_cast<const uint2*>(mix.cache_in + ((size_t)n * Km1 + len + i) * C + c);
+            *reinterpret_cast<uint2*>(mix.cache_out + ((size_t)n * Km1 + i) * C + c) = v;
+        }
+    }
+}
+
 // The whole chunk chain of one (sequence n, V head h), run by the kChainThreads
 // threads of a block (tid 0 .. 415, synchronised by the named barrier sync_id) on
 // the tensor memory `tmem` (512 columns). With `flags`, a chunk's record is
 // copied only once a prep worker has published it.
-template <int kM>
+template <int kM, bool kNorm>
 __device__ __forceinline__ void chain_unit(
     const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
     const CUtensorMap& tm_o, const float* S0g, const int32_t* __restrict__ cu_seqlens,
@@ -707,8 +849,9 @@ __device__ __forceinline__ void chain_unit(
     float* Sfg, const StateIndex sref, int* status,
     const unsigned long long* flags, unsigned long long epoch, uint8_t* sm, const int tid,
     const int n, const int h, const int hv, const uint32_t tmem,
-    const int sync_id, const long long wait_cycles) {
+    const int sync_id, const long long wait_cycles, const MixerFusion& mix) {
     static_assert(kM == 128 || kM == 64, "a chain block owns all 128 value rows or one half");
+    static_assert(!kNorm || kM == 128, "the fused gated norm needs whole value rows");
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + CS_BAR);  // [3] slot landed
     uint64_t* mbar = full + kRing;         // chain MMA completions
     uint64_t* obar = mbar + 1;             // [2] chunk parity b: output accumulators complete
@@ -747,7 +890,8 @@ __device__ __forceinline__ void chain_unit(
 
     // chunk c of this sequence -> its ring slot (issued by one lane). The K, Q, V tiles
     // need nothing from the prep workers and go first; the record follows once its
-    // flag is seen (the slot's barrier expects both).
+    // flag is seen (the slot's barrier expects both). With the convolution fused into
+    // the preparation the tiles are its output too, so they wait for the flag as well.
     auto load_tiles = [&](int c) {
         const int st = c % kRing;
         uint8_t* slot = sm + st * kSlotBytes;
@@ -786,20 +930,59 @@ __device__ __forceinline__ void chain_unit(
         uint8_t* ost = sm + CS_OST;
         const bool loader = warp == kLoadWarp && lane == 0;
         float* egq = reinterpret_cast<float*>(sm + CS_EGQ);
+        float* s_nw = reinterpret_cast<float*>(sm + CS_NW);
+        if (kNorm && to < kD / 4)  // read by the norm after the loop's first barrier
+            reinterpret_cast<float4*>(s_nw)[to] = reinterpret_cast<const float4*>(mix.norm_w)[to];
         int issued = 0;   // chunks whose tiles and record were issued
         if (loader) {
-            for (int c = 0; c < kRing && c < nchunks; ++c) load_tiles(c);
-            for (int c = 0; c < kRing && c < nchunks; ++c) {
-                record_ready(c);
-                load_record(c);
-                issued = c + 1;
+            if (mix.x) {
+                for (int c = 0; c < kRing && c < nchunks; ++c) {
+                    record_ready(c);
+                    if (flags) asm volatile("fence.proxy.async.global;" ::: "memory");
+                    load_tiles(c);
+                    load_record(c);
+                    issued = c + 1;
+                }
+            } else {
+                for (int c = 0; c < kRing && c < nchunks; ++c) load_tiles(c);
+                for (int c = 0; c < kRing && c < nchunks; ++c) {
+                    record_ready(c);
+                    load_record(c);
+                    issued = c + 1;
+                }
             }
         }
         __syncwarp();
+        // Gate rows for the fused norm: chunk c's are loaded into registers at the end of
+        // chunk c-1's iteration (the output warps reach a chunk when its MMAs are long
+        // done, so a load issued at its start would be waited for in full), after being
+        // prefetched into L2 two chunks ahead.
+        uint4 zv[kNorm ? 8 : 1];
+        auto load_gate_rows = [&](int c) {
+            const int64_t tz = s0 + (int64_t)c * kC + (to >> 1);
+            if (c < nchunks && tz < s1) {
+                const bf16* zr = mix.z + ((size_t)tz * H_v + h) * kD + (to & 1) * 64;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) zv[q] = *reinterpret_cast<const uint4*>(zr + q * 8);
+            }
+        };
+        if constexpr (kNorm) {
+            for (int c2 = 1; c2 < 3 && c2 < nchunks; ++c2) {
+                const int64_t t2 = s0 + (int64_t)c2 * kC + (to >> 1);
+                if (t2 < s1) prefetch_l2(mix.z + ((size_t)t2 * H_v + h) * kD + (to & 1) * 64);
+            }
+            load_gate_rows(0);
+        }
 #pragma unroll 1
         for (int cp = 0; cp < nchunks; ++cp) {
             const int b = cp & 1;
             const int cn = cp + kRing;  // the chunk that will reuse this chunk's slot
+            const int64_t t0 = s0 + (int64_t)cp * kC;
+            const int L = (int)min((int64_t)kC, s1 - t0);
+            if constexpr (kNorm) {
+                const int64_t t3 = t0 + 3 * kC + (to >> 1);
+                if (t3 < s1) prefetch_l2(mix.z + ((size_t)t3 * H_v + h) * kD + (to & 1) * 64);
+            }
             // its record's flag is checked while this chunk's MMAs still run
             const bool next = loader && cn < nchunks && issued == cn;
             const bool ok = mbar_wait_bounded(&obar[b], (cp >> 1) & 1, wait_cycles);
@@ -873,6 +1056,7 @@ __device__ __forceinline__ void chain_unit(
             // flag is an L2 round trip; before the read it delayed every chunk's output).
             if (next) {
                 record_ready(cn);
+                if (mix.x && flags) asm volatile("fence.proxy.async.global;" ::: "memory");
                 load_tiles(cn);
                 load_record(cn);
                 issued = cn + 1;
@@ -880,8 +1064,55 @@ __device__ __forceinline__ void chain_unit(
             __syncwarp();
             fence_proxy_async_smem();
             named_bar_sync(2, kOut);  // staged; every output warp is done with the slot
-            const int64_t t0 = s0 + (int64_t)cp * kC;
-            const int L = (int)min((int64_t)kC, s1 - t0);
+            if constexpr (kNorm) {
+                {
+                    // The gated RMSNorm over each staged o row ("Qwen3.5-MoE-35B-A3B architecture
+                    // teardown", 3.3 phase 4: RMSNorm(o) * w * SiLU(z)): two threads per token,
+                    // 64 values each, the sum of squares of the bf16 o, then y over o in place.
+                    const int t = to >> 1, half = to & 1;
+                    uint8_t* rowp = ost + half * 8192 + t * 128;
+                    float ss = 0.f;
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        const uint4 w = *reinterpret_cast<const uint4*>(rowp + ((ch ^ (t & 7)) << 4));
+                        const uint32_t* u = &w.x;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u[e]));
+                            ss = fmaf(f.x, f.x, ss);
+                            ss = fmaf(f.y, f.y, ss);
+                        }
+                    }
+                    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                    const float inv = rsqrtf(ss * (1.f / kD) + mix.eps);
+                    if (t < L) {
+                        const float4* wr4 = reinterpret_cast<const float4*>(s_nw + half * 64);
+#pragma unroll
+                        for (int ch = 0; ch < 8; ++ch) {
+                            uint4* p = reinterpret_cast<uint4*>(rowp + ((ch ^ (t & 7)) << 4));
+                            const uint4 ov = *p;
+                            const float4 w0 = wr4[2 * ch], w1 = wr4[2 * ch + 1];
+                            const float wv[8] = {w0.x * inv, w0.y * inv, w0.z * inv, w0.w * inv,
+                                                 w1.x * inv, w1.y * inv, w1.z * inv, w1.w * inv};
+                            const uint32_t* ou = &ov.x;
+                            const uint32_t* zu = &zv[ch].x;
+                            uint32_t res[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 of = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ou[e]));
+                                const float2 zf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&zu[e]));
+                                res[e] = pack_bf16x2(of.x * wv[2 * e] * silu_tanh(zf.x),
+                                                     of.y * wv[2 * e + 1] * silu_tanh(zf.y));
+                            }
+                            *p = make_uint4(res[0], res[1], res[2], res[3]);
+                        }
+                    }
+                    __syncwarp();
+                    fence_proxy_async_smem();
+                    named_bar_sync(2, kOut);
+                    load_gate_rows(cp + 1);  // the next chunk's, a whole chunk ahead of use
+                }
+            }
             constexpr int kOutCh = kM / 8;  // 16-byte chunks per staged row
             if (L == kC) {
                 if (loader) {
@@ -905,6 +1136,8 @@ __device__ __forceinline__ void chain_unit(
             }
             __syncwarp();
         }
+        if (mix.cache_out && hv == 0 && *s_err == 0)
+            write_conv_cache(mix, n, s0, s1, h, j, h % (H_v / H_qk) == 0, H_qk, to, kOut);
         if (loader) {
             bulk_wait_group<0>();  // o stores complete
             // Leave nothing in flight into shared memory (loads the chain did not
@@ -1338,13 +1571,14 @@ __device__ __forceinline__ void chain_unit(
     if (tid == 0 && *s_err) set_status(status, kStatusTimeout);
 }
 
+template <bool kNorm>
 __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
     const float* S0g, const int32_t* __restrict__ cu_seqlens,
     const int32_t* __restrict__ choff, int64_t T_total, int H_qk, int H_v,
     const uint8_t* __restrict__ rec, bf16* __restrict__ o, float* Sfg, const StateIndex sref,
-    int* status, long long wait_cycles) {
+    int* status, long long wait_cycles, const MixerFusion mix) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1358,9 +1592,9 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
-    chain_unit<128>(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v, rec, o,
+    chain_unit<128, kNorm>(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v, rec, o,
                     Sfg, sref, status, nullptr, 0, sm, threadIdx.x, blockIdx.x / H_v,
-                    blockIdx.x % H_v, 0, tmem, 1, wait_cycles);
+                    blockIdx.x % H_v, 0, tmem, 1, wait_cycles, mix);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1383,7 +1617,7 @@ constexpr size_t kFusedSmem =
 constexpr int kChainSync = 5;  // named barrier of the chain threads in the fused kernel
 constexpr int kFusedMaxSeqs = 255;  // the fused kernel computes the chunk offsets itself
 
-template <int kM>
+template <int kM, bool kMix>
 __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -1394,7 +1628,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
     int64_t T_total, int H_qk, int H_v, float scale, uint8_t* __restrict__ rec,
     bf16* __restrict__ o, float* Sfg, const StateIndex sref,
     int* status, unsigned long long* flags, unsigned long long epoch, int c0,
-    long long wait_cycles, int withhold_records) {
+    long long wait_cycles, int withhold_records, const MixerFusion mix) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ int32_t s_choff[kFusedMaxSeqs + 1];
     __shared__ int s_bad;
@@ -1435,10 +1669,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
     if ((int)blockIdx.x >= c0) {
         const int sub = tid >> 8;
         // a fault-injection call withholds every record: the chains' waits run out
-        prep_worker(q, k, a, b, A_log, dt_bias, cu_seqlens, choff, N, H_qk, H_v, scale, rec,
+        prep_worker<kMix>(q, k, a, b, A_log, dt_bias, cu_seqlens, choff, N, H_qk, H_v, scale, rec,
                     status, withhold_records ? nullptr : flags, epoch, sm + sub * kPrepRegion,
                     tid & 255, 3 + sub, 2 * ((int)blockIdx.x - c0) + sub,
-                    2 * ((int)gridDim.x - c0), false, wait_cycles);
+                    2 * ((int)gridDim.x - c0), false, wait_cycles, mix, (int64_t)H_qk * kD);
         return;
     }
     if (tid >= kChainThreads) return;
@@ -1454,9 +1688,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
     // block u: (sequence, V head) u, or with half-row blocks its half u & 1 of unit u >> 1
     const int u = kM == 64 ? (int)blockIdx.x >> 1 : (int)blockIdx.x;
     const int hv = kM == 64 ? (int)blockIdx.x & 1 : 0;
-    chain_unit<kM>(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v, rec, o,
+    chain_unit<kM, kMix>(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v, rec, o,
                    Sfg, sref, status, flags, epoch, sm, tid, u / H_v, u % H_v, hv, tmem,
-                   kChainSync, wait_cycles);
+                   kChainSync, wait_cycles, mix);
     tc_fence_before();
     named_bar_sync(kChainSync, kChainThreads);
     tc_fence_after();
@@ -1534,12 +1768,15 @@ EncodeTiledFn encode_tiled() {
 
 // [T][heads][128] bf16 rows as a 3-D tensor (d, head, token); boxes of 64 d x 1
 // head x 64 tokens move as 64 rows of 128 bytes in the 128-byte swizzle. Tokens
-// past T read as zeros and are not written.
-bool make_rows_map(CUtensorMap* m, const void* base, int heads, int64_t T) {
+// past T read as zeros and are not written. token_elems: elements from one token's
+// rows to the next one's (0: heads x 128, a dense tensor).
+bool make_rows_map(CUtensorMap* m, const void* base, int heads, int64_t T,
+                   int64_t token_elems = 0) {
     EncodeTiledFn fn = encode_tiled();
     if (!fn) return false;
+    if (token_elems == 0) token_elems = (int64_t)heads * kD;
     const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)heads, (cuuint64_t)(T > 0 ? T : 1)};
-    const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)heads * kD * 2};
+    const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)token_elems * 2};
     const cuuint32_t box[3] = {64, 1, (cuuint32_t)kC};
     const cuuint32_t estride[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
@@ -1553,7 +1790,7 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
                               const float* S0, const int32_t* cu_seqlens, int32_t N, int64_t T,
                               int32_t H_qk, int32_t H_v, float scale, void* o, float* S_final,
                               StateIndex sref, void* workspace, const PrefillOpts& opt,
-                              int* status, cudaStream_t s) {
+                              int* status, cudaStream_t s, const MixerFusion& mix) {
     if (N == 0) return cudaSuccess;
     if (T > (int64_t)0x7FFFFFFF - kC) return cudaErrorInvalidValue;  // TMA token coordinates
     const TcWorkspace ws = tc_workspace_layout(N, T, H_v);
@@ -1562,10 +1799,18 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
     unsigned long long* flags = reinterpret_cast<unsigned long long*>(wb + ws.off_flags);
     uint8_t* rec = wb + ws.off_rec;
     // With no tokens the maps are never read; any aligned device address will do.
+    // In the mixer, q, k and v are the convolution's output: views of the post-conv
+    // buffer [T][conv_dim] (q | k | v), written by the preparation (convolution fused into
+    // its loads) or by the standalone convolution kernel before it.
     CUtensorMap tm_q, tm_k, tm_v, tm_o;
-    if (!make_rows_map(&tm_q, T > 0 ? q : workspace, H_qk, T) ||
-        !make_rows_map(&tm_k, T > 0 ? k : workspace, H_qk, T) ||
-        !make_rows_map(&tm_v, T > 0 ? v : workspace, H_v, T) ||
+    const bool mixer = mix.qkvc != nullptr;
+    const int64_t tok = mixer ? (int64_t)mix.conv_dim : 0;
+    const void* qv = mixer ? (const void*)mix.qkvc : q;
+    const void* kv = mixer ? (const void*)(mix.qkvc + (size_t)H_qk * kD) : k;
+    const void* vv = mixer ? (const void*)(mix.qkvc + (size_t)2 * H_qk * kD) : v;
+    if (!make_rows_map(&tm_q, T > 0 ? qv : workspace, H_qk, T, tok) ||
+        !make_rows_map(&tm_k, T > 0 ? kv : workspace, H_qk, T, tok) ||
+        !make_rows_map(&tm_v, T > 0 ? vv : workspace, H_v, T, tok) ||
         !make_rows_map(&tm_o, T > 0 ? o : workspace, H_v, T))
         return cudaErrorInvalidValue;
     int dev = 0, num_sms = 0, coop = 0;
@@ -1586,8 +1831,11 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
         // phases at full occupancy. With at most a quarter as many chains as SMs each
         // chain runs as two blocks of 64 value rows (half the per-thread state work on
         // the critical path).
-        const bool half = !whole_rows && 4 * chain_units <= num_sms;
-        const void* kfn = half ? (const void*)fused_kernel<64> : (const void*)fused_kernel<128>;
+        // (the fused gated norm needs all 128 values of a token in one block)
+        const bool half = !whole_rows && !mixer && 4 * chain_units <= num_sms;
+        const void* kfn = mixer ? (const void*)fused_kernel<128, true>
+                        : half  ? (const void*)fused_kernel<64, false>
+                                : (const void*)fused_kernel<128, false>;
         e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kFusedSmem);
         if (e != cudaSuccess) return e;
@@ -1607,7 +1855,7 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
             void* args[] = {&tm_q, &tm_k, &tm_v, &tm_o, &qb, &kb, &a, &b, &A_log, &dt_bias, &S0,
                             &cu_seqlens, &choff, &N, &T, &H_qk, &H_v, &scale, &rec, &ob,
                             &S_final, &sref, &status, &flags, &epoch, &c0v, &wait_cycles,
-                            &withhold};
+                            &withhold, const_cast<MixerFusion*>(&mix)};
             timer_before(opt.timer, s);
             e = cudaLaunchCooperativeKernel(kfn, dim3(grid), dim3(kFusedThreads), args, kFusedSmem,
                                             s);
@@ -1616,13 +1864,36 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
         }
     }
 
-    e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    // Separate launches. In the mixer the convolution then runs as its own streaming
+    // kernel first (the preparation is the slower stage here, and the convolution would
+    // add to it): it writes the post-conv buffer and the conv cache, the preparation
+    // reads its q and k rows from that buffer, and the chain applies the gated norm.
+    MixerFusion mix_split = mix;
+    mix_split.x = nullptr;
+    mix_split.cache_out = nullptr;
+    if (mixer && T > 0) {
+        timer_before(opt.timer, s);
+        e = launch_conv1d_silu(mix.x, GDN_BF16, mix.conv_w, mix.conv_b, mix.cache_in, cu_seqlens,
+                               N, T, mix.conv_dim, mix.K, mix.qkvc, mix.cache_out, status, s);
+        if (e != cudaSuccess) return e;
+        timer_after(opt.timer, s, "conv1d_silu");
+    } else if (mixer && mix.cache_out) {  // no tokens: only the cache (kept) to write
+        e = launch_conv1d_silu(mix.x, GDN_BF16, mix.conv_w, mix.conv_b, mix.cache_in, cu_seqlens,
+                               N, T, mix.conv_dim, mix.K, mix.qkvc, mix.cache_out, status, s);
+        if (e != cudaSuccess) return e;
+    }
+    const bf16* q_rows = mixer ? mix.qkvc : static_cast<const bf16*>(q);
+    const bf16* k_rows = mixer ? mix.qkvc + (size_t)H_qk * kD : static_cast<const bf16*>(k);
+    const int64_t qk_tok = mixer ? (int64_t)mix.conv_dim : (int64_t)H_qk * kD;
+    const auto prep_fn = prep_kernel<false>;
+    const auto chain_fn = mixer ? chain_kernel<true> : chain_kernel<false>;
+    e = cudaFuncSetAttribute(prep_fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kPrepSmem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+    e = cudaFuncSetAttribute(prep_fn, cudaFuncAttributePreferredSharedMemoryCarveout,
                              (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(chain_fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kChainSmem);
     if (e != cudaSuccess) return e;
     timer_before(opt.timer, s);
@@ -1638,17 +1909,17 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
     const int prep_grid = (int)(unit_bound < grid_cap ? unit_bound : grid_cap);
     if (prep_grid > 0) {
         timer_before(opt.timer, s);
-        prep_kernel<<<prep_grid, kPrepThreads, kPrepSmem, s>>>(
-            static_cast<const bf16*>(q), static_cast<const bf16*>(k), a, b, A_log, dt_bias,
-            cu_seqlens, choff, N, H_qk, H_v, scale, rec, status, wait_cycles);
+        prep_fn<<<prep_grid, kPrepThreads, kPrepSmem, s>>>(
+            q_rows, k_rows, a, b, A_log, dt_bias, cu_seqlens, choff, N, H_qk, H_v, scale, rec,
+            status, wait_cycles, mix_split, qk_tok);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         timer_after(opt.timer, s, "prep");
     }
     timer_before(opt.timer, s);
-    chain_kernel<<<(unsigned)chain_units, kChainThreads, kChainSmem, s>>>(
+    chain_fn<<<(unsigned)chain_units, kChainThreads, kChainSmem, s>>>(
         tm_q, tm_k, tm_v, tm_o, S0, cu_seqlens, choff, T, H_qk, H_v, rec, static_cast<bf16*>(o),
-        S_final, sref, status, wait_cycles);
+        S_final, sref, status, wait_cycles, mix_split);
     e = cudaGetLastError();
     if (e == cudaSuccess) timer_after(opt.timer, s, "chain");
     return e;

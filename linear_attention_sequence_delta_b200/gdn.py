@@ -37,7 +37,8 @@ EXPORTS = ["gdn_status_string", "gdn_version", "gdn_prefill_workspace_size", "gd
            "gdn_prefill_noalloc", "gdn_timer_create", "gdn_timer_destroy", "gdn_timer_read",
            "gdn_timer_kernel_name", "gdn_conv1d_silu", "gdn_conv1d_silu_decode",
            "gdn_rmsnorm_gated", "gdn_decode_slots", "gdn_decode_step_bf16_state",
-           "gdn_prefill_slots", "gdn_prefill_slots_ex"]
+           "gdn_prefill_slots", "gdn_prefill_slots_ex", "gdn_mixer_prefill",
+           "gdn_mixer_prefill_workspace_size"]
 GDN_IMPL_AUTO, GDN_IMPL_CUDA_CORE, GDN_IMPL_TENSOR_CORE, GDN_IMPL_TENSOR_CORE_SPLIT = 0, 1, 2, 3
 GDN_IMPL_TENSOR_CORE_WHOLE_ROWS = 4
 GDN_FAULT_NONE, GDN_FAULT_WITHHOLD_RECORDS = 0, 1
@@ -112,6 +113,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gdn_decode_slots.restype = ctypes.c_int
     lib.gdn_decode_slots.argtypes = [P, P, P, i32, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32,
                                      i32, f32, P, P, P]
+    lib.gdn_mixer_prefill_workspace_size.restype = sz
+    lib.gdn_mixer_prefill_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32, i32]
+    lib.gdn_mixer_prefill.restype = ctypes.c_int
+    lib.gdn_mixer_prefill.argtypes = [P, i32, P, P, P, P, i32, P, P, P, P, P, P, i32, i64, i32,
+                                      i32, i32, i32, f32, P, P, f32, P, P, P, sz, P, P]
     lib.gdn_rmsnorm_gated.restype = ctypes.c_int
     lib.gdn_rmsnorm_gated.argtypes = [P, P, i32, P, f32, i64, i32, P, P]
     _lib = lib
@@ -410,3 +416,54 @@ def gdn_rmsnorm_gated(o, z, weight, eps: float = 1e-6, *, out=None):
                                _ptr(y), _stream(o.device))
     _check(st, "gdn_rmsnorm_gated")
     return y
+
+
+def mixer_workspace_size(num_seqs, total_tokens, H_qk, H_v, d, io_dtype=torch.bfloat16) -> int:
+    io = GDN_BF16 if io_dtype == torch.bfloat16 else GDN_FP32
+    return int(load_library().gdn_mixer_prefill_workspace_size(num_seqs, total_tokens, H_qk,
+                                                               H_v, d, d, io))
+
+
+def gdn_mixer_prefill(x, conv_weight, conv_bias, cu_seqlens, a, b, A_log, dt_bias, z,
+                      norm_weight, *, H_qk: int, conv_state_in=None, conv_state_out=None,
+                      initial_state=None, eps: float = 1e-6, scale: float = 1.0,
+                      output_final_state: bool = True, out=None, final_state=None,
+                      workspace=None, impl: int = GDN_IMPL_AUTO,
+                      timer: Optional[Timer] = None, fault: int = GDN_FAULT_NONE,
+                      wait_limit_cycles: int = 0):
+    """The mixer core in one call: y = RMSNorm(o) * w * SiLU(z) with o the gated delta
+    rule over the causal conv1d + SiLU of x. Returns (y, final_state or None).
+
+    x [T, (2 H_qk + H_v) d] (q | k | v channels, bf16 or fp32); conv_weight [C, K] fp32;
+    conv_bias [C] fp32 or None; cu_seqlens int32 [N+1]; a, b [T, H_v] fp32; A_log, dt_bias
+    [H_v] fp32; z [T, H_v, d] (x's dtype); norm_weight [d] fp32; conv_state_in /
+    conv_state_out [N, K-1, C] or None (out may be in: updated in place); initial_state
+    [N, H_v, d, d] fp32 or None.
+    """
+    lib = load_library()
+    _need_cuda(x, conv_weight, conv_bias, cu_seqlens, a, b, A_log, dt_bias, z, norm_weight,
+               conv_state_in, conv_state_out, initial_state, out, final_state, workspace)
+    io = _io_dtype(x)
+    T, C = x.shape
+    _, H_v, d = z.shape
+    K = conv_weight.shape[1]
+    N = cu_seqlens.numel() - 1
+    if C != (2 * H_qk + H_v) * d:
+        raise ValueError("x must have (2 H_qk + H_v) d channels")
+    y = out if out is not None else torch.empty_like(z)
+    if output_final_state and final_state is None:
+        final_state = torch.empty((N, H_v, d, d), device=x.device, dtype=torch.float32)
+    if not output_final_state:
+        final_state = None
+    need = lib.gdn_mixer_prefill_workspace_size(N, T, H_qk, H_v, d, d, io)
+    if workspace is None:
+        workspace = torch.empty((max(int(need), 1),), device=x.device, dtype=torch.uint8)
+    opts = _options(impl, fault, wait_limit_cycles, timer)
+    st = lib.gdn_mixer_prefill(_ptr(x), io, _ptr(conv_weight), _ptr(conv_bias),
+                               _ptr(conv_state_in), _ptr(conv_state_out), K, _ptr(a), _ptr(b),
+                               _ptr(A_log), _ptr(dt_bias), _ptr(initial_state), _ptr(cu_seqlens),
+                               N, T, H_qk, H_v, d, d, float(scale), _ptr(z), _ptr(norm_weight),
+                               float(eps), _ptr(y), _ptr(final_state), _ptr(workspace),
+                               workspace.numel(), opts, _stream(x.device))
+    _check(st, "gdn_mixer_prefill")
+    return y, final_state

@@ -182,6 +182,75 @@ def make_mixer_inputs(lengths=None, *, num_seqs: int = 1, seq_len: int = 256,
     return MixerInputs(x, w, bias, st, o, z, nw, cu_t)
 
 
+@dataclass
+class MixerPrefillInputs:
+    x: torch.Tensor              # [T, C] pre-conv q | k | v channels
+    conv_weight: torch.Tensor    # [C, K] fp32
+    conv_bias: torch.Tensor      # [C] fp32
+    conv_state: torch.Tensor     # [N, K-1, C]
+    a: torch.Tensor              # [T, H_v] fp32
+    b: torch.Tensor
+    A_log: torch.Tensor          # [H_v] fp32
+    dt_bias: torch.Tensor
+    initial_state: Optional[torch.Tensor]  # [N, H_v, d_v, d_k] fp32
+    z: torch.Tensor              # [T, H_v, d_v]
+    norm_weight: torch.Tensor    # [d_v] fp32
+    cu_seqlens: torch.Tensor     # int32 [N+1]
+    H_qk: int
+
+    @property
+    def num_seqs(self) -> int:
+        return self.cu_seqlens.numel() - 1
+
+    def to(self, device) -> "MixerPrefillInputs":
+        mv = lambda t: t.to(device) if isinstance(t, torch.Tensor) else t
+        return MixerPrefillInputs(*(mv(getattr(self, f)) for f in self.__dataclass_fields__))
+
+
+def make_mixer_prefill_inputs(lengths=None, *, num_seqs: int = 1, seq_len: int = 256,
+                              len_lo: int = 128, len_hi: int = 8192, H_qk: int = 16,
+                              H_v: int = 32, d: int = 128, kernel_size: int = 4,
+                              io_dtype: torch.dtype = torch.bfloat16,
+                              state_std: Optional[float] = None, seed: int = 0,
+                              device="cpu") -> MixerPrefillInputs:
+    """Inputs of the whole mixer core (conv -> delta rule -> gated norm), drawn in this
+    order: lengths (as make_prefill_inputs); x [T, C] ~ N(0, 1) (C = (2 H_qk + H_v) d,
+    rounded to the I/O type); conv weight [C, K] ~ U(-1/sqrt(K), 1/sqrt(K)), conv bias
+    [C] ~ N(0, 0.1^2); conv cache [N, K-1, C] ~ N(0, 1) (rounded); a, b [T, H_v] ~ N(0, 1);
+    A_log ~ U(0, ln 16), dt_bias ~ U(-1, 1); initial state ~ N(0, state_std^2) (when
+    asked for); z [T, H_v, d] ~ N(0, 1) (rounded); norm weight [d] ~ U(0.5, 1.5)."""
+    g = _gen(device, seed)
+    if isinstance(lengths, str) and lengths == "random":
+        lens = torch.randint(len_lo, len_hi + 1, (num_seqs,), generator=g, device=device)
+        lens = [int(x) for x in lens.cpu()]
+    elif lengths is None:
+        lens = [seq_len] * num_seqs
+    else:
+        lens = [int(x) for x in lengths]
+    cu = [0]
+    for n in lens:
+        cu.append(cu[-1] + n)
+    T, N, K = cu[-1], len(lens), kernel_size
+    C = (2 * H_qk + H_v) * d
+    f32 = torch.float32
+    x = torch.randn((T, C), generator=g, device=device, dtype=f32).to(io_dtype)
+    bound = 1.0 / math.sqrt(K)
+    w = (torch.rand((C, K), generator=g, device=device, dtype=f32) * 2.0 - 1.0) * bound
+    bias = torch.randn((C,), generator=g, device=device, dtype=f32) * 0.1
+    st = torch.randn((N, K - 1, C), generator=g, device=device, dtype=f32).to(io_dtype)
+    a = torch.randn((T, H_v), generator=g, device=device, dtype=f32)
+    b = torch.randn((T, H_v), generator=g, device=device, dtype=f32)
+    A_log = torch.rand((H_v,), generator=g, device=device, dtype=f32) * math.log(16.0)
+    dt_bias = torch.rand((H_v,), generator=g, device=device, dtype=f32) * 2.0 - 1.0
+    S0 = None
+    if state_std is not None:
+        S0 = torch.randn((N, H_v, d, d), generator=g, device=device, dtype=f32) * state_std
+    z = torch.randn((T, H_v, d), generator=g, device=device, dtype=f32).to(io_dtype)
+    nw = torch.rand((d,), generator=g, device=device, dtype=f32) + 0.5
+    cu_t = torch.tensor(cu, dtype=torch.int32, device=device)
+    return MixerPrefillInputs(x, w, bias, st, a, b, A_log, dt_bias, S0, z, nw, cu_t, H_qk)
+
+
 # The five workloads, by name. Sizes are those of the Qwen3.5 GDN layers.
 WORKLOADS = {
     "tiny_fp32": dict(num_seqs=1, seq_len=256, H_qk=2, H_v=4, d_k=64, d_v=64,

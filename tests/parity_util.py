@@ -38,3 +38,23 @@ def oracle_prefill_heads(P, heads, seqs=None, scale=1.0):
                                    P.dt_bias[h:h + 1].cpu(), [0, s1 - s0], S0, scale=scale)
             out[(n, h)] = (o[:, 0], Sf[0, 0])
     return out
+
+
+def oracle_mixer(P, eps=1e-6, scale=1.0):
+    """The mixer core composed from the oracle's steps: the causal conv1d + SiLU over the
+    q | k | v channels (the conv cache in and out), its output rounded to the I/O type as
+    the API states, split into q, k and v heads, the gated delta rule, then the gated
+    RMSNorm with z. Returns (y, final_state, conv_state_out)."""
+    cu = P.cu_seqlens.cpu().numpy().astype(np.int64)
+    T, C = P.x.shape
+    H_v, d = P.z.shape[1], P.z.shape[2]
+    H_qk = P.H_qk
+    yc, so = oracle.conv1d_silu(P.x, P.conv_weight, P.conv_bias, cu, P.conv_state)
+    yc = torch.from_numpy(yc).to(P.x.dtype)  # the post-conv q, k, v in the I/O type
+    q = yc[:, :H_qk * d].reshape(T, H_qk, d)
+    k = yc[:, H_qk * d:2 * H_qk * d].reshape(T, H_qk, d)
+    v = yc[:, 2 * H_qk * d:].reshape(T, H_v, d)
+    o, Sf = oracle.forward(q, k, v, P.a, P.b, P.A_log, P.dt_bias, cu, P.initial_state,
+                           scale=scale)
+    y = oracle.rmsnorm_gated(o, P.z, P.norm_weight, eps)
+    return y, Sf, so

@@ -332,3 +332,48 @@ def test_timer_host_checks(lib):
     assert lib.gdn_timer_read(None, ms, 4) == -1
     assert lib.gdn_timer_kernel_name(None, 0) is None
     lib.gdn_timer_destroy(None)  # ignored
+
+
+def _call_mixer(lib, **over):
+    a = dict(x=F, io=gdn.GDN_BF16, w=F + 0x1000, bias=None, cin=None, cout=None, K=4,
+             a=F + 0x3000, b=F + 0x4000, A_log=F + 0x5000, dt_bias=F + 0x6000, S0=None,
+             cu=F + 0x7000, N=1, T=128, H_qk=2, H_v=4, d=64, scale=1.0, z=F + 0x8000,
+             nw=F + 0x9000, eps=1e-6, y=F + 0xA000, Sf=None, ws=F + 0x10000, ws_bytes=1 << 30,
+             opts=None)
+    a.update(over)
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.gdn_mixer_prefill(v(a["x"]), a["io"], v(a["w"]), v(a["bias"]), v(a["cin"]),
+                                 v(a["cout"]), a["K"], v(a["a"]), v(a["b"]), v(a["A_log"]),
+                                 v(a["dt_bias"]), v(a["S0"]), v(a["cu"]), a["N"], a["T"],
+                                 a["H_qk"], a["H_v"], a["d"], a["d"], a["scale"], v(a["z"]),
+                                 v(a["nw"]), a["eps"], v(a["y"]), v(a["Sf"]), v(a["ws"]),
+                                 a["ws_bytes"], a["opts"], None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(io=3), 1),
+    (dict(K=5), 2), (dict(K=1), 2),
+    (dict(d=96), 2),
+    (dict(H_v=3), 1),
+    (dict(eps=-1.0), 1), (dict(eps=math.inf), 1), (dict(scale=math.nan), 1),
+    (dict(N=0, T=5), 1),
+    (dict(x=None), 1), (dict(z=None), 1), (dict(y=None), 1), (dict(w=None), 1),
+    (dict(nw=None), 1), (dict(cu=None), 1),
+    (dict(y=F), 1),                     # y must not be x
+    (dict(y=F + 0x8000), 1),            # nor z
+    (dict(nw=F + 4), 1), (dict(cout=F + 8), 1), (dict(x=F + 2), 1), (dict(bias=F + 2), 1),
+    (dict(ws_bytes=1000), 3), (dict(ws=F + 0x10010), 3), (dict(ws=None), 3),
+    (dict(N=0, T=0), 0),                # nothing to do
+])
+def test_mixer_prefill_rejects(lib, over, code):
+    assert _call_mixer(lib, **over) == code
+
+
+def test_mixer_workspace_size(lib):
+    f = lib.gdn_mixer_prefill_workspace_size
+    pre = lib.gdn_prefill_workspace_size(1, 4096, 16, 32, 128, 128)
+    conv_dim = (2 * 16 + 32) * 128
+    assert f(1, 4096, 16, 32, 128, 128, gdn.GDN_BF16) == 4096 * conv_dim * 2 + pre
+    assert f(1, 4096, 16, 32, 128, 128, gdn.GDN_FP32) == 4096 * conv_dim * 4 + pre
+    assert f(1, 4096, 16, 32, 128, 128, 7) == 0
+    assert f(1, 10, 16, 24, 128, 128, gdn.GDN_BF16) == 0
