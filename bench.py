@@ -196,6 +196,89 @@ def run_mixer(rank, dev, flush, stream, hbm, peak_src, iters):
     return out, iters * 4
 
 
+def mixer_call_bytes(T, N, H_qk, H_v, d, K, io_bytes, with_initial):
+    """Algorithmic HBM bytes of one gdn_mixer_prefill call: x read, z read, y written
+    (io_bytes each element), a and b read, the conv taps read, the conv cache read and
+    written, the final states written (and the initial states read)."""
+    C = (2 * H_qk + H_v) * d
+    b = T * C * io_bytes + 2 * T * H_v * d * io_bytes + 2 * T * H_v * 4 + C * K * 4
+    b += 2 * N * (K - 1) * C * io_bytes
+    b += N * H_v * d * d * 4 * (2 if with_initial else 1)
+    return b
+
+
+def run_mixer_prefill(rank, dev, flush, stream, hbm, peak_src, iters):
+    """gdn_mixer_prefill (conv1d + SiLU fused into the prefill's preparation, gated
+    RMSNorm into the chain's output) against the same steps as separate kernels: the
+    conv of the q, k and v parts (dense tensors), gdn_prefill, gdn_rmsnorm_gated. On
+    the 35B-A3B layer shape (T=4096) and the packed varlen batch (64 sequences)."""
+    from linear_attention_sequence_delta_b200 import gdn
+    from linear_attention_sequence_delta_b200.inputs import WORKLOADS, make_mixer_prefill_inputs
+    out, launches = {}, 0
+    timer = gdn.Timer()
+    for name in ("prefill_35b", "varlen_64"):
+        W = WORKLOADS[name]
+        lens = "random" if W.get("lengths") == "random" else None
+        P = make_mixer_prefill_inputs(lens, num_seqs=W["num_seqs"], seq_len=W.get("seq_len", 256),
+                                      len_lo=W.get("len_lo", 128), len_hi=W.get("len_hi", 8192),
+                                      H_qk=W["H_qk"], H_v=W["H_v"], d=W["d_k"],
+                                      state_std=W.get("state_std"), seed=rank, device=dev)
+        T, C = P.x.shape
+        N, H_qk, H_v, d = P.num_seqs, P.H_qk, P.z.shape[1], P.z.shape[2]
+        K = P.conv_weight.shape[1]
+        y = torch.empty_like(P.z)
+        Sf = torch.empty((N, H_v, d, d), device=dev, dtype=torch.float32)
+        cout = torch.empty_like(P.conv_state)
+        ws = torch.empty((gdn.mixer_workspace_size(N, T, H_qk, H_v, d),), device=dev,
+                         dtype=torch.uint8)
+        fused = lambda tm=None: gdn.gdn_mixer_prefill(
+            P.x, P.conv_weight, P.conv_bias, P.cu_seqlens, P.a, P.b, P.A_log, P.dt_bias, P.z,
+            P.norm_weight, H_qk=H_qk, conv_state_in=P.conv_state, conv_state_out=cout,
+            initial_state=P.initial_state, out=y, final_state=Sf, workspace=ws, timer=tm)
+        # the separate steps on dense parts (q, k, v each its own [T, H d] tensor)
+        bounds = [(0, H_qk * d), (H_qk * d, 2 * H_qk * d), (2 * H_qk * d, C)]
+        xs = [P.x[:, a_:b_].contiguous() for a_, b_ in bounds]
+        wsp = [P.conv_weight[a_:b_].contiguous() for a_, b_ in bounds]
+        bsp = [P.conv_bias[a_:b_].contiguous() for a_, b_ in bounds]
+        csp = [P.conv_state[:, :, a_:b_].contiguous() for a_, b_ in bounds]
+        ys = [torch.empty_like(x_) for x_ in xs]
+        cos = [torch.empty_like(c_) for c_ in csp]
+        o = torch.empty_like(P.z)
+        pws = torch.empty((gdn.workspace_size(N, T, H_qk, H_v, d, d),), device=dev,
+                          dtype=torch.uint8)
+
+        def steps():
+            for x_, w_, b_, c_, y_, co_ in zip(xs, wsp, bsp, csp, ys, cos):
+                gdn.gdn_conv1d_silu(x_, w_, b_, P.cu_seqlens, c_, out=y_, conv_state_out=co_)
+            gdn.gdn_prefill(ys[0].view(T, H_qk, d), ys[1].view(T, H_qk, d), ys[2].view(T, H_v, d),
+                            P.a, P.b, P.A_log, P.dt_bias, P.cu_seqlens, P.initial_state, out=o,
+                            final_state=Sf, workspace=pws)
+            gdn.gdn_rmsnorm_gated(o, P.z, P.norm_weight, 1e-6, out=y)
+
+        ms_f = _time_op(fused, iters, flush, stream)
+        ms_s = _time_op(steps, iters, flush, stream)
+        fused(timer)
+        kn = timer.times()
+        launches += 2 * (iters + 3) * 6
+        byts = mixer_call_bytes(T, N, H_qk, H_v, d, K, 2, P.initial_state is not None)
+        out[name] = {
+            "workload": f"N={N}, T_total={T}, H_qk={H_qk}, H_v={H_v}, d={d}, conv_dim={C}, K={K}, "
+                        "bf16 x/z/y, conv cache in and out"
+                        + (", initial states in" if P.initial_state is not None else "")
+                        + ", final states out",
+            "fused_ms": ms_f, "separate_steps_ms": ms_s,
+            "separate_steps": "3 conv1d_silu (q, k, v parts) + gdn_prefill + gdn_rmsnorm_gated",
+            "fused_kernels_ms": {k_: v_ for k_, v_ in kn},
+            "tokens_per_s": T / (ms_f / 1e3), "algorithmic_bytes": byts,
+            "achieved_gbs": byts / (ms_f / 1e3) / 1e9,
+            "frac_hbm": byts / (ms_f / 1e3) / 1e9 / hbm, "peak_source": peak_src}
+        del P, y, Sf, cout, ws, xs, ys, o, pws
+    timer.close()
+    out["l2"] = "flushed (512 MiB write) before every timed call"
+    out["iters"] = iters
+    return out, launches
+
+
 def run_decode_variants(rank, dev, flush, stream, hbm, peak_src, iters):
     """gdn_decode_slots on the 397B-A17B decode shape (256 sequences, 64 V heads, d=128):
     L = 1 with the states scattered over a pool of 512 slots (continuous batching), and
@@ -468,6 +551,10 @@ def run_ours(args):
         if not args.no_decode:
             dvar, dvar_launches = run_decode_variants(rank, dev, flush, stream, hbm, peak_src,
                                                       args.mixer_iters)
+        mixp, mixp_launches = None, 0
+        if not args.no_mixer:
+            mixp, mixp_launches = run_mixer_prefill(rank, dev, flush, stream, hbm, peak_src,
+                                                    args.other_iters)
         other, other_launches = None, 0
         if not args.no_other_prefill:
             other, other_launches = run_other_prefill(rank, dev, flush, stream, hbm, tc_burst,
@@ -513,12 +600,13 @@ def run_ours(args):
         "e2e": e2e,
         "gpu_launches": sum(len(v_) for v_ in kernel_ms.values()),
         "gpu_launches_other_blocks": (args.decode_steps if dec else 0) + mixer_launches
-                                     + dvar_launches + other_launches,
+                                     + dvar_launches + other_launches + mixp_launches,
         "clocks": clocks.summary(),
         "prefill_other_configs": other,
         "decode": dec,
         "decode_slots": dvar,
         "mixer": mixer,
+        "mixer_prefill": mixp,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()

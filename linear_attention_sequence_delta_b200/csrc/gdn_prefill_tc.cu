@@ -442,17 +442,24 @@ __device__ __forceinline__ void prep_worker(
     const int hh = warp >> 2;                 // which 32 columns of that row
     uint32_t mphase = 0;
     bool failed = false;
+    // A worker's units only move forward, so the sequence of each is found by a short
+    // forward scan from the previous one's (the first by bisection): one dependent load
+    // of the offsets per unit instead of a bisection's worth.
+    int n = 0;
+    if (worker < total_units) {
+        const int cg = worker / H_qk;
+        int hi = N;
+        while (hi - n > 1) {
+            const int mid = (n + hi) >> 1;
+            if (choff[mid] <= cg) n = mid; else hi = mid;
+        }
+    }
 
 #pragma unroll 1
     for (int unit = worker; unit < total_units; unit += nworkers) {
         const int cg = unit / H_qk;
         const int j = unit - cg * H_qk;
-        int lo = 0, hi = N;  // sequence n with choff[n] <= cg < choff[n+1]
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (choff[mid] <= cg) lo = mid; else hi = mid;
-        }
-        const int n = lo;
+        while (choff[n + 1] <= cg) ++n;  // sequence n: choff[n] <= cg < choff[n + 1]
         const int64_t t0 = (int64_t)cu_seqlens[n] + (int64_t)(cg - choff[n]) * kC;
         const int L = (int)min((int64_t)kC, (int64_t)cu_seqlens[n + 1] - t0);
 
@@ -583,6 +590,22 @@ __device__ __forceinline__ void prep_worker(
         // every later head's are built while the head before writes its record.
         exp_tables(sGall, sU, sE, sCI, tid);
         named_bar_sync(bar_id, kPrepThreads);
+        {
+            const int un = unit + nworkers;
+            if (un < total_units) {
+                const int cgn = un / H_qk, jn = un - cgn * H_qk;
+                int nn = n;
+                while (choff[nn + 1] <= cgn) ++nn;
+                const int64_t t0n = (int64_t)cu_seqlens[nn] + (int64_t)(cgn - choff[nn]) * kC;
+                const int Ln = (int)min((int64_t)kC, (int64_t)cu_seqlens[nn + 1] - t0n);
+                const int rr = tid >> 2;
+                if (rr < Ln)
+                    prefetch_l2(((tid & 2) ? q : k) + (size_t)(t0n + rr) * qk_tok + (size_t)jn * kD +
+                                (tid & 1) * 64);
+                if (tid < 2 * kC && (tid & 63) < Ln)
+                    prefetch_l2(((tid >> 6) ? b : a) + (size_t)(t0n + (tid & 63)) * H_v + jn * r);
+            }
+        }
 
 #pragma unroll 1
         for (int hr = 0; hr < r; ++hr) {
