@@ -182,6 +182,10 @@ class Timer:
         self._t = self._lib.gdn_timer_create()
         if not self._t:
             raise GDNError(4, "gdn_timer_create")
+        # held here so that close() needs no module global (at interpreter exit those
+        # may already be gone when the finaliser runs)
+        self._handle = ctypes.c_void_p(self._t)
+        self._destroy = self._lib.gdn_timer_destroy
 
     def times(self) -> list:
         """[(kernel name, milliseconds)] of the most recent call made with this timer
@@ -195,7 +199,7 @@ class Timer:
 
     def close(self):
         if getattr(self, "_t", None):
-            self._lib.gdn_timer_destroy(ctypes.c_void_p(self._t))
+            self._destroy(self._handle)
             self._t = None
 
     def __del__(self):

@@ -228,6 +228,23 @@ def test_kernel_timing_names_and_durations():
     timer.close()
 
 
+def test_timer_left_open_at_exit():
+    """A timer still alive when the interpreter exits is released by its finaliser
+    without an error (module globals may already be gone by then)."""
+    import os
+    import subprocess
+    import sys
+    code = ("import torch\n"
+            "from linear_attention_sequence_delta_b200 import gdn\n"
+            "torch.zeros(1, device='cuda')\n"
+            "t = gdn.Timer()\n")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                       timeout=300, cwd=root)
+    assert r.returncode == 0, r.stderr
+    assert "Exception ignored" not in r.stderr and "Error" not in r.stderr, r.stderr
+
+
 @pytest.mark.parametrize("wl", ["prefill_35b", "varlen_64"])
 def test_fused_equals_split(wl):
     """The overlapped single launch (half-row chain blocks for the 35B layer's 32 chains,
