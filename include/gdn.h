@@ -59,7 +59,9 @@ typedef enum {
     GDN_ERR_CUDA = 4,        /* a CUDA runtime call failed (launch, attribute)    */
     GDN_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out                */
     GDN_ERR_BAD_SEQLENS = 6, /* cu_seqlens not non-decreasing / out of range      */
-    GDN_ERR_BAD_SLOT = 7     /* a state / cache slot index >= the pool size       */
+    GDN_ERR_BAD_SLOT = 7,    /* a state / cache slot index >= the pool size       */
+    GDN_ERR_BAD_INDEX = 8    /* an index a kernel formed lies outside its buffer  */
+                             /* (checked only by libgdn_debug.so, see below)      */
 } gdn_status;
 
 typedef enum { GDN_BF16 = 0, GDN_FP32 = 1 } gdn_dtype;
@@ -159,6 +161,12 @@ int gdn_prefill(const void* q, const void* k, const void* v, int32_t io_dtype,
  *                      the call then ends with GDN_ERR_TIMEOUT in the device
  *                      status word (outputs undefined) and the context stays
  *                      usable. Nothing faults. Other launches ignore it.
+ *                      GDN_FAULT_BAD_INDEX (libgdn_debug.so only; GDN_ERR_UNSUPPORTED
+ *                      in libgdn.so): every chain of the tensor-core path passes one
+ *                      index just past the end of the record array through its index
+ *                      check before its first chunk, and reads nothing there; the
+ *                      check records GDN_ERR_BAD_INDEX and its site, and the call
+ *                      computes its results as without the option.
  *   wait_limit_cycles  limit of every bounded device-side wait of the tensor-core
  *                      path, in SM clock cycles; 0 = the default (4e9, about 2 s).
  *   timer              NULL, or a timer from gdn_timer_create: CUDA events are
@@ -171,7 +179,7 @@ enum {
     GDN_IMPL_TENSOR_CORE_SPLIT = 3,
     GDN_IMPL_TENSOR_CORE_WHOLE_ROWS = 4
 };
-enum { GDN_FAULT_NONE = 0, GDN_FAULT_WITHHOLD_RECORDS = 1 };
+enum { GDN_FAULT_NONE = 0, GDN_FAULT_WITHHOLD_RECORDS = 1, GDN_FAULT_BAD_INDEX = 2 };
 
 typedef struct gdn_timer gdn_timer;
 
@@ -456,10 +464,32 @@ int gdn_mixer_prefill(const void* x, int32_t io_dtype, const float* conv_weight,
 
 /*
  * Synchronise `stream`, then return and clear the device status word of the
- * current device (GDN_OK, GDN_ERR_BAD_SEQLENS, GDN_ERR_BAD_SLOT or GDN_ERR_TIMEOUT), or
- * GDN_ERR_CUDA if the synchronisation itself failed.
+ * current device (GDN_OK, GDN_ERR_BAD_SEQLENS, GDN_ERR_BAD_SLOT, GDN_ERR_TIMEOUT or,
+ * in libgdn_debug.so, GDN_ERR_BAD_INDEX), or GDN_ERR_CUDA if the synchronisation
+ * itself failed.
  */
 int gdn_sync_status(void* stream);
+
+/*
+ * The debug build. `python -m linear_attention_sequence_delta_b200.build --debug`
+ * builds libgdn_debug.so: the same ABI, in which the kernels of the tensor-core
+ * prefill (chunk offsets, preparation, chains, the overlapped launch, with the fused
+ * convolution and norm) check each global-memory index they form against the extent
+ * of its buffer before the access (the decode kernels' only index taken from data, the
+ * state slot, is checked in every build: GDN_ERR_BAD_SLOT). An index outside
+ * records GDN_ERR_BAD_INDEX in the device status word and the source line of the
+ * first failed check in a second device word, and the access is skipped (a load
+ * reads zeros): nothing faults or traps. In libgdn.so the checks are compiled out.
+ * Tensor-memory-accelerator copies are not checked: the hardware bounds their
+ * coordinates itself (reads past a tensor's end fill zeros, writes there are dropped).
+ *   gdn_debug_build           1 in libgdn_debug.so, 0 in libgdn.so; touches no GPU.
+ *   gdn_debug_bad_index_site  synchronises `stream`, then returns and clears the
+ *                             source line of the first failed index check on the
+ *                             current device since the last call (0: none), or
+ *                             -GDN_ERR_CUDA if the synchronisation failed.
+ */
+int gdn_debug_build(void);
+int gdn_debug_bad_index_site(void* stream);
 
 #ifdef __cplusplus
 }

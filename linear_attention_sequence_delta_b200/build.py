@@ -1,12 +1,14 @@
 """Build libgdn.so (the CUDA kernels and the C ABI) in-tree, for sm_100a only.
 
-    python -m linear_attention_sequence_delta_b200.build [--force] [--verbose]
+    python -m linear_attention_sequence_delta_b200.build [--force] [--verbose] [--debug]
 
 Each csrc/*.cu is compiled by nvcc to an object under _build/ (in parallel),
 then linked into linear_attention_sequence_delta_b200/libgdn.so with the CUDA
 runtime linked statically, so the library loads on a machine without a GPU
 (no CUDA call happens at load time) and does not depend on the runtime that
-torch ships.
+torch ships. With --debug the same sources are compiled with GDN_DEBUG=1 (the
+kernels' index checks, see include/gdn.h) into libgdn_debug.so, objects under
+_build/debug/.
 """
 from __future__ import annotations
 
@@ -24,6 +26,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libgdn.so")
+DEBUG_LIB = os.path.join(PKG, "libgdn_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC,
@@ -42,15 +45,19 @@ def _deps_mtime() -> float:
     return max(os.path.getmtime(f) for f in files)
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
+def build(force: bool = False, verbose: bool = False, extra_flags=(), debug: bool = False) -> str:
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= _deps_mtime():
-        return LIB
-    os.makedirs(BUILD, exist_ok=True)
+    lib = DEBUG_LIB if debug else LIB
+    objdir = os.path.join(BUILD, "debug") if debug else BUILD
+    if debug:
+        extra_flags = (*extra_flags, "-DGDN_DEBUG=1")
+    if not force and os.path.exists(lib) and os.path.getmtime(lib) >= _deps_mtime():
+        return lib
+    os.makedirs(objdir, exist_ok=True)
     cc = nvcc()
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+        obj = os.path.join(objdir, os.path.basename(src) + ".o")
         cmd = [cc, *ARCH, *NVCC_FLAGS, *extra_flags, "-c", src, "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
@@ -63,18 +70,20 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
 
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
         objs = list(ex.map(compile_one, srcs))
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [cc, *ARCH, "-shared", "-cudart", "static", *objs, "-o", tmp]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true", help="print ptxas register/smem usage")
+    ap.add_argument("--debug", action="store_true",
+                    help="build libgdn_debug.so (kernels with index checks, GDN_DEBUG=1)")
     args = ap.parse_args()
-    print(build(force=args.force, verbose=args.verbose))
+    print(build(force=args.force, verbose=args.verbose, debug=args.debug))

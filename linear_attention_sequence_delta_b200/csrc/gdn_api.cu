@@ -12,7 +12,7 @@ namespace gdn {
 
 // One status word per device: kernels record content errors (bad cu_seqlens,
 // an expired bounded wait) here instead of trapping.
-__device__ int g_status_word;
+__device__ int g_status_word[2];  // [0] status, [1] first failed index check (debug build)
 
 namespace {
 constexpr int kMaxDevices = 64;
@@ -95,6 +95,7 @@ const char* gdn_status_string(int status) {
         case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
         case GDN_ERR_BAD_SEQLENS: return "GDN_ERR_BAD_SEQLENS";
         case GDN_ERR_BAD_SLOT: return "GDN_ERR_BAD_SLOT";
+        case GDN_ERR_BAD_INDEX: return "GDN_ERR_BAD_INDEX";
         default: return "GDN_ERR_UNKNOWN";
     }
 }
@@ -143,8 +144,10 @@ int prefill_common(const void* q, const void* k, const void* v, int32_t io_dtype
     if (options) {
         if (options->impl < GDN_IMPL_AUTO || options->impl > GDN_IMPL_TENSOR_CORE_WHOLE_ROWS)
             return GDN_ERR_INVALID_ARG;
-        if (options->fault != GDN_FAULT_NONE && options->fault != GDN_FAULT_WITHHOLD_RECORDS)
+        if (options->fault != GDN_FAULT_NONE && options->fault != GDN_FAULT_WITHHOLD_RECORDS &&
+            options->fault != GDN_FAULT_BAD_INDEX)
             return GDN_ERR_INVALID_ARG;
+        if (options->fault == GDN_FAULT_BAD_INDEX && !kDebugBuild) return GDN_ERR_UNSUPPORTED;
         if (options->wait_limit_cycles < 0) return GDN_ERR_INVALID_ARG;
         opt.impl = options->impl;
         opt.fault = options->fault;
@@ -300,8 +303,10 @@ int gdn_mixer_prefill(const void* x, int32_t io_dtype, const float* conv_weight,
     if (options) {
         if (options->impl < GDN_IMPL_AUTO || options->impl > GDN_IMPL_TENSOR_CORE_WHOLE_ROWS)
             return GDN_ERR_INVALID_ARG;
-        if (options->fault != GDN_FAULT_NONE && options->fault != GDN_FAULT_WITHHOLD_RECORDS)
+        if (options->fault != GDN_FAULT_NONE && options->fault != GDN_FAULT_WITHHOLD_RECORDS &&
+            options->fault != GDN_FAULT_BAD_INDEX)
             return GDN_ERR_INVALID_ARG;
+        if (options->fault == GDN_FAULT_BAD_INDEX && !kDebugBuild) return GDN_ERR_UNSUPPORTED;
         if (options->wait_limit_cycles < 0) return GDN_ERR_INVALID_ARG;
         opt.impl = options->impl;
         opt.fault = options->fault;
@@ -562,6 +567,21 @@ int gdn_timer_read(gdn_timer* t, float* ms, int32_t max_kernels) {
 
 const char* gdn_timer_kernel_name(const gdn_timer* t, int32_t i) {
     return (t && i >= 0 && i < t->n) ? t->name[i] : nullptr;
+}
+
+int gdn_debug_build(void) { return kDebugBuild ? 1 : 0; }
+
+int gdn_debug_bad_index_site(void* stream) {
+    int* st = device_status_ptr();
+    if (!st) return -GDN_ERR_CUDA;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return -GDN_ERR_CUDA;
+    int val = 0;
+    if (cudaMemcpy(&val, st + 1, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return -GDN_ERR_CUDA;
+    const int zero = 0;
+    if (val != 0 && cudaMemcpy(st + 1, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+        return -GDN_ERR_CUDA;
+    return val;
 }
 
 int gdn_sync_status(void* stream) {

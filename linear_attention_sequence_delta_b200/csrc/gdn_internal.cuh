@@ -18,10 +18,19 @@ constexpr float kL2Eps = 1e-6f;     // inside the square root of the QK L2 norm
 // otherwise turn G_i - G_j into inf - inf = NaN.
 constexpr float kMinLogDecay = -128.f;
 
-// Device status word values (written by kernels, read by gdn_sync_status).
+// Device status word values (written by kernels, read by gdn_sync_status). The status
+// pointer kernels receive addresses two words: [0] the status, [1] (debug build) the
+// source line of the first failed index check.
 constexpr int kStatusBadSeqlens = GDN_ERR_BAD_SEQLENS;
 constexpr int kStatusTimeout = GDN_ERR_TIMEOUT;
 constexpr int kStatusBadSlot = GDN_ERR_BAD_SLOT;
+constexpr int kStatusBadIndex = GDN_ERR_BAD_INDEX;
+
+// The debug build (libgdn_debug.so) is compiled with GDN_DEBUG=1.
+#ifndef GDN_DEBUG
+#define GDN_DEBUG 0
+#endif
+constexpr bool kDebugBuild = GDN_DEBUG != 0;
 
 // ---- small device helpers ---------------------------------------------------
 
@@ -66,6 +75,26 @@ __device__ __forceinline__ float gate_beta(float b) { return 1.f / (1.f + expf(-
 __device__ __forceinline__ void set_status(int* status, int code) {
     if (status) atomicCAS(status, 0, code);
 }
+
+// Index check of the debug build: true when 0 <= idx < count. Otherwise it records
+// GDN_ERR_BAD_INDEX in the status word and `line` in the second word (the first failed
+// check's), and the caller skips the access. Compiled out (always true) in libgdn.so.
+__device__ __forceinline__ bool in_bounds_at(long long idx, long long count, int* status,
+                                             int line) {
+#if GDN_DEBUG
+    if (idx >= 0 && idx < count) return true;
+    if (status) {
+        atomicCAS(status, 0, GDN_ERR_BAD_INDEX);
+        atomicCAS(status + 1, 0, line);
+    }
+    return false;
+#else
+    (void)idx; (void)count; (void)status; (void)line;
+    return true;
+#endif
+}
+#define GDN_IN_BOUNDS(idx, count, status) \
+    ::gdn::in_bounds_at((long long)(idx), (long long)(count), (status), __LINE__)
 
 // Where each sequence's initial and final states live. Without slots sequence n uses
 // state n of the initial / final arrays. With slots it uses entry slots[n] of one pool,

@@ -297,7 +297,8 @@ __device__ __forceinline__ float silu_tanh(float x) {
 // standalone convolution kernel, so both give the same bits. A thread takes 4 channels x
 // 8 tokens at a time; consecutive threads take consecutive channel groups.
 __device__ __forceinline__ void conv_unit(const MixerFusion& mix, int n, int64_t s0, int64_t t0,
-                                          int L, int j, int r, int H_qk, uint8_t* KQ, int tid) {
+                                          int L, int j, int r, int H_qk, uint8_t* KQ, int tid,
+                                          int64_t T_total, int N, int* status) {
     const int C = mix.conv_dim, K = mix.K;
     const int nv4 = 64 + 32 * r;  // 4-channel groups: q 32, k 32, v 32 per V head
     const int items = nv4 * 8;    // x 8 segments of 8 tokens
@@ -317,11 +318,14 @@ __device__ __forceinline__ void conv_unit(const MixerFusion& mix, int n, int64_t
             raw[s_] = make_uint2(0u, 0u);
             const int64_t p = t0 + tt0 - (K - 1) + s_;
             if (s_ < 7 + K && p < t0 + L) {
-                if (p >= s0)
-                    raw[s_] = *reinterpret_cast<const uint2*>(mix.x + (size_t)p * C + c);
-                else if (mix.cache_in)
-                    raw[s_] = *reinterpret_cast<const uint2*>(
-                        mix.cache_in + ((size_t)n * (K - 1) + (K - 1) + (p - s0)) * C + c);
+                if (p >= s0) {
+                    if (GDN_IN_BOUNDS(p * C + c + 3, T_total * C, status))
+                        raw[s_] = *reinterpret_cast<const uint2*>(mix.x + (size_t)p * C + c);
+                } else if (mix.cache_in) {
+                    const int64_t ci = ((int64_t)n * (K - 1) + (K - 1) + (p - s0)) * C + c;
+                    if (GDN_IN_BOUNDS(ci + 3, (int64_t)N * (K - 1) * C, status))
+                        raw[s_] = *reinterpret_cast<const uint2*>(mix.cache_in + ci);
+                }
             }
         }
     };
@@ -359,7 +363,8 @@ __device__ __forceinline__ void conv_unit(const MixerFusion& mix, int n, int64_t
                                  pack_bf16x2(silu_fast(acc[2]), silu_fast(acc[3])));
             if (v4 < 64)
                 *reinterpret_cast<uint2*>(kq + sw128_off((uint32_t)(row0 + tt), (uint32_t)((cc & 63) >> 3))) = out;
-            if (live) *reinterpret_cast<uint2*>(mix.qkvc + (size_t)(t0 + tt) * C + c) = out;
+            if (live && GDN_IN_BOUNDS((t0 + tt) * C + c + 3, T_total * C, status))
+                *reinterpret_cast<uint2*>(mix.qkvc + (size_t)(t0 + tt) * C + c) = out;
         }
     };
     // two items in flight: both windows are loaded before either is computed
@@ -400,7 +405,8 @@ __device__ __forceinline__ void prep_worker(
     uint8_t* __restrict__ rec, int* status,
     unsigned long long* flags, unsigned long long epoch, uint8_t* sm, const int tid,
     const int bar_id, const int worker, const int nworkers, const bool relinquish,
-    const long long wait_cycles, const MixerFusion& mix, const int64_t qk_tok) {
+    const long long wait_cycles, const MixerFusion& mix, const int64_t qk_tok,
+    const int64_t T_total) {
     uint8_t* KQ = sm + PS_KQ;
     float* Ts = reinterpret_cast<float*>(sm + PS_TS);
     float* As = reinterpret_cast<float*>(sm + PS_AS);
@@ -421,6 +427,10 @@ __device__ __forceinline__ void prep_worker(
     const int warp = tid >> 5, lane = tid & 31;
     const int r = H_v / H_qk;
     const int total_units = choff[N] * H_qk;
+    // extents of the debug build's index checks: records, and q / k rows from the pointer
+    // (the last token's row of the last QK head ends there)
+    const int64_t total_records = (int64_t)choff[N] * H_v;
+    const int64_t qk_extent = T_total > 0 ? (T_total - 1) * qk_tok + (int64_t)H_qk * kD : 0;
 
     constexpr uint32_t tcols = 64u;
     if (warp == 0) {
@@ -459,22 +469,23 @@ __device__ __forceinline__ void prep_worker(
     for (int unit = worker; unit < total_units; unit += nworkers) {
         const int cg = unit / H_qk;
         const int j = unit - cg * H_qk;
-        while (choff[n + 1] <= cg) ++n;  // sequence n: choff[n] <= cg < choff[n + 1]
+        // sequence n: choff[n] <= cg < choff[n + 1]
+        while (GDN_IN_BOUNDS(n + 1, N + 1, status) && choff[n + 1] <= cg) ++n;
         const int64_t t0 = (int64_t)cu_seqlens[n] + (int64_t)(cg - choff[n]) * kC;
         const int L = (int)min((int64_t)kC, (int64_t)cu_seqlens[n + 1] - t0);
 
         // ---- raw K and Q rows (sw128), or the convolution that makes them; gates of
         // the r V heads
         if constexpr (kConv) {
-            conv_unit(mix, n, cu_seqlens[n], t0, L, j, r, H_qk, KQ, tid);
+            conv_unit(mix, n, cu_seqlens[n], t0, L, j, r, H_qk, KQ, tid, T_total, N, status);
         } else {
 #pragma unroll
             for (int it = 0; it < 4; ++it) {
                 const int idx = tid + kPrepThreads * it;  // 0 .. 1023
                 const int rr = idx >> 4, ch = idx & 15;
-                const bool live = rr < L;
-                const int64_t tok = live ? t0 + rr : 0;
+                const int64_t tok = rr < L ? t0 + rr : 0;
                 const size_t rowk = (size_t)tok * qk_tok + (size_t)j * kD + ch * 8;
+                const bool live = rr < L && GDN_IN_BOUNDS(rowk + 7, qk_extent, status);
                 const uint32_t off = (uint32_t)(ch >> 3) * 16384u;
                 cp_async_16(KQ + off + sw128_off(rr, ch & 7), k + rowk, live ? 16u : 0u);
                 cp_async_16(KQ + off + sw128_off(rr + 64, ch & 7), q + rowk, live ? 16u : 0u);
@@ -484,15 +495,16 @@ __device__ __forceinline__ void prep_worker(
             const int which = idx / (r * kC);            // 0: a, 1: b
             const int rem = idx - which * r * kC;
             const int hr = rem >> 6, t = rem & 63;
-            const bool live = t < L;
-            const int64_t tok = live ? t0 + t : 0;
+            const int64_t tok = t < L ? t0 + t : 0;
+            const bool live = t < L && GDN_IN_BOUNDS(tok * H_v + j * r + hr, T_total * H_v, status);
             const float* src = (which ? b : a) + (size_t)tok * H_v + j * r + hr;
             cp_async_4(AB + (which * kMaxGroup + hr) * kC + t, src, live ? 4u : 0u);
         }
         if (tid < 2 * r) {
             const int hr = tid >> 1;
-            cp_async_4(sPar + (tid & 1) * kMaxGroup + hr, ((tid & 1) ? dt_bias : A_log) + j * r + hr,
-                       4u);
+            const bool ok = GDN_IN_BOUNDS(j * r + hr, H_v, status);
+            cp_async_4(sPar + (tid & 1) * kMaxGroup + hr,
+                       ((tid & 1) ? dt_bias : A_log) + (ok ? j * r + hr : 0), ok ? 4u : 0u);
         }
         cp_async_commit();
         cp_async_wait<0>();
@@ -556,6 +568,7 @@ __device__ __forceinline__ void prep_worker(
             *reinterpret_cast<float2*>(sGall + hr * kC + ta) = make_float2(Ga, Gb);
             *reinterpret_cast<float2*>(sBall + hr * kC + ta) = make_float2(ba, bb);
             float* rg = reinterpret_cast<float*>(rec + ((size_t)cg * H_v + h) * kRecBytes + REC_G);
+            if (!GDN_IN_BOUNDS((int64_t)cg * H_v + h, total_records, status)) continue;
             const float ea = __expf(Ga), eb = __expf(Gb);
             const float2 rk2 = *reinterpret_cast<const float2*>(rk + ta);
             const float2 rq2 = *reinterpret_cast<const float2*>(rq + ta);
@@ -595,14 +608,16 @@ __device__ __forceinline__ void prep_worker(
             if (un < total_units) {
                 const int cgn = un / H_qk, jn = un - cgn * H_qk;
                 int nn = n;
-                while (choff[nn + 1] <= cgn) ++nn;
+                while (GDN_IN_BOUNDS(nn + 1, N + 1, status) && choff[nn + 1] <= cgn) ++nn;
                 const int64_t t0n = (int64_t)cu_seqlens[nn] + (int64_t)(cgn - choff[nn]) * kC;
                 const int Ln = (int)min((int64_t)kC, (int64_t)cu_seqlens[nn + 1] - t0n);
                 const int rr = tid >> 2;
-                if (rr < Ln)
+                if (rr < Ln && GDN_IN_BOUNDS((t0n + rr) * qk_tok + (int64_t)jn * kD + 127, qk_extent,
+                                             status))
                     prefetch_l2(((tid & 2) ? q : k) + (size_t)(t0n + rr) * qk_tok + (size_t)jn * kD +
                                 (tid & 1) * 64);
-                if (tid < 2 * kC && (tid & 63) < Ln)
+                if (tid < 2 * kC && (tid & 63) < Ln &&
+                    GDN_IN_BOUNDS((t0n + (tid & 63)) * H_v + jn * r, T_total * H_v, status))
                     prefetch_l2(((tid >> 6) ? b : a) + (size_t)(t0n + (tid & 63)) * H_v + jn * r);
             }
         }
@@ -611,6 +626,7 @@ __device__ __forceinline__ void prep_worker(
         for (int hr = 0; hr < r; ++hr) {
             const int h = j * r + hr;
             uint8_t* R = rec + ((size_t)cg * H_v + h) * kRecBytes;
+            const bool rec_ok = GDN_IN_BOUNDS((int64_t)cg * H_v + h, total_records, status);
             const float* hBeta = sBall + hr * kC;  // this head's beta
 
             // ---- A rows 0-63 -> As (fp32); P rows 64-127 -> staging (bf16 image);
@@ -720,12 +736,14 @@ __device__ __forceinline__ void prep_worker(
                 w.y = pack_bf16x2(f0.z * b0.z, f0.w * b0.w);
                 w.z = pack_bf16x2(f1.x * b1.x, f1.y * b1.y);
                 w.w = pack_bf16x2(f1.z * b1.z, f1.w * b1.w);
-                *reinterpret_cast<uint4*>(R + REC_T + sw128_off(row, ch)) = w;
-                reinterpret_cast<uint4*>(R + REC_P)[idx] = reinterpret_cast<const uint4*>(Pst)[idx];
+                if (rec_ok) {
+                    *reinterpret_cast<uint4*>(R + REC_T + sw128_off(row, ch)) = w;
+                    reinterpret_cast<uint4*>(R + REC_P)[idx] = reinterpret_cast<const uint4*>(Pst)[idx];
+                }
             }
             if (hr + 1 < r) exp_tables(sGall + (hr + 1) * kC, sU, sE, sCI, tid);
             named_bar_sync(bar_id, kPrepThreads);  // Ts, As, Xs, the staging and tables are reused
-            if (flags && tid == 0) publish_record(flags, (size_t)cg * H_v + h, epoch);
+            if (flags && tid == 0 && rec_ok) publish_record(flags, (size_t)cg * H_v + h, epoch);
         }
         tc_fence_before();  // this unit's TMEM reads precede the next unit's MMA
     }
@@ -744,13 +762,13 @@ __global__ void __launch_bounds__(kPrepThreads, kPrepBlocksPerSm) prep_kernel(
     const float* __restrict__ dt_bias, const int32_t* __restrict__ cu_seqlens,
     const int32_t* __restrict__ choff, int32_t N, int H_qk, int H_v, float scale,
     uint8_t* __restrict__ rec, int* status, long long wait_cycles, const MixerFusion mix,
-    int64_t qk_tok) {
+    int64_t qk_tok, int64_t T_total) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     prep_worker<kConv>(q, k, a, b, A_log, dt_bias, cu_seqlens, choff, N, H_qk, H_v, scale, rec,
                        status, nullptr, 0, sm, threadIdx.x, 1, blockIdx.x, gridDim.x, true,
-                       wait_cycles, mix, qk_tok);
+                       wait_cycles, mix, qk_tok, T_total);
 }
 
 // ==================================== chain =======================================
@@ -838,7 +856,8 @@ __device__ __forceinline__ bool wait_record(const unsigned long long* flag,
 // overwritten.
 __device__ __forceinline__ void write_conv_cache(const MixerFusion& mix, int n, int64_t s0,
                                                  int64_t s1, int h, int j, bool qk, int H_qk,
-                                                 int to, int nthreads) {
+                                                 int to, int nthreads, int64_t T_total, int N,
+                                                 int* status) {
     const int C = mix.conv_dim, Km1 = mix.K - 1;
     const int64_t len = s1 - s0;
     const int ng = qk ? 96 : 32;
@@ -850,11 +869,16 @@ __device__ __forceinline__ void write_conv_cache(const MixerFusion& mix, int n, 
         for (int i = 0; i < Km1; ++i) {
             const int64_t p = len - Km1 + i;
             uint2 v = make_uint2(0u, 0u);
-            if (p >= 0)
-                v = *reinterpret_cast<const uint2*>(mix.x + (size_t)(s0 + p) * C + c);
-            else if (mix.cache_in)
-                v = *reinterpret_cast<const uint2*>(mix.cache_in + ((size_t)n * Km1 + len + i) * C + c);
-            *reinterpret_cast<uint2*>(mix.cache_out + ((size_t)n * Km1 + i) * C + c) = v;
+            const int64_t cache_extent = (int64_t)N * Km1 * C;
+            if (p >= 0) {
+                if (GDN_IN_BOUNDS((s0 + p) * C + c + 3, T_total * C, status))
+                    v = *reinterpret_cast<const uint2*>(mix.x + (size_t)(s0 + p) * C + c);
+            } else if (mix.cache_in) {
+                if (GDN_IN_BOUNDS(((int64_t)n * Km1 + len + i) * C + c + 3, cache_extent, status))
+                    v = *reinterpret_cast<const uint2*>(mix.cache_in + ((size_t)n * Km1 + len + i) * C + c);
+            }
+            if (GDN_IN_BOUNDS(((int64_t)n * Km1 + i) * C + c + 3, cache_extent, status))
+                *reinterpret_cast<uint2*>(mix.cache_out + ((size_t)n * Km1 + i) * C + c) = v;
         }
     }
 }
@@ -872,7 +896,8 @@ __device__ __forceinline__ void chain_unit(
     float* Sfg, const StateIndex sref, int* status,
     const unsigned long long* flags, unsigned long long epoch, uint8_t* sm, const int tid,
     const int n, const int h, const int hv, const uint32_t tmem,
-    const int sync_id, const long long wait_cycles, const MixerFusion& mix) {
+    const int sync_id, const long long wait_cycles, const MixerFusion& mix, const int N,
+    const bool inject_bad_index) {
     static_assert(kM == 128 || kM == 64, "a chain block owns all 128 value rows or one half");
     static_assert(!kNorm || kM == 128, "the fused gated norm needs whole value rows");
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + CS_BAR);  // [3] slot landed
@@ -884,11 +909,14 @@ __device__ __forceinline__ void chain_unit(
 
     const int warp = tid >> 5, lane = tid & 31;
     const int j = h / (H_v / H_qk);
+    if (!GDN_IN_BOUNDS(n, N, status)) return;
     const int64_t s0 = cu_seqlens[n];
     const int64_t s1 = cu_seqlens[n + 1];
     if (bad_seq(s0, s1, T_total, n)) return;  // reported by the offsets kernel
     const int nchunks = (int)((s1 - s0 + kC - 1) / kC);
     const int cg0 = choff[n];
+    // records of the batch: the extent of the debug build's record index checks
+    const int64_t total_records = kDebugBuild ? (int64_t)choff[N] * H_v : 0;
 
     if (tid == 0) {
         for (int i = 0; i < kRing; ++i) mbar_init(&full[i], 1);
@@ -931,6 +959,7 @@ __device__ __forceinline__ void chain_unit(
     // results are discarded), so that the slot's barrier completes and no copy is left
     // in flight when the block exits.
     auto record_ready = [&](int c) -> bool {
+        if (!GDN_IN_BOUNDS((int64_t)(cg0 + c) * H_v + h, total_records, status)) return true;
         if (flags && !wait_record(flags + (size_t)(cg0 + c) * H_v + h, epoch, wait_cycles)) {
             *s_err = 1;
             return false;
@@ -940,8 +969,11 @@ __device__ __forceinline__ void chain_unit(
     auto load_record = [&](int c) {
         const int st = c % kRing;
         if (flags) asm volatile("fence.proxy.async.global;" ::: "memory");  // read by TMA
-        bulk_g2s(sm + st * kSlotBytes + SLOT_REC, rec + ((size_t)(cg0 + c) * H_v + h) * kRecBytes,
-                 kRecBytes, &full[st]);
+        // (debug build: an index outside copies the first record of this head instead, so
+        // that the slot's transaction count still completes)
+        size_t ri = (size_t)(cg0 + c) * H_v + h;
+        if (!GDN_IN_BOUNDS(ri, total_records, status)) ri = (size_t)h;
+        bulk_g2s(sm + st * kSlotBytes + SLOT_REC, rec + ri * kRecBytes, kRecBytes, &full[st]);
     };
 
     if (warp > kIssueWarp) {
@@ -957,6 +989,8 @@ __device__ __forceinline__ void chain_unit(
         if (kNorm && to < kD / 4)  // read by the norm after the loop's first barrier
             reinterpret_cast<float4*>(s_nw)[to] = reinterpret_cast<const float4*>(mix.norm_w)[to];
         int issued = 0;   // chunks whose tiles and record were issued
+        // a test of the index checks: one index just past the record array, nothing read
+        if (inject_bad_index && loader) (void)GDN_IN_BOUNDS(total_records, total_records, status);
         if (loader) {
             if (mix.x) {
                 for (int c = 0; c < kRing && c < nchunks; ++c) {
@@ -983,7 +1017,7 @@ __device__ __forceinline__ void chain_unit(
         uint4 zv[kNorm ? 8 : 1];
         auto load_gate_rows = [&](int c) {
             const int64_t tz = s0 + (int64_t)c * kC + (to >> 1);
-            if (c < nchunks && tz < s1) {
+            if (c < nchunks && tz < s1 && GDN_IN_BOUNDS(tz, T_total, status)) {
                 const bf16* zr = mix.z + ((size_t)tz * H_v + h) * kD + (to & 1) * 64;
 #pragma unroll
                 for (int q = 0; q < 8; ++q) zv[q] = *reinterpret_cast<const uint4*>(zr + q * 8);
@@ -1152,15 +1186,17 @@ __device__ __forceinline__ void chain_unit(
                 for (int idx = to; idx < L * kOutCh; idx += kOut) {
                     const int r = idx / kOutCh, ch = idx % kOutCh;
                     const uint4 w = *reinterpret_cast<const uint4*>(ost + tile64_off(r, ch * 8));
-                    *reinterpret_cast<uint4*>(o + ((size_t)(t0 + r) * H_v + h) * kD +
-                                              (kM == 64 ? 64 * hv : 0) + ch * 8) = w;
+                    if (GDN_IN_BOUNDS(t0 + r, T_total, status))
+                        *reinterpret_cast<uint4*>(o + ((size_t)(t0 + r) * H_v + h) * kD +
+                                                  (kM == 64 ? 64 * hv : 0) + ch * 8) = w;
                 }
                 named_bar_sync(2, kOut);
             }
             __syncwarp();
         }
         if (mix.cache_out && hv == 0 && *s_err == 0)
-            write_conv_cache(mix, n, s0, s1, h, j, h % (H_v / H_qk) == 0, H_qk, to, kOut);
+            write_conv_cache(mix, n, s0, s1, h, j, h % (H_v / H_qk) == 0, H_qk, to, kOut, T_total,
+                             N, status);
         if (loader) {
             bulk_wait_group<0>();  // o stores complete
             // Leave nothing in flight into shared memory (loads the chain did not
@@ -1278,6 +1314,7 @@ __device__ __forceinline__ void chain_unit(
             const uint32_t ctl = tmem + ((uint32_t)(qd * 32) << 16);
             bool rd, wr;  // the sequence's state (or pool slot): read at the start, written at the end
             const int sidx = sref.resolve(n, rd, wr, tid == 0 ? status : nullptr);
+            if (!GDN_IN_BOUNDS(sidx, sref.slots ? sref.num_slots : N, status)) rd = wr = false;
             const float* S0s = rd ? S0g : nullptr;
             float* Sfs = wr ? Sfg : nullptr;
             const size_t sbase = ((size_t)sidx * H_v + h) * kD * kD + (size_t)row * kD + 64 * hh;
@@ -1443,6 +1480,7 @@ __device__ __forceinline__ void chain_unit(
             const uint32_t ctl = tmem + ((uint32_t)(qd * 32) << 16);
             bool rd, wr;  // the sequence's state (or pool slot): read at the start, written at the end
             const int sidx = sref.resolve(n, rd, wr, tid == 0 ? status : nullptr);
+            if (!GDN_IN_BOUNDS(sidx, sref.slots ? sref.num_slots : N, status)) rd = wr = false;
             const float* S0s = rd ? S0g : nullptr;
             float* Sfs = wr ? Sfg : nullptr;
             const size_t hbase = ((size_t)sidx * H_v + h) * kD * kD;
@@ -1601,7 +1639,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
     const float* S0g, const int32_t* __restrict__ cu_seqlens,
     const int32_t* __restrict__ choff, int64_t T_total, int H_qk, int H_v,
     const uint8_t* __restrict__ rec, bf16* __restrict__ o, float* Sfg, const StateIndex sref,
-    int* status, long long wait_cycles, const MixerFusion mix) {
+    int* status, long long wait_cycles, const MixerFusion mix, int N, int inject_bad_index) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1617,7 +1655,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
     const uint32_t tmem = *s_tmem;
     chain_unit<128, kNorm>(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v, rec, o,
                     Sfg, sref, status, nullptr, 0, sm, threadIdx.x, blockIdx.x / H_v,
-                    blockIdx.x % H_v, 0, tmem, 1, wait_cycles, mix);
+                    blockIdx.x % H_v, 0, tmem, 1, wait_cycles, mix, N, inject_bad_index != 0);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1651,7 +1689,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
     int64_t T_total, int H_qk, int H_v, float scale, uint8_t* __restrict__ rec,
     bf16* __restrict__ o, float* Sfg, const StateIndex sref,
     int* status, unsigned long long* flags, unsigned long long epoch, int c0,
-    long long wait_cycles, int withhold_records, const MixerFusion mix) {
+    long long wait_cycles, int withhold_records, const MixerFusion mix, int inject_bad_index) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ int32_t s_choff[kFusedMaxSeqs + 1];
     __shared__ int s_bad;
@@ -1695,7 +1733,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
         prep_worker<kMix>(q, k, a, b, A_log, dt_bias, cu_seqlens, choff, N, H_qk, H_v, scale, rec,
                     status, withhold_records ? nullptr : flags, epoch, sm + sub * kPrepRegion,
                     tid & 255, 3 + sub, 2 * ((int)blockIdx.x - c0) + sub,
-                    2 * ((int)gridDim.x - c0), false, wait_cycles, mix, (int64_t)H_qk * kD);
+                    2 * ((int)gridDim.x - c0), false, wait_cycles, mix, (int64_t)H_qk * kD,
+                    T_total);
         return;
     }
     if (tid >= kChainThreads) return;
@@ -1713,7 +1752,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
     const int hv = kM == 64 ? (int)blockIdx.x & 1 : 0;
     chain_unit<kM, kMix>(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v, rec, o,
                    Sfg, sref, status, flags, epoch, sm, tid, u / H_v, u % H_v, hv, tmem,
-                   kChainSync, wait_cycles, mix);
+                   kChainSync, wait_cycles, mix, N, inject_bad_index != 0);
     tc_fence_before();
     named_bar_sync(kChainSync, kChainThreads);
     tc_fence_after();
@@ -1875,10 +1914,11 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
             bf16* ob = static_cast<bf16*>(o);
             int c0v = (int)chain_blocks;
             int withhold = opt.fault == GDN_FAULT_WITHHOLD_RECORDS ? 1 : 0;
+            int inject = opt.fault == GDN_FAULT_BAD_INDEX ? 1 : 0;
             void* args[] = {&tm_q, &tm_k, &tm_v, &tm_o, &qb, &kb, &a, &b, &A_log, &dt_bias, &S0,
                             &cu_seqlens, &choff, &N, &T, &H_qk, &H_v, &scale, &rec, &ob,
                             &S_final, &sref, &status, &flags, &epoch, &c0v, &wait_cycles,
-                            &withhold, const_cast<MixerFusion*>(&mix)};
+                            &withhold, const_cast<MixerFusion*>(&mix), &inject};
             timer_before(opt.timer, s);
             e = cudaLaunchCooperativeKernel(kfn, dim3(grid), dim3(kFusedThreads), args, kFusedSmem,
                                             s);
@@ -1934,7 +1974,7 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
         timer_before(opt.timer, s);
         prep_fn<<<prep_grid, kPrepThreads, kPrepSmem, s>>>(
             q_rows, k_rows, a, b, A_log, dt_bias, cu_seqlens, choff, N, H_qk, H_v, scale, rec,
-            status, wait_cycles, mix_split, qk_tok);
+            status, wait_cycles, mix_split, qk_tok, T);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         timer_after(opt.timer, s, "prep");
@@ -1942,7 +1982,8 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
     timer_before(opt.timer, s);
     chain_fn<<<(unsigned)chain_units, kChainThreads, kChainSmem, s>>>(
         tm_q, tm_k, tm_v, tm_o, S0, cu_seqlens, choff, T, H_qk, H_v, rec, static_cast<bf16*>(o),
-        S_final, sref, status, wait_cycles, mix_split);
+        S_final, sref, status, wait_cycles, mix_split, N,
+        opt.fault == GDN_FAULT_BAD_INDEX ? 1 : 0);
     e = cudaGetLastError();
     if (e == cudaSuccess) timer_after(opt.timer, s, "chain");
     return e;

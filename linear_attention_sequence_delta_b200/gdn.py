@@ -24,12 +24,16 @@ from typing import Optional, Tuple
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libgdn.so")
+DEFAULT_LIB_PATH = os.path.join(_HERE, "libgdn.so")
+DEBUG_LIB_PATH = os.path.join(_HERE, "libgdn_debug.so")  # kernels with index checks
+# The library a process loads: libgdn.so, or the file GDN_LIBRARY names (for instance
+# libgdn_debug.so, the same ABI with the kernels' index checks compiled in).
+LIB_PATH = os.environ.get("GDN_LIBRARY") or DEFAULT_LIB_PATH
 
 GDN_BF16, GDN_FP32 = 0, 1
 _STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "GDN_ERR_WORKSPACE",
            4: "GDN_ERR_CUDA", 5: "GDN_ERR_TIMEOUT", 6: "GDN_ERR_BAD_SEQLENS",
-           7: "GDN_ERR_BAD_SLOT"}
+           7: "GDN_ERR_BAD_SLOT", 8: "GDN_ERR_BAD_INDEX"}
 
 # Every symbol include/gdn.h declares (the tests check the library exports them all).
 EXPORTS = ["gdn_status_string", "gdn_version", "gdn_prefill_workspace_size", "gdn_gates",
@@ -38,10 +42,10 @@ EXPORTS = ["gdn_status_string", "gdn_version", "gdn_prefill_workspace_size", "gd
            "gdn_timer_kernel_name", "gdn_conv1d_silu", "gdn_conv1d_silu_decode",
            "gdn_rmsnorm_gated", "gdn_decode_slots", "gdn_decode_step_bf16_state",
            "gdn_prefill_slots", "gdn_prefill_slots_ex", "gdn_mixer_prefill",
-           "gdn_mixer_prefill_workspace_size"]
+           "gdn_mixer_prefill_workspace_size", "gdn_debug_build", "gdn_debug_bad_index_site"]
 GDN_IMPL_AUTO, GDN_IMPL_CUDA_CORE, GDN_IMPL_TENSOR_CORE, GDN_IMPL_TENSOR_CORE_SPLIT = 0, 1, 2, 3
 GDN_IMPL_TENSOR_CORE_WHOLE_ROWS = 4
-GDN_FAULT_NONE, GDN_FAULT_WITHHOLD_RECORDS = 0, 1
+GDN_FAULT_NONE, GDN_FAULT_WITHHOLD_RECORDS, GDN_FAULT_BAD_INDEX = 0, 1, 2
 
 
 class PrefillOptions(ctypes.Structure):
@@ -86,6 +90,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                     P]
     lib.gdn_sync_status.restype = ctypes.c_int
     lib.gdn_sync_status.argtypes = [P]
+    lib.gdn_debug_build.restype = ctypes.c_int
+    lib.gdn_debug_build.argtypes = []
+    lib.gdn_debug_bad_index_site.restype = ctypes.c_int
+    lib.gdn_debug_bad_index_site.argtypes = [P]
     lib.gdn_prefill_ex.restype = ctypes.c_int
     lib.gdn_prefill_ex.argtypes = [P, P, P, i32, P, P, P, P, P, P, i32, i64, i32, i32, i32, i32,
                                    f32, P, P, P, sz, P, P]
@@ -360,6 +368,20 @@ def gdn_sync_status(device=None) -> int:
     """Synchronise the current stream and return (and clear) the device status word."""
     lib = load_library()
     return int(lib.gdn_sync_status(_stream(device)))
+
+
+def debug_build() -> bool:
+    """True when the loaded library is libgdn_debug.so (kernels with index checks)."""
+    return bool(load_library().gdn_debug_build())
+
+
+def debug_bad_index_site(device=None) -> int:
+    """Synchronise the current stream; return (and clear) the source line of the first
+    failed index check of the debug build since the last call (0: none)."""
+    r = int(load_library().gdn_debug_bad_index_site(_stream(device)))
+    if r < 0:
+        raise GDNError(-r, "gdn_debug_bad_index_site")
+    return r
 
 
 def gdn_conv1d_silu(x, weight, bias, cu_seqlens, conv_state_in=None, *, want_state=True,

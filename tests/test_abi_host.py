@@ -120,7 +120,8 @@ def _call_prefill_ex(lib, opts, **over):
 @pytest.mark.parametrize("opts,over,code", [
     (dict(impl=5), {}, 1),                          # no such implementation
     (dict(impl=-1), {}, 1),
-    (dict(fault=2), {}, 1),                         # no such fault
+    (dict(fault=3), {}, 1),                         # no such fault
+    (dict(fault=2), {}, 2),                         # index-check injection: debug build only
     (dict(wait_limit_cycles=-1), {}, 1),
     (dict(impl=2), {}, 2),                          # tensor cores forced, d = 64: unsupported
     (dict(impl=3), dict(io=gdn.GDN_FP32, d_k=128, d_v=128), 2),  # fp32 I/O
@@ -133,6 +134,37 @@ def test_prefill_ex_rejects(lib, opts, over, code):
     for k_, v_ in opts.items():
         setattr(o, k_, v_)
     assert _call_prefill_ex(lib, o, **over) == code
+
+
+@pytest.fixture(scope="module")
+def debug_lib(lib):
+    """libgdn_debug.so through a handle of its own (the module's library stays loaded),
+    with the same argument and result types as the binding gives libgdn.so."""
+    d = ctypes.CDLL(build.build(debug=True))
+    for name in gdn.EXPORTS:
+        f, g = getattr(lib, name), getattr(d, name)
+        g.restype = f.restype
+        if f.argtypes is not None:
+            g.argtypes = f.argtypes
+    return d
+
+
+def test_debug_library_exports_and_flag(lib, debug_lib):
+    for name in _declared():
+        assert hasattr(debug_lib, name), name
+    assert lib.gdn_debug_build() == 0
+    assert debug_lib.gdn_debug_build() == 1
+    assert debug_lib.gdn_status_string(8) == b"GDN_ERR_BAD_INDEX"
+
+
+def test_debug_library_accepts_injection_option(debug_lib):
+    """The debug build takes GDN_FAULT_BAD_INDEX and goes on to the ordinary checks (here
+    a workspace too small: GDN_ERR_WORKSPACE, before any launch)."""
+    o = gdn.PrefillOptions()
+    o.fault = gdn.GDN_FAULT_BAD_INDEX
+    assert _call_prefill_ex(debug_lib, o, ws_bytes=100) == 3
+    o.fault = 3
+    assert _call_prefill_ex(debug_lib, o) == 1
 
 
 def test_prefill_ex_null_options_is_prefill(lib):
