@@ -101,6 +101,38 @@ def _source_sha1(path=TC_SOURCE):
         return hashlib.sha1(f.read()).hexdigest()
 
 
+def run_metadata(dev):
+    """Where the number was measured: the GPU (name, SM count, memory, driver and CUDA
+    runtime of the process), the library that ran (a hash of the kernel sources and
+    the public header, whether it is the debug build) and, where the checkout has its
+    history, the git commit."""
+    from linear_attention_sequence_delta_b200 import gdn
+    props = torch.cuda.get_device_properties(dev)
+    h = hashlib.sha1()
+    csrc = os.path.join(ROOT, "linear_attention_sequence_delta_b200", "csrc")
+    files = [os.path.join(csrc, f) for f in sorted(os.listdir(csrc)) if f.endswith((".cu", ".cuh"))]
+    for path in files + [os.path.join(ROOT, "include", "gdn.h")]:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    try:
+        sha = subprocess.run(["git", "-C", ROOT, "rev-parse", "HEAD"], capture_output=True,
+                             text=True, timeout=10).stdout.strip() or None
+    except Exception:
+        sha = None
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        driver = pynvml.nvmlSystemGetDriverVersion()
+        driver = driver.decode() if isinstance(driver, bytes) else driver
+    except Exception:
+        driver = None
+    return {"gpu": {"name": props.name, "sm_count": props.multi_processor_count,
+                    "memory_gib": round(props.total_memory / 2**30, 1),
+                    "driver": driver, "torch_cuda": torch.version.cuda},
+            "library": {"sources_sha1": h.hexdigest(), "debug_build": gdn.debug_build(),
+                        "git_sha": sha}}
+
+
 def kernel_traffic(kernel, workload):
     """DRAM bytes per launch of `kernel` on `workload` from the committed ncu record,
     or None (no record, or one taken on another build of the kernel source)."""
@@ -607,6 +639,7 @@ def run_ours(args):
         "decode_slots": dvar,
         "mixer": mixer,
         "mixer_prefill": mixp,
+        "run": run_metadata(dev),
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()

@@ -201,7 +201,8 @@ constexpr uint32_t PS_RK = 71680;  // [64] rk, [64] rq (rq includes the scale)
 constexpr uint32_t PS_PAR = 72192; // [2][kMaxGroup] A_log, dt_bias of those heads
 constexpr uint32_t PS_BAR = 72320; // mbarrier (MMA)
 constexpr uint32_t PS_TMEM = 72328;
-constexpr size_t kPrepSmem = 72336 + 1024;
+constexpr uint32_t PS_LDBAR = 72336; // mbarrier (TMA loads of the K and Q rows)
+constexpr size_t kPrepSmem = 72344 + 1024;
 static_assert(PS_CI + 64 * 4 <= PS_TS, "the per-head area must fit where K and Q were");
 
 // Half a row (32 columns from 32 H) of A (row i < 64, to the A matrix) or of P (row
@@ -406,7 +407,7 @@ __device__ __forceinline__ void prep_worker(
     unsigned long long* flags, unsigned long long epoch, uint8_t* sm, const int tid,
     const int bar_id, const int worker, const int nworkers, const bool relinquish,
     const long long wait_cycles, const MixerFusion& mix, const int64_t qk_tok,
-    const int64_t T_total) {
+    const int64_t T_total, const CUtensorMap* tm_q, const CUtensorMap* tm_k) {
     uint8_t* KQ = sm + PS_KQ;
     float* Ts = reinterpret_cast<float*>(sm + PS_TS);
     float* As = reinterpret_cast<float*>(sm + PS_AS);
@@ -422,6 +423,7 @@ __device__ __forceinline__ void prep_worker(
     float* sCI = reinterpret_cast<float*>(sm + PS_CI);
     float* rq = rk + 64;
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + PS_BAR);
+    uint64_t* ldbar = reinterpret_cast<uint64_t*>(sm + PS_LDBAR);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + PS_TMEM);
 
     const int warp = tid >> 5, lane = tid & 31;
@@ -432,13 +434,14 @@ __device__ __forceinline__ void prep_worker(
     const int64_t total_records = (int64_t)choff[N] * H_v;
     const int64_t qk_extent = T_total > 0 ? (T_total - 1) * qk_tok + (int64_t)H_qk * kD : 0;
 
-    constexpr uint32_t tcols = 64u;
+    constexpr uint32_t tcols = 128u;  // [K; Q] [K; Q]^T
     if (warp == 0) {
         tmem_alloc(s_tmem, tcols);
         if (relinquish) tmem_relinquish();
     }
     if (tid == 0) {
         mbar_init(bar, 1);
+        mbar_init(ldbar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     // entries of T above its diagonal blocks are never written: zero them once
@@ -450,8 +453,10 @@ __device__ __forceinline__ void prep_worker(
     const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const int trow = (warp & 3) * 32 + lane;  // TMEM lane = row of [K; Q] K^T
     const int hh = warp >> 2;                 // which 32 columns of that row
-    uint32_t mphase = 0;
+    uint32_t mphase = 0, lphase = 0;
     bool failed = false;
+    bool ld_pending = false;  // (thread 0) a TMA load of K and Q rows not yet waited for
+    uint32_t ld_phase = 0;    // (thread 0) the phase that load completes
     // A worker's units only move forward, so the sequence of each is found by a short
     // forward scan from the previous one's (the first by bisection): one dependent load
     // of the offsets per unit instead of a bisection's worth.
@@ -474,22 +479,18 @@ __device__ __forceinline__ void prep_worker(
         const int64_t t0 = (int64_t)cu_seqlens[n] + (int64_t)(cg - choff[n]) * kC;
         const int L = (int)min((int64_t)kC, (int64_t)cu_seqlens[n + 1] - t0);
 
-        // ---- raw K and Q rows (sw128), or the convolution that makes them; gates of
-        // the r V heads
+        // ---- raw K and Q rows (sw128: four TMA boxes of 64 rows x 128 bytes, the chain's
+        // tile layout), or the convolution that makes them; gates of the r V heads
         if constexpr (kConv) {
             conv_unit(mix, n, cu_seqlens[n], t0, L, j, r, H_qk, KQ, tid, T_total, N, status);
-        } else {
-#pragma unroll
-            for (int it = 0; it < 4; ++it) {
-                const int idx = tid + kPrepThreads * it;  // 0 .. 1023
-                const int rr = idx >> 4, ch = idx & 15;
-                const int64_t tok = rr < L ? t0 + rr : 0;
-                const size_t rowk = (size_t)tok * qk_tok + (size_t)j * kD + ch * 8;
-                const bool live = rr < L && GDN_IN_BOUNDS(rowk + 7, qk_extent, status);
-                const uint32_t off = (uint32_t)(ch >> 3) * 16384u;
-                cp_async_16(KQ + off + sw128_off(rr, ch & 7), k + rowk, live ? 16u : 0u);
-                cp_async_16(KQ + off + sw128_off(rr + 64, ch & 7), q + rowk, live ? 16u : 0u);
-            }
+        } else if (tid == 0) {
+            mbar_arrive_expect_tx(ldbar, 4u * 8192u);
+            tma_load_3d(KQ, tm_k, 0, j, (int32_t)t0, ldbar);
+            tma_load_3d(KQ + 16384, tm_k, 64, j, (int32_t)t0, ldbar);
+            tma_load_3d(KQ + 8192, tm_q, 0, j, (int32_t)t0, ldbar);
+            tma_load_3d(KQ + 16384 + 8192, tm_q, 64, j, (int32_t)t0, ldbar);
+            ld_pending = true;
+            ld_phase = lphase;
         }
         for (int idx = tid; idx < 2 * r * kC; idx += kPrepThreads) {
             const int which = idx / (r * kC);            // 0: a, 1: b
@@ -508,49 +509,47 @@ __device__ __forceinline__ void prep_worker(
         }
         cp_async_commit();
         cp_async_wait<0>();
+        if (!kConv && L < kC) {
+            // the rows past the sequence's end hold the next tokens (or zeros past T): zero
+            // them, 16 bytes a thread at a time (whole 128-byte rows, so no swizzle matters)
+            if (!mbar_wait_bounded(ldbar, lphase, wait_cycles)) failed = true;
+            else if (tid == 0) ld_pending = false;
+            const int nz = (kC - L) * 8;  // 16-byte pieces per 64-row tile
+            for (int idx = tid; idx < 4 * nz; idx += kPrepThreads) {
+                const int tile = idx / nz, rr = L + (idx % nz) / 8, ch = idx & 7;
+                *reinterpret_cast<uint4*>(KQ + (tile >> 1) * 16384 + (tile & 1) * 8192 + rr * 128 +
+                                          ch * 16) = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
         fence_proxy_async_smem();
         named_bar_sync(bar_id, kPrepThreads);
 
-        // ---- inverse row norms (two threads per row), then Dkq = [K; Q] K^T ---------
-        {
-            const int row = tid >> 1;
-            const uint8_t* base = KQ + (uint32_t)(tid & 1) * 16384u;
-            float ss = 0.f;
+        // ---- Dkq = [K; Q] [K; Q]^T: columns 0-63 ([K; Q] K^T) feed A and P, the diagonal
+        // gives the row norms
+        if (tid == 0) {
+            bool ok = true;
+            if (!kConv && L == kC) {
+                ok = mbar_wait_bounded(ldbar, lphase, wait_cycles);
+                if (ok) ld_pending = false;
+            }
+            if (!ok) failed = true;
+            const uint32_t kq = smem_u32(KQ);
+            constexpr uint32_t id_kq = idesc_bf16_f32(128, 128, 0, 0);
+            if (ok) {
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                const uint4 w = *reinterpret_cast<const uint4*>(base + sw128_off(row, ch));
-                const uint32_t* u = &w.x;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 x2 =
-                        __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u[e]));
-                    ss = fmaf(x2.x, x2.x, ss);
-                    ss = fmaf(x2.y, x2.y, ss);
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t off = (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u;
+                    mma_bf16_ss(tmem, smem_desc_sw128(kq + off, 16, 1024),
+                                smem_desc_sw128(kq + off, 16, 1024), id_kq, ks > 0);
                 }
             }
-            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-            if ((tid & 1) == 0) {
-                const float inv = 1.f / sqrtf(ss + kL2Eps);
-                if (row < 64) rk[row] = inv;
-                else rq[row - 64] = inv * scale;
-            }
+            mma_commit(bar);  // (after a failed load: arrives at once, the error follows)
         }
-        named_bar_sync(bar_id, kPrepThreads);  // rk, rq
-        if (tid == 0) {
-            const uint32_t kq = smem_u32(KQ);
-            constexpr uint32_t id_kq = idesc_bf16_f32(128, 64, 0, 0);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t off = (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u;
-                mma_bf16_ss(tmem, smem_desc_sw128(kq + off, 16, 1024),
-                            smem_desc_sw128(kq + off, 16, 1024), id_kq, ks > 0);
-            }
-            mma_commit(bar);
-        }
+        if (!kConv) lphase ^= 1u;
         // ---- gates of every V head of the group: one warp per head, two tokens a lane:
-        // g, beta, the in-chunk inclusive cumsum G, and the record's per-token factors
+        // g, beta and the in-chunk inclusive cumsum G (the record's per-token factors
+        // follow once the row norms are known)
         for (int hr = warp; hr < r; hr += kPrepThreads / 32) {
-            const int h = j * r + hr;
             const float A_l = sPar[hr], dtb = sPar[kMaxGroup + hr];
             const int ta = 2 * lane, tb = 2 * lane + 1;
             const float ga = ta < L ? gate_g(AB[hr * kC + ta], A_l, dtb) : 0.f;
@@ -563,26 +562,46 @@ __device__ __forceinline__ void prep_worker(
                 const float y = __shfl_up_sync(0xffffffffu, sc, off);
                 if (lane >= off) sc += y;
             }
-            const float Gb = sc, Ga = sc - gb;  // G_{L-1} = G of the last lane (g = 0 past L)
-            const float G_last = __shfl_sync(0xffffffffu, sc, 31);
-            *reinterpret_cast<float2*>(sGall + hr * kC + ta) = make_float2(Ga, Gb);
+            *reinterpret_cast<float2*>(sGall + hr * kC + ta) = make_float2(sc - gb, sc);
             *reinterpret_cast<float2*>(sBall + hr * kC + ta) = make_float2(ba, bb);
-            float* rg = reinterpret_cast<float*>(rec + ((size_t)cg * H_v + h) * kRecBytes + REC_G);
-            if (!GDN_IN_BOUNDS((int64_t)cg * H_v + h, total_records, status)) continue;
-            const float ea = __expf(Ga), eb = __expf(Gb);
-            const float2 rk2 = *reinterpret_cast<const float2*>(rk + ta);
-            const float2 rq2 = *reinterpret_cast<const float2*>(rq + ta);
-            *reinterpret_cast<float2*>(rg + RG_FK + ta) = make_float2(ea * rk2.x, eb * rk2.y);
-            *reinterpret_cast<float2*>(rg + RG_EGQ + ta) = make_float2(ea * rq2.x, eb * rq2.y);
-            *reinterpret_cast<float2*>(rg + RG_EGL + ta) =
-                make_float2(__expf(G_last - Ga) * rk2.x, __expf(G_last - Gb) * rk2.y);
-            if (lane == 0) rg[RG_GAMMA] = __expf(G_last);
         }
         const bool ok = mbar_wait_bounded(bar, mphase, wait_cycles);
         mphase ^= 1u;
         if (!ok) failed = true;
         if (named_bar_any(bar_id, kPrepThreads, failed)) { failed = true; break; }
         tc_fence_after();
+        // ---- inverse row norms from the diagonal (K K^T)_ii, (Q Q^T)_tt: the warps of the
+        // first column half load the 32 columns of their own 32 rows and keep their lane's
+        {
+            if (hh == 0) {
+                float xd[32];
+                tmem_ld32_sync(tl + 32 * (warp & 3), xd);
+                float d = xd[0];
+#pragma unroll
+                for (int e = 1; e < 32; ++e) d = lane == e ? xd[e] : d;
+                const float inv = 1.f / sqrtf(d + kL2Eps);
+                if (trow < 64) rk[trow] = inv;
+                else rq[trow - 64] = inv * scale;
+            }
+        }
+        named_bar_sync(bar_id, kPrepThreads);  // rk, rq
+        // the record's per-token factors of every V head of the group
+        for (int hr = warp; hr < r; hr += kPrepThreads / 32) {
+            const int h = j * r + hr;
+            const int ta = 2 * lane;
+            const float2 G2 = *reinterpret_cast<const float2*>(sGall + hr * kC + ta);
+            const float G_last = sGall[hr * kC + kC - 1];  // G_{L-1} (g = 0 past L)
+            float* rg = reinterpret_cast<float*>(rec + ((size_t)cg * H_v + h) * kRecBytes + REC_G);
+            if (!GDN_IN_BOUNDS((int64_t)cg * H_v + h, total_records, status)) continue;
+            const float ea = __expf(G2.x), eb = __expf(G2.y);
+            const float2 rk2 = *reinterpret_cast<const float2*>(rk + ta);
+            const float2 rq2 = *reinterpret_cast<const float2*>(rq + ta);
+            *reinterpret_cast<float2*>(rg + RG_FK + ta) = make_float2(ea * rk2.x, eb * rk2.y);
+            *reinterpret_cast<float2*>(rg + RG_EGQ + ta) = make_float2(ea * rq2.x, eb * rq2.y);
+            *reinterpret_cast<float2*>(rg + RG_EGL + ta) =
+                make_float2(__expf(G_last - G2.x) * rk2.x, __expf(G_last - G2.y) * rk2.y);
+            if (lane == 0) rg[RG_GAMMA] = __expf(G_last);
+        }
         // this thread's half row of [K; Q] K^T, shared by the r V heads, columns scaled
         // by rk once for all of them
         float x[32];
@@ -598,7 +617,7 @@ __device__ __forceinline__ void prep_worker(
                 x[4 * e4 + 3] *= r4.w;
             }
         }
-        // The K and Q rows have been read (norms, MMA): their area now takes A, the P
+        // The K and Q rows have been read (MMA): their area now takes A, the P
         // staging image and the tables. The first head's tables get a phase of their own;
         // every later head's are built while the head before writes its record.
         exp_tables(sGall, sU, sE, sCI, tid);
@@ -747,6 +766,8 @@ __device__ __forceinline__ void prep_worker(
         }
         tc_fence_before();  // this unit's TMEM reads precede the next unit's MMA
     }
+    // no copy into shared memory may still be in flight when the worker ends
+    if (tid == 0 && ld_pending && !mbar_wait_bounded(ldbar, ld_phase, wait_cycles)) failed = true;
     tc_fence_before();
     named_bar_sync(bar_id, kPrepThreads);
     tc_fence_after();
@@ -757,6 +778,7 @@ __device__ __forceinline__ void prep_worker(
 constexpr int kPrepBlocksPerSm = 3;
 template <bool kConv>
 __global__ void __launch_bounds__(kPrepThreads, kPrepBlocksPerSm) prep_kernel(
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const bf16* __restrict__ q, const bf16* __restrict__ k, const float* __restrict__ a,
     const float* __restrict__ b, const float* __restrict__ A_log,
     const float* __restrict__ dt_bias, const int32_t* __restrict__ cu_seqlens,
@@ -768,7 +790,7 @@ __global__ void __launch_bounds__(kPrepThreads, kPrepBlocksPerSm) prep_kernel(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     prep_worker<kConv>(q, k, a, b, A_log, dt_bias, cu_seqlens, choff, N, H_qk, H_v, scale, rec,
                        status, nullptr, 0, sm, threadIdx.x, 1, blockIdx.x, gridDim.x, true,
-                       wait_cycles, mix, qk_tok, T_total);
+                       wait_cycles, mix, qk_tok, T_total, &tm_q, &tm_k);
 }
 
 // ==================================== chain =======================================
@@ -1734,7 +1756,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
                     status, withhold_records ? nullptr : flags, epoch, sm + sub * kPrepRegion,
                     tid & 255, 3 + sub, 2 * ((int)blockIdx.x - c0) + sub,
                     2 * ((int)gridDim.x - c0), false, wait_cycles, mix, (int64_t)H_qk * kD,
-                    T_total);
+                    T_total, &tm_q, &tm_k);
         return;
     }
     if (tid >= kChainThreads) return;
@@ -1973,7 +1995,7 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
     if (prep_grid > 0) {
         timer_before(opt.timer, s);
         prep_fn<<<prep_grid, kPrepThreads, kPrepSmem, s>>>(
-            q_rows, k_rows, a, b, A_log, dt_bias, cu_seqlens, choff, N, H_qk, H_v, scale, rec,
+            tm_q, tm_k, q_rows, k_rows, a, b, A_log, dt_bias, cu_seqlens, choff, N, H_qk, H_v, scale, rec,
             status, wait_cycles, mix_split, qk_tok, T);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
