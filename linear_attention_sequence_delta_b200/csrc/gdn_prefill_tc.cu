@@ -87,11 +87,17 @@ __device__ __forceinline__ bool bad_seq(int64_t s0, int64_t s1, int64_t T_total,
 }
 
 // =============================== chunk offsets ===================================
-// choff[n] = number of 64-token chunks in sequences 0 .. n-1 (choff[N] = total).
+// choff[n] = number of 64-token chunks in sequences 0 .. n-1 (choff[N] = total), and
+// order[]: the sequences by chunk count, most first (ties by index), for the chain
+// blocks of the separate-launch path to take the longest sequences first (a list
+// schedule); with more than kOrderMax sequences, or bad lengths, the identity.
+constexpr int kOrderMax = 1024;
 __global__ void __launch_bounds__(256) chunk_offsets_kernel(const int32_t* __restrict__ cu,
                                                             int32_t N, int64_t T_total,
                                                             int32_t* __restrict__ choff,
+                                                            int32_t* __restrict__ order,
                                                             int* status) {
+    __shared__ int32_t s_nc[kOrderMax];
     __shared__ int32_t warp_tot[8];
     __shared__ int32_t carry;
     __shared__ int bad;
@@ -128,6 +134,23 @@ __global__ void __launch_bounds__(256) chunk_offsets_kernel(const int32_t* __res
             set_status(status, kStatusBadSeqlens);
             for (int n = 0; n < N; ++n) choff[n] = 0;
         }
+    }
+    // rank of sequence n = how many sequences come before it in the order
+    const bool sort = !bad && N <= kOrderMax;
+    if (sort)
+        for (int n = threadIdx.x; n < N; n += 256) s_nc[n] = (int32_t)((cu[n + 1] - cu[n] + kC - 1) / kC);
+    __syncthreads();
+    for (int n = threadIdx.x; n < N; n += 256) {
+        int rank = n;
+        if (sort) {
+            const int32_t c = s_nc[n];
+            rank = 0;
+            for (int m = 0; m < N; ++m) {
+                const int32_t cm = s_nc[m];
+                rank += (cm > c || (cm == c && m < n)) ? 1 : 0;
+            }
+        }
+        order[rank] = n;
     }
 }
 
@@ -1661,7 +1684,8 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
     const float* S0g, const int32_t* __restrict__ cu_seqlens,
     const int32_t* __restrict__ choff, int64_t T_total, int H_qk, int H_v,
     const uint8_t* __restrict__ rec, bf16* __restrict__ o, float* Sfg, const StateIndex sref,
-    int* status, long long wait_cycles, const MixerFusion mix, int N, int inject_bad_index) {
+    int* status, long long wait_cycles, const MixerFusion mix, int N, int inject_bad_index,
+    const int32_t* __restrict__ order) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1676,7 +1700,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
     chain_unit<128, kNorm>(tm_q, tm_k, tm_v, tm_o, S0g, cu_seqlens, choff, T_total, H_qk, H_v, rec, o,
-                    Sfg, sref, status, nullptr, 0, sm, threadIdx.x, blockIdx.x / H_v,
+                    Sfg, sref, status, nullptr, 0, sm, threadIdx.x, order[blockIdx.x / H_v],
                     blockIdx.x % H_v, 0, tmem, 1, wait_cycles, mix, N, inject_bad_index != 0);
     tc_fence_before();
     __syncthreads();
@@ -1787,13 +1811,13 @@ struct TcWorkspace {
     size_t off_flags, off_rec, total;
 };
 
-// Workspace: chunk offsets [N + 1] | record flags [records] (64-bit call numbers) |
-// records [chunks][H_v].
+// Workspace: chunk offsets [N + 1], chain order [N] | record flags [records] (64-bit call
+// numbers) | records [chunks][H_v].
 TcWorkspace tc_workspace_layout(int32_t N, int64_t T, int32_t H_v) {
     const size_t chunks = (size_t)((T + kC - 1) / kC) + (size_t)N;
     const size_t records = chunks * H_v;
     TcWorkspace w;
-    w.off_flags = align256((size_t)(N + 1) * sizeof(int32_t));
+    w.off_flags = align256((size_t)(2 * N + 1) * sizeof(int32_t));
     w.off_rec = w.off_flags + align256(records * sizeof(unsigned long long));
     w.total = w.off_rec + records * kRecBytes;
     return w;
@@ -1982,7 +2006,7 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
                              (int)kChainSmem);
     if (e != cudaSuccess) return e;
     timer_before(opt.timer, s);
-    chunk_offsets_kernel<<<1, 256, 0, s>>>(cu_seqlens, N, T, choff, status);
+    chunk_offsets_kernel<<<1, 256, 0, s>>>(cu_seqlens, N, T, choff, choff + N + 1, status);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     timer_after(opt.timer, s, "chunk_offsets");
@@ -2005,7 +2029,7 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
     chain_fn<<<(unsigned)chain_units, kChainThreads, kChainSmem, s>>>(
         tm_q, tm_k, tm_v, tm_o, S0, cu_seqlens, choff, T, H_qk, H_v, rec, static_cast<bf16*>(o),
         S_final, sref, status, wait_cycles, mix_split, N,
-        opt.fault == GDN_FAULT_BAD_INDEX ? 1 : 0);
+        opt.fault == GDN_FAULT_BAD_INDEX ? 1 : 0, choff + N + 1);
     e = cudaGetLastError();
     if (e == cudaSuccess) timer_after(opt.timer, s, "chain");
     return e;

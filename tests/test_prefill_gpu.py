@@ -278,6 +278,28 @@ def test_many_chains_use_separate_launches():
     assert [n for n, _ in timer.times()] == ["chunk_offsets", "prep", "chain"]
 
 
+def test_chain_order_longest_first():
+    """The separate launches run the chains of the sequences with the most chunks first:
+    the order the offsets kernel leaves in the workspace (after the N + 1 chunk offsets)
+    is the sequences by chunk count, most first, ties by index; the results match the
+    oracle whatever the order."""
+    lens = [100, 700, 0, 64, 65, 700, 1, 300, 128, 129, 5, 640]
+    P = make_prefill_inputs(lens, H_qk=4, H_v=8, d_k=128, d_v=128, state_std=0.05, seed=61)
+    Pd = P.to("cuda")
+    N, T = len(lens), sum(lens)
+    work = torch.zeros(gdn.workspace_size(N, T, 4, 8, 128, 128), dtype=torch.uint8,
+                       device="cuda")
+    o, Sf = gdn_prefill(Pd.q, Pd.k, Pd.v, Pd.a, Pd.b, Pd.A_log, Pd.dt_bias, Pd.cu_seqlens,
+                        Pd.initial_state, workspace=work, impl=gdn.GDN_IMPL_TENSOR_CORE_SPLIT)
+    assert gdn_sync_status() == 0
+    words = work[: (2 * N + 1) * 4].view(torch.int32).cpu().tolist()
+    chunks = [(n_ + 63) // 64 for n_ in lens]
+    assert words[:N + 1] == [sum(chunks[:i]) for i in range(N + 1)]
+    assert words[N + 1:] == sorted(range(N), key=lambda i: (-chunks[i], i))
+    o_ref, S_ref = _full_oracle(P)
+    assert rel_err(o, o_ref) <= TOL_BF16 and rel_err(Sf, S_ref) <= TOL_BF16
+
+
 # ------------------------------------------------ workspace contents, failures ----
 
 def _ws_fill(work, pattern):
