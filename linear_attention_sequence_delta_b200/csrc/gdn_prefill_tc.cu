@@ -292,8 +292,11 @@ __device__ __forceinline__ void exp_tables(const float* hG, float* sU, float* sE
     sU[tid] = (jj < 16 * ab4) ? __expf(hG[16 * ab4] - hG[jj]) : 0.f;
 #pragma unroll
     for (int q4 = 0; q4 < 4; ++q4) {
+        // a warp writes rows ii and ii + 4 of a block (20 ii and 20 ii + 80 differ by 16
+        // banks: no conflict); over the 16 row selectors rs every row ii once
         const int idx = tid + kPrepThreads * q4;  // 0..1023
-        const int bb = idx >> 8, ii = (idx >> 4) & 15, jb = idx & 15;
+        const int rs = (idx >> 4) & 15;
+        const int bb = idx >> 8, ii = ((rs & 1) << 2) | ((rs >> 1) & 3) | (rs & 8), jb = idx & 15;
         sE[bb * (16 * kEStride) + ii * kEStride + jb] =
             jb <= ii ? __expf(hG[16 * bb + ii] - hG[16 * bb + jb]) : 0.f;
     }
@@ -686,9 +689,13 @@ __device__ __forceinline__ void prep_worker(
                 const int rr = i & 7;
                 const int b0 = i & ~7;
                 const int src0 = lane & ~7;
-                float Ad[8];
+                // the row's 8 entries of its diagonal block as two 16-byte loads (the rows of a
+                // load's 8-thread phase are 68 words apart: distinct bank groups)
+                const float4 q0 = *reinterpret_cast<const float4*>(As + i * kAsStride + b0);
+                const float4 q1 = *reinterpret_cast<const float4*>(As + i * kAsStride + b0 + 4);
+                float Ad[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
-                for (int r2 = 0; r2 < 8; ++r2) Ad[r2] = (r2 < rr) ? As[i * kAsStride + b0 + r2] : 0.f;
+                for (int r2 = 0; r2 < 8; ++r2) Ad[r2] = (r2 < rr) ? Ad[r2] : 0.f;
                 float Rr[8];
 #pragma unroll
                 for (int jj = 0; jj < 8; ++jj) Rr[jj] = 0.f;
@@ -702,9 +709,12 @@ __device__ __forceinline__ void prep_worker(
                     }
                     if (rr > m) Rr[m] += am;
                 }
-                float* Trow = Ts + i * kTsStride + b0;
+                float Tv[8];
 #pragma unroll
-                for (int r2 = 0; r2 < 8; ++r2) Trow[r2] = r2 < rr ? -Rr[r2] : (r2 == rr ? 1.f : 0.f);
+                for (int r2 = 0; r2 < 8; ++r2) Tv[r2] = r2 < rr ? -Rr[r2] : (r2 == rr ? 1.f : 0.f);
+                float4* Trow = reinterpret_cast<float4*>(Ts + i * kTsStride + b0);
+                Trow[0] = make_float4(Tv[0], Tv[1], Tv[2], Tv[3]);
+                Trow[1] = make_float4(Tv[4], Tv[5], Tv[6], Tv[7]);
             }
             named_bar_sync(bar_id, kPrepThreads);
 
@@ -767,17 +777,33 @@ __device__ __forceinline__ void prep_worker(
             // as coalesced 16-byte stores; the next head's tables meanwhile -------------
 #pragma unroll
             for (int it = 0; it < 2; ++it) {
+                // The 8 threads of a row read its columns 4 c8 .. + 3 and 32 + 4 c8 .. + 3
+                // (two contiguous 128-byte runs: no bank conflict), times beta of those
+                // columns; each pair of neighbours then swaps halves, so that the even one
+                // holds 16-byte chunk c8 / 2 of the bf16 row and the odd one chunk 4 + c8 / 2.
                 const int idx = tid + kPrepThreads * it;  // 0..511
-                const int row = idx >> 3, ch = idx & 7;
-                const float4 f0 = *reinterpret_cast<const float4*>(Ts + row * kTsStride + ch * 8);
-                const float4 f1 = *reinterpret_cast<const float4*>(Ts + row * kTsStride + ch * 8 + 4);
-                const float4 b0 = *reinterpret_cast<const float4*>(hBeta + ch * 8);
-                const float4 b1 = *reinterpret_cast<const float4*>(hBeta + ch * 8 + 4);
+                const int row = idx >> 3, c8 = idx & 7;
+                const bool odd = (c8 & 1) != 0;
+                const float* trow = Ts + row * kTsStride;
+                const float4 ta = *reinterpret_cast<const float4*>(trow + 4 * c8);
+                const float4 tb = *reinterpret_cast<const float4*>(trow + 32 + 4 * c8);
+                const float4 ba = *reinterpret_cast<const float4*>(hBeta + 4 * c8);
+                const float4 bb = *reinterpret_cast<const float4*>(hBeta + 32 + 4 * c8);
+                const float4 pa = make_float4(ta.x * ba.x, ta.y * ba.y, ta.z * ba.z, ta.w * ba.w);
+                const float4 pb = make_float4(tb.x * bb.x, tb.y * bb.y, tb.z * bb.z, tb.w * bb.w);
+                const float4 snd = odd ? pa : pb;
+                float4 rcv;
+                rcv.x = __shfl_xor_sync(0xffffffffu, snd.x, 1);
+                rcv.y = __shfl_xor_sync(0xffffffffu, snd.y, 1);
+                rcv.z = __shfl_xor_sync(0xffffffffu, snd.z, 1);
+                rcv.w = __shfl_xor_sync(0xffffffffu, snd.w, 1);
+                const float4 lo = odd ? rcv : pa, hi = odd ? pb : rcv;
                 uint4 w;  // column s of T times beta_s
-                w.x = pack_bf16x2(f0.x * b0.x, f0.y * b0.y);
-                w.y = pack_bf16x2(f0.z * b0.z, f0.w * b0.w);
-                w.z = pack_bf16x2(f1.x * b1.x, f1.y * b1.y);
-                w.w = pack_bf16x2(f1.z * b1.z, f1.w * b1.w);
+                w.x = pack_bf16x2(lo.x, lo.y);
+                w.y = pack_bf16x2(lo.z, lo.w);
+                w.z = pack_bf16x2(hi.x, hi.y);
+                w.w = pack_bf16x2(hi.z, hi.w);
+                const int ch = odd ? 4 + (c8 >> 1) : (c8 >> 1);
                 if (rec_ok) {
                     *reinterpret_cast<uint4*>(R + REC_T + sw128_off(row, ch)) = w;
                     reinterpret_cast<uint4*>(R + REC_P)[idx] = reinterpret_cast<const uint4*>(Pst)[idx];
@@ -809,8 +835,9 @@ __global__ void __launch_bounds__(kPrepThreads, kPrepBlocksPerSm) prep_kernel(
     uint8_t* __restrict__ rec, int* status, long long wait_cycles, const MixerFusion mix,
     int64_t qk_tok, int64_t T_total) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned (128-byte swizzle), as an offset from the shared array itself so
+    // that every pointer derived from it stays a shared-memory address for the compiler
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     prep_worker<kConv>(q, k, a, b, A_log, dt_bias, cu_seqlens, choff, N, H_qk, H_v, scale, rec,
                        status, nullptr, 0, sm, threadIdx.x, 1, blockIdx.x, gridDim.x, true,
                        wait_cycles, mix, qk_tok, T_total, &tm_q, &tm_k);
@@ -1687,8 +1714,9 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
     int* status, long long wait_cycles, const MixerFusion mix, int N, int inject_bad_index,
     const int32_t* __restrict__ order) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned (128-byte swizzle), as an offset from the shared array itself so
+    // that every pointer derived from it stays a shared-memory address for the compiler
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + CS_TMEM);
     const int warp = threadIdx.x >> 5;
     if (warp == 0) {
@@ -1739,8 +1767,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
     extern __shared__ uint8_t smem_raw[];
     __shared__ int32_t s_choff[kFusedMaxSeqs + 1];
     __shared__ int s_bad;
-    uint8_t* sm = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned (128-byte swizzle), as an offset from the shared array itself so
+    // that every pointer derived from it stays a shared-memory address for the compiler
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x;
     // chunk offsets of the sequences (prefix sum of ceil(len / 64)), by one warp
     if (tid < 32) {
