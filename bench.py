@@ -240,10 +240,12 @@ def mixer_call_bytes(T, N, H_qk, H_v, d, K, io_bytes, with_initial):
 
 
 def run_mixer_prefill(rank, dev, flush, stream, hbm, peak_src, iters):
-    """gdn_mixer_prefill (conv1d + SiLU fused into the prefill's preparation, gated
-    RMSNorm into the chain's output) against the same steps as separate kernels: the
-    conv of the q, k and v parts (dense tensors), gdn_prefill, gdn_rmsnorm_gated. On
-    the 35B-A3B layer shape (T=4096) and the packed varlen batch (64 sequences)."""
+    """gdn_mixer_prefill in its default schedule (the convolution, the tensor-core prefill
+    reading the post-conv buffer, the norm in place) and in the fused one (conv1d + SiLU
+    in the prefill's preparation, gated RMSNorm in the chain's output), against the same
+    steps as separate calls: the conv of the q, k and v parts (dense tensors), gdn_prefill,
+    gdn_rmsnorm_gated. On the 35B-A3B layer shape (T=4096) and the packed varlen batch
+    (64 sequences)."""
     from linear_attention_sequence_delta_b200 import gdn
     from linear_attention_sequence_delta_b200.inputs import WORKLOADS, make_mixer_prefill_inputs
     out, launches = {}, 0
@@ -263,10 +265,12 @@ def run_mixer_prefill(rank, dev, flush, stream, hbm, peak_src, iters):
         cout = torch.empty_like(P.conv_state)
         ws = torch.empty((gdn.mixer_workspace_size(N, T, H_qk, H_v, d),), device=dev,
                          dtype=torch.uint8)
-        fused = lambda tm=None: gdn.gdn_mixer_prefill(
+        call = lambda tm=None, impl=gdn.GDN_IMPL_AUTO: gdn.gdn_mixer_prefill(
             P.x, P.conv_weight, P.conv_bias, P.cu_seqlens, P.a, P.b, P.A_log, P.dt_bias, P.z,
             P.norm_weight, H_qk=H_qk, conv_state_in=P.conv_state, conv_state_out=cout,
-            initial_state=P.initial_state, out=y, final_state=Sf, workspace=ws, timer=tm)
+            initial_state=P.initial_state, out=y, final_state=Sf, workspace=ws, timer=tm,
+            impl=impl)
+        fused = lambda tm=None: call(tm, gdn.GDN_IMPL_TENSOR_CORE)
         # the separate steps on dense parts (q, k, v each its own [T, H d] tensor)
         bounds = [(0, H_qk * d), (H_qk * d, 2 * H_qk * d), (2 * H_qk * d, C)]
         xs = [P.x[:, a_:b_].contiguous() for a_, b_ in bounds]
@@ -287,23 +291,27 @@ def run_mixer_prefill(rank, dev, flush, stream, hbm, peak_src, iters):
                             final_state=Sf, workspace=pws)
             gdn.gdn_rmsnorm_gated(o, P.z, P.norm_weight, 1e-6, out=y)
 
+        ms_a = _time_op(call, iters, flush, stream)
         ms_f = _time_op(fused, iters, flush, stream)
         ms_s = _time_op(steps, iters, flush, stream)
+        call(timer)
+        ka = timer.times()
         fused(timer)
         kn = timer.times()
-        launches += 2 * (iters + 3) * 6
+        launches += 3 * (iters + 3) * 6
         byts = mixer_call_bytes(T, N, H_qk, H_v, d, K, 2, P.initial_state is not None)
         out[name] = {
             "workload": f"N={N}, T_total={T}, H_qk={H_qk}, H_v={H_v}, d={d}, conv_dim={C}, K={K}, "
                         "bf16 x/z/y, conv cache in and out"
                         + (", initial states in" if P.initial_state is not None else "")
                         + ", final states out",
-            "fused_ms": ms_f, "separate_steps_ms": ms_s,
+            "call_ms": ms_a, "call_kernels_ms": {k_: v_ for k_, v_ in ka},
+            "fused_ms": ms_f, "fused_kernels_ms": {k_: v_ for k_, v_ in kn},
+            "separate_steps_ms": ms_s,
             "separate_steps": "3 conv1d_silu (q, k, v parts) + gdn_prefill + gdn_rmsnorm_gated",
-            "fused_kernels_ms": {k_: v_ for k_, v_ in kn},
-            "tokens_per_s": T / (ms_f / 1e3), "algorithmic_bytes": byts,
-            "achieved_gbs": byts / (ms_f / 1e3) / 1e9,
-            "frac_hbm": byts / (ms_f / 1e3) / 1e9 / hbm, "peak_source": peak_src}
+            "tokens_per_s": T / (ms_a / 1e3), "algorithmic_bytes": byts,
+            "achieved_gbs": byts / (ms_a / 1e3) / 1e9,
+            "frac_hbm": byts / (ms_a / 1e3) / 1e9 / hbm, "peak_source": peak_src}
         del P, y, Sf, cout, ws, xs, ys, o, pws
     timer.close()
     out["l2"] = "flushed (512 MiB write) before every timed call"

@@ -200,18 +200,19 @@ int gdn_prefill_ex(const void* q, const void* k, const void* v, int32_t io_dtype
 
 /*
  * Kernel timing of gdn_prefill_ex -- a measurement aid; the pages have no
- * counterpart. A timer owns 8 CUDA events of the device current at creation (it
+ * counterpart. A timer owns 16 CUDA events of the device current at creation (it
  * is the only object of this library that allocates, and only here).
  *   gdn_timer_create      returns a timer, or NULL if the events cannot be made.
  *   gdn_timer_destroy     frees it (NULL is ignored).
  *   gdn_timer_read        waits for the events of the most recent call that used
  *                         the timer and writes the durations of its first
  *                         min(count, max_kernels) kernels, in milliseconds, to ms
- *                         (host array); returns the kernel count (at most 4), or
+ *                         (host array); returns the kernel count (at most 8), or
  *                         -GDN_ERR_INVALID_ARG / -GDN_ERR_CUDA.
  *   gdn_timer_kernel_name name of kernel i of that call ("chunk_offsets", "prep",
  *                         "chain", "fused", "fused_half_rows" on the tensor-core
- *                         path; "gates", "prefill_simt" on the CUDA-core path), or
+ *                         path; "gates", "prefill_simt" on the CUDA-core path;
+ *                         "conv1d_silu", "rmsnorm_gated" in gdn_mixer_prefill), or
  *                         NULL.
  * A timer may be used by one call at a time.
  */
@@ -440,14 +441,20 @@ int gdn_rmsnorm_gated(const void* o, const void* z, int32_t io_dtype, const floa
  *                   the post-conv q | k | v ([T, conv_dim] io_dtype), then the
  *                   prefill's workspace
  *   options         as gdn_prefill_ex, or NULL
- * For bf16 with d = 128 (at most 16 V heads per QK head) the steps are fused into the
- * tensor-core prefill: its preparation stage reads x (with each sequence's K-1 earlier
- * positions from the conv cache), convolves the q and k channels it needs itself and
- * writes all post-conv channels once for the chain stage, which applies the gated norm
- * to each tile of o before it is stored, and writes the conv cache at the end of each
- * sequence. The convolution's arithmetic is that of gdn_conv1d_silu (bit for bit);
- * the norm's sum of squares is taken in another order than gdn_rmsnorm_gated's. For
- * other shapes and types (and with GDN_IMPL_CUDA_CORE) the call runs the convolution,
+ * For bf16 with d = 128 (at most 16 V heads per QK head) there are two schedules:
+ *   GDN_IMPL_AUTO (default): the convolution into the workspace, the tensor-core
+ *     prefill with its own schedule reading q, k and v there (token stride conv_dim)
+ *     and writing o to y, then the norm over y in place -- the faster schedule on
+ *     every measured workload, and the same bits as the three calls.
+ *   GDN_IMPL_TENSOR_CORE, _SPLIT, _WHOLE_ROWS: the steps fused into the tensor-core
+ *     prefill: its preparation stage reads x (with each sequence's K-1 earlier
+ *     positions from the conv cache), convolves the q and k channels it needs itself
+ *     and writes all post-conv channels once for the chain stage, which applies the
+ *     gated norm to each tile of o before it is stored, and writes the conv cache at
+ *     the end of each sequence (with many chains the convolution runs as its own kernel
+ *     first). The convolution's arithmetic is that of gdn_conv1d_silu (bit for bit);
+ *     the norm's sum of squares is taken in another order than gdn_rmsnorm_gated's.
+ * For other shapes and types (and with GDN_IMPL_CUDA_CORE) the call runs the convolution,
  * the CUDA-core prefill and the norm one after another on the same buffers.
  */
 size_t gdn_mixer_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t H_qk,

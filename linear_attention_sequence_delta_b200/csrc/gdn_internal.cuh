@@ -202,7 +202,8 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
                               const float* S0, const int32_t* cu_seqlens, int32_t N, int64_t T,
                               int32_t H_qk, int32_t H_v, float scale, void* o, float* S_final,
                               StateIndex sref, void* workspace, const PrefillOpts& opt,
-                              int* status, cudaStream_t s, const MixerFusion& mix = MixerFusion{});
+                              int* status, cudaStream_t s, const MixerFusion& mix = MixerFusion{},
+                              int64_t qkv_tok = 0);
 
 // Steps around the delta rule (gdn_mixer.cu): causal depthwise conv1d + SiLU with
 // the per-sequence conv cache, its single-token decode form, and the gated RMSNorm.

@@ -657,8 +657,9 @@ __device__ __forceinline__ void prep_worker(
                 const int64_t t0n = (int64_t)cu_seqlens[nn] + (int64_t)(cgn - choff[nn]) * kC;
                 const int Ln = (int)min((int64_t)kC, (int64_t)cu_seqlens[nn + 1] - t0n);
                 const int rr = tid >> 2;
-                if (rr < Ln && GDN_IN_BOUNDS((t0n + rr) * qk_tok + (int64_t)jn * kD + 127, qk_extent,
-                                             status))
+                // (with the convolution fused in, the rows are made from x: nothing to fetch)
+                if (!kConv && rr < Ln &&
+                    GDN_IN_BOUNDS((t0n + rr) * qk_tok + (int64_t)jn * kD + 127, qk_extent, status))
                     prefetch_l2(((tid & 2) ? q : k) + (size_t)(t0n + rr) * qk_tok + (size_t)jn * kD +
                                 (tid & 1) * 64);
                 if (tid < 2 * kC && (tid & 63) < Ln &&
@@ -1763,7 +1764,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
     int64_t T_total, int H_qk, int H_v, float scale, uint8_t* __restrict__ rec,
     bf16* __restrict__ o, float* Sfg, const StateIndex sref,
     int* status, unsigned long long* flags, unsigned long long epoch, int c0,
-    long long wait_cycles, int withhold_records, const MixerFusion mix, int inject_bad_index) {
+    long long wait_cycles, int withhold_records, const MixerFusion mix, int inject_bad_index,
+    int64_t qk_tok) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ int32_t s_choff[kFusedMaxSeqs + 1];
     __shared__ int s_bad;
@@ -1808,7 +1810,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_kernel(
         prep_worker<kMix>(q, k, a, b, A_log, dt_bias, cu_seqlens, choff, N, H_qk, H_v, scale, rec,
                     status, withhold_records ? nullptr : flags, epoch, sm + sub * kPrepRegion,
                     tid & 255, 3 + sub, 2 * ((int)blockIdx.x - c0) + sub,
-                    2 * ((int)gridDim.x - c0), false, wait_cycles, mix, (int64_t)H_qk * kD,
+                    2 * ((int)gridDim.x - c0), false, wait_cycles, mix, qk_tok,
                     T_total, &tm_q, &tm_k);
         return;
     }
@@ -1927,7 +1929,8 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
                               const float* S0, const int32_t* cu_seqlens, int32_t N, int64_t T,
                               int32_t H_qk, int32_t H_v, float scale, void* o, float* S_final,
                               StateIndex sref, void* workspace, const PrefillOpts& opt,
-                              int* status, cudaStream_t s, const MixerFusion& mix) {
+                              int* status, cudaStream_t s, const MixerFusion& mix,
+                              int64_t qkv_tok) {
     if (N == 0) return cudaSuccess;
     if (T > (int64_t)0x7FFFFFFF - kC) return cudaErrorInvalidValue;  // TMA token coordinates
     const TcWorkspace ws = tc_workspace_layout(N, T, H_v);
@@ -1940,8 +1943,11 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
     // buffer [T][conv_dim] (q | k | v), written by the preparation (convolution fused into
     // its loads) or by the standalone convolution kernel before it.
     CUtensorMap tm_q, tm_k, tm_v, tm_o;
+    // q, k and v rows are token_stride apart (0: dense [T][heads][128] tensors): views of
+    // one [T][conv_dim] buffer in the mixer, fused or not
     const bool mixer = mix.qkvc != nullptr;
-    const int64_t tok = mixer ? (int64_t)mix.conv_dim : 0;
+    const int64_t tok = mixer ? (int64_t)mix.conv_dim : qkv_tok;
+    const int64_t qk_tok = tok ? tok : (int64_t)H_qk * kD;  // elements from one q/k row to the next token's
     const void* qv = mixer ? (const void*)mix.qkvc : q;
     const void* kv = mixer ? (const void*)(mix.qkvc + (size_t)H_qk * kD) : k;
     const void* vv = mixer ? (const void*)(mix.qkvc + (size_t)2 * H_qk * kD) : v;
@@ -1993,7 +1999,8 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
             void* args[] = {&tm_q, &tm_k, &tm_v, &tm_o, &qb, &kb, &a, &b, &A_log, &dt_bias, &S0,
                             &cu_seqlens, &choff, &N, &T, &H_qk, &H_v, &scale, &rec, &ob,
                             &S_final, &sref, &status, &flags, &epoch, &c0v, &wait_cycles,
-                            &withhold, const_cast<MixerFusion*>(&mix), &inject};
+                            &withhold, const_cast<MixerFusion*>(&mix), &inject,
+                            const_cast<int64_t*>(&qk_tok)};
             timer_before(opt.timer, s);
             e = cudaLaunchCooperativeKernel(kfn, dim3(grid), dim3(kFusedThreads), args, kFusedSmem,
                                             s);
@@ -2022,7 +2029,6 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, const
     }
     const bf16* q_rows = mixer ? mix.qkvc : static_cast<const bf16*>(q);
     const bf16* k_rows = mixer ? mix.qkvc + (size_t)H_qk * kD : static_cast<const bf16*>(k);
-    const int64_t qk_tok = mixer ? (int64_t)mix.conv_dim : (int64_t)H_qk * kD;
     const auto prep_fn = prep_kernel<false>;
     const auto chain_fn = mixer ? chain_kernel<true> : chain_kernel<false>;
     e = cudaFuncSetAttribute(prep_fn, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -198,12 +198,12 @@ class Timer:
     def times(self) -> list:
         """[(kernel name, milliseconds)] of the most recent call made with this timer
         (waits for its events)."""
-        ms = (ctypes.c_float * 4)()
-        n = int(self._lib.gdn_timer_read(ctypes.c_void_p(self._t), ms, 4))
+        ms = (ctypes.c_float * 8)()
+        n = int(self._lib.gdn_timer_read(ctypes.c_void_p(self._t), ms, 8))
         if n < 0:
             raise GDNError(-n, "gdn_timer_read")
         return [(self._lib.gdn_timer_kernel_name(ctypes.c_void_p(self._t), i).decode(),
-                 float(ms[i])) for i in range(min(n, 4))]
+                 float(ms[i])) for i in range(min(n, 8))]
 
     def close(self):
         if getattr(self, "_t", None):

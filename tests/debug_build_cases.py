@@ -80,7 +80,8 @@ def main():
         ("ragged_split", lambda: _prefill(ragged, gdn.GDN_IMPL_TENSOR_CORE_SPLIT)),
         ("many_chains_auto", lambda: _prefill(many, gdn.GDN_IMPL_AUTO)),
         ("slots_padding", _slots),
-        ("mixer_fused", lambda: _mixer([70, 1, 129, 0, 33], gdn.GDN_IMPL_AUTO)),
+        ("mixer_auto", lambda: _mixer([70, 1, 129, 0, 33], gdn.GDN_IMPL_AUTO)),
+        ("mixer_fused", lambda: _mixer([70, 1, 129, 0, 33], gdn.GDN_IMPL_TENSOR_CORE)),
         ("mixer_split", lambda: _mixer([70, 1, 129, 0, 33], gdn.GDN_IMPL_TENSOR_CORE_SPLIT)),
         ("inject_split", lambda: _prefill(ragged, gdn.GDN_IMPL_TENSOR_CORE_SPLIT,
                                           gdn.GDN_FAULT_BAD_INDEX)),

@@ -48,17 +48,22 @@ def _no_cache(P):
     return dataclasses.replace(P, conv_state=torch.zeros_like(P.conv_state))
 
 
-def test_mixer_35b_layer():
+@pytest.mark.parametrize("impl,kernels", [
+    (gdn.GDN_IMPL_AUTO, ["conv1d_silu", "fused_half_rows", "rmsnorm_gated"]),
+    (gdn.GDN_IMPL_TENSOR_CORE, ["fused"])])
+def test_mixer_35b_layer(impl, kernels):
     """The 35B-A3B layer (T=4096, 16 QK / 32 V heads, d=128, K=4), conv cache in and
-    out, initial states in: one overlapped launch (whole-row chain blocks)."""
+    out, initial states in: by default the convolution, the prefill (overlapped, half-row
+    chain blocks) and the norm; with the fused schedule one overlapped launch."""
     P = make_mixer_prefill_inputs([4096], H_qk=16, H_v=32, d=128, state_std=0.02, seed=1)
     timer = gdn.Timer()
-    _check(P, TOL_BF16, timer=timer)
-    assert [n for n, _ in timer.times()] == ["fused"]
+    _check(P, TOL_BF16, impl=impl, timer=timer)
+    assert [n for n, _ in timer.times()] == kernels
 
 
 @pytest.mark.parametrize("K", [2, 3, 4])
-@pytest.mark.parametrize("impl", [gdn.GDN_IMPL_AUTO, gdn.GDN_IMPL_TENSOR_CORE_SPLIT])
+@pytest.mark.parametrize("impl", [gdn.GDN_IMPL_AUTO, gdn.GDN_IMPL_TENSOR_CORE,
+                                  gdn.GDN_IMPL_TENSOR_CORE_SPLIT])
 def test_mixer_ragged_and_short(K, impl):
     """Empty sequences, sequences shorter than the cache, one token, a whole chunk, a
     ragged tail; overlapped and separate launches."""
@@ -67,7 +72,8 @@ def test_mixer_ragged_and_short(K, impl):
     _check(P, TOL_BF16, impl=impl)
 
 
-@pytest.mark.parametrize("impl", [gdn.GDN_IMPL_AUTO, gdn.GDN_IMPL_TENSOR_CORE_SPLIT])
+@pytest.mark.parametrize("impl", [gdn.GDN_IMPL_AUTO, gdn.GDN_IMPL_TENSOR_CORE,
+                                  gdn.GDN_IMPL_TENSOR_CORE_SPLIT])
 def test_mixer_cache_in_place_and_absent(impl):
     P = make_mixer_prefill_inputs([130, 1, 0, 65], H_qk=2, H_v=8, d=128, state_std=0.05,
                                   seed=21)
@@ -76,13 +82,17 @@ def test_mixer_cache_in_place_and_absent(impl):
     _check(P2, TOL_BF16, impl=impl, cache=False)
 
 
-def test_mixer_many_chains_separate_launches():
+@pytest.mark.parametrize("impl,kernels", [
+    (gdn.GDN_IMPL_AUTO, ["conv1d_silu", "chunk_offsets", "prep", "chain", "rmsnorm_gated"]),
+    (gdn.GDN_IMPL_TENSOR_CORE, ["conv1d_silu", "chunk_offsets", "prep", "chain"])])
+def test_mixer_many_chains_separate_launches(impl, kernels):
     """More chains than half the SMs: the convolution as its own streaming kernel, then
-    preparation and chains (with the fused gated norm) as separate launches."""
+    preparation and chains as separate launches, and the norm as its own kernel (by
+    default) or in the chains' output (fused schedule)."""
     P = make_mixer_prefill_inputs([300] * 6, H_qk=16, H_v=32, d=128, state_std=0.02, seed=5)
     timer = gdn.Timer()
-    _check(P, TOL_BF16, timer=timer)
-    assert [n for n, _ in timer.times()] == ["conv1d_silu", "chunk_offsets", "prep", "chain"]
+    _check(P, TOL_BF16, impl=impl, timer=timer)
+    assert [n for n, _ in timer.times()] == kernels
 
 
 @pytest.mark.parametrize("lengths,d", [([100, 0, 37], 64), ([70, 3], 128)])
@@ -95,14 +105,17 @@ def test_mixer_fp32_runs_the_steps_in_turn(lengths, d):
                                              "rmsnorm_gated"]
 
 
-def test_mixer_equals_the_three_calls():
-    """The fused call against gdn_conv1d_silu -> gdn_prefill -> gdn_rmsnorm_gated on the
-    GPU: the convolution has the same arithmetic (same q, k, v bits), so the final states
-    and the conv cache agree to the last bit; y differs only by the norm's order of
-    summation (within one bf16 rounding)."""
+@pytest.mark.parametrize("impl", [gdn.GDN_IMPL_AUTO, gdn.GDN_IMPL_TENSOR_CORE])
+def test_mixer_equals_the_three_calls(impl):
+    """The call against gdn_conv1d_silu -> gdn_prefill -> gdn_rmsnorm_gated on the GPU:
+    the default schedule runs those kernels (the prefill reading the post-conv buffer with
+    a token stride), so everything agrees to the last bit; in the fused schedule the
+    convolution has the same arithmetic (same q, k, v bits), so the final states and the
+    conv cache agree to the last bit and y differs only by the norm's order of summation
+    (within one bf16 rounding)."""
     P = make_mixer_prefill_inputs([700, 64, 1, 333], H_qk=4, H_v=8, d=128, state_std=0.05,
                                   seed=41)
-    y, Sf, cout = _run(P)
+    y, Sf, cout = _run(P, impl=impl)
     Pd = P.to("cuda")
     yc, c2 = gdn_conv1d_silu(Pd.x, Pd.conv_weight, Pd.conv_bias, Pd.cu_seqlens, Pd.conv_state)
     T, C = Pd.x.shape
@@ -116,11 +129,14 @@ def test_mixer_equals_the_three_calls():
     assert gdn_sync_status() == 0
     assert torch.equal(Sf, S2)
     assert torch.equal(cout, c2)
+    if impl == gdn.GDN_IMPL_AUTO:
+        assert torch.equal(y, y2)
     dy = (y.float() - y2.float()).abs()
     assert bool((dy <= 2.0 ** -7 * y2.float().abs() + 1e-3).all()), float(dy.max())
 
 
-@pytest.mark.parametrize("impl", [gdn.GDN_IMPL_AUTO, gdn.GDN_IMPL_TENSOR_CORE_SPLIT])
+@pytest.mark.parametrize("impl", [gdn.GDN_IMPL_AUTO, gdn.GDN_IMPL_TENSOR_CORE,
+                                  gdn.GDN_IMPL_TENSOR_CORE_SPLIT])
 def test_mixer_writes_nothing_outside_its_outputs(impl):
     """Guard regions around y and the conv cache (a stand-in for a memory checker)."""
     P = make_mixer_prefill_inputs([70, 0, 1, 130], H_qk=2, H_v=4, d=128, state_std=0.05,
