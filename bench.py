@@ -97,8 +97,16 @@ def prefill_flops(T, N, H_qk, H_v, d, C=64):
 
 
 def _source_sha1(path=TC_SOURCE):
-    with open(path, "rb") as f:
-        return hashlib.sha1(f.read()).hexdigest()
+    """SHA-1 of the kernel source's code: comments removed and every run of blank space
+    turned into one space, so that a traffic record stays valid across edits of comments
+    and layout only."""
+    import re
+    with open(path, encoding="utf-8") as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    src = re.sub(r"\s+", " ", src).strip()
+    return hashlib.sha1(src.encode()).hexdigest()
 
 
 def run_metadata(dev):

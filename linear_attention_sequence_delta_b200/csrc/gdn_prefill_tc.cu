@@ -23,9 +23,11 @@
 //
 // Two stages:
 //   prep           everything that does not depend on the state, for all chunks:
-//                  workers walk (chunk, QK head) units; each forms K K^T / Q K^T once
-//                  (one MMA into TMEM), then for each V head sharing that QK head the
-//                  gates, A, P and T = (I + A)^-1 in fp32 (8x8 diagonal blocks by
+//                  workers walk (chunk, QK head) units; each loads its K and Q rows
+//                  by TMA and forms [K; Q] [K; Q]^T once (one MMA into TMEM: K K^T and
+//                  Q K^T, and on the diagonal the squared row norms), then for each V
+//                  head sharing that QK head the gates, A, P and T = (I + A)^-1 in fp32
+//                  (8x8 diagonal blocks by
 //                  forward substitution in registers, then doubling steps 8 -> 16 ->
 //                  32 -> 64 with T_10 = -D_1 A_10 D_0, the last two on tf32 tensor
 //                  cores). T diag(beta), P and the per-token factors go to the
@@ -41,7 +43,8 @@
 // cooperative launch (fused_kernel), chain blocks consuming records as prep blocks
 // publish them (per-record flags holding the call's number); with at most a quarter
 // as many chains as SMs each chain is split over two blocks of 64 value rows (M = 64
-// MMAs). Otherwise three launches: chunk offsets, prep_kernel, chain_kernel.
+// MMAs). Otherwise three launches: chunk offsets (and the chains' order, longest
+// sequences first), prep_kernel, chain_kernel.
 //
 // Every wait is bounded; on expiry a block records GDN_ERR_TIMEOUT in the status
 // word, leaves its loops, drains its copies, frees its tensor memory and exits.
