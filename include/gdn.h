@@ -76,9 +76,10 @@ int gdn_version(void);
  * Bytes of device workspace gdn_prefill needs for these sizes. For d = 128 it
  * covers the tensor-core path: the chunk offsets of the sequences and the order
  * in which their chains run (two int32 per sequence, plus one), then per
- * (64-token chunk, V head) an 8-byte ready flag and a 17,664-byte record (the
- * chunk's T diag(beta) and P matrices and per-token factors), i.e. about 276
- * bytes per token and V head (with one extra chunk per sequence), the first two
+ * (64-token chunk, V head) an 8-byte ready flag and an 11,520-byte record (the
+ * chunk's T diag(beta) and P matrices, lower triangular, in 16-row bands, and
+ * per-token factors), i.e. about 180 bytes per token and V head (with one extra
+ * chunk per sequence), the first two
  * parts rounded up to 256 bytes; for d = 64 (CUDA-core path) it is the per-token
  * G and beta, fp32 [T, H_v] each. Returns 0 for invalid sizes (and for
  * num_seqs = 0).

@@ -71,14 +71,29 @@ constexpr int kC = kChunk;  // 64
 constexpr int kMaxGroup = 16;                    // V heads per QK head handled by prep
 
 // ---- workspace record of one (chunk, V head), written by prep, bulk-copied by chain
-constexpr uint32_t REC_T = 0;        // [64][128 B] T diag(beta), bf16, sw128 image
-constexpr uint32_t REC_P = 8192;     // [64][128 B] P, bf16, sw128 image
-constexpr uint32_t REC_G = 16384;    // factors (floats):
+// T diag(beta) and P are lower triangular, and each enters the chain as the B operand
+// (K-major, N = K = 64) of four K steps of 16. Step s needs only the rows 16 s .. 63 of
+// its 16 columns (the rows above are zero), so a matrix is kept as four bands, band s =
+// those rows and columns, in the plain (unswizzled) K-major core-matrix layout: 16-byte
+// chunk (row i, columns 8 c .. 8 c + 7), s = c / 2, at chunk index
+//   kBandStart[s] + ((i - 16 s) / 8) * 16 + (c % 2) * 8 + i % 8
+// (8-row groups 256 bytes apart, the two core matrices of a step 128 bytes apart):
+// 320 chunks (5,120 bytes) instead of the 512 of the full tile.
+constexpr int kTriChunks = 320;
+__host__ __device__ constexpr int band_start(int s) { return 16 * s * (9 - s); }  // 0 128 224 288
+__device__ __forceinline__ int tri_chunk(int i, int c) {
+    const int s = c >> 1;
+    return band_start(s) + ((i - 16 * s) >> 3) * 16 + (c & 1) * 8 + (i & 7);
+}
+constexpr uint32_t REC_T = 0;        // T diag(beta), bf16, banded
+constexpr uint32_t REC_P = 5120;     // P, bf16, banded
+constexpr uint32_t REC_G = 10240;    // factors (floats):
 constexpr int RG_FK = 0;             //   [64] e^{G_t} rk_t
 constexpr int RG_EGQ = 128;          //   [64] e^{G_t} rq_t
 constexpr int RG_EGL = 192;          //   [64] e^{G_L - G_t} rk_t
 constexpr int RG_GAMMA = 256;        //   e^{G_L}
-constexpr uint32_t kRecBytes = 17664;  // 69 x 256
+constexpr uint32_t kRecBytes = 11520;  // 45 x 256
+static_assert(band_start(4) == kTriChunks && 16 * kTriChunks == REC_P, "band layout");
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -214,7 +229,7 @@ constexpr int kEStride = 20;   // rows of the in-block exponential table (16 use
 // P and the exponential tables of the V head being worked on.
 constexpr uint32_t PS_KQ = 0;      // [2 col blocks][128 rows][128 B], raw K then Q, sw128
 constexpr uint32_t PS_AS = 0;      // [64][68] fp32 A (strictly-lower part used)
-constexpr uint32_t PS_PST = 17408; // [64][128 B] P, bf16 sw128 image (the record's P)
+constexpr uint32_t PS_PST = 17408; // P, bf16, banded (the record's P; 5,120 of 8,192 B)
 constexpr uint32_t PS_E = 25600;   // [4][16][20] exp(G_i - G_j) inside 16-blocks
 constexpr uint32_t PS_U = 30720;   // [4][64] exp(G_{16 a} - G_j)
 constexpr uint32_t PS_CI = 31744;  // [64] exp(G_i - G_{16-block start of i})
@@ -232,7 +247,7 @@ constexpr size_t kPrepSmem = 72344 + 1024;
 static_assert(PS_CI + 64 * 4 <= PS_TS, "the per-head area must fit where K and Q were");
 
 // Half a row (32 columns from 32 H) of A (row i < 64, to the A matrix) or of P (row
-// t = i - 64, to the staging image) from the matching half row x of [K; Q] K^T, whose
+// t = i - 64, to the banded staging image) from the matching half row x of [K; Q] K^T, whose
 // columns are already scaled by rk. Columns left of the row's 16-block use
 // exp(G_i - G_j) = exp(G_i - G_a0) U_j (both factors <= 1); the at most 16 columns
 // inside the block take their own exponential; columns right of the row are zero.
@@ -271,7 +286,7 @@ __device__ __forceinline__ void ap_half_row(const float (&x)[32], int row, const
 #pragma unroll
             for (int e4 = 0; e4 < 4; ++e4)
                 Arow[e4] = make_float4(v[4 * e4], v[4 * e4 + 1], v[4 * e4 + 2], v[4 * e4 + 3]);
-        } else {
+        } else if (c0 <= a0) {  // (16-column groups right of the row's block: not kept)
 #pragma unroll
             for (int q2 = 0; q2 < 2; ++q2) {
                 uint4 w;
@@ -279,7 +294,7 @@ __device__ __forceinline__ void ap_half_row(const float (&x)[32], int row, const
                 w.y = live ? pack_bf16x2(v[8 * q2 + 2], v[8 * q2 + 3]) : 0u;
                 w.z = live ? pack_bf16x2(v[8 * q2 + 4], v[8 * q2 + 5]) : 0u;
                 w.w = live ? pack_bf16x2(v[8 * q2 + 6], v[8 * q2 + 7]) : 0u;
-                *reinterpret_cast<uint4*>(Pst + sw128_off((uint32_t)i, (uint32_t)(4 * H + 2 * g + q2))) = w;
+                reinterpret_cast<uint4*>(Pst)[tri_chunk(i, 4 * H + 2 * g + q2)] = w;
             }
         }
     }
@@ -777,40 +792,33 @@ __device__ __forceinline__ void prep_worker(
             }
             named_bar_sync(bar_id, kPrepThreads);
 
-            // ---- T diag(beta) -> record (bf16 sw128 image), the staged P -> record, both
-            // as coalesced 16-byte stores; the next head's tables meanwhile -------------
+            // ---- T diag(beta) -> record, the staged P -> record, both banded, as
+            // coalesced 16-byte stores; the next head's tables meanwhile ----------------
 #pragma unroll
             for (int it = 0; it < 2; ++it) {
-                // The 8 threads of a row read its columns 4 c8 .. + 3 and 32 + 4 c8 .. + 3
-                // (two contiguous 128-byte runs: no bank conflict), times beta of those
-                // columns; each pair of neighbours then swaps halves, so that the even one
-                // holds 16-byte chunk c8 / 2 of the bf16 row and the odd one chunk 4 + c8 / 2.
-                const int idx = tid + kPrepThreads * it;  // 0..511
-                const int row = idx >> 3, c8 = idx & 7;
-                const bool odd = (c8 & 1) != 0;
-                const float* trow = Ts + row * kTsStride;
-                const float4 ta = *reinterpret_cast<const float4*>(trow + 4 * c8);
-                const float4 tb = *reinterpret_cast<const float4*>(trow + 32 + 4 * c8);
-                const float4 ba = *reinterpret_cast<const float4*>(hBeta + 4 * c8);
-                const float4 bb = *reinterpret_cast<const float4*>(hBeta + 32 + 4 * c8);
-                const float4 pa = make_float4(ta.x * ba.x, ta.y * ba.y, ta.z * ba.z, ta.w * ba.w);
-                const float4 pb = make_float4(tb.x * bb.x, tb.y * bb.y, tb.z * bb.z, tb.w * bb.w);
-                const float4 snd = odd ? pa : pb;
-                float4 rcv;
-                rcv.x = __shfl_xor_sync(0xffffffffu, snd.x, 1);
-                rcv.y = __shfl_xor_sync(0xffffffffu, snd.y, 1);
-                rcv.z = __shfl_xor_sync(0xffffffffu, snd.z, 1);
-                rcv.w = __shfl_xor_sync(0xffffffffu, snd.w, 1);
-                const float4 lo = odd ? rcv : pa, hi = odd ? pb : rcv;
-                uint4 w;  // column s of T times beta_s
-                w.x = pack_bf16x2(lo.x, lo.y);
-                w.y = pack_bf16x2(lo.z, lo.w);
-                w.z = pack_bf16x2(hi.x, hi.y);
-                w.w = pack_bf16x2(hi.z, hi.w);
-                const int ch = odd ? 4 + (c8 >> 1) : (c8 >> 1);
-                if (rec_ok) {
-                    *reinterpret_cast<uint4*>(R + REC_T + sw128_off(row, ch)) = w;
-                    reinterpret_cast<uint4*>(R + REC_P)[idx] = reinterpret_cast<const uint4*>(Pst)[idx];
+                // chunk o of the banded image: rows i .. of one 8-row group, columns
+                // 8 c .. 8 c + 7; the 8 threads of a load phase read one column run of 8
+                // consecutive rows (68 words apart: distinct bank groups)
+                const int o = tid + kPrepThreads * it;
+                if (o < kTriChunks) {
+                    const int sb = (o >= band_start(1)) + (o >= band_start(2)) + (o >= band_start(3));
+                    const int rest = o - band_start(sb);
+                    const int i = 16 * sb + (rest >> 4) * 8 + (rest & 7);
+                    const int c = 2 * sb + ((rest >> 3) & 1);
+                    const float* trow = Ts + i * kTsStride + 8 * c;
+                    const float4 ta = *reinterpret_cast<const float4*>(trow);
+                    const float4 tb = *reinterpret_cast<const float4*>(trow + 4);
+                    const float4 ba = *reinterpret_cast<const float4*>(hBeta + 8 * c);
+                    const float4 bb = *reinterpret_cast<const float4*>(hBeta + 8 * c + 4);
+                    uint4 w;  // column s of T times beta_s
+                    w.x = pack_bf16x2(ta.x * ba.x, ta.y * ba.y);
+                    w.y = pack_bf16x2(ta.z * ba.z, ta.w * ba.w);
+                    w.z = pack_bf16x2(tb.x * bb.x, tb.y * bb.y);
+                    w.w = pack_bf16x2(tb.z * bb.z, tb.w * bb.w);
+                    if (rec_ok) {
+                        reinterpret_cast<uint4*>(R + REC_T)[o] = w;
+                        reinterpret_cast<uint4*>(R + REC_P)[o] = reinterpret_cast<const uint4*>(Pst)[o];
+                    }
                 }
             }
             if (hr + 1 < r) exp_tables(sGall + (hr + 1) * kC, sU, sE, sCI, tid);
@@ -860,7 +868,8 @@ constexpr int kRing = 3;
 constexpr uint32_t SLOT_KQ = 0;        // [2 col blocks][K rows 0-63, Q rows 64-127][128 B], sw128
 constexpr uint32_t SLOT_V = 32768;     // [2 col blocks][64 rows][128 B] V, sw128
 constexpr uint32_t SLOT_REC = 49152;   // the (chunk, V head) record: T diag(beta), P, factors
-constexpr uint32_t kSlotBytes = 67584;
+constexpr uint32_t kSlotBytes = 61440;  // (the next slot's tiles 1024-byte aligned)
+static_assert(SLOT_REC + kRecBytes <= kSlotBytes && kSlotBytes % 1024 == 0, "slot layout");
 constexpr uint32_t kSlotTx = 6 * 8192 + kRecBytes;  // six 64x64 tiles + the record
 constexpr uint32_t CS_OST = kRing * kSlotBytes;     // [2 col blocks][64 t][128 B] o, sw128
 constexpr uint32_t CS_BAR = CS_OST + 16384;         // barriers (see below)
@@ -1292,8 +1301,12 @@ __device__ __forceinline__ void chain_unit(
         };
         bool dead = false;
         constexpr uint32_t id64 = idesc_bf16_f32(kM, 64, 0, 0);
-        constexpr uint32_t id_v = idesc_bf16_f32(kM, 64, 1, 0);
         constexpr uint32_t id_s = idesc_bf16_f32(kM, 128, 0, 1);
+        // the K steps of a banded B (T diag(beta), P): N = 64 - 16 s
+        constexpr uint32_t id_tri[4] = {id64, idesc_bf16_f32(kM, 48, 0, 0),
+                                        idesc_bf16_f32(kM, 32, 0, 0), idesc_bf16_f32(kM, 16, 0, 0)};
+        constexpr uint32_t id_tri_v[4] = {idesc_bf16_f32(kM, 64, 1, 0), idesc_bf16_f32(kM, 48, 1, 0),
+                                          idesc_bf16_f32(kM, 32, 1, 0), idesc_bf16_f32(kM, 16, 1, 0)};
         // TMEM A operands (fixed for the whole unit)
         uint32_t aS0[4], aS1[4], aZ[4], aU[4], aN[4];
 #pragma unroll
@@ -1326,9 +1339,9 @@ __device__ __forceinline__ void chain_unit(
                 dQ1[ks] = smem_desc_sw128(kq + 16384u + 8192u + ks * 32u, 16, 1024);
                 // V^T rows = value rows: this block's half of them when kM = 64
                 dV[ks] = smem_desc_sw128(vt + (kM == 64 ? 8192u * hv : 0u) + ks * 2048u, 8192, 1024);
-                dT[ks] = smem_desc_sw128(tt + ks * 32u, 16, 1024);
+                dT[ks] = smem_desc_kmajor_plain(tt + 16u * band_start(ks), 128, 256);
                 dKm[ks] = smem_desc_sw128(kq + ks * 2048u, 16384, 1024);
-                dP[ks] = smem_desc_sw128(ptile + ks * 32u, 16, 1024);
+                dP[ks] = smem_desc_kmajor_plain(ptile + 16u * band_start(ks), 128, 256);
             }
             if (!dead) check(mbar_wait_bounded(&full[st], (c / kRing) & 1, wait_cycles));
             // (1) the bf16 state is written: S0 K^T, then V^T (T diag(beta))^T
@@ -1338,14 +1351,14 @@ __device__ __forceinline__ void chain_unit(
                 mma_ts_group4(tmem + TM_D1K, aS0, dK0, id64, 0);
                 mma_ts_group4(tmem + TM_D1K, aS1, dK1, id64, 1);
                 mma_commit_warp(mbar);
-                mma_ss_group4(tmem + TM_D3, dV, dT, id_v, 0);
+                mma_ss_tri4(tmem + TM_D3, dV, dT, id_tri_v, 0);
             }
             // (2) Z^T is written: Vn^T += Z^T (T diag(beta))^T; then S0 Q^T into the
             // accumulator of parity c & 1, last read for chunk c - 2
             wait_rdy();
             check(true);
             if (!dead) {
-                mma_ts_group4(tmem + TM_D3, aZ, dT, id64, 1);
+                mma_ts_tri4(tmem + TM_D3, aZ, dT, id_tri, 1);
                 mma_commit_warp(mbar);
                 if (c >= 2)
                     check(mbar_wait_bounded(&ofree[c & 1], ((c - 2) >> 1) & 1, wait_cycles));
@@ -1366,7 +1379,7 @@ __device__ __forceinline__ void chain_unit(
                                             wait_cycles));
             }
             if (!dead) {
-                mma_ts_group4(tmem + TM_D4, aN, dP, id64, 0);
+                mma_ts_tri4(tmem + TM_D4, aN, dP, id_tri, 0);
                 mma_commit_warp(&obar[c & 1]);
             }
         }

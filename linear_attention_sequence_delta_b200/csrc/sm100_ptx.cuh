@@ -131,6 +131,19 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
     return d;
 }
 
+// The same for a K-major operand without swizzle: core matrices of 8 rows x 16 bytes
+// (rows 16 bytes apart), `lbo_bytes` from the first to the second core matrix of a
+// 16-element K step, `sbo_bytes` from one 8-row group to the next (swizzle mode 0).
+__device__ __forceinline__ uint64_t smem_desc_kmajor_plain(uint32_t saddr, uint32_t lbo_bytes,
+                                                           uint32_t sbo_bytes) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    return d;
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.
 // a_mn / b_mn: 1 if that operand is MN-major (contiguous along M / N).
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn) {
@@ -281,6 +294,48 @@ __device__ __forceinline__ void mma_ss_group4(uint32_t d, const uint64_t (&a)[4]
         "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %8, %9, p1;\n\t}"
         ::"r"(d), "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]),
         "l"(b[3]), "r"(idesc), "r"(acc_first)
+        : "memory");
+}
+
+// Four K steps of 16 into a 64-column accumulator whose B (N x K, K-major) is lower
+// triangular in 16 x 16 blocks: B rows n < 16 s are zero in K step s, so step s reads
+// only rows 16 s .. 63 (descriptor b[s]) and updates only accumulator columns
+// 16 s .. 63 (address d + 16 s, instruction descriptor idesc[s] with N = 64 - 16 s).
+// The first step, N = 64, accumulates only if `acc_first`. A from TMEM (a[s]) or shared
+// memory (ad[s]); one elected lane of a converged warp issues.
+__device__ __forceinline__ void mma_ts_tri4(uint32_t d, const uint32_t (&a)[4],
+                                            const uint64_t (&b)[4], const uint32_t (&idesc)[4],
+                                            uint32_t acc_first) {
+    asm volatile(
+        "{\n\t.reg .pred e, p0, p1;\n\t"
+        "setp.ne.b32 p0, %16, 0;\n\t"
+        "setp.eq.b32 p1, %16, %16;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %8, %12, p0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%1], [%5], %9, %13, p1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%2], [%6], %10, %14, p1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%3], [%7], %11, %15, p1;\n\t}"
+        ::"r"(d), "r"(d + 16u), "r"(d + 32u), "r"(d + 48u), "r"(a[0]), "r"(a[1]), "r"(a[2]),
+        "r"(a[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "r"(idesc[0]), "r"(idesc[1]),
+        "r"(idesc[2]), "r"(idesc[3]), "r"(acc_first)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_ss_tri4(uint32_t d, const uint64_t (&ad)[4],
+                                            const uint64_t (&b)[4], const uint32_t (&idesc)[4],
+                                            uint32_t acc_first) {
+    asm volatile(
+        "{\n\t.reg .pred e, p0, p1;\n\t"
+        "setp.ne.b32 p0, %16, 0;\n\t"
+        "setp.eq.b32 p1, %16, %16;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %8, %12, p0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%1], %5, %9, %13, p1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%2], %6, %10, %14, p1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%3], %7, %11, %15, p1;\n\t}"
+        ::"r"(d), "r"(d + 16u), "r"(d + 32u), "r"(d + 48u), "l"(ad[0]), "l"(ad[1]), "l"(ad[2]),
+        "l"(ad[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "r"(idesc[0]), "r"(idesc[1]),
+        "r"(idesc[2]), "r"(idesc[3]), "r"(acc_first)
         : "memory");
 }
 

@@ -45,8 +45,8 @@ def test_workspace_size(lib):
     ws = lib.gdn_prefill_workspace_size
     a256 = lambda x: (x + 255) // 256 * 256
     # d = 128: chunk offsets and chain order (2 N + 1 int32), an 8-byte flag per record
-    # and one 17,664-byte record per (chunk, V head), with at most ceil(T / 64) + N chunks
-    tc = lambda N, ch, hv: a256((2 * N + 1) * 4) + a256(ch * hv * 8) + ch * hv * 17664
+    # and one 11,520-byte record per (chunk, V head), with at most ceil(T / 64) + N chunks
+    tc = lambda N, ch, hv: a256((2 * N + 1) * 4) + a256(ch * hv * 8) + ch * hv * 11520
     assert ws(1, 4096, 16, 32, 128, 128) == tc(1, 64 + 1, 32)
     assert ws(4, 4 * 16384, 16, 64, 128, 128) == tc(4, 1024 + 4, 64)
     assert ws(64, 274156, 16, 32, 128, 128) == tc(64, (274156 + 63) // 64 + 64, 32)
