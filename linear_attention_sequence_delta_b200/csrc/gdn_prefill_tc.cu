@@ -191,17 +191,31 @@ __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
+// Four 8 x 8 matrices of 16-bit elements from shared memory, lane l giving the address of
+// row l % 8 of matrix l / 8 (16-byte aligned); register i of lane l receives elements
+// 2 (l % 4) and 2 (l % 4) + 1 of row l / 4 of matrix i, i.e. with 32-bit elements
+// (rows of four) element l % 4 of row l / 4.
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_u32(p))
+                 : "memory");
+}
+
 // d (16 x 8 tile at rows r0, columns c0 of the product) += M1[r0.., k0..k0+kn) M2[k0.., c0..)
 // with M1, M2 row-major fp32 in shared memory (row strides s1, s2), kn a multiple of 8.
+// M1's rows and k0 are 16-byte aligned: its four 8 x 4 pieces of a step are one ldmatrix
+// (rows r0 + l % 8 and r0 + 8 + l % 8, columns k and k + 4).
 __device__ __forceinline__ void tile_mma_tf32(float (&d)[4], const float* M1, int s1,
                                               const float* M2, int s2, int r0, int c0, int k0,
                                               int kn, int lane) {
     const int g = lane >> 2, t = lane & 3;
+    const float* arow = M1 + (r0 + (lane & 7) + ((lane >> 3) & 1) * 8) * s1 + ((lane >> 4) << 2);
     for (int k = k0; k < k0 + kn; k += 8) {
-        const uint32_t a[4] = {to_tf32(M1[(r0 + g) * s1 + k + t]),
-                               to_tf32(M1[(r0 + g + 8) * s1 + k + t]),
-                               to_tf32(M1[(r0 + g) * s1 + k + t + 4]),
-                               to_tf32(M1[(r0 + g + 8) * s1 + k + t + 4])};
+        uint32_t ar[4];
+        ldsm_x4(ar, arow + k);
+        const uint32_t a[4] = {to_tf32(__uint_as_float(ar[0])), to_tf32(__uint_as_float(ar[1])),
+                               to_tf32(__uint_as_float(ar[2])), to_tf32(__uint_as_float(ar[3]))};
         const uint32_t b[2] = {to_tf32(M2[(k + t) * s2 + c0 + g]),
                                to_tf32(M2[(k + t + 4) * s2 + c0 + g])};
         mma_tf32_16x8x8(d, a, b);
@@ -235,15 +249,17 @@ constexpr uint32_t PS_U = 30720;   // [4][64] exp(G_{16 a} - G_j)
 constexpr uint32_t PS_CI = 31744;  // [64] exp(G_i - G_{16-block start of i})
 constexpr uint32_t PS_TS = 32768;  // [64][68] fp32 T (entries above its diagonal blocks stay 0)
 constexpr uint32_t PS_XS = 50176;  // [32][40] fp32 merge scratch
-constexpr uint32_t PS_AB = 55296;  // [2][kMaxGroup][64] fp32 a, b
-constexpr uint32_t PS_GA = 63488;  // [kMaxGroup][64] G of every V head of the unit
-constexpr uint32_t PS_BA = 67584;  // [kMaxGroup][64] beta of every V head of the unit
-constexpr uint32_t PS_RK = 71680;  // [64] rk, [64] rq (rq includes the scale)
-constexpr uint32_t PS_PAR = 72192; // [2][kMaxGroup] A_log, dt_bias of those heads
-constexpr uint32_t PS_BAR = 72320; // mbarrier (MMA)
-constexpr uint32_t PS_TMEM = 72328;
-constexpr uint32_t PS_LDBAR = 72336; // mbarrier (TMA loads of the K and Q rows)
-constexpr size_t kPrepSmem = 72344 + 1024;
+constexpr uint32_t PS_GA = 55296;  // [kMaxGroup][64] G of every V head of the unit
+constexpr uint32_t PS_BA = 59392;  // [kMaxGroup][64] beta of every V head of the unit
+constexpr uint32_t PS_RK = 63488;  // [64] rk, [64] rq (rq includes the scale)
+constexpr uint32_t PS_BAR = 64000; // mbarrier (MMA)
+constexpr uint32_t PS_TMEM = 64008;
+constexpr uint32_t PS_LDBAR = 64016; // mbarrier (TMA loads of the K and Q rows)
+constexpr uint32_t PS_NEXT = 64032;  // [2][16 B] a coming unit's first token (int64),
+                                     // sequence and length (int32 each)
+constexpr uint32_t PS_AB = 64512;    // [2][kMaxGroup][64] fp32 a, b of the unit (copied in
+                                     // during the unit before)
+constexpr size_t kPrepSmem = PS_AB + 2 * kMaxGroup * 64 * 4 + 1024;
 static_assert(PS_CI + 64 * 4 <= PS_TS, "the per-head area must fit where K and Q were");
 
 // Half a row (32 columns from 32 H) of A (row i < 64, to the A matrix) or of P (row
@@ -456,19 +472,19 @@ __device__ __forceinline__ void prep_worker(
     float* Ts = reinterpret_cast<float*>(sm + PS_TS);
     float* As = reinterpret_cast<float*>(sm + PS_AS);
     float* Xs = reinterpret_cast<float*>(sm + PS_XS);
-    float* AB = reinterpret_cast<float*>(sm + PS_AB);
     float* sU = reinterpret_cast<float*>(sm + PS_U);   // per-head exp tables (see exp_tables)
     uint8_t* Pst = sm + PS_PST;                        // P staging image
     float* rk = reinterpret_cast<float*>(sm + PS_RK);
     float* sGall = reinterpret_cast<float*>(sm + PS_GA);
     float* sBall = reinterpret_cast<float*>(sm + PS_BA);
-    float* sPar = reinterpret_cast<float*>(sm + PS_PAR);
     float* sE = reinterpret_cast<float*>(sm + PS_E);
     float* sCI = reinterpret_cast<float*>(sm + PS_CI);
     float* rq = rk + 64;
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + PS_BAR);
     uint64_t* ldbar = reinterpret_cast<uint64_t*>(sm + PS_LDBAR);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + PS_TMEM);
+    int64_t* s_next = reinterpret_cast<int64_t*>(sm + PS_NEXT);
+    float* AB = reinterpret_cast<float*>(sm + PS_AB);
 
     const int warp = tid >> 5, lane = tid & 31;
     const int r = H_v / H_qk;
@@ -501,10 +517,33 @@ __device__ __forceinline__ void prep_worker(
     bool failed = false;
     bool ld_pending = false;  // (thread 0) a TMA load of K and Q rows not yet waited for
     uint32_t ld_phase = 0;    // (thread 0) the phase that load completes
-    // A worker's units only move forward, so the sequence of each is found by a short
-    // forward scan from the previous one's (the first by bisection): one dependent load
-    // of the offsets per unit instead of a bisection's worth.
-    int n = 0;
+    // A unit's sequence n (choff[n] <= chunk < choff[n + 1]), first token t0 and length L.
+    // A worker's units only move forward, so each unit's are found by a short forward
+    // scan from the previous one's (the first by bisection), one unit ahead: thread 0
+    // looks up the next unit while the current unit's K and Q rows are in flight and
+    // leaves the result in slot par ^ 1 of s_next, read after the barriers that follow
+    // (by the L2 prefetch of the next unit's rows, and at the end of the iteration).
+    auto locate = [&](int cgx, int& nx, int64_t& t0x, int& Lx) {
+        while (GDN_IN_BOUNDS(nx + 1, N + 1, status) && choff[nx + 1] <= cgx) ++nx;
+        t0x = (int64_t)cu_seqlens[nx] + (int64_t)(cgx - choff[nx]) * kC;
+        Lx = (int)min((int64_t)kC, (int64_t)cu_seqlens[nx + 1] - t0x);
+    };
+    // a and b of a unit's V heads (tokens past its length read as zeros) into AB, as one
+    // cp.async group of this thread
+    auto fetch_ab = [&](int64_t t0x, int Lx, int jx) {
+        for (int idx = tid; idx < 2 * r * kC; idx += kPrepThreads) {
+            const int which = idx / (r * kC);            // 0: a, 1: b
+            const int rem = idx - which * r * kC;
+            const int hr = rem >> 6, t = rem & 63;
+            const int64_t tok = t < Lx ? t0x + t : 0;
+            const bool live = t < Lx && GDN_IN_BOUNDS(tok * H_v + jx * r + hr, T_total * H_v, status);
+            const float* src = (which ? b : a) + (size_t)tok * H_v + jx * r + hr;
+            cp_async_4(AB + (which * kMaxGroup + hr) * kC + t, src, live ? 4u : 0u);
+        }
+        cp_async_commit();
+    };
+    int n = 0, L = 0, par = 0;
+    int64_t t0 = 0;
     if (worker < total_units) {
         const int cg = worker / H_qk;
         int hi = N;
@@ -512,16 +551,14 @@ __device__ __forceinline__ void prep_worker(
             const int mid = (n + hi) >> 1;
             if (choff[mid] <= cg) n = mid; else hi = mid;
         }
+        locate(cg, n, t0, L);
+        fetch_ab(t0, L, worker % H_qk);
     }
 
 #pragma unroll 1
     for (int unit = worker; unit < total_units; unit += nworkers) {
         const int cg = unit / H_qk;
         const int j = unit - cg * H_qk;
-        // sequence n: choff[n] <= cg < choff[n + 1]
-        while (GDN_IN_BOUNDS(n + 1, N + 1, status) && choff[n + 1] <= cg) ++n;
-        const int64_t t0 = (int64_t)cu_seqlens[n] + (int64_t)(cg - choff[n]) * kC;
-        const int L = (int)min((int64_t)kC, (int64_t)cu_seqlens[n + 1] - t0);
 
         // ---- raw K and Q rows (sw128: four TMA boxes of 64 rows x 128 bytes, the chain's
         // tile layout), or the convolution that makes them; gates of the r V heads
@@ -536,23 +573,7 @@ __device__ __forceinline__ void prep_worker(
             ld_pending = true;
             ld_phase = lphase;
         }
-        for (int idx = tid; idx < 2 * r * kC; idx += kPrepThreads) {
-            const int which = idx / (r * kC);            // 0: a, 1: b
-            const int rem = idx - which * r * kC;
-            const int hr = rem >> 6, t = rem & 63;
-            const int64_t tok = t < L ? t0 + t : 0;
-            const bool live = t < L && GDN_IN_BOUNDS(tok * H_v + j * r + hr, T_total * H_v, status);
-            const float* src = (which ? b : a) + (size_t)tok * H_v + j * r + hr;
-            cp_async_4(AB + (which * kMaxGroup + hr) * kC + t, src, live ? 4u : 0u);
-        }
-        if (tid < 2 * r) {
-            const int hr = tid >> 1;
-            const bool ok = GDN_IN_BOUNDS(j * r + hr, H_v, status);
-            cp_async_4(sPar + (tid & 1) * kMaxGroup + hr,
-                       ((tid & 1) ? dt_bias : A_log) + (ok ? j * r + hr : 0), ok ? 4u : 0u);
-        }
-        cp_async_commit();
-        cp_async_wait<0>();
+        const int un = unit + nworkers;
         if (!kConv && L < kC) {
             // the rows past the sequence's end hold the next tokens (or zeros past T): zero
             // them, 16 bytes a thread at a time (whole 128-byte rows, so no swizzle matters)
@@ -565,6 +586,7 @@ __device__ __forceinline__ void prep_worker(
                                           ch * 16) = make_uint4(0u, 0u, 0u, 0u);
             }
         }
+        cp_async_wait<0>();  // this unit's a and b (copied in during the unit before)
         fence_proxy_async_smem();
         named_bar_sync(bar_id, kPrepThreads);
 
@@ -593,13 +615,19 @@ __device__ __forceinline__ void prep_worker(
         // ---- gates of every V head of the group: one warp per head, two tokens a lane:
         // g, beta and the in-chunk inclusive cumsum G (the record's per-token factors
         // follow once the row norms are known)
-        for (int hr = warp; hr < r; hr += kPrepThreads / 32) {
-            const float A_l = sPar[hr], dtb = sPar[kMaxGroup + hr];
+        // (warps 1.., while thread 0 waits for the rows and issues the MMA)
+        for (int hr = warp - 1; hr >= 0 && hr < r; hr += kPrepThreads / 32 - 1) {
+            const int hv = j * r + hr;
+            const bool hok = GDN_IN_BOUNDS(hv, H_v, status);
+            const float A_l = hok ? A_log[hv] : 0.f, dtb = hok ? dt_bias[hv] : 0.f;
             const int ta = 2 * lane, tb = 2 * lane + 1;
-            const float ga = ta < L ? gate_g(AB[hr * kC + ta], A_l, dtb) : 0.f;
-            const float gb = tb < L ? gate_g(AB[hr * kC + tb], A_l, dtb) : 0.f;
-            const float ba = ta < L ? gate_beta(AB[(kMaxGroup + hr) * kC + ta]) : 0.f;
-            const float bb = tb < L ? gate_beta(AB[(kMaxGroup + hr) * kC + tb]) : 0.f;
+            const bool la = ta < L, lb = tb < L;
+            const float2 av = *reinterpret_cast<const float2*>(AB + hr * kC + ta);
+            const float2 bv = *reinterpret_cast<const float2*>(AB + (kMaxGroup + hr) * kC + ta);
+            const float ga = la ? gate_g(av.x, A_l, dtb) : 0.f;
+            const float gb = lb ? gate_g(av.y, A_l, dtb) : 0.f;
+            const float ba = la ? gate_beta(bv.x) : 0.f;
+            const float bb = lb ? gate_beta(bv.y) : 0.f;
             float sc = ga + gb;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
@@ -609,11 +637,36 @@ __device__ __forceinline__ void prep_worker(
             *reinterpret_cast<float2*>(sGall + hr * kC + ta) = make_float2(sc - gb, sc);
             *reinterpret_cast<float2*>(sBall + hr * kC + ta) = make_float2(ba, bb);
         }
+        // ---- the next unit, by the last warp meanwhile: its sequence, first token and
+        // length (into slot par ^ 1 of s_next, read after the barriers that follow) and
+        // its K and Q rows fetched into L2 (the four boxes its loads will read)
+        if (warp == kPrepThreads / 32 - 1 && un < total_units) {
+            int nn = n, Ln = 0;
+            int64_t t0n = 0;
+            if (lane == 0) {
+                locate(un / H_qk, nn, t0n, Ln);
+                s_next[2 * (par ^ 1)] = t0n;
+                reinterpret_cast<int*>(s_next + 2 * (par ^ 1) + 1)[0] = nn;
+                reinterpret_cast<int*>(s_next + 2 * (par ^ 1) + 1)[1] = Ln;
+            }
+            // (with the convolution fused in, the rows are made from x: nothing to fetch)
+            if (!kConv && lane == 0 && Ln > 0) {
+                const int jn = un % H_qk;
+                tma_prefetch_l2_3d(tm_k, 0, jn, (int32_t)t0n);
+                tma_prefetch_l2_3d(tm_k, 64, jn, (int32_t)t0n);
+                tma_prefetch_l2_3d(tm_q, 0, jn, (int32_t)t0n);
+                tma_prefetch_l2_3d(tm_q, 64, jn, (int32_t)t0n);
+            }
+        }
         const bool ok = mbar_wait_bounded(bar, mphase, wait_cycles);
         mphase ^= 1u;
         if (!ok) failed = true;
         if (named_bar_any(bar_id, kPrepThreads, failed)) { failed = true; break; }
         tc_fence_after();
+        // the gates have read this unit's a and b: the next unit's come in meanwhile
+        if (un < total_units)
+            fetch_ab(s_next[2 * (par ^ 1)],
+                     reinterpret_cast<const int*>(s_next + 2 * (par ^ 1) + 1)[1], un % H_qk);
         // ---- inverse row norms from the diagonal (K K^T)_ii, (Q Q^T)_tt: the warps of the
         // first column half load the 32 columns of their own 32 rows and keep their lane's
         {
@@ -666,25 +719,6 @@ __device__ __forceinline__ void prep_worker(
         // every later head's are built while the head before writes its record.
         exp_tables(sGall, sU, sE, sCI, tid);
         named_bar_sync(bar_id, kPrepThreads);
-        {
-            const int un = unit + nworkers;
-            if (un < total_units) {
-                const int cgn = un / H_qk, jn = un - cgn * H_qk;
-                int nn = n;
-                while (GDN_IN_BOUNDS(nn + 1, N + 1, status) && choff[nn + 1] <= cgn) ++nn;
-                const int64_t t0n = (int64_t)cu_seqlens[nn] + (int64_t)(cgn - choff[nn]) * kC;
-                const int Ln = (int)min((int64_t)kC, (int64_t)cu_seqlens[nn + 1] - t0n);
-                const int rr = tid >> 2;
-                // (with the convolution fused in, the rows are made from x: nothing to fetch)
-                if (!kConv && rr < Ln &&
-                    GDN_IN_BOUNDS((t0n + rr) * qk_tok + (int64_t)jn * kD + 127, qk_extent, status))
-                    prefetch_l2(((tid & 2) ? q : k) + (size_t)(t0n + rr) * qk_tok + (size_t)jn * kD +
-                                (tid & 1) * 64);
-                if (tid < 2 * kC && (tid & 63) < Ln &&
-                    GDN_IN_BOUNDS((t0n + (tid & 63)) * H_v + jn * r, T_total * H_v, status))
-                    prefetch_l2(((tid >> 6) ? b : a) + (size_t)(t0n + (tid & 63)) * H_v + jn * r);
-            }
-        }
 
 #pragma unroll 1
         for (int hr = 0; hr < r; ++hr) {
@@ -741,17 +775,21 @@ __device__ __forceinline__ void prep_worker(
             {
                 const int a0 = (tid >> 6) * 16;
                 const int rr = (tid >> 3) & 7, cc = tid & 7;
-                const float* Arow = As + (a0 + 8 + rr) * kAsStride + a0;
+                const float4* Arow = reinterpret_cast<const float4*>(As + (a0 + 8 + rr) * kAsStride + a0);
+                const float4 Al = Arow[0], Ah = Arow[1];
+                const float Av[8] = {Al.x, Al.y, Al.z, Al.w, Ah.x, Ah.y, Ah.z, Ah.w};
                 float acc = 0.f;
 #pragma unroll
-                for (int m = 0; m < 8; ++m) acc = fmaf(Arow[m], Ts[(a0 + m) * kTsStride + a0 + cc], acc);
+                for (int m = 0; m < 8; ++m) acc = fmaf(Av[m], Ts[(a0 + m) * kTsStride + a0 + cc], acc);
                 Xs[tid] = acc;
                 named_bar_sync(bar_id, kPrepThreads);
-                const float* Drow = Ts + (a0 + 8 + rr) * kTsStride + a0 + 8;
+                const float4* Drow = reinterpret_cast<const float4*>(Ts + (a0 + 8 + rr) * kTsStride + a0 + 8);
+                const float4 Dl = Drow[0], Dh = Drow[1];
+                const float Dv[8] = {Dl.x, Dl.y, Dl.z, Dl.w, Dh.x, Dh.y, Dh.z, Dh.w};
                 const float* Xb = Xs + (tid & ~63);
                 float t1 = 0.f;
 #pragma unroll
-                for (int m = 0; m < 8; ++m) t1 = fmaf(Drow[m], Xb[m * 8 + cc], t1);
+                for (int m = 0; m < 8; ++m) t1 = fmaf(Dv[m], Xb[m * 8 + cc], t1);
                 Ts[(a0 + 8 + rr) * kTsStride + a0 + cc] = -t1;
             }
             named_bar_sync(bar_id, kPrepThreads);
@@ -826,8 +864,13 @@ __device__ __forceinline__ void prep_worker(
             if (flags && tid == 0 && rec_ok) publish_record(flags, (size_t)cg * H_v + h, epoch);
         }
         tc_fence_before();  // this unit's TMEM reads precede the next unit's MMA
+        par ^= 1;
+        t0 = s_next[2 * par];
+        n = reinterpret_cast<const int*>(s_next + 2 * par + 1)[0];
+        L = reinterpret_cast<const int*>(s_next + 2 * par + 1)[1];
     }
     // no copy into shared memory may still be in flight when the worker ends
+    cp_async_wait<0>();
     if (tid == 0 && ld_pending && !mbar_wait_bounded(ldbar, ld_phase, wait_cycles)) failed = true;
     tc_fence_before();
     named_bar_sync(bar_id, kPrepThreads);

@@ -387,6 +387,15 @@ __device__ __forceinline__ void bulk_wait_group() {
 }
 
 // Bring the cache line holding `p` into L2 (a hint; no value is returned).
+// ---- TMA: the rows of one 3-D tiled box fetched into L2 only (nothing lands in shared
+// memory; rows outside the tensor are skipped).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const void* tmap, int32_t c0, int32_t c1,
+                                                   int32_t c2) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];"
+                 ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+
 __device__ __forceinline__ void prefetch_l2(const void* p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
