@@ -528,10 +528,10 @@ __device__ __forceinline__ void prep_worker(
         t0x = (int64_t)cu_seqlens[nx] + (int64_t)(cgx - choff[nx]) * kC;
         Lx = (int)min((int64_t)kC, (int64_t)cu_seqlens[nx + 1] - t0x);
     };
-    // a and b of a unit's V heads (tokens past its length read as zeros) into AB, as one
-    // cp.async group of this thread
-    auto fetch_ab = [&](int64_t t0x, int Lx, int jx) {
-        for (int idx = tid; idx < 2 * r * kC; idx += kPrepThreads) {
+    // a and b of a unit's V heads (tokens past its length read as zeros) into AB, element
+    // i0, i0 + step, ... by this thread, as one cp.async group of it
+    auto fetch_ab = [&](int64_t t0x, int Lx, int jx, int i0, int step) {
+        for (int idx = i0; idx < 2 * r * kC; idx += step) {
             const int which = idx / (r * kC);            // 0: a, 1: b
             const int rem = idx - which * r * kC;
             const int hr = rem >> 6, t = rem & 63;
@@ -552,7 +552,7 @@ __device__ __forceinline__ void prep_worker(
             if (choff[mid] <= cg) n = mid; else hi = mid;
         }
         locate(cg, n, t0, L);
-        fetch_ab(t0, L, worker % H_qk);
+        fetch_ab(t0, L, worker % H_qk, tid, kPrepThreads);
     }
 
 #pragma unroll 1
@@ -663,10 +663,12 @@ __device__ __forceinline__ void prep_worker(
         if (!ok) failed = true;
         if (named_bar_any(bar_id, kPrepThreads, failed)) { failed = true; break; }
         tc_fence_after();
-        // the gates have read this unit's a and b: the next unit's come in meanwhile
-        if (un < total_units)
+        // the gates have read this unit's a and b: the next unit's come in meanwhile, asked
+        // for by the warps of the second column half (the first load the row norms)
+        if (un < total_units && hh == 1)
             fetch_ab(s_next[2 * (par ^ 1)],
-                     reinterpret_cast<const int*>(s_next + 2 * (par ^ 1) + 1)[1], un % H_qk);
+                     reinterpret_cast<const int*>(s_next + 2 * (par ^ 1) + 1)[1], un % H_qk,
+                     tid - kPrepThreads / 2, kPrepThreads / 2);
         // ---- inverse row norms from the diagonal (K K^T)_ii, (Q Q^T)_tt: the warps of the
         // first column half load the 32 columns of their own 32 rows and keep their lane's
         {
