@@ -327,11 +327,11 @@ int gdn_prefill_slots_ex(const void* q, const void* k, const void* v, int32_t io
  * array inside the library.
  *   - It always runs the fp32 CUDA-core chunk kernel (the gate kernel, then the
  *     CUDA-core prefill), whatever the shape and type: the tensor-core path needs
- *     a workspace proportional to the tokens (about 276 bytes per token and V
+ *     a workspace proportional to the tokens (about 180 bytes per token and V
  *     head), which a fixed array cannot hold for useful sizes. The results agree
  *     with gdn_prefill within the same tolerances; for bf16 with d = 128 the call
  *     is much slower (on the 35B-A3B layer shape, T = 4096 with 32 V heads: about
- *     3.5 ms against about 0.14 ms for gdn_prefill).
+ *     3.5 ms against about 0.12 ms for gdn_prefill).
  *   - Capacity: total_tokens * H_v <= GDN_NOALLOC_MAX_GATE_ELEMS; larger calls
  *     return GDN_ERR_WORKSPACE and launch nothing (use gdn_prefill for them).
  *     The array (8 MiB) is held on every GPU that loads the library until the
