@@ -31,8 +31,11 @@
 //                  forward substitution in registers, then doubling steps 8 -> 16 ->
 //                  32 -> 64 with T_10 = -D_1 A_10 D_0, the last two on tf32 tensor
 //                  cores). T diag(beta), P and the per-token factors go to the
-//                  workspace as a record per (chunk, V head): images of the chain's
-//                  shared-memory tiles.
+//                  workspace as a record per (chunk, V head): the two lower-triangular
+//                  matrices as the 16-row bands the chain's MMAs read (see the record
+//                  layout below), copied into the chain's shared memory as they are.
+//                  Each worker finds the next unit's sequence and prefetches its rows
+//                  and gate inputs one unit ahead.
 //   chain          one (sequence, V head) walks its chunks in order. The fp32 state
 //                  lives in the registers of eight state warps; every A operand they
 //                  produce (the bf16 state, Z^T, Vn^T and its decay-scaled copy) goes to
@@ -1802,7 +1805,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) chain_kernel(
 // Prep and chain in one cooperative launch (every block resident at once), so the
 // chain of the first sequences runs while prep workers produce the later records.
 // Block u < c0 runs chain unit u (sequence u / H_v, V head u % H_v); the others run
-// two prep workers each (256 threads, their own 90 KB of shared memory and 64 TMEM
+// two prep workers each (256 threads, their own 72 KB of shared memory and 128 TMEM
 // columns). A chain's loader waits (bounded) for each record's flag to carry this
 // call's number before its bulk copy, and prep workers never wait on chains, so
 // every wait ends. Nothing in the workspace needs clearing between calls.
