@@ -1,6 +1,6 @@
 """Cases for the debug build, run by tests/test_debug_build_gpu.py in a process of its own
 that loads libgdn_debug.so (GDN_LIBRARY): the tensor-core prefill's schedules on ragged
-and empty sequences, pool slots with padding entries, the mixer core with the
+and empty sequences, more preparation units than workers, pool slots with padding entries, the mixer core with the
 convolution and the norm fused in, and a call with one injected index check. Each call is
 compared with the oracle, and the status word and the first failed check's site are read
 after it. Prints one JSON list of {case, err, status, site} (test infrastructure).
@@ -74,11 +74,18 @@ def main():
                                  state_std=0.05, seed=44)
     many = make_prefill_inputs([100] * 8, H_qk=16, H_v=32, d_k=128, d_v=128, state_std=0.05,
                                seed=45)
+    # more (chunk, QK head) units than preparation workers, over many short sequences: each
+    # worker looks the next unit up (often across several sequence boundaries) and fetches
+    # its rows and gate inputs one unit ahead
+    rng = np.random.default_rng(47)
+    units = make_prefill_inputs([int(x) for x in rng.integers(1, 300, size=96)], H_qk=8, H_v=32,
+                                d_k=128, d_v=128, state_std=0.05, seed=48)
     cases = [
         ("ragged_half_rows", lambda: _prefill(ragged, gdn.GDN_IMPL_TENSOR_CORE)),
         ("ragged_whole_rows", lambda: _prefill(ragged, gdn.GDN_IMPL_TENSOR_CORE_WHOLE_ROWS)),
         ("ragged_split", lambda: _prefill(ragged, gdn.GDN_IMPL_TENSOR_CORE_SPLIT)),
         ("many_chains_auto", lambda: _prefill(many, gdn.GDN_IMPL_AUTO)),
+        ("many_units_split", lambda: _prefill(units, gdn.GDN_IMPL_TENSOR_CORE_SPLIT)),
         ("slots_padding", _slots),
         ("mixer_auto", lambda: _mixer([70, 1, 129, 0, 33], gdn.GDN_IMPL_AUTO)),
         ("mixer_fused", lambda: _mixer([70, 1, 129, 0, 33], gdn.GDN_IMPL_TENSOR_CORE)),

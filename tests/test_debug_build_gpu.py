@@ -32,7 +32,7 @@ def results():
 
 
 CLEAN = ["ragged_half_rows", "ragged_whole_rows", "ragged_split", "many_chains_auto",
-         "slots_padding", "mixer_auto", "mixer_fused", "mixer_split", "after_injection"]
+         "many_units_split", "slots_padding", "mixer_auto", "mixer_fused", "mixer_split", "after_injection"]
 
 
 @pytest.mark.parametrize("case", CLEAN)
